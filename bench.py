@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the masked HLA forward on B200.
+
+Default workload: ratio-normalised second-order HLA, bf16 inputs, fp32 output,
+B=4, H=16, T=4096, d=dv=64 (262,144 tokens per step), synthetic seeded inputs.
+One step = one full forward (segment summaries, Blelloch scan, output pass).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  Device timing: CUDA events recorded by the
+library on the launching stream around every phase of every timed step; L2 is
+flushed (a 512 MiB write) before every step, outside the events.  Multi-GPU
+(torchrun): every rank runs its own batch of the same shape (no collective on
+the data path: heads are independent), time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import hla_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "hla2n_bf16_4x16x4096x64"
+METRIC = "HLA-2 masked fwd tokens/sec (B·H·T/s) at d=64 bf16; % of B200 bf16 tensor peak"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(hla_inputs.WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if args.steps < 1:
+        p.error("--steps must be >= 1")
+    return args
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def dist_init(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, max_seconds_per_step: float) -> float:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / max_seconds_per_step
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled while the GPU works
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="hla_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        busy = [x for x in sm if smax and x > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# roofline bookkeeping
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def output_kernel_model(path: str, w: hla_inputs.Workload):
+    """Algorithmic work of the output kernel per token ('Roofline')."""
+    D = w.d
+    if path == "tc":
+        c = 128
+        # A = Q K^T, P = Q S0, W = [P|A][Q|A]^T, O = [Q|W][R0;V], state walk (Z, S, R)
+        flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c) + 2 * c * D + 2 * D * (D + 16) + 2 * D * D
+        return {"bound": "tensor", "flops_per_token": flops, "chunk": c}
+    c = 64
+    flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
+    return {"bound": "alu", "flops_per_token": flops, "chunk": c}
+
+
+def alu_peak_tflops(sm_mhz: float) -> float:
+    """FP32 FFMA peak of a B200: 148 SMs x 128 lanes x 2 flop x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import higher_order_linear_chunked_b200 as hla
+
+    rank, world, local_rank = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (this library has no CPU path)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist_init(world, "nccl")
+    base = hla_inputs.workload(args.workload)
+    w = base.scaled(seed=base.seed + rank)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    tokens = w.tokens
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    gd = g.to(dev) if g is not None else None
+    out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
+    op = hla.OP_CODES[w.op]
+    ws = hla.make_workspace(op, qd, vd, decayed=gd is not None)
+    dcode = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
+    launches_per_step = hla.kernel_launches(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv)
+    path = "tc" if hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv) else "simt"
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def new_events():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for e in evs:
+            e.record()
+        return evs
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        hla.forward(w.op, qd, kd, vd, gamma=gd, eps=w.eps, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    if hla.read_device_status(ws) != 0:
+        raise SystemExit("device status word set during warm-up")
+    events = [new_events() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()                                            # outside the timed events
+        hla.forward_profiled(w.op, qd, kd, vd, events[i], gamma=gd, eps=w.eps, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.stop()
+    step_ms = [ev[0].elapsed_time(ev[3]) for ev in events]
+    out_ms = [ev[2].elapsed_time(ev[3]) for ev in events]
+    sum_ms = [ev[0].elapsed_time(ev[1]) for ev in events]
+    scan_ms = [ev[1].elapsed_time(ev[2]) for ev in events]
+    status = hla.read_device_status(ws)
+    total_ms = sum(step_ms)
+    max_total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = max_total_ms / args.steps
+    value = weak_scaling_value(tokens, world, ms_per_step / 1e3)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+        oh = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32).pin_memory()
+        st = torch.cuda.current_stream(dev)
+        e_ms = []
+        for i in range(args.e2e_steps + 2):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            hla.forward(w.op, qd, kd, vd, gamma=gd, eps=w.eps, out=out, workspace=ws)
+            oh.copy_(out, non_blocking=True)
+            b.record(st)
+            torch.cuda.synchronize()
+            if i >= 2:
+                e_ms.append(a.elapsed_time(b))
+        e2e_ms = max_over_ranks(sum(e_ms) / len(e_ms), world, dev)
+        h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
+        e2e = {"value": weak_scaling_value(tokens, world, e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+               "ms_per_step": e2e_ms}
+
+    peaks, peak_kind = load_peaks()
+    clk = clocks.summary()
+    model = output_kernel_model(path, w)
+    out_avg_ms = statistics.mean(out_ms)
+    achieved = model["flops_per_token"] * tokens / (out_avg_ms / 1e3) / 1e12
+    if model["bound"] == "tensor":
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_note = f"bf16 dense burst ({peak_kind})"
+    else:
+        smax = float(peaks.get("sm_max_mhz", 1965.0))
+        peak = alu_peak_tflops(smax)
+        peak_note = f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"
+    roofline = {"kernel": "output", "bound": model["bound"], "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
+                "flops_per_token": model["flops_per_token"], "kernel_ms": out_avg_ms,
+                "phase_ms": {"summary": statistics.mean(sum_ms), "scan": statistics.mean(scan_ms),
+                             "output": out_avg_ms}}
+    roofline["traffic"] = _traffic_from_profiles(path, w)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, q, k, v, g)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "op": w.op, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "dv": w.dv,
+                       "tokens_per_gpu": tokens, "path": path, "chunk": model["chunk"],
+                       "l2": "flushed before every step (512 MiB write, outside the timed events)",
+                       "parallelism": f"dp{world} (independent heads per rank, no collective)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": launches_per_step * args.steps, "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def _traffic_from_profiles(path, w):
+    """DRAM bytes per launch of the output kernel from the committed ncu summary, if it matches."""
+    f = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(f):
+        return None
+    try:
+        rec = json.load(open(f)).get(f"{path}:{w.name}")
+    except (OSError, ValueError):
+        return None
+    return rec.get("dram_bytes_per_launch") if rec else None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline and the reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, q, k, v, g, max_tokens: int = 1 << 30):
+    import oracle
+    threads = os.cpu_count() or 1
+    B, H, T = w.B, w.H, w.T
+    # the whole workload (every head, every token) unless it is larger than max_tokens
+    Ts = min(T, max(1, max_tokens // (B * H)))
+    qs, ks, vs = q[:, :, :Ts], k[:, :, :Ts], v[:, :, :Ts]
+    t0 = time.perf_counter()
+    oracle.recur(w.op, qs, ks, vs, gamma=g, eps=w.eps, nthreads=threads)
+    dt = time.perf_counter() - t0
+    n = B * H * Ts
+    return {"value": n / dt, "unit": UNIT, "cores": min(threads, B * H), "kind": "oracle",
+            "sample": f"{B}x{H} heads x {Ts} tokens ({n} tokens) of the same workload, serial fp64 "
+                      f"recurrence, one host thread per head, {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = hla_inputs.workload(args.workload)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    threads = os.cpu_count() or 1
+    Ts = min(w.T, 1024)                         # bounded sample per step: every head, first Ts tokens
+    qs, ks, vs = q[:, :, :Ts], k[:, :, :Ts], v[:, :, :Ts]
+    n = w.B * w.H * Ts
+    for _ in range(args.warmup):
+        oracle.recur(w.op, qs, ks, vs, gamma=g, eps=w.eps, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recur(w.op, qs, ks, vs, gamma=g, eps=w.eps, nthreads=threads)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"{w.B}x{w.H} heads x first {Ts} tokens ({n} tokens) per step, serial fp64 recurrence "
+              f"(the oracle), one host thread per head")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "op": w.op, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "dv": w.dv},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, w.B * w.H), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,248 @@
+"""B200 (sm_100a) masked Higher-order Linear Attention forward.
+
+A thin ctypes binding over the C ABI of ``libhla.so`` (declared in
+``include/hla.h``).  This module only marshals arguments: every step of the
+computation runs in the library's CUDA kernels, on the tensors' device, on the
+current torch stream.  PyTorch supplies device memory and streams.  There is no
+CPU implementation here and no fallback: if the library is missing or the
+tensors are not CUDA tensors, the calls raise.
+
+Operations ("Higher-order Linear Attention" summary, gist.science 2510.27258):
+
+* :func:`hla2` - second-order masked output (Metodología 1), optional per-head
+  decay ``gamma`` (Contribuciones 2);
+* :func:`hla2_normalized` - the ratio-normalised variant (Metodología 1);
+* :func:`ahla` - asymmetric AHLA (Metodología 2);
+* :func:`hla3` - third-order masked output (Metodología 3).
+
+Inputs are ``[B, H, T, d]`` (``v``: ``[B, H, T, dv]``) contiguous fp32 or
+bf16 tensors; the output is fp32 ``[B, H, T, dv]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhla.so")
+
+HLA_OK = 0
+HLA_F32, HLA_BF16 = 0, 1
+OP_HLA2, OP_HLA2_NORM, OP_AHLA, OP_HLA3 = 0, 1, 2, 3
+
+STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_ALIGN", 4: "HLA_ERR_DTYPE",
+                5: "HLA_ERR_UNSUPPORTED", 6: "HLA_ERR_WORKSPACE", 7: "HLA_ERR_CUDA", 8: "HLA_ERR_TIMEOUT"}
+
+# Every symbol include/hla.h declares.
+EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
+           "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_read_device_status", "hla_selftest_umma")
+
+
+class HLAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """Load ``libhla.so`` (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise OSError(f"libhla.so not found at {p}: run higher_order_linear_chunked_b200.build.build() first")
+    lib = ctypes.CDLL(p)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.hla_abi_version.argtypes, lib.hla_abi_version.restype = [], i
+    lib.hla_status_str.argtypes, lib.hla_status_str.restype = [i], ctypes.c_char_p
+    lib.hla_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.hla_workspace_bytes.restype = sz
+    common = [vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    for name in ("hla2_forward", "ahla_forward", "hla3_forward"):
+        fn = getattr(lib, name)
+        fn.argtypes = common + [vp, sz, vp]
+        fn.restype = i
+    lib.hla2_forward_normalized.argtypes = common + [f, vp, sz, vp]
+    lib.hla2_forward_normalized.restype = i
+    lib.hla_forward_profiled.argtypes = [i] + common + [f, vp, sz, vp, vp]
+    lib.hla_forward_profiled.restype = i
+    lib.hla_kernel_launches.argtypes = [i, i, i, i, i, i, i, i]
+    lib.hla_kernel_launches.restype = i
+    lib.hla_uses_tensor_cores.argtypes = [i, i, i, i, i, i, i, i]
+    lib.hla_uses_tensor_cores.restype = i
+    lib.hla_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i)]
+    lib.hla_read_device_status.restype = i
+    lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
+    lib.hla_selftest_umma.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return HLA_F32
+    if t.dtype == torch.bfloat16:
+        return HLA_BF16
+    raise TypeError(f"q, k, v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _check(q, k, v):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, T, d]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if q.shape != k.shape or q.shape[:3] != v.shape[:3]:
+        raise ValueError("shape mismatch: q, k [B,H,T,d], v [B,H,T,dv]")
+
+
+def workspace_bytes(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> int:
+    return int(load_library().hla_workspace_bytes(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
+
+
+def kernel_launches(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> int:
+    return int(load_library().hla_kernel_launches(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
+
+
+def uses_tensor_cores(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> bool:
+    return bool(load_library().hla_uses_tensor_cores(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
+
+
+def make_workspace(op: int, q, v, decayed: bool = False):
+    """Allocate (with torch, on q's device) a workspace sized for this call."""
+    torch = _torch()
+    B, H, T, d = q.shape
+    n = workspace_bytes(op, _dtype_code(q), decayed, B, H, T, d, v.shape[-1])
+    if n == 0:
+        raise HLAError(5, "unsupported shape/dtype for this op")
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def _call(op: int, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):
+    torch = _torch()
+    _check(q, k, v)
+    lib = load_library()
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=q.device)
+    if gamma is not None:
+        if not gamma.is_cuda or gamma.dtype != torch.float32 or gamma.numel() != H or not gamma.is_contiguous():
+            raise ValueError("gamma must be a contiguous CUDA float32 tensor of shape [H]")
+    if workspace is None:
+        workspace = make_workspace(op, q, v, decayed=gamma is not None)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    sptr = ctypes.c_void_p(st.cuda_stream)
+    gptr = ctypes.c_void_p(gamma.data_ptr()) if gamma is not None else ctypes.c_void_p(0)
+    args = [ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+            ctypes.c_void_p(out.data_ptr()), B, H, T, d, dv, _dtype_code(q), gptr]
+    ws = [ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel() * workspace.element_size()), sptr]
+    if op == OP_HLA2:
+        rc = lib.hla2_forward(*args, *ws)
+    elif op == OP_HLA2_NORM:
+        rc = lib.hla2_forward_normalized(*args, ctypes.c_float(eps), *ws)
+    elif op == OP_AHLA:
+        rc = lib.ahla_forward(*args, *ws)
+    elif op == OP_HLA3:
+        rc = lib.hla3_forward(*args, *ws)
+    else:
+        raise ValueError(op)
+    if rc != HLA_OK:
+        raise HLAError(rc, "HLA forward rejected the call")
+    return out
+
+
+def hla2(q, k, v, gamma=None, out=None, workspace=None, stream=None):
+    """Second-order masked HLA forward (optional per-head decay gamma [H])."""
+    return _call(OP_HLA2, q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
+
+
+def hla2_normalized(q, k, v, eps: float = 1e-6, gamma=None, out=None, workspace=None, stream=None):
+    """Ratio-normalised second-order masked HLA forward."""
+    return _call(OP_HLA2_NORM, q, k, v, gamma=gamma, eps=eps, out=out, workspace=workspace, stream=stream)
+
+
+def ahla(q, k, v, out=None, workspace=None, stream=None):
+    """AHLA masked forward."""
+    return _call(OP_AHLA, q, k, v, out=out, workspace=workspace, stream=stream)
+
+
+def hla3(q, k, v, out=None, workspace=None, stream=None):
+    """Third-order masked HLA forward."""
+    return _call(OP_HLA3, q, k, v, out=out, workspace=workspace, stream=stream)
+
+
+def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):
+    """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3"."""
+    if op_name == "hla2":
+        return hla2(q, k, v, out=out, workspace=workspace, stream=stream)
+    if op_name == "hla2n":
+        return hla2_normalized(q, k, v, eps=eps, gamma=gamma, out=out, workspace=workspace, stream=stream)
+    if op_name == "hla2d":
+        if gamma is None:
+            raise ValueError("hla2d needs gamma")
+        return hla2(q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
+    if op_name == "ahla":
+        return ahla(q, k, v, out=out, workspace=workspace, stream=stream)
+    if op_name == "hla3":
+        return hla3(q, k, v, out=out, workspace=workspace, stream=stream)
+    raise ValueError(op_name)
+
+
+OP_CODES = {"hla2": OP_HLA2, "hla2n": OP_HLA2_NORM, "hla2d": OP_HLA2, "ahla": OP_AHLA, "hla3": OP_HLA3}
+
+
+def read_device_status(workspace, stream=None) -> int:
+    """Synchronise and return the device status word of the last call on ``workspace``."""
+    torch = _torch()
+    st = stream if stream is not None else torch.cuda.current_stream(workspace.device)
+    s = ctypes.c_int(-1)
+    rc = load_library().hla_read_device_status(ctypes.c_void_p(workspace.data_ptr()),
+                                                ctypes.c_void_p(st.cuda_stream), ctypes.byref(s))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla_read_device_status")
+    return s.value
+
+
+def forward_profiled(op_name: str, q, k, v, events, gamma=None, eps: float = 1e-6, out=None, workspace=None,
+                     stream=None):
+    """Same as :func:`forward` through ``hla_forward_profiled``: ``events`` are four recorded-once
+    ``torch.cuda.Event(enable_timing=True)`` objects the library records before the summary kernel,
+    after it, after the scan and after the output kernel (on the call's stream)."""
+    torch = _torch()
+    _check(q, k, v)
+    lib = load_library()
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=torch.float32, device=q.device)
+    op = OP_CODES[op_name]
+    if workspace is None:
+        workspace = make_workspace(op, q, v, decayed=gamma is not None)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    handles = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    rc = lib.hla_forward_profiled(
+        op, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+        ctypes.c_void_p(out.data_ptr()), B, H, T, d, dv, _dtype_code(q),
+        ctypes.c_void_p(gamma.data_ptr()) if gamma is not None else ctypes.c_void_p(0), ctypes.c_float(eps),
+        ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()),
+        ctypes.c_void_p(st.cuda_stream), ctypes.cast(handles, ctypes.c_void_p))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla_forward_profiled rejected the call")
+    return out

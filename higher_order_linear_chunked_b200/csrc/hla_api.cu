@@ -1,0 +1,175 @@
+// C ABI of the HLA forward library: argument checks, workspace sizing, path choice, launches.
+// Declarations and the contract of every entry point: include/hla.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hla.h"
+#include "common.cuh"
+#include "simt.h"
+#include "tc.h"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Request {
+    int op;        // internal op id
+    bool norm;     // ratio-normalised
+    bool bf16;
+    int B, H, T, d, dv;
+};
+
+// Shape / dtype checks shared by the size query and the forward calls.
+hla_status_t check_shape(hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
+    if (dtype != HLA_F32 && dtype != HLA_BF16) return HLA_ERR_DTYPE;
+    if (B < 1 || H < 1 || T < 1 || d < 1 || dv < 1) return HLA_ERR_SHAPE;
+    if ((long long)B * H * T >= (1LL << 31)) return HLA_ERR_SHAPE;
+    if (d != dv) return HLA_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64) return HLA_ERR_UNSUPPORTED;
+    return HLA_OK;
+}
+
+Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
+    Request r{};
+    r.norm = (op == HLA_OP_HLA2_NORM);
+    r.bf16 = (dtype == HLA_BF16);
+    if (op == HLA_OP_HLA2 || op == HLA_OP_HLA2_NORM) r.op = decayed ? hla::OP_HLA2D : hla::OP_HLA2;
+    else if (op == HLA_OP_AHLA) r.op = hla::OP_AHLA;
+    else r.op = hla::OP_HLA3;
+    r.B = B; r.H = H; r.T = T; r.d = d; r.dv = dv;
+    return r;
+}
+
+bool use_tc(const Request& r) { return hla::tc::supported(r.op, r.norm, r.bf16, r.d); }
+
+size_t workspace_for(const Request& r) {
+    const int BH = r.B * r.H;
+    if (use_tc(r)) return hla::kStatusBytes + hla::tc::workspace_bytes(r.op, r.norm, BH, r.T);
+    return hla::kStatusBytes + sizeof(float) * hla::simt::workspace_floats(r.op, r.d, BH, r.T);
+}
+
+hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, float* o, int B, int H, int T,
+                     int d, int dv, hla_dtype_t dtype, const float* gamma, float eps, void* workspace,
+                     size_t workspace_bytes, void* stream, void* const* phase_events = nullptr) {
+    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o) return HLA_ERR_NULL;
+    hla_status_t s = check_shape(dtype, B, H, T, d, dv);
+    if (s != HLA_OK) return s;
+    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HLA_ERR_ALIGN;
+    if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
+    const Request r = make_request(op, gamma != nullptr, dtype, B, H, T, d, dv);
+    if (!workspace) return HLA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HLA_ERR_ALIGN;
+    if (workspace_bytes < workspace_for(r)) return HLA_ERR_WORKSPACE;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
+    char* body = static_cast<char*>(workspace) + hla::kStatusBytes;
+    cudaEvent_t* ev = phase_events ? reinterpret_cast<cudaEvent_t*>(const_cast<void**>(phase_events)) : nullptr;
+    cudaError_t e;
+    if (use_tc(r)) {
+        e = hla::tc::forward(r.op, r.norm, q, k, v, eps, o, B * H, T, body, status, st, ev);
+    } else {
+        e = hla::simt::forward(r.op, r.norm, r.bf16, r.d, q, k, v, gamma, eps, o, B * H, H, T,
+                               reinterpret_cast<float*>(body), st, ev);
+    }
+    return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hla_abi_version(void) { return kAbiVersion; }
+
+const char* hla_status_str(hla_status_t s) {
+    switch (s) {
+    case HLA_OK: return "HLA_OK";
+    case HLA_ERR_NULL: return "HLA_ERR_NULL: a required pointer is NULL";
+    case HLA_ERR_SHAPE: return "HLA_ERR_SHAPE: B, H, T, d or dv out of range";
+    case HLA_ERR_ALIGN: return "HLA_ERR_ALIGN: a base address is not 16-byte aligned";
+    case HLA_ERR_DTYPE: return "HLA_ERR_DTYPE: unknown dtype";
+    case HLA_ERR_UNSUPPORTED: return "HLA_ERR_UNSUPPORTED: no kernel for this (op, dtype, d, dv, gamma)";
+    case HLA_ERR_WORKSPACE: return "HLA_ERR_WORKSPACE: workspace missing or too small";
+    case HLA_ERR_CUDA: return "HLA_ERR_CUDA: a CUDA call or launch failed";
+    case HLA_ERR_TIMEOUT: return "HLA_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    }
+    return "unknown hla_status_t";
+}
+
+size_t hla_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
+    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return 0;
+    if (check_shape(dtype, B, H, T, d, dv) != HLA_OK) return 0;
+    if (decayed && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return 0;
+    return workspace_for(make_request(op, decayed != 0, dtype, B, H, T, d, dv));
+}
+
+int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
+    if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
+    const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
+    if (use_tc(r)) return hla::tc::kernel_launches(r.op, r.norm, B * H, T);
+    return hla::simt::kernel_launches(T);
+}
+
+int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
+    if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
+    return use_tc(make_request(op, decayed != 0, dtype, B, H, T, d, dv)) ? 1 : 0;
+}
+
+hla_status_t hla2_forward(const void* q, const void* k, const void* v, float* o, int B, int H, int T, int d,
+                          int dv, hla_dtype_t dtype, const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    return forward(HLA_OP_HLA2, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace, workspace_bytes, stream);
+}
+
+hla_status_t hla2_forward_normalized(const void* q, const void* k, const void* v, float* o, int B, int H, int T,
+                                     int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    return forward(HLA_OP_HLA2_NORM, q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, workspace, workspace_bytes,
+                   stream);
+}
+
+hla_status_t ahla_forward(const void* q, const void* k, const void* v, float* o, int B, int H, int T, int d,
+                          int dv, hla_dtype_t dtype, const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    return forward(HLA_OP_AHLA, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace, workspace_bytes, stream);
+}
+
+hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o, int B, int H, int T, int d,
+                          int dv, hla_dtype_t dtype, const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    return forward(HLA_OP_HLA3, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace, workspace_bytes, stream);
+}
+
+hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, const void* v, float* o, int B,
+                                  int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
+                                  void* workspace, size_t workspace_bytes, void* stream,
+                                  void* const* phase_events) {
+    return forward(op, q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, workspace, workspace_bytes, stream,
+                   phase_events);
+}
+
+hla_status_t hla_read_device_status(const void* workspace, void* stream, int* device_status) {
+    if (!workspace || !device_status) return HLA_ERR_NULL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HLA_ERR_CUDA;
+    int s = 0;
+    if (cudaMemcpy(&s, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return HLA_ERR_CUDA;
+    *device_status = s;
+    return HLA_OK;
+}
+
+hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, float* d, int N, int K,
+                               void* stream) {
+    if (!a || !b || !d) return HLA_ERR_NULL;
+    if (layout_case < 0 || layout_case > 3) return HLA_ERR_UNSUPPORTED;
+    if ((N != 64 && N != 128) || (K != 64 && K != 128)) return HLA_ERR_SHAPE;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return HLA_ERR_ALIGN;
+    cudaError_t e = hla::tc::selftest(layout_case, a, b, d, N, K, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,635 @@
+// CUDA-core (FFMA, fp32) chunk-parallel path for every HLA op.
+//
+// "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 4:
+// the sequence is cut into chunks; each chunk's summary is built on its own
+// (chunk kernel), a Blelloch exclusive scan with the semidirect-product combine
+// turns them into carried-in prefixes (scan kernel, one launch per tree level),
+// and each chunk's output applies its prefix (output kernel).  This path serves
+// the fp32 workloads (whose tolerance rules out single-pass TF32 tensor cores),
+// every op at d in {32, 64}, and bf16 inputs the tcgen05 path does not cover.
+//
+// Per chunk (c tokens, local 0-based index; A* = Q K^T, A = L (.) A*):
+//   second order   summary  S = K^T K, C = Q^T V, m = Q^T 1,
+//                           R = S C - G = K^T (A^T V), r = S m - h = K^T (A^T 1)
+//                  combine  R_AB = R_A + R_B + S_A C_B, r_AB = r_A + r_B + S_A m_B
+//                  output   W = L (.) (Q S0 Q^T + A A^T), O = Q R0 + W V,
+//                           den = Q r0 + W 1 (ratio-normalised)
+//   decayed        state (S, C, G, Khat, m, h, rho), rho = gamma^len, Khat = K^T K;
+//                  combine and output formulas in combine_into / k_output below
+//   AHLA           summary  P = K^T V, Dm = K^T Q, E = K^T (A V);
+//                  combine  E_AB = E_A + E_B + Dm_B P_A; output O = Q E0 + A (Q P0 + A V)
+//   third order    summary  S, Q2 = Q^T Q, P, X = Q^T (A V), Z = K^T (A^T Q),
+//                           F = K^T (A^T (A V));
+//                  output   W as above, O = Q F0 + W (Q P0 + A V)
+#include "common.cuh"
+#include "simt.h"
+
+namespace hla {
+namespace simt {
+
+constexpr int C = 64;        // chunk length
+constexpr int LDC = C + 1;   // padded row stride of c x c tiles in shared memory
+constexpr int NT = 256;      // threads per block
+
+template <int D>
+struct Dim {
+    static constexpr int LD = D + 1;  // padded row stride of c x D / D x D tiles
+};
+
+// ---------------------------------------------------------------------------
+// Summary layout: NMAT matrices D x D, then NVEC vectors D, then one scalar.
+// ---------------------------------------------------------------------------
+template <int OP, int D>
+struct Sum {
+    static constexpr int DD = D * D;
+    static constexpr int NMAT = OP == OP_HLA3 ? 6 : OP == OP_HLA2D ? 4 : 3;
+    static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D) ? 2 : 0;
+    static constexpr int VEC0 = NMAT * DD;
+    static constexpr int SCAL = VEC0 + NVEC * D;
+    static constexpr int SIZE = (SCAL + 4 + 31) / 32 * 32;
+    __host__ __device__ static constexpr int mat(int i) { return i * DD; }
+    __host__ __device__ static constexpr int vec(int i) { return VEC0 + i * D; }
+};
+// Matrix / vector slots.
+//   OP_HLA2 : S=0 C=1 R=2 ; m=0 r=1
+//   OP_HLA2D: S=0 C=1 G=2 Khat=3 ; m=0 h=1 ; scalar rho
+//   OP_AHLA : P=0 E=1 Dm=2
+//   OP_HLA3 : S=0 Q2=1 P=2 F=3 X=4 Z=5
+
+size_t summary_floats(int op, int d) {
+    switch (op) {
+    case OP_HLA2: return d == 32 ? Sum<OP_HLA2, 32>::SIZE : Sum<OP_HLA2, 64>::SIZE;
+    case OP_HLA2D: return d == 32 ? Sum<OP_HLA2D, 32>::SIZE : Sum<OP_HLA2D, 64>::SIZE;
+    case OP_AHLA: return d == 32 ? Sum<OP_AHLA, 32>::SIZE : Sum<OP_AHLA, 64>::SIZE;
+    case OP_HLA3: return d == 32 ? Sum<OP_HLA3, 32>::SIZE : Sum<OP_HLA3, 64>::SIZE;
+    }
+    return 0;
+}
+
+// ---------------------------------------------------------------------------
+// Block-cooperative small matrix products in shared/global memory.
+//   out(m,n) = init(m,n) + sum_k a1(m,k) b1(k,n) [+ sum_k a2(m,k) b2(k,n) ...]
+// Thread owns the 4x4 outputs (tm + i*M/4, tn + j*N/4): a() reads are
+// broadcasts within a warp, b() reads walk consecutive n (conflict-free).
+// ---------------------------------------------------------------------------
+struct Zero {
+    __device__ float operator()(int, int) const { return 0.f; }
+};
+
+template <int M, int N, int K1, int K2, int K3, class A1, class B1, class A2, class B2, class A3,
+          class B3, class FI, class FS>
+__device__ __forceinline__ void mm3(A1 a1, B1 b1, A2 a2, B2 b2, A3 a3, B3 b3, FI init, FS store) {
+    static_assert(M % 4 == 0 && N % 4 == 0, "tile");
+    constexpr int RM = M / 4, RN = N / 4;
+    for (int tile = threadIdx.x; tile < RM * RN; tile += blockDim.x) {
+        const int tm = tile / RN, tn = tile % RN;
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = init(tm + i * RM, tn + j * RN);
+#pragma unroll 4
+        for (int kk = 0; kk < K1; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) av[i] = a1(tm + i * RM, kk);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bv[j] = b1(kk, tn + j * RN);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+#pragma unroll 4
+        for (int kk = 0; kk < K2; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) av[i] = a2(tm + i * RM, kk);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bv[j] = b2(kk, tn + j * RN);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+#pragma unroll 4
+        for (int kk = 0; kk < K3; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) av[i] = a3(tm + i * RM, kk);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bv[j] = b3(kk, tn + j * RN);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) store(tm + i * RM, tn + j * RN, acc[i][j]);
+    }
+}
+
+template <int M, int N, int K, class A1, class B1, class FI, class FS>
+__device__ __forceinline__ void mm(A1 a, B1 b, FI init, FS store) {
+    mm3<M, N, K, 0, 0>(a, b, a, b, a, b, init, store);
+}
+
+template <int M, int N, int K1, int K2, class A1, class B1, class A2, class B2, class FI, class FS>
+__device__ __forceinline__ void mm2(A1 a1, B1 b1, A2 a2, B2 b2, FI init, FS store) {
+    mm3<M, N, K1, K2, 0>(a1, b1, a2, b2, a1, b1, init, store);
+}
+
+// Row-major shared tile accessors.
+struct Tile {                      // element (r, c) of a tile with row stride ld
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[r * ld + c]; }
+};
+struct TileT {                     // transposed view: element (r, c) = tile[c][r]
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[c * ld + r]; }
+};
+struct Put {                    // plain store into a tile
+    float* p;
+    int ld;
+    __device__ void operator()(int r, int c, float x) const { p[r * ld + c] = x; }
+};
+
+// Load `rows` chunk rows (zero beyond T) of a [T][D] head slice into a padded fp32 tile.
+template <int D, typename TIn>
+__device__ __forceinline__ void load_rows(float* dst, const TIn* src, int t0, int T) {
+    constexpr int LD = Dim<D>::LD;
+    for (int e = threadIdx.x; e < C * D; e += blockDim.x) {
+        const int r = e / D, c = e % D;
+        const int t = t0 + r;
+        dst[r * LD + c] = (t < T) ? to_f32(src[(size_t)t * D + c]) : 0.f;
+    }
+}
+
+// Load a D x D matrix (global, dense) into a padded tile; `scale` applied.
+template <int D>
+__device__ __forceinline__ void load_mat(float* dst, const float* src) {
+    constexpr int LD = Dim<D>::LD;
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) dst[(e / D) * LD + (e % D)] = src[e];
+}
+
+__device__ __forceinline__ float gpow(float g, int n) {  // gamma^n, n >= 0
+    return n == 0 ? 1.f : powf(g, (float)n);
+}
+
+// Identity element of each op's combine: zeros, rho = 1.
+template <int OP, int D>
+__device__ void write_identity(float* out) {
+    using S = Sum<OP, D>;
+    for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) out[e] = (OP == OP_HLA2D && e == S::SCAL) ? 1.f : 0.f;
+}
+
+// ---------------------------------------------------------------------------
+// Chunk kernel: one block per (chunk, head); writes the chunk's summary.
+// Slots NC..NCp-1 (scan padding) receive the identity.
+// ---------------------------------------------------------------------------
+template <int OP, int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                                const TIn* __restrict__ v, const float* __restrict__ gamma,
+                                                int H, int T, int NC, int NCp, float* __restrict__ sums) {
+    using S = Sum<OP, D>;
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    float* out = sums + ((size_t)bh * NCp + chunk) * S::SIZE;
+    if (chunk >= NC) {
+        write_identity<OP, D>(out);
+        return;
+    }
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Ks = Qs + C * LD;
+    float* Vs = Ks + C * LD;
+    float* As = Vs + C * LD;      // C x LDC
+    float* Ys = As + C * LDC;     // C x LD
+    float* Y2 = Ys + C * LD;      // C x LD
+    float* us = Y2 + C * LD;      // C
+    float* lam = us + C;          // C  (decay weights)
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Ks, k + head, t0, T);
+    load_rows<D>(Vs, v + head, t0, T);
+    float g = 1.f;
+    if (OP == OP_HLA2D) {
+        g = gamma[bh % H];
+        for (int j = threadIdx.x; j < C; j += blockDim.x) lam[j] = gpow(g, C - 1 - j);  // gamma^(len - tau)
+    }
+    __syncthreads();
+    // A* = Q K^T (masked to A = L (.) A* except for the decayed op, which needs both parts)
+    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
+        As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
+    });
+    __syncthreads();
+
+    auto store_mat = [&](int slot) {
+        return [=](int r, int c, float x) { out[S::mat(slot) + r * D + c] = x; };
+    };
+
+    if (OP == OP_HLA2) {
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(0));        // S = K^T K
+        mm<D, D, C>(TileT{Qs, LD}, Tile{Vs, LD}, Zero{}, store_mat(1));        // C = Q^T V
+        mm<C, D, C>(TileT{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});        // Y = A^T V
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {              // u = A^T 1
+            float s = 0.f;
+            for (int j = 0; j < C; ++j) s += As[j * LDC + i];
+            us[i] = s;
+        }
+        __syncthreads();
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ys, LD}, Zero{}, store_mat(2));        // R = K^T Y
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sr = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Qs[i * LD + a];
+                sr += Ks[i * LD + a] * us[i];
+            }
+            out[S::vec(0) + a] = sm_;                                    // m = Q^T 1
+            out[S::vec(1) + a] = sr;                                     // r = K^T (A^T 1)
+        }
+    } else if (OP == OP_HLA2D) {
+        // S = K^T diag(lam) K, C = Q^T diag(lam) V, Khat = K^T K
+        mm<D, D, C>([&](int r, int c) { return Ks[c * LD + r] * lam[c]; }, Tile{Ks, LD}, Zero{}, store_mat(0));
+        mm<D, D, C>([&](int r, int c) { return Qs[c * LD + r] * lam[c]; }, Tile{Vs, LD}, Zero{}, store_mat(1));
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(3));
+        // Y_G[i] = sum_{j<i} (q_j.k_i) lam_j v_j ;  u_i = sum_{j<i} (q_j.k_i) lam_j
+        auto ug = [&](int i, int j) { return j < i ? As[j * LDC + i] * lam[j] : 0.f; };
+        mm<C, D, C>(ug, Tile{Vs, LD}, Zero{}, Put{Ys, LD});
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+            float s = 0.f;
+            for (int j = 0; j < i; ++j) s += As[j * LDC + i] * lam[j];
+            us[i] = s;
+        }
+        __syncthreads();
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ys, LD}, Zero{}, store_mat(2));        // G = K^T Y_G
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sh = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Qs[i * LD + a] * lam[i];
+                sh += Ks[i * LD + a] * us[i];
+            }
+            out[S::vec(0) + a] = sm_;                                    // m
+            out[S::vec(1) + a] = sh;                                     // h = K^T u
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = gpow(g, C);                 // rho = gamma^len
+    } else if (OP == OP_AHLA) {
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Vs, LD}, Zero{}, store_mat(0));        // P = K^T V
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Qs, LD}, Zero{}, store_mat(2));        // Dm = K^T Q
+        mm<C, D, C>(Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});         // Y = A V
+        __syncthreads();
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ys, LD}, Zero{}, store_mat(1));        // E = K^T Y
+    } else {  // OP_HLA3
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(0));        // S
+        mm<D, D, C>(TileT{Qs, LD}, Tile{Qs, LD}, Zero{}, store_mat(1));        // Q2
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Vs, LD}, Zero{}, store_mat(2));        // P
+        mm<C, D, C>(Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});         // Yl = A V
+        mm<C, D, C>(TileT{As, LDC}, Tile{Qs, LD}, Zero{}, Put{Y2, LD});        // A^T Q
+        __syncthreads();
+        mm<D, D, C>(TileT{Qs, LD}, Tile{Ys, LD}, Zero{}, store_mat(4));        // X = Q^T Yl
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Y2, LD}, Zero{}, store_mat(5));        // Z = K^T (A^T Q)
+        __syncthreads();
+        mm<C, D, C>(TileT{As, LDC}, Tile{Ys, LD}, Zero{}, Put{Y2, LD});        // A^T Yl
+        __syncthreads();
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Y2, LD}, Zero{}, store_mat(3));        // F = K^T (A^T Yl)
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Scan kernel: one Blelloch level; one block per (pair, head).
+//   up-sweep:   X[R] = X[L] o X[R]
+//   down-sweep: X[L], X[R] = X[R], X[R] o X[L]   (root: X[R] read as identity)
+// combine(A, B) summarises "A then B".
+// ---------------------------------------------------------------------------
+template <int OP, int D>
+__device__ void combine_into(const float* A, const float* B, float* out, float* tmp) {
+    using S = Sum<OP, D>;
+    constexpr int DD = D * D;
+    auto G = [](const float* p, int slot) { return Tile{p + S::mat(slot), D}; };
+    auto add2 = [&](int slot) {
+        for (int e = threadIdx.x; e < DD; e += blockDim.x) out[S::mat(slot) + e] = A[S::mat(slot) + e] + B[S::mat(slot) + e];
+    };
+    auto dst = [&](int slot) {
+        return [=](int r, int c, float x) { out[S::mat(slot) + r * D + c] = x; };
+    };
+    if (OP == OP_HLA2) {
+        add2(0);
+        add2(1);
+        mm<D, D, D>(G(A, 0), G(B, 1),
+                    [&](int r, int c) { return A[S::mat(2) + r * D + c] + B[S::mat(2) + r * D + c]; }, dst(2));
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float s = 0.f;
+            for (int b = 0; b < D; ++b) s += A[S::mat(0) + a * D + b] * B[S::vec(0) + b];
+            out[S::vec(0) + a] = A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = A[S::vec(1) + a] + B[S::vec(1) + a] + s;
+        }
+    } else if (OP == OP_HLA2D) {
+        const float rb = B[S::SCAL];
+        for (int e = threadIdx.x; e < DD; e += blockDim.x) {
+            out[S::mat(0) + e] = rb * A[S::mat(0) + e] + B[S::mat(0) + e];
+            out[S::mat(1) + e] = rb * A[S::mat(1) + e] + B[S::mat(1) + e];
+            out[S::mat(3) + e] = A[S::mat(3) + e] + B[S::mat(3) + e];
+        }
+        mm<D, D, D>([&](int r, int c) { return rb * B[S::mat(3) + r * D + c]; }, G(A, 1),
+                    [&](int r, int c) { return rb * A[S::mat(2) + r * D + c] + B[S::mat(2) + r * D + c]; },
+                    dst(2));
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float s = 0.f;
+            for (int b = 0; b < D; ++b) s += B[S::mat(3) + a * D + b] * A[S::vec(0) + b];
+            out[S::vec(0) + a] = rb * A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = rb * A[S::vec(1) + a] + B[S::vec(1) + a] + rb * s;
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = A[S::SCAL] * rb;
+    } else if (OP == OP_AHLA) {
+        add2(0);
+        add2(2);
+        mm<D, D, D>(G(B, 2), G(A, 0),
+                    [&](int r, int c) { return A[S::mat(1) + r * D + c] + B[S::mat(1) + r * D + c]; }, dst(1));
+    } else {  // OP_HLA3
+        // tmp = S_A Q2_B
+        mm<D, D, D>(G(A, 0), G(B, 1), Zero{}, [&](int r, int c, float x) { tmp[r * D + c] = x; });
+        __syncthreads();
+        add2(0);
+        add2(1);
+        add2(2);
+        for (int e = threadIdx.x; e < DD; e += blockDim.x) out[S::mat(5) + e] = A[S::mat(5) + e] + B[S::mat(5) + e] + tmp[e];
+        mm<D, D, D>(G(B, 1), G(A, 2),
+                    [&](int r, int c) { return A[S::mat(4) + r * D + c] + B[S::mat(4) + r * D + c]; }, dst(4));
+        mm3<D, D, D, D, D>(Tile{tmp, D}, G(A, 2), G(A, 0), G(B, 4), G(B, 5), G(A, 2),
+                           [&](int r, int c) { return A[S::mat(3) + r * D + c] + B[S::mat(3) + r * D + c]; },
+                           dst(3));
+    }
+}
+
+template <int OP, int D>
+__global__ void __launch_bounds__(NT) k_scan_level(float* __restrict__ sums, int NCp, int step, int down, int root) {
+    using S = Sum<OP, D>;
+    extern __shared__ float sm[];
+    float* As = sm;
+    float* Bs = As + S::SIZE;
+    float* tmp = Bs + S::SIZE;
+    const int pair = blockIdx.x, bh = blockIdx.y;
+    const int L = pair * 2 * step + step - 1, R = pair * 2 * step + 2 * step - 1;
+    float* base = sums + (size_t)bh * NCp * S::SIZE;
+    float* XL = base + (size_t)L * S::SIZE;
+    float* XR = base + (size_t)R * S::SIZE;
+    if (!down) {
+        for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) {
+            As[e] = XL[e];
+            Bs[e] = XR[e];
+        }
+        __syncthreads();
+        combine_into<OP, D>(As, Bs, XR, tmp);
+    } else {
+        // A = parent prefix (X[R], identity at the root), B = left subtree total (X[L])
+        if (root) write_identity<OP, D>(As);
+        else
+            for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) As[e] = XR[e];
+        for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) Bs[e] = XL[e];
+        __syncthreads();
+        for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) XL[e] = As[e];
+        combine_into<OP, D>(As, Bs, XR, tmp);
+    }
+}
+
+template <int OP, int D>
+__global__ void k_identity(float* sums, int NCp) {
+    using S = Sum<OP, D>;
+    write_identity<OP, D>(sums + (size_t)blockIdx.x * NCp * S::SIZE);
+}
+
+// ---------------------------------------------------------------------------
+// Output kernel: one block per (chunk, head); applies the chunk's prefix.
+// ---------------------------------------------------------------------------
+template <int OP, bool NORM, int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                               const TIn* __restrict__ v, const float* __restrict__ gamma,
+                                               float eps, int H, int T, int NCp, const float* __restrict__ sums,
+                                               float* __restrict__ o) {
+    using S = Sum<OP, D>;
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const float* pre = sums + ((size_t)bh * NCp + chunk) * S::SIZE;
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Ks = Qs + C * LD;
+    float* Vs = Ks + C * LD;
+    float* As = Vs + C * LD;      // C x LDC
+    float* Ws = As + C * LDC;     // C x LDC
+    float* Ps = Ws + C * LDC;     // C x LD
+    float* Ys = Ps + C * LD;      // C x LD
+    float* M0 = Ys + C * LD;      // D x LD  (prefix matrices)
+    float* M1 = M0 + D * LD;
+    float* M2 = M1 + D * LD;
+    float* vec = M2 + D * LD;     // 2 D
+    float* den = vec + 2 * D;     // C
+    float* gp = den + C;          // C + 1
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Ks, k + head, t0, T);
+    load_rows<D>(Vs, v + head, t0, T);
+    float g = 1.f;
+    if (OP == OP_HLA2) {
+        load_mat<D>(M0, pre + S::mat(0));   // S0
+        load_mat<D>(M1, pre + S::mat(2));   // R0
+        for (int a = threadIdx.x; a < D; a += blockDim.x) vec[a] = pre[S::vec(1) + a];  // r0
+    } else if (OP == OP_HLA2D) {
+        load_mat<D>(M0, pre + S::mat(0));   // S0
+        load_mat<D>(M1, pre + S::mat(1));   // C0
+        load_mat<D>(M2, pre + S::mat(2));   // G0
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            vec[a] = pre[S::vec(0) + a];      // m0
+            vec[D + a] = pre[S::vec(1) + a];  // h0
+        }
+        g = gamma[bh % H];
+        for (int j = threadIdx.x; j <= C; j += blockDim.x) gp[j] = gpow(g, j);
+    } else if (OP == OP_AHLA) {
+        load_mat<D>(M0, pre + S::mat(0));   // P0
+        load_mat<D>(M1, pre + S::mat(1));   // E0
+    } else {
+        load_mat<D>(M0, pre + S::mat(0));   // S0
+        load_mat<D>(M1, pre + S::mat(2));   // P0
+        load_mat<D>(M2, pre + S::mat(3));   // F0
+    }
+    __syncthreads();
+    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
+        As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
+    });
+    if (OP == OP_HLA2 || OP == OP_HLA3)
+        mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, Put{Ps, LD});                      // P = Q S0
+    if (OP == OP_HLA2D)
+        mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, [&](int r, int c, float x) {         // P~ = Gamma Q S0
+            Ps[r * LD + c] = gp[r + 1] * x;
+        });
+    __syncthreads();
+
+    const size_t obase = ((size_t)bh * T + t0) * D;
+    auto emit = [&](int r, int c, float x) {
+        if (t0 + r < T) o[obase + (size_t)r * D + c] = NORM ? x / (den[r] + eps) : x;
+    };
+
+    if (OP == OP_HLA2) {
+        // W = L (.) (P Q^T + A A^T)
+        mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Tile{As, LDC}, TileT{As, LDC}, Zero{},
+                        [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
+        __syncthreads();
+        if (NORM) {
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[a];
+                for (int j = 0; j <= r; ++j) s += Ws[r * LDC + j];
+                den[r] = s;
+            }
+            __syncthreads();
+        }
+        mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{Ws, LDC}, Tile{Vs, LD}, Zero{}, emit);   // O = Q R0 + W V
+    } else if (OP == OP_HLA2D) {
+        // W_tj = [j<=t] g^(t-j) ( g^(t+1) (P Q^T)_tj + sum_{i<=t} A*_ti A*_ji (g^(t-i) - [i>j]) )
+        //      = [j<=t] g^(t-j) ( (P~ Q^T) + (A~ A*^T) - (A U^T) )_tj
+        auto At = [&](int r, int c) { return c <= r ? gp[r - c] * As[r * LDC + c] : 0.f; };   // A~
+        auto Am = [&](int r, int c) { return c <= r ? -As[r * LDC + c] : 0.f; };            // -A
+        auto Ut = [&](int kk, int n) { return kk > n ? As[n * LDC + kk] : 0.f; };           // U^T
+        mm3<C, C, D, C, C>(Tile{Ps, LD}, TileT{Qs, LD}, At, TileT{As, LDC}, Am, Ut, Zero{},
+                           [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? gp[r - c] * x : 0.f; });
+        // Z' = P~ + (A~ - A) K
+        mm<C, D, C>([&](int r, int c) { return c <= r ? (gp[r - c] - 1.f) * As[r * LDC + c] : 0.f; },
+                    Tile{Ks, LD}, Tile{Ps, LD}, Put{Ys, LD});
+        __syncthreads();
+        if (NORM) {
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f, zm = 0.f, qh = 0.f;
+                for (int j = 0; j <= r; ++j) s += Ws[r * LDC + j];
+                for (int a = 0; a < D; ++a) {
+                    zm += Ys[r * LD + a] * vec[a];
+                    qh += Qs[r * LD + a] * vec[D + a];
+                }
+                den[r] = s + gp[r + 1] * (zm - qh);
+            }
+            __syncthreads();
+        }
+        // O = W V + Gamma Z' C0 - Gamma Q G0
+        mm3<C, D, C, D, D>(Tile{Ws, LDC}, Tile{Vs, LD},
+                           [&](int r, int c) { return gp[r + 1] * Ys[r * LD + c]; }, Tile{M1, LD},
+                           [&](int r, int c) { return -gp[r + 1] * Qs[r * LD + c]; }, Tile{M2, LD}, Zero{}, emit);
+    } else if (OP == OP_AHLA) {
+        mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M0, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y = Q P0 + A V
+        __syncthreads();
+        mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{As, LDC}, Tile{Ys, LD}, Zero{}, emit);          // O = Q E0 + A Y
+    } else {  // OP_HLA3
+        mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Tile{As, LDC}, TileT{As, LDC}, Zero{},
+                        [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
+        mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y = Q P0 + A V
+        __syncthreads();
+        mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M2, LD}, Tile{Ws, LDC}, Tile{Ys, LD}, Zero{}, emit);          // O = Q F0 + W Y
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+static int next_pow2(int n) {
+    int p = 1;
+    while (p < n) p *= 2;
+    return p;
+}
+
+template <int D>
+static size_t summary_smem() {
+    constexpr int LD = Dim<D>::LD;
+    return sizeof(float) * (size_t)(3 * C * LD + C * LDC + 2 * C * LD + 2 * C);
+}
+template <int D>
+static size_t output_smem() {
+    constexpr int LD = Dim<D>::LD;
+    return sizeof(float) * (size_t)(3 * C * LD + 2 * C * LDC + 2 * C * LD + 3 * D * LD + 2 * D + 2 * C + 1);
+}
+template <int OP, int D>
+static size_t scan_smem() {
+    return sizeof(float) * (size_t)(2 * Sum<OP, D>::SIZE + D * D);
+}
+
+int kernel_launches(int T) {
+    const int NCp = next_pow2((T + C - 1) / C);
+    int levels = 0;
+    for (int p = 1; p < NCp; p *= 2) ++levels;
+    return 2 + (NCp == 1 ? 1 : 2 * levels);
+}
+
+size_t workspace_floats(int op, int d, int BH, int T) {
+    const int NC = (T + C - 1) / C;
+    return (size_t)BH * next_pow2(NC) * summary_floats(op, d);
+}
+
+template <int OP, bool NORM, int D, typename TIn>
+static cudaError_t run(const void* q, const void* k, const void* v, const float* gamma, float eps, float* o,
+                       int BH, int H, int T, float* sums, cudaStream_t st, cudaEvent_t* ev) {
+    const int NC = (T + C - 1) / C;
+    const int NCp = next_pow2(NC);
+    auto ks = k_summary<OP, D, TIn>;
+    auto kl = k_scan_level<OP, D>;
+    auto ko = k_output<OP, NORM, D, TIn>;
+    const size_t s1 = summary_smem<D>(), s2 = scan_smem<OP, D>(), s3 = output_smem<D>();
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
+    ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, H, T, NC, NCp, sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
+    if (NCp == 1) {
+        k_identity<OP, D><<<BH, NT, 0, st>>>(sums, NCp);
+    } else {
+        for (int step = 1; step < NCp; step *= 2) {
+            kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 0, 0);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        for (int step = NCp / 2; step >= 1; step /= 2) {
+            kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 1, step == NCp / 2);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
+    ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H, T, NCp, sums, o);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
+    return cudaSuccess;
+}
+
+template <typename TIn, int D>
+static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma,
+                               float eps, float* o, int BH, int H, int T, float* sums, cudaStream_t st,
+                               cudaEvent_t* ev) {
+    switch (op) {
+    case OP_HLA2:
+        return norm ? run<OP_HLA2, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_HLA2, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_HLA2D:
+        return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_AHLA: return run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_HLA3: return run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,
+                    const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, cudaStream_t st,
+                    cudaEvent_t* ev) {
+    if (bf16) {
+        if (d == 32) return dispatch_op<__nv_bfloat16, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return dispatch_op<__nv_bfloat16, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    }
+    if (d == 32) return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+}
+
+}  // namespace simt
+}  // namespace hla

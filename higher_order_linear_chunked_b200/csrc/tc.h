@@ -1,0 +1,22 @@
+// tcgen05 (5th-generation tensor core) path: declarations used by the C ABI layer.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace hla {
+namespace tc {
+
+// true when (internal op, normalised, bf16, d) runs on the tcgen05 kernels
+bool supported(int op, bool norm, bool bf16, int d);
+// kernels one forward enqueues
+int kernel_launches(int op, bool norm, int BH, int T);
+// workspace bytes the path needs after the status block
+size_t workspace_bytes(int op, bool norm, int BH, int T);
+// enqueue the segment-summary walker, the Blelloch scan levels and the output walker
+cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
+                    int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
+// one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
+cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace hla

@@ -1,0 +1,93 @@
+// tcgen05 layout self-check: one bf16 MMA (M = 128) with K-major / MN-major operands in
+// 128-byte-swizzled shared memory, accumulator read back through tcgen05.ld.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tc.h"
+
+namespace hla {
+namespace tc {
+
+using bf16 = __nv_bfloat16;
+
+// Place element (row r of the operand's M/N extent, column kk along K) of an R x K operand.
+__device__ __forceinline__ uint32_t operand_offset(bool mn_major, int R, int K, int r, int kk) {
+    if (!mn_major) return static_cast<uint32_t>((kk / 64) * (R * 128)) + ptx::sw128_offset(r, kk % 64);
+    return static_cast<uint32_t>((r / 64) * (K * 128)) + ptx::sw128_offset(kk, r % 64);
+}
+
+// Descriptor of K-step s (16 elements) of an R x K operand.
+__device__ __forceinline__ uint64_t operand_desc(bool mn_major, uint32_t base, int R, int K, int s) {
+    if (!mn_major) return ptx::desc_sw128(base + (s / 4) * (R * 128) + (s % 4) * 32, 16, 1024);
+    return ptx::desc_sw128(base + s * 2048, K * 128, 1024);
+}
+
+__global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict__ a, const bf16* __restrict__ b,
+                                                   float* __restrict__ d, int N, int K) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int M = 128;
+    const bool a_mn = (cs & 2) != 0, b_mn = (cs & 1) != 0;
+    uint8_t* As = smem;
+    uint8_t* Bs = smem + M * K * 2;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    for (int e = tid; e < M * K; e += blockDim.x) {
+        int r, kk;
+        if (!a_mn) { r = e / K; kk = e % K; } else { kk = e / M; r = e % M; }
+        const bf16 x = a_mn ? a[kk * M + r] : a[r * K + kk];
+        *reinterpret_cast<bf16*>(As + operand_offset(a_mn, M, K, r, kk)) = x;
+    }
+    for (int e = tid; e < N * K; e += blockDim.x) {
+        int r, kk;
+        if (!b_mn) { r = e / K; kk = e % K; } else { kk = e / N; r = e % N; }
+        const bf16 x = b_mn ? b[kk * N + r] : b[r * K + kk];
+        *reinterpret_cast<bf16*>(Bs + operand_offset(b_mn, N, K, r, kk)) = x;
+    }
+    ptx::fence_proxy_async();
+    if (warp == 0) {
+        ptx::tmem_alloc(&tmem_base, 128);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tbase = tmem_base;
+    if (tid == 0) {
+        const uint32_t idesc = ptx::idesc_bf16(M, N, a_mn, b_mn);
+        const uint32_t abase = ptx::smem_u32(As), bbase = ptx::smem_u32(Bs);
+        for (int s = 0; s < K / 16; ++s)
+            ptx::umma_bf16(tbase, operand_desc(a_mn, abase, M, K, s), operand_desc(b_mn, bbase, N, K, s), idesc,
+                           s > 0);
+        ptx::umma_commit(&bar);
+    }
+    bool ok = ptx::mbar_wait(&bar, 0);
+    if (!ok) ok = ptx::mbar_wait(&bar, 0);  // second bounded wait before touching TMEM
+    ptx::tc_fence_after();
+    const uint32_t taddr = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    for (int col = 0; col < N; col += 16) {
+        float v[16];
+        ptx::tmem_ld16(taddr + col, v);
+        for (int i = 0; i < 16; ++i) d[(warp * 32 + lane) * N + col + i] = ok ? v[i] : __int_as_float(0x7fc00000);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) ptx::tmem_dealloc(tbase, 128);
+}
+
+cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st) {
+    const int smem = 128 * K * 2 + N * K * 2 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_selftest, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_selftest<<<1, 128, smem, st>>>(layout_case, static_cast<const bf16*>(a), static_cast<const bf16*>(b), d, N, K);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace hla

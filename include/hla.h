@@ -1,0 +1,171 @@
+/*
+ * hla.h - C ABI of the B200 (sm_100a) masked Higher-order Linear Attention forward.
+ *
+ * The operations are those of "Resumen Técnico: Atención Lineal de Orden
+ * Superior (HLA)" (gist.science, paper 2510.27258):
+ *
+ *   hla2_forward            Metodología 1: second-order masked output
+ *                           o_t = q_t^T (S^K_t C^QV_t - G_t)
+ *                               = sum_{j<=t} sum_{i<=j} (q_t.k_i)(q_j.k_i) v_j.
+ *                           With gamma != NULL: the masked operator with
+ *                           exponential decay (Contribuciones 2), read as "every
+ *                           prefix state is multiplied by gamma_h before each
+ *                           token's update".
+ *   hla2_forward_normalized Metodología 1, "Normalización": the same numerator
+ *                           divided by q_t^T (S^K_t m^Q_t - h_t) + eps.
+ *   ahla_forward            Metodología 2: AHLA, Q (K^T Q)(K^T V), masked:
+ *                           o_t = sum_{j<=t} (q_t.k_j) sum_{i<=j} (q_j.k_i) v_i.
+ *   hla3_forward            Metodología 3: third order A A^T A, masked:
+ *                           O = (M A) V, M = L (.) (A A^T), A = L (.) Q K^T.
+ *
+ * The mask L includes the diagonal (j <= t).  All four are computed with the
+ * chunk-parallel scheme of Metodología 4: per-segment summaries, a Blelloch
+ * exclusive scan with the semidirect-product combine, and a per-chunk output
+ * pass that applies each chunk's carried-in prefix.
+ *
+ * Layout.  q, k: [B][H][T][d]; v: [B][H][T][dv]; o: [B][H][T][dv], contiguous
+ * row-major.  q, k, v are fp32 (HLA_F32) or bf16 (HLA_BF16), all three the same
+ * type; o is always fp32.  gamma, when given, is fp32 [H], shared across B,
+ * each value in (0, 1].  Base addresses must be 16-byte aligned.
+ *
+ * Supported shapes.  d == dv.  HLA_F32: d in {32, 64}, every op (fp32 CUDA-core
+ * path).  HLA_BF16: d in {32, 64}, every op; d == 64 without decay runs the
+ * tcgen05 tensor-core path for hla2 / hla2_normalized / ahla.  T >= 1 (any
+ * value; the tail chunk is padded), B, H >= 1, B*H*T < 2^31.  Anything else
+ * returns HLA_ERR_UNSUPPORTED or HLA_ERR_SHAPE before any launch.
+ *
+ * Memory ownership.  Every pointer (q, k, v, o, gamma, workspace) is DEVICE
+ * memory owned by the caller.  The library never allocates or frees device
+ * memory and keeps no pointer after a call returns.  The workspace holds the
+ * segment summaries, the scanned prefixes and a device status word; size it
+ * with hla_workspace_bytes() for the same (op, dtype, decayed, B, H, T, d, dv).
+ *
+ * Execution.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and the call returns without synchronising.  Calls that share
+ * a workspace must not overlap on the device.
+ *
+ * Errors.  Status codes only: nothing aborts, throws or traps.  Argument errors
+ * are found on the host before anything is enqueued.  A failed launch returns
+ * HLA_ERR_CUDA.  Kernels that wait on a barrier give up after a bounded time,
+ * set the device status word and return; hla_read_device_status() fetches it.
+ */
+#ifndef HLA_H_
+#define HLA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HLA_OK = 0,
+    HLA_ERR_NULL = 1,        /* a required pointer is NULL */
+    HLA_ERR_SHAPE = 2,       /* B, H, T, d or dv out of range, or d != dv */
+    HLA_ERR_ALIGN = 3,       /* a base address is not 16-byte aligned */
+    HLA_ERR_DTYPE = 4,       /* unknown hla_dtype_t */
+    HLA_ERR_UNSUPPORTED = 5, /* valid request this build has no kernel for */
+    HLA_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than hla_workspace_bytes() */
+    HLA_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed */
+    HLA_ERR_TIMEOUT = 8      /* device status: a kernel's bounded wait ran out */
+} hla_status_t;
+
+typedef enum { HLA_F32 = 0, HLA_BF16 = 1 } hla_dtype_t;
+
+typedef enum {
+    HLA_OP_HLA2 = 0,       /* hla2_forward */
+    HLA_OP_HLA2_NORM = 1,  /* hla2_forward_normalized */
+    HLA_OP_AHLA = 2,       /* ahla_forward */
+    HLA_OP_HLA3 = 3        /* hla3_forward */
+} hla_op_t;
+
+/* Version of this ABI (bumped on any signature change). */
+int hla_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hla_status_str(hla_status_t status);
+
+/*
+ * Bytes of device workspace one call needs, or 0 when the request is invalid
+ * or unsupported.  decayed: nonzero when gamma will be passed (hla2 only).
+ */
+size_t hla_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed,
+                           int B, int H, int T, int d, int dv);
+
+/* Second-order masked forward (Metodología 1; decay: Contribuciones 2).
+ * gamma: device fp32 [H], or NULL for no decay. */
+hla_status_t hla2_forward(const void* q, const void* k, const void* v, float* o,
+                          int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                          const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Ratio-normalised second-order masked forward (Metodología 1, Normalización):
+ * o_t = num_t / (den_t + eps), den_t = q_t^T (S^K_t m^Q_t - h_t). */
+hla_status_t hla2_forward_normalized(const void* q, const void* k, const void* v, float* o,
+                                     int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                     const float* gamma, float eps,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* AHLA masked forward (Metodología 2).  gamma must be NULL (no decayed AHLA). */
+hla_status_t ahla_forward(const void* q, const void* k, const void* v, float* o,
+                          int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                          const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Third-order masked forward (Metodología 3).  gamma must be NULL. */
+hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
+                          int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                          const float* gamma, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * Same computation as the four entry points above, selected by `op`, with
+ * timing hooks: when `phase_events` is non-NULL it points to four cudaEvent_t
+ * handles (created by the caller, timing enabled) that are recorded on
+ * `stream` before the segment-summary kernel, after it, after the scan, and
+ * after the output kernel.  gamma is accepted for HLA_OP_HLA2 and
+ * HLA_OP_HLA2_NORM only; eps is used by HLA_OP_HLA2_NORM only.
+ */
+hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, const void* v, float* o,
+                                  int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                  const float* gamma, float eps, void* workspace,
+                                  size_t workspace_bytes, void* stream, void* const* phase_events);
+
+/*
+ * Number of kernel launches one forward call of this request enqueues
+ * (summary kernel + scan levels + output kernel), or 0 when the request is
+ * invalid or unsupported.  Same arguments as hla_workspace_bytes().
+ */
+int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
+
+/*
+ * 1 when this request runs on the tcgen05 tensor-core kernels, 0 when it runs
+ * on the CUDA-core (fp32 FFMA) kernels or is invalid.  Same arguments as
+ * hla_workspace_bytes().
+ */
+int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
+
+/*
+ * Synchronises `stream` and copies the device status word of the last call
+ * that used `workspace` into *device_status (HLA_OK, or HLA_ERR_TIMEOUT when a
+ * bounded wait ran out).  Returns HLA_ERR_CUDA if the copy fails.
+ */
+hla_status_t hla_read_device_status(const void* workspace, void* stream, int* device_status);
+
+/*
+ * Tensor-core layout self-check (diagnostic; no counterpart on the pages).
+ * Runs one tcgen05 bf16 MMA of shape M=128 x N x K on one CTA:
+ *   D[M][N] = sum_k A(m,k) B(k,n), fp32 accumulate,
+ * with A given row-major as a[M][K] (case 0, 1: K-major) or as a[K][M]
+ * (case 2, 3: MN-major), and B given as b[N][K] (case 0, 2: K-major) or as
+ * b[K][N] (case 1, 3: MN-major); K and N multiples of 64 (<= 128).
+ * a, b: device bf16; d: device fp32 [M][N].  Enqueued on `stream`.
+ */
+hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, float* d,
+                               int N, int K, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HLA_H_ */

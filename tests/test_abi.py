@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls).
+
+The library must load on a machine without a GPU, export every function
+include/hla.h declares, size workspaces, and reject bad arguments with the
+documented status codes before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import higher_order_linear_chunked_b200 as hla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(hla.LIB_PATH):
+        from higher_order_linear_chunked_b200 import build
+        build.build()
+    return hla.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:a?hla)\w*)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(hla.EXPORTS), names
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.hla_abi_version() == 1
+    for code in range(9):
+        s = lib.hla_status_str(code).decode()
+        assert s.startswith(hla.STATUS_NAMES[code])
+    assert lib.hla_status_str(99).decode() == "unknown hla_status_t"
+
+
+def test_workspace_sizes(lib):
+    ws = lambda *a: lib.hla_workspace_bytes(*a)
+    # supported requests have a positive size, growing with the sequence
+    for op in range(4):
+        for dtype in (hla.HLA_F32, hla.HLA_BF16):
+            for d in (32, 64):
+                a = ws(op, dtype, 0, 1, 2, 256, d, d)
+                b = ws(op, dtype, 0, 1, 2, 4096, d, d)
+                assert 0 < a <= b
+    assert ws(hla.OP_HLA2, hla.HLA_BF16, 1, 2, 16, 16384, 64, 64) > 0       # decayed
+    # invalid or unsupported requests size to 0
+    assert ws(hla.OP_HLA2, hla.HLA_F32, 0, 1, 1, 10, 48, 48) == 0          # d not in {32, 64}
+    assert ws(hla.OP_HLA2, hla.HLA_F32, 0, 1, 1, 10, 64, 32) == 0          # d != dv
+    assert ws(hla.OP_HLA2, hla.HLA_F32, 0, 0, 1, 10, 64, 64) == 0          # B = 0
+    assert ws(hla.OP_HLA2, 7, 0, 1, 1, 10, 64, 64) == 0                    # bad dtype
+    assert ws(hla.OP_AHLA, hla.HLA_F32, 1, 1, 1, 10, 64, 64) == 0          # no decayed AHLA
+    assert ws(9, hla.HLA_F32, 0, 1, 1, 10, 64, 64) == 0                    # bad op
+
+
+def _call(lib, name, q=16, k=16, v=16, o=16, B=1, H=1, T=8, d=32, dv=32, dtype=0, gamma=0, ws=16,
+          wsb=1 << 30, eps=None):
+    vp = ctypes.c_void_p
+    args = [vp(q), vp(k), vp(v), vp(o), B, H, T, d, dv, dtype, vp(gamma)]
+    tail = [vp(ws), ctypes.c_size_t(wsb), vp(0)]
+    fn = getattr(lib, name)
+    if name == "hla2_forward_normalized":
+        return fn(*args, ctypes.c_float(1e-6 if eps is None else eps), *tail)
+    return fn(*args, *tail)
+
+
+@pytest.mark.parametrize("name", ["hla2_forward", "hla2_forward_normalized", "ahla_forward", "hla3_forward"])
+def test_argument_errors_are_reported_before_any_launch(lib, name):
+    assert _call(lib, name, q=0) == 1                      # HLA_ERR_NULL
+    assert _call(lib, name, o=0) == 1
+    assert _call(lib, name, B=0) == 2                      # HLA_ERR_SHAPE
+    assert _call(lib, name, T=0) == 2
+    assert _call(lib, name, B=1 << 16, H=1 << 10, T=1 << 10) == 2
+    assert _call(lib, name, dtype=5) == 4                  # HLA_ERR_DTYPE
+    assert _call(lib, name, d=32, dv=64) == 5              # HLA_ERR_UNSUPPORTED
+    assert _call(lib, name, d=48, dv=48) == 5
+    assert _call(lib, name, q=24) == 3                     # HLA_ERR_ALIGN
+    assert _call(lib, name, ws=0) == 6                     # HLA_ERR_WORKSPACE
+    assert _call(lib, name, wsb=64) == 6
+    assert _call(lib, name, ws=32 + 8) == 3
+    if name in ("ahla_forward", "hla3_forward"):
+        assert _call(lib, name, gamma=64) == 5             # gamma only for second order
+    else:
+        assert _call(lib, name, gamma=66) == 3             # misaligned gamma
+
+
+def test_selftest_argument_errors(lib):
+    vp = ctypes.c_void_p
+    assert lib.hla_selftest_umma(0, vp(0), vp(16), vp(16), 64, 64, vp(0)) == 1
+    assert lib.hla_selftest_umma(4, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
+    assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 96, 64, vp(0)) == 2
+    assert lib.hla_read_device_status(vp(0), vp(0), None) == 1
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package (binding + CUDA sources) must not import, call or link oracle/."""
+    pkg = os.path.join(ROOT, "higher_order_linear_chunked_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"\boracle\b", text), os.path.join(dirpath, f)
+
+
+def test_python_binding_rejects_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 1, 4, 32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        hla.hla2(q, q, q)

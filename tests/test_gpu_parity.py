@@ -1,0 +1,186 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Inputs come from the seeded generators of ``hla_inputs``; the oracle consumes
+exactly the values the kernels receive (bf16 workloads are rounded once, then
+widened).  Bar: max row-wise relative L2 error <= 1e-4 for fp32 inputs and
+<= 2e-2 for bf16 inputs (the problem's stated tolerances).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import hla_inputs
+import oracle
+import oracle.brute as brute
+
+torch = pytest.importorskip("torch")
+import higher_order_linear_chunked_b200 as hla  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3"]
+
+
+def recipe(op, dtype, B, H, T, d, seed=0):
+    qk = "softplus" if op == "hla2n" else "scaled"
+    v = "unit" if op == "hla2n" else "scaled"
+    g = (0.95, 0.999) if op == "hla2d" else None
+    return hla_inputs.Workload(f"{op}_{dtype}_{B}x{H}x{T}x{d}", op, dtype, B, H, T, d, d, qk, v,
+                               gamma_range=g, seed=seed)
+
+
+def gpu_forward(op, q, k, v, gamma, eps=1e-6):
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    gd = gamma.to(dev) if gamma is not None else None
+    o = hla.forward(op, qd, kd, vd, gamma=gd, eps=eps)
+    torch.cuda.synchronize()
+    return o
+
+
+def reference(op, q, k, v, gamma, eps=1e-6):
+    if q.shape[2] <= 256:
+        return brute.forward(op, q, k, v, gamma=gamma, eps=eps)
+    return oracle.recur(op, q, k, v, gamma=gamma, eps=eps)
+
+
+# ---------------------------------------------------------------------------
+# tensor-core layout self-check (one tcgen05 MMA), against fp64 on the host
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", [0, 1, 2, 3])
+@pytest.mark.parametrize("N,K", [(64, 64), (128, 64), (64, 128), (128, 128)])
+def test_umma_layouts(case, N, K):
+    g = torch.Generator().manual_seed(case * 7 + N + K)
+    M = 128
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(K, N, generator=g).to(torch.bfloat16)
+    a = A if not (case & 2) else A.t().contiguous()        # [M][K] or [K][M]
+    b = B.t().contiguous() if not (case & 1) else B        # [N][K] or [K][N]
+    ad, bd = a.cuda(), b.cuda()
+    d = torch.full((M, N), float("nan"), device="cuda")
+    import ctypes
+    lib = hla.load_library()
+    rc = lib.hla_selftest_umma(case, ctypes.c_void_p(ad.data_ptr()), ctypes.c_void_p(bd.data_ptr()),
+                               ctypes.c_void_p(d.data_ptr()), N, K,
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    ref = A.double() @ B.double()
+    err = (d.cpu().double() - ref).abs().max().item()
+    assert err <= 1e-4 * max(1.0, ref.abs().max().item()), err
+
+
+# ---------------------------------------------------------------------------
+# small shapes: every op x dtype x d, ragged tails, several chunks
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 333])
+def test_small_parity(op, dtype, d, T):
+    w = recipe(op, dtype, 1, 2, T, d, seed=T)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(op, q, k, v, g)
+    ref = reference(op, q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), ref)
+    assert err <= TOL[dtype], err
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_many_heads_short_sequences(op):
+    w = recipe(op, "bf16", 3, 5, 97, 64, seed=3)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(op, q, k, v, g)
+    assert oracle.max_row_rel_err(o.cpu(), reference(op, q, k, v, g)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla"])
+@pytest.mark.parametrize("T", [127, 128, 129, 1000, 1024, 2049])
+def test_bf16_d64_parity_across_segments(op, T):
+    """bf16 d = 64 (the tensor-core shapes) over many chunks and a ragged tail."""
+    w = recipe(op, "bf16", 1, 3, T, 64, seed=T + 1)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(op, q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g))
+    assert err <= TOL["bf16"], err
+
+
+# ---------------------------------------------------------------------------
+# properties
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_deterministic_and_causal(op, dtype):
+    w = recipe(op, dtype, 1, 2, 300, 64, seed=11)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    a = gpu_forward(op, q, k, v, g)
+    b = gpu_forward(op, q, k, v, g)
+    assert torch.equal(a, b)                                  # run-to-run bitwise
+    s = 150
+    q2, k2, v2 = q.clone(), k.clone(), v.clone()
+    q2[:, :, s:] = q2[:, :, s:] * 2
+    k2[:, :, s:] = -k2[:, :, s:]
+    v2[:, :, s:] = v2[:, :, s:] + 1
+    c = gpu_forward(op, q2, k2, v2, g)
+    assert torch.equal(a[:, :, :s], c[:, :, :s])              # rows before s untouched
+    assert not torch.equal(a[:, :, s:], c[:, :, s:])
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_no_write_outside_output(op):
+    w = recipe(op, "bf16", 1, 2, 190, 64, seed=5)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    dev = torch.device("cuda:0")
+    n = q.shape[0] * q.shape[1] * q.shape[2] * 64
+    guard = 4096
+    buf = torch.full((n + 2 * guard,), float("nan"), device=dev)
+    out = buf[guard:guard + n].view(1, 2, 190, 64)
+    ws = hla.make_workspace(hla.OP_CODES[op], q.to(dev), v.to(dev), decayed=g is not None)
+    hla.forward(op, q.to(dev), k.to(dev), v.to(dev), gamma=g.to(dev) if g is not None else None,
+                out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[guard + n:]).all()
+    assert torch.isfinite(out).all()
+    assert hla.read_device_status(ws) == 0
+
+
+def test_normalized_constant_v_gives_den_ratio():
+    w = recipe("hla2n", "bf16", 1, 2, 300, 64, seed=9)
+    q, k, _, _ = hla_inputs.make_inputs(w)
+    v = torch.full((1, 2, 300, 64), 2.5, dtype=torch.bfloat16)
+    o = gpu_forward("hla2n", q, k, v, None).cpu().double()
+    # den >> eps for positive q, k: the output is 2.5 up to rounding
+    assert (o - 2.5).abs().max().item() < 2.5 * 2e-2
+
+
+def test_decay_gamma_one_matches_undecayed():
+    w = recipe("hla2", "f32", 1, 2, 200, 32, seed=4)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    a = gpu_forward("hla2d", q, k, v, torch.ones(2))
+    b = gpu_forward("hla2", q, k, v, None)
+    assert oracle.max_row_rel_err(a.cpu(), b.cpu()) < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# the five full-size workloads: whole GPU forward, oracle on sampled heads
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(hla_inputs.WORKLOADS))
+def test_full_size_workloads(name):
+    w = hla_inputs.workload(name)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(w.op, q, k, v, g, eps=w.eps).cpu()
+    assert torch.isfinite(o).all()
+    BH = w.B * w.H
+    for bh in sorted({0, BH // 2, BH - 1}):
+        b, h = divmod(bh, w.H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        gh = g[h:h + 1] if g is not None else None
+        ref = oracle.recur(w.op, q[sl], k[sl], v[sl], gamma=gh, eps=w.eps)
+        err = oracle.max_row_rel_err(o[sl], ref)
+        assert err <= TOL[w.dtype], (name, bh, err)
