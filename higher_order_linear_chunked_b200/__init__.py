@@ -36,7 +36,7 @@ STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_
 
 # Every symbol include/hla.h declares.
 EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
-           "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_read_device_status", "hla_selftest_umma")
+           "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma")
 
 
 class HLAError(RuntimeError):
@@ -75,6 +75,8 @@ def load_library(path: Optional[str] = None):
     lib.hla_kernel_launches.restype = i
     lib.hla_uses_tensor_cores.argtypes = [i, i, i, i, i, i, i, i]
     lib.hla_uses_tensor_cores.restype = i
+    lib.hla_set_segment_chunks.argtypes = [i]
+    lib.hla_set_segment_chunks.restype = i
     lib.hla_read_device_status.argtypes = [vp, vp, ctypes.POINTER(i)]
     lib.hla_read_device_status.restype = i
     lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
@@ -122,6 +124,13 @@ def kernel_launches(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: 
 
 def uses_tensor_cores(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> bool:
     return bool(load_library().hla_uses_tensor_cores(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
+
+
+def set_segment_chunks(chunks: int) -> None:
+    """Tensor-core path tuning: 128-token chunks per segment (0 = automatic)."""
+    rc = load_library().hla_set_segment_chunks(int(chunks))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla_set_segment_chunks")
 
 
 def make_workspace(op: int, q, v, decayed: bool = False):

@@ -153,6 +153,10 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
                    phase_events);
 }
 
+hla_status_t hla_set_segment_chunks(int chunks) {
+    return hla::tc::set_segment_chunks(chunks) ? HLA_OK : HLA_ERR_SHAPE;
+}
+
 hla_status_t hla_read_device_status(const void* workspace, void* stream, int* device_status) {
     if (!workspace || !device_status) return HLA_ERR_NULL;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HLA_ERR_CUDA;

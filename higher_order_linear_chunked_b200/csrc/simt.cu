@@ -554,16 +554,50 @@ static size_t scan_smem() {
     return sizeof(float) * (size_t)(2 * Sum<OP, D>::SIZE + D * D);
 }
 
-int kernel_launches(int T) {
-    const int NCp = next_pow2((T + C - 1) / C);
-    int levels = 0;
-    for (int p = 1; p < NCp; p *= 2) ++levels;
-    return 2 + (NCp == 1 ? 1 : 2 * levels);
-}
 
 size_t workspace_floats(int op, int d, int BH, int T) {
     const int NC = (T + C - 1) / C;
     return (size_t)BH * next_pow2(NC) * summary_floats(op, d);
+}
+
+// Blelloch exclusive scan over NCp (a power of two) summaries per head, in place:
+// log2(NCp) up-sweep launches, then log2(NCp) down-sweep launches (the first one
+// reads the root as the identity).  One block per (pair, head) per level.
+template <int OP, int D>
+static cudaError_t scan_levels(float* sums, int NCp, int BH, cudaStream_t st) {
+    auto kl = k_scan_level<OP, D>;
+    const size_t s2 = scan_smem<OP, D>();
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
+    if (NCp == 1) {
+        k_identity<OP, D><<<BH, NT, 0, st>>>(sums, NCp);
+        return cudaGetLastError();
+    }
+    for (int step = 1; step < NCp; step *= 2) {
+        kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 0, 0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    for (int step = NCp / 2; step >= 1; step /= 2) {
+        kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 1, step == NCp / 2);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t scan(int op, int d, float* sums, int NCp, int BH, cudaStream_t st) {
+    switch (op) {
+    case OP_HLA2: return d == 32 ? scan_levels<OP_HLA2, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA2, 64>(sums, NCp, BH, st);
+    case OP_HLA2D: return d == 32 ? scan_levels<OP_HLA2D, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA2D, 64>(sums, NCp, BH, st);
+    case OP_AHLA: return d == 32 ? scan_levels<OP_AHLA, 32>(sums, NCp, BH, st) : scan_levels<OP_AHLA, 64>(sums, NCp, BH, st);
+    case OP_HLA3: return d == 32 ? scan_levels<OP_HLA3, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA3, 64>(sums, NCp, BH, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+int scan_launches(int NCp) {
+    int levels = 0;
+    for (int p = 1; p < NCp; p *= 2) ++levels;
+    return NCp == 1 ? 1 : 2 * levels;
 }
 
 template <int OP, bool NORM, int D, typename TIn>
@@ -572,30 +606,16 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     const int NC = (T + C - 1) / C;
     const int NCp = next_pow2(NC);
     auto ks = k_summary<OP, D, TIn>;
-    auto kl = k_scan_level<OP, D>;
     auto ko = k_output<OP, NORM, D, TIn>;
-    const size_t s1 = summary_smem<D>(), s2 = scan_smem<OP, D>(), s3 = output_smem<D>();
+    const size_t s1 = summary_smem<D>(), s3 = output_smem<D>();
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
     ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, H, T, NC, NCp, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if (NCp == 1) {
-        k_identity<OP, D><<<BH, NT, 0, st>>>(sums, NCp);
-    } else {
-        for (int step = 1; step < NCp; step *= 2) {
-            kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 0, 0);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        for (int step = NCp / 2; step >= 1; step /= 2) {
-            kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 1, step == NCp / 2);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = scan_levels<OP, D>(sums, NCp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H, T, NCp, sums, o);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -630,6 +650,8 @@ cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const vo
     if (d == 32) return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
 }
+
+int kernel_launches(int T) { return 2 + scan_launches(next_pow2((T + C - 1) / C)); }
 
 }  // namespace simt
 }  // namespace hla

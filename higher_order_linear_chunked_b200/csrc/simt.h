@@ -12,6 +12,14 @@ size_t summary_floats(int op, int d);
 int kernel_launches(int T);
 // floats of workspace the path needs after the status block
 size_t workspace_floats(int op, int d, int BH, int T);
+// summary layout helpers for other paths: offsets (in floats) of matrix / vector slots
+// (second order: S=0 C=1 R=2 ; m=0 r=1; AHLA: P=0 E=1 Dm=2)
+inline size_t mat_offset(int slot, int d) { return (size_t)slot * d * d; }
+inline size_t vec_offset(int op, int slot, int d) { return (size_t)(op == 3 ? 6 : op == 1 ? 4 : 3) * d * d + (size_t)slot * d; }
+// in-place Blelloch exclusive scan over NCp (power of two) summaries per head
+cudaError_t scan(int op, int d, float* sums, int NCp, int BH, cudaStream_t st);
+// kernels scan() enqueues
+int scan_launches(int NCp);
 // enqueue chunk kernel, Blelloch scan levels and output kernel on `st`; `ev` (NULL or
 // 4 events) is recorded before the chunk kernel, after it, after the scan, after the output kernel
 cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,

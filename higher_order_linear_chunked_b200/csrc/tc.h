@@ -8,6 +8,8 @@ namespace tc {
 
 // true when (internal op, normalised, bf16, d) runs on the tcgen05 kernels
 bool supported(int op, bool norm, bool bf16, int d);
+// process-wide segment length (chunks); 0 = automatic; false if invalid
+bool set_segment_chunks(int chunks);
 // kernels one forward enqueues
 int kernel_launches(int op, bool norm, int BH, int T);
 // workspace bytes the path needs after the status block

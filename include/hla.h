@@ -146,6 +146,15 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
 
 /*
+ * Tuning knob of the tensor-core path: chunks of 128 tokens per segment (the
+ * unit one CTA walks).  0 restores the automatic choice.  Values outside
+ * {0, 1, 2, 4, 8, 16} return HLA_ERR_SHAPE.  Process-wide setting: it changes
+ * hla_workspace_bytes() and must not be changed while calls are being made
+ * from other threads.  Results do not depend on it beyond rounding.
+ */
+hla_status_t hla_set_segment_chunks(int chunks);
+
+/*
  * Synchronises `stream` and copies the device status word of the last call
  * that used `workspace` into *device_status (HLA_OK, or HLA_ERR_TIMEOUT when a
  * bounded wait ran out).  Returns HLA_ERR_CUDA if the copy fails.

@@ -95,6 +95,17 @@ def test_argument_errors_are_reported_before_any_launch(lib, name):
         assert _call(lib, name, gamma=66) == 3             # misaligned gamma
 
 
+def test_segment_chunks_knob(lib):
+    base = lib.hla_workspace_bytes(hla.OP_HLA2, hla.HLA_BF16, 0, 1, 2, 4096, 64, 64)
+    for n in (1, 2, 4, 8, 16):
+        assert lib.hla_set_segment_chunks(n) == 0
+        assert lib.hla_workspace_bytes(hla.OP_HLA2, hla.HLA_BF16, 0, 1, 2, 4096, 64, 64) > 0
+    for bad in (-1, 3, 5, 32):
+        assert lib.hla_set_segment_chunks(bad) == 2
+    assert lib.hla_set_segment_chunks(0) == 0
+    assert lib.hla_workspace_bytes(hla.OP_HLA2, hla.HLA_BF16, 0, 1, 2, 4096, 64, 64) == base
+
+
 def test_selftest_argument_errors(lib):
     vp = ctypes.c_void_p
     assert lib.hla_selftest_umma(0, vp(0), vp(16), vp(16), 64, 64, vp(0)) == 1

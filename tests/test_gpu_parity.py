@@ -109,6 +109,29 @@ def test_bf16_d64_parity_across_segments(op, T):
     assert err <= TOL["bf16"], err
 
 
+@pytest.mark.parametrize("op", ["hla2", "hla2n"])
+@pytest.mark.parametrize("nch", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("T", [129, 1000, 2049])
+def test_segment_length_invariance(op, nch, T):
+    """Tensor-core walk over 1..16 chunks per segment: same result (to rounding) as the oracle."""
+    w = recipe(op, "bf16", 2, 2, T, 64, seed=nch + T)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    hla.set_segment_chunks(nch)
+    try:
+        o = gpu_forward(op, q, k, v, g)
+    finally:
+        hla.set_segment_chunks(0)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g))
+    assert err <= TOL["bf16"], err
+
+
+def test_tensor_core_path_is_used_for_bf16_d64():
+    assert hla.uses_tensor_cores(hla.OP_HLA2_NORM, hla.HLA_BF16, False, 4, 16, 4096, 64, 64)
+    assert hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, False, 1, 1, 100, 64, 64)
+    assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_F32, False, 1, 1, 100, 64, 64)
+    assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, True, 1, 1, 100, 64, 64)
+
+
 # ---------------------------------------------------------------------------
 # properties
 # ---------------------------------------------------------------------------
