@@ -162,6 +162,38 @@ hla_status_t hla_set_segment_chunks(int chunks);
 hla_status_t hla_read_device_status(const void* workspace, void* stream, int* device_status);
 
 /*
+ * Size of the device scratch array built into the library for
+ * hla2_forward_normalized_noalloc(): 32 MiB, held on every GPU that loads
+ * the library until the process exits.
+ */
+#define HLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * hla2_forward_normalized() for callers that cannot supply a workspace
+ * (the paper has no counterpart; this is a deployment convenience).
+ *
+ * Who needs it: code that may not allocate device memory while it runs, such
+ * as a plugin executing inside another framework that owns the device memory,
+ * or a serving loop that allocates everything at start-up because cudaMalloc
+ * and cudaFree can synchronise the device and stall unrelated streams.
+ *
+ * Same arguments and result as hla2_forward_normalized() minus the workspace:
+ * the scratch lives in a fixed array of HLA_NOALLOC_SCRATCH_BYTES inside the
+ * library.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).  A request whose hla_workspace_bytes() exceeds
+ * HLA_NOALLOC_SCRATCH_BYTES returns HLA_ERR_WORKSPACE before anything is
+ * enqueued.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  All calls on a device share the one array:
+ * calls whose work overlaps on the GPU race and must be serialised by the
+ * caller.  The array keeps the last call's contents; each call clears what
+ * must start at zero.
+ */
+hla_status_t hla2_forward_normalized_noalloc(const void* q, const void* k, const void* v, float* o,
+                                             int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                             const float* gamma, float eps, void* stream);
+
+/*
  * Tensor-core layout self-check (diagnostic; no counterpart on the pages).
  * Runs one tcgen05 bf16 MMA of shape M=128 x N x K on one CTA:
  *   D[M][N] = sum_k A(m,k) B(k,n), fp32 accumulate,
