@@ -5,8 +5,8 @@
 //
 //  1. k_walk<SUMMARY>: one CTA per (segment, head) walks its chunks from the zero
 //     state and writes the segment summary (S, C, m, R = S C - G, r = S m - h) in fp32.
-//  2. the Blelloch exclusive scan with the semidirect-product combine (shared with the
-//     CUDA-core path) turns segment summaries into carried-in prefixes.
+//  2. k_scan_tree: the Blelloch exclusive scan with the semidirect-product combine turns
+//     the segment summaries into carried-in prefixes (one launch, one CTA per head).
 //  3. k_walk<OUTPUT>: one CTA per (segment, head) starts from its prefix and walks its
 //     chunks again, emitting o for every token and carrying (S, R, r) to the next chunk.
 //
@@ -36,7 +36,7 @@ using bf16 = __nv_bfloat16;
 
 constexpr int C = 128;             // chunk length (tokens) = MMA M
 constexpr int D = 64;              // head dim (d = dv)
-constexpr int NT = 128;            // threads: 4 warps <-> 128 TMEM lanes
+constexpr int NT = 256;            // threads: 8 warps, two per TMEM lane quadrant
 constexpr int DEFAULT_NCH = 4;     // chunks per segment
 constexpr uint32_t TILE = C * D * 2;   // one [128][64] bf16 tile = 16 KB
 
@@ -49,16 +49,18 @@ constexpr uint32_t SM_ONES = SM_Z + TILE;        // MN-major [tok][64], column 0
 constexpr uint32_t SM_A = SM_ONES + TILE;        // A, then W: [128][128] K-major (2 atoms)
 constexpr uint32_t SM_S0 = SM_A + 2 * TILE;      // S0^T: [64 n][64 k] K-major
 constexpr uint32_t SM_R0 = SM_S0 + 64 * 128;     // [R0 | r0]^T: [80 n][64 k] K-major
-constexpr uint32_t SM_BAR = SM_R0 + 80 * 128;    // mbarriers
+constexpr uint32_t SM_RS = SM_R0 + 80 * 128;     // [2][128] fp32 partial row sums of W
+constexpr uint32_t SM_BAR = SM_RS + 2 * C * 4;   // mbarriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024; // + alignment slack
 
 // TMEM columns (fp32 accumulators, 128 lanes).
 constexpr uint32_t TM_A = 0;      // A, then W            (128 cols)
 constexpr uint32_t TM_P = 128;    // P, then Z            (64)
-constexpr uint32_t TM_O = 192;    // O | q.r0             (80)
+constexpr uint32_t TM_O0 = 192;   // O | q.r0, even chunks (80)
 constexpr uint32_t TM_CR = 272;   // lanes 0-63 [C|m], lanes 64-127 [R|r]  (80)
 constexpr uint32_t TM_S = 352;    // lanes 0-63 S         (64)
+constexpr uint32_t TM_O1 = 416;   // O | q.r0, odd chunks  (80)
 constexpr uint32_t TM_COLS = 512;
 
 enum Mode { SUMMARY = 0, OUTPUT = 1 };
@@ -110,6 +112,28 @@ __device__ __forceinline__ void st_row16(uint8_t* tile, uint32_t atom_bytes, int
         *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
     }
 }
+// 32 consecutive columns c0..c0+31 (c0 a multiple of 32) of row `row` into a K-major
+// [rows][128] tile made of two 64-wide atoms TILE bytes apart (or one atom when c0 < 64).
+__device__ __forceinline__ void st_row32(uint8_t* tile, int row, int c0, const float (&v)[32]) {
+    uint8_t* atom = tile + (c0 >> 6) * TILE;
+    const int cin = c0 & 63;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint4 u;
+        u.x = ptx::pack_bf16(v[8 * h + 0], v[8 * h + 1]);
+        u.y = ptx::pack_bf16(v[8 * h + 2], v[8 * h + 3]);
+        u.z = ptx::pack_bf16(v[8 * h + 4], v[8 * h + 5]);
+        u.w = ptx::pack_bf16(v[8 * h + 6], v[8 * h + 7]);
+        const int chunk = (cin >> 3) + h;
+        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
+    }
+}
+// Transposed write of 32 values: v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
+__device__ __forceinline__ void st_col32(uint8_t* tile, int kcol, int c0, const float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
+}
 // Transposed write: value v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
 __device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const float (&v)[16]) {
 #pragma unroll
@@ -118,6 +142,19 @@ __device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const 
 }
 
 // ---------------------------------------------------------------- the walker
+// Threads: 8 warps.  Warp w reads TMEM lane quadrant (w & 3), i.e. tile rows
+// 32 (w & 3) .. + 31, and handles half (w >> 2) of each tile's columns.  Thread 0
+// also issues the TMA loads and the MMAs.
+//
+// Rounds of MMAs per chunk n, each followed by an epilogue:
+//   R1(n): A = Q K^T, P = Q S0                      -> E1(n): A, P to bf16 tiles
+//   R2(n): W = P Q^T + A A^T, Z = P + A K,
+//          S += K^T K, O[n&1] = Q [R0|r0]^T         -> E2(n): W, Z, S0^T to bf16 tiles
+//   R3(n): O[n&1] += W V,
+//          [C|m ; R|r] += [Q^T;Z^T][V|1]            -> E3(n): [R0|r0]^T; O[n&1] to HBM
+// R3(n) and R1(n+1) are issued together and their epilogues run together.  The O
+// accumulator is double buffered in TMEM, so the store of O(n) to HBM runs while
+// the tensor core works on R2(n+1).
 template <int MODE>
 __global__ void __launch_bounds__(NT, 1)
 k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -127,49 +164,32 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + SM_BAR);       // [2]
     uint64_t* bar_mma = bar_load + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    float* rowsum_x = reinterpret_cast<float*>(sm + SM_RS);               // [2][128] partial row sums of W
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;                                     // TMEM lane = tile row
     const int seg = blockIdx.x, bh = blockIdx.y;
     using S = simt_layout;
     float* slot = p.sums + ((size_t)bh * p.NSp + seg) * S::size;
     if (seg >= p.NS) {                       // scan padding: identity (zeros)
-        if (MODE == SUMMARY)
-            for (int e = tid; e < S::size; e += NT) slot[e] = 0.f;
+        if (MODE == SUMMARY) {
+            float4* s4 = reinterpret_cast<float4*>(slot);
+            for (int e = tid; e < S::size / 4; e += NT) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         return;
     }
     const int chunk0 = seg * p.NCH;
     const int nchunks_total = (p.T + C - 1) / C;
     const int nch = min(p.NCH, nchunks_total - chunk0);
 
-    // ---- set-up: barriers, TMEM, constant tiles, carried-in state
+    // ---- set-up: barriers, first loads, TMEM, the ones tile
     if (tid == 0) {
         ptx::mbar_init(&bar_load[0], 1);
         ptx::mbar_init(&bar_load[1], 1);
         ptx::mbar_init(bar_mma, 1);
         ptx::fence_mbar_init();
-        ptx::prefetch_tmap(&tq);
-        ptx::prefetch_tmap(&tk);
-        ptx::prefetch_tmap(&tv);
-    }
-    if (warp == 0) {
-        ptx::tmem_alloc(tmem_slot, TM_COLS);
-        ptx::tmem_relinquish();
-    }
-    {   // ones tile: MN-major, element (token kk, column 0) = 1
-        uint32_t* w = reinterpret_cast<uint32_t*>(sm + SM_ONES);
-        for (int e = tid; e < (int)(TILE / 4); e += NT) w[e] = 0u;
     }
     __syncthreads();
-    {
-        const bf16 one = __float2bfloat16_rn(1.f);
-        *reinterpret_cast<bf16*>(sm + SM_ONES + ptx::sw128_offset(tid, 0)) = one;   // tid = token row 0..127
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-
-    // Issue the TMA loads of chunk `n` (local index) into buffer n & 1.
     auto issue_load = [&](int n) {
         const int b = n & 1;
         const int t0 = (chunk0 + n) * C;
@@ -182,27 +202,75 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         issue_load(0);
         if (nch > 1) issue_load(1);
     }
-
-    // Carried-in state: fp32 into TMEM (S in TM_S lanes 0-63, [R|r] in TM_CR lanes 64-127),
-    // bf16 transposed copies into SM_S0 / SM_R0.  The summary walk starts from zero.
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, TM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid < C) {
+        // ones tile, MN-major [token][64]: the N = 80 MMAs read only columns 0..15 of it,
+        // i.e. logical 16-byte chunks 0 and 1 of every token row: chunk 0 = (1, 0, ..., 0).
+        uint8_t* r = sm + SM_ONES + tid * 128;
+        *reinterpret_cast<uint4*>(r + (((0 ^ tid) & 7) << 4)) = make_uint4(0x3F80u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(r + (((1 ^ tid) & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // Carried-in state (OUTPUT): the prefix (S, R, r) is staged in shared memory with
+    // coalesced loads (rows swizzled by 16-byte chunk), then every thread takes its row.
+    float* stage = reinterpret_cast<float*>(sm + SM_A);                   // S [64][64] | R [64][64]
+    float* stage_r = reinterpret_cast<float*>(sm + SM_Z);                 // r [64]
+    if (MODE == OUTPUT) {
+        const float4* s4 = reinterpret_cast<const float4*>(slot + S::mat(0));
+        const float4* r4 = reinterpret_cast<const float4*>(slot + S::mat(2));
+        float4 xs[4], xr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xs[i] = s4[tid + NT * i];
+            xr[i] = r4[tid + NT * i];
+        }
+        const float rv = tid < D ? slot[S::vec(1) + tid] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int f = tid + NT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
+            reinterpret_cast<float4*>(stage)[rr * 16 + ch] = xs[i];
+            reinterpret_cast<float4*>(stage + D * D)[rr * 16 + ch] = xr[i];
+        }
+        if (tid < D) stage_r[tid] = rv;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     {
+        // state -> TMEM (fp32) and bf16 transposed copies (S0^T, [R0|r0]^T); zeros for the summary walk
         float v[16];
-        if (warp < 2) {                      // S row `tid`
-            const float* src = slot + S::mat(0) + tid * D;
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                for (int i = 0; i < 16; ++i) v[i] = (MODE == OUTPUT) ? src[c0 + i] : 0.f;
+        if (quad < 2) {                      // S row `row`, columns half*32 .. +31
+            for (int c0 = half * 32; c0 < half * 32 + 32; c0 += 16) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int ch = (c0 / 4 + j) ^ (row & 7);
+                    const float4 x = MODE == OUTPUT ? reinterpret_cast<const float4*>(stage)[row * 16 + ch]
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                }
                 if (MODE == OUTPUT) ptx::tmem_st16(tmem + lane_base + TM_S + c0, v);
-                st_col16(sm + SM_S0, tid, c0, v);
+                st_col16(sm + SM_S0, row, c0, v);
             }
-        } else {                             // [R | r] row tid - 64
-            const int r = tid - 64;
-            const float* src = slot + S::mat(2) + r * D;
-            for (int c0 = 0; c0 < 80; c0 += 16) {
-                for (int i = 0; i < 16; ++i) {
-                    const int c = c0 + i;
-                    float x = 0.f;
-                    if (MODE == OUTPUT) x = c < D ? src[c] : (c == D ? slot[S::vec(1) + r] : 0.f);
-                    v[i] = x;
+        } else {                             // [R | r] row `row - 64`, columns 0..47 / 48..79
+            const int r = row - 64;
+            const int cb = half ? 48 : 0, ce = half ? 80 : 48;
+            for (int c0 = cb; c0 < ce; c0 += 16) {
+                if (c0 < D) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int ch = (c0 / 4 + j) ^ (r & 7);
+                        const float4 x = MODE == OUTPUT ? reinterpret_cast<const float4*>(stage + D * D)[r * 16 + ch]
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                        v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                    if (MODE == OUTPUT) v[0] = stage_r[r];
                 }
                 if (MODE == OUTPUT) ptx::tmem_st16(tmem + lane_base + TM_CR + c0, v);
                 st_col16(sm + SM_R0, r, c0, v);
@@ -222,11 +290,49 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     constexpr uint32_t I_N64_MM = ptx::idesc_bf16(128, 64, true, true);
     constexpr uint32_t I_N80_KK = ptx::idesc_bf16(128, 80, false, false);
     constexpr uint32_t I_N80_MM = ptx::idesc_bf16(128, 80, true, true);
+    // Descriptor of K-step s from the step-0 descriptor: only the 14-bit start address moves.
+    auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
+    auto k2 = [](uint64_t d0, int s) { return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4); };
+    auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };                       // +2048 B
+    auto bufQ = [&](int n) { return sbase + ((n & 1) ? SM_Q1 : SM_Q0); };
+    auto bufK = [&](int n) { return sbase + ((n & 1) ? SM_K1 : SM_K0); };
+    auto bufV = [&](int n) { return sbase + ((n & 1) ? SM_V1 : SM_V0); };
+    const uint64_t dS0 = kdesc(sbase + SM_S0, 0), dR0 = kdesc(sbase + SM_R0, 0);
+    const uint64_t dZk = kdesc(sbase + SM_Z, 0), dA2 = kdesc2(sbase + SM_A, 0);
+    auto tm_o = [&](int n) { return tmem + ((n & 1) ? TM_O1 : TM_O0); };
+
+    auto issue_r1 = [&](int n) {             // A = Q K^T, P = Q S0
+        const uint64_t dQ = kdesc(bufQ(n), 0), dK = kdesc(bufK(n), 0);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_A, k1(dQ, s), k1(dK, s), I_QK, s > 0);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_P, k1(dQ, s), k1(dS0, s), I_N64_KK, s > 0);
+    };
+    auto issue_r2 = [&](int n) {             // W, O = Q [R0|r0]^T, Z, S
+        const uint32_t sK = bufK(n), sV = bufV(n);
+        const uint64_t dQ = kdesc(bufQ(n), 0);
+        const uint64_t dKm = mdesc(sK, TILE, 0), dKV = mdesc(sK, sV - sK, 0);
+        if (MODE == OUTPUT) {
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_A, k1(dZk, s), k1(dQ, s), I_QK, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_A, k2(dA2, s), k2(dA2, s), I_QK, 1);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tm_o(n), k1(dQ, s), k1(dR0, s), I_N80_KK, s > 0);
+        }
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_P, k2(dA2, s), mn(dKm, s), I_N64_KM, 1);
+        for (int s = 0; s < 8; ++s)
+            ptx::umma_bf16(tmem + TM_S, mn(dKV, s), mn(dKm, s), I_N64_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
+    };
+    auto issue_r3 = [&](int n) {             // O += W V ; [C|m ; R|r] += [Q^T ; Z^T] [V | 1]
+        const uint32_t sQ = bufQ(n), sV = bufV(n);
+        const uint64_t dVm = mdesc(sV, TILE, 0), dQZ = mdesc(sQ, sbase + SM_Z - sQ, 0);
+        const uint64_t dV1 = mdesc(sV, sbase + SM_ONES - sV, 0);
+        if (MODE == OUTPUT)
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tm_o(n), k2(dA2, s), mn(dVm, s), I_N64_KM, 1);
+        for (int s = 0; s < 8; ++s)
+            ptx::umma_bf16(tmem + TM_CR, mn(dQZ, s), mn(dV1, s), I_N80_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
+    };
 
     uint32_t mma_phase = 0;
     bool ok = true;
-    // Thread 0 waits on the MMA barrier (bounded); the block agrees on the outcome.
-    auto wait_mma = [&]() -> bool {
+    // Thread 0 commits the MMAs issued so far and waits for them (bounded); the block agrees.
+    auto commit_wait = [&]() -> bool {
         bool good = true;
         if (tid == 0) {
             ptx::umma_commit(bar_mma);
@@ -244,145 +350,160 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tc_fence_after();
     };
 
-    const int row = tid;                      // TMEM lane = row of the 128-row tiles
-    const int t_base = chunk0 * C;
-    for (int n = 0; n < nch && ok; ++n) {
-        const int b = n & 1;
-        const uint32_t sQ = sbase + (b ? SM_Q1 : SM_Q0);
-        const uint32_t sK = sbase + (b ? SM_K1 : SM_K0);
-        const uint32_t sV = sbase + (b ? SM_V1 : SM_V0);
-        // ---- phase 1: A = Q K^T, P = Q S0
-        if (tid == 0) {
-            ok = ptx::mbar_wait(&bar_load[b], (n >> 1) & 1);
-            if (ok) {
-                ptx::tc_fence_after();
-                for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_A, kdesc(sQ, s), kdesc(sK, s), I_QK, s > 0);
-                for (int s = 0; s < 4; ++s)
-                    ptx::umma_bf16(tmem + TM_P, kdesc(sQ, s), kdesc(sbase + SM_S0, s), I_N64_KK, s > 0);
-            }
+    // E1: A (masked) -> SM_A (this thread: columns half*64 .. +63); P -> SM_Z (OUTPUT only)
+    auto epi1 = [&]() {
+        float v0[32], v1[32];
+        const int c0 = half * 64;
+        ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (c0 + i > row) v0[i] = 0.f;
+            if (c0 + 32 + i > row) v1[i] = 0.f;
         }
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-        if (!wait_mma()) { ok = false; break; }
-        // ---- epilogue 1: A (masked) and P to bf16 tiles
-        {
-            float v[16];
-            for (int c0 = 0; c0 < C; c0 += 16) {
-                ptx::tmem_ld16(tmem + lane_base + TM_A + c0, v);
-                for (int i = 0; i < 16; ++i)
-                    if (c0 + i > row) v[i] = 0.f;
-                st_row16(sm + SM_A, TILE, row, c0, v);
-            }
-            if (MODE == OUTPUT)
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    ptx::tmem_ld16(tmem + lane_base + TM_P + c0, v);
-                    st_row16(sm + SM_Z, TILE, row, c0, v);
-                }
-        }
-        sync_for_mma();
-        // ---- phase 2: W = P Q^T + A A^T ; Z = P + A K ; S += K^T K ; O = Q [R0|r0]
-        if (tid == 0) {
-            if (MODE == OUTPUT) {
-                for (int s = 0; s < 4; ++s)
-                    ptx::umma_bf16(tmem + TM_A, kdesc(sbase + SM_Z, s), kdesc(sQ, s), I_QK, s > 0);
-                for (int s = 0; s < 8; ++s)
-                    ptx::umma_bf16(tmem + TM_A, kdesc2(sbase + SM_A, s), kdesc2(sbase + SM_A, s), I_QK, 1);
-                for (int s = 0; s < 4; ++s)
-                    ptx::umma_bf16(tmem + TM_O, kdesc(sQ, s), kdesc(sbase + SM_R0, s), I_N80_KK, s > 0);
-            }
-            for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + TM_P, kdesc2(sbase + SM_A, s), mdesc(sK, TILE, s), I_N64_KM, 1);
-            for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + TM_S, mdesc(sK, sV - sK, s), mdesc(sK, TILE, s), I_N64_MM,
-                               (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
-        }
-        if (!wait_mma()) { ok = false; break; }
-        // ---- epilogue 2: W (masked) -> bf16 (+ row sums), Z -> bf16, S -> bf16 S0^T
-        float rowsum = 0.f;
-        {
-            float v[16];
-            if (MODE == OUTPUT)
-                for (int c0 = 0; c0 < C; c0 += 16) {
-                    ptx::tmem_ld16(tmem + lane_base + TM_A + c0, v);
-                    for (int i = 0; i < 16; ++i) {
-                        const float x = (c0 + i > row) ? 0.f : __bfloat162float(__float2bfloat16_rn(v[i]));
-                        v[i] = x;
-                        rowsum += x;
-                    }
-                    st_row16(sm + SM_A, TILE, row, c0, v);
-                }
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                ptx::tmem_ld16(tmem + lane_base + TM_P + c0, v);
-                st_row16(sm + SM_Z, TILE, row, c0, v);
-            }
-            if (warp < 2)
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    ptx::tmem_ld16(tmem + lane_base + TM_S + c0, v);
-                    st_col16(sm + SM_S0, row, c0, v);
-                }
-        }
-        sync_for_mma();
-        // ---- phase 3: O += W V ; [C|m ; R|r] += [Q^T ; Z^T] [V | 1]
-        if (tid == 0) {
-            if (MODE == OUTPUT)
-                for (int s = 0; s < 8; ++s)
-                    ptx::umma_bf16(tmem + TM_O, kdesc2(sbase + SM_A, s), mdesc(sV, TILE, s), I_N64_KM, 1);
-            for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + TM_CR, mdesc(sQ, sbase + SM_Z - sQ, s), mdesc(sV, sbase + SM_ONES - sV, s),
-                               I_N80_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
-        }
-        if (!wait_mma()) { ok = false; break; }
-        // ---- epilogue 3: output rows; [R|r] -> bf16 transposed copy; next loads
-        if (tid == 0 && n + 2 < nch) issue_load(n + 2);
+        st_row32(sm + SM_A, row, c0, v0);
+        st_row32(sm + SM_A, row, c0 + 32, v1);
         if (MODE == OUTPUT) {
-            float v[16];
-            ptx::tmem_ld16(tmem + lane_base + TM_O + 64, v);
-            const float den = v[0] + rowsum;
-            const float scale = p.norm ? 1.f / (den + p.eps) : 1.f;
-            const int t = t_base + n * C + row;
-            float* orow = p.o + ((size_t)bh * p.T + t) * D;
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                ptx::tmem_ld16(tmem + lane_base + TM_O + c0, v);
-                if (t < p.T)
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4*>(orow + c0 + i) =
-                            make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
-            }
-            if (warp >= 2)
-                for (int c0 = 0; c0 < 80; c0 += 16) {
-                    ptx::tmem_ld16(tmem + lane_base + TM_CR + c0, v);
-                    st_col16(sm + SM_R0, row - 64, c0, v);
-                }
+            ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
+            st_row32(sm + SM_Z, row, half * 32, v0);
         }
+    };
+    // E2: W (masked, bf16-rounded, partial row sums) -> SM_A; Z -> SM_Z; S -> SM_S0 (transposed)
+    auto epi2 = [&]() {
+        float v0[32], v1[32];
+        if (MODE == OUTPUT) {
+            const int c0 = half * 64;
+            ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
+            float rs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float a = (c0 + i > row) ? 0.f : __bfloat162float(__float2bfloat16_rn(v0[i]));
+                const float b = (c0 + 32 + i > row) ? 0.f : __bfloat162float(__float2bfloat16_rn(v1[i]));
+                v0[i] = a;
+                v1[i] = b;
+                rs += a + b;
+            }
+            rowsum_x[half * C + row] = rs;
+            st_row32(sm + SM_A, row, c0, v0);
+            st_row32(sm + SM_A, row, c0 + 32, v1);
+        }
+        if (quad < 2) {
+            ptx::tmem_ld32x2(tmem + lane_base + TM_P + half * 32, tmem + lane_base + TM_S + half * 32, v0, v1);
+            st_row32(sm + SM_Z, row, half * 32, v0);
+            st_col32(sm + SM_S0, row, half * 32, v1);
+        } else {
+            ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
+            st_row32(sm + SM_Z, row, half * 32, v0);
+        }
+    };
+    // E3, state part: [R|r] -> SM_R0 (transposed), rows 64..127 of TM_CR
+    auto epi3_state = [&]() {
+        if (quad < 2) return;
+        float v[32];
+        float d[16];
+        const int r = row - 64;
+        if (half == 0) {
+            ptx::tmem_ld32(tmem + lane_base + TM_CR, v);
+            st_col32(sm + SM_R0, r, 0, v);
+            ptx::tmem_ld16(tmem + lane_base + TM_CR + 32, d);
+            st_col16(sm + SM_R0, r, 32, d);
+        } else {
+            ptx::tmem_ld32(tmem + lane_base + TM_CR + 48, v);
+            st_col32(sm + SM_R0, r, 48, v);
+        }
+    };
+    // E3, output part: O rows of chunk n -> HBM (normalised)
+    auto epi3_out = [&](int n) {
+        float v[32];
+        float d[16];
+        const uint32_t to = tm_o(n) + lane_base;
+        ptx::tmem_ld16(to + 64, d);
+        const float den = d[0] + rowsum_x[row] + rowsum_x[C + row];
+        const float scale = p.norm ? 1.f / (den + p.eps) : 1.f;
+        const int t = (chunk0 + n) * C + row;
+        ptx::tmem_ld32(to + half * 32, v);
+        if (t < p.T) {
+            float* orow = p.o + ((size_t)bh * p.T + t) * D + half * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4*>(orow + i) =
+                    make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
+        }
+    };
+
+    // ---- the walk
+    if (tid == 0) {
+        ok = ptx::mbar_wait(&bar_load[0], 0);
+        if (ok) {
+            ptx::tc_fence_after();
+            issue_r1(0);
+        }
+    }
+    ok = __syncthreads_and(ok) != 0;
+    for (int n = 0; n < nch && ok; ++n) {
+        if (!commit_wait()) { ok = false; break; }          // R1(n) [+ R3(n-1)] done
+        epi1();
+        if (MODE == OUTPUT && n > 0) epi3_state();
+        if (tid == 0 && n >= 1 && n + 1 < nch) issue_load(n + 1);   // buffer freed by R3(n-1)
         sync_for_mma();
+        if (tid == 0) issue_r2(n);
+        if (MODE == OUTPUT && n > 0) epi3_out(n - 1);       // overlaps R2(n)
+        if (!commit_wait()) { ok = false; break; }          // R2(n) done
+        epi2();
+        sync_for_mma();
+        if (tid == 0) {
+            issue_r3(n);
+            if (n + 1 < nch) {
+                ok = ptx::mbar_wait(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    issue_r1(n + 1);
+                }
+            }
+        }
+        ok = __syncthreads_and(ok) != 0;
+    }
+    if (ok) {
+        ok = commit_wait();                                  // R3(last) done
+        if (ok && MODE == OUTPUT) epi3_out(nch - 1);
     }
 
-    // ---- summary: write the segment's state (fp32)
+    // ---- summary: stage the segment's state (fp32) in shared memory, then coalesced stores
     if (MODE == SUMMARY && ok) {
-        float v[16];
-        if (warp < 2) {
-            for (int c0 = 0; c0 < D; c0 += 16) {            // S row
-                ptx::tmem_ld16(tmem + lane_base + TM_S + c0, v);
-                for (int i = 0; i < 16; ++i) slot[S::mat(0) + row * D + c0 + i] = v[i];
-            }
-            for (int c0 = 0; c0 < 80; c0 += 16) {           // [C | m] row
-                ptx::tmem_ld16(tmem + lane_base + TM_CR + c0, v);
-                for (int i = 0; i < 16; ++i) {
-                    const int c = c0 + i;
-                    if (c < D) slot[S::mat(1) + row * D + c] = v[i];
-                    else if (c == D) slot[S::vec(0) + row] = v[i];
-                }
+        float* st = reinterpret_cast<float*>(sm + SM_Q0);   // the slot layout, rows chunk-swizzled
+        float v[32];
+        float d[16];
+        auto put_row = [&](int m, int rr, int c0, const float (&x)[32]) {
+            float4* dst = reinterpret_cast<float4*>(st + S::mat(m) + rr * D);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                dst[(c0 / 4 + j) ^ (rr & 7)] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+        };
+        if (quad < 2) {
+            ptx::tmem_ld32(tmem + lane_base + TM_S + half * 32, v);
+            put_row(0, row, half * 32, v);
+            ptx::tmem_ld32(tmem + lane_base + TM_CR + half * 32, v);
+            put_row(1, row, half * 32, v);
+            if (half == 0) {
+                ptx::tmem_ld16(tmem + lane_base + TM_CR + 64, d);
+                st[S::vec(0) + row] = d[0];
             }
         } else {
             const int r = row - 64;
-            for (int c0 = 0; c0 < 80; c0 += 16) {           // [R | r] row
-                ptx::tmem_ld16(tmem + lane_base + TM_CR + c0, v);
-                for (int i = 0; i < 16; ++i) {
-                    const int c = c0 + i;
-                    if (c < D) slot[S::mat(2) + r * D + c] = v[i];
-                    else if (c == D) slot[S::vec(1) + r] = v[i];
-                }
+            ptx::tmem_ld32(tmem + lane_base + TM_CR + half * 32, v);
+            put_row(2, r, half * 32, v);
+            if (half == 0) {
+                ptx::tmem_ld16(tmem + lane_base + TM_CR + 64, d);
+                st[S::vec(1) + r] = d[0];
             }
         }
+        __syncthreads();
+        float4* out4 = reinterpret_cast<float4*>(slot);
+        const float4* st4 = reinterpret_cast<const float4*>(st);
+        for (int f = tid; f < 3 * D * D / 4; f += NT) {
+            const int rr = (f >> 4) & (D - 1);
+            out4[f] = st4[(f & ~15) | ((f & 15) ^ (rr & 7))];
+        }
+        for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += NT) out4[f] = st4[f];
     }
     if (!ok) {
         if (tid == 0) {
@@ -396,7 +517,195 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0) ptx::tmem_dealloc(tmem, TM_COLS);
+    if (warp == 1) ptx::tmem_dealloc(tmem, TM_COLS);
+}
+
+// ---------------------------------------------------------------- segment scan
+// Blelloch exclusive scan over the NSp segment summaries of one head, all tree levels
+// in one launch.  One CTA per head; four groups of 128 threads, each group combines one
+// pair of a level (pairs beyond four take further passes).  The semidirect-product
+// combine of the second-order summaries (A earlier, B later):
+//     S = S_A + S_B,  C = C_A + C_B,  m = m_A + m_B,
+//     R = R_A + R_B + S_A C_B,  r = r_A + r_B + S_A m_B.
+// Up-sweep:   X[R] <- X[L] o X[R].
+// Down-sweep: X[L] <- X[R], X[R] <- X[R] o X[L]  (the root is read as the identity).
+// Every pair is updated in place: the factors of the cross term (S of the earlier
+// operand, C and m of the later one) are first staged in shared memory, then each
+// thread rewrites only the elements it owns.
+constexpr int SCAN_GROUPS = 4;
+constexpr int SCAN_GT = 128;                         // threads per group
+constexpr int SCAN_LDS = D + 1;                      // padded row stride of the staged S
+constexpr int SCAN_GROUP_FLOATS = D * SCAN_LDS + D * D + D;
+constexpr size_t SCAN_SMEM = sizeof(float) * SCAN_GROUP_FLOATS * SCAN_GROUPS;
+
+__device__ __forceinline__ void group_sync(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(SCAN_GT) : "memory");
+}
+
+// Stage S of `a` and (C, m) of `b`; then this thread's 32 elements of S_a C_b (row lt/2,
+// columns (lt%2)*32..+31) and, for lt < 64, element lt of S_a m_b.  All global loads of a
+// step are issued before any is used (8 float4 per thread per matrix).
+__device__ __forceinline__ void cross_term(const float* a, const float* b, float* Ss, float* Cs, float* ms, int g,
+                                           int lt, float (&acc)[32], float& accv) {
+    using S = simt_layout;
+    const float4* a4 = reinterpret_cast<const float4*>(a + S::mat(0));
+    const float4* b4 = reinterpret_cast<const float4*>(b + S::mat(1));
+    float4 x[8], y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[i] = a4[lt + SCAN_GT * i];
+        y[i] = b4[lt + SCAN_GT * i];
+    }
+    const float mv = lt < D ? b[S::vec(0) + lt] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = 4 * (lt + SCAN_GT * i), rr = e / D, cc = e % D;
+        float* d = Ss + rr * SCAN_LDS + cc;
+        d[0] = x[i].x; d[1] = x[i].y; d[2] = x[i].z; d[3] = x[i].w;
+        reinterpret_cast<float4*>(Cs)[lt + SCAN_GT * i] = y[i];
+    }
+    if (lt < D) ms[lt] = mv;
+    group_sync(g);
+    const int r = lt >> 1, c0 = (lt & 1) * 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+        const float xv = Ss[r * SCAN_LDS + k];
+        const float4* crow = reinterpret_cast<const float4*>(Cs + k * D + c0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 c = crow[j];
+            acc[4 * j + 0] = fmaf(xv, c.x, acc[4 * j + 0]);
+            acc[4 * j + 1] = fmaf(xv, c.y, acc[4 * j + 1]);
+            acc[4 * j + 2] = fmaf(xv, c.z, acc[4 * j + 2]);
+            acc[4 * j + 3] = fmaf(xv, c.w, acc[4 * j + 3]);
+        }
+    }
+    accv = 0.f;
+    if (lt < D)
+        for (int k = 0; k < D; ++k) accv = fmaf(Ss[lt * SCAN_LDS + k], ms[k], accv);
+    group_sync(g);
+}
+
+// out[e] = f(p[e], t[e]) over one D x D matrix, 8 float4 per thread, loads first.
+template <class F>
+__device__ __forceinline__ void mat_pass(const float* pm, const float* tm, int lt, F f) {
+    const float4* p4 = reinterpret_cast<const float4*>(pm);
+    const float4* t4 = reinterpret_cast<const float4*>(tm);
+    float4 x[8], y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[i] = p4[lt + SCAN_GT * i];
+        y[i] = t4[lt + SCAN_GT * i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f(lt + SCAN_GT * i, x[i], y[i]);
+}
+
+__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+
+__global__ void __launch_bounds__(SCAN_GROUPS * SCAN_GT) k_scan_tree(float* __restrict__ sums, int NSp) {
+    using S = simt_layout;
+    extern __shared__ float scan_sm[];
+    const int g = threadIdx.x / SCAN_GT, lt = threadIdx.x % SCAN_GT;
+    float* Ss = scan_sm + g * SCAN_GROUP_FLOATS;
+    float* Cs = Ss + D * SCAN_LDS;
+    float* ms = Cs + D * D;
+    float* base = sums + (size_t)blockIdx.x * NSp * S::size;
+    const int r = lt >> 1, c0 = (lt & 1) * 32;
+    float acc[32];
+    float accv;
+    for (int step = 1; step < NSp; step *= 2) {                  // up-sweep: X[R] <- X[L] o X[R]
+        const int npairs = NSp / (2 * step);
+        for (int p0 = 0; p0 < npairs; p0 += SCAN_GROUPS) {
+            const int pair = p0 + g;
+            if (pair < npairs) {
+                const float* A = base + (size_t)(pair * 2 * step + step - 1) * S::size;
+                float* B = base + (size_t)(pair * 2 * step + 2 * step - 1) * S::size;
+                cross_term(A, B, Ss, Cs, ms, g, lt, acc, accv);
+                {   // R row r, columns c0..c0+31
+                    const float4* a4 = reinterpret_cast<const float4*>(A + S::mat(2) + r * D + c0);
+                    float4* b4 = reinterpret_cast<float4*>(B + S::mat(2) + r * D + c0);
+                    float4 x[8], y[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) { x[j] = a4[j]; y[j] = b4[j]; }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        b4[j] = make_float4(x[j].x + y[j].x + acc[4 * j], x[j].y + y[j].y + acc[4 * j + 1],
+                                            x[j].z + y[j].z + acc[4 * j + 2], x[j].w + y[j].w + acc[4 * j + 3]);
+                }
+                for (int m = 0; m < 2; ++m) {
+                    float4* b4 = reinterpret_cast<float4*>(B + S::mat(m));
+                    mat_pass(A + S::mat(m), B + S::mat(m), lt, [&](int f, float4 a, float4 b) { b4[f] = add4(a, b); });
+                }
+                if (lt < D) {
+                    B[S::vec(1) + lt] = A[S::vec(1) + lt] + B[S::vec(1) + lt] + accv;
+                    B[S::vec(0) + lt] += A[S::vec(0) + lt];
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int step = NSp / 2; step >= 1; step /= 2) {              // down-sweep
+        const int npairs = NSp / (2 * step);
+        const bool root = (step == NSp / 2);
+        for (int p0 = 0; p0 < npairs; p0 += SCAN_GROUPS) {
+            const int pair = p0 + g;
+            if (pair < npairs) {
+                float* XL = base + (size_t)(pair * 2 * step + step - 1) * S::size;
+                float* XR = base + (size_t)(pair * 2 * step + 2 * step - 1) * S::size;
+                if (root) {                                      // parent prefix = identity
+                    for (int m = 0; m < 3; ++m) {
+                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(m));
+                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(m));
+                        mat_pass(XL + S::mat(m), XR + S::mat(m), lt, [&](int f, float4 t, float4) {
+                            r4[f] = t;
+                            l4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        });
+                    }
+                    if (lt < 2 * D) {
+                        XR[S::vec(0) + lt] = XL[S::vec(0) + lt];
+                        XL[S::vec(0) + lt] = 0.f;
+                    }
+                } else {                                         // P = X[R] (prefix), T = X[L] (left total)
+                    cross_term(XR, XL, Ss, Cs, ms, g, lt, acc, accv);
+                    {
+                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(2) + r * D + c0);
+                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(2) + r * D + c0);
+                        float4 x[8], y[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) { x[j] = r4[j]; y[j] = l4[j]; }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            l4[j] = x[j];
+                            r4[j] = make_float4(x[j].x + y[j].x + acc[4 * j], x[j].y + y[j].y + acc[4 * j + 1],
+                                                x[j].z + y[j].z + acc[4 * j + 2], x[j].w + y[j].w + acc[4 * j + 3]);
+                        }
+                    }
+                    for (int m = 0; m < 2; ++m) {
+                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(m));
+                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(m));
+                        mat_pass(XR + S::mat(m), XL + S::mat(m), lt, [&](int f, float4 pv, float4 tv) {
+                            l4[f] = pv;
+                            r4[f] = add4(pv, tv);
+                        });
+                    }
+                    if (lt < D) {
+                        const float pm = XR[S::vec(0) + lt], tm = XL[S::vec(0) + lt];
+                        const float pr = XR[S::vec(1) + lt], tr = XL[S::vec(1) + lt];
+                        XL[S::vec(0) + lt] = pm;
+                        XR[S::vec(0) + lt] = pm + tm;
+                        XL[S::vec(1) + lt] = pr;
+                        XR[S::vec(1) + lt] = pr + tr + accv;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (NSp == 1)
+        for (int e = threadIdx.x; e < S::size; e += blockDim.x) base[e] = 0.f;
 }
 
 // ---------------------------------------------------------------- host side
@@ -473,7 +782,7 @@ size_t workspace_bytes(int /*op*/, bool /*norm*/, int BH, int T) {
     return sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-int kernel_launches(int /*op*/, bool /*norm*/, int BH, int T) { return 2 + simt::scan_launches(plan(BH, T).NSp); }
+int kernel_launches(int /*op*/, bool /*norm*/, int /*BH*/, int /*T*/) { return 3; }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
                     int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
@@ -500,7 +809,11 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     k_walk<SUMMARY><<<dim3(pl.NSp, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = simt::scan(OP_HLA2, D, prm.sums, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k_scan_tree, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCAN_SMEM)) !=
+        cudaSuccess)
+        return e;
+    k_scan_tree<<<BH, SCAN_GROUPS * SCAN_GT, SCAN_SMEM, st>>>(prm.sums, pl.NSp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_walk<OUTPUT><<<dim3(pl.NS, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
