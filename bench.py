@@ -50,6 +50,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(hla_inputs.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--segment-chunks", type=int, default=0,
+                   help="tensor-core path: 128-token chunks per segment (0 = the library's choice)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -199,11 +201,15 @@ def run_ours(args):
     gd = g.to(dev) if g is not None else None
     out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
     op = hla.OP_CODES[w.op]
+    if args.segment_chunks:
+        hla.set_segment_chunks(args.segment_chunks)
     ws = hla.make_workspace(op, qd, vd, decayed=gd is not None)
     dcode = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
     launches_per_step = hla.kernel_launches(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv)
     path = "tc" if hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv) else "simt"
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    if args.segment_chunks:
+        hla.set_segment_chunks(args.segment_chunks)
 
     def new_events():
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -297,6 +303,7 @@ def run_ours(args):
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "op": w.op, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "dv": w.dv,
                        "tokens_per_gpu": tokens, "path": path, "chunk": model["chunk"],
+                       "segment_chunks": args.segment_chunks or "auto",
                        "l2": "flushed before every step (512 MiB write, outside the timed events)",
                        "parallelism": f"dp{world} (independent heads per rank, no collective)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,

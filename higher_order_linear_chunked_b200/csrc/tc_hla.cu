@@ -5,8 +5,8 @@
 //
 //  1. k_walk<SUMMARY>: one CTA per (segment, head) walks its chunks from the zero
 //     state and writes the segment summary (S, C, m, R = S C - G, r = S m - h) in fp32.
-//  2. k_scan_tree: the Blelloch exclusive scan with the semidirect-product combine turns
-//     the segment summaries into carried-in prefixes (one launch, one CTA per head).
+//  2. k_prefix_cross + k_prefix_sum: the exclusive prefix of the segment summaries under
+//     the semidirect-product combine, in its factored form (see "segment prefixes").
 //  3. k_walk<OUTPUT>: one CTA per (segment, head) starts from its prefix and walks its
 //     chunks again, emitting o for every token and carrying (S, R, r) to the next chunk.
 //
@@ -37,7 +37,7 @@ using bf16 = __nv_bfloat16;
 constexpr int C = 128;             // chunk length (tokens) = MMA M
 constexpr int D = 64;              // head dim (d = dv)
 constexpr int NT = 256;            // threads: 8 warps, two per TMEM lane quadrant
-constexpr int DEFAULT_NCH = 4;     // chunks per segment
+constexpr int kSMs = 148;          // B200 streaming multiprocessors
 constexpr uint32_t TILE = C * D * 2;   // one [128][64] bf16 tile = 16 KB
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
@@ -77,7 +77,8 @@ struct Params {
     int T, BH, NCH, NS, NSp;
     float eps;
     int norm;
-    float* sums;     // [BH][NSp][summary floats]
+    float* sums;     // [BH][NSp][summary floats]: segment summaries
+    float* pre;      // [BH][NSp][summary floats]: carried-in prefixes
     float* o;        // [BH][T][64]
     int* status;
 };
@@ -170,8 +171,8 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     const int row = quad * 32 + lane;                                     // TMEM lane = tile row
     const int seg = blockIdx.x, bh = blockIdx.y;
     using S = simt_layout;
-    float* slot = p.sums + ((size_t)bh * p.NSp + seg) * S::size;
-    if (seg >= p.NS) {                       // scan padding: identity (zeros)
+    float* slot = (MODE == OUTPUT ? p.pre : p.sums) + ((size_t)bh * p.NSp + seg) * S::size;
+    if (seg >= p.NS) {                       // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
             for (int e = tid; e < S::size / 4; e += NT) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -520,192 +521,120 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     if (warp == 1) ptx::tmem_dealloc(tmem, TM_COLS);
 }
 
-// ---------------------------------------------------------------- segment scan
-// Blelloch exclusive scan over the NSp segment summaries of one head, all tree levels
-// in one launch.  One CTA per head; four groups of 128 threads, each group combines one
-// pair of a level (pairs beyond four take further passes).  The semidirect-product
-// combine of the second-order summaries (A earlier, B later):
-//     S = S_A + S_B,  C = C_A + C_B,  m = m_A + m_B,
-//     R = R_A + R_B + S_A C_B,  r = r_A + r_B + S_A m_B.
-// Up-sweep:   X[R] <- X[L] o X[R].
-// Down-sweep: X[L] <- X[R], X[R] <- X[R] o X[L]  (the root is read as the identity).
-// Every pair is updated in place: the factors of the cross term (S of the earlier
-// operand, C and m of the later one) are first staged in shared memory, then each
-// thread rewrites only the elements it owns.
-constexpr int SCAN_GROUPS = 4;
-constexpr int SCAN_GT = 128;                         // threads per group
-constexpr int SCAN_LDS = D + 1;                      // padded row stride of the staged S
-constexpr int SCAN_GROUP_FLOATS = D * SCAN_LDS + D * D + D;
-constexpr size_t SCAN_SMEM = sizeof(float) * SCAN_GROUP_FLOATS * SCAN_GROUPS;
+// ---------------------------------------------------------------- segment prefixes
+// Exclusive prefix of the segment summaries under the semidirect-product combine
+//     (S, C, m, R, r)_A o (S, C, m, R, r)_B
+//       = (S_A + S_B, C_A + C_B, m_A + m_B, R_A + R_B + S_A C_B, r_A + r_B + S_A m_B).
+// Unrolled, the prefix of segments 0..n-1 is
+//     S0(n) = sum_{l<n} S_l,   R0(n) = sum_{l<n} (R_l + S0(l) C_l),
+//     r0(n) = sum_{l<n} (r_l + S0(l) m_l):
+// the cross term of the combine depends on the earlier part only through its S, so
+// the scan splits into a prefix of S, one independent product per segment and a
+// prefix of the corrected R.  Both prefixes are plain sums, so every segment and every
+// matrix element runs in parallel; the result equals the Blelloch tree's (up to the
+// order of fp32 additions).
+//   k_prefix_cross (one CTA per segment x head): S0(l), m0(l) by summation, then
+//       Y_l = R_l + S0(l) C_l and y_l = r_l + S0(l) m_l, written to the prefix slot l;
+//   k_prefix_sum (one thread per matrix element): R0(n) = sum_{l<n} Y_l in place.
+constexpr int PX_NT = 256;
 
-__device__ __forceinline__ void group_sync(int g) {
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(SCAN_GT) : "memory");
-}
-
-// Stage S of `a` and (C, m) of `b`; then this thread's 32 elements of S_a C_b (row lt/2,
-// columns (lt%2)*32..+31) and, for lt < 64, element lt of S_a m_b.  All global loads of a
-// step are issued before any is used (8 float4 per thread per matrix).
-__device__ __forceinline__ void cross_term(const float* a, const float* b, float* Ss, float* Cs, float* ms, int g,
-                                           int lt, float (&acc)[32], float& accv) {
+__global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict__ sums, float* __restrict__ pre,
+                                                        int NSp) {
     using S = simt_layout;
-    const float4* a4 = reinterpret_cast<const float4*>(a + S::mat(0));
-    const float4* b4 = reinterpret_cast<const float4*>(b + S::mat(1));
-    float4 x[8], y[8];
+    __shared__ __align__(16) float S0s[D * (D + 4)];   // padded rows: conflict-free column walks
+    __shared__ __align__(16) float Cs[D * D];
+    __shared__ float ms[D];
+    const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const float* sb = sums + (size_t)bh * NSp * S::size;
+    float* out = pre + ((size_t)bh * NSp + l) * S::size;
+    // S0(l) = sum_{m<l} S_m : this thread owns float4 items tid + 256 i (i < 4)
+    float4 acc[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[i] = a4[lt + SCAN_GT * i];
-        y[i] = b4[lt + SCAN_GT * i];
+    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int m = 0; m < l; ++m) {
+        const float4* src = reinterpret_cast<const float4*>(sb + (size_t)m * S::size + S::mat(0));
+        float4 x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = src[tid + PX_NT * i];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = make_float4(acc[i].x + x[i].x, acc[i].y + x[i].y, acc[i].z + x[i].z,
+                                                         acc[i].w + x[i].w);
     }
-    const float mv = lt < D ? b[S::vec(0) + lt] : 0.f;
+    float m0 = 0.f;
+    if (tid < D)
+        for (int m = 0; m < l; ++m) m0 += sb[(size_t)m * S::size + S::vec(0) + tid];
+    {
+        const float* cl = sb + (size_t)l * S::size;
+        float4 c[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = 4 * (lt + SCAN_GT * i), rr = e / D, cc = e % D;
-        float* d = Ss + rr * SCAN_LDS + cc;
-        d[0] = x[i].x; d[1] = x[i].y; d[2] = x[i].z; d[3] = x[i].w;
-        reinterpret_cast<float4*>(Cs)[lt + SCAN_GT * i] = y[i];
-    }
-    if (lt < D) ms[lt] = mv;
-    group_sync(g);
-    const int r = lt >> 1, c0 = (lt & 1) * 32;
+        for (int i = 0; i < 4; ++i) c[i] = reinterpret_cast<const float4*>(cl + S::mat(1))[tid + PX_NT * i];
+        const float mv = tid < D ? cl[S::vec(0) + tid] : 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < D; ++k) {
-        const float xv = Ss[r * SCAN_LDS + k];
-        const float4* crow = reinterpret_cast<const float4*>(Cs + k * D + c0);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 c = crow[j];
-            acc[4 * j + 0] = fmaf(xv, c.x, acc[4 * j + 0]);
-            acc[4 * j + 1] = fmaf(xv, c.y, acc[4 * j + 1]);
-            acc[4 * j + 2] = fmaf(xv, c.z, acc[4 * j + 2]);
-            acc[4 * j + 3] = fmaf(xv, c.w, acc[4 * j + 3]);
+        for (int i = 0; i < 4; ++i) {
+            const int f = tid + PX_NT * i, r = f >> 4, c4 = f & 15;
+            *reinterpret_cast<float4*>(S0s + r * (D + 4) + 4 * c4) = acc[i];
+            reinterpret_cast<float4*>(Cs)[f] = c[i];
+            reinterpret_cast<float4*>(out + S::mat(0))[f] = acc[i];          // S0(l)
+        }
+        if (tid < D) {
+            ms[tid] = mv;
+            out[S::vec(0) + tid] = m0;                                       // m0(l)
         }
     }
-    accv = 0.f;
-    if (lt < D)
-        for (int k = 0; k < D; ++k) accv = fmaf(Ss[lt * SCAN_LDS + k], ms[k], accv);
-    group_sync(g);
-}
-
-// out[e] = f(p[e], t[e]) over one D x D matrix, 8 float4 per thread, loads first.
-template <class F>
-__device__ __forceinline__ void mat_pass(const float* pm, const float* tm, int lt, F f) {
-    const float4* p4 = reinterpret_cast<const float4*>(pm);
-    const float4* t4 = reinterpret_cast<const float4*>(tm);
-    float4 x[8], y[8];
+    __syncthreads();
+    // Y_l = R_l + S0 C_l: thread owns rows 4 (tid / 16) .. +3, columns 4 (tid % 16) .. +3
+    {
+        const int r = 4 * (tid >> 4), c = 4 * (tid & 15);
+        float y[4][4];
+        const float* Rl = sb + (size_t)l * S::size + S::mat(2);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[i] = p4[lt + SCAN_GT * i];
-        y[i] = t4[lt + SCAN_GT * i];
+        for (int a = 0; a < 4; ++a) {
+            const float4 x = *reinterpret_cast<const float4*>(Rl + (r + a) * D + c);
+            y[a][0] = x.x; y[a][1] = x.y; y[a][2] = x.z; y[a][3] = x.w;
+        }
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) {
+            const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float sv = S0s[(r + a) * (D + 4) + k];
+                y[a][0] = fmaf(sv, cv.x, y[a][0]);
+                y[a][1] = fmaf(sv, cv.y, y[a][1]);
+                y[a][2] = fmaf(sv, cv.z, y[a][2]);
+                y[a][3] = fmaf(sv, cv.w, y[a][3]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            *reinterpret_cast<float4*>(out + S::mat(2) + (r + a) * D + c) = make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
+        if (tid < D) {
+            float yv = sb[(size_t)l * S::size + S::vec(1) + tid];
+            for (int k = 0; k < D; ++k) yv = fmaf(S0s[tid * (D + 4) + k], ms[k], yv);
+            out[S::vec(1) + tid] = yv;                                       // y_l
+        }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f(lt + SCAN_GT * i, x[i], y[i]);
 }
 
-__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
-
-__global__ void __launch_bounds__(SCAN_GROUPS * SCAN_GT) k_scan_tree(float* __restrict__ sums, int NSp) {
+// R0(n) = sum_{l<n} Y_l and r0(n) = sum_{l<n} y_l, elementwise and in place.
+__global__ void __launch_bounds__(PX_NT) k_prefix_sum(float* __restrict__ pre, int NS, int NSp) {
     using S = simt_layout;
-    extern __shared__ float scan_sm[];
-    const int g = threadIdx.x / SCAN_GT, lt = threadIdx.x % SCAN_GT;
-    float* Ss = scan_sm + g * SCAN_GROUP_FLOATS;
-    float* Cs = Ss + D * SCAN_LDS;
-    float* ms = Cs + D * D;
-    float* base = sums + (size_t)blockIdx.x * NSp * S::size;
-    const int r = lt >> 1, c0 = (lt & 1) * 32;
-    float acc[32];
-    float accv;
-    for (int step = 1; step < NSp; step *= 2) {                  // up-sweep: X[R] <- X[L] o X[R]
-        const int npairs = NSp / (2 * step);
-        for (int p0 = 0; p0 < npairs; p0 += SCAN_GROUPS) {
-            const int pair = p0 + g;
-            if (pair < npairs) {
-                const float* A = base + (size_t)(pair * 2 * step + step - 1) * S::size;
-                float* B = base + (size_t)(pair * 2 * step + 2 * step - 1) * S::size;
-                cross_term(A, B, Ss, Cs, ms, g, lt, acc, accv);
-                {   // R row r, columns c0..c0+31
-                    const float4* a4 = reinterpret_cast<const float4*>(A + S::mat(2) + r * D + c0);
-                    float4* b4 = reinterpret_cast<float4*>(B + S::mat(2) + r * D + c0);
-                    float4 x[8], y[8];
+    const int e = blockIdx.x * PX_NT + threadIdx.x;     // element of the R | r region
+    if (e >= D * D + D) return;
+    const int off = e < D * D ? S::mat(2) + e : S::vec(1) + (e - D * D);
+    float* p = pre + (size_t)blockIdx.y * NSp * S::size + off;
+    float run = 0.f;
+    for (int l0 = 0; l0 < NS; l0 += 8) {
+        float y[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) { x[j] = a4[j]; y[j] = b4[j]; }
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NS) y[i] = p[(size_t)(l0 + i) * S::size];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        b4[j] = make_float4(x[j].x + y[j].x + acc[4 * j], x[j].y + y[j].y + acc[4 * j + 1],
-                                            x[j].z + y[j].z + acc[4 * j + 2], x[j].w + y[j].w + acc[4 * j + 3]);
-                }
-                for (int m = 0; m < 2; ++m) {
-                    float4* b4 = reinterpret_cast<float4*>(B + S::mat(m));
-                    mat_pass(A + S::mat(m), B + S::mat(m), lt, [&](int f, float4 a, float4 b) { b4[f] = add4(a, b); });
-                }
-                if (lt < D) {
-                    B[S::vec(1) + lt] = A[S::vec(1) + lt] + B[S::vec(1) + lt] + accv;
-                    B[S::vec(0) + lt] += A[S::vec(0) + lt];
-                }
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NS) {
+                p[(size_t)(l0 + i) * S::size] = run;
+                run += y[i];
             }
-            __syncthreads();
-        }
     }
-    for (int step = NSp / 2; step >= 1; step /= 2) {              // down-sweep
-        const int npairs = NSp / (2 * step);
-        const bool root = (step == NSp / 2);
-        for (int p0 = 0; p0 < npairs; p0 += SCAN_GROUPS) {
-            const int pair = p0 + g;
-            if (pair < npairs) {
-                float* XL = base + (size_t)(pair * 2 * step + step - 1) * S::size;
-                float* XR = base + (size_t)(pair * 2 * step + 2 * step - 1) * S::size;
-                if (root) {                                      // parent prefix = identity
-                    for (int m = 0; m < 3; ++m) {
-                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(m));
-                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(m));
-                        mat_pass(XL + S::mat(m), XR + S::mat(m), lt, [&](int f, float4 t, float4) {
-                            r4[f] = t;
-                            l4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        });
-                    }
-                    if (lt < 2 * D) {
-                        XR[S::vec(0) + lt] = XL[S::vec(0) + lt];
-                        XL[S::vec(0) + lt] = 0.f;
-                    }
-                } else {                                         // P = X[R] (prefix), T = X[L] (left total)
-                    cross_term(XR, XL, Ss, Cs, ms, g, lt, acc, accv);
-                    {
-                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(2) + r * D + c0);
-                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(2) + r * D + c0);
-                        float4 x[8], y[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) { x[j] = r4[j]; y[j] = l4[j]; }
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            l4[j] = x[j];
-                            r4[j] = make_float4(x[j].x + y[j].x + acc[4 * j], x[j].y + y[j].y + acc[4 * j + 1],
-                                                x[j].z + y[j].z + acc[4 * j + 2], x[j].w + y[j].w + acc[4 * j + 3]);
-                        }
-                    }
-                    for (int m = 0; m < 2; ++m) {
-                        float4* l4 = reinterpret_cast<float4*>(XL + S::mat(m));
-                        float4* r4 = reinterpret_cast<float4*>(XR + S::mat(m));
-                        mat_pass(XR + S::mat(m), XL + S::mat(m), lt, [&](int f, float4 pv, float4 tv) {
-                            l4[f] = pv;
-                            r4[f] = add4(pv, tv);
-                        });
-                    }
-                    if (lt < D) {
-                        const float pm = XR[S::vec(0) + lt], tm = XL[S::vec(0) + lt];
-                        const float pr = XR[S::vec(1) + lt], tr = XL[S::vec(1) + lt];
-                        XL[S::vec(0) + lt] = pm;
-                        XR[S::vec(0) + lt] = pm + tm;
-                        XL[S::vec(1) + lt] = pr;
-                        XR[S::vec(1) + lt] = pr + tr + accv;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-    if (NSp == 1)
-        for (int e = threadIdx.x; e < S::size; e += blockDim.x) base[e] = 0.f;
 }
 
 // ---------------------------------------------------------------- host side
@@ -758,9 +687,20 @@ Plan plan(int BH, int T) {
     if (g_segment_chunks > 0) {
         pl.NCH = g_segment_chunks;
     } else {
-        pl.NCH = DEFAULT_NCH;
-        // keep at least two waves of CTAs on 148 SMs when the sequence allows it
-        while (pl.NCH > 1 && (long long)BH * ((pl.NC + pl.NCH - 1) / pl.NCH) < 2 * 148) pl.NCH /= 2;
+        // One CTA walks one segment, one at a time per SM: the walk's makespan is
+        // (waves of CTAs) x (chunks per segment + about one chunk of per-CTA set-up).
+        // Pick the segment length that minimises it (ties: the longer segment).
+        long long best = -1;
+        for (int nch = 1; nch <= 16; nch *= 2) {
+            const long long ctas = (long long)BH * ((pl.NC + nch - 1) / nch);
+            const long long waves = (ctas + kSMs - 1) / kSMs;
+            const long long cost = waves * (nch + 1);
+            if (best < 0 || cost <= best) {
+                best = cost;
+                pl.NCH = nch;
+            }
+            if (nch >= pl.NC) break;
+        }
     }
     pl.NS = (pl.NC + pl.NCH - 1) / pl.NCH;
     pl.NSp = next_pow2(pl.NS);
@@ -779,10 +719,10 @@ bool supported(int op, bool /*norm*/, bool bf16, int d) { return op == OP_HLA2 &
 
 size_t workspace_bytes(int /*op*/, bool /*norm*/, int BH, int T) {
     const Plan pl = plan(BH, T);
-    return sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
+    return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-int kernel_launches(int /*op*/, bool /*norm*/, int /*BH*/, int /*T*/) { return 3; }
+int kernel_launches(int /*op*/, bool /*norm*/, int /*BH*/, int /*T*/) { return 4; }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
                     int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
@@ -796,6 +736,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp;
     prm.eps = eps; prm.norm = norm ? 1 : 0;
     prm.sums = static_cast<float*>(ws);
+    prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
     cudaError_t e;
@@ -809,10 +750,9 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     k_walk<SUMMARY><<<dim3(pl.NSp, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(k_scan_tree, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCAN_SMEM)) !=
-        cudaSuccess)
-        return e;
-    k_scan_tree<<<BH, SCAN_GROUPS * SCAN_GT, SCAN_SMEM, st>>>(prm.sums, pl.NSp);
+    k_prefix_cross<<<dim3(pl.NS, BH), PX_NT, 0, st>>>(prm.sums, prm.pre, pl.NSp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(prm.pre, pl.NS, pl.NSp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_walk<OUTPUT><<<dim3(pl.NS, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);

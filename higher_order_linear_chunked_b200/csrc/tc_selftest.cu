@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     __shared__ uint64_t bar;
     __shared__ uint32_t tmem_base;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int M = 128;
+    const int M = (cs & 4) ? 64 : 128;          // bit 2: M = 64 (half-lane-quadrant accumulator)
+    const int loff = (cs & 8) ? 16 : 0;         // bit 3: accumulator at TMEM lane offset 16
     const bool a_mn = (cs & 2) != 0, b_mn = (cs & 1) != 0;
     uint8_t* As = smem;
     uint8_t* Bs = smem + M * K * 2;
@@ -62,8 +63,9 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     if (tid == 0) {
         const uint32_t idesc = ptx::idesc_bf16(M, N, a_mn, b_mn);
         const uint32_t abase = ptx::smem_u32(As), bbase = ptx::smem_u32(Bs);
+        const uint32_t dt = tbase + (static_cast<uint32_t>(loff) << 16);
         for (int s = 0; s < K / 16; ++s)
-            ptx::umma_bf16(tbase, operand_desc(a_mn, abase, M, K, s), operand_desc(b_mn, bbase, N, K, s), idesc,
+            ptx::umma_bf16(dt, operand_desc(a_mn, abase, M, K, s), operand_desc(b_mn, bbase, N, K, s), idesc,
                            s > 0);
         ptx::umma_commit(&bar);
     }
@@ -71,10 +73,15 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     if (!ok) ok = ptx::mbar_wait(&bar, 0);  // second bounded wait before touching TMEM
     ptx::tc_fence_after();
     const uint32_t taddr = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    // M = 128: row m in lane m.  M = 64: row m in lane (m % 16) + 32 (m / 16) + loff.
+    int m = -1;
+    if (M == 128) m = warp * 32 + lane;
+    else if (lane >= loff && lane < loff + 16) m = warp * 16 + (lane - loff);
     for (int col = 0; col < N; col += 16) {
         float v[16];
         ptx::tmem_ld16(taddr + col, v);
-        for (int i = 0; i < 16; ++i) d[(warp * 32 + lane) * N + col + i] = ok ? v[i] : __int_as_float(0x7fc00000);
+        if (m >= 0)
+            for (int i = 0; i < 16; ++i) d[m * N + col + i] = ok ? v[i] : __int_as_float(0x7fc00000);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -82,7 +89,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
 }
 
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st) {
-    const int smem = 128 * K * 2 + N * K * 2 + 1024;
+    const int smem = 128 * K * 2 + N * K * 2 + 1024;   // A sized for M = 128 in every case
     cudaError_t e = cudaFuncSetAttribute(k_selftest, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k_selftest<<<1, 128, smem, st>>>(layout_case, static_cast<const bf16*>(a), static_cast<const bf16*>(b), d, N, K);

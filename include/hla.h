@@ -163,10 +163,10 @@ hla_status_t hla_read_device_status(const void* workspace, void* stream, int* de
 
 /*
  * Size of the device scratch array built into the library for
- * hla2_forward_normalized_noalloc(): 32 MiB, held on every GPU that loads
+ * hla2_forward_normalized_noalloc(): 64 MiB, held on every GPU that loads
  * the library until the process exits.
  */
-#define HLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define HLA_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /*
  * hla2_forward_normalized() for callers that cannot supply a workspace
@@ -195,11 +195,13 @@ hla_status_t hla2_forward_normalized_noalloc(const void* q, const void* k, const
 
 /*
  * Tensor-core layout self-check (diagnostic; no counterpart on the pages).
- * Runs one tcgen05 bf16 MMA of shape M=128 x N x K on one CTA:
+ * Runs one tcgen05 bf16 MMA of shape M x N x K on one CTA:
  *   D[M][N] = sum_k A(m,k) B(k,n), fp32 accumulate,
- * with A given row-major as a[M][K] (case 0, 1: K-major) or as a[K][M]
- * (case 2, 3: MN-major), and B given as b[N][K] (case 0, 2: K-major) or as
- * b[K][N] (case 1, 3: MN-major); K and N multiples of 64 (<= 128).
+ * with A given row-major as a[M][K] (bit 1 clear: K-major) or as a[K][M]
+ * (bit 1 set: MN-major), and B given as b[N][K] (bit 0 clear: K-major) or as
+ * b[K][N] (bit 0 set: MN-major).  Bit 2 selects M = 64 (else 128); bit 3 (with
+ * bit 2) places the M = 64 accumulator at TMEM lane offset 16.  K and N are
+ * multiples of 64 (<= 128).
  * a, b: device bf16; d: device fp32 [M][N].  Enqueued on `stream`.
  */
 hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, float* d,

@@ -109,7 +109,8 @@ def test_segment_chunks_knob(lib):
 def test_selftest_argument_errors(lib):
     vp = ctypes.c_void_p
     assert lib.hla_selftest_umma(0, vp(0), vp(16), vp(16), 64, 64, vp(0)) == 1
-    assert lib.hla_selftest_umma(4, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
+    assert lib.hla_selftest_umma(16, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
+    assert lib.hla_selftest_umma(8, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 96, 64, vp(0)) == 2
     assert lib.hla_read_device_status(vp(0), vp(0), None) == 1
 

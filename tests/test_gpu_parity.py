@@ -50,11 +50,11 @@ def reference(op, q, k, v, gamma, eps=1e-6):
 # tensor-core layout self-check (one tcgen05 MMA), against fp64 on the host
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("case", [0, 1, 2, 3])
+@pytest.mark.parametrize("case", [0, 1, 2, 3, 4, 5, 6, 7, 12, 13, 14, 15])
 @pytest.mark.parametrize("N,K", [(64, 64), (128, 64), (64, 128), (128, 128)])
 def test_umma_layouts(case, N, K):
     g = torch.Generator().manual_seed(case * 7 + N + K)
-    M = 128
+    M = 64 if case & 4 else 128
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
     B = torch.randn(K, N, generator=g).to(torch.bfloat16)
     a = A if not (case & 2) else A.t().contiguous()        # [M][K] or [K][M]
@@ -122,6 +122,20 @@ def test_segment_length_invariance(op, nch, T):
     finally:
         hla.set_segment_chunks(0)
     err = oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g))
+    assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("nch,T", [(1, 4097), (1, 8193), (2, 8193)])
+def test_many_segments_per_head(nch, T):
+    """More than 32 segments per head (the scan leaves shared memory) and exactly 32 / 64."""
+    w = recipe("hla2n", "bf16", 1, 2, T, 64, seed=nch * 7 + T)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    hla.set_segment_chunks(nch)
+    try:
+        o = gpu_forward("hla2n", q, k, v, g)
+    finally:
+        hla.set_segment_chunks(0)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2n", q, k, v, gamma=g))
     assert err <= TOL["bf16"], err
 
 

@@ -24,7 +24,7 @@ import higher_order_linear_chunked_b200 as hla  # noqa: E402
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2   # bf16-input tolerance used by every parity test
-SCRATCH = 32 << 20
+SCRATCH = 64 << 20
 
 
 def _inputs(seed, T=4096, op="hla2n"):
