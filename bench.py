@@ -164,14 +164,10 @@ def load_peaks():
 def output_kernel_model(path: str, w: hla_inputs.Workload):
     """Algorithmic work of the output kernel per token ('Roofline')."""
     D = w.d
-    if path == "tc":
-        c = 128
-        # A = Q K^T, P = Q S0, W = [P|A][Q|A]^T, O = [Q|W][R0;V], state walk (Z, S, R)
-        flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c) + 2 * c * D + 2 * D * (D + 16) + 2 * D * D
-        return {"bound": "tensor", "flops_per_token": flops, "chunk": c}
-    c = 64
+    # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
+    c = 128 if path == "tc" else 64
     flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
-    return {"bound": "alu", "flops_per_token": flops, "chunk": c}
+    return {"bound": "tensor" if path == "tc" else "alu", "flops_per_token": flops, "chunk": c}
 
 
 def alu_peak_tflops(sm_mhz: float) -> float:
@@ -316,7 +312,9 @@ def run_ours(args):
 
 
 def _traffic_from_profiles(path, w):
-    """DRAM bytes per launch of the output kernel from the committed ncu summary, if it matches."""
+    """DRAM bytes per launch of the output kernel from the committed ncu summary, when it was
+    taken on this workload and on the kernel source as it is now (else None)."""
+    import hashlib
     f = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(f):
         return None
@@ -324,7 +322,13 @@ def _traffic_from_profiles(path, w):
         rec = json.load(open(f)).get(f"{path}:{w.name}")
     except (OSError, ValueError):
         return None
-    return rec.get("dram_bytes_per_launch") if rec else None
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "higher_order_linear_chunked_b200", "csrc", "tc_hla.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest() if os.path.exists(src) else None
+    if rec.get("kernel_source_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
