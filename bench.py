@@ -164,9 +164,13 @@ def load_peaks():
 def output_kernel_model(path: str, w: hla_inputs.Workload):
     """Algorithmic work of the output kernel per token ('Roofline')."""
     D = w.d
-    # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
     c = 128 if path == "tc" else 64
-    flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
+    if w.op == "ahla":
+        # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
+        flops = 6 * c * D + 4 * D * D
+    else:
+        # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
+        flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
     return {"bound": "tensor" if path == "tc" else "alu", "flops_per_token": flops, "chunk": c}
 
 

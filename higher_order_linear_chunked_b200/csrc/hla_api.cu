@@ -170,7 +170,7 @@ hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, fl
                                void* stream) {
     if (!a || !b || !d) return HLA_ERR_NULL;
     if (layout_case < 0 || layout_case > 15 || (layout_case & 8 && !(layout_case & 4))) return HLA_ERR_UNSUPPORTED;
-    if ((N != 64 && N != 128) || (K != 64 && K != 128)) return HLA_ERR_SHAPE;
+    if ((N != 64 && N != 128 && N != 192 && N != 256) || (K != 64 && K != 128)) return HLA_ERR_SHAPE;
     if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return HLA_ERR_ALIGN;
     cudaError_t e = hla::tc::selftest(layout_case, a, b, d, N, K, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;

@@ -1,0 +1,343 @@
+// tcgen05 tensor-core path for the asymmetric HLA forward (AHLA; bf16 inputs, d = dv = 64).
+//
+// "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 2 and 4.
+// Streaming state after token t: P_t = sum_{s<=t} k_s v_s^T and
+// E_t = sum_{s<=t} k_s (q_s^T P_s); the output is o_t = q_t^T E_t.
+//
+// Per chunk of c = 128 tokens (Q, K, V: 128 x 64 tiles; P0, E0: state carried in):
+//     A = L (.) (Q K^T)              (inclusive causal mask)
+//     Y = Q P0 + A V                 (row s is q_s^T P_s)
+//     O = Q E0 + A Y
+//     P0 += K^T V,   E0 += K^T Y
+// A segment of chunks walked from the zero state is summarised by (P, E, D = K^T Q);
+// two segments combine as (P_A + P_B, E_A + E_B + D_B P_A).  The summary slot holds the
+// transposes (P^T, D^T, E^T) in the places of (S, C, R) of the second-order slot: the
+// transposed combine, E^T_AB = E^T_A + E^T_B + P^T_A D^T_B, is the second-order one
+// (R_AB = R_A + R_B + S_A C_B), so the same factored prefix kernels serve both.
+//
+// The walker keeps the fp32 state in registers (thread = one row of [P^T ; E^T], half of
+// its columns) and its bf16 copy in shared memory right after the K tile, so one MMA of
+// N = 256 gives [A | Q P0 | Q E0] at once.  96 KB of shared memory and 256 TMEM columns
+// per CTA: two CTAs share an SM, and one's epilogues overlap the other's MMAs.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tc.h"
+#include "tc_common.cuh"
+
+namespace hla {
+namespace tc {
+namespace {
+
+constexpr int ANT = 256;                 // 8 warps, two per TMEM lane quadrant
+constexpr int kCtasPerSM = 2;
+
+// Shared-memory map (offsets from a 1024-byte aligned base).
+constexpr uint32_t AS_V = 0;             // V  [tok][feat]
+constexpr uint32_t AS_Q = AS_V + TILE;   // Q, then Y  [tok][feat]
+constexpr uint32_t AS_K = AS_Q + TILE;   // K  [tok][feat]
+constexpr uint32_t AS_ST = AS_K + TILE;  // [P0^T ; E0^T] K-major [128 n][64 k], directly after K
+constexpr uint32_t AS_A = AS_ST + TILE;  // A: [128][128] K-major (two 64-wide atoms)
+constexpr uint32_t AS_BAR = AS_A + 2 * TILE;
+constexpr uint32_t AS_TOTAL = AS_BAR + 64;
+constexpr uint32_t ASMEM_BYTES = AS_TOTAL + 1024;   // + alignment slack
+
+// TMEM columns (fp32, 128 lanes).
+constexpr uint32_t TA_A = 0;      // A (128), then the state increment [dP^T ; dE^T] (64)
+constexpr uint32_t TA_Y = 128;    // Q P0, then Y (64)
+constexpr uint32_t TA_O = 192;    // output walk: Q E0, then O (64)
+constexpr uint32_t TA_D = 192;    // summary walk: lanes 0-63 D^T of the segment (64)
+constexpr uint32_t TA_COLS = 256;
+
+enum Mode { SUMMARY = 0, OUTPUT = 1 };
+
+// Threads: warp w reads TMEM lane quadrant (w & 3), i.e. tile rows 32 (w & 3) .. + 31,
+// and half (w >> 2) of each tile's columns.  Thread 0 also issues the TMA loads and MMAs.
+//
+// Rounds of MMAs per chunk n, each followed by an epilogue:
+//   R1: [A | Q P0 | Q E0] = Q [K ; P0^T ; E0^T]^T      -> E1: A masked to bf16
+//   R2: Y += A V  (summary: also D^T += Q^T K)          -> E2: Y to bf16 (over Q)
+//   R3: O += A Y  (output only), [dP^T ; dE^T] = [V^T ; Y^T] K
+//                                                      -> E3: state += increment, to bf16;
+//                                                             O to HBM; next chunk's loads
+template <int MODE>
+__global__ void __launch_bounds__(ANT, kCtasPerSM)
+k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+            const __grid_constant__ CUtensorMap tv, Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + AS_BAR);
+    uint64_t* bar_mma = bar_load + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;                     // TMEM lane = tile row
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    using S = simt_layout;
+    float* slot = (MODE == OUTPUT ? p.pre : p.sums) + ((size_t)bh * p.NSp + seg) * S::size;
+    if (seg >= p.NS) {                                    // padding slots: identity (zeros)
+        if (MODE == SUMMARY) {
+            float4* s4 = reinterpret_cast<float4*>(slot);
+            for (int e = tid; e < S::size / 4; e += ANT) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+    const int chunk0 = seg * p.NCH;
+    const int nch = min(p.NCH, (p.T + C - 1) / C - chunk0);
+
+    if (tid == 0) {
+        ptx::mbar_init(bar_load, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    int loads_issued = 0;                                 // thread 0's count of chunk loads
+    auto issue_load = [&](int n) {
+        const int t0 = (chunk0 + n) * C;
+        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE);
+        ptx::tma_load_3d(sm + AS_Q, &tq, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + AS_K, &tk, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + AS_V, &tv, bar_load, 0, t0, bh);
+        ++loads_issued;
+    };
+    if (tid == 0) issue_load(0);
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, TA_COLS);
+        ptx::tmem_relinquish();
+    }
+
+    // This thread's part of the fp32 state: row `row` of [P^T ; E^T], columns half*32 .. +31.
+    float st[32];
+    if (MODE == OUTPUT) {
+        // the carried-in prefix (P^T, E^T) through shared memory: coalesced loads, rows
+        // swizzled by 16-byte chunk, then every thread takes its row
+        float* stage = reinterpret_cast<float*>(sm + AS_A);   // P^T [64][64] | E^T [64][64]
+        const float4* p4 = reinterpret_cast<const float4*>(slot + S::mat(0));
+        const float4* e4 = reinterpret_cast<const float4*>(slot + S::mat(2));
+        float4 xp[4], xe[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xp[i] = p4[tid + ANT * i];
+            xe[i] = e4[tid + ANT * i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int f = tid + ANT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
+            reinterpret_cast<float4*>(stage)[rr * 16 + ch] = xp[i];
+            reinterpret_cast<float4*>(stage + D * D)[rr * 16 + ch] = xe[i];
+        }
+        __syncthreads();
+        const int r = row & 63;
+        const float4* src = reinterpret_cast<const float4*>(stage + (row >> 6) * D * D) + r * 16;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = src[(half * 8 + j) ^ (r & 7)];
+            st[4 * j] = x.x; st[4 * j + 1] = x.y; st[4 * j + 2] = x.z; st[4 * j + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) st[i] = 0.f;
+    }
+    st_row32(sm + AS_ST, row, half * 32, st);
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+
+    const uint32_t sbase = ptx::smem_u32(sm);
+    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, MODE == OUTPUT ? 256 : 192, false, false);
+    constexpr uint32_t I_N64_KM = ptx::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t I_N64_MM = ptx::idesc_bf16(128, 64, true, true);
+    auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
+    auto k2 = [](uint64_t d0, int s) { return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4); };
+    auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };                       // +2048 B
+    const uint64_t dQ = kdesc(sbase + AS_Q, 0);
+    const uint64_t dKS = kdesc(sbase + AS_K, 0);                     // B rows: K, then P0^T, E0^T
+    const uint64_t dA2 = kdesc2(sbase + AS_A, 0);
+    const uint64_t dVm = mdesc(sbase + AS_V, TILE, 0);
+    const uint64_t dYm = mdesc(sbase + AS_Q, TILE, 0);
+    const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
+    const uint64_t dVY = mdesc(sbase + AS_V, AS_Q - AS_V, 0);        // stacked [V^T ; Y^T]
+    const uint64_t dQK = mdesc(sbase + AS_Q, AS_K - AS_Q, 0);        // stacked [Q^T ; K^T]
+
+    auto issue_r1 = [&]() {
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TA_A, k1(dQ, s), k1(dKS, s), I_R1, s > 0);
+    };
+    auto issue_r2 = [&](int n) {
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_Y, k2(dA2, s), mn(dVm, s), I_N64_KM, 1);
+        if (MODE == SUMMARY)     // lanes 0-63: D^T += Q^T K (lanes 64-127 take K^T K, unused)
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + TA_D, mn(dQK, s), mn(dKm, s), I_N64_MM, (n > 0 || s > 0) ? 1u : 0u);
+    };
+    auto issue_r3 = [&]() {
+        if (MODE == OUTPUT)
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_O, k2(dA2, s), mn(dYm, s), I_N64_KM, 1);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_A, mn(dVY, s), mn(dKm, s), I_N64_MM, s > 0);
+    };
+
+    uint32_t mma_phase = 0;
+    bool ok = true;
+    auto commit_wait = [&]() -> bool {
+        bool good = true;
+        if (tid == 0) {
+            ptx::umma_commit(bar_mma);
+            good = ptx::mbar_wait(bar_mma, mma_phase);
+        }
+        mma_phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
+    auto sync_for_mma = [&]() {
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+    };
+
+    // E1: A (masked, inclusive diagonal) -> AS_A; this thread: columns half*64 .. +63
+    auto epi1 = [&]() {
+        float v[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            ptx::tmem_ld32(tmem + lane_base + TA_A + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i > row) v[i] = 0.f;
+            st_row32(sm + AS_A, row, c0, v);
+        }
+    };
+    // E2: Y -> AS_Q (the Q tile is no longer read)
+    auto epi2 = [&]() {
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + TA_Y + half * 32, v);
+        st_row32(sm + AS_Q, row, half * 32, v);
+    };
+    // E3: state += increment, its bf16 copy -> AS_ST; O rows of chunk n -> HBM
+    auto epi3 = [&](int n) {
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + TA_A + half * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) st[i] += v[i];
+        if (MODE == OUTPUT || row < 64) st_row32(sm + AS_ST, row, half * 32, st);
+        if (MODE == OUTPUT) {
+            ptx::tmem_ld32(tmem + lane_base + TA_O + half * 32, v);
+            const int t = (chunk0 + n) * C + row;
+            if (t < p.T) {
+                float* orow = p.o + ((size_t)bh * p.T + t) * D + half * 32;
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4*>(orow + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            }
+        }
+    };
+
+    // ---- the walk
+    for (int n = 0; n < nch && ok; ++n) {
+        if (tid == 0) {
+            ok = ptx::mbar_wait(bar_load, n & 1);
+            if (ok) {
+                ptx::tc_fence_after();
+                issue_r1();
+            }
+        }
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        if (!commit_wait()) { ok = false; break; }          // R1 done
+        epi1();
+        sync_for_mma();
+        if (tid == 0) issue_r2(n);
+        if (!commit_wait()) { ok = false; break; }          // R2 done
+        epi2();
+        sync_for_mma();
+        if (tid == 0) issue_r3();
+        if (!commit_wait()) { ok = false; break; }          // R3 done: Q/Y, K, V free
+        if (tid == 0 && n + 1 < nch) issue_load(n + 1);
+        epi3(n);
+        sync_for_mma();
+    }
+
+    // ---- summary: stage (P^T, D^T, E^T) in shared memory, then coalesced stores
+    if (MODE == SUMMARY && ok) {
+        float* stg = reinterpret_cast<float*>(sm + AS_V);  // 48 KB over V, Q, K (all MMAs done)
+        auto put_row = [&](int m, int rr, const float (&x)[32]) {
+            float4* dst = reinterpret_cast<float4*>(stg + S::mat(m) + rr * D);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                dst[(half * 8 + j) ^ (rr & 7)] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+        };
+        if (quad < 2) {
+            float v[32];
+            put_row(0, row, st);                                   // P^T
+            ptx::tmem_ld32(tmem + lane_base + TA_D + half * 32, v);
+            put_row(1, row, v);                                    // D^T
+        } else {
+            put_row(2, row - 64, st);                              // E^T
+        }
+        __syncthreads();
+        float4* out4 = reinterpret_cast<float4*>(slot);
+        const float4* st4 = reinterpret_cast<const float4*>(stg);
+        for (int f = tid; f < 3 * D * D / 4; f += ANT) {
+            const int rr = (f >> 4) & (D - 1);
+            out4[f] = st4[(f & ~15) | ((f & 15) ^ (rr & 7))];
+        }
+        for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += ANT) out4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (!ok && tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        // let a load and MMAs already in flight land before TMEM and smem are released
+        if (loads_issued > 0) ptx::mbar_wait(bar_load, (loads_issued - 1) & 1, 100000000ull);
+        ptx::umma_commit(bar_mma);
+        ptx::mbar_wait(bar_mma, mma_phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, TA_COLS);
+}
+
+}  // namespace
+
+size_t ahla_workspace_bytes(int BH, int T) {
+    const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
+    return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
+}
+
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
+                         int* status, cudaStream_t st, cudaEvent_t* ev) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH))
+        return cudaErrorInvalidValue;
+    const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
+    Params prm;
+    prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp;
+    prm.eps = 0.f; prm.norm = 0;
+    prm.sums = static_cast<float*>(ws);
+    prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
+    prm.o = o;
+    prm.status = status;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k_ahla_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ASMEM_BYTES)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_ahla_walk<OUTPUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ASMEM_BYTES)) != cudaSuccess)
+        return e;
+    if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
+    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
+    if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
+    k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
+    return cudaSuccess;
+}
+
+}  // namespace tc
+}  // namespace hla

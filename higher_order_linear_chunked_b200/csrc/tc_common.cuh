@@ -1,0 +1,123 @@
+// Pieces shared by the tcgen05 walkers (second order in tc_hla.cu, AHLA in tc_ahla.cu):
+// tile geometry, UMMA shared-memory descriptors, epilogue stores into 128B-swizzled
+// tiles, the segment-summary slot layout and the host-side set-up (tensor maps, the
+// segment plan, the segment-prefix launches).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace hla {
+namespace tc {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int C = 128;             // chunk length (tokens) = MMA M
+constexpr int D = 64;              // head dim (d = dv)
+constexpr int kSMs = 148;          // B200 streaming multiprocessors
+constexpr uint32_t TILE = C * D * 2;   // one [128][64] bf16 tile = 16 KB
+
+// Segment summaries use the layout of the shared scan kernel (second order, d = 64):
+// S, C, R as 64 x 64 row-major matrices, then m, r, then padding.
+struct simt_layout {
+    static constexpr int size = (3 * D * D + 2 * D + 4 + 31) / 32 * 32;
+    __host__ __device__ static constexpr int mat(int i) { return i * D * D; }
+    __host__ __device__ static constexpr int vec(int i) { return 3 * D * D + i * D; }
+};
+
+struct Params {
+    int T, BH, NCH, NS, NSp;
+    float eps;
+    int norm;       // second order: divide by the denominator
+    float* sums;     // [BH][NSp][summary floats]: segment summaries
+    float* pre;      // [BH][NSp][summary floats]: carried-in prefixes
+    float* o;        // [BH][T][64]
+    int* status;
+};
+
+// ---------------------------------------------------------------- descriptors
+// K-major tile of `rows` rows, K = 64 per atom; K-step s (16 elements).
+__device__ __forceinline__ uint64_t kdesc(uint32_t base, int s) { return ptx::desc_sw128(base + s * 32, 16, 1024); }
+// K-major [128][128] tile in two 64-wide atoms.
+__device__ __forceinline__ uint64_t kdesc2(uint32_t base, int s) {
+    return ptx::desc_sw128(base + (s >> 2) * TILE + (s & 3) * 32, 16, 1024);
+}
+// MN-major tile: one 128-byte row per token; K-step s covers tokens 16s..16s+15;
+// lbo = distance to the next 64-wide M/N block.
+__device__ __forceinline__ uint64_t mdesc(uint32_t base, uint32_t lbo, int s) {
+    return ptx::desc_sw128(base + s * 2048, lbo, 1024);
+}
+
+// ---------------------------------------------------------------- epilogue helpers
+// Write 16 consecutive fp32 values (columns c0..c0+15 of row `row`) as bf16 into a
+// K-major 128B-swizzled tile whose atoms are `atom_bytes` apart.
+__device__ __forceinline__ void st_row16(uint8_t* tile, uint32_t atom_bytes, int row, int c0, const float (&v)[16]) {
+    uint8_t* atom = tile + (c0 >> 6) * atom_bytes;
+    const int cin = c0 & 63;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint4 u;
+        u.x = ptx::pack_bf16(v[8 * h + 0], v[8 * h + 1]);
+        u.y = ptx::pack_bf16(v[8 * h + 2], v[8 * h + 3]);
+        u.z = ptx::pack_bf16(v[8 * h + 4], v[8 * h + 5]);
+        u.w = ptx::pack_bf16(v[8 * h + 6], v[8 * h + 7]);
+        const int chunk = (cin >> 3) + h;
+        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
+    }
+}
+// 32 consecutive columns c0..c0+31 (c0 a multiple of 32) of row `row` into a K-major
+// [rows][128] tile made of two 64-wide atoms TILE bytes apart (or one atom when c0 < 64).
+__device__ __forceinline__ void st_row32(uint8_t* tile, int row, int c0, const float (&v)[32]) {
+    uint8_t* atom = tile + (c0 >> 6) * TILE;
+    const int cin = c0 & 63;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        uint4 u;
+        u.x = ptx::pack_bf16(v[8 * h + 0], v[8 * h + 1]);
+        u.y = ptx::pack_bf16(v[8 * h + 2], v[8 * h + 3]);
+        u.z = ptx::pack_bf16(v[8 * h + 4], v[8 * h + 5]);
+        u.w = ptx::pack_bf16(v[8 * h + 6], v[8 * h + 7]);
+        const int chunk = (cin >> 3) + h;
+        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
+    }
+}
+// Transposed write of 32 values: v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
+__device__ __forceinline__ void st_col32(uint8_t* tile, int kcol, int c0, const float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
+}
+// Transposed write: value v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
+__device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const float (&v)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
+}
+
+// ---------------------------------------------------------------- host side
+// [BH][T][64] bf16 tensor, box = one 128-token chunk, 128-byte swizzle, zero fill past T.
+bool make_map(CUtensorMap* map, const void* base, int T, int BH);
+
+struct Plan {
+    int NC;    // chunks per head
+    int NCH;   // chunks per segment
+    int NS;    // segments per head
+    int NSp;   // NS rounded up to a power of two (summary slots per head)
+};
+// Segment length for BH heads of T tokens when `slots` walker CTAs can run at once.
+Plan plan(int BH, int T, int slots);
+
+// Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for
+// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
+cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st);
+
+// The AHLA forward on the tcgen05 walkers (tc_ahla.cu).
+size_t ahla_workspace_bytes(int BH, int T);
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
+                         int* status, cudaStream_t st, cudaEvent_t* ev);
+
+}  // namespace tc
+}  // namespace hla

@@ -28,17 +28,12 @@
 #include "ptx.cuh"
 #include "simt.h"
 #include "tc.h"
+#include "tc_common.cuh"
 
 namespace hla {
 namespace tc {
 
-using bf16 = __nv_bfloat16;
-
-constexpr int C = 128;             // chunk length (tokens) = MMA M
-constexpr int D = 64;              // head dim (d = dv)
 constexpr int NT = 256;            // threads: 8 warps, two per TMEM lane quadrant
-constexpr int kSMs = 148;          // B200 streaming multiprocessors
-constexpr uint32_t TILE = C * D * 2;   // one [128][64] bf16 tile = 16 KB
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 constexpr uint32_t SM_Q0 = 0, SM_Q1 = SM_Q0 + TILE;
@@ -64,83 +59,6 @@ constexpr uint32_t TM_O1 = 416;   // O | q.r0, odd chunks  (80)
 constexpr uint32_t TM_COLS = 512;
 
 enum Mode { SUMMARY = 0, OUTPUT = 1 };
-
-// Segment summaries use the layout of the shared scan kernel (second order, d = 64):
-// S, C, R as 64 x 64 row-major matrices, then m, r, then padding.
-struct simt_layout {
-    static constexpr int size = (3 * D * D + 2 * D + 4 + 31) / 32 * 32;
-    __host__ __device__ static constexpr int mat(int i) { return i * D * D; }
-    __host__ __device__ static constexpr int vec(int i) { return 3 * D * D + i * D; }
-};
-
-struct Params {
-    int T, BH, NCH, NS, NSp;
-    float eps;
-    int norm;
-    float* sums;     // [BH][NSp][summary floats]: segment summaries
-    float* pre;      // [BH][NSp][summary floats]: carried-in prefixes
-    float* o;        // [BH][T][64]
-    int* status;
-};
-
-// ---------------------------------------------------------------- descriptors
-// K-major tile of `rows` rows, K = 64 per atom; K-step s (16 elements).
-__device__ __forceinline__ uint64_t kdesc(uint32_t base, int s) { return ptx::desc_sw128(base + s * 32, 16, 1024); }
-// K-major [128][128] tile in two 64-wide atoms.
-__device__ __forceinline__ uint64_t kdesc2(uint32_t base, int s) {
-    return ptx::desc_sw128(base + (s >> 2) * TILE + (s & 3) * 32, 16, 1024);
-}
-// MN-major tile: one 128-byte row per token; K-step s covers tokens 16s..16s+15;
-// lbo = distance to the next 64-wide M/N block.
-__device__ __forceinline__ uint64_t mdesc(uint32_t base, uint32_t lbo, int s) {
-    return ptx::desc_sw128(base + s * 2048, lbo, 1024);
-}
-
-// ---------------------------------------------------------------- epilogue helpers
-// Write 16 consecutive fp32 values (columns c0..c0+15 of row `row`) as bf16 into a
-// K-major 128B-swizzled tile whose atoms are `atom_bytes` apart.
-__device__ __forceinline__ void st_row16(uint8_t* tile, uint32_t atom_bytes, int row, int c0, const float (&v)[16]) {
-    uint8_t* atom = tile + (c0 >> 6) * atom_bytes;
-    const int cin = c0 & 63;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint4 u;
-        u.x = ptx::pack_bf16(v[8 * h + 0], v[8 * h + 1]);
-        u.y = ptx::pack_bf16(v[8 * h + 2], v[8 * h + 3]);
-        u.z = ptx::pack_bf16(v[8 * h + 4], v[8 * h + 5]);
-        u.w = ptx::pack_bf16(v[8 * h + 6], v[8 * h + 7]);
-        const int chunk = (cin >> 3) + h;
-        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
-    }
-}
-// 32 consecutive columns c0..c0+31 (c0 a multiple of 32) of row `row` into a K-major
-// [rows][128] tile made of two 64-wide atoms TILE bytes apart (or one atom when c0 < 64).
-__device__ __forceinline__ void st_row32(uint8_t* tile, int row, int c0, const float (&v)[32]) {
-    uint8_t* atom = tile + (c0 >> 6) * TILE;
-    const int cin = c0 & 63;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        uint4 u;
-        u.x = ptx::pack_bf16(v[8 * h + 0], v[8 * h + 1]);
-        u.y = ptx::pack_bf16(v[8 * h + 2], v[8 * h + 3]);
-        u.z = ptx::pack_bf16(v[8 * h + 4], v[8 * h + 5]);
-        u.w = ptx::pack_bf16(v[8 * h + 6], v[8 * h + 7]);
-        const int chunk = (cin >> 3) + h;
-        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
-    }
-}
-// Transposed write of 32 values: v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
-__device__ __forceinline__ void st_col32(uint8_t* tile, int kcol, int c0, const float (&v)[32]) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
-}
-// Transposed write: value v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
-__device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const float (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
-}
 
 // ---------------------------------------------------------------- the walker
 // Threads: 8 warps.  Warp w reads TMEM lane quadrant (w & 3), i.e. tile rows
@@ -656,7 +574,16 @@ EncodeTiled encode_fn() {
     return fn;
 }
 
-// [BH][T][64] bf16 tensor, box = one 128-token chunk, 128-byte swizzle, zero fill past T.
+int next_pow2(int n) {
+    int p = 1;
+    while (p < n) p *= 2;
+    return p;
+}
+
+int g_segment_chunks = 0;   // 0 = automatic
+
+}  // namespace
+
 bool make_map(CUtensorMap* map, const void* base, int T, int BH) {
     EncodeTiled fn = encode_fn();
     if (!fn) return false;
@@ -669,31 +596,19 @@ bool make_map(CUtensorMap* map, const void* base, int T, int BH) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int next_pow2(int n) {
-    int p = 1;
-    while (p < n) p *= 2;
-    return p;
-}
-
-struct Plan {
-    int NC, NCH, NS, NSp;
-};
-
-int g_segment_chunks = 0;   // 0 = automatic
-
-Plan plan(int BH, int T) {
+Plan plan(int BH, int T, int slots) {
     Plan pl;
     pl.NC = (T + C - 1) / C;
     if (g_segment_chunks > 0) {
         pl.NCH = g_segment_chunks;
     } else {
-        // One CTA walks one segment, one at a time per SM: the walk's makespan is
+        // One CTA walks one segment; `slots` CTAs run at once: the walk's makespan is
         // (waves of CTAs) x (chunks per segment + about one chunk of per-CTA set-up).
         // Pick the segment length that minimises it (ties: the longer segment).
         long long best = -1;
         for (int nch = 1; nch <= 16; nch *= 2) {
             const long long ctas = (long long)BH * ((pl.NC + nch - 1) / nch);
-            const long long waves = (ctas + kSMs - 1) / kSMs;
+            const long long waves = (ctas + slots - 1) / slots;
             const long long cost = waves * (nch + 1);
             if (best < 0 || cost <= best) {
                 best = cost;
@@ -707,7 +622,13 @@ Plan plan(int BH, int T) {
     return pl;
 }
 
-}  // namespace
+cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st) {
+    k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(pre, NS, NSp);
+    return cudaGetLastError();
+}
 
 bool set_segment_chunks(int chunks) {
     if (chunks != 0 && chunks != 1 && chunks != 2 && chunks != 4 && chunks != 8 && chunks != 16) return false;
@@ -715,10 +636,11 @@ bool set_segment_chunks(int chunks) {
     return true;
 }
 
-bool supported(int op, bool /*norm*/, bool bf16, int d) { return op == OP_HLA2 && bf16 && d == D; }
+bool supported(int op, bool /*norm*/, bool bf16, int d) { return (op == OP_HLA2 || op == OP_AHLA) && bf16 && d == D; }
 
-size_t workspace_bytes(int /*op*/, bool /*norm*/, int BH, int T) {
-    const Plan pl = plan(BH, T);
+size_t workspace_bytes(int op, bool /*norm*/, int BH, int T) {
+    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T);
+    const Plan pl = plan(BH, T, kSMs);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
@@ -726,12 +648,13 @@ int kernel_launches(int /*op*/, bool /*norm*/, int /*BH*/, int /*T*/) { return 4
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
                     int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
+    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH))
         return cudaErrorInvalidValue;
-    const Plan pl = plan(BH, T);
+    const Plan pl = plan(BH, T, kSMs);
     Params prm;
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp;
     prm.eps = eps; prm.norm = norm ? 1 : 0;
@@ -750,10 +673,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     k_walk<SUMMARY><<<dim3(pl.NSp, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    k_prefix_cross<<<dim3(pl.NS, BH), PX_NT, 0, st>>>(prm.sums, prm.pre, pl.NSp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(prm.pre, pl.NS, pl.NSp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_walk<OUTPUT><<<dim3(pl.NS, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

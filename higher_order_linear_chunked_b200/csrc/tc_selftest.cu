@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     }
     ptx::fence_proxy_async();
     if (warp == 0) {
-        ptx::tmem_alloc(&tmem_base, 128);
+        ptx::tmem_alloc(&tmem_base, 256);
         ptx::tmem_relinquish();
     }
     if (tid == 0) {
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0) ptx::tmem_dealloc(tbase, 128);
+    if (warp == 0) ptx::tmem_dealloc(tbase, 256);
 }
 
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st) {

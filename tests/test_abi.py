@@ -112,6 +112,7 @@ def test_selftest_argument_errors(lib):
     assert lib.hla_selftest_umma(16, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
     assert lib.hla_selftest_umma(8, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 96, 64, vp(0)) == 2
+    assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 320, 64, vp(0)) == 2
     assert lib.hla_read_device_status(vp(0), vp(0), None) == 1
 
 

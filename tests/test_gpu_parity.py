@@ -51,7 +51,7 @@ def reference(op, q, k, v, gamma, eps=1e-6):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("case", [0, 1, 2, 3, 4, 5, 6, 7, 12, 13, 14, 15])
-@pytest.mark.parametrize("N,K", [(64, 64), (128, 64), (64, 128), (128, 128)])
+@pytest.mark.parametrize("N,K", [(64, 64), (128, 64), (64, 128), (128, 128), (192, 64), (256, 64), (256, 128)])
 def test_umma_layouts(case, N, K):
     g = torch.Generator().manual_seed(case * 7 + N + K)
     M = 64 if case & 4 else 128
@@ -109,7 +109,7 @@ def test_bf16_d64_parity_across_segments(op, T):
     assert err <= TOL["bf16"], err
 
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla"])
 @pytest.mark.parametrize("nch", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T", [129, 1000, 2049])
 def test_segment_length_invariance(op, nch, T):
@@ -125,17 +125,18 @@ def test_segment_length_invariance(op, nch, T):
     assert err <= TOL["bf16"], err
 
 
+@pytest.mark.parametrize("op", ["hla2n", "ahla"])
 @pytest.mark.parametrize("nch,T", [(1, 4097), (1, 8193), (2, 8193)])
-def test_many_segments_per_head(nch, T):
+def test_many_segments_per_head(op, nch, T):
     """More than 32 segments per head (the scan leaves shared memory) and exactly 32 / 64."""
-    w = recipe("hla2n", "bf16", 1, 2, T, 64, seed=nch * 7 + T)
+    w = recipe(op, "bf16", 1, 2, T, 64, seed=nch * 7 + T)
     q, k, v, g = hla_inputs.make_inputs(w)
     hla.set_segment_chunks(nch)
     try:
-        o = gpu_forward("hla2n", q, k, v, g)
+        o = gpu_forward(op, q, k, v, g)
     finally:
         hla.set_segment_chunks(0)
-    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2n", q, k, v, gamma=g))
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g))
     assert err <= TOL["bf16"], err
 
 
@@ -144,6 +145,9 @@ def test_tensor_core_path_is_used_for_bf16_d64():
     assert hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, False, 1, 1, 100, 64, 64)
     assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_F32, False, 1, 1, 100, 64, 64)
     assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, True, 1, 1, 100, 64, 64)
+    assert hla.uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, False, 4, 16, 8192, 64, 64)
+    assert not hla.uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, False, 1, 1, 100, 32, 32)
+    assert not hla.uses_tensor_cores(hla.OP_HLA3, hla.HLA_BF16, False, 1, 1, 100, 64, 64)
 
 
 # ---------------------------------------------------------------------------
