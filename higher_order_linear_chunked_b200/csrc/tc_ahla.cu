@@ -62,11 +62,12 @@ enum Mode { SUMMARY = 0, OUTPUT = 1 };
 //   R2: Y += A V  (summary: also D^T += Q^T K)          -> E2: Y to bf16 (over Q)
 //   R3: O += A Y  (output only), [dP^T ; dE^T] = [V^T ; Y^T] K
 //                                                      -> E3: state += increment, to bf16;
-//                                                             O to HBM; next chunk's loads
+//                                                             O staged over A; next loads
+// The staged O goes to HBM by TMA bulk stores while the next chunk's R1 runs.
 template <int MODE>
 __global__ void __launch_bounds__(ANT, kCtasPerSM)
 k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-            const __grid_constant__ CUtensorMap tv, Params p) {
+            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + AS_BAR);
@@ -156,27 +157,30 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
     auto k2 = [](uint64_t d0, int s) { return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4); };
     auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };                       // +2048 B
-    const uint64_t dQ = kdesc(sbase + AS_Q, 0);
-    const uint64_t dKS = kdesc(sbase + AS_K, 0);                     // B rows: K, then P0^T, E0^T
-    const uint64_t dA2 = kdesc2(sbase + AS_A, 0);
-    const uint64_t dVm = mdesc(sbase + AS_V, TILE, 0);
-    const uint64_t dYm = mdesc(sbase + AS_Q, TILE, 0);
-    const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
-    const uint64_t dVY = mdesc(sbase + AS_V, AS_Q - AS_V, 0);        // stacked [V^T ; Y^T]
-    const uint64_t dQK = mdesc(sbase + AS_Q, AS_K - AS_Q, 0);        // stacked [Q^T ; K^T]
-
+    // Operand descriptors (built where they are used: only thread 0 issues MMAs).
+    //   Q [K ; P0^T ; E0^T]^T : K-major Q and K-major B rows K, then P0^T, E0^T
+    //   A V, A Y              : K-major A (two atoms), MN-major V / Y
+    //   [V^T ; Y^T] K, [Q^T ; K^T] K : stacked MN-major A operands, MN-major K
     auto issue_r1 = [&]() {
+        const uint64_t dQ = kdesc(sbase + AS_Q, 0), dKS = kdesc(sbase + AS_K, 0);
         for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TA_A, k1(dQ, s), k1(dKS, s), I_R1, s > 0);
     };
     auto issue_r2 = [&](int n) {
+        const uint64_t dA2 = kdesc2(sbase + AS_A, 0), dVm = mdesc(sbase + AS_V, TILE, 0);
         for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_Y, k2(dA2, s), mn(dVm, s), I_N64_KM, 1);
-        if (MODE == SUMMARY)     // lanes 0-63: D^T += Q^T K (lanes 64-127 take K^T K, unused)
+        if (MODE == SUMMARY) {   // lanes 0-63: D^T += Q^T K (lanes 64-127 take K^T K, unused)
+            const uint64_t dQK = mdesc(sbase + AS_Q, AS_K - AS_Q, 0), dKm = mdesc(sbase + AS_K, TILE, 0);
             for (int s = 0; s < 8; ++s)
                 ptx::umma_bf16(tmem + TA_D, mn(dQK, s), mn(dKm, s), I_N64_MM, (n > 0 || s > 0) ? 1u : 0u);
+        }
     };
     auto issue_r3 = [&]() {
-        if (MODE == OUTPUT)
+        const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
+        if (MODE == OUTPUT) {
+            const uint64_t dA2 = kdesc2(sbase + AS_A, 0), dYm = mdesc(sbase + AS_Q, TILE, 0);
             for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_O, k2(dA2, s), mn(dYm, s), I_N64_KM, 1);
+        }
+        const uint64_t dVY = mdesc(sbase + AS_V, AS_Q - AS_V, 0);
         for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_A, mn(dVY, s), mn(dKm, s), I_N64_MM, s > 0);
     };
 
@@ -218,8 +222,9 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         ptx::tmem_ld32(tmem + lane_base + TA_Y + half * 32, v);
         st_row32(sm + AS_Q, row, half * 32, v);
     };
-    // E3: state += increment, its bf16 copy -> AS_ST; O rows of chunk n -> HBM
-    auto epi3 = [&](int n) {
+    // E3: state += increment, its bf16 copy -> AS_ST; O of the chunk (fp32) staged over the
+    // A tile as two [128 rows][32 cols] boxes in the 128B-swizzled TMA layout
+    auto epi3 = [&]() {
         float v[32];
         ptx::tmem_ld32(tmem + lane_base + TA_A + half * 32, v);
 #pragma unroll
@@ -227,24 +232,30 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if (MODE == OUTPUT || row < 64) st_row32(sm + AS_ST, row, half * 32, st);
         if (MODE == OUTPUT) {
             ptx::tmem_ld32(tmem + lane_base + TA_O + half * 32, v);
-            const int t = (chunk0 + n) * C + row;
-            if (t < p.T) {
-                float* orow = p.o + ((size_t)bh * p.T + t) * D + half * 32;
+            float4* box = reinterpret_cast<float4*>(sm + AS_A + half * (C * 128) + row * 128);
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4*>(orow + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            }
+            for (int j = 0; j < 8; ++j)
+                box[j ^ (row & 7)] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
+    };
+    // Thread 0: store the staged O of chunk n (rows past T are clipped by the tensor map).
+    auto store_o = [&](int n) {
+        const int t0 = (chunk0 + n) * C;
+        ptx::tma_store_3d(&to, sm + AS_A, 0, t0, bh);
+        ptx::tma_store_3d(&to, sm + AS_A + C * 128, 32, t0, bh);
+        ptx::bulk_commit();
     };
 
     // ---- the walk
     for (int n = 0; n < nch && ok; ++n) {
         if (tid == 0) {
+            if (MODE == OUTPUT && n > 0) store_o(n - 1);
             ok = ptx::mbar_wait(bar_load, n & 1);
             if (ok) {
                 ptx::tc_fence_after();
                 issue_r1();
             }
+            if (MODE == OUTPUT) ptx::bulk_wait_read();      // the A tile is free for E1 again
         }
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
@@ -258,9 +269,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if (tid == 0) issue_r3();
         if (!commit_wait()) { ok = false; break; }          // R3 done: Q/Y, K, V free
         if (tid == 0 && n + 1 < nch) issue_load(n + 1);
-        epi3(n);
+        epi3();
         sync_for_mma();
     }
+    if (MODE == OUTPUT && ok && tid == 0) store_o(nch - 1);
 
     // ---- summary: stage (P^T, D^T, E^T) in shared memory, then coalesced stores
     if (MODE == SUMMARY && ok) {
@@ -288,6 +300,7 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += ANT) out4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    if (MODE == OUTPUT && tid == 0) ptx::bulk_wait_all();  // O stores done before the CTA exits
     if (!ok && tid == 0) {
         set_status(p.status, DEV_TIMEOUT);
         // let a load and MMAs already in flight land before TMEM and smem are released
@@ -309,8 +322,9 @@ size_t ahla_workspace_bytes(int BH, int T) {
 
 cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
                          int* status, cudaStream_t st, cudaEvent_t* ev) {
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
+        !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
     Params prm;
@@ -328,12 +342,12 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
                                   ASMEM_BYTES)) != cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, prm);
+    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, prm);
+    k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;

@@ -100,6 +100,8 @@ __device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const 
 // ---------------------------------------------------------------- host side
 // [BH][T][64] bf16 tensor, box = one 128-token chunk, 128-byte swizzle, zero fill past T.
 bool make_map(CUtensorMap* map, const void* base, int T, int BH);
+// [BH][T][64] fp32 output, box = 32 columns x one chunk, 128-byte swizzle (TMA stores).
+bool make_map_out(CUtensorMap* map, float* base, int T, int BH);
 
 struct Plan {
     int NC;    // chunks per head

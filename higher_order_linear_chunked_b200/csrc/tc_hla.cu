@@ -33,7 +33,9 @@
 namespace hla {
 namespace tc {
 
-constexpr int NT = 256;            // threads: 8 warps, two per TMEM lane quadrant
+constexpr int NT = 256;            // epilogue threads: 8 warps, two per TMEM lane quadrant
+constexpr int NTH = NT + 32;       // + one warp that issues the TMA loads and the MMAs
+constexpr int ISSUER = NT;         // the issuing thread (lane 0 of warp 8)
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 constexpr uint32_t SM_Q0 = 0, SM_Q1 = SM_Q0 + TILE;
@@ -44,8 +46,8 @@ constexpr uint32_t SM_ONES = SM_Z + TILE;        // MN-major [tok][64], column 0
 constexpr uint32_t SM_A = SM_ONES + TILE;        // A, then W: [128][128] K-major (2 atoms)
 constexpr uint32_t SM_S0 = SM_A + 2 * TILE;      // S0^T: [64 n][64 k] K-major
 constexpr uint32_t SM_R0 = SM_S0 + 64 * 128;     // [R0 | r0]^T: [80 n][64 k] K-major
-constexpr uint32_t SM_RS = SM_R0 + 80 * 128;     // [2][128] fp32 partial row sums of W
-constexpr uint32_t SM_BAR = SM_RS + 2 * C * 4;   // mbarriers
+constexpr uint32_t SM_OST = SM_R0 + 80 * 128;    // O staging: two [128][32] fp32 TMA boxes
+constexpr uint32_t SM_BAR = SM_OST + 2 * C * 128; // mbarriers
 constexpr uint32_t SM_TOTAL = SM_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024; // + alignment slack
 
@@ -61,39 +63,40 @@ constexpr uint32_t TM_COLS = 512;
 enum Mode { SUMMARY = 0, OUTPUT = 1 };
 
 // ---------------------------------------------------------------- the walker
-// Threads: 8 warps.  Warp w reads TMEM lane quadrant (w & 3), i.e. tile rows
-// 32 (w & 3) .. + 31, and handles half (w >> 2) of each tile's columns.  Thread 0
-// also issues the TMA loads and the MMAs.
+// Threads: 8 epilogue warps and one issuing warp.  Epilogue warp w reads TMEM lane
+// quadrant (w & 3), i.e. tile rows 32 (w & 3) .. + 31, and handles half (w >> 2) of
+// each tile's columns.  Lane 0 of warp 8 issues the TMA loads and the MMAs, so the
+// epilogue warps never wait for an issue in progress.
 //
 // Rounds of MMAs per chunk n, each followed by an epilogue:
 //   R1(n): A = Q K^T, P = Q S0                      -> E1(n): A, P to bf16 tiles
 //   R2(n): W = P Q^T + A A^T, Z = P + A K,
-//          S += K^T K, O[n&1] = Q [R0|r0]^T         -> E2(n): W, Z, S0^T to bf16 tiles
+//          S += K^T K, O[n&1] = Q [R0|r0]^T         -> E2(n): W, Z, S0 to bf16 tiles
 //   R3(n): O[n&1] += W V,
 //          [C|m ; R|r] += [Q^T;Z^T][V|1]            -> E3(n): [R0|r0]^T; O[n&1] to HBM
 // R3(n) and R1(n+1) are issued together and their epilogues run together.  The O
 // accumulator is double buffered in TMEM, so the store of O(n) to HBM runs while
 // the tensor core works on R2(n+1).
 template <int MODE>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NTH, 1)
 k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-       const __grid_constant__ CUtensorMap tv, Params p) {
+       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + SM_BAR);       // [2]
     uint64_t* bar_mma = bar_load + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
-    float* rowsum_x = reinterpret_cast<float*>(sm + SM_RS);               // [2][128] partial row sums of W
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, half = (warp >> 2) & 1;
     const int row = quad * 32 + lane;                                     // TMEM lane = tile row
+    const bool epi = warp < NT / 32;                                      // an epilogue warp
     const int seg = blockIdx.x, bh = blockIdx.y;
     using S = simt_layout;
     float* slot = (MODE == OUTPUT ? p.pre : p.sums) + ((size_t)bh * p.NSp + seg) * S::size;
     if (seg >= p.NS) {                       // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
-            for (int e = tid; e < S::size / 4; e += NT) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = tid; e < S::size / 4; e += NTH) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
@@ -102,7 +105,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     const int nch = min(p.NCH, nchunks_total - chunk0);
 
     // ---- set-up: barriers, first loads, TMEM, the ones tile
-    if (tid == 0) {
+    if (tid == ISSUER) {
         ptx::mbar_init(&bar_load[0], 1);
         ptx::mbar_init(&bar_load[1], 1);
         ptx::mbar_init(bar_mma, 1);
@@ -117,7 +120,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tma_load_3d(sm + (b ? SM_K1 : SM_K0), &tk, &bar_load[b], 0, t0, bh);
         ptx::tma_load_3d(sm + (b ? SM_V1 : SM_V0), &tv, &bar_load[b], 0, t0, bh);
     };
-    if (tid == 0) {
+    if (tid == ISSUER) {
         issue_load(0);
         if (nch > 1) issue_load(1);
     }
@@ -136,7 +139,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     // coalesced loads (rows swizzled by 16-byte chunk), then every thread takes its row.
     float* stage = reinterpret_cast<float*>(sm + SM_A);                   // S [64][64] | R [64][64]
     float* stage_r = reinterpret_cast<float*>(sm + SM_Z);                 // r [64]
-    if (MODE == OUTPUT) {
+    if (MODE == OUTPUT && epi) {
         const float4* s4 = reinterpret_cast<const float4*>(slot + S::mat(0));
         const float4* r4 = reinterpret_cast<const float4*>(slot + S::mat(2));
         float4 xs[4], xr[4];
@@ -159,8 +162,9 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    {
-        // state -> TMEM (fp32) and bf16 transposed copies (S0^T, [R0|r0]^T); zeros for the summary walk
+    if (epi) {
+        // state -> TMEM (fp32) and bf16 copies (S0 rows: S is symmetric; [R0|r0]^T); zeros
+        // for the summary walk
         float v[16];
         if (quad < 2) {                      // S row `row`, columns half*32 .. +31
             for (int c0 = half * 32; c0 < half * 32 + 32; c0 += 16) {
@@ -172,7 +176,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
                     v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
                 if (MODE == OUTPUT) ptx::tmem_st16(tmem + lane_base + TM_S + c0, v);
-                st_col16(sm + SM_S0, row, c0, v);
+                st_row16(sm + SM_S0, TILE, row, c0, v);
             }
         } else {                             // [R | r] row `row - 64`, columns 0..47 / 48..79
             const int r = row - 64;
@@ -208,6 +212,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     constexpr uint32_t I_N64_KM = ptx::idesc_bf16(128, 64, false, true);
     constexpr uint32_t I_N64_MM = ptx::idesc_bf16(128, 64, true, true);
     constexpr uint32_t I_N80_KK = ptx::idesc_bf16(128, 80, false, false);
+    constexpr uint32_t I_N80_KM = ptx::idesc_bf16(128, 80, false, true);
     constexpr uint32_t I_N80_MM = ptx::idesc_bf16(128, 80, true, true);
     // Descriptor of K-step s from the step-0 descriptor: only the 14-bit start address moves.
     auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
@@ -238,12 +243,12 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         for (int s = 0; s < 8; ++s)
             ptx::umma_bf16(tmem + TM_S, mn(dKV, s), mn(dKm, s), I_N64_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
     };
-    auto issue_r3 = [&](int n) {             // O += W V ; [C|m ; R|r] += [Q^T ; Z^T] [V | 1]
+    auto issue_r3 = [&](int n) {             // [O | den] += W [V | 1] ; [C|m ; R|r] += [Q^T ; Z^T] [V | 1]
         const uint32_t sQ = bufQ(n), sV = bufV(n);
-        const uint64_t dVm = mdesc(sV, TILE, 0), dQZ = mdesc(sQ, sbase + SM_Z - sQ, 0);
+        const uint64_t dQZ = mdesc(sQ, sbase + SM_Z - sQ, 0);
         const uint64_t dV1 = mdesc(sV, sbase + SM_ONES - sV, 0);
         if (MODE == OUTPUT)
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tm_o(n), k2(dA2, s), mn(dVm, s), I_N64_KM, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tm_o(n), k2(dA2, s), mn(dV1, s), I_N80_KM, 1);
         for (int s = 0; s < 8; ++s)
             ptx::umma_bf16(tmem + TM_CR, mn(dQZ, s), mn(dV1, s), I_N80_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
     };
@@ -253,7 +258,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     // Thread 0 commits the MMAs issued so far and waits for them (bounded); the block agrees.
     auto commit_wait = [&]() -> bool {
         bool good = true;
-        if (tid == 0) {
+        if (tid == ISSUER) {
             ptx::umma_commit(bar_mma);
             good = ptx::mbar_wait(bar_mma, mma_phase);
         }
@@ -292,23 +297,18 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         if (MODE == OUTPUT) {
             const int c0 = half * 64;
             ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
-            float rs = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a = (c0 + i > row) ? 0.f : __bfloat162float(__float2bfloat16_rn(v0[i]));
-                const float b = (c0 + 32 + i > row) ? 0.f : __bfloat162float(__float2bfloat16_rn(v1[i]));
-                v0[i] = a;
-                v1[i] = b;
-                rs += a + b;
+                if (c0 + i > row) v0[i] = 0.f;
+                if (c0 + 32 + i > row) v1[i] = 0.f;
             }
-            rowsum_x[half * C + row] = rs;
             st_row32(sm + SM_A, row, c0, v0);
             st_row32(sm + SM_A, row, c0 + 32, v1);
         }
         if (quad < 2) {
             ptx::tmem_ld32x2(tmem + lane_base + TM_P + half * 32, tmem + lane_base + TM_S + half * 32, v0, v1);
             st_row32(sm + SM_Z, row, half * 32, v0);
-            st_col32(sm + SM_S0, row, half * 32, v1);
+            st_row32(sm + SM_S0, row, half * 32, v1);
         } else {
             ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
             st_row32(sm + SM_Z, row, half * 32, v0);
@@ -330,27 +330,32 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             st_col32(sm + SM_R0, r, 48, v);
         }
     };
-    // E3, output part: O rows of chunk n -> HBM (normalised)
+    // E3, output part: O rows of chunk n (normalised by column 64, q.r0 + rowsum W) staged
+    // as two [128 rows][32 cols] fp32 boxes in the 128B-swizzled TMA layout
     auto epi3_out = [&](int n) {
         float v[32];
         float d[16];
-        const uint32_t to = tm_o(n) + lane_base;
-        ptx::tmem_ld16(to + 64, d);
-        const float den = d[0] + rowsum_x[row] + rowsum_x[C + row];
-        const float scale = p.norm ? 1.f / (den + p.eps) : 1.f;
-        const int t = (chunk0 + n) * C + row;
-        ptx::tmem_ld32(to + half * 32, v);
-        if (t < p.T) {
-            float* orow = p.o + ((size_t)bh * p.T + t) * D + half * 32;
+        const uint32_t tmo = tm_o(n) + lane_base;
+        ptx::tmem_ld16(tmo + 64, d);
+        const float scale = p.norm ? 1.f / (d[0] + p.eps) : 1.f;
+        ptx::tmem_ld32(tmo + half * 32, v);
+        float4* box = reinterpret_cast<float4*>(sm + SM_OST + half * (C * 128) + row * 128);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(orow + i) =
-                    make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
-        }
+        for (int j = 0; j < 8; ++j)
+            box[j ^ (row & 7)] = make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale,
+                                             v[4 * j + 3] * scale);
+        ptx::fence_proxy_async();
+    };
+    // Issuing thread: store the staged O of chunk n (rows past T are clipped by the map).
+    auto store_o = [&](int n) {
+        const int t0 = (chunk0 + n) * C;
+        ptx::tma_store_3d(&to, sm + SM_OST, 0, t0, bh);
+        ptx::tma_store_3d(&to, sm + SM_OST + C * 128, 32, t0, bh);
+        ptx::bulk_commit();
     };
 
     // ---- the walk
-    if (tid == 0) {
+    if (tid == ISSUER) {
         ok = ptx::mbar_wait(&bar_load[0], 0);
         if (ok) {
             ptx::tc_fence_after();
@@ -360,16 +365,22 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     ok = __syncthreads_and(ok) != 0;
     for (int n = 0; n < nch && ok; ++n) {
         if (!commit_wait()) { ok = false; break; }          // R1(n) [+ R3(n-1)] done
-        epi1();
-        if (MODE == OUTPUT && n > 0) epi3_state();
-        if (tid == 0 && n >= 1 && n + 1 < nch) issue_load(n + 1);   // buffer freed by R3(n-1)
+        if (epi) {
+            epi1();
+            if (MODE == OUTPUT && n > 0) epi3_state();
+        }
+        if (tid == ISSUER) {
+            if (n >= 1 && n + 1 < nch) issue_load(n + 1);   // buffer freed by R3(n-1)
+            if (MODE == OUTPUT) ptx::bulk_wait_read();     // the O staging is free again
+        }
         sync_for_mma();
-        if (tid == 0) issue_r2(n);
-        if (MODE == OUTPUT && n > 0) epi3_out(n - 1);       // overlaps R2(n)
+        if (tid == ISSUER) issue_r2(n);
+        if (MODE == OUTPUT && n > 0 && epi) epi3_out(n - 1);   // overlaps R2(n)
         if (!commit_wait()) { ok = false; break; }          // R2(n) done
-        epi2();
+        if (MODE == OUTPUT && n > 0 && tid == ISSUER) store_o(n - 1);
+        if (epi) epi2();
         sync_for_mma();
-        if (tid == 0) {
+        if (tid == ISSUER) {
             issue_r3(n);
             if (n + 1 < nch) {
                 ok = ptx::mbar_wait(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1);
@@ -382,9 +393,15 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ok = __syncthreads_and(ok) != 0;
     }
     if (ok) {
+        if (MODE == OUTPUT && tid == ISSUER) ptx::bulk_wait_read();
         ok = commit_wait();                                  // R3(last) done
-        if (ok && MODE == OUTPUT) epi3_out(nch - 1);
+        if (ok && MODE == OUTPUT) {
+            if (epi) epi3_out(nch - 1);
+            __syncthreads();
+            if (tid == ISSUER) store_o(nch - 1);
+        }
     }
+    if (MODE == OUTPUT && tid == ISSUER) ptx::bulk_wait_all();   // O stores done before the CTA exits
 
     // ---- summary: stage the segment's state (fp32) in shared memory, then coalesced stores
     if (MODE == SUMMARY && ok) {
@@ -397,7 +414,8 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             for (int j = 0; j < 8; ++j)
                 dst[(c0 / 4 + j) ^ (rr & 7)] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
         };
-        if (quad < 2) {
+        if (!epi) {
+        } else if (quad < 2) {
             ptx::tmem_ld32(tmem + lane_base + TM_S + half * 32, v);
             put_row(0, row, half * 32, v);
             ptx::tmem_ld32(tmem + lane_base + TM_CR + half * 32, v);
@@ -418,14 +436,14 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         __syncthreads();
         float4* out4 = reinterpret_cast<float4*>(slot);
         const float4* st4 = reinterpret_cast<const float4*>(st);
-        for (int f = tid; f < 3 * D * D / 4; f += NT) {
+        for (int f = tid; f < 3 * D * D / 4; f += NTH) {
             const int rr = (f >> 4) & (D - 1);
             out4[f] = st4[(f & ~15) | ((f & 15) ^ (rr & 7))];
         }
-        for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += NT) out4[f] = st4[f];
+        for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += NTH) out4[f] = st4[f];
     }
     if (!ok) {
-        if (tid == 0) {
+        if (tid == ISSUER) {
             set_status(p.status, DEV_TIMEOUT);
             // let copies and MMAs already in flight land before TMEM and smem are released
             ptx::mbar_wait(&bar_load[0], 0, 100000000ull);
@@ -596,6 +614,18 @@ bool make_map(CUtensorMap* map, const void* base, int T, int BH) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_map_out(CUtensorMap* map, float* base, int T, int BH) {
+    EncodeTiled fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
+    const cuuint32_t box[3] = {32, (cuuint32_t)C, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 Plan plan(int BH, int T, int slots) {
     Plan pl;
     pl.NC = (T + C - 1) / C;
@@ -651,8 +681,9 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
+        !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, kSMs);
     Params prm;
@@ -670,12 +701,12 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_walk<SUMMARY><<<dim3(pl.NSp, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
+    k_walk<SUMMARY><<<dim3(pl.NSp, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    k_walk<OUTPUT><<<dim3(pl.NS, BH), NT, SMEM_BYTES, st>>>(mq, mk, mv, prm);
+    k_walk<OUTPUT><<<dim3(pl.NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
