@@ -328,7 +328,7 @@ def _traffic_from_profiles(path, w):
         return None
     if not rec:
         return None
-    src = os.path.join(ROOT, "higher_order_linear_chunked_b200", "csrc", "tc_hla.cu")
+    src = os.path.join(ROOT, rec.get("kernel_source", "higher_order_linear_chunked_b200/csrc/tc_hla.cu"))
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest() if os.path.exists(src) else None
     if rec.get("kernel_source_sha256") != sha:
         return None
