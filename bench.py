@@ -168,6 +168,10 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     if w.op == "ahla":
         # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
         flops = 6 * c * D + 4 * D * D
+    elif w.op == "hla2d" and path == "tc":
+        # per token: A* = Q K^T, Gam P Q^T, H K, W V (2cD each); Q S0, Q G0, Q M0, (Gam H K) C0
+        # (2D^2 each); H A*^T and A A^T (2c^2 each)
+        flops = 8 * c * D + 8 * D * D + 4 * c * c
     else:
         # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
         flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)

@@ -16,7 +16,7 @@ enum Op : int {
 };
 
 // Device status word values (first int of every workspace).
-enum DevStatus : int { DEV_OK = 0, DEV_TIMEOUT = 8 };
+enum DevStatus : int { DEV_OK = 0, DEV_ALIGN = 3, DEV_TIMEOUT = 8 };
 
 // Bytes reserved at the start of every workspace for the status word.
 constexpr size_t kStatusBytes = 256;

@@ -72,7 +72,7 @@ hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, f
     cudaEvent_t* ev = phase_events ? reinterpret_cast<cudaEvent_t*>(const_cast<void**>(phase_events)) : nullptr;
     cudaError_t e;
     if (use_tc(r)) {
-        e = hla::tc::forward(r.op, r.norm, q, k, v, eps, o, B * H, T, body, status, st, ev);
+        e = hla::tc::forward(r.op, r.norm, q, k, v, gamma, eps, o, B * H, H, T, body, status, st, ev);
     } else {
         e = hla::simt::forward(r.op, r.norm, r.bf16, r.d, q, k, v, gamma, eps, o, B * H, H, T,
                                reinterpret_cast<float*>(body), st, ev);

@@ -14,9 +14,9 @@ bool set_segment_chunks(int chunks);
 int kernel_launches(int op, bool norm, int BH, int T);
 // workspace bytes the path needs after the status block
 size_t workspace_bytes(int op, bool norm, int BH, int T);
-// enqueue the segment-summary walker, the Blelloch scan levels and the output walker
-cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
-                    int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
+// enqueue the forward (summaries, prefixes, output); gamma: device [H] decay factors or null
+cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
+                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 

@@ -116,6 +116,12 @@ Plan plan(int BH, int T, int slots);
 // every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st);
 
+// The decayed second-order forward, chunk-parallel (tc_decay.cu).
+size_t decay_workspace_bytes(int BH, int T);
+int decay_kernel_launches();
+cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
+                          int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
+
 // The AHLA forward on the tcgen05 walkers (tc_ahla.cu).
 size_t ahla_workspace_bytes(int BH, int T);
 cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,

@@ -1,0 +1,633 @@
+// tcgen05 path for the second-order forward with per-head decay (bf16 inputs, d = dv = 64,
+// not ratio-normalised).
+//
+// "Higher-order Linear Attention" summary (gist.science 2510.27258), Contribuciones 2 (masked
+// operators with exponential decay) and Metodología 4 (chunked scan).  Decay reading: before
+// each token's update every state is multiplied by gamma_h, then the undecayed updates run:
+//     S_t = g S_{t-1} + k k^T,   C_t = g C_{t-1} + q v^T,   G_t = g G_{t-1} + k k^T (g C_{t-1}),
+//     o_t = q_t^T (S_t C_t - G_t).
+//
+// Chunk algebra.  c = 128 tokens, local index tau.  Gam_tau = g^(tau+1), lam_tau = g^(c-1-tau),
+// rho = g^c.  A* = Q K^T (no mask), A = L (.) A*, U = strict upper part of A*,
+// At[tau][i] = g^(tau-i) A*[tau][i] for i <= tau, H[tau][i] = (g^(tau-i) - 1) A*[tau][i] for
+// i < tau (0 elsewhere).
+//   summary of a chunk from the zero state:
+//     S = K^T Lam K,   C = Q^T Lam V,   Khat = K^T K,   G = K^T (U^T Lam V)
+//   state entering chunk l (every earlier chunk is full):
+//     S0(l+1) = rho S0(l) + S_l,   C0(l+1) = rho C0(l) + C_l,
+//     G0(l+1) = rho G0(l) + G_l + rho Khat_l C0(l)
+//   output of a chunk with carried-in (S0, C0, G0), P = Q S0, M0 = S0 C0:
+//     W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T),   Dg[tau][j] = g^(tau-j)
+//     O = W V + Gam (H K) C0 + Gam^2 (Q M0) - Gam (Q G0)
+// The three cross terms are the carried-in S0 times the chunk's C (through P Q^T), the chunk's
+// decayed-minus-undecayed key moment times C0 (through H K), and the carried-in S0 C0 - G0.
+// Inside the chunk, the pair weight g^(tau-i) - [i > j] is split by i <= j (At A^T) and i > j
+// (H U^T), so every weight is applied in fp32 before the one rounding of an operand to bf16:
+// writing it as a difference of separately rounded products would lose the weight to bf16
+// rounding at strong decay (H A*^T + A A^T) or at weak decay (At A*^T - A U^T).
+//
+// Kernels (one CTA per chunk x head, every chunk independent):
+//   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G), fp32
+//   k_dec_prefix_sc, k_dec_cross, k_dec_prefix_g (CUDA cores)
+//                                               S0, C0; Y = G + rho Khat C0 and M0 = S0 C0; G0
+//   k_dec_tiles (CUDA cores)                    S0, G0^T, M0^T, C0 as bf16 operand tiles
+//                                               in the 128-byte-swizzled shared-memory layout
+//   k_dec_output (tcgen05)                      O, written by TMA bulk tensor stores
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tc.h"
+#include "tc_common.cuh"
+
+namespace hla {
+namespace tc {
+namespace {
+
+constexpr int DNT = 256;                  // 8 warps, two per TMEM lane quadrant
+constexpr int DSUM = 4 * D * D;           // summary slot: S, C, Khat (then M0), G (then Y, G0)
+constexpr uint32_t DPRE = 4 * D * D * 2;  // prefix tiles: S0, G0^T, M0^T, C0 (bf16) = 32 KB
+constexpr uint32_t QTILE = D * D * 2;     // one 64 x 64 bf16 tile = 8 KB
+
+struct DParams {
+    int T, BH, H, NC;
+    const float* gamma;
+    float* sums;      // [BH][NC][DSUM] fp32
+    uint8_t* pre;     // [BH][NC][DPRE] bf16 tiles
+    int* status;
+};
+
+// g^n for n >= 0 (binary powering).
+__device__ __forceinline__ float gpow_n(float g, int n) {
+    float r = 1.f, b = g;
+    while (n) {
+        if (n & 1) r *= b;
+        b *= b;
+        n >>= 1;
+    }
+    return r;
+}
+
+// Shared bounded commit-and-wait of the issuing thread; the block agrees on the result.
+struct MmaSync {
+    uint64_t* bar;
+    uint32_t phase;
+    __device__ bool commit_wait(bool issuer) {
+        bool good = true;
+        if (issuer) {
+            ptx::umma_commit(bar);
+            good = ptx::mbar_wait(bar, phase);
+        }
+        phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    }
+};
+
+__device__ __forceinline__ void sync_for_mma() {
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+}
+
+__device__ __forceinline__ auto k1s(uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); }
+__device__ __forceinline__ auto k2s(uint64_t d0, int s) {
+    return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4);
+}
+__device__ __forceinline__ auto mns(uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); }
+
+// ---------------------------------------------------------------- chunk summaries
+// Shared memory (offsets from the dynamic base, which is 1024-byte aligned):
+constexpr uint32_t S1_U = 0;                // U: [128 j][128 i] K-major, two atoms
+constexpr uint32_t S1_LK = S1_U + 2 * TILE; // Lam K  [tok][feat]   } equally spaced: the
+constexpr uint32_t S1_LV = S1_LK + TILE;    // Lam V  [tok][feat]   } N = 192 MN-major operand
+constexpr uint32_t S1_K = S1_LV + TILE;     // K      [tok][feat]   } [Lam K | Lam V | K]
+constexpr uint32_t S1_Q = S1_K + TILE;      // Q, then Y = U^T Lam V
+constexpr uint32_t S1_V = S1_Q + TILE;      // V
+constexpr uint32_t S1_TAB = S1_V + TILE;    // lam[128]
+constexpr uint32_t S1_BAR = S1_TAB + C * 4;
+constexpr uint32_t S1_BYTES = S1_BAR + 64;  // no slack: checked at run time
+// The summary is staged (fp32, rows swizzled by 16-byte chunk) over U, Lam K, Lam V.
+
+// Threads: warp w reads TMEM lane quadrant (w & 3) and half (w >> 2) of the columns.
+// Rounds: R1 A* = Q K^T                                -> E1: U to bf16; Lam K, Lam V
+//         R2 Y = U^T Lam V; [K^T ; Q^T][Lam K | Lam V | K]  (S, -, Khat ; -, C, -)
+//                                                      -> E2: Y to bf16; S, C, Khat staged
+//         R3 [K^T ; Y^T] Y   (lanes 0-63: G)            -> E3: G staged; summary stored
+__global__ void __launch_bounds__(DNT, 2)
+k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+              const __grid_constant__ CUtensorMap tv, DParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    if (ptx::smem_u32(sm) & 1023) {            // the swizzled tiles need a 1024-byte base
+        if (tid == 0) set_status(p.status, DEV_ALIGN);
+        return;
+    }
+    float* lam = reinterpret_cast<float*>(sm + S1_TAB);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S1_BAR);
+    MmaSync ms{bar_load + 1, 0};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
+    const float g = p.gamma[bh % p.H];
+    if (tid == 0) {
+        ptx::mbar_init(bar_load, 1);
+        ptx::mbar_init(ms.bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int t0 = chunk * C;
+        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE);
+        ptx::tma_load_3d(sm + S1_Q, &tq, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + S1_K, &tk, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + S1_V, &tv, bar_load, 0, t0, bh);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 256);
+        ptx::tmem_relinquish();
+    }
+    if (tid < C) lam[tid] = gpow_n(g, C - 1 - tid);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    bool ok = ptx::mbar_wait(bar_load, 0);     // every thread: the tiles are read below
+    if (ok && tid == 0) {
+        ptx::tc_fence_after();
+        const uint64_t dQ = kdesc(sb + S1_Q, 0), dK = kdesc(sb + S1_K, 0);
+        constexpr uint32_t I_QK = ptx::idesc_bf16(128, 128, false, false);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem, k1s(dQ, s), k1s(dK, s), I_QK, s > 0);
+    }
+    // Lam K and Lam V: scale each token row by lam; the swizzle moves 16-byte chunks within a
+    // row, so a chunk keeps its place.
+    if (ok) {
+        const float l = lam[row];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t off = row * 128 + (half * 4 + c) * 16;
+            const uint4 kx = *reinterpret_cast<const uint4*>(sm + S1_K + off);
+            const uint4 vx = *reinterpret_cast<const uint4*>(sm + S1_V + off);
+            auto scale = [&](uint32_t w) {
+                __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w);
+                const float2 f = __bfloat1622float2(h);
+                return ptx::pack_bf16(f.x * l, f.y * l);
+            };
+            *reinterpret_cast<uint4*>(sm + S1_LK + off) = make_uint4(scale(kx.x), scale(kx.y), scale(kx.z), scale(kx.w));
+            *reinterpret_cast<uint4*>(sm + S1_LV + off) = make_uint4(scale(vx.x), scale(vx.y), scale(vx.z), scale(vx.w));
+        }
+    }
+    ok = __syncthreads_and(ok) != 0;
+    if (ok) ok = ms.commit_wait(tid == 0);      // R1 done
+    if (ok) {
+        // E1: U = strict upper part of A*, row `row` (this thread: columns half*64 .. +63)
+        float v[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            ptx::tmem_ld32(tmem + lane_base + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i <= row) v[i] = 0.f;
+            st_row32(sm + S1_U, row, c0, v);
+        }
+        sync_for_mma();
+        if (tid == 0) {
+            constexpr uint32_t I_Y = ptx::idesc_bf16(128, 64, true, true);
+            constexpr uint32_t I_ST = ptx::idesc_bf16(128, 192, true, true);
+            const uint64_t dU = mdesc(sb + S1_U, TILE, 0), dLV = mdesc(sb + S1_LV, TILE, 0);
+            const uint64_t dKQ = mdesc(sb + S1_K, S1_Q - S1_K, 0), dB3 = mdesc(sb + S1_LK, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 192, mns(dU, s), mns(dLV, s), I_Y, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dKQ, s), mns(dB3, s), I_ST, s > 0);
+        }
+        ok = ms.commit_wait(tid == 0);          // R2 done
+    }
+    float* stg = reinterpret_cast<float*>(sm + S1_U);   // [4][64][64] fp32, rows chunk-swizzled
+    auto put_row = [&](int m, int r, int c0, const float (&x)[32]) {
+        float4* dst = reinterpret_cast<float4*>(stg + m * D * D + r * D);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            dst[(c0 / 4 + j) ^ (r & 7)] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+    };
+    if (ok) {
+        // E2: Y -> bf16 over Q; S (lanes 0-63, cols 0-63), Khat (lanes 0-63, cols 128-191),
+        // C (lanes 64-127, cols 64-127) staged
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + 192 + half * 32, v);
+        st_row32(sm + S1_Q, row, half * 32, v);
+        if (quad < 2) {
+            ptx::tmem_ld32(tmem + lane_base + half * 32, v);
+            put_row(0, row, half * 32, v);
+            ptx::tmem_ld32(tmem + lane_base + 128 + half * 32, v);
+            put_row(2, row, half * 32, v);
+        } else {
+            ptx::tmem_ld32(tmem + lane_base + 64 + half * 32, v);
+            put_row(1, row - 64, half * 32, v);
+        }
+        sync_for_mma();
+        if (tid == 0) {
+            constexpr uint32_t I_G = ptx::idesc_bf16(128, 64, true, true);
+            const uint64_t dKY = mdesc(sb + S1_K, S1_Q - S1_K, 0), dY = mdesc(sb + S1_Q, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dKY, s), mns(dY, s), I_G, s > 0);
+        }
+        ok = ms.commit_wait(tid == 0);          // R3 done
+    }
+    if (ok) {
+        if (quad < 2) {
+            float v[32];
+            ptx::tmem_ld32(tmem + lane_base + half * 32, v);
+            put_row(3, row, half * 32, v);
+        }
+        __syncthreads();
+        float4* out4 = reinterpret_cast<float4*>(p.sums + ((size_t)bh * p.NC + chunk) * DSUM);
+        const float4* st4 = reinterpret_cast<const float4*>(stg);
+        for (int f = tid; f < DSUM / 4; f += DNT) {
+            const int r = (f >> 4) & (D - 1);
+            out4[f] = st4[(f & ~15) | ((f & 15) ^ (r & 7))];
+        }
+    } else if (tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        ptx::mbar_wait(bar_load, 0, 100000000ull);
+        ptx::umma_commit(ms.bar);
+        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------- prefixes (CUDA cores)
+constexpr int PNT = 256;
+
+// Exclusive decayed prefix over chunks of S (slot matrix 0) and C (matrix 1), in place:
+// X0(0) = 0, X0(l+1) = rho X0(l) + X_l.  One thread per matrix element.
+__global__ void __launch_bounds__(PNT) k_dec_prefix_sc(DParams p) {
+    const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
+    if (e >= 2 * D * D) return;
+    const float rho = gpow_n(p.gamma[bh % p.H], C);
+    float* x = p.sums + (size_t)bh * p.NC * DSUM + e;
+    float run = 0.f;
+    for (int l0 = 0; l0 < p.NC; l0 += 8) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < p.NC) {
+                x[(size_t)(l0 + i) * DSUM] = run;
+                run = fmaf(rho, run, y[i]);
+            }
+    }
+}
+
+// Per chunk: Y = G + rho Khat C0 (into matrix 3) and M0 = S0 C0 (into matrix 2).
+constexpr int XLD = D + 4;   // padded row stride of the left operands
+__global__ void __launch_bounds__(PNT) k_dec_cross(DParams p) {
+    extern __shared__ __align__(16) float xs[];
+    float* Kh = xs;                 // [64][XLD]
+    float* S0 = Kh + D * XLD;       // [64][XLD]
+    float* C0 = S0 + D * XLD;       // [64][64]
+    const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    float* slot = p.sums + ((size_t)bh * p.NC + l) * DSUM;
+    const float rho = gpow_n(p.gamma[bh % p.H], C);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int f = tid + PNT * i, r = f >> 4, c4 = f & 15;
+        const float4 s = reinterpret_cast<const float4*>(slot)[f];
+        const float4 c = reinterpret_cast<const float4*>(slot + D * D)[f];
+        const float4 k = reinterpret_cast<const float4*>(slot + 2 * D * D)[f];
+        *reinterpret_cast<float4*>(S0 + r * XLD + 4 * c4) = s;
+        *reinterpret_cast<float4*>(Kh + r * XLD + 4 * c4) = k;
+        reinterpret_cast<float4*>(C0)[f] = c;
+    }
+    __syncthreads();
+    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);
+    float y[4][4], m[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const float4 gx = *reinterpret_cast<const float4*>(slot + 3 * D * D + (r + a) * D + c);
+        y[a][0] = gx.x; y[a][1] = gx.y; y[a][2] = gx.z; y[a][3] = gx.w;
+        m[a][0] = m[a][1] = m[a][2] = m[a][3] = 0.f;
+    }
+#pragma unroll 8
+    for (int k = 0; k < D; ++k) {
+        const float4 cv = *reinterpret_cast<const float4*>(C0 + k * D + c);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float kv = rho * Kh[(r + a) * XLD + k], sv = S0[(r + a) * XLD + k];
+            y[a][0] = fmaf(kv, cv.x, y[a][0]); y[a][1] = fmaf(kv, cv.y, y[a][1]);
+            y[a][2] = fmaf(kv, cv.z, y[a][2]); y[a][3] = fmaf(kv, cv.w, y[a][3]);
+            m[a][0] = fmaf(sv, cv.x, m[a][0]); m[a][1] = fmaf(sv, cv.y, m[a][1]);
+            m[a][2] = fmaf(sv, cv.z, m[a][2]); m[a][3] = fmaf(sv, cv.w, m[a][3]);
+        }
+    }
+    __syncthreads();   // every thread has read Khat before M0 overwrites it
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        *reinterpret_cast<float4*>(slot + 3 * D * D + (r + a) * D + c) = make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
+        *reinterpret_cast<float4*>(slot + 2 * D * D + (r + a) * D + c) = make_float4(m[a][0], m[a][1], m[a][2], m[a][3]);
+    }
+}
+
+// Exclusive decayed prefix of Y (matrix 3) into G0, in place.
+__global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
+    const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
+    if (e >= D * D) return;
+    const float rho = gpow_n(p.gamma[bh % p.H], C);
+    float* x = p.sums + (size_t)bh * p.NC * DSUM + 3 * D * D + e;
+    float run = 0.f;
+    for (int l0 = 0; l0 < p.NC; l0 += 8) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < p.NC) {
+                x[(size_t)(l0 + i) * DSUM] = run;
+                run = fmaf(rho, run, y[i]);
+            }
+    }
+}
+
+// Per chunk: the bf16 operand tiles of the output kernel, in the 128-byte-swizzled layout
+// (row r of a tile at r * 128 bytes, 16-byte chunk j at position j ^ (r & 7)):
+//   tile 0: S0^T (row n = column n of S0)     B operand of Q S0 (K-major)
+//   tile 1: G0^T                               B operand of Q G0 (K-major)
+//   tile 2: M0^T                               B operand of Q M0 (K-major)
+//   tile 3: C0 (row k = row k of C0)           B operand of (H K) C0 (MN-major)
+__global__ void __launch_bounds__(PNT) k_dec_tiles(DParams p) {
+    __shared__ float ts[D * (D + 1)];
+    const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    const float* slot = p.sums + ((size_t)bh * p.NC + l) * DSUM;
+    uint8_t* out = p.pre + ((size_t)bh * p.NC + l) * DPRE;
+    const int src[4] = {0, 3, 2, 1};           // slot matrices: S0, G0, M0, C0
+    for (int t = 0; t < 4; ++t) {
+        const float* m = slot + src[t] * D * D;
+        for (int e = tid; e < D * D; e += PNT) ts[(e >> 6) * (D + 1) + (e & 63)] = m[e];
+        __syncthreads();
+        // this thread: 16-byte chunks (r, j) = (f / 8, f % 8) for f = tid, tid + 256
+        for (int f = tid; f < D * 8; f += PNT) {
+            const int r = f >> 3, j = f & 7;
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = 8 * j + i;
+                x[i] = (t < 3) ? ts[c * (D + 1) + r] : ts[r * (D + 1) + c];   // transposed for 0-2
+            }
+            const uint4 u = make_uint4(ptx::pack_bf16(x[0], x[1]), ptx::pack_bf16(x[2], x[3]),
+                                       ptx::pack_bf16(x[4], x[5]), ptx::pack_bf16(x[6], x[7]));
+            *reinterpret_cast<uint4*>(out + t * QTILE + r * 128 + ((j ^ (r & 7)) << 4)) = u;
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- output
+// Shared memory:
+constexpr uint32_t S3_Q = 0;                 // Q [tok][feat]
+constexpr uint32_t S3_K = S3_Q + TILE;       // K                    } B rows of R1:
+constexpr uint32_t S3_SG = S3_K + TILE;      // S0^T, G0^T tiles      } [K ; S0^T ; G0^T]
+constexpr uint32_t S3_M0 = S3_SG + 2 * QTILE;   // M0^T
+constexpr uint32_t S3_C0 = S3_M0 + QTILE;    // C0
+constexpr uint32_t S3_V = S3_C0 + QTILE;     // V
+constexpr uint32_t S3_AT = S3_V + TILE;      // At, later the O staging boxes
+constexpr uint32_t S3_H = S3_AT + 2 * TILE;  // H, later W
+constexpr uint32_t S3_A = S3_H + 2 * TILE;   // A
+constexpr uint32_t S3_U = S3_A + 2 * TILE;   // U
+constexpr uint32_t S3_P = S3_U + 2 * TILE;   // Gam P, later Gam (H K)
+constexpr uint32_t S3_TAB = S3_P + TILE;     // g^n, n = 0..256
+constexpr uint32_t S3_BAR = S3_TAB + 260 * 4;
+constexpr uint32_t S3_BYTES = S3_BAR + 64 + 1024;   // + alignment slack
+
+// TMEM columns
+constexpr uint32_t T3_AS = 0;     // A*, then W   (128)
+constexpr uint32_t T3_P = 128;    // P, then H K  (64)
+constexpr uint32_t T3_QG = 192;   // Q G0         (64)
+constexpr uint32_t T3_QM = 256;   // Q M0         (64)
+constexpr uint32_t T3_O = 320;    // O            (64)
+
+// Rounds: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T, Q M0    -> E1: At, H, A, U, Gam P to bf16
+//         R2 W = Gam P Q^T + At A^T + H U^T; H K               -> E2: W (masked, Dg), Gam H K
+//         R3 O = W V + (Gam H K) C0                            -> E3: O + Gam^2 Q M0 - Gam Q G0
+__global__ void __launch_bounds__(DNT, 1)
+k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, DParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    float* gp = reinterpret_cast<float*>(sm + S3_TAB);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S3_BAR);
+    MmaSync ms{bar_load + 1, 0};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
+    const float g = p.gamma[bh % p.H];
+    if (tid == 0) {
+        ptx::mbar_init(bar_load, 1);
+        ptx::mbar_init(ms.bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int t0 = chunk * C;
+        const uint8_t* pre = p.pre + ((size_t)bh * p.NC + chunk) * DPRE;
+        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE + DPRE);
+        ptx::tma_load_3d(sm + S3_Q, &tq, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + S3_K, &tk, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + S3_V, &tv, bar_load, 0, t0, bh);
+        ptx::bulk_load(sm + S3_SG, pre, 3 * QTILE, bar_load);          // S0^T, G0^T, M0^T
+        ptx::bulk_load(sm + S3_C0, pre + 3 * QTILE, QTILE, bar_load);  // C0
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    bool ok = true;
+    if (tid == 0) {
+        ok = ptx::mbar_wait(bar_load, 0);
+        if (ok) {
+            ptx::tc_fence_after();
+            constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 256, false, false);
+            constexpr uint32_t I_N64 = ptx::idesc_bf16(128, 64, false, false);
+            const uint64_t dQ = kdesc(sb + S3_Q, 0), dKSG = kdesc(sb + S3_K, 0), dM = kdesc(sb + S3_M0, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dQ, s), k1s(dKSG, s), I_R1, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_QM, k1s(dQ, s), k1s(dM, s), I_N64, s > 0);
+        }
+    }
+    ok = __syncthreads_and(ok) != 0;
+    if (ok) ok = ms.commit_wait(tid == 0);      // R1 done
+    if (ok) {
+        // E1: from A* row `row` (columns half*64 .. +63): At, H, A, U; Gam P (columns half*32 .. +31)
+        float v[32], w[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int d = row - (c0 + i);                          // tau - i
+                w[i] = d >= 0 ? gp[d] * v[i] : 0.f;                    // At
+            }
+            st_row32(sm + S3_AT, row, c0, w);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int d = row - (c0 + i);
+                w[i] = d > 0 ? (gp[d] - 1.f) * v[i] : 0.f;            // H
+            }
+            st_row32(sm + S3_H, row, c0, w);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = (c0 + i <= row) ? v[i] : 0.f;   // A
+            st_row32(sm + S3_A, row, c0, w);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = (c0 + i > row) ? v[i] : 0.f;    // U
+            st_row32(sm + S3_U, row, c0, w);
+        }
+        ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
+        const float gam = gp[row + 1];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= gam;
+        st_row32(sm + S3_P, row, half * 32, v);
+        sync_for_mma();
+        if (tid == 0) {
+            constexpr uint32_t I_W = ptx::idesc_bf16(128, 128, false, false);
+            constexpr uint32_t I_HK = ptx::idesc_bf16(128, 64, false, true);
+            const uint64_t dP = kdesc(sb + S3_P, 0), dQ = kdesc(sb + S3_Q, 0);
+            const uint64_t dAt = kdesc2(sb + S3_AT, 0), dA = kdesc2(sb + S3_A, 0);
+            const uint64_t dH = kdesc2(sb + S3_H, 0), dU = kdesc2(sb + S3_U, 0);
+            const uint64_t dKm = mdesc(sb + S3_K, TILE, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dP, s), k1s(dQ, s), I_W, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dAt, s), k2s(dA, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dH, s), k2s(dU, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_P, k2s(dH, s), mns(dKm, s), I_HK, s > 0);
+        }
+        ok = ms.commit_wait(tid == 0);          // R2 done
+    }
+    if (ok) {
+        // E2: W[tau][j] = g^(tau-j) x for j <= tau -> over H; Gam (H K) -> over Gam P
+        float v[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int d = row - (c0 + i);
+                v[i] = d >= 0 ? gp[d] * v[i] : 0.f;
+            }
+            st_row32(sm + S3_H, row, c0, v);
+        }
+        ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
+        const float gam = gp[row + 1];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= gam;
+        st_row32(sm + S3_P, row, half * 32, v);
+        sync_for_mma();
+        if (tid == 0) {
+            constexpr uint32_t I_O = ptx::idesc_bf16(128, 64, false, true);
+            const uint64_t dW = kdesc2(sb + S3_H, 0), dVm = mdesc(sb + S3_V, TILE, 0);
+            const uint64_t dP = kdesc(sb + S3_P, 0), dC = mdesc(sb + S3_C0, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_O, k2s(dW, s), mns(dVm, s), I_O, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_O, k1s(dP, s), mns(dC, s), I_O, 1);
+        }
+        ok = ms.commit_wait(tid == 0);          // R3 done
+    }
+    if (ok) {
+        // E3: O + Gam^2 (Q M0) - Gam (Q G0), staged as two [128][32] fp32 boxes over At
+        float o[32], m[32];
+        ptx::tmem_ld32(tmem + lane_base + T3_O + half * 32, o);
+        ptx::tmem_ld32(tmem + lane_base + T3_QM + half * 32, m);
+        const float gam = gp[row + 1], gam2 = gp[2 * row + 2];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = fmaf(gam2, m[i], o[i]);
+        ptx::tmem_ld32(tmem + lane_base + T3_QG + half * 32, m);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = fmaf(-gam, m[i], o[i]);
+        float4* box = reinterpret_cast<float4*>(sm + S3_AT + half * (C * 128) + row * 128);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) box[j ^ (row & 7)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+        ptx::fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            ptx::tma_store_3d(&to, sm + S3_AT, 0, chunk * C, bh);
+            ptx::tma_store_3d(&to, sm + S3_AT + C * 128, 32, chunk * C, bh);
+            ptx::bulk_commit();
+            ptx::bulk_wait_all();
+        }
+    } else if (tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        ptx::mbar_wait(bar_load, 0, 100000000ull);
+        ptx::umma_commit(ms.bar);
+        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+size_t decay_workspace_bytes(int BH, int T) {
+    const size_t NC = (size_t)(T + C - 1) / C;
+    return (size_t)BH * NC * (DSUM * sizeof(float) + DPRE);
+}
+
+int decay_kernel_launches() { return 6; }
+
+cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
+                          int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
+    if (!gamma || H < 1) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
+        !make_map_out(&mo, o, T, BH))
+        return cudaErrorInvalidValue;
+    DParams prm;
+    prm.T = T; prm.BH = BH; prm.H = H; prm.NC = (T + C - 1) / C;
+    prm.gamma = gamma;
+    prm.sums = static_cast<float*>(ws);
+    prm.pre = reinterpret_cast<uint8_t*>(prm.sums + (size_t)BH * prm.NC * DSUM);
+    prm.status = status;
+    const int NC = prm.NC;
+    const size_t cross_smem = sizeof(float) * (2 * D * XLD + D * D);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k_dec_summary, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_BYTES)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_dec_cross, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cross_smem)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(k_dec_output, cudaFuncAttributeMaxDynamicSharedMemorySize, S3_BYTES)) != cudaSuccess)
+        return e;
+    if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
+    k_dec_summary<<<dim3(NC, BH), DNT, S1_BYTES, st>>>(mq, mk, mv, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
+    k_dec_prefix_sc<<<dim3((2 * D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_dec_cross<<<dim3(NC, BH), PNT, cross_smem, st>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_dec_prefix_g<<<dim3((D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_dec_tiles<<<dim3(NC, BH), PNT, 0, st>>>(prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
+    k_dec_output<<<dim3(NC, BH), DNT, S3_BYTES, st>>>(mq, mk, mv, mo, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
+    return cudaSuccess;
+}
+
+}  // namespace tc
+}  // namespace hla

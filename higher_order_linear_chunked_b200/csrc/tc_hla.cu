@@ -666,19 +666,26 @@ bool set_segment_chunks(int chunks) {
     return true;
 }
 
-bool supported(int op, bool /*norm*/, bool bf16, int d) { return (op == OP_HLA2 || op == OP_AHLA) && bf16 && d == D; }
+bool supported(int op, bool norm, bool bf16, int d) {
+    if (!bf16 || d != D) return false;
+    return op == OP_HLA2 || op == OP_AHLA || (op == OP_HLA2D && !norm);
+}
 
 size_t workspace_bytes(int op, bool /*norm*/, int BH, int T) {
     if (op == OP_AHLA) return ahla_workspace_bytes(BH, T);
+    if (op == OP_HLA2D) return decay_workspace_bytes(BH, T);
     const Plan pl = plan(BH, T, kSMs);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-int kernel_launches(int /*op*/, bool /*norm*/, int /*BH*/, int /*T*/) { return 4; }
+int kernel_launches(int op, bool /*norm*/, int /*BH*/, int /*T*/) {
+    return op == OP_HLA2D ? decay_kernel_launches() : 4;
+}
 
-cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, float eps, float* o, int BH,
-                    int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
+cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
+                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
     if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev);
+    if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;

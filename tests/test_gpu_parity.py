@@ -98,7 +98,7 @@ def test_many_heads_short_sequences(op):
     assert oracle.max_row_rel_err(o.cpu(), reference(op, q, k, v, g)) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla"])
 @pytest.mark.parametrize("T", [127, 128, 129, 1000, 1024, 2049])
 def test_bf16_d64_parity_across_segments(op, T):
     """bf16 d = 64 (the tensor-core shapes) over many chunks and a ragged tail."""
@@ -144,7 +144,8 @@ def test_tensor_core_path_is_used_for_bf16_d64():
     assert hla.uses_tensor_cores(hla.OP_HLA2_NORM, hla.HLA_BF16, False, 4, 16, 4096, 64, 64)
     assert hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, False, 1, 1, 100, 64, 64)
     assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_F32, False, 1, 1, 100, 64, 64)
-    assert not hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, True, 1, 1, 100, 64, 64)
+    assert hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_BF16, True, 2, 16, 16384, 64, 64)       # decayed
+    assert not hla.uses_tensor_cores(hla.OP_HLA2_NORM, hla.HLA_BF16, True, 1, 1, 100, 64, 64)  # normalised + decay
     assert hla.uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, False, 4, 16, 8192, 64, 64)
     assert not hla.uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, False, 1, 1, 100, 32, 32)
     assert not hla.uses_tensor_cores(hla.OP_HLA3, hla.HLA_BF16, False, 1, 1, 100, 64, 64)
@@ -205,6 +206,30 @@ def test_decay_gamma_one_matches_undecayed():
     a = gpu_forward("hla2d", q, k, v, torch.ones(2))
     b = gpu_forward("hla2", q, k, v, None)
     assert oracle.max_row_rel_err(a.cpu(), b.cpu()) < 1e-5
+
+
+@pytest.mark.parametrize("T", [300, 2049])
+def test_decay_gamma_one_matches_undecayed_tensor_cores(T):
+    """bf16 d = 64: the decayed tensor-core path at gamma = 1 against the undecayed one (both
+    differ from the oracle only by bf16 operand rounding)."""
+    w = recipe("hla2", "bf16", 1, 2, T, 64, seed=T)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    a = gpu_forward("hla2d", q, k, v, torch.ones(2))
+    b = gpu_forward("hla2", q, k, v, None)
+    ref = oracle.recur("hla2", q, k, v)
+    assert oracle.max_row_rel_err(a.cpu(), ref) <= TOL["bf16"]
+    assert oracle.max_row_rel_err(a.cpu(), b.cpu()) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("gam", [0.5, 0.95, 0.999])
+def test_decay_strong_and_weak_tensor_cores(gam):
+    """bf16 d = 64 decayed path for one gamma per run, strong to weak decay, ragged tail."""
+    w = recipe("hla2d", "bf16", 1, 2, 777, 64, seed=int(gam * 1000))
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    g = torch.full((2,), gam)
+    o = gpu_forward("hla2d", q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2d", q, k, v, gamma=g))
+    assert err <= TOL["bf16"], err
 
 
 # ---------------------------------------------------------------------------
