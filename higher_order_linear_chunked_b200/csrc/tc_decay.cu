@@ -16,11 +16,12 @@
 //   state entering chunk l (every earlier chunk is full):
 //     S0(l+1) = rho S0(l) + S_l,   C0(l+1) = rho C0(l) + C_l,
 //     G0(l+1) = rho G0(l) + G_l + rho Khat_l C0(l)
-//   output of a chunk with carried-in (S0, C0, G0), P = Q S0, M0 = S0 C0:
+//   output of a chunk with carried-in (S0, C0, G0), P = Q S0:
 //     W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T),   Dg[tau][j] = g^(tau-j)
-//     O = W V + Gam (H K) C0 + Gam^2 (Q M0) - Gam (Q G0)
-// The three cross terms are the carried-in S0 times the chunk's C (through P Q^T), the chunk's
-// decayed-minus-undecayed key moment times C0 (through H K), and the carried-in S0 C0 - G0.
+//     O = W V + Gam (Gam P + H K) C0 - Gam (Q G0)
+// The cross terms are the carried-in S0 times the chunk's C (through P Q^T), the chunk's
+// decayed-minus-undecayed key moment times C0 (through H K), and the carried-in
+// Gam S0 C0 - G0 (through Gam P C0 and Q G0).
 // Inside the chunk, the pair weight g^(tau-i) - [i > j] is split by i <= j (At A^T) and i > j
 // (H U^T), so every weight is applied in fp32 before the one rounding of an operand to bf16:
 // writing it as a difference of separately rounded products would lose the weight to bf16
@@ -29,10 +30,10 @@
 // Kernels (one CTA per chunk x head, every chunk independent):
 //   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G), fp32
 //   k_dec_prefix_sc, k_dec_cross, k_dec_prefix_g (CUDA cores)
-//                                               S0, C0; Y = G + rho Khat C0 and M0 = S0 C0; G0
-//   k_dec_tiles (CUDA cores)                    S0, G0^T, M0^T, C0 as bf16 operand tiles
-//                                               in the 128-byte-swizzled shared-memory layout
-//   k_dec_output (tcgen05)                      O, written by TMA bulk tensor stores
+//                                               in place: S0, C0; Y = G + rho Khat C0; G0
+//   k_dec_output (tcgen05)                      turns (S0, C0, G0) into bf16 operand tiles
+//                                               while its Q/K/V loads are in flight; O,
+//                                               written by TMA bulk tensor stores
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -47,15 +48,13 @@ namespace tc {
 namespace {
 
 constexpr int DNT = 256;                  // 8 warps, two per TMEM lane quadrant
-constexpr int DSUM = 4 * D * D;           // summary slot: S, C, Khat (then M0), G (then Y, G0)
-constexpr uint32_t DPRE = 4 * D * D * 2;  // prefix tiles: S0, G0^T, M0^T, C0 (bf16) = 32 KB
+constexpr int DSUM = 4 * D * D;           // summary slot: S, C, Khat, G (then Y, then G0)
 constexpr uint32_t QTILE = D * D * 2;     // one 64 x 64 bf16 tile = 8 KB
 
 struct DParams {
     int T, BH, H, NC;
     const float* gamma;
     float* sums;      // [BH][NC][DSUM] fp32
-    uint8_t* pre;     // [BH][NC][DPRE] bf16 tiles
     int* status;
 };
 
@@ -274,13 +273,13 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_sc(DParams p) {
     const float rho = gpow_n(p.gamma[bh % p.H], C);
     float* x = p.sums + (size_t)bh * p.NC * DSUM + e;
     float run = 0.f;
-    for (int l0 = 0; l0 < p.NC; l0 += 8) {
-        float y[8];
+    for (int l0 = 0; l0 < p.NC; l0 += 16) {
+        float y[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) {
                 x[(size_t)(l0 + i) * DSUM] = run;
                 run = fmaf(rho, run, y[i]);
@@ -288,53 +287,43 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_sc(DParams p) {
     }
 }
 
-// Per chunk: Y = G + rho Khat C0 (into matrix 3) and M0 = S0 C0 (into matrix 2).
-constexpr int XLD = D + 4;   // padded row stride of the left operands
+// Per chunk: Y = G + rho Khat C0, in place of G (matrix 3).
+constexpr int XLD = D + 4;   // padded row stride of the left operand
 __global__ void __launch_bounds__(PNT) k_dec_cross(DParams p) {
-    extern __shared__ __align__(16) float xs[];
-    float* Kh = xs;                 // [64][XLD]
-    float* S0 = Kh + D * XLD;       // [64][XLD]
-    float* C0 = S0 + D * XLD;       // [64][64]
+    __shared__ __align__(16) float Kh[D * XLD];
+    __shared__ __align__(16) float C0[D * D];
     const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     float* slot = p.sums + ((size_t)bh * p.NC + l) * DSUM;
     const float rho = gpow_n(p.gamma[bh % p.H], C);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int f = tid + PNT * i, r = f >> 4, c4 = f & 15;
-        const float4 s = reinterpret_cast<const float4*>(slot)[f];
         const float4 c = reinterpret_cast<const float4*>(slot + D * D)[f];
         const float4 k = reinterpret_cast<const float4*>(slot + 2 * D * D)[f];
-        *reinterpret_cast<float4*>(S0 + r * XLD + 4 * c4) = s;
-        *reinterpret_cast<float4*>(Kh + r * XLD + 4 * c4) = k;
+        *reinterpret_cast<float4*>(Kh + r * XLD + 4 * c4) = make_float4(rho * k.x, rho * k.y, rho * k.z, rho * k.w);
         reinterpret_cast<float4*>(C0)[f] = c;
     }
     __syncthreads();
     const int r = 4 * (tid >> 4), c = 4 * (tid & 15);
-    float y[4][4], m[4][4];
+    float y[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
         const float4 gx = *reinterpret_cast<const float4*>(slot + 3 * D * D + (r + a) * D + c);
         y[a][0] = gx.x; y[a][1] = gx.y; y[a][2] = gx.z; y[a][3] = gx.w;
-        m[a][0] = m[a][1] = m[a][2] = m[a][3] = 0.f;
     }
 #pragma unroll 8
     for (int k = 0; k < D; ++k) {
         const float4 cv = *reinterpret_cast<const float4*>(C0 + k * D + c);
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-            const float kv = rho * Kh[(r + a) * XLD + k], sv = S0[(r + a) * XLD + k];
+            const float kv = Kh[(r + a) * XLD + k];
             y[a][0] = fmaf(kv, cv.x, y[a][0]); y[a][1] = fmaf(kv, cv.y, y[a][1]);
             y[a][2] = fmaf(kv, cv.z, y[a][2]); y[a][3] = fmaf(kv, cv.w, y[a][3]);
-            m[a][0] = fmaf(sv, cv.x, m[a][0]); m[a][1] = fmaf(sv, cv.y, m[a][1]);
-            m[a][2] = fmaf(sv, cv.z, m[a][2]); m[a][3] = fmaf(sv, cv.w, m[a][3]);
         }
     }
-    __syncthreads();   // every thread has read Khat before M0 overwrites it
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
+    for (int a = 0; a < 4; ++a)
         *reinterpret_cast<float4*>(slot + 3 * D * D + (r + a) * D + c) = make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
-        *reinterpret_cast<float4*>(slot + 2 * D * D + (r + a) * D + c) = make_float4(m[a][0], m[a][1], m[a][2], m[a][3]);
-    }
 }
 
 // Exclusive decayed prefix of Y (matrix 3) into G0, in place.
@@ -344,13 +333,13 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
     const float rho = gpow_n(p.gamma[bh % p.H], C);
     float* x = p.sums + (size_t)bh * p.NC * DSUM + 3 * D * D + e;
     float run = 0.f;
-    for (int l0 = 0; l0 < p.NC; l0 += 8) {
-        float y[8];
+    for (int l0 = 0; l0 < p.NC; l0 += 16) {
+        float y[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) {
                 x[(size_t)(l0 + i) * DSUM] = run;
                 run = fmaf(rho, run, y[i]);
@@ -358,48 +347,14 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
     }
 }
 
-// Per chunk: the bf16 operand tiles of the output kernel, in the 128-byte-swizzled layout
-// (row r of a tile at r * 128 bytes, 16-byte chunk j at position j ^ (r & 7)):
-//   tile 0: S0^T (row n = column n of S0)     B operand of Q S0 (K-major)
-//   tile 1: G0^T                               B operand of Q G0 (K-major)
-//   tile 2: M0^T                               B operand of Q M0 (K-major)
-//   tile 3: C0 (row k = row k of C0)           B operand of (H K) C0 (MN-major)
-__global__ void __launch_bounds__(PNT) k_dec_tiles(DParams p) {
-    __shared__ float ts[D * (D + 1)];
-    const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const float* slot = p.sums + ((size_t)bh * p.NC + l) * DSUM;
-    uint8_t* out = p.pre + ((size_t)bh * p.NC + l) * DPRE;
-    const int src[4] = {0, 3, 2, 1};           // slot matrices: S0, G0, M0, C0
-    for (int t = 0; t < 4; ++t) {
-        const float* m = slot + src[t] * D * D;
-        for (int e = tid; e < D * D; e += PNT) ts[(e >> 6) * (D + 1) + (e & 63)] = m[e];
-        __syncthreads();
-        // this thread: 16-byte chunks (r, j) = (f / 8, f % 8) for f = tid, tid + 256
-        for (int f = tid; f < D * 8; f += PNT) {
-            const int r = f >> 3, j = f & 7;
-            float x[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = 8 * j + i;
-                x[i] = (t < 3) ? ts[c * (D + 1) + r] : ts[r * (D + 1) + c];   // transposed for 0-2
-            }
-            const uint4 u = make_uint4(ptx::pack_bf16(x[0], x[1]), ptx::pack_bf16(x[2], x[3]),
-                                       ptx::pack_bf16(x[4], x[5]), ptx::pack_bf16(x[6], x[7]));
-            *reinterpret_cast<uint4*>(out + t * QTILE + r * 128 + ((j ^ (r & 7)) << 4)) = u;
-        }
-        __syncthreads();
-    }
-}
-
 // ---------------------------------------------------------------- output
 // Shared memory:
 constexpr uint32_t S3_Q = 0;                 // Q [tok][feat]
 constexpr uint32_t S3_K = S3_Q + TILE;       // K                    } B rows of R1:
-constexpr uint32_t S3_SG = S3_K + TILE;      // S0^T, G0^T tiles      } [K ; S0^T ; G0^T]
-constexpr uint32_t S3_M0 = S3_SG + 2 * QTILE;   // M0^T
-constexpr uint32_t S3_C0 = S3_M0 + QTILE;    // C0
+constexpr uint32_t S3_SG = S3_K + TILE;      // S0 (rows), G0^T tiles } [K ; S0^T ; G0^T]
+constexpr uint32_t S3_C0 = S3_SG + 2 * QTILE;   // C0 (rows: MN-major B operand)
 constexpr uint32_t S3_V = S3_C0 + QTILE;     // V
-constexpr uint32_t S3_AT = S3_V + TILE;      // At, later the O staging boxes
+constexpr uint32_t S3_AT = S3_V + TILE;      // G0 staging (fp32), At, later the O staging boxes
 constexpr uint32_t S3_H = S3_AT + 2 * TILE;  // H, later W
 constexpr uint32_t S3_A = S3_H + 2 * TILE;   // A
 constexpr uint32_t S3_U = S3_A + 2 * TILE;   // U
@@ -410,14 +365,17 @@ constexpr uint32_t S3_BYTES = S3_BAR + 64 + 1024;   // + alignment slack
 
 // TMEM columns
 constexpr uint32_t T3_AS = 0;     // A*, then W   (128)
-constexpr uint32_t T3_P = 128;    // P, then H K  (64)
+constexpr uint32_t T3_P = 128;    // P            (64)
 constexpr uint32_t T3_QG = 192;   // Q G0         (64)
-constexpr uint32_t T3_QM = 256;   // Q M0         (64)
+constexpr uint32_t T3_HK = 256;   // H K          (64)
 constexpr uint32_t T3_O = 320;    // O            (64)
 
-// Rounds: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T, Q M0    -> E1: At, H, A, U, Gam P to bf16
-//         R2 W = Gam P Q^T + At A^T + H U^T; H K               -> E2: W (masked, Dg), Gam H K
-//         R3 O = W V + (Gam H K) C0                            -> E3: O + Gam^2 Q M0 - Gam Q G0
+// Prologue: (S0, C0, G0) fp32 from the summary slot to bf16 tiles (S0 = S0^T: the key moment
+// is symmetric), overlapping the Q/K/V loads.
+// Rounds: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T          -> E1: At, H, A, U, Gam P to bf16
+//         R2 W = Gam P Q^T + At A^T + H U^T; H K               -> E2: W (masked, Dg); Gam Z,
+//                                                                   Z = Gam P + H K
+//         R3 O = W V + (Gam Z) C0                              -> E3: O - Gam Q G0
 __global__ void __launch_bounds__(DNT, 1)
 k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, DParams p) {
@@ -440,19 +398,49 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     __syncthreads();
     if (tid == 0) {
         const int t0 = chunk * C;
-        const uint8_t* pre = p.pre + ((size_t)bh * p.NC + chunk) * DPRE;
-        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE + DPRE);
+        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE);
         ptx::tma_load_3d(sm + S3_Q, &tq, bar_load, 0, t0, bh);
         ptx::tma_load_3d(sm + S3_K, &tk, bar_load, 0, t0, bh);
         ptx::tma_load_3d(sm + S3_V, &tv, bar_load, 0, t0, bh);
-        ptx::bulk_load(sm + S3_SG, pre, 3 * QTILE, bar_load);          // S0^T, G0^T, M0^T
-        ptx::bulk_load(sm + S3_C0, pre + 3 * QTILE, QTILE, bar_load);  // C0
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
     for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
+    {
+        // carried-in state -> bf16 operand tiles (row r, 16-byte chunk j at j ^ (r & 7))
+        const float* slot = p.sums + ((size_t)bh * p.NC + chunk) * DSUM;
+        auto put8 = [&](uint32_t tile, int r, int j, const float (&x)[8]) {
+            *reinterpret_cast<uint4*>(sm + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
+                make_uint4(ptx::pack_bf16(x[0], x[1]), ptx::pack_bf16(x[2], x[3]), ptx::pack_bf16(x[4], x[5]),
+                           ptx::pack_bf16(x[6], x[7]));
+        };
+        float* gst = reinterpret_cast<float*>(sm + S3_AT);   // G0 [64][65] fp32
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int f = tid + DNT * i, rr = f >> 4, c4 = f & 15;
+            const float4 x = reinterpret_cast<const float4*>(slot + 3 * D * D)[f];
+            float* d = gst + rr * (D + 1) + 4 * c4;
+            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+        }
+        for (int f = tid; f < 2 * D * 8; f += DNT) {          // S0 rows (tile 0), C0 rows
+            const int m = f >> 9, r = (f >> 3) & 63, j = f & 7;
+            const float4* src = reinterpret_cast<const float4*>(slot + m * D * D + r * D + 8 * j);
+            const float4 a = src[0], b = src[1];
+            const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            put8(m ? S3_C0 : S3_SG, r, j, x);
+        }
+        __syncthreads();
+        for (int f = tid; f < D * 8; f += DNT) {              // G0^T: row n = column n of G0
+            const int n = f >> 3, j = f & 7;
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = gst[(8 * j + i) * (D + 1) + n];
+            put8(S3_SG + QTILE, n, j, x);
+        }
+    }
+    ptx::fence_proxy_async();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -465,10 +453,8 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
         if (ok) {
             ptx::tc_fence_after();
             constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 256, false, false);
-            constexpr uint32_t I_N64 = ptx::idesc_bf16(128, 64, false, false);
-            const uint64_t dQ = kdesc(sb + S3_Q, 0), dKSG = kdesc(sb + S3_K, 0), dM = kdesc(sb + S3_M0, 0);
+            const uint64_t dQ = kdesc(sb + S3_Q, 0), dKSG = kdesc(sb + S3_K, 0);
             for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dQ, s), k1s(dKSG, s), I_R1, s > 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_QM, k1s(dQ, s), k1s(dM, s), I_N64, s > 0);
         }
     }
     ok = __syncthreads_and(ok) != 0;
@@ -514,13 +500,13 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
             for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dP, s), k1s(dQ, s), I_W, s > 0);
             for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dAt, s), k2s(dA, s), I_W, 1);
             for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dH, s), k2s(dU, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_P, k2s(dH, s), mns(dKm, s), I_HK, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_HK, k2s(dH, s), mns(dKm, s), I_HK, s > 0);
         }
         ok = ms.commit_wait(tid == 0);          // R2 done
     }
     if (ok) {
-        // E2: W[tau][j] = g^(tau-j) x for j <= tau -> over H; Gam (H K) -> over Gam P
-        float v[32];
+        // E2: W[tau][j] = g^(tau-j) x for j <= tau -> over H; Gam (Gam P + H K) -> over Gam P
+        float v[32], w[32];
 #pragma unroll
         for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
             ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
@@ -531,10 +517,10 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
             }
             st_row32(sm + S3_H, row, c0, v);
         }
-        ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
+        ptx::tmem_ld32x2(tmem + lane_base + T3_P + half * 32, tmem + lane_base + T3_HK + half * 32, v, w);
         const float gam = gp[row + 1];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= gam;
+        for (int i = 0; i < 32; ++i) v[i] = gam * fmaf(gam, v[i], w[i]);
         st_row32(sm + S3_P, row, half * 32, v);
         sync_for_mma();
         if (tid == 0) {
@@ -547,14 +533,10 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
         ok = ms.commit_wait(tid == 0);          // R3 done
     }
     if (ok) {
-        // E3: O + Gam^2 (Q M0) - Gam (Q G0), staged as two [128][32] fp32 boxes over At
+        // E3: O - Gam (Q G0), staged as two [128][32] fp32 boxes over At
         float o[32], m[32];
-        ptx::tmem_ld32(tmem + lane_base + T3_O + half * 32, o);
-        ptx::tmem_ld32(tmem + lane_base + T3_QM + half * 32, m);
-        const float gam = gp[row + 1], gam2 = gp[2 * row + 2];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = fmaf(gam2, m[i], o[i]);
-        ptx::tmem_ld32(tmem + lane_base + T3_QG + half * 32, m);
+        ptx::tmem_ld32x2(tmem + lane_base + T3_O + half * 32, tmem + lane_base + T3_QG + half * 32, o, m);
+        const float gam = gp[row + 1];
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = fmaf(-gam, m[i], o[i]);
         float4* box = reinterpret_cast<float4*>(sm + S3_AT + half * (C * 128) + row * 128);
@@ -583,10 +565,10 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
 
 size_t decay_workspace_bytes(int BH, int T) {
     const size_t NC = (size_t)(T + C - 1) / C;
-    return (size_t)BH * NC * (DSUM * sizeof(float) + DPRE);
+    return (size_t)BH * NC * DSUM * sizeof(float);
 }
 
-int decay_kernel_launches() { return 6; }
+int decay_kernel_launches() { return 5; }
 
 cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
                           int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
@@ -599,14 +581,10 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
     prm.T = T; prm.BH = BH; prm.H = H; prm.NC = (T + C - 1) / C;
     prm.gamma = gamma;
     prm.sums = static_cast<float*>(ws);
-    prm.pre = reinterpret_cast<uint8_t*>(prm.sums + (size_t)BH * prm.NC * DSUM);
     prm.status = status;
     const int NC = prm.NC;
-    const size_t cross_smem = sizeof(float) * (2 * D * XLD + D * D);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_dec_summary, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_BYTES)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(k_dec_cross, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cross_smem)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(k_dec_output, cudaFuncAttributeMaxDynamicSharedMemorySize, S3_BYTES)) != cudaSuccess)
         return e;
@@ -616,11 +594,9 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     k_dec_prefix_sc<<<dim3((2 * D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_dec_cross<<<dim3(NC, BH), PNT, cross_smem, st>>>(prm);
+    k_dec_cross<<<dim3(NC, BH), PNT, 0, st>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_dec_prefix_g<<<dim3((D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_dec_tiles<<<dim3(NC, BH), PNT, 0, st>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_dec_output<<<dim3(NC, BH), DNT, S3_BYTES, st>>>(mq, mk, mv, mo, prm);
