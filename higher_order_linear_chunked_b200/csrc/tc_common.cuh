@@ -84,6 +84,16 @@ __device__ __forceinline__ void st_row32(uint8_t* tile, int row, int c0, const f
         *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = u;
     }
 }
+// 32 zero columns c0..c0+31 of row `row` (a block that the causal mask clears).
+__device__ __forceinline__ void st_row32_zero(uint8_t* tile, int row, int c0) {
+    uint8_t* atom = tile + (c0 >> 6) * TILE;
+    const int cin = c0 & 63;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const int chunk = (cin >> 3) + h;
+        *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
 // Transposed write of 32 values: v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
 __device__ __forceinline__ void st_col32(uint8_t* tile, int kcol, int c0, const float (&v)[32]) {
 #pragma unroll

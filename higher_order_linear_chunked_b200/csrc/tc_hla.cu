@@ -278,14 +278,19 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     auto epi1 = [&]() {
         float v0[32], v1[32];
         const int c0 = half * 64;
-        ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
+        if (c0 > row) {                      // rows 0..63, columns 64..127: cleared by the mask
+            st_row32_zero(sm + SM_A, row, c0);
+            st_row32_zero(sm + SM_A, row, c0 + 32);
+        } else {
+            ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (c0 + i > row) v0[i] = 0.f;
-            if (c0 + 32 + i > row) v1[i] = 0.f;
+            for (int i = 0; i < 32; ++i) {
+                if (c0 + i > row) v0[i] = 0.f;
+                if (c0 + 32 + i > row) v1[i] = 0.f;
+            }
+            st_row32(sm + SM_A, row, c0, v0);
+            st_row32(sm + SM_A, row, c0 + 32, v1);
         }
-        st_row32(sm + SM_A, row, c0, v0);
-        st_row32(sm + SM_A, row, c0 + 32, v1);
         if (MODE == OUTPUT) {
             ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
             st_row32(sm + SM_Z, row, half * 32, v0);
@@ -296,14 +301,19 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         float v0[32], v1[32];
         if (MODE == OUTPUT) {
             const int c0 = half * 64;
-            ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
+            if (c0 > row) {
+                st_row32_zero(sm + SM_A, row, c0);
+                st_row32_zero(sm + SM_A, row, c0 + 32);
+            } else {
+                ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (c0 + i > row) v0[i] = 0.f;
-                if (c0 + 32 + i > row) v1[i] = 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    if (c0 + i > row) v0[i] = 0.f;
+                    if (c0 + 32 + i > row) v1[i] = 0.f;
+                }
+                st_row32(sm + SM_A, row, c0, v0);
+                st_row32(sm + SM_A, row, c0 + 32, v1);
             }
-            st_row32(sm + SM_A, row, c0, v0);
-            st_row32(sm + SM_A, row, c0 + 32, v1);
         }
         if (quad < 2) {
             ptx::tmem_ld32x2(tmem + lane_base + TM_P + half * 32, tmem + lane_base + TM_S + half * 32, v0, v1);

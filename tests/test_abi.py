@@ -64,6 +64,32 @@ def test_workspace_sizes(lib):
     assert ws(9, hla.HLA_F32, 0, 1, 1, 10, 64, 64) == 0                    # bad op
 
 
+def test_tensor_core_routing_launches_and_workspace(lib):
+    """Host-side routing: which requests take the tcgen05 kernels, how many launches a
+    forward enqueues, and the workspace each path sizes (no GPU needed)."""
+    use = lambda op, dt, dec, T=4096, d=64: lib.hla_uses_tensor_cores(op, dt, dec, 4, 16, T, d, d)
+    launches = lambda op, dt, dec, T=4096, d=64: lib.hla_kernel_launches(op, dt, dec, 4, 16, T, d, d)
+    bf16, f32 = hla.HLA_BF16, hla.HLA_F32
+    # bf16, d = 64: second order (plain, normalised, decayed) and AHLA run on the tensor cores
+    for op, dec in ((hla.OP_HLA2, 0), (hla.OP_HLA2_NORM, 0), (hla.OP_HLA2, 1), (hla.OP_AHLA, 0)):
+        assert use(op, bf16, dec) == 1, (op, dec)
+    # the rest on CUDA cores: fp32 inputs, d = 32, third order, normalised with decay
+    assert use(hla.OP_HLA2, f32, 0) == 0
+    assert use(hla.OP_HLA2, bf16, 0, d=32) == 0
+    assert use(hla.OP_HLA3, bf16, 0) == 0
+    assert use(hla.OP_HLA2_NORM, bf16, 1) == 0
+    # launches per forward: summary walker, two prefix kernels, output walker; the decayed
+    # path has chunk summaries, three prefix kernels and the output kernel
+    assert launches(hla.OP_HLA2_NORM, bf16, 0) == 4
+    assert launches(hla.OP_AHLA, bf16, 0) == 4
+    assert launches(hla.OP_HLA2, bf16, 1) == 5
+    # decayed workspace: 256 B status block + one 4 x 64 x 64 fp32 slot per 128-token chunk
+    T = 16384
+    assert lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, T, 64, 64) == 256 + 32 * (T // 128) * 4 * 64 * 64 * 4
+    assert lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, T + 1, 64, 64) == \
+        256 + 32 * (T // 128 + 1) * 4 * 64 * 64 * 4
+
+
 def _call(lib, name, q=16, k=16, v=16, o=16, B=1, H=1, T=8, d=32, dv=32, dtype=0, gamma=0, ws=16,
           wsb=1 << 30, eps=None):
     vp = ctypes.c_void_p
