@@ -55,7 +55,8 @@ constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024; // + alignment slack
 constexpr uint32_t TM_A = 0;      // A, then W            (128 cols)
 constexpr uint32_t TM_P = 128;    // P, then Z            (64)
 constexpr uint32_t TM_O0 = 192;   // O | q.r0, even chunks (80)
-constexpr uint32_t TM_CR = 272;   // lanes 0-63 [C|m], lanes 64-127 [R|r]  (80)
+constexpr uint32_t TM_CR = 272;   // summary: lanes 0-63 [C|m], lanes 64-127 [R|r]  (80)
+                                  // output: lanes 0-63 R^T, lane 64 r^T, rest 0   (64)
 constexpr uint32_t TM_S = 352;    // lanes 0-63 S         (64)
 constexpr uint32_t TM_O1 = 416;   // O | q.r0, odd chunks  (80)
 constexpr uint32_t TM_COLS = 512;
@@ -72,8 +73,9 @@ enum Mode { SUMMARY = 0, OUTPUT = 1 };
 //   R1(n): A = Q K^T, P = Q S0                      -> E1(n): A, P to bf16 tiles
 //   R2(n): W = P Q^T + A A^T, Z = P + A K,
 //          S += K^T K, O[n&1] = Q [R0|r0]^T         -> E2(n): W, Z, S0 to bf16 tiles
-//   R3(n): O[n&1] += W V,
-//          [C|m ; R|r] += [Q^T;Z^T][V|1]            -> E3(n): [R0|r0]^T; O[n&1] to HBM
+//   R3(n): [O|den][n&1] += W [V|1],
+//          summary: [C|m ; R|r] += [Q^T;Z^T][V|1]
+//          output:  [R^T ; r^T] += [V^T ; 1^T] Z    -> E3(n): [R0|r0]^T; O[n&1] to HBM
 // R3(n) and R1(n+1) are issued together and their epilogues run together.  The O
 // accumulator is double buffered in TMEM, so the store of O(n) to HBM runs while
 // the tensor core works on R2(n+1).
@@ -129,11 +131,13 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tmem_relinquish();
     }
     if (tid < C) {
-        // ones tile, MN-major [token][64]: the N = 80 MMAs read only columns 0..15 of it,
-        // i.e. logical 16-byte chunks 0 and 1 of every token row: chunk 0 = (1, 0, ..., 0).
+        // ones tile, [token][64]: column 0 = 1, the rest 0.  As the second N block of an
+        // MN-major B operand it appends a ones column ([V | 1]); as the second M block of a
+        // stacked MN-major A operand it appends a row of column sums ([V^T ; 1^T]).
         uint8_t* r = sm + SM_ONES + tid * 128;
-        *reinterpret_cast<uint4*>(r + (((0 ^ tid) & 7) << 4)) = make_uint4(0x3F80u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(r + (((1 ^ tid) & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(r + (((j ^ tid) & 7) << 4)) = make_uint4(j == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
     }
     // Carried-in state (OUTPUT): the prefix (S, R, r) is staged in shared memory with
     // coalesced loads (rows swizzled by 16-byte chunk), then every thread takes its row.
@@ -178,25 +182,32 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
                 if (MODE == OUTPUT) ptx::tmem_st16(tmem + lane_base + TM_S + c0, v);
                 st_row16(sm + SM_S0, TILE, row, c0, v);
             }
-        } else {                             // [R | r] row `row - 64`, columns 0..47 / 48..79
-            const int r = row - 64;
-            const int cb = half ? 48 : 0, ce = half ? 80 : 48;
-            for (int c0 = cb; c0 < ce; c0 += 16) {
-                if (c0 < D) {
+        } else if (MODE == SUMMARY) {        // [R0|r0]^T starts at zero: rows n = row - 64 < 80
+            const int n = row - 64;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int ch = (c0 / 4 + j) ^ (r & 7);
-                        const float4 x = MODE == OUTPUT ? reinterpret_cast<const float4*>(stage + D * D)[r * 16 + ch]
-                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-                        v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            for (int c0 = half * 32; c0 < half * 32 + 32; c0 += 16) {
+                st_row16(sm + SM_R0, TILE, n, c0, v);
+                if (n < 16) st_row16(sm + SM_R0, TILE, 64 + n, c0, v);
+            }
+        }
+        if (MODE == OUTPUT && quad < 3) {
+            // [R^T ; r^T] rows: row n < 64 is column n of R; row 64 is r; rows 65.. are 0.
+            // TMEM lanes 0..95 of TM_CR and tile rows 0..79 (rows n < 64 by quads 0-1,
+            // rows 64..79 by lanes 0..15 of quad 2).
+            for (int c0 = half * 32; c0 < half * 32 + 32; c0 += 16) {
+                if (quad < 2) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int k = c0 + i;                                 // R[k][row]
+                        v[i] = stage[D * D + k * D + ((((row >> 2) ^ (k & 7)) << 2) | (row & 3))];
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-                    if (MODE == OUTPUT) v[0] = stage_r[r];
+                    for (int i = 0; i < 16; ++i) v[i] = (lane == 0) ? stage_r[c0 + i] : 0.f;
                 }
-                if (MODE == OUTPUT) ptx::tmem_st16(tmem + lane_base + TM_CR + c0, v);
-                st_col16(sm + SM_R0, r, c0, v);
+                ptx::tmem_st16(tmem + lane_base + TM_CR + c0, v);
+                if (quad < 2 || lane < 16) st_row16(sm + SM_R0, TILE, quad < 2 ? row : 64 + lane, c0, v);
             }
         }
         if (MODE == OUTPUT) ptx::tmem_st_wait();
@@ -223,6 +234,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     auto bufV = [&](int n) { return sbase + ((n & 1) ? SM_V1 : SM_V0); };
     const uint64_t dS0 = kdesc(sbase + SM_S0, 0), dR0 = kdesc(sbase + SM_R0, 0);
     const uint64_t dZk = kdesc(sbase + SM_Z, 0), dA2 = kdesc2(sbase + SM_A, 0);
+    const uint64_t dZm = mdesc(sbase + SM_Z, TILE, 0);
     auto tm_o = [&](int n) { return tmem + ((n & 1) ? TM_O1 : TM_O0); };
 
     auto issue_r1 = [&](int n) {             // A = Q K^T, P = Q S0
@@ -247,10 +259,14 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         const uint32_t sQ = bufQ(n), sV = bufV(n);
         const uint64_t dQZ = mdesc(sQ, sbase + SM_Z - sQ, 0);
         const uint64_t dV1 = mdesc(sV, sbase + SM_ONES - sV, 0);
-        if (MODE == OUTPUT)
+        if (MODE == OUTPUT) {
+            const uint64_t dV1t = mdesc(sV, sbase + SM_ONES - sV, 0);     // stacked [V^T ; 1^T]
             for (int s = 0; s < 8; ++s) ptx::umma_bf16(tm_o(n), k2(dA2, s), mn(dV1, s), I_N80_KM, 1);
-        for (int s = 0; s < 8; ++s)
-            ptx::umma_bf16(tmem + TM_CR, mn(dQZ, s), mn(dV1, s), I_N80_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_CR, mn(dV1t, s), mn(dZm, s), I_N64_MM, 1);
+        } else {
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + TM_CR, mn(dQZ, s), mn(dV1, s), I_N80_MM, (n > 0 || s > 0) ? 1u : 0u);
+        }
     };
 
     uint32_t mma_phase = 0;
@@ -324,21 +340,12 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             st_row32(sm + SM_Z, row, half * 32, v0);
         }
     };
-    // E3, state part: [R|r] -> SM_R0 (transposed), rows 64..127 of TM_CR
+    // E3, state part (output walk): [R^T ; r^T] rows 0..64 of TM_CR -> [R0|r0]^T tile rows
     auto epi3_state = [&]() {
-        if (quad < 2) return;
+        if (quad == 3) return;
         float v[32];
-        float d[16];
-        const int r = row - 64;
-        if (half == 0) {
-            ptx::tmem_ld32(tmem + lane_base + TM_CR, v);
-            st_col32(sm + SM_R0, r, 0, v);
-            ptx::tmem_ld16(tmem + lane_base + TM_CR + 32, d);
-            st_col16(sm + SM_R0, r, 32, d);
-        } else {
-            ptx::tmem_ld32(tmem + lane_base + TM_CR + 48, v);
-            st_col32(sm + SM_R0, r, 48, v);
-        }
+        ptx::tmem_ld32(tmem + lane_base + TM_CR + half * 32, v);   // warp-collective
+        if (quad < 2 || lane < 16) st_row32(sm + SM_R0, quad < 2 ? row : 64 + lane, half * 32, v);
     };
     // E3, output part: O rows of chunk n (normalised by column 64, q.r0 + rowsum W) staged
     // as two [128 rows][32 cols] fp32 boxes in the 128B-swizzled TMA layout
