@@ -28,9 +28,10 @@
 // rounding at strong decay (H A*^T + A A^T) or at weak decay (At A*^T - A U^T).
 //
 // Kernels (one CTA per chunk x head, every chunk independent):
-//   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G), fp32
+//   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G^T), fp32
 //   k_dec_prefix_sc, k_dec_cross, k_dec_prefix_g (CUDA cores)
-//                                               in place: S0, C0; Y = G + rho Khat C0; G0
+//                                               in place: S0, C0; Y^T = G^T + rho C0^T Khat;
+//                                               G0^T (Khat is symmetric)
 //   k_dec_output (tcgen05)                      turns (S0, C0, G0) into bf16 operand tiles
 //                                               while its Q/K/V loads are in flight; O,
 //                                               written by TMA bulk tensor stores
@@ -48,15 +49,24 @@ namespace tc {
 namespace {
 
 constexpr int DNT = 256;                  // 8 warps, two per TMEM lane quadrant
-constexpr int DSUM = 4 * D * D;           // summary slot: S, C, Khat, G (then Y, then G0)
+constexpr int DSUM = 4 * D * D;           // chunk state: S, C, Khat, G^T (then Y^T, then G0^T)
 constexpr uint32_t QTILE = D * D * 2;     // one 64 x 64 bf16 tile = 8 KB
 
 struct DParams {
     int T, BH, H, NC;
     const float* gamma;
-    float* sums;      // [BH][NC][DSUM] fp32
+    float* sums;      // per head NC x DSUM fp32, in the blocked layout of dsum()
     int* status;
 };
+
+// Chunk states of a head are stored in blocks of 32 consecutive elements of one matrix,
+// chunk-major inside a block: element e (0 .. DSUM) of chunk l sits at
+//     sums + bh NC DSUM + (e / 32) NC 32 + l 32 + e % 32.
+// A warp that follows one block across the chunks reads one contiguous run, and one chunk's
+// state is 512 whole 128-byte lines.
+__device__ __forceinline__ float* dsum(const DParams& p, int bh, int l, int e) {
+    return p.sums + (size_t)bh * p.NC * DSUM + (size_t)(e >> 5) * p.NC * 32 + l * 32 + (e & 31);
+}
 
 // g^n for n >= 0 (binary powering).
 __device__ __forceinline__ float gpow_n(float g, int n) {
@@ -116,7 +126,7 @@ constexpr uint32_t S1_BYTES = S1_BAR + 64;  // no slack: checked at run time
 // Rounds: R1 A* = Q K^T                                -> E1: U to bf16; Lam K, Lam V
 //         R2 Y = U^T Lam V; [K^T ; Q^T][Lam K | Lam V | K]  (S, -, Khat ; -, C, -)
 //                                                      -> E2: Y to bf16; S, C, Khat staged
-//         R3 [K^T ; Y^T] Y   (lanes 0-63: G)            -> E3: G staged; summary stored
+//         R3 [Y^T ; V^T] K   (lanes 0-63: G^T)          -> E3: G^T staged; summary stored
 __global__ void __launch_bounds__(DNT, 2)
 k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
               const __grid_constant__ CUtensorMap tv, DParams p) {
@@ -233,8 +243,8 @@ k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         sync_for_mma();
         if (tid == 0) {
             constexpr uint32_t I_G = ptx::idesc_bf16(128, 64, true, true);
-            const uint64_t dKY = mdesc(sb + S1_K, S1_Q - S1_K, 0), dY = mdesc(sb + S1_Q, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dKY, s), mns(dY, s), I_G, s > 0);
+            const uint64_t dYV = mdesc(sb + S1_Q, S1_V - S1_Q, 0), dK = mdesc(sb + S1_K, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dYV, s), mns(dK, s), I_G, s > 0);
         }
         ok = ms.commit_wait(tid == 0);          // R3 done
     }
@@ -245,11 +255,10 @@ k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
             put_row(3, row, half * 32, v);
         }
         __syncthreads();
-        float4* out4 = reinterpret_cast<float4*>(p.sums + ((size_t)bh * p.NC + chunk) * DSUM);
         const float4* st4 = reinterpret_cast<const float4*>(stg);
         for (int f = tid; f < DSUM / 4; f += DNT) {
             const int r = (f >> 4) & (D - 1);
-            out4[f] = st4[(f & ~15) | ((f & 15) ^ (r & 7))];
+            *reinterpret_cast<float4*>(dsum(p, bh, chunk, 4 * f)) = st4[(f & ~15) | ((f & 15) ^ (r & 7))];
         }
     } else if (tid == 0) {
         set_status(p.status, DEV_TIMEOUT);
@@ -271,77 +280,78 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_sc(DParams p) {
     const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
     if (e >= 2 * D * D) return;
     const float rho = gpow_n(p.gamma[bh % p.H], C);
-    float* x = p.sums + (size_t)bh * p.NC * DSUM + e;
+    float* x = dsum(p, bh, 0, e);             // chunk l at x + 32 l
     float run = 0.f;
     for (int l0 = 0; l0 < p.NC; l0 += 16) {
         float y[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
+            if (l0 + i < p.NC) y[i] = x[(l0 + i) * 32];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) {
-                x[(size_t)(l0 + i) * DSUM] = run;
+                x[(l0 + i) * 32] = run;
                 run = fmaf(rho, run, y[i]);
             }
     }
 }
 
-// Per chunk: Y = G + rho Khat C0, in place of G (matrix 3).
-constexpr int XLD = D + 4;   // padded row stride of the left operand
+// Per chunk: Y^T = G^T + rho C0^T Khat, in place of G^T (matrix 3).  (Y = G + rho Khat C0 and
+// Khat is symmetric.)
 __global__ void __launch_bounds__(PNT) k_dec_cross(DParams p) {
-    __shared__ __align__(16) float Kh[D * XLD];
+    __shared__ __align__(16) float Kh[D * D];
     __shared__ __align__(16) float C0[D * D];
     const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    float* slot = p.sums + ((size_t)bh * p.NC + l) * DSUM;
     const float rho = gpow_n(p.gamma[bh % p.H], C);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int f = tid + PNT * i, r = f >> 4, c4 = f & 15;
-        const float4 c = reinterpret_cast<const float4*>(slot + D * D)[f];
-        const float4 k = reinterpret_cast<const float4*>(slot + 2 * D * D)[f];
-        *reinterpret_cast<float4*>(Kh + r * XLD + 4 * c4) = make_float4(rho * k.x, rho * k.y, rho * k.z, rho * k.w);
+        const int f = tid + PNT * i;
+        const float4 c = *reinterpret_cast<const float4*>(dsum(p, bh, l, D * D + 4 * f));
+        const float4 k = *reinterpret_cast<const float4*>(dsum(p, bh, l, 2 * D * D + 4 * f));
         reinterpret_cast<float4*>(C0)[f] = c;
+        reinterpret_cast<float4*>(Kh)[f] = make_float4(rho * k.x, rho * k.y, rho * k.z, rho * k.w);
     }
     __syncthreads();
-    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);
+    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);   // rows r.. of Y^T (columns of C0), columns c..
     float y[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
-        const float4 gx = *reinterpret_cast<const float4*>(slot + 3 * D * D + (r + a) * D + c);
+        const float4 gx = *reinterpret_cast<const float4*>(dsum(p, bh, l, 3 * D * D + (r + a) * D + c));
         y[a][0] = gx.x; y[a][1] = gx.y; y[a][2] = gx.z; y[a][3] = gx.w;
     }
 #pragma unroll 8
     for (int k = 0; k < D; ++k) {
-        const float4 cv = *reinterpret_cast<const float4*>(C0 + k * D + c);
+        const float4 cv = *reinterpret_cast<const float4*>(C0 + k * D + r);
+        const float4 kv = *reinterpret_cast<const float4*>(Kh + k * D + c);
+        const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-            const float kv = Kh[(r + a) * XLD + k];
-            y[a][0] = fmaf(kv, cv.x, y[a][0]); y[a][1] = fmaf(kv, cv.y, y[a][1]);
-            y[a][2] = fmaf(kv, cv.z, y[a][2]); y[a][3] = fmaf(kv, cv.w, y[a][3]);
+            y[a][0] = fmaf(cc[a], kv.x, y[a][0]); y[a][1] = fmaf(cc[a], kv.y, y[a][1]);
+            y[a][2] = fmaf(cc[a], kv.z, y[a][2]); y[a][3] = fmaf(cc[a], kv.w, y[a][3]);
         }
     }
 #pragma unroll
     for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4*>(slot + 3 * D * D + (r + a) * D + c) = make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
+        *reinterpret_cast<float4*>(dsum(p, bh, l, 3 * D * D + (r + a) * D + c)) =
+            make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
 }
 
-// Exclusive decayed prefix of Y (matrix 3) into G0, in place.
+// Exclusive decayed prefix of Y^T (matrix 3) into G0^T, in place.
 __global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
     const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
     if (e >= D * D) return;
     const float rho = gpow_n(p.gamma[bh % p.H], C);
-    float* x = p.sums + (size_t)bh * p.NC * DSUM + 3 * D * D + e;
+    float* x = dsum(p, bh, 0, 3 * D * D + e);
     float run = 0.f;
     for (int l0 = 0; l0 < p.NC; l0 += 16) {
         float y[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) y[i] = x[(size_t)(l0 + i) * DSUM];
+            if (l0 + i < p.NC) y[i] = x[(l0 + i) * 32];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             if (l0 + i < p.NC) {
-                x[(size_t)(l0 + i) * DSUM] = run;
+                x[(l0 + i) * 32] = run;
                 run = fmaf(rho, run, y[i]);
             }
     }
@@ -354,7 +364,7 @@ constexpr uint32_t S3_K = S3_Q + TILE;       // K                    } B rows of
 constexpr uint32_t S3_SG = S3_K + TILE;      // S0 (rows), G0^T tiles } [K ; S0^T ; G0^T]
 constexpr uint32_t S3_C0 = S3_SG + 2 * QTILE;   // C0 (rows: MN-major B operand)
 constexpr uint32_t S3_V = S3_C0 + QTILE;     // V
-constexpr uint32_t S3_AT = S3_V + TILE;      // G0 staging (fp32), At, later the O staging boxes
+constexpr uint32_t S3_AT = S3_V + TILE;      // At, later the O staging boxes
 constexpr uint32_t S3_H = S3_AT + 2 * TILE;  // H, later W
 constexpr uint32_t S3_A = S3_H + 2 * TILE;   // A
 constexpr uint32_t S3_U = S3_A + 2 * TILE;   // U
@@ -370,7 +380,7 @@ constexpr uint32_t T3_QG = 192;   // Q G0         (64)
 constexpr uint32_t T3_HK = 256;   // H K          (64)
 constexpr uint32_t T3_O = 320;    // O            (64)
 
-// Prologue: (S0, C0, G0) fp32 from the summary slot to bf16 tiles (S0 = S0^T: the key moment
+// Prologue: (S0, C0, G0^T) fp32 from the chunk state to bf16 tiles (S0 = S0^T: the key moment
 // is symmetric), overlapping the Q/K/V loads.
 // Rounds: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T          -> E1: At, H, A, U, Gam P to bf16
 //         R2 W = Gam P Q^T + At A^T + H U^T; H K               -> E2: W (masked, Dg); Gam Z,
@@ -409,35 +419,25 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     }
     for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
     {
-        // carried-in state -> bf16 operand tiles (row r, 16-byte chunk j at j ^ (r & 7))
-        const float* slot = p.sums + ((size_t)bh * p.NC + chunk) * DSUM;
-        auto put8 = [&](uint32_t tile, int r, int j, const float (&x)[8]) {
+        // carried-in S0, C0 and G0^T -> bf16 operand tiles, row for row (row r, 16-byte chunk j
+        // at j ^ (r & 7)); S0 is symmetric, so its rows serve as the K-major S0^T
+        constexpr int NI = 3 * D * 8 / DNT;                // 16-byte chunks per thread
+        float4 x[NI][2];
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
+            const int e = (t == 2 ? 3 : t) * D * D + r * D + 8 * j;
+            const float4* src = reinterpret_cast<const float4*>(dsum(p, bh, chunk, e));
+            x[i][0] = src[0];
+            x[i][1] = src[1];
+        }
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+            const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
+            const uint32_t tile = t == 0 ? S3_SG : t == 1 ? S3_C0 : S3_SG + QTILE;
             *reinterpret_cast<uint4*>(sm + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
-                make_uint4(ptx::pack_bf16(x[0], x[1]), ptx::pack_bf16(x[2], x[3]), ptx::pack_bf16(x[4], x[5]),
-                           ptx::pack_bf16(x[6], x[7]));
-        };
-        float* gst = reinterpret_cast<float*>(sm + S3_AT);   // G0 [64][65] fp32
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int f = tid + DNT * i, rr = f >> 4, c4 = f & 15;
-            const float4 x = reinterpret_cast<const float4*>(slot + 3 * D * D)[f];
-            float* d = gst + rr * (D + 1) + 4 * c4;
-            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
-        }
-        for (int f = tid; f < 2 * D * 8; f += DNT) {          // S0 rows (tile 0), C0 rows
-            const int m = f >> 9, r = (f >> 3) & 63, j = f & 7;
-            const float4* src = reinterpret_cast<const float4*>(slot + m * D * D + r * D + 8 * j);
-            const float4 a = src[0], b = src[1];
-            const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            put8(m ? S3_C0 : S3_SG, r, j, x);
-        }
-        __syncthreads();
-        for (int f = tid; f < D * 8; f += DNT) {              // G0^T: row n = column n of G0
-            const int n = f >> 3, j = f & 7;
-            float x[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) x[i] = gst[(8 * j + i) * (D + 1) + n];
-            put8(S3_SG + QTILE, n, j, x);
+                make_uint4(ptx::pack_bf16(x[i][0].x, x[i][0].y), ptx::pack_bf16(x[i][0].z, x[i][0].w),
+                           ptx::pack_bf16(x[i][1].x, x[i][1].y), ptx::pack_bf16(x[i][1].z, x[i][1].w));
         }
     }
     ptx::fence_proxy_async();
