@@ -201,6 +201,10 @@ k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CU
         float v[32];
 #pragma unroll
         for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 + 31 < quad * 32) {                                 // wholly below the diagonal
+                st_row32_zero(sm + S1_U, row, c0);
+                continue;
+            }
             ptx::tmem_ld32(tmem + lane_base + c0, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -461,10 +465,19 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     if (ok) ok = ms.commit_wait(tid == 0);      // R1 done
     if (ok) {
         // E1: from A* row `row` (columns half*64 .. +63): At, H, A, U; Gam P (columns half*32 .. +31)
+        // 32 x 32 blocks wholly above the diagonal are zero in At, H and A, and wholly below
+        // it zero in U: those are written without conversions (the test is warp-uniform).
         float v[32], w[32];
 #pragma unroll
         for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
             ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
+            if (c0 > quad * 32 + 31) {                                 // above the diagonal
+                st_row32_zero(sm + S3_AT, row, c0);
+                st_row32_zero(sm + S3_H, row, c0);
+                st_row32_zero(sm + S3_A, row, c0);
+                st_row32(sm + S3_U, row, c0, v);
+                continue;
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int d = row - (c0 + i);                          // tau - i
@@ -477,6 +490,11 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
                 w[i] = d > 0 ? (gp[d] - 1.f) * v[i] : 0.f;            // H
             }
             st_row32(sm + S3_H, row, c0, w);
+            if (c0 + 31 < quad * 32) {                                 // below the diagonal
+                st_row32(sm + S3_A, row, c0, v);
+                st_row32_zero(sm + S3_U, row, c0);
+                continue;
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i) w[i] = (c0 + i <= row) ? v[i] : 0.f;   // A
             st_row32(sm + S3_A, row, c0, w);
@@ -509,6 +527,10 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
         float v[32], w[32];
 #pragma unroll
         for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 > quad * 32 + 31) {                                 // above the diagonal
+                st_row32_zero(sm + S3_H, row, c0);
+                continue;
+            }
             ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

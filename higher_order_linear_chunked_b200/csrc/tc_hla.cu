@@ -290,45 +290,42 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tc_fence_after();
     };
 
-    // E1: A (masked) -> SM_A (this thread: columns half*64 .. +63); P -> SM_Z (OUTPUT only)
+    // E1: A (masked) -> SM_A (this thread: columns half*64 .. +63; blocks wholly above the
+    // diagonal are written as zeros); P -> SM_Z (OUTPUT only)
     auto epi1 = [&]() {
-        float v0[32], v1[32];
-        const int c0 = half * 64;
-        if (c0 > row) {                      // rows 0..63, columns 64..127: cleared by the mask
-            st_row32_zero(sm + SM_A, row, c0);
-            st_row32_zero(sm + SM_A, row, c0 + 32);
-        } else {
-            ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
+        float v0[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (c0 + i > row) v0[i] = 0.f;
-                if (c0 + 32 + i > row) v1[i] = 0.f;
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 > quad * 32 + 31) {       // a 32 x 32 block wholly above the diagonal
+                st_row32_zero(sm + SM_A, row, c0);
+                continue;
             }
+            ptx::tmem_ld32(tmem + lane_base + TM_A + c0, v0);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i > row) v0[i] = 0.f;
             st_row32(sm + SM_A, row, c0, v0);
-            st_row32(sm + SM_A, row, c0 + 32, v1);
         }
         if (MODE == OUTPUT) {
             ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
             st_row32(sm + SM_Z, row, half * 32, v0);
         }
     };
-    // E2: W (masked, bf16-rounded, partial row sums) -> SM_A; Z -> SM_Z; S -> SM_S0 (transposed)
+    // E2: W (masked) -> SM_A; Z -> SM_Z; S -> SM_S0 (by rows: S is symmetric)
     auto epi2 = [&]() {
         float v0[32], v1[32];
         if (MODE == OUTPUT) {
-            const int c0 = half * 64;
-            if (c0 > row) {
-                st_row32_zero(sm + SM_A, row, c0);
-                st_row32_zero(sm + SM_A, row, c0 + 32);
-            } else {
-                ptx::tmem_ld32x2(tmem + lane_base + TM_A + c0, tmem + lane_base + TM_A + c0 + 32, v0, v1);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    if (c0 + i > row) v0[i] = 0.f;
-                    if (c0 + 32 + i > row) v1[i] = 0.f;
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) {
+                    st_row32_zero(sm + SM_A, row, c0);
+                    continue;
                 }
+                ptx::tmem_ld32(tmem + lane_base + TM_A + c0, v0);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i > row) v0[i] = 0.f;
                 st_row32(sm + SM_A, row, c0, v0);
-                st_row32(sm + SM_A, row, c0 + 32, v1);
             }
         }
         if (quad < 2) {
