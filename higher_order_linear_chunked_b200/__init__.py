@@ -36,7 +36,7 @@ STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_
 
 # Every symbol include/hla.h declares.
 EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
-           "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma",
+           "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
            "hla2_forward_normalized_noalloc")
 
 
@@ -84,6 +84,8 @@ def load_library(path: Optional[str] = None):
     lib.hla2_forward_normalized_noalloc.restype = i
     lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
     lib.hla_selftest_umma.restype = i
+    lib.hla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]
+    lib.hla_selftest_wait_timeout.restype = i
     if path is None:
         _lib = lib
     return lib

@@ -176,4 +176,16 @@ hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, fl
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 
+hla_status_t hla_selftest_wait_timeout(void* workspace, size_t workspace_bytes, unsigned timeout_us, void* stream) {
+    if (!workspace) return HLA_ERR_NULL;
+    if (!aligned16(workspace)) return HLA_ERR_ALIGN;
+    if (workspace_bytes < hla::kStatusBytes) return HLA_ERR_WORKSPACE;
+    if (timeout_us < 1 || timeout_us > 1000000) return HLA_ERR_SHAPE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int* status = static_cast<int*>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
+    const cudaError_t e = hla::tc::selftest_wait_timeout(status, timeout_us, st);
+    return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
+}
+
 }  // extern "C"

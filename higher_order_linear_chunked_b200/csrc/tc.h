@@ -19,6 +19,8 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
                     float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
+// a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)
+cudaError_t selftest_wait_timeout(int* status, unsigned timeout_us, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace hla

@@ -88,6 +88,38 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     if (warp == 0) ptx::tmem_dealloc(tbase, 256);
 }
 
+// A bounded wait that runs out on purpose: an mbarrier nothing arrives on, waited on with the
+// same helper the walkers use.  On the timeout the kernel records DEV_TIMEOUT in the status
+// word and frees its TMEM, exactly as the walkers' error path does, then returns normally.
+__global__ void __launch_bounds__(64) k_wait_timeout(int* status, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        ptx::tmem_alloc(&tmem_base, 32);
+        ptx::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    bool ok = true;
+    if (threadIdx.x == 0) ok = ptx::mbar_wait(&bar, 0, timeout_ns);
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok && threadIdx.x == 0) set_status(status, DEV_TIMEOUT);
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) ptx::tmem_dealloc(tmem_base, 32);
+}
+
+cudaError_t selftest_wait_timeout(int* status, unsigned timeout_us, cudaStream_t st) {
+    k_wait_timeout<<<1, 64, 0, st>>>(status, static_cast<unsigned long long>(timeout_us) * 1000ull);
+    return cudaGetLastError();
+}
+
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st) {
     const int smem = 128 * K * 2 + N * K * 2 + 1024;   // A sized for M = 128 in every case
     cudaError_t e = cudaFuncSetAttribute(k_selftest, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

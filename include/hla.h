@@ -207,6 +207,21 @@ hla_status_t hla2_forward_normalized_noalloc(const void* q, const void* k, const
 hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, float* d,
                                int N, int K, void* stream);
 
+/*
+ * Failure-path self-check (diagnostic; no counterpart on the pages).  Launches one small
+ * kernel whose bounded mbarrier wait runs out on purpose (nothing ever arrives): after
+ * `timeout_us` microseconds of %globaltimer it records HLA_ERR_TIMEOUT in the status word
+ * at the start of `workspace`, frees the tensor memory it allocated and returns, as the
+ * forward kernels do when one of their waits runs out.  No fault, trap or hang: the context
+ * stays usable.  Read the outcome with hla_read_device_status.
+ *   workspace: device memory of at least 256 bytes (16-byte aligned); its status word is
+ *              cleared by this call.
+ *   timeout_us: 1 .. 1000000 (else HLA_ERR_SHAPE).
+ * Enqueued on `stream`; returns HLA_OK once launched.
+ */
+hla_status_t hla_selftest_wait_timeout(void* workspace, size_t workspace_bytes, unsigned timeout_us,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -140,6 +140,12 @@ def test_selftest_argument_errors(lib):
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 96, 64, vp(0)) == 2
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 320, 64, vp(0)) == 2
     assert lib.hla_read_device_status(vp(0), vp(0), None) == 1
+    wt = lib.hla_selftest_wait_timeout
+    assert wt(vp(0), 256, 1000, vp(0)) == 1                     # NULL workspace
+    assert wt(vp(8), 256, 1000, vp(0)) == 3                     # not 16-byte aligned
+    assert wt(vp(16), 64, 1000, vp(0)) == 6                     # smaller than the status block
+    assert wt(vp(16), 256, 0, vp(0)) == 2                       # timeout out of range
+    assert wt(vp(16), 256, 2000000, vp(0)) == 2
 
 
 def test_product_path_never_touches_the_oracle():
