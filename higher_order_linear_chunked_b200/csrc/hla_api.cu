@@ -169,7 +169,8 @@ hla_status_t hla_read_device_status(const void* workspace, void* stream, int* de
 hla_status_t hla_selftest_umma(int layout_case, const void* a, const void* b, float* d, int N, int K,
                                void* stream) {
     if (!a || !b || !d) return HLA_ERR_NULL;
-    if (layout_case < 0 || layout_case > 15 || (layout_case & 8 && !(layout_case & 4))) return HLA_ERR_UNSUPPORTED;
+    if (layout_case < 0 || layout_case > 31 || (layout_case & 8 && !(layout_case & 4))) return HLA_ERR_UNSUPPORTED;
+    if ((layout_case & 16) && (layout_case & 14)) return HLA_ERR_UNSUPPORTED;   // A in TMEM: M = 128, K-major
     if ((N != 64 && N != 128 && N != 192 && N != 256) || (K != 64 && K != 128)) return HLA_ERR_SHAPE;
     if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return HLA_ERR_ALIGN;
     cudaError_t e = hla::tc::selftest(layout_case, a, b, d, N, K, static_cast<cudaStream_t>(stream));

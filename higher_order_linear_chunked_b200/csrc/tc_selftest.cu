@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int M = (cs & 4) ? 64 : 128;          // bit 2: M = 64 (half-lane-quadrant accumulator)
     const int loff = (cs & 8) ? 16 : 0;         // bit 3: accumulator at TMEM lane offset 16
+    const bool a_tm = (cs & 16) != 0;           // bit 4: A read from tensor memory (M = 128, K-major)
     const bool a_mn = (cs & 2) != 0, b_mn = (cs & 1) != 0;
     uint8_t* As = smem;
     uint8_t* Bs = smem + M * K * 2;
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     }
     ptx::fence_proxy_async();
     if (warp == 0) {
-        ptx::tmem_alloc(&tmem_base, 256);
+        ptx::tmem_alloc(&tmem_base, 512);
         ptx::tmem_relinquish();
     }
     if (tid == 0) {
@@ -60,13 +61,36 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tbase = tmem_base;
+    constexpr uint32_t kAcol = 256;             // A's columns when it is read from tensor memory
+    if (a_tm) {
+        // row m = lane m: K bf16 values packed two per column from column kAcol on
+        const int m = warp * 32 + lane;
+        for (int c0 = 0; c0 < K / 2; c0 += 16) {
+            uint32_t r[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int kk = 2 * (c0 + i);
+                const float lo = __bfloat162float(a[m * K + kk]), hi = __bfloat162float(a[m * K + kk + 1]);
+                r[i] = ptx::pack_bf16(lo, hi);
+            }
+            ptx::tmem_st16u(tbase + (static_cast<uint32_t>(warp * 32) << 16) + kAcol + c0, r);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+    }
     if (tid == 0) {
         const uint32_t idesc = ptx::idesc_bf16(M, N, a_mn, b_mn);
         const uint32_t abase = ptx::smem_u32(As), bbase = ptx::smem_u32(Bs);
         const uint32_t dt = tbase + (static_cast<uint32_t>(loff) << 16);
-        for (int s = 0; s < K / 16; ++s)
-            ptx::umma_bf16(dt, operand_desc(a_mn, abase, M, K, s), operand_desc(b_mn, bbase, N, K, s), idesc,
-                           s > 0);
+        for (int s = 0; s < K / 16; ++s) {
+            if (a_tm)
+                ptx::umma_bf16_ts(dt, tbase + kAcol + 8 * s, operand_desc(b_mn, bbase, N, K, s), idesc, s > 0);
+            else
+                ptx::umma_bf16(dt, operand_desc(a_mn, abase, M, K, s), operand_desc(b_mn, bbase, N, K, s), idesc,
+                               s > 0);
+        }
         ptx::umma_commit(&bar);
     }
     bool ok = ptx::mbar_wait(&bar, 0);
@@ -85,7 +109,7 @@ __global__ void __launch_bounds__(128) k_selftest(int cs, const bf16* __restrict
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0) ptx::tmem_dealloc(tbase, 256);
+    if (warp == 0) ptx::tmem_dealloc(tbase, 512);
 }
 
 // A bounded wait that runs out on purpose: an mbarrier nothing arrives on, waited on with the

@@ -200,7 +200,8 @@ hla_status_t hla2_forward_normalized_noalloc(const void* q, const void* k, const
  * with A given row-major as a[M][K] (bit 1 clear: K-major) or as a[K][M]
  * (bit 1 set: MN-major), and B given as b[N][K] (bit 0 clear: K-major) or as
  * b[K][N] (bit 0 set: MN-major).  Bit 2 selects M = 64 (else 128); bit 3 (with
- * bit 2) places the M = 64 accumulator at TMEM lane offset 16.  N is 64, 128,
+ * bit 2) places the M = 64 accumulator at TMEM lane offset 16.  Bit 4 reads A from
+ * tensor memory (M = 128 and a given as a[M][K]; not with bits 1-3).  N is 64, 128,
  * 192 or 256; K is 64 or 128 (else HLA_ERR_SHAPE).
  * a, b: device bf16; d: device fp32 [M][N].  Enqueued on `stream`.
  */

@@ -135,7 +135,9 @@ def test_segment_chunks_knob(lib):
 def test_selftest_argument_errors(lib):
     vp = ctypes.c_void_p
     assert lib.hla_selftest_umma(0, vp(0), vp(16), vp(16), 64, 64, vp(0)) == 1
-    assert lib.hla_selftest_umma(16, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
+    assert lib.hla_selftest_umma(32, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
+    assert lib.hla_selftest_umma(18, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5   # TMEM A, MN-major
+    assert lib.hla_selftest_umma(20, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5   # TMEM A, M = 64
     assert lib.hla_selftest_umma(8, vp(16), vp(16), vp(16), 64, 64, vp(0)) == 5
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 96, 64, vp(0)) == 2
     assert lib.hla_selftest_umma(0, vp(16), vp(16), vp(16), 320, 64, vp(0)) == 2

@@ -50,7 +50,7 @@ def reference(op, q, k, v, gamma, eps=1e-6):
 # tensor-core layout self-check (one tcgen05 MMA), against fp64 on the host
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("case", [0, 1, 2, 3, 4, 5, 6, 7, 12, 13, 14, 15])
+@pytest.mark.parametrize("case", [0, 1, 2, 3, 4, 5, 6, 7, 12, 13, 14, 15, 16, 17])
 @pytest.mark.parametrize("N,K", [(64, 64), (128, 64), (64, 128), (128, 128), (192, 64), (256, 64), (256, 128)])
 def test_umma_layouts(case, N, K):
     g = torch.Generator().manual_seed(case * 7 + N + K)
