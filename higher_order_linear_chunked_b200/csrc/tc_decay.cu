@@ -27,14 +27,14 @@
 // writing it as a difference of separately rounded products would lose the weight to bf16
 // rounding at strong decay (H A*^T + A A^T) or at weak decay (At A*^T - A U^T).
 //
-// Kernels (one CTA per chunk x head, every chunk independent):
+// Kernels (every chunk independent):
 //   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G^T), fp32
 //   k_dec_prefix_sc, k_dec_cross, k_dec_prefix_g (CUDA cores)
 //                                               in place: S0, C0; Y^T = G^T + rho C0^T Khat;
 //                                               G0^T (Khat is symmetric)
-//   k_dec_output (tcgen05)                      turns (S0, C0, G0) into bf16 operand tiles
-//                                               while its Q/K/V loads are in flight; O,
-//                                               written by TMA bulk tensor stores
+//   k_dec_output (tcgen05, persistent: one CTA per SM over the chunks)
+//                                               turns (S0, C0, G0^T) into bf16 operand tiles
+//                                               and forms O, written by TMA bulk tensor stores
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -361,35 +361,40 @@ __global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
     }
 }
 
-// ---------------------------------------------------------------- output
-// Shared memory:
-constexpr uint32_t S3_Q = 0;                 // Q [tok][feat]
-constexpr uint32_t S3_K = S3_Q + TILE;       // K                    } B rows of R1:
-constexpr uint32_t S3_SG = S3_K + TILE;      // S0 (rows), G0^T tiles } [K ; S0^T ; G0^T]
-constexpr uint32_t S3_C0 = S3_SG + 2 * QTILE;   // C0 (rows: MN-major B operand)
-constexpr uint32_t S3_V = S3_C0 + QTILE;     // V
-constexpr uint32_t S3_AT = S3_V + TILE;      // At, later the O staging boxes
-constexpr uint32_t S3_H = S3_AT + 2 * TILE;  // H, later W
-constexpr uint32_t S3_A = S3_H + 2 * TILE;   // A
-constexpr uint32_t S3_U = S3_A + 2 * TILE;   // U
-constexpr uint32_t S3_P = S3_U + 2 * TILE;   // Gam P, later Gam (H K)
-constexpr uint32_t S3_TAB = S3_P + TILE;     // g^n, n = 0..256
-constexpr uint32_t S3_BAR = S3_TAB + 260 * 4;
+// ---------------------------------------------------------------- output (persistent)
+// One CTA per SM takes the (chunk, head) items w = blockIdx.x, blockIdx.x + gridDim.x, ...;
+// items are independent.  Q, K, V and the carried-in state tiles are double buffered: the
+// next item's TMA loads are issued as an item starts, and the epilogue warps turn the next
+// item's fp32 state into bf16 tiles while the current item's second MMA round runs.  At, H,
+// W and Gam Z are MMA A operands read from tensor memory.
+//
+// Shared memory: two stages of [Q | K | S0, G0^T | C0 | V] (72 KB each; K sits directly
+// before S0, G0^T so that [K ; S0^T ; G0^T] is one B operand), then A, U (B operands), Gam P,
+// the table of gamma powers and the barriers.
+constexpr uint32_t SQ_ = 0, SK_ = TILE, SSG_ = 2 * TILE, SC0_ = 2 * TILE + 2 * QTILE;
+constexpr uint32_t SV_ = 2 * TILE + 3 * QTILE;
+constexpr uint32_t STAGE3 = 3 * TILE + 3 * QTILE;   // 72 KB
+constexpr uint32_t S3_A = 2 * STAGE3;               // A, later the O staging boxes
+constexpr uint32_t S3_U = S3_A + 2 * TILE;          // U
+constexpr uint32_t S3_P = S3_U + 2 * TILE;          // Gam P
+constexpr uint32_t S3_TAB = S3_P + TILE;            // g^n, n = 0..256
+constexpr uint32_t S3_BAR = S3_TAB + 260 * 4;       // 2 load barriers, the MMA barrier, TMEM slot
 constexpr uint32_t S3_BYTES = S3_BAR + 64 + 1024;   // + alignment slack
 
 // TMEM columns
-constexpr uint32_t T3_AS = 0;     // A*, then W   (128)
-constexpr uint32_t T3_P = 128;    // P            (64)
-constexpr uint32_t T3_QG = 192;   // Q G0         (64)
-constexpr uint32_t T3_HK = 256;   // H K          (64)
-constexpr uint32_t T3_O = 320;    // O            (64)
+constexpr uint32_t T3_AS = 0;     // A*, then W (fp32)        (128)
+constexpr uint32_t T3_P = 128;    // P                        (64)
+constexpr uint32_t T3_QG = 192;   // Q G0                     (64)
+constexpr uint32_t T3_HK = 256;   // H K                      (64)
+constexpr uint32_t T3_O = 320;    // O                        (64)
+constexpr uint32_t T3_AT = 384;   // At, then W (bf16 pairs)  (64)
+constexpr uint32_t T3_H = 448;    // H, then Gam Z (bf16)     (64)
 
-// Prologue: (S0, C0, G0^T) fp32 from the chunk state to bf16 tiles (S0 = S0^T: the key moment
-// is symmetric), overlapping the Q/K/V loads.
-// Rounds: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T          -> E1: At, H, A, U, Gam P to bf16
-//         R2 W = Gam P Q^T + At A^T + H U^T; H K               -> E2: W (masked, Dg); Gam Z,
-//                                                                   Z = Gam P + H K
-//         R3 O = W V + (Gam Z) C0                              -> E3: O - Gam Q G0
+// Rounds per item: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T  -> E1: At, H to TMEM; A, U,
+//                                                                  Gam P to shared memory
+//                  R2 W = Gam P Q^T + At A^T + H U^T; H K      -> E2: W (masked, Dg) and
+//                                                                  Gam Z = Gam (Gam P + H K) to TMEM
+//                  R3 O = W V + (Gam Z) C0                     -> E3: O - Gam Q G0, TMA store
 __global__ void __launch_bounds__(DNT, 1)
 k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, DParams p) {
@@ -398,52 +403,59 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int items = p.NC * p.BH;
+    const int w0 = blockIdx.x;
+    if (w0 >= items) return;
     float* gp = reinterpret_cast<float*>(sm + S3_TAB);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S3_BAR);
-    MmaSync ms{bar_load + 1, 0};
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
-    const float g = p.gamma[bh % p.H];
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S3_BAR);   // [2]
+    MmaSync ms{bar_load + 2, 0};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 3);
     if (tid == 0) {
-        ptx::mbar_init(bar_load, 1);
+        ptx::mbar_init(&bar_load[0], 1);
+        ptx::mbar_init(&bar_load[1], 1);
         ptx::mbar_init(ms.bar, 1);
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    if (tid == 0) {
-        const int t0 = chunk * C;
-        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE);
-        ptx::tma_load_3d(sm + S3_Q, &tq, bar_load, 0, t0, bh);
-        ptx::tma_load_3d(sm + S3_K, &tk, bar_load, 0, t0, bh);
-        ptx::tma_load_3d(sm + S3_V, &tv, bar_load, 0, t0, bh);
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 512);
-        ptx::tmem_relinquish();
-    }
-    for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
-    {
-        // carried-in S0, C0 and G0^T -> bf16 operand tiles, row for row (row r, 16-byte chunk j
-        // at j ^ (r & 7)); S0 is symmetric, so its rows serve as the K-major S0^T
-        constexpr int NI = 3 * D * 8 / DNT;                // 16-byte chunks per thread
+    int issued[2] = {0, 0}, waited[2] = {0, 0};       // thread 0's load bookkeeping
+    auto issue_loads = [&](int w, int b) {
+        uint8_t* st = sm + b * STAGE3;
+        const int bh = w / p.NC, t0 = (w % p.NC) * C;
+        ptx::mbar_arrive_expect_tx(&bar_load[b], 3 * TILE);
+        ptx::tma_load_3d(st + SQ_, &tq, &bar_load[b], 0, t0, bh);
+        ptx::tma_load_3d(st + SK_, &tk, &bar_load[b], 0, t0, bh);
+        ptx::tma_load_3d(st + SV_, &tv, &bar_load[b], 0, t0, bh);
+        ++issued[b];
+    };
+    // carried-in S0, C0 and G0^T of item w -> bf16 operand tiles of stage b, row for row (row r,
+    // 16-byte chunk j at j ^ (r & 7)); S0 is symmetric, so its rows serve as the K-major S0^T
+    auto convert_state = [&](int w, int b) {
+        uint8_t* st = sm + b * STAGE3;
+        const int bh = w / p.NC, l = w % p.NC;
+        constexpr int NI = 3 * D * 8 / DNT;
         float4 x[NI][2];
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
             const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
-            const int e = (t == 2 ? 3 : t) * D * D + r * D + 8 * j;
-            const float4* src = reinterpret_cast<const float4*>(dsum(p, bh, chunk, e));
+            const float4* src = reinterpret_cast<const float4*>(dsum(p, bh, l, (t == 2 ? 3 : t) * D * D + r * D + 8 * j));
             x[i][0] = src[0];
             x[i][1] = src[1];
         }
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
             const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
-            const uint32_t tile = t == 0 ? S3_SG : t == 1 ? S3_C0 : S3_SG + QTILE;
-            *reinterpret_cast<uint4*>(sm + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
+            const uint32_t tile = t == 0 ? SSG_ : t == 1 ? SC0_ : SSG_ + QTILE;
+            *reinterpret_cast<uint4*>(st + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
                 make_uint4(ptx::pack_bf16(x[i][0].x, x[i][0].y), ptx::pack_bf16(x[i][0].z, x[i][0].w),
                            ptx::pack_bf16(x[i][1].x, x[i][1].y), ptx::pack_bf16(x[i][1].z, x[i][1].w));
         }
+    };
+    if (tid == 0) issue_loads(w0, 0);
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
     }
+    convert_state(w0, 0);
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
     __syncthreads();
@@ -451,132 +463,168 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t sb = ptx::smem_u32(sm);
+    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 256, false, false);
+    constexpr uint32_t I_W = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
+    // packed bf16 pairs of 32 values (columns c0 .. c0+31) into 16 TMEM columns of this lane
+    auto st_pairs = [&](uint32_t tcol, const float (&x)[32]) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = ptx::pack_bf16(x[2 * i], x[2 * i + 1]);
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    auto st_pairs_zero = [&](uint32_t tcol) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+
     bool ok = true;
-    if (tid == 0) {
-        ok = ptx::mbar_wait(bar_load, 0);
-        if (ok) {
-            ptx::tc_fence_after();
-            constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 256, false, false);
-            const uint64_t dQ = kdesc(sb + S3_Q, 0), dKSG = kdesc(sb + S3_K, 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dQ, s), k1s(dKSG, s), I_R1, s > 0);
+    int cur_bh = -1;
+    int it = 0;
+    for (int w = w0; w < items && ok; w += gridDim.x, ++it) {
+        const int b = it & 1;
+        const uint32_t st = b * STAGE3;
+        const int bh = w / p.NC, chunk = w % p.NC;
+        const int wn = w + gridDim.x;
+        if (bh != cur_bh) {                  // gamma powers of this item's head (block-uniform)
+            cur_bh = bh;
+            const float g = p.gamma[bh % p.H];
+            for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
         }
-    }
-    ok = __syncthreads_and(ok) != 0;
-    if (ok) ok = ms.commit_wait(tid == 0);      // R1 done
-    if (ok) {
-        // E1: from A* row `row` (columns half*64 .. +63): At, H, A, U; Gam P (columns half*32 .. +31)
-        // 32 x 32 blocks wholly above the diagonal are zero in At, H and A, and wholly below
-        // it zero in U: those are written without conversions (the test is warp-uniform).
-        float v[32], w[32];
-#pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
-            if (c0 > quad * 32 + 31) {                                 // above the diagonal
-                st_row32_zero(sm + S3_AT, row, c0);
-                st_row32_zero(sm + S3_H, row, c0);
-                st_row32_zero(sm + S3_A, row, c0);
-                st_row32(sm + S3_U, row, c0, v);
-                continue;
+        if (tid == 0) {
+            if (wn < items) issue_loads(wn, b ^ 1);        // stage b^1 was freed by the last item
+            ok = ptx::mbar_wait(&bar_load[b], (it >> 1) & 1);
+            if (ok) {
+                ++waited[b];
+                ptx::tc_fence_after();
+                const uint64_t dQ = kdesc(sb + st + SQ_, 0), dKSG = kdesc(sb + st + SK_, 0);
+                for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dQ, s), k1s(dKSG, s), I_R1, s > 0);
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int d = row - (c0 + i);                          // tau - i
-                w[i] = d >= 0 ? gp[d] * v[i] : 0.f;                    // At
-            }
-            st_row32(sm + S3_AT, row, c0, w);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int d = row - (c0 + i);
-                w[i] = d > 0 ? (gp[d] - 1.f) * v[i] : 0.f;            // H
-            }
-            st_row32(sm + S3_H, row, c0, w);
-            if (c0 + 31 < quad * 32) {                                 // below the diagonal
-                st_row32(sm + S3_A, row, c0, v);
-                st_row32_zero(sm + S3_U, row, c0);
-                continue;
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = (c0 + i <= row) ? v[i] : 0.f;   // A
-            st_row32(sm + S3_A, row, c0, w);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = (c0 + i > row) ? v[i] : 0.f;    // U
-            st_row32(sm + S3_U, row, c0, w);
+            ptx::bulk_wait_read();                          // the last item's O boxes (over A) are read
         }
-        ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
-        const float gam = gp[row + 1];
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R1 done
+        {
+            // E1: from A* row `row`, columns half*64 .. +63 in two blocks of 32: At, H (TMEM, bf16
+            // pairs), A, U (shared memory); Gam P (columns half*32 .. +31).  Blocks wholly above
+            // the diagonal are zero in At, H and A, blocks wholly below it zero in U.
+            float v[32], w32[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= gam;
-        st_row32(sm + S3_P, row, half * 32, v);
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
+                if (c0 > quad * 32 + 31) {
+                    st_pairs_zero(T3_AT + c0 / 2);
+                    st_pairs_zero(T3_H + c0 / 2);
+                    st_row32_zero(sm + S3_A, row, c0);
+                    st_row32(sm + S3_U, row, c0, v);
+                    continue;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int d = row - (c0 + i);                      // tau - i
+                    w32[i] = d >= 0 ? gp[d] * v[i] : 0.f;              // At
+                }
+                st_pairs(T3_AT + c0 / 2, w32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int d = row - (c0 + i);
+                    w32[i] = d > 0 ? (gp[d] - 1.f) * v[i] : 0.f;      // H
+                }
+                st_pairs(T3_H + c0 / 2, w32);
+                if (c0 + 31 < quad * 32) {
+                    st_row32(sm + S3_A, row, c0, v);
+                    st_row32_zero(sm + S3_U, row, c0);
+                    continue;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i <= row) ? v[i] : 0.f;   // A
+                st_row32(sm + S3_A, row, c0, w32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i > row) ? v[i] : 0.f;    // U
+                st_row32(sm + S3_U, row, c0, w32);
+            }
+            ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
+            const float gam = gp[row + 1];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= gam;
+            st_row32(sm + S3_P, row, half * 32, v);
+            ptx::tmem_st_wait();
+        }
         sync_for_mma();
         if (tid == 0) {
-            constexpr uint32_t I_W = ptx::idesc_bf16(128, 128, false, false);
-            constexpr uint32_t I_HK = ptx::idesc_bf16(128, 64, false, true);
-            const uint64_t dP = kdesc(sb + S3_P, 0), dQ = kdesc(sb + S3_Q, 0);
-            const uint64_t dAt = kdesc2(sb + S3_AT, 0), dA = kdesc2(sb + S3_A, 0);
-            const uint64_t dH = kdesc2(sb + S3_H, 0), dU = kdesc2(sb + S3_U, 0);
-            const uint64_t dKm = mdesc(sb + S3_K, TILE, 0);
+            const uint64_t dP = kdesc(sb + S3_P, 0), dQ = kdesc(sb + st + SQ_, 0);
+            const uint64_t dA = kdesc2(sb + S3_A, 0), dU = kdesc2(sb + S3_U, 0);
+            const uint64_t dKm = mdesc(sb + st + SK_, TILE, 0);
             for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dP, s), k1s(dQ, s), I_W, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dAt, s), k2s(dA, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_AS, k2s(dH, s), k2s(dU, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_HK, k2s(dH, s), mns(dKm, s), I_HK, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_AS, tmem + T3_AT + 8 * s, k2s(dA, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_AS, tmem + T3_H + 8 * s, k2s(dU, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_HK, tmem + T3_H + 8 * s, mns(dKm, s), I_KM, s > 0);
         }
-        ok = ms.commit_wait(tid == 0);          // R2 done
-    }
-    if (ok) {
-        // E2: W[tau][j] = g^(tau-j) x for j <= tau -> over H; Gam (Gam P + H K) -> over Gam P
-        float v[32], w[32];
+        if (wn < items) convert_state(wn, b ^ 1);                  // overlaps R2
+        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R2 done
+        {
+            // E2: W[tau][j] = g^(tau-j) x for j <= tau -> TMEM over At; Gam (Gam P + H K) -> over H
+            float v[32], w32[32];
 #pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 > quad * 32 + 31) {                                 // above the diagonal
-                st_row32_zero(sm + S3_H, row, c0);
-                continue;
-            }
-            ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) {
+                    st_pairs_zero(T3_AT + c0 / 2);
+                    continue;
+                }
+                ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int d = row - (c0 + i);
-                v[i] = d >= 0 ? gp[d] * v[i] : 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    const int d = row - (c0 + i);
+                    v[i] = d >= 0 ? gp[d] * v[i] : 0.f;
+                }
+                st_pairs(T3_AT + c0 / 2, v);
             }
-            st_row32(sm + S3_H, row, c0, v);
+            ptx::tmem_ld32x2(tmem + lane_base + T3_P + half * 32, tmem + lane_base + T3_HK + half * 32, v, w32);
+            const float gam = gp[row + 1];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = gam * fmaf(gam, v[i], w32[i]);
+            st_pairs(T3_H + half * 16, v);
+            ptx::tmem_st_wait();
         }
-        ptx::tmem_ld32x2(tmem + lane_base + T3_P + half * 32, tmem + lane_base + T3_HK + half * 32, v, w);
-        const float gam = gp[row + 1];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = gam * fmaf(gam, v[i], w[i]);
-        st_row32(sm + S3_P, row, half * 32, v);
         sync_for_mma();
         if (tid == 0) {
-            constexpr uint32_t I_O = ptx::idesc_bf16(128, 64, false, true);
-            const uint64_t dW = kdesc2(sb + S3_H, 0), dVm = mdesc(sb + S3_V, TILE, 0);
-            const uint64_t dP = kdesc(sb + S3_P, 0), dC = mdesc(sb + S3_C0, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3_O, k2s(dW, s), mns(dVm, s), I_O, s > 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_O, k1s(dP, s), mns(dC, s), I_O, 1);
+            const uint64_t dVm = mdesc(sb + st + SV_, TILE, 0), dC = mdesc(sb + st + SC0_, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_O, tmem + T3_AT + 8 * s, mns(dVm, s), I_KM, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16_ts(tmem + T3_O, tmem + T3_H + 8 * s, mns(dC, s), I_KM, 1);
         }
-        ok = ms.commit_wait(tid == 0);          // R3 done
-    }
-    if (ok) {
-        // E3: O - Gam (Q G0), staged as two [128][32] fp32 boxes over At
-        float o[32], m[32];
-        ptx::tmem_ld32x2(tmem + lane_base + T3_O + half * 32, tmem + lane_base + T3_QG + half * 32, o, m);
-        const float gam = gp[row + 1];
+        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R3 done
+        {
+            // E3: O - Gam (Q G0), staged as two [128][32] fp32 boxes over A, then TMA stores
+            float o[32], m[32];
+            ptx::tmem_ld32x2(tmem + lane_base + T3_O + half * 32, tmem + lane_base + T3_QG + half * 32, o, m);
+            const float gam = gp[row + 1];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = fmaf(-gam, m[i], o[i]);
-        float4* box = reinterpret_cast<float4*>(sm + S3_AT + half * (C * 128) + row * 128);
+            for (int i = 0; i < 32; ++i) o[i] = fmaf(-gam, m[i], o[i]);
+            float4* box = reinterpret_cast<float4*>(sm + S3_A + half * (C * 128) + row * 128);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) box[j ^ (row & 7)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-        ptx::fence_proxy_async();
+            for (int j = 0; j < 8; ++j) box[j ^ (row & 7)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            ptx::fence_proxy_async();
+        }
         __syncthreads();
         if (tid == 0) {
-            ptx::tma_store_3d(&to, sm + S3_AT, 0, chunk * C, bh);
-            ptx::tma_store_3d(&to, sm + S3_AT + C * 128, 32, chunk * C, bh);
+            ptx::tma_store_3d(&to, sm + S3_A, 0, chunk * C, bh);
+            ptx::tma_store_3d(&to, sm + S3_A + C * 128, 32, chunk * C, bh);
             ptx::bulk_commit();
-            ptx::bulk_wait_all();
         }
-    } else if (tid == 0) {
-        set_status(p.status, DEV_TIMEOUT);
-        ptx::mbar_wait(bar_load, 0, 100000000ull);
-        ptx::umma_commit(ms.bar);
-        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+    }
+    if (tid == 0) {
+        ptx::bulk_wait_all();
+        if (!ok) {
+            set_status(p.status, DEV_TIMEOUT);
+            // let loads and MMAs already in flight land before TMEM and shared memory are released
+            for (int b = 0; b < 2; ++b)
+                if (issued[b] > waited[b]) ptx::mbar_wait(&bar_load[b], (issued[b] - 1) & 1, 100000000ull);
+            ptx::umma_commit(ms.bar);
+            ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+        }
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -621,7 +669,8 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
     k_dec_prefix_g<<<dim3((D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    k_dec_output<<<dim3(NC, BH), DNT, S3_BYTES, st>>>(mq, mk, mv, mo, prm);
+    const int items = NC * BH;
+    k_dec_output<<<items < kSMs ? items : kSMs, DNT, S3_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
