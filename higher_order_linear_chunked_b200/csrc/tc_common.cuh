@@ -94,18 +94,6 @@ __device__ __forceinline__ void st_row32_zero(uint8_t* tile, int row, int c0) {
         *reinterpret_cast<uint4*>(atom + row * 128 + (((chunk ^ row) & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
     }
 }
-// Transposed write of 32 values: v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
-__device__ __forceinline__ void st_col32(uint8_t* tile, int kcol, int c0, const float (&v)[32]) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
-}
-// Transposed write: value v[i] is element (n = c0 + i, k = kcol) of a K-major tile.
-__device__ __forceinline__ void st_col16(uint8_t* tile, int kcol, int c0, const float (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        *reinterpret_cast<bf16*>(tile + ptx::sw128_offset(c0 + i, kcol)) = __float2bfloat16_rn(v[i]);
-}
 
 // ---------------------------------------------------------------- host side
 // [BH][T][64] bf16 tensor, box = one 128-token chunk, 128-byte swizzle, zero fill past T.
