@@ -78,7 +78,8 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const int row = quad * 32 + lane;                     // TMEM lane = tile row
     const int seg = blockIdx.x, bh = blockIdx.y;
     using S = simt_layout;
-    float* slot = (MODE == OUTPUT ? p.pre : p.sums) + ((size_t)bh * p.NSp + seg) * S::size;
+    float* slot = MODE == OUTPUT ? p.pre + ((size_t)bh * p.NSp + seg * p.ratio) * S::size
+                                 : p.sums + ((size_t)bh * p.NSp + seg) * S::size;
     if (seg >= p.NS) {                                    // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
@@ -327,13 +328,15 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
-    Params prm;
-    prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp;
+    Params prm;                              // the output walk
+    prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = 0.f; prm.norm = 0;
     prm.sums = static_cast<float*>(ws);
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
+    Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
+    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_ahla_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ASMEM_BYTES)) != cudaSuccess)
@@ -342,10 +345,10 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
                                   ASMEM_BYTES)) != cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
+    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if ((e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -30,6 +30,7 @@ struct simt_layout {
 
 struct Params {
     int T, BH, NCH, NS, NSp;
+    int ratio;      // output walk: summary slots per output segment (prefix of segment s at s * ratio)
     float eps;
     int norm;       // second order: divide by the denominator
     float* sums;     // [BH][NSp][summary floats]: segment summaries
@@ -103,11 +104,16 @@ bool make_map_out(CUtensorMap* map, float* base, int T, int BH);
 
 struct Plan {
     int NC;    // chunks per head
-    int NCH;   // chunks per segment
-    int NS;    // segments per head
-    int NSp;   // NS rounded up to a power of two (summary slots per head)
+    int NCH;   // chunks per output segment
+    int NS;    // output segments per head
+    int NCHs;  // chunks per summary segment (divides NCH)
+    int NSf;   // summary segments per head: they cover the chunks before the last output segment
+    int NSp;   // NSf + 1 rounded up to a power of two (summary / prefix slots per head)
+    int ratio; // NCH / NCHs
 };
-// Segment length for BH heads of T tokens when `slots` walker CTAs can run at once.
+// Segment lengths for BH heads of T tokens when `slots` walker CTAs can run at once.  The
+// last output segment's summary is never needed, so summaries cover (NS - 1) NCH chunks per
+// head, in segments short enough to fill the machine.
 Plan plan(int BH, int T, int slots);
 
 // Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for

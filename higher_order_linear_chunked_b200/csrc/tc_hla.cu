@@ -94,7 +94,8 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     const bool epi = warp < NT / 32;                                      // an epilogue warp
     const int seg = blockIdx.x, bh = blockIdx.y;
     using S = simt_layout;
-    float* slot = (MODE == OUTPUT ? p.pre : p.sums) + ((size_t)bh * p.NSp + seg) * S::size;
+    float* slot = MODE == OUTPUT ? p.pre + ((size_t)bh * p.NSp + seg * p.ratio) * S::size
+                                 : p.sums + ((size_t)bh * p.NSp + seg) * S::size;
     if (seg >= p.NS) {                       // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
@@ -643,26 +644,44 @@ bool make_map_out(CUtensorMap* map, float* base, int T, int BH) {
 Plan plan(int BH, int T, int slots) {
     Plan pl;
     pl.NC = (T + C - 1) / C;
+    // Costs in chunk-times.  One walk over CTAs of `len` chunks takes (waves of CTAs) x (len +
+    // about one chunk of set-up); the prefix kernels take about one per summary slot of a head.
+    auto cost = [&](long long ctas, int len) { return ((ctas + slots - 1) / slots) * (long long)(len + 1); };
+    // Summaries are needed for the chunks before the last output segment; shorter summary
+    // segments shorten the summary walk but lengthen the prefix.
+    auto summary_cost = [&](int nch, int& len_out) -> long long {
+        const int ncsum = ((pl.NC + nch - 1) / nch - 1) * nch;
+        len_out = nch;
+        if (ncsum == 0) return 0;
+        long long best = -1;
+        for (int len = nch; len >= 1; len /= 2) {
+            const long long c = cost((long long)BH * (ncsum / len), len) + ncsum / len;
+            if (best < 0 || c < best) {
+                best = c;
+                len_out = len;
+            }
+        }
+        return best;
+    };
     if (g_segment_chunks > 0) {
         pl.NCH = g_segment_chunks;
     } else {
-        // One CTA walks one segment; `slots` CTAs run at once: the walk's makespan is
-        // (waves of CTAs) x (chunks per segment + about one chunk of per-CTA set-up).
-        // Pick the segment length that minimises it (ties: the longer segment).
-        long long best = -1;
+        long long best = -1;                 // ties: the longer output segment
         for (int nch = 1; nch <= 16; nch *= 2) {
-            const long long ctas = (long long)BH * ((pl.NC + nch - 1) / nch);
-            const long long waves = (ctas + slots - 1) / slots;
-            const long long cost = waves * (nch + 1);
-            if (best < 0 || cost <= best) {
-                best = cost;
+            int len;
+            const long long c = cost((long long)BH * ((pl.NC + nch - 1) / nch), nch) + summary_cost(nch, len);
+            if (best < 0 || c <= best) {
+                best = c;
                 pl.NCH = nch;
             }
             if (nch >= pl.NC) break;
         }
     }
     pl.NS = (pl.NC + pl.NCH - 1) / pl.NCH;
-    pl.NSp = next_pow2(pl.NS);
+    summary_cost(pl.NCH, pl.NCHs);
+    pl.NSf = (pl.NS - 1) * pl.NCH / pl.NCHs;
+    pl.ratio = pl.NCH / pl.NCHs;
+    pl.NSp = next_pow2(pl.NSf + 1);
     return pl;
 }
 
@@ -707,13 +726,15 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, kSMs);
-    Params prm;
-    prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp;
+    Params prm;                              // the output walk
+    prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = eps; prm.norm = norm ? 1 : 0;
     prm.sums = static_cast<float*>(ws);
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
+    Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
+    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
         cudaSuccess)
@@ -722,10 +743,10 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_walk<SUMMARY><<<dim3(pl.NSp, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
+    k_walk<SUMMARY><<<dim3(pl.NSp, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = launch_prefix(prm.sums, prm.pre, pl.NS, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if ((e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_walk<OUTPUT><<<dim3(pl.NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
