@@ -316,6 +316,8 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 }  // namespace
 
+int ahla_ctas_per_sm() { return kCtasPerSM; }
+
 size_t ahla_workspace_bytes(int BH, int T) {
     const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;

@@ -117,7 +117,8 @@ struct Plan {
 Plan plan(int BH, int T, int slots);
 
 // Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for
-// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
+// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  One launch for up to
+// nine slots per head, two beyond.
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st);
 
 // The decayed second-order forward, chunk-parallel (tc_decay.cu).
@@ -128,6 +129,7 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
 
 // The AHLA forward on the tcgen05 walkers (tc_ahla.cu).
 size_t ahla_workspace_bytes(int BH, int T);
+int ahla_ctas_per_sm();
 cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
                          int* status, cudaStream_t st, cudaEvent_t* ev);
 
