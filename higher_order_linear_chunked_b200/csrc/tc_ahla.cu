@@ -339,6 +339,7 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     prm.status = status;
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
     sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1;
+    prm.fold = sprm.fold = 0;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_ahla_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ASMEM_BYTES)) != cudaSuccess)

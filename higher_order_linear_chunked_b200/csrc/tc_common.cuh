@@ -31,6 +31,7 @@ struct simt_layout {
 struct Params {
     int T, BH, NCH, NS, NSp;
     int ratio;      // output walk: summary slots per output segment (prefix of segment s at s * ratio)
+    int fold;       // output walk: fold the prefix from the summaries (no prefix kernels)
     float eps;
     int norm;       // second order: divide by the denominator
     float* sums;     // [BH][NSp][summary floats]: segment summaries

@@ -140,11 +140,90 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         for (int j = 0; j < 8; ++j)
             *reinterpret_cast<uint4*>(r + (((j ^ tid) & 7) << 4)) = make_uint4(j == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
     }
-    // Carried-in state (OUTPUT): the prefix (S, R, r) is staged in shared memory with
-    // coalesced loads (rows swizzled by 16-byte chunk), then every thread takes its row.
+    // Carried-in state (OUTPUT): the prefix (S, R, r) is staged in shared memory (rows swizzled
+    // by 16-byte chunk: element (i, j) at i*64 + ((j/4 ^ (i & 7)) * 4) + j % 4), then every
+    // thread takes its row.  With p.fold the CTA folds the summaries of slots 0 .. seg*ratio - 1
+    // itself (R0 += R_l + S0 C_l, r0 += r_l + S0 m_l, then S0 += S_l), while its first loads
+    // are in flight; otherwise it reads the prefix the prefix kernels wrote.
     float* stage = reinterpret_cast<float*>(sm + SM_A);                   // S [64][64] | R [64][64]
     float* stage_r = reinterpret_cast<float*>(sm + SM_Z);                 // r [64]
-    if (MODE == OUTPUT && epi) {
+    auto sw = [](int i, int j) { return i * D + ((((j >> 2) ^ (i & 7)) << 2) | (j & 3)); };
+    if (MODE == OUTPUT && epi && p.fold) {
+        // n = seg * ratio slots: S0 = sum_l S_l, R0 = sum_l R_l + sum_{m < n-1} S_m Csuf(m+1),
+        // r0 = sum_l r_l + sum_{m < n-1} S_m msuf(m+1), with Csuf(m) = sum_{m <= l < n} C_l (the
+        // factored prefix, cross terms grouped by their S factor).  The plain sums are one batch
+        // of loads; each cross term is one 64 x 64 x 64 product.
+        const int n = seg * p.ratio;
+        const float* sb = p.sums + (size_t)bh * p.NSp * S::size;
+        float* Cs = reinterpret_cast<float*>(sm + SM_OST);                // Csuf [64][64]
+        float* msuf = Cs + D * D;                                         // msuf [64]
+        float* Sm = stage + D * D;                                        // S_m [64][64] (R part, for now)
+        const int r = 4 * (tid >> 4), c = 4 * (tid & 15);                 // this thread's 4 x 4 of R0
+        constexpr int NF = D * D / 4 / NT;                                // float4 per thread
+        float racc[4][4];
+        float4 sacc[NF];
+        float r0 = 0.f;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) racc[a][b] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NF; ++i) sacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int l = 0; l < n; ++l) {
+            const float* sl = sb + (size_t)l * S::size;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float4 x = *reinterpret_cast<const float4*>(sl + S::mat(2) + (r + a) * D + c);
+                racc[a][0] += x.x; racc[a][1] += x.y; racc[a][2] += x.z; racc[a][3] += x.w;
+            }
+#pragma unroll
+            for (int i = 0; i < NF; ++i) {
+                const float4 x = reinterpret_cast<const float4*>(sl + S::mat(0))[tid + NT * i];
+                sacc[i] = make_float4(sacc[i].x + x.x, sacc[i].y + x.y, sacc[i].z + x.z, sacc[i].w + x.w);
+            }
+            if (tid < D) r0 += sl[S::vec(1) + tid];
+        }
+        for (int m = n - 2; m >= 0; --m) {
+            const float* cl = sb + (size_t)(m + 1) * S::size;
+            const float* smp = sb + (size_t)m * S::size;
+            for (int f = tid; f < D * D / 4; f += NT) {
+                const float4 x = reinterpret_cast<const float4*>(cl + S::mat(1))[f];
+                const float4 o = m == n - 2 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<float4*>(Cs)[f];
+                reinterpret_cast<float4*>(Cs)[f] = make_float4(o.x + x.x, o.y + x.y, o.z + x.z, o.w + x.w);
+                reinterpret_cast<float4*>(Sm)[f] = reinterpret_cast<const float4*>(smp + S::mat(0))[f];
+            }
+            if (tid < D) msuf[tid] = (m == n - 2 ? 0.f : msuf[tid]) + cl[S::vec(0) + tid];
+            ptx::named_sync(1, NT);          // the epilogue warps only
+#pragma unroll 8
+            for (int k = 0; k < D; ++k) {
+                const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const float sv = Sm[(r + a) * D + k];
+                    racc[a][0] = fmaf(sv, cv.x, racc[a][0]);
+                    racc[a][1] = fmaf(sv, cv.y, racc[a][1]);
+                    racc[a][2] = fmaf(sv, cv.z, racc[a][2]);
+                    racc[a][3] = fmaf(sv, cv.w, racc[a][3]);
+                }
+            }
+            if (tid < D) {                   // (S_m msuf)[tid] = sum_k S_m[k][tid] msuf[k] (S_m is symmetric)
+                float y = 0.f;
+                for (int k = 0; k < D; ++k) y = fmaf(Sm[k * D + tid], msuf[k], y);
+                r0 += y;
+            }
+            ptx::named_sync(1, NT);
+        }
+#pragma unroll
+        for (int i = 0; i < NF; ++i) {
+            const int f = tid + NT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
+            reinterpret_cast<float4*>(stage)[rr * 16 + ch] = sacc[i];
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) stage[D * D + sw(r + a, c + b)] = racc[a][b];
+        if (tid < D) stage_r[tid] = r0;
+    } else if (MODE == OUTPUT && epi) {
         const float4* s4 = reinterpret_cast<const float4*>(slot + S::mat(0));
         const float4* r4 = reinterpret_cast<const float4*>(slot + S::mat(2));
         float4 xs[4], xr[4];
@@ -797,9 +876,11 @@ size_t workspace_bytes(int op, bool /*norm*/, int BH, int T) {
 
 int kernel_launches(int op, bool /*norm*/, int BH, int T) {
     if (op == OP_HLA2D) return decay_kernel_launches();
-    // summary walk, the prefix (one launch up to PH_MAX slots per head, else two), output walk
+    // summary walk, the prefix (second order up to PH_MAX slots per head: folded into the output
+    // walk; AHLA: one launch up to PH_MAX slots, else two), output walk
     const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm() * kSMs : kSMs);
-    return pl.NSf + 1 <= PH_MAX ? 3 : 4;
+    if (pl.NSf + 1 > PH_MAX) return 4;
+    return op == OP_AHLA ? 3 : 2;            // second order: the output walker folds the prefix
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
@@ -820,8 +901,9 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
+    prm.fold = pl.NSf + 1 <= PH_MAX ? 1 : 0;  // few slots: each output CTA folds its own prefix
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
-    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1;
+    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
         cudaSuccess)
@@ -833,7 +915,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     k_walk<SUMMARY><<<dim3(pl.NSp, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_walk<OUTPUT><<<dim3(pl.NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
