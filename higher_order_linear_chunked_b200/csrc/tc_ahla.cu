@@ -117,19 +117,88 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // the carried-in prefix (P^T, E^T) through shared memory: coalesced loads, rows
         // swizzled by 16-byte chunk, then every thread takes its row
         float* stage = reinterpret_cast<float*>(sm + AS_A);   // P^T [64][64] | E^T [64][64]
-        const float4* p4 = reinterpret_cast<const float4*>(slot + S::mat(0));
-        const float4* e4 = reinterpret_cast<const float4*>(slot + S::mat(2));
-        float4 xp[4], xe[4];
+        if (p.fold) {
+            // n = seg * ratio slots: P0^T = sum_l P^T_l and
+            // E0^T = sum_l E^T_l + sum_{m < n-1} P^T_m Dsuf^T(m+1), Dsuf^T(m) = sum_{m <= l < n} D^T_l
+            // (the factored prefix, cross terms grouped by their P factor), while the first
+            // loads are in flight.
+            const int n = seg * p.ratio;
+            const float* sb = p.sums + (size_t)bh * p.NSp * S::size;
+            float* Cs = reinterpret_cast<float*>(sm + AS_ST);  // Dsuf^T [64][64] (the state tile comes later)
+            float* Sm = stage + D * D;                         // P^T_m (the E^T half, for now)
+            const int r = 4 * (tid >> 4), c = 4 * (tid & 15);  // this thread's 4 x 4 of E0^T
+            float racc[4][4];
+            float4 sacc[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            xp[i] = p4[tid + ANT * i];
-            xe[i] = e4[tid + ANT * i];
-        }
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int f = tid + ANT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
-            reinterpret_cast<float4*>(stage)[rr * 16 + ch] = xp[i];
-            reinterpret_cast<float4*>(stage + D * D)[rr * 16 + ch] = xe[i];
+                for (int b = 0; b < 4; ++b) racc[a][b] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int l = 0; l < n; ++l) {
+                const float* sl = sb + (size_t)l * S::size;
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const float4 x = *reinterpret_cast<const float4*>(sl + S::mat(2) + (r + a) * D + c);
+                    racc[a][0] += x.x; racc[a][1] += x.y; racc[a][2] += x.z; racc[a][3] += x.w;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 x = reinterpret_cast<const float4*>(sl + S::mat(0))[tid + ANT * i];
+                    sacc[i] = make_float4(sacc[i].x + x.x, sacc[i].y + x.y, sacc[i].z + x.z, sacc[i].w + x.w);
+                }
+            }
+            for (int m = n - 2; m >= 0; --m) {
+                const float* cl = sb + (size_t)(m + 1) * S::size;
+                const float* smp = sb + (size_t)m * S::size;
+                for (int f = tid; f < D * D / 4; f += ANT) {
+                    const float4 x = reinterpret_cast<const float4*>(cl + S::mat(1))[f];
+                    const float4 o = m == n - 2 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<float4*>(Cs)[f];
+                    reinterpret_cast<float4*>(Cs)[f] = make_float4(o.x + x.x, o.y + x.y, o.z + x.z, o.w + x.w);
+                    reinterpret_cast<float4*>(Sm)[f] = reinterpret_cast<const float4*>(smp + S::mat(0))[f];
+                }
+                __syncthreads();
+#pragma unroll 8
+                for (int k = 0; k < D; ++k) {
+                    const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const float sv = Sm[(r + a) * D + k];
+                        racc[a][0] = fmaf(sv, cv.x, racc[a][0]);
+                        racc[a][1] = fmaf(sv, cv.y, racc[a][1]);
+                        racc[a][2] = fmaf(sv, cv.z, racc[a][2]);
+                        racc[a][3] = fmaf(sv, cv.w, racc[a][3]);
+                    }
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int f = tid + ANT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
+                reinterpret_cast<float4*>(stage)[rr * 16 + ch] = sacc[i];
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int i = r + a, j = c + b;
+                    stage[D * D + i * D + ((((j >> 2) ^ (i & 7)) << 2) | (j & 3))] = racc[a][b];
+                }
+        } else {
+            const float4* p4 = reinterpret_cast<const float4*>(slot + S::mat(0));
+            const float4* e4 = reinterpret_cast<const float4*>(slot + S::mat(2));
+            float4 xp[4], xe[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                xp[i] = p4[tid + ANT * i];
+                xe[i] = e4[tid + ANT * i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int f = tid + ANT * i, rr = f >> 4, ch = (f & 15) ^ (rr & 7);
+                reinterpret_cast<float4*>(stage)[rr * 16 + ch] = xp[i];
+                reinterpret_cast<float4*>(stage + D * D)[rr * 16 + ch] = xe[i];
+            }
         }
         __syncthreads();
         const int r = row & 63;
@@ -337,9 +406,9 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
+    prm.fold = pl.NSf + 1 <= PH_MAX ? 1 : 0;  // few slots: each output CTA folds its own prefix
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
-    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1;
-    prm.fold = sprm.fold = 0;
+    sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k_ahla_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ASMEM_BYTES)) != cudaSuccess)
@@ -351,7 +420,7 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if ((e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

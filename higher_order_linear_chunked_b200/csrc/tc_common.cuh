@@ -117,9 +117,11 @@ struct Plan {
 // head, in segments short enough to fill the machine.
 Plan plan(int BH, int T, int slots);
 
+// Up to this many summary slots per head, an output walker folds its prefix itself.
+constexpr int PH_MAX = 9;
+
 // Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for
-// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  One launch for up to
-// nine slots per head, two beyond.
+// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st);
 
 // The decayed second-order forward, chunk-parallel (tc_decay.cu).

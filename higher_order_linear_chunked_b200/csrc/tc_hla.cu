@@ -667,86 +667,6 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_sum(float* __restrict__ pre, i
     }
 }
 
-// The same prefixes for a head with few summary slots, in one launch: one CTA per head folds
-// the slots in order, writing each exclusive prefix before adding the slot's summary
-// (R0 += R_l + S0 C_l, r0 += r_l + S0 m_l, then S0 += S_l, m0 += m_l).
-constexpr int PH_MAX = 9;    // slots handled this way
-__global__ void __launch_bounds__(PX_NT) k_prefix_head(const float* __restrict__ sums, float* __restrict__ pre,
-                                                       int NS, int NSp) {
-    using S = simt_layout;
-    __shared__ __align__(16) float S0s[D * (D + 4)];   // running S0, padded rows
-    __shared__ __align__(16) float Cs[D * D];
-    __shared__ float ms[D];
-    const int bh = blockIdx.x, tid = threadIdx.x;
-    const float* sb = sums + (size_t)bh * NSp * S::size;
-    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);   // this thread's 4 x 4 block of R0
-    float racc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) racc[a][b] = 0.f;
-    float m0 = 0.f, r0 = 0.f;                           // thread tid < D: element tid
-    for (int e = tid; e < D * (D + 4); e += PX_NT) S0s[e] = 0.f;
-    __syncthreads();
-    for (int l = 0; l < NS; ++l) {
-        float* out = pre + ((size_t)bh * NSp + l) * S::size;
-        // the exclusive prefix at l
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int f = tid + PX_NT * i, rr = f >> 4, c4 = f & 15;
-            reinterpret_cast<float4*>(out + S::mat(0))[f] = *reinterpret_cast<const float4*>(S0s + rr * (D + 4) + 4 * c4);
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-            *reinterpret_cast<float4*>(out + S::mat(2) + (r + a) * D + c) =
-                make_float4(racc[a][0], racc[a][1], racc[a][2], racc[a][3]);
-        if (tid < D) {
-            out[S::vec(0) + tid] = m0;
-            out[S::vec(1) + tid] = r0;
-        }
-        if (l + 1 == NS) break;
-        // fold slot l
-        const float* sl = sb + (size_t)l * S::size;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) reinterpret_cast<float4*>(Cs)[tid + PX_NT * i] = reinterpret_cast<const float4*>(sl + S::mat(1))[tid + PX_NT * i];
-        if (tid < D) ms[tid] = sl[S::vec(0) + tid];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const float4 x = *reinterpret_cast<const float4*>(sl + S::mat(2) + (r + a) * D + c);
-            racc[a][0] += x.x; racc[a][1] += x.y; racc[a][2] += x.z; racc[a][3] += x.w;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) {
-            const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const float sv = S0s[(r + a) * (D + 4) + k];
-                racc[a][0] = fmaf(sv, cv.x, racc[a][0]);
-                racc[a][1] = fmaf(sv, cv.y, racc[a][1]);
-                racc[a][2] = fmaf(sv, cv.z, racc[a][2]);
-                racc[a][3] = fmaf(sv, cv.w, racc[a][3]);
-            }
-        }
-        if (tid < D) {
-            float y = sl[S::vec(1) + tid];
-            for (int k = 0; k < D; ++k) y = fmaf(S0s[tid * (D + 4) + k], ms[k], y);
-            r0 += y;
-            m0 += ms[tid];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int f = tid + PX_NT * i, rr = f >> 4, c4 = f & 15;
-            const float4 x = reinterpret_cast<const float4*>(sl + S::mat(0))[f];
-            float4* d = reinterpret_cast<float4*>(S0s + rr * (D + 4) + 4 * c4);
-            const float4 o = *d;
-            *d = make_float4(o.x + x.x, o.y + x.y, o.z + x.z, o.w + x.w);
-        }
-        __syncthreads();
-    }
-}
-
 // ---------------------------------------------------------------- host side
 namespace {
 
@@ -845,10 +765,6 @@ Plan plan(int BH, int T, int slots) {
 }
 
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st) {
-    if (NS <= PH_MAX) {
-        k_prefix_head<<<BH, PX_NT, 0, st>>>(sums, pre, NS, NSp);
-        return cudaGetLastError();
-    }
     k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -876,11 +792,10 @@ size_t workspace_bytes(int op, bool /*norm*/, int BH, int T) {
 
 int kernel_launches(int op, bool /*norm*/, int BH, int T) {
     if (op == OP_HLA2D) return decay_kernel_launches();
-    // summary walk, the prefix (second order up to PH_MAX slots per head: folded into the output
-    // walk; AHLA: one launch up to PH_MAX slots, else two), output walk
+    // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
+    // two launches), output walk
     const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm() * kSMs : kSMs);
-    if (pl.NSf + 1 > PH_MAX) return 4;
-    return op == OP_AHLA ? 3 : 2;            // second order: the output walker folds the prefix
+    return pl.NSf + 1 > PH_MAX ? 4 : 2;     // else the output walker folds the prefix itself
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,

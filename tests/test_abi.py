@@ -78,12 +78,11 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert use(hla.OP_HLA2, bf16, 0, d=32) == 0
     assert use(hla.OP_HLA3, bf16, 0) == 0
     assert use(hla.OP_HLA2_NORM, bf16, 1) == 0
-    # launches per forward: summary walker, the prefix (with up to nine summary slots per
-    # head: folded into the second-order output walker, one kernel for AHLA; else two
-    # kernels), output walker; the decayed path has chunk summaries, three prefix kernels and
-    # the output kernel
+    # launches per forward: summary walker, the prefix (with up to nine summary slots per head
+    # folded into the output walker; else two kernels), output walker; the decayed path has
+    # chunk summaries, three prefix kernels and the output kernel
     assert launches(hla.OP_HLA2_NORM, bf16, 0) == 2   # the output walker folds the prefix
-    assert launches(hla.OP_AHLA, bf16, 0) == 3
+    assert launches(hla.OP_AHLA, bf16, 0) == 2
     assert lib.hla_kernel_launches(hla.OP_HLA2_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 4   # many slots
     assert launches(hla.OP_HLA2, bf16, 1) == 5
     # decayed workspace: 256 B status block + one 4 x 64 x 64 fp32 slot per 128-token chunk
