@@ -1,25 +1,29 @@
 // tcgen05 tensor-core path for the second-order masked HLA forward (bf16 inputs, d = dv = 64).
 //
 // "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 1 and 4.
-// The sequence of each head is cut into segments of NCH chunks of c = 128 tokens.
+// The sequence of each head is cut into output segments of NCH chunks of c = 128 tokens;
+// the chunks before the last output segment are also cut into summary segments of NCHs
+// chunks (see plan()).
 //
-//  1. k_walk<SUMMARY>: one CTA per (segment, head) walks its chunks from the zero
+//  1. k_walk<SUMMARY>: one CTA per (summary segment, head) walks its chunks from the zero
 //     state and writes the segment summary (S, C, m, R = S C - G, r = S m - h) in fp32.
-//  2. k_prefix_cross + k_prefix_sum: the exclusive prefix of the segment summaries under
-//     the semidirect-product combine, in its factored form (see "segment prefixes").
-//  3. k_walk<OUTPUT>: one CTA per (segment, head) starts from its prefix and walks its
-//     chunks again, emitting o for every token and carrying (S, R, r) to the next chunk.
+//  2. The exclusive prefix of the summaries under the semidirect-product combine, in its
+//     factored form (see "segment prefixes"): folded by each output CTA in its prologue when
+//     a head has few summary slots, else k_prefix_cross + k_prefix_sum.
+//  3. k_walk<OUTPUT>: one CTA per (output segment, head) starts from its prefix and walks
+//     its chunks again, emitting o for every token and carrying (S, R, r) to the next chunk.
 //
 // Per chunk (Q, K, V: 128 x 64 tiles; S0, R0, r0: state carried into the chunk):
 //     A  = L (.) (Q K^T)                         (tcgen05, M=128 N=128 K=64)
 //     P  = Q S0                                  (M=128 N=64  K=64)
 //     W  = L (.) (P Q^T + A A^T)                 (M=128 N=128 K=64+128)
-//     O  = Q [R0 | r0] + W V,  den = q.r0 + W 1  (M=128 N=80 K=64; N=64 K=128)
+//     O  = Q [R0 | r0] + W [V | 1]               (M=128 N=80 K=64; N=80 K=128; column 64: den)
 //     Z  = P + A K        (Z_j = S_j q_j, S_j the key moment up to token j)
 //     S0 += K^T K;  [R0 | r0] += Z^T [V | 1]      (stacked M=128 MN-major operands)
 // The tensor-core state lives in TMEM (fp32) across the walk; its bf16 copies feed
 // the next chunk's MMAs.  TMA stages Q, K, V (128B swizzle, no multicast), double
-// buffered; one thread issues TMA and MMA; four warps run the TMEM epilogues.
+// buffered; one warp issues TMA and MMA; eight warps run the TMEM epilogues; O leaves
+// through shared memory by TMA bulk tensor stores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
