@@ -1,0 +1,310 @@
+"""The chunk algebra of the tensor-core kernels, checked in fp64 on the CPU.
+
+The CUDA kernels do not run the token recurrence; they run a rewritten form of it:
+per-chunk matrix products, segment summaries and factored prefixes.  The GPU parity
+tests check the end result; these tests check each rewrite on its own, in fp64,
+against the oracle's serial recurrence and its semidirect-product combine maps, so a
+derivation error (a dropped cross term, a wrong decay exponent, a transposed
+operand) shows up here, away from bf16 rounding.  Every emulation below restates the
+formulas written in the header comments of the kernel sources; none of them calls
+into the CUDA path.
+
+Sources: "Higher-order Linear Attention" summary (gist.science 2510.27258),
+Metodología 1 (second-order state, ratio normalisation), Metodología 2 (AHLA),
+Metodología 4 (chunked, scan-parallel evaluation), Contribuciones 2 (decay).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.segments as seg
+
+EPS = 1e-6
+
+
+def rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+def rand_head(T, d, dv, seed):
+    rng = np.random.default_rng(seed)
+    s = 1.0 / np.sqrt(d)
+    q = rng.standard_normal((T, d)) * s
+    k = rng.standard_normal((T, d)) * s
+    v = rng.standard_normal((T, dv))
+    return q, k, v
+
+
+def chunks(x, c):
+    """Zero-pad the token axis to whole chunks of c and split; zero tokens add nothing."""
+    T = x.shape[0]
+    n = -(-T // c)
+    xp = np.vstack([x, np.zeros((n * c - T, x.shape[1]))])
+    return [xp[i * c:(i + 1) * c] for i in range(n)]
+
+
+def recur(op, q, k, v, gamma=None):
+    g = None if gamma is None else np.array([gamma])
+    return oracle.recur(op, q[None, None], k[None, None], v[None, None], gamma=g, eps=EPS)[0, 0]
+
+
+# ---------------------------------------------------------------------------
+# second order, undecayed: the walker's per-chunk step (R-form state)
+# ---------------------------------------------------------------------------
+
+def hla2_chunk(Q, K, V1, S0, R0):
+    """One chunk of the second-order walker.  V1 = [V | 1] for the normalised form.
+
+    State carried in: S0 (key moment) and R0 = S0 C0 - G0 (with r0 as its last column
+    when V1 carries the ones column).  Returns (O, S0', R0')."""
+    c = Q.shape[0]
+    L = np.tril(np.ones((c, c)))
+    A = L * (Q @ K.T)
+    P = Q @ S0
+    W = L * (P @ Q.T + A @ A.T)
+    O = Q @ R0 + W @ V1
+    Z = P + A @ K                     # row j: S_j q_j
+    return O, S0 + K.T @ K, R0 + Z.T @ V1
+
+
+def hla2_walk(q, k, v, c, normalized, S0=None, R0=None):
+    d, dv = q.shape[1], v.shape[1] + (1 if normalized else 0)
+    S0 = np.zeros((d, d)) if S0 is None else S0
+    R0 = np.zeros((d, dv)) if R0 is None else R0
+    outs = []
+    for Q, K, V in zip(chunks(q, c), chunks(k, c), chunks(v, c)):
+        V1 = np.hstack([V, np.ones((V.shape[0], 1))]) if normalized else V
+        O, S0, R0 = hla2_chunk(Q, K, V1, S0, R0)
+        outs.append(O)
+    O = np.vstack(outs)[:q.shape[0]]
+    if normalized:
+        O = O[:, :-1] / (O[:, -1:] + EPS)
+    return O, S0, R0
+
+
+@pytest.mark.parametrize("normalized", [False, True])
+@pytest.mark.parametrize("T,c", [(1, 8), (7, 8), (8, 8), (37, 8), (64, 16), (100, 32)])
+def test_hla2_chunk_step_matches_recurrence(T, c, normalized):
+    q, k, v = rand_head(T, 5, 3, seed=T * 7 + c)
+    if normalized:
+        k = np.abs(k)                 # keep the denominator away from zero
+        q = np.abs(q)
+    O, _, _ = hla2_walk(q, k, v, c, normalized)
+    ref = recur("hla2n" if normalized else "hla2", q, k, v)
+    assert rel(O, ref) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# segment prefixes: the factored forms against the exclusive fold of the combine
+# ---------------------------------------------------------------------------
+
+def r_form(s):
+    """(S, C, m, R = S C - G, r = S m - h) of an oracle second-order summary."""
+    return dict(S=s["S"], C=s["C"], m=s["m"], R=s["S"] @ s["C"] - s["G"], r=s["S"] @ s["m"] - s["h"])
+
+
+def prefix_cross_sum(slots):
+    """The two-kernel form: Y_l = R_l + S0(l) C_l, then R0(n) = sum_{l<n} Y_l."""
+    out, S0, R0, r0 = [], 0.0 * slots[0]["S"], 0.0 * slots[0]["R"], 0.0 * slots[0]["r"]
+    for s in slots:
+        out.append(dict(S=S0, R=R0, r=r0))
+        R0 = R0 + s["R"] + S0 @ s["C"]
+        r0 = r0 + s["r"] + S0 @ s["m"]
+        S0 = S0 + s["S"]
+    return out
+
+
+def prefix_fold(slots, n):
+    """The in-prologue fold for the prefix of slots 0..n-1: plain sums of S, R, r plus the
+    cross terms sum_{m<n-1} S_m Csuf(m+1), Csuf(m+1) = sum_{m<l<n} C_l (likewise m)."""
+    S0 = sum((s["S"] for s in slots[:n]), 0.0 * slots[0]["S"])
+    R0 = sum((s["R"] for s in slots[:n]), 0.0 * slots[0]["R"])
+    r0 = sum((s["r"] for s in slots[:n]), 0.0 * slots[0]["r"])
+    Csuf, msuf = 0.0 * slots[0]["C"], 0.0 * slots[0]["m"]
+    for m in range(n - 2, -1, -1):
+        Csuf = Csuf + slots[m + 1]["C"]
+        msuf = msuf + slots[m + 1]["m"]
+        R0 = R0 + slots[m]["S"] @ Csuf
+        r0 = r0 + slots[m]["S"] @ msuf
+    return dict(S=S0, R=R0, r=r0)
+
+
+@pytest.mark.parametrize("lengths", [[5], [3, 9, 1], [8, 8, 8, 8, 8], [1, 2, 3, 4, 5, 6, 7]])
+def test_factored_prefixes_equal_the_combine_fold(lengths):
+    T, d, dv = sum(lengths), 4, 3
+    q, k, v = rand_head(T, d, dv, seed=len(lengths))
+    b = seg.split_points(T, lengths)
+    sums = [seg.hla2_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]]) for i in range(len(lengths))]
+    ref = seg.fold_exclusive(sums, seg.hla2_combine, seg.hla2_identity(d, dv))
+    slots = [r_form(s) for s in sums]
+    two_kernel = prefix_cross_sum(slots)
+    for n in range(len(lengths)):
+        want = r_form(ref[n])
+        folded = prefix_fold(slots, n)
+        for key in ("S", "R", "r"):
+            np.testing.assert_allclose(two_kernel[n][key], want[key], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(folded[key], want[key], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("normalized", [False, True])
+@pytest.mark.parametrize("T,c,NCH,ratio", [(200, 8, 5, 1), (200, 8, 6, 3), (129, 16, 2, 2), (70, 8, 9, 1)])
+def test_segment_plan_matches_recurrence(T, c, NCH, ratio, normalized):
+    """Summary segments of NCH/ratio chunks walked from zero, their prefix, then output
+    segments of NCH chunks walked from that prefix: the three kernel stages end to end."""
+    d, dv = 4, 3
+    q, k, v = rand_head(T, d, dv, seed=T + NCH)
+    if normalized:
+        q, k = np.abs(q), np.abs(k)
+    nchunks = -(-T // c)
+    NCHs = NCH // ratio
+    seg_tok = NCHs * c
+    n_out = -(-nchunks // NCH)
+    n_sum = (n_out - 1) * ratio      # only the chunks before the last output segment
+    slots = []
+    for i in range(n_sum):
+        sl = slice(i * seg_tok, (i + 1) * seg_tok)
+        _, S, R = hla2_walk(q[sl], k[sl], v[sl], c, normalized)
+        slots.append(dict(S=S, C=q[sl].T @ v[sl], m=q[sl].sum(0), R=R[:, :dv],
+                          r=R[:, dv] if normalized else np.zeros(d)))
+    outs = []
+    for n in range(n_out):
+        if n == 0:
+            S0, R0, r0 = np.zeros((d, d)), np.zeros((d, dv)), np.zeros(d)
+        else:
+            p = prefix_fold(slots, n * ratio)
+            S0, R0, r0 = p["S"], p["R"], p["r"]
+        R0 = np.hstack([R0, r0[:, None]]) if normalized else R0
+        sl = slice(n * NCH * c, min((n + 1) * NCH * c, T))
+        O, _, _ = hla2_walk(q[sl], k[sl], v[sl], c, normalized, S0=S0, R0=R0)
+        outs.append(O)
+    ref = recur("hla2n" if normalized else "hla2", q, k, v)
+    assert rel(np.vstack(outs), ref) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# AHLA: the walker's chunk step and the transposed summary slot
+# ---------------------------------------------------------------------------
+
+def ahla_walk(q, k, v, c, P0=None, E0=None):
+    d, dv = q.shape[1], v.shape[1]
+    P0 = np.zeros((d, dv)) if P0 is None else P0
+    E0 = np.zeros((d, dv)) if E0 is None else E0
+    outs = []
+    for Q, K, V in zip(chunks(q, c), chunks(k, c), chunks(v, c)):
+        A = np.tril(Q @ K.T)
+        Y = Q @ P0 + A @ V            # row s: q_s^T P_s
+        outs.append(Q @ E0 + A @ Y)
+        P0 = P0 + K.T @ V
+        E0 = E0 + K.T @ Y
+    return np.vstack(outs)[:q.shape[0]], P0, E0
+
+
+@pytest.mark.parametrize("T,c", [(1, 8), (13, 8), (64, 16), (99, 32)])
+def test_ahla_chunk_step_matches_recurrence(T, c):
+    q, k, v = rand_head(T, 5, 3, seed=T + 1000)
+    O, _, _ = ahla_walk(q, k, v, c)
+    assert rel(O, recur("ahla", q, k, v)) < 1e-12
+
+
+@pytest.mark.parametrize("lengths", [[4, 4], [3, 9, 1, 6], [8, 8, 8, 8, 8, 8]])
+def test_ahla_transposed_slot_uses_the_second_order_prefix(lengths):
+    """(P^T, D^T, E^T) in the places of (S, C, R): the second-order factored prefix of the
+    transposed slots is the transpose of the AHLA combine fold."""
+    T, d, dv = sum(lengths), 5, 3
+    q, k, v = rand_head(T, d, dv, seed=77 + len(lengths))
+    b = seg.split_points(T, lengths)
+    sums = [seg.ahla_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]]) for i in range(len(lengths))]
+    ref = seg.fold_exclusive(sums, seg.ahla_combine, seg.ahla_identity(d, dv))
+    slots = [dict(S=s["P"].T, C=s["D"].T, m=np.zeros(d), R=s["E"].T, r=np.zeros(dv)) for s in sums]
+    two_kernel = prefix_cross_sum(slots)
+    for n in range(len(lengths)):
+        folded = prefix_fold(slots, n)
+        for got in (two_kernel[n], folded):
+            np.testing.assert_allclose(got["S"], ref[n]["P"].T, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(got["R"], ref[n]["E"].T, rtol=0, atol=1e-12)
+
+
+def test_ahla_segment_plan_matches_recurrence():
+    T, c, NCH, d, dv = 150, 8, 4, 4, 3
+    q, k, v = rand_head(T, d, dv, seed=5)
+    seg_tok = NCH * c
+    n_out = -(-T // seg_tok)
+    slots = []
+    for i in range(n_out - 1):
+        sl = slice(i * seg_tok, (i + 1) * seg_tok)
+        _, P, E = ahla_walk(q[sl], k[sl], v[sl], c)
+        slots.append(dict(S=P.T, C=(k[sl].T @ q[sl]).T, m=np.zeros(d), R=E.T, r=np.zeros(dv)))
+    outs = []
+    for n in range(n_out):
+        P0, E0 = np.zeros((d, dv)), np.zeros((d, dv))
+        if n:
+            p = prefix_fold(slots, n)
+            P0, E0 = p["S"].T, p["R"].T
+        sl = slice(n * seg_tok, min((n + 1) * seg_tok, T))
+        outs.append(ahla_walk(q[sl], k[sl], v[sl], c, P0=P0, E0=E0)[0])
+    assert rel(np.vstack(outs), recur("ahla", q, k, v)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# decayed second order: chunk summaries, prefix recurrences and the output split
+# ---------------------------------------------------------------------------
+
+def decay_forward(q, k, v, g, c, drop=None):
+    """The decay kernels' algebra, chunk by chunk.  ``drop`` zeroes one named term (used
+    only to show that each term is needed)."""
+    T, d = q.shape
+    tau = np.arange(c)
+    lam = g ** (c - 1 - tau)
+    rho = g ** c
+    Gam = g ** (tau + 1)
+    Dl = tau[:, None] - tau[None, :]
+    Dg = np.where(Dl >= 0, g ** np.maximum(Dl, 0), 0.0)
+    L = (Dl >= 0).astype(float)
+    keep = lambda name, x: 0.0 * x if drop == name else x
+    Qs, Ks, Vs = chunks(q, c), chunks(k, c), chunks(v, c)
+    # k_dec_summary: every chunk from the zero state
+    sums = []
+    for Q, K, V in zip(Qs, Ks, Vs):
+        As = Q @ K.T
+        U = np.triu(As, 1)
+        sums.append(dict(S=K.T @ (lam[:, None] * K), C=Q.T @ (lam[:, None] * V), Khat=K.T @ K,
+                         G=K.T @ (U.T @ (lam[:, None] * V))))
+    # prefix kernels, then k_dec_output
+    dv = v.shape[1]
+    S0, C0, G0 = np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv))
+    outs = []
+    for (Q, K, V), s in zip(zip(Qs, Ks, Vs), sums):
+        As = Q @ K.T
+        A = L * As
+        U = np.triu(As, 1)
+        At = Dg * As
+        H = np.where(Dl > 0, (Dg - 1.0) * As, 0.0)
+        P = Q @ S0
+        W = Dg * (Gam[:, None] * (P @ Q.T) + At @ A.T + keep("HU", H @ U.T))
+        O = W @ V + Gam[:, None] * ((Gam[:, None] * P + keep("HK", H @ K)) @ C0) - keep("QG0", Gam[:, None] * (Q @ G0))
+        outs.append(O)
+        G0 = rho * G0 + s["G"] + keep("KhatC0", rho * s["Khat"] @ C0)
+        S0 = rho * S0 + s["S"]
+        C0 = rho * C0 + s["C"]
+    return np.vstack(outs)[:T]
+
+
+@pytest.mark.parametrize("gamma", [1.0, 0.999, 0.95, 0.5])
+@pytest.mark.parametrize("T,c", [(5, 8), (37, 8), (64, 16), (100, 16)])
+def test_decay_chunk_algebra_matches_recurrence(T, c, gamma):
+    q, k, v = rand_head(T, 4, 3, seed=T + int(gamma * 1000))
+    assert rel(decay_forward(q, k, v, gamma, c), recur("hla2d", q, k, v, gamma=gamma)) < 1e-12
+
+
+def test_decay_gamma_one_reduces_to_the_undecayed_walk():
+    q, k, v = rand_head(61, 4, 3, seed=3)
+    np.testing.assert_allclose(decay_forward(q, k, v, 1.0, 8), hla2_walk(q, k, v, 8, False)[0],
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("term", ["HU", "HK", "QG0", "KhatC0"])
+def test_decay_every_term_is_needed(term):
+    """Removing any one cross term breaks the match: the test above is not vacuous."""
+    q, k, v = rand_head(48, 4, 3, seed=9)
+    ref = recur("hla2d", q, k, v, gamma=0.9)
+    assert rel(decay_forward(q, k, v, 0.9, 16, drop=term), ref) > 1e-3
