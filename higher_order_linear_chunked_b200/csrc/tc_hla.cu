@@ -20,6 +20,10 @@
 //     O  = Q [R0 | r0] + W [V | 1]               (M=128 N=80 K=64; N=80 K=128; column 64: den)
 //     Z  = P + A K        (Z_j = S_j q_j, S_j the key moment up to token j)
 //     S0 += K^T K;  [R0 | r0] += Z^T [V | 1]      (stacked M=128 MN-major operands)
+// W_tj = q_t^T S_j q_j (j <= t) is the pair weight of the masked definition.  It equals
+// q_t . Z_j too, but that dot product of the rounded Z can cancel far below its terms
+// when q and k have mixed signs, while P Q^T + A A^T sums it key by key from the rounded
+// scores, so its rounding error stays relative to the terms of the sum itself.
 // The tensor-core state lives in TMEM (fp32) across the walk; its bf16 copies feed
 // the next chunk's MMAs.  TMA stages Q, K, V (128B swizzle, no multicast), double
 // buffered; one warp issues TMA and MMA; eight warps run the TMEM epilogues; O leaves
@@ -45,9 +49,10 @@ constexpr int ISSUER = NT;         // the issuing thread (lane 0 of warp 8)
 constexpr uint32_t SM_Q0 = 0, SM_Q1 = SM_Q0 + TILE;
 constexpr uint32_t SM_K0 = SM_Q1 + TILE, SM_V0 = SM_K0 + TILE;
 constexpr uint32_t SM_K1 = SM_V0 + TILE, SM_V1 = SM_K1 + TILE;
-constexpr uint32_t SM_Z = SM_V1 + TILE;          // P, then Z  ([tok][feat])
+constexpr uint32_t SM_Z = SM_V1 + TILE;          // Z  ([tok][feat])
 constexpr uint32_t SM_ONES = SM_Z + TILE;        // MN-major [tok][64], column 0 = 1
-constexpr uint32_t SM_A = SM_ONES + TILE;        // A, then W: [128][128] K-major (2 atoms)
+constexpr uint32_t SM_A = SM_ONES + TILE;        // output: masked A [128][128] K-major (2 atoms);
+                                                 // set-up: the carried-in state, fp32 S | R
 constexpr uint32_t SM_S0 = SM_A + 2 * TILE;      // S0^T: [64 n][64 k] K-major
 constexpr uint32_t SM_R0 = SM_S0 + 64 * 128;     // [R0 | r0]^T: [80 n][64 k] K-major
 constexpr uint32_t SM_OST = SM_R0 + 80 * 128;    // O staging: two [128][32] fp32 TMA boxes
@@ -56,33 +61,46 @@ constexpr uint32_t SM_TOTAL = SM_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SM_TOTAL + 1024; // + alignment slack
 
 // TMEM columns (fp32 accumulators, 128 lanes).
-constexpr uint32_t TM_A = 0;      // A, then W            (128 cols)
+constexpr uint32_t TM_A = 0;      // A; output walk: then W (128 cols)
 constexpr uint32_t TM_P = 128;    // P, then Z            (64)
-constexpr uint32_t TM_O0 = 192;   // O | q.r0, even chunks (80)
+constexpr uint32_t TM_O = 192;    // output: [O | den]    (80)
 constexpr uint32_t TM_CR = 272;   // summary: lanes 0-63 [C|m], lanes 64-127 [R|r]  (80)
                                   // output: lanes 0-63 R^T, lane 64 r^T, rest 0   (64)
 constexpr uint32_t TM_S = 352;    // lanes 0-63 S         (64)
-constexpr uint32_t TM_O1 = 416;   // O | q.r0, odd chunks  (80)
+constexpr uint32_t TM_W = 416;    // summary: masked A; output: masked W; as bf16 pairs, the A
+                                  // operand of K-step s (16 tokens) at TM_W + 8 s  (64)
+constexpr uint32_t TM_PP = 480;   // output: P as bf16 pairs  (32)
 constexpr uint32_t TM_COLS = 512;
 
 enum Mode { SUMMARY = 0, OUTPUT = 1 };
 
 // ---------------------------------------------------------------- the walker
 // Threads: 8 epilogue warps and one issuing warp.  Epilogue warp w reads TMEM lane
-// quadrant (w & 3), i.e. tile rows 32 (w & 3) .. + 31, and handles half (w >> 2) of
-// each tile's columns.  Lane 0 of warp 8 issues the TMA loads and the MMAs, so the
-// epilogue warps never wait for an issue in progress.
+// quadrant (w & 3), i.e. tile rows 32 (w & 3) .. + 31 (the hardware ties a warp to the
+// quadrant w mod 4, and so to one SM sub-partition), and handles half (w >> 2) of each
+// tile's columns.  Lane 0 of warp 8 issues the TMA loads and the MMAs, so the epilogue
+// warps never wait for an issue in progress.
 //
-// Rounds of MMAs per chunk n, each followed by an epilogue:
-//   R1(n): A = Q K^T, P = Q S0                      -> E1(n): A, P to bf16 tiles
-//   R2(n): W = P Q^T + A A^T, Z = P + A K,
-//          S += K^T K, O[n&1] = Q [R0|r0]^T         -> E2(n): W, Z, S0 to bf16 tiles
-//   R3(n): [O|den][n&1] += W [V|1],
-//          summary: [C|m ; R|r] += [Q^T;Z^T][V|1]
-//          output:  [R^T ; r^T] += [V^T ; 1^T] Z    -> E3(n): [R0|r0]^T; O[n&1] to HBM
-// R3(n) and R1(n+1) are issued together and their epilogues run together.  The O
-// accumulator is double buffered in TMEM, so the store of O(n) to HBM runs while
-// the tensor core works on R2(n+1).
+// Summary walk, rounds of MMAs per chunk n, each followed by an epilogue:
+//   R1(n): A = Q K^T, P = Q S0                      -> E1(n): A to a bf16 tile
+//   R2(n): Z = P + A K, S += K^T K                  -> E2(n): Z, S0 to bf16 tiles
+//   R3(n): [C|m ; R|r] += [Q^T;Z^T][V|1]
+// R3(n) and R1(n+1) are issued together and their epilogues run together.
+//
+// Output walk, per chunk n (products marked * run while an epilogue converts something else):
+//   R1(n): A = Q K^T, P = Q S0              -> E1: A (masked) to a bf16 tile, P to bf16 pairs
+//                                                   in TMEM; [R0|r0]^T tile of chunk n
+//          * S += K^T K
+//   R2(n): W = P Q^T + A A^T, Z = P + A K   -> E2: W (masked) to bf16 pairs in TMEM; Z, S0 to
+//          (P read from TMEM)                      bf16 tiles
+//          * O = Q [R0|r0]^T
+//   R3(n): [O|den] += W [V|1] (W read from TMEM), [R^T ; r^T] += [V^T ; 1^T] Z
+// with R3(n) and R1(n+1) issued together.  Blocks above the diagonal of the masked A tile
+// and of the masked pairs in TMEM are zeroed once.  The 32 x 32 blocks that the mask keeps
+// and the other conversions are spread so that no warp does more than three 32-column
+// pieces in one epilogue: a warp pair on one quadrant shares that sub-partition's issue
+// slots, and quadrant 3 holds the longest rows.  O(n-1) leaves TMEM while R2(n) runs, and
+// HBM by TMA stores.
 template <int MODE>
 __global__ void __launch_bounds__(NTH, 1)
 k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -294,7 +312,17 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
                 if (quad < 2 || lane < 16) st_row16(sm + SM_R0, TILE, quad < 2 ? row : 64 + lane, c0, v);
             }
         }
-        if (MODE == OUTPUT) ptx::tmem_st_wait();
+        {
+            // The 32 x 32 blocks of the masked A (and W) above the diagonal (token block b of a
+            // row in quadrant q < b) are zero in every chunk: written once, here.
+            uint32_t z[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                if (2 * half + j > quad) ptx::tmem_st16u(tmem + lane_base + TM_W + 16 * (2 * half + j), z);
+            ptx::tmem_st_wait();
+        }
     }
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
@@ -317,27 +345,33 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     auto bufK = [&](int n) { return sbase + ((n & 1) ? SM_K1 : SM_K0); };
     auto bufV = [&](int n) { return sbase + ((n & 1) ? SM_V1 : SM_V0); };
     const uint64_t dS0 = kdesc(sbase + SM_S0, 0), dR0 = kdesc(sbase + SM_R0, 0);
-    const uint64_t dZk = kdesc(sbase + SM_Z, 0), dA2 = kdesc2(sbase + SM_A, 0);
+    const uint64_t dA2 = kdesc2(sbase + SM_A, 0);
     const uint64_t dZm = mdesc(sbase + SM_Z, TILE, 0);
-    auto tm_o = [&](int n) { return tmem + ((n & 1) ? TM_O1 : TM_O0); };
 
     auto issue_r1 = [&](int n) {             // A = Q K^T, P = Q S0
         const uint64_t dQ = kdesc(bufQ(n), 0), dK = kdesc(bufK(n), 0);
         for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_A, k1(dQ, s), k1(dK, s), I_QK, s > 0);
         for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_P, k1(dQ, s), k1(dS0, s), I_N64_KK, s > 0);
     };
-    auto issue_r2 = [&](int n) {             // W, O = Q [R0|r0]^T, Z, S
+    auto issue_s = [&](int n) {              // S += K^T K (rows 0-63 of [K^T ; V^T] K)
         const uint32_t sK = bufK(n), sV = bufV(n);
-        const uint64_t dQ = kdesc(bufQ(n), 0);
         const uint64_t dKm = mdesc(sK, TILE, 0), dKV = mdesc(sK, sV - sK, 0);
-        if (MODE == OUTPUT) {
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_A, k1(dZk, s), k1(dQ, s), I_QK, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_A, k2(dA2, s), k2(dA2, s), I_QK, 1);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tm_o(n), k1(dQ, s), k1(dR0, s), I_N80_KK, s > 0);
-        }
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_P, k2(dA2, s), mn(dKm, s), I_N64_KM, 1);
         for (int s = 0; s < 8; ++s)
             ptx::umma_bf16(tmem + TM_S, mn(dKV, s), mn(dKm, s), I_N64_MM, (MODE == OUTPUT || n > 0 || s > 0) ? 1u : 0u);
+    };
+    auto issue_z = [&](int n) {              // summary: Z = P + A K, masked A read from TMEM as bf16 pairs
+        const uint64_t dKm = mdesc(bufK(n), TILE, 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TM_P, tmem + TM_W + 8 * s, mn(dKm, s), I_N64_KM, 1);
+    };
+    auto issue_wz = [&](int n) {             // output: W = P Q^T + A A^T, Z = P + A K (A from the bf16 tile)
+        const uint64_t dQ = kdesc(bufQ(n), 0), dKm = mdesc(bufK(n), TILE, 0);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16_ts(tmem + TM_A, tmem + TM_PP + 8 * s, k1(dQ, s), I_QK, s > 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_A, k2(dA2, s), k2(dA2, s), I_QK, 1);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_P, k2(dA2, s), mn(dKm, s), I_N64_KM, 1);
+    };
+    auto issue_qr0 = [&](int n) {            // [O | q.r0] = Q [R0|r0]^T
+        const uint64_t dQ = kdesc(bufQ(n), 0);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TM_O, k1(dQ, s), k1(dR0, s), I_N80_KK, s > 0);
     };
     auto issue_r3 = [&](int n) {             // [O | den] += W [V | 1] ; [C|m ; R|r] += [Q^T ; Z^T] [V | 1]
         const uint32_t sQ = bufQ(n), sV = bufV(n);
@@ -345,7 +379,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         const uint64_t dV1 = mdesc(sV, sbase + SM_ONES - sV, 0);
         if (MODE == OUTPUT) {
             const uint64_t dV1t = mdesc(sV, sbase + SM_ONES - sV, 0);     // stacked [V^T ; 1^T]
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tm_o(n), k2(dA2, s), mn(dV1, s), I_N80_KM, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TM_O, tmem + TM_W + 8 * s, mn(dV1, s), I_N80_KM, 1);
             for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TM_CR, mn(dV1t, s), mn(dZm, s), I_N64_MM, 1);
         } else {
             for (int s = 0; s < 8; ++s)
@@ -358,6 +392,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     // Thread 0 commits the MMAs issued so far and waits for them (bounded); the block agrees.
     auto commit_wait = [&]() -> bool {
         bool good = true;
+        ptx::tc_fence_before();              // this thread's TMEM reads before MMAs issued after
         if (tid == ISSUER) {
             ptx::umma_commit(bar_mma);
             good = ptx::mbar_wait(bar_mma, mma_phase);
@@ -374,44 +409,68 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tc_fence_after();
     };
 
-    // E1: A (masked) -> SM_A (this thread: columns half*64 .. +63; blocks wholly above the
-    // diagonal are written as zeros); P -> SM_Z (OUTPUT only)
-    auto epi1 = [&]() {
-        float v0[32];
+    // 32 fp32 columns of this lane -> 16 bf16 pairs in TMEM (column 2i in the low half).  On
+    // the diagonal block (diag), the columns past this lane's token are cleared first.
+    auto st_pairs = [&](uint32_t tcol, const float (&x)[32], bool diag) {
+        uint32_t r[16];
+        if (diag) {
 #pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 > quad * 32 + 31) {       // a 32 x 32 block wholly above the diagonal
-                st_row32_zero(sm + SM_A, row, c0);
-                continue;
-            }
-            ptx::tmem_ld32(tmem + lane_base + TM_A + c0, v0);
+            for (int i = 0; i < 16; ++i)
+                r[i] = ptx::pack_bf16(2 * i > lane ? 0.f : x[2 * i], 2 * i + 1 > lane ? 0.f : x[2 * i + 1]);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i > row) v0[i] = 0.f;
-            st_row32(sm + SM_A, row, c0, v0);
+            for (int i = 0; i < 16; ++i) r[i] = ptx::pack_bf16(x[2 * i], x[2 * i + 1]);
         }
-        if (MODE == OUTPUT) {
-            ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v0);
-            st_row32(sm + SM_Z, row, half * 32, v0);
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    // Masked A (summary E1) or masked W (output E2): TM_A (fp32) -> bf16 pairs at TM_W.  Warp
+    // (quad, half) converts its rows' token blocks 2 half and 2 half + 1 where the mask keeps
+    // them (block b <= quad); the blocks above stay the zeros written at set-up.
+    auto epi_mask = [&]() {
+        const int b0 = 2 * half;
+        if (b0 > quad) return;
+        float v0[32], v1[32];
+        if (b0 + 1 <= quad) {
+            ptx::tmem_ld32x2(tmem + lane_base + TM_A + 32 * b0, tmem + lane_base + TM_A + 32 * (b0 + 1), v0, v1);
+            st_pairs(TM_W + 16 * b0, v0, false);
+            st_pairs(TM_W + 16 * (b0 + 1), v1, b0 + 1 == quad);
+        } else {                             // b0 == quad
+            ptx::tmem_ld32(tmem + lane_base + TM_A + 32 * b0, v0);
+            st_pairs(TM_W + 16 * b0, v0, true);
         }
     };
-    // E2: W (masked) -> SM_A; Z -> SM_Z; S -> SM_S0 (by rows: S is symmetric)
-    auto epi2 = [&]() {
+    // Output E1: masked A -> SM_A (the K-major tile that is both operands of
+    // A A^T); blocks above the diagonal stay the zeros of set-up
+    auto epi_a_tile = [&]() {
+        const int b0 = 2 * half;
+        if (b0 > quad) return;
         float v0[32], v1[32];
-        if (MODE == OUTPUT) {
-#pragma unroll
-            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-                if (c0 > quad * 32 + 31) {
-                    st_row32_zero(sm + SM_A, row, c0);
-                    continue;
-                }
-                ptx::tmem_ld32(tmem + lane_base + TM_A + c0, v0);
+        if (b0 + 1 <= quad) {
+            ptx::tmem_ld32x2(tmem + lane_base + TM_A + 32 * b0, tmem + lane_base + TM_A + 32 * (b0 + 1), v0, v1);
+            if (b0 + 1 == quad) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (c0 + i > row) v0[i] = 0.f;
-                st_row32(sm + SM_A, row, c0, v0);
+                    if (i > lane) v1[i] = 0.f;
             }
+            st_row32(sm + SM_A, row, 32 * b0, v0);
+            st_row32(sm + SM_A, row, 32 * (b0 + 1), v1);
+        } else {
+            ptx::tmem_ld32(tmem + lane_base + TM_A + 32 * b0, v0);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (i > lane) v0[i] = 0.f;
+            st_row32(sm + SM_A, row, 32 * b0, v0);
         }
+    };
+    // Output E1: P -> bf16 pairs at TM_PP (this warp: columns half*32 .. +31)
+    auto epi_p_pairs = [&]() {
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v);
+        st_pairs(TM_PP + 16 * half, v, false);
+    };
+    // Summary E2: Z -> SM_Z; S -> SM_S0 (by rows: S is symmetric)
+    auto epi2_sum = [&]() {
+        float v0[32], v1[32];
         if (quad < 2) {
             ptx::tmem_ld32x2(tmem + lane_base + TM_P + half * 32, tmem + lane_base + TM_S + half * 32, v0, v1);
             st_row32(sm + SM_Z, row, half * 32, v0);
@@ -421,19 +480,39 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             st_row32(sm + SM_Z, row, half * 32, v0);
         }
     };
-    // E3, state part (output walk): [R^T ; r^T] rows 0..64 of TM_CR -> [R0|r0]^T tile rows
-    auto epi3_state = [&]() {
-        if (quad == 3) return;
+    // Output E2, beside epi_mask: Z -> SM_Z
+    auto epi2_out = [&]() {
         float v[32];
-        ptx::tmem_ld32(tmem + lane_base + TM_CR + half * 32, v);   // warp-collective
-        if (quad < 2 || lane < 16) st_row32(sm + SM_R0, quad < 2 ? row : 64 + lane, half * 32, v);
+        ptx::tmem_ld32(tmem + lane_base + TM_P + half * 32, v);
+        st_row32(sm + SM_Z, row, half * 32, v);
     };
-    // E3, output part: O rows of chunk n (normalised by column 64, q.r0 + rowsum W) staged
-    // as two [128 rows][32 cols] fp32 boxes in the 128B-swizzled TMA layout
-    auto epi3_out = [&](int n) {
+    // Output E2, beside epi_mask: S -> SM_S0 rows, by the two warps that convert no mask block
+    auto epi_s0 = [&]() {
+        if (half != 1 || quad >= 2) return;
+        float v0[32], v1[32];
+        ptx::tmem_ld32x2(tmem + lane_base + TM_S, tmem + lane_base + TM_S + 32, v0, v1);
+        st_row32(sm + SM_S0, row, 0, v0);
+        st_row32(sm + SM_S0, row, 32, v1);
+    };
+    // Output E1, beside epi_mask: [R^T ; r^T] rows 0..64 of TM_CR -> [R0|r0]^T tile rows
+    // (rows 65..79 stay the zeros of set-up), by the half-1 warps of quadrants 0-2, which
+    // convert at most one mask block.
+    auto epi3_state = [&]() {
+        if (half != 1 || quad == 3) return;
+        float v0[32], v1[32];
+        ptx::tmem_ld32x2(tmem + lane_base + TM_CR, tmem + lane_base + TM_CR + 32, v0, v1);   // warp-collective
+        if (quad < 2 || lane == 0) {
+            const int r = quad < 2 ? row : 64;
+            st_row32(sm + SM_R0, r, 0, v0);
+            st_row32(sm + SM_R0, r, 32, v1);
+        }
+    };
+    // Output: O rows of the last finished chunk (normalised by column 64, q.r0 + rowsum W)
+    // staged as two [128 rows][32 cols] fp32 boxes in the 128B-swizzled TMA layout
+    auto epi3_out = [&]() {
         float v[32];
         float d[16];
-        const uint32_t tmo = tm_o(n) + lane_base;
+        const uint32_t tmo = tmem + TM_O + lane_base;
         ptx::tmem_ld16(tmo + 64, d);
         const float scale = p.norm ? 1.f / (d[0] + p.eps) : 1.f;
         ptx::tmem_ld32(tmo + half * 32, v);
@@ -451,8 +530,25 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
         ptx::tma_store_3d(&to, sm + SM_OST + C * 128, 32, t0, bh);
         ptx::bulk_commit();
     };
+    // Issuing thread: wait for the loads of chunk n + 1, then issue R3(n) and R1(n + 1).
+    auto issue_r3_r1 = [&](int n) -> bool {
+        issue_r3(n);
+        if (n + 1 < nch) {
+            if (!ptx::mbar_wait(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1)) return false;
+            ptx::tc_fence_after();
+            issue_r1(n + 1);
+        }
+        return true;
+    };
 
     // ---- the walk
+    if (MODE == OUTPUT && epi) {
+        // masked-A tile blocks above the diagonal: zero in every chunk (the set-up staging that
+        // shared this space has been read); the first E1's proxy fence publishes them
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            if (2 * half + j > quad) st_row32_zero(sm + SM_A, row, 32 * (2 * half + j));
+    }
     if (tid == ISSUER) {
         ok = ptx::mbar_wait(&bar_load[0], 0);
         if (ok) {
@@ -463,38 +559,52 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     ok = __syncthreads_and(ok) != 0;
     for (int n = 0; n < nch && ok; ++n) {
         if (!commit_wait()) { ok = false; break; }          // R1(n) [+ R3(n-1)] done
-        if (epi) {
-            epi1();
-            if (MODE == OUTPUT && n > 0) epi3_state();
-        }
         if (tid == ISSUER) {
+            issue_s(n);                                     // runs during E1
             if (n >= 1 && n + 1 < nch) issue_load(n + 1);   // buffer freed by R3(n-1)
             if (MODE == OUTPUT) ptx::bulk_wait_read();     // the O staging is free again
         }
-        sync_for_mma();
-        if (tid == ISSUER) issue_r2(n);
-        if (MODE == OUTPUT && n > 0 && epi) epi3_out(n - 1);   // overlaps R2(n)
-        if (!commit_wait()) { ok = false; break; }          // R2(n) done
-        if (MODE == OUTPUT && n > 0 && tid == ISSUER) store_o(n - 1);
-        if (epi) epi2();
+        if (epi) {
+            if (MODE == OUTPUT) {
+                epi_a_tile();
+                epi_p_pairs();
+                if (n > 0) epi3_state();
+            } else {
+                epi_mask();
+            }
+            ptx::tmem_st_wait();
+        }
         sync_for_mma();
         if (tid == ISSUER) {
-            issue_r3(n);
-            if (n + 1 < nch) {
-                ok = ptx::mbar_wait(&bar_load[(n + 1) & 1], ((n + 1) >> 1) & 1);
-                if (ok) {
-                    ptx::tc_fence_after();
-                    issue_r1(n + 1);
-                }
-            }
+            if (MODE == OUTPUT) issue_wz(n);
+            else issue_z(n);
         }
+        if (MODE == OUTPUT) {
+            if (n > 0 && epi) epi3_out();                   // O(n-1), while W(n), Z(n) run
+            if (!commit_wait()) { ok = false; break; }      // W(n), Z(n) and S done
+            if (tid == ISSUER) {
+                if (n > 0) store_o(n - 1);
+                issue_qr0(n);                               // runs during E2
+            }
+            if (epi) {
+                epi_mask();
+                epi2_out();
+                epi_s0();
+                ptx::tmem_st_wait();
+            }
+        } else {
+            if (!commit_wait()) { ok = false; break; }      // Z(n) and S done
+            if (epi) epi2_sum();
+        }
+        sync_for_mma();
+        if (tid == ISSUER) ok = issue_r3_r1(n);
         ok = __syncthreads_and(ok) != 0;
     }
     if (ok) {
         if (MODE == OUTPUT && tid == ISSUER) ptx::bulk_wait_read();
         ok = commit_wait();                                  // R3(last) done
         if (ok && MODE == OUTPUT) {
-            if (epi) epi3_out(nch - 1);
+            if (epi) epi3_out();
             __syncthreads();
             if (tid == ISSUER) store_o(nch - 1);
         }

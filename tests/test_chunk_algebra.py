@@ -61,7 +61,7 @@ def hla2_chunk(Q, K, V1, S0, R0):
     L = np.tril(np.ones((c, c)))
     A = L * (Q @ K.T)
     P = Q @ S0
-    W = L * (P @ Q.T + A @ A.T)
+    W = L * (P @ Q.T + A @ A.T)       # W_tj = q_t^T S_j q_j
     O = Q @ R0 + W @ V1
     Z = P + A @ K                     # row j: S_j q_j
     return O, S0 + K.T @ K, R0 + Z.T @ V1
@@ -80,6 +80,25 @@ def hla2_walk(q, k, v, c, normalized, S0=None, R0=None):
     if normalized:
         O = O[:, :-1] / (O[:, -1:] + EPS)
     return O, S0, R0
+
+
+def test_pair_weight_two_forms():
+    """L (.) (Q S0 Q^T + A A^T) equals L (.) (Q Z^T) with Z = Q S0 + A K: the weight of the
+    pair (t, j) sums (q_t . k_i)(q_j . k_i) over the carried-in keys and the keys i <= j."""
+    rng = np.random.default_rng(4)
+    c, d = 16, 5
+    Q, K = rng.standard_normal((c, d)), rng.standard_normal((c, d))
+    G = rng.standard_normal((d, d))
+    S0 = G @ G.T
+    L = np.tril(np.ones((c, c)))
+    A = L * (Q @ K.T)
+    Z = Q @ S0 + A @ K
+    np.testing.assert_allclose(L * (Q @ Z.T), L * (Q @ S0 @ Q.T + A @ A.T), rtol=0, atol=1e-12)
+    # the brute-force pair weight, entry by entry
+    for t in range(c):
+        for j in range(t + 1):
+            w = Q[t] @ S0 @ Q[j] + sum((Q[t] @ K[i]) * (Q[j] @ K[i]) for i in range(j + 1))
+            assert abs((Q[t] @ Z[j]) - w) < 1e-12
 
 
 @pytest.mark.parametrize("normalized", [False, True])
