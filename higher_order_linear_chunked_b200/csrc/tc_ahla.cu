@@ -40,13 +40,16 @@ constexpr uint32_t AS_V = 0;             // V  [tok][feat]
 constexpr uint32_t AS_Q = AS_V + TILE;   // Q, then Y  [tok][feat]
 constexpr uint32_t AS_K = AS_Q + TILE;   // K  [tok][feat]
 constexpr uint32_t AS_ST = AS_K + TILE;  // [P0^T ; E0^T] K-major [128 n][64 k], directly after K
-constexpr uint32_t AS_A = AS_ST + TILE;  // A: [128][128] K-major (two 64-wide atoms)
+constexpr uint32_t AS_A = AS_ST + TILE;  // O staging (output walk); set-up: the carried-in state
 constexpr uint32_t AS_BAR = AS_A + 2 * TILE;
 constexpr uint32_t AS_TOTAL = AS_BAR + 64;
 constexpr uint32_t ASMEM_BYTES = AS_TOTAL + 1024;   // + alignment slack
 
 // TMEM columns (fp32, 128 lanes).
-constexpr uint32_t TA_A = 0;      // A (128), then the state increment [dP^T ; dE^T] (64)
+constexpr uint32_t TA_A = 0;      // A (128); then the masked A as bf16 pairs at columns 0-31
+                                  // (tokens 0-63) and 96-127 (tokens 64-127), the state
+                                  // increment [dP^T ; dE^T] between them (TA_INC, 64)
+constexpr uint32_t TA_INC = 32;
 constexpr uint32_t TA_Y = 128;    // Q P0, then Y (64)
 constexpr uint32_t TA_O = 192;    // output walk: Q E0, then O (64)
 constexpr uint32_t TA_D = 192;    // summary walk: lanes 0-63 D^T of the segment (64)
@@ -58,7 +61,7 @@ enum Mode { SUMMARY = 0, OUTPUT = 1 };
 // and half (w >> 2) of each tile's columns.  Thread 0 also issues the TMA loads and MMAs.
 //
 // Rounds of MMAs per chunk n, each followed by an epilogue:
-//   R1: [A | Q P0 | Q E0] = Q [K ; P0^T ; E0^T]^T      -> E1: A masked to bf16
+//   R1: [A | Q P0 | Q E0] = Q [K ; P0^T ; E0^T]^T      -> E1: A masked to bf16 pairs in TMEM
 //   R2: Y += A V  (summary: also D^T += Q^T K)          -> E2: Y to bf16 (over Q)
 //   R3: O += A Y  (output only), [dP^T ; dE^T] = [V^T ; Y^T] K
 //                                                      -> E3: state += increment, to bf16;
@@ -225,7 +228,6 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     constexpr uint32_t I_N64_KM = ptx::idesc_bf16(128, 64, false, true);
     constexpr uint32_t I_N64_MM = ptx::idesc_bf16(128, 64, true, true);
     auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
-    auto k2 = [](uint64_t d0, int s) { return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4); };
     auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };                       // +2048 B
     // Operand descriptors (built where they are used: only thread 0 issues MMAs).
     //   Q [K ; P0^T ; E0^T]^T : K-major Q and K-major B rows K, then P0^T, E0^T
@@ -235,9 +237,11 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         const uint64_t dQ = kdesc(sbase + AS_Q, 0), dKS = kdesc(sbase + AS_K, 0);
         for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TA_A, k1(dQ, s), k1(dKS, s), I_R1, s > 0);
     };
+    // masked A as bf16 pairs: K-step s (tokens 16 s .. 16 s + 15)
+    auto a_pairs = [&](int s) { return tmem + TA_A + (s < 4 ? 8 * s : 96 + 8 * (s - 4)); };
     auto issue_r2 = [&](int n) {
-        const uint64_t dA2 = kdesc2(sbase + AS_A, 0), dVm = mdesc(sbase + AS_V, TILE, 0);
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_Y, k2(dA2, s), mn(dVm, s), I_N64_KM, 1);
+        const uint64_t dVm = mdesc(sbase + AS_V, TILE, 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TA_Y, a_pairs(s), mn(dVm, s), I_N64_KM, 1);
         if (MODE == SUMMARY) {   // lanes 0-63: D^T += Q^T K (lanes 64-127 take K^T K, unused)
             const uint64_t dQK = mdesc(sbase + AS_Q, AS_K - AS_Q, 0), dKm = mdesc(sbase + AS_K, TILE, 0);
             for (int s = 0; s < 8; ++s)
@@ -247,20 +251,24 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     auto issue_r3 = [&]() {
         const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
         if (MODE == OUTPUT) {
-            const uint64_t dA2 = kdesc2(sbase + AS_A, 0), dYm = mdesc(sbase + AS_Q, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_O, k2(dA2, s), mn(dYm, s), I_N64_KM, 1);
+            const uint64_t dYm = mdesc(sbase + AS_Q, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TA_O, a_pairs(s), mn(dYm, s), I_N64_KM, 1);
         }
         const uint64_t dVY = mdesc(sbase + AS_V, AS_Q - AS_V, 0);
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_A, mn(dVY, s), mn(dKm, s), I_N64_MM, s > 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_INC, mn(dVY, s), mn(dKm, s), I_N64_MM, s > 0);
     };
 
     uint32_t mma_phase = 0;
-    bool ok = true;
+    bool ok = true;                          // agreed by the whole block
+    bool issuer_ok = true;                   // thread 0's load waits since the last agreement
+    // Thread 0 commits the MMAs issued so far and waits for them (bounded); the block agrees,
+    // on that and on thread 0's own load waits.
     auto commit_wait = [&]() -> bool {
         bool good = true;
+        ptx::tc_fence_before();
         if (tid == 0) {
             ptx::umma_commit(bar_mma);
-            good = ptx::mbar_wait(bar_mma, mma_phase);
+            good = ptx::mbar_wait(bar_mma, mma_phase) && issuer_ok;
         }
         mma_phase ^= 1;
         good = __syncthreads_and(good) != 0;
@@ -274,17 +282,44 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         ptx::tc_fence_after();
     };
 
-    // E1: A (masked, inclusive diagonal) -> AS_A; this thread: columns half*64 .. +63
-    auto epi1 = [&]() {
-        float v[32];
+    // 32 fp32 columns of this lane -> 16 bf16 pairs in TMEM (column 2i in the low half); on
+    // the diagonal block the columns past this lane's token are cleared; nullptr: zeros.
+    auto st_pairs = [&](uint32_t tcol, const float* x, bool diag) {
+        uint32_t r[16];
+        if (x == nullptr) {
 #pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            ptx::tmem_ld32(tmem + lane_base + TA_A + c0, v);
+            for (int i = 0; i < 16; ++i) r[i] = 0u;
+        } else if (diag) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i > row) v[i] = 0.f;
-            st_row32(sm + AS_A, row, c0, v);
+            for (int i = 0; i < 16; ++i)
+                r[i] = ptx::pack_bf16(2 * i > lane ? 0.f : x[2 * i], 2 * i + 1 > lane ? 0.f : x[2 * i + 1]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = ptx::pack_bf16(x[2 * i], x[2 * i + 1]);
         }
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    // E1: A (masked, inclusive diagonal) -> bf16 pairs, in place: this warp reads its token
+    // blocks b0 = 2 half and b0 + 1 (columns 64 half .. +63) and writes their pairs to columns
+    // 96 half .. +31, which it has read itself.  Blocks above the diagonal (b > quad) become
+    // zeros (the A of every chunk overwrites them).
+    auto epi1 = [&]() {
+        const int b0 = 2 * half;
+        const uint32_t pc = TA_A + 96 * half;
+        float v0[32], v1[32];
+        if (b0 + 1 <= quad) {
+            ptx::tmem_ld32x2(tmem + lane_base + TA_A + 32 * b0, tmem + lane_base + TA_A + 32 * (b0 + 1), v0, v1);
+            st_pairs(pc, v0, false);
+            st_pairs(pc + 16, v1, b0 + 1 == quad);
+        } else if (b0 == quad) {
+            ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * b0, v0);
+            st_pairs(pc, v0, true);
+            st_pairs(pc + 16, nullptr, false);
+        } else {
+            st_pairs(pc, nullptr, false);
+            st_pairs(pc + 16, nullptr, false);
+        }
+        ptx::tmem_st_wait();
     };
     // E2: Y -> AS_Q (the Q tile is no longer read)
     auto epi2 = [&]() {
@@ -296,7 +331,7 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // A tile as two [128 rows][32 cols] boxes in the 128B-swizzled TMA layout
     auto epi3 = [&]() {
         float v[32];
-        ptx::tmem_ld32(tmem + lane_base + TA_A + half * 32, v);
+        ptx::tmem_ld32(tmem + lane_base + TA_INC + half * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[i] += v[i];
         if (MODE == OUTPUT || row < 64) st_row32(sm + AS_ST, row, half * 32, st);
@@ -317,26 +352,27 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     };
 
     // ---- the walk
+    // ok changes only where the block agrees, so every thread runs the same barriers.
     for (int n = 0; n < nch && ok; ++n) {
         if (tid == 0) {
             if (MODE == OUTPUT && n > 0) store_o(n - 1);
-            ok = ptx::mbar_wait(bar_load, n & 1);
-            if (ok) {
+            issuer_ok = ptx::mbar_wait(bar_load, n & 1);
+            if (issuer_ok) {
                 ptx::tc_fence_after();
                 issue_r1();
             }
-            if (MODE == OUTPUT) ptx::bulk_wait_read();      // the A tile is free for E1 again
         }
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (!commit_wait()) { ok = false; break; }          // R1 done
+        if (!commit_wait()) { ok = false; break; }          // loads and R1 done
         epi1();
         sync_for_mma();
         if (tid == 0) issue_r2(n);
         if (!commit_wait()) { ok = false; break; }          // R2 done
         epi2();
         sync_for_mma();
-        if (tid == 0) issue_r3();
+        if (tid == 0) {
+            issue_r3();
+            if (MODE == OUTPUT) ptx::bulk_wait_read();      // the O staging is free for E3 again
+        }
         if (!commit_wait()) { ok = false; break; }          // R3 done: Q/Y, K, V free
         if (tid == 0 && n + 1 < nch) issue_load(n + 1);
         epi3();
