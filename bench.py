@@ -50,6 +50,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(hla_inputs.WORKLOADS))
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--decode-steps", type=int, default=20,
+                   help="streaming decode steps timed after the forward (0: skip)")
     p.add_argument("--segment-chunks", type=int, default=0,
                    help="tensor-core path: 128-token chunks per segment (0 = the library's choice)")
     args = p.parse_args(argv)
@@ -295,6 +297,9 @@ def run_ours(args):
                "pipeline": f"{G} batch slices on {G} streams: copy in, forward, copy out per slice"}
 
     peaks, peak_kind = load_peaks()
+    decode = None
+    if args.decode_steps > 0:
+        decode = decode_measure(w, qd, kd, vd, gd, flush, args.decode_steps, peaks, peak_kind)
     clk = clocks.summary()
     model = output_kernel_model(path, w)
     out_avg_ms = statistics.mean(out_ms)
@@ -327,13 +332,54 @@ def run_ours(args):
                        "segment_chunks": args.segment_chunks or "auto",
                        "l2": "flushed before every step (512 MiB write, outside the timed events)",
                        "parallelism": f"dp{world} (independent heads per rank, no collective)"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "clocks": clk,
             "gpu_launches": launches_per_step * args.steps, "device_status": status,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
+    """Streaming form: the prefill state of the workload's T tokens (hla_state), then `steps`
+    one-token decode steps per head (hla_step), each timed alone with CUDA events after an L2
+    flush.  A step reads and writes every head's state once: HBM-bound."""
+    import torch
+
+    import higher_order_linear_chunked_b200 as hla
+    B, H, T, d = qd.shape
+    dev = qd.device
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    flush.zero_()
+    ev[0].record()
+    st = hla.state(w.op, qd, kd, vd, gamma=gd)
+    ev[1].record()
+    torch.cuda.synchronize()
+    prefill_ms = ev[0].elapsed_time(ev[1])
+    toks = [(qd[:, :, t].contiguous(), kd[:, :, t].contiguous(), vd[:, :, t].contiguous()) for t in range(steps)]
+    o = torch.empty((B, H, vd.shape[-1]), dtype=torch.float32, device=dev)
+    for t in range(3):                                              # warm-up on a copy of the state
+        hla.step(w.op, st.clone(), *toks[t % steps], gamma=gd, eps=w.eps, out=o)
+    times = []
+    for t in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        hla.step(w.op, st, *toks[t], gamma=gd, eps=w.eps, out=o)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    step_ms = statistics.mean(times)
+    esz = qd.element_size()
+    nbytes = B * H * (2 * st.shape[-1] * 4 + 3 * d * esz + vd.shape[-1] * 4)   # state in and out, q k v, o
+    gbs = nbytes / (step_ms / 1e3) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"prefill_ms": prefill_ms, "prefill_tokens": B * H * T, "steps": steps, "us_per_step": step_ms * 1e3,
+            "tokens_per_s": B * H / (step_ms / 1e3), "gpu_launches_per_step": 1,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "bytes_per_step": nbytes, "peak_source": f"HBM copy ({peak_kind})"},
+            "l2": "flushed before every step (outside the events)"}
 
 
 def _traffic_from_profiles(path, w):

@@ -37,7 +37,8 @@ STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_
 # Every symbol include/hla.h declares.
 EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
            "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
-           "hla2_forward_normalized_noalloc")
+           "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
+           "hla_state_kernel_launches", "hla_state", "hla_step")
 
 
 class HLAError(RuntimeError):
@@ -86,6 +87,15 @@ def load_library(path: Optional[str] = None):
     lib.hla_selftest_umma.restype = i
     lib.hla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]
     lib.hla_selftest_wait_timeout.restype = i
+    lib.hla_state_floats.argtypes, lib.hla_state_floats.restype = [i, i, i, i], sz
+    lib.hla_state_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+    lib.hla_state_workspace_bytes.restype = sz
+    lib.hla_state_kernel_launches.argtypes = [i, i, i, i, i, i, i, i]
+    lib.hla_state_kernel_launches.restype = i
+    lib.hla_state.argtypes = [i, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, sz, vp]
+    lib.hla_state.restype = i
+    lib.hla_step.argtypes = [i, vp, vp, vp, vp, vp, i, i, i, i, i, vp, f, vp]
+    lib.hla_step.restype = i
     if path is None:
         _lib = lib
     return lib
@@ -259,4 +269,83 @@ def forward_profiled(op_name: str, q, k, v, events, gamma=None, eps: float = 1e-
         ctypes.c_void_p(st.cuda_stream), ctypes.cast(handles, ctypes.c_void_p))
     if rc != HLA_OK:
         raise HLAError(rc, "hla_forward_profiled rejected the call")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# streaming state: prefill (state after T tokens) and one-token decode steps
+# ---------------------------------------------------------------------------
+
+def state_floats(op_name: str, d: int, dv: int, decayed=None) -> int:
+    """Floats of one head's streaming state for ``op_name`` (see ``hla_state_floats``);
+    ``decayed`` defaults to ``op_name == "hla2d"`` (pass True for "hla2n" with gamma)."""
+    dec = op_name == "hla2d" if decayed is None else bool(decayed)
+    return int(load_library().hla_state_floats(OP_CODES[op_name], int(dec), d, dv))
+
+
+def new_state(op_name: str, B: int, H: int, d: int, device="cuda", decayed=None):
+    """The state of zero tokens: zeros, with rho = 1 for the decayed form."""
+    torch = _torch()
+    dec = op_name == "hla2d" if decayed is None else bool(decayed)
+    n = state_floats(op_name, d, d, decayed=dec)
+    if n == 0:
+        raise HLAError(5, "no streaming state for this op / d")
+    st = torch.zeros((B, H, n), dtype=torch.float32, device=device)
+    if dec:
+        st[..., 4 * d * d + 2 * d] = 1.0       # rho, after four d x d matrices and two vectors
+    return st
+
+
+def state(op_name: str, q, k, v, gamma=None, out=None, workspace=None, stream=None):
+    """Prefill: the streaming state [B, H, state_floats] of every head after its T tokens."""
+    torch = _torch()
+    _check(q, k, v)
+    lib = load_library()
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    op = OP_CODES[op_name]
+    decayed = op_name == "hla2d" or (op_name == "hla2n" and gamma is not None)
+    if op_name == "hla2d" and gamma is None:
+        raise ValueError("hla2d needs gamma")
+    n = int(lib.hla_state_floats(op, int(decayed), d, dv))
+    if out is None:
+        out = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nb = int(lib.hla_state_workspace_bytes(op, _dtype_code(q), int(decayed), B, H, T, d, dv))
+        if nb == 0:
+            raise HLAError(5, "unsupported shape/dtype for this op")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=q.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = lib.hla_state(op, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                       ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), B, H, T, d, dv,
+                       _dtype_code(q), ctypes.c_void_p(gamma.data_ptr()) if gamma is not None else ctypes.c_void_p(0),
+                       ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()),
+                       ctypes.c_void_p(st.cuda_stream))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla_state rejected the call")
+    return out
+
+
+def step(op_name: str, state_io, q, k, v, gamma=None, eps: float = 1e-6, out=None, stream=None):
+    """Decode one token per head: q, k, v [B, H, d]; advances ``state_io`` in place; returns o [B, H, dv]."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("state", state_io)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q.dim() != 3 or q.shape != k.shape or q.shape[:2] != v.shape[:2]:
+        raise ValueError("q, k [B,H,d], v [B,H,dv]")
+    if state_io.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    B, H, d = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = load_library().hla_step(
+        OP_CODES[op_name], ctypes.c_void_p(state_io.data_ptr()), ctypes.c_void_p(q.data_ptr()),
+        ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+        B, H, d, dv, _dtype_code(q), ctypes.c_void_p(gamma.data_ptr()) if gamma is not None else ctypes.c_void_p(0),
+        ctypes.c_float(eps), ctypes.c_void_p(st.cuda_stream))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla_step rejected the call")
     return out

@@ -80,6 +80,11 @@ hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, f
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 
+// Streaming-state requests run on the CUDA-core kernels (fp32 state, any supported dtype).
+size_t state_workspace_for(const Request& r) {
+    return hla::kStatusBytes + sizeof(float) * hla::simt::workspace_floats(r.op, r.d, r.B * r.H, r.T);
+}
+
 }  // namespace
 
 extern "C" {
@@ -151,6 +156,59 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
                                   void* const* phase_events) {
     return forward(op, q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, workspace, workspace_bytes, stream,
                    phase_events);
+}
+
+size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv) {
+    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return 0;
+    if (d != dv || (d != 32 && d != 64)) return 0;
+    if (decayed && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return 0;
+    return hla::simt::summary_floats(make_request(op, decayed != 0, HLA_F32, 1, 1, 1, d, dv).op, d);
+}
+
+size_t hla_state_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
+    if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
+    return state_workspace_for(make_request(op, decayed != 0, dtype, B, H, T, d, dv));
+}
+
+int hla_state_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
+    if (hla_state_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
+    return hla::simt::state_launches(T);
+}
+
+hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v, float* state, int B, int H, int T,
+                       int d, int dv, hla_dtype_t dtype, const float* gamma, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !state) return HLA_ERR_NULL;
+    hla_status_t s = check_shape(dtype, B, H, T, d, dv);
+    if (s != HLA_OK) return s;
+    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state)) return HLA_ERR_ALIGN;
+    if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
+    const Request r = make_request(op, gamma != nullptr, dtype, B, H, T, d, dv);
+    if (!workspace) return HLA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HLA_ERR_ALIGN;
+    if (workspace_bytes < state_workspace_for(r)) return HLA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
+    float* sums = reinterpret_cast<float*>(static_cast<char*>(workspace) + hla::kStatusBytes);
+    const cudaError_t e = hla::simt::state(r.op, r.bf16, d, q, k, v, gamma, B * H, H, T, sums, state, st);
+    return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
+}
+
+hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, const void* v, float* o, int B, int H,
+                      int d, int dv, hla_dtype_t dtype, const float* gamma, float eps, void* stream) {
+    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!state || !q || !k || !v || !o) return HLA_ERR_NULL;
+    hla_status_t s = check_shape(dtype, B, H, 1, d, dv);
+    if (s != HLA_OK) return s;
+    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HLA_ERR_ALIGN;
+    if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
+    const Request r = make_request(op, gamma != nullptr, dtype, B, H, 1, d, dv);
+    const cudaError_t e = hla::simt::step(r.op, r.norm, r.bf16, d, state, q, k, v, gamma, eps, B * H, H, o,
+                                          static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 
 hla_status_t hla_set_segment_chunks(int chunks) {

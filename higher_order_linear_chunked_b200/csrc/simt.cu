@@ -218,9 +218,12 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     load_rows<D>(Ks, k + head, t0, T);
     load_rows<D>(Vs, v + head, t0, T);
     float g = 1.f;
+    const int len = min(C, T - t0);      // tokens in this chunk (the last one may be short)
     if (OP == OP_HLA2D) {
+        // gamma^(len - 1 - tau): decayed to the chunk's own last token, so that the summary of
+        // a short last chunk is the state after the sequence's last token (the streaming state)
         g = gamma[bh % H];
-        for (int j = threadIdx.x; j < C; j += blockDim.x) lam[j] = gpow(g, C - 1 - j);  // gamma^(len - tau)
+        for (int j = threadIdx.x; j < C; j += blockDim.x) lam[j] = j < len ? gpow(g, len - 1 - j) : 0.f;
     }
     __syncthreads();
     // A* = Q K^T (masked to A = L (.) A* except for the decayed op, which needs both parts)
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
             out[S::vec(0) + a] = sm_;                                    // m
             out[S::vec(1) + a] = sh;                                     // h = K^T u
         }
-        if (threadIdx.x == 0) out[S::SCAL] = gpow(g, C);                 // rho = gamma^len
+        if (threadIdx.x == 0) out[S::SCAL] = gpow(g, len);               // rho = gamma^len
     } else if (OP == OP_AHLA) {
         mm<D, D, C>(TileT{Ks, LD}, Tile{Vs, LD}, Zero{}, store_mat(0));        // P = K^T V
         mm<D, D, C>(TileT{Ks, LD}, Tile{Qs, LD}, Zero{}, store_mat(2));        // Dm = K^T Q
@@ -652,6 +655,277 @@ cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const vo
 }
 
 int kernel_launches(int T) { return 2 + scan_launches(next_pow2((T + C - 1) / C)); }
+
+// ---------------------------------------------------------------------------
+// Streaming state.  A head's state after t tokens is the summary of those t
+// tokens in the layout above (the state the recurrence reaches from zero, with
+// the maps the combine needs), so the chunk kernel and the up-sweep of the scan
+// export it and the step kernel below advances it one token at a time.
+// ---------------------------------------------------------------------------
+
+// Copy the root of each head's up-sweep tree (slot NCp-1: every chunk combined) out.
+template <int OP, int D>
+__global__ void __launch_bounds__(NT) k_copy_root(const float* __restrict__ sums, int NCp, float* __restrict__ state) {
+    using S = Sum<OP, D>;
+    const float* src = sums + ((size_t)blockIdx.x * NCp + NCp - 1) * S::SIZE;
+    float* dst = state + (size_t)blockIdx.x * S::SIZE;
+    for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) dst[e] = src[e];
+}
+
+template <int OP, int D, typename TIn>
+static cudaError_t state_run(const void* q, const void* k, const void* v, const float* gamma, int BH, int H, int T,
+                             float* sums, float* state, cudaStream_t st) {
+    const int NC = (T + C - 1) / C;
+    const int NCp = next_pow2(NC);
+    auto ks = k_summary<OP, D, TIn>;
+    auto kl = k_scan_level<OP, D>;
+    const size_t s1 = summary_smem<D>(), s2 = scan_smem<OP, D>();
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
+    ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, H, T, NC, NCp, sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    for (int step = 1; step < NCp; step *= 2) {            // up-sweep only: the root ends as the total
+        kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 0, 0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    k_copy_root<OP, D><<<BH, NT, 0, st>>>(sums, NCp, state);
+    return cudaGetLastError();
+}
+
+template <typename TIn, int D>
+static cudaError_t state_op(int op, const void* q, const void* k, const void* v, const float* gamma, int BH, int H,
+                            int T, float* sums, float* state, cudaStream_t st) {
+    switch (op) {
+    case OP_HLA2: return state_run<OP_HLA2, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_HLA2D: return state_run<OP_HLA2D, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_AHLA: return state_run<OP_AHLA, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_HLA3: return state_run<OP_HLA3, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t state(int op, bool bf16, int d, const void* q, const void* k, const void* v, const float* gamma, int BH,
+                  int H, int T, float* sums, float* state_out, cudaStream_t st) {
+    if (bf16) {
+        if (d == 32) return state_op<__nv_bfloat16, 32>(op, q, k, v, gamma, BH, H, T, sums, state_out, st);
+        return state_op<__nv_bfloat16, 64>(op, q, k, v, gamma, BH, H, T, sums, state_out, st);
+    }
+    if (d == 32) return state_op<float, 32>(op, q, k, v, gamma, BH, H, T, sums, state_out, st);
+    return state_op<float, 64>(op, q, k, v, gamma, BH, H, T, sums, state_out, st);
+}
+
+int state_launches(int T) {
+    int levels = 0;
+    for (int p = 1; p < next_pow2((T + C - 1) / C); p *= 2) ++levels;
+    return 2 + levels;                                       // chunk kernel, up-sweep levels, copy
+}
+
+// One token per head: the recurrence's update, on the summary layout, in fp32.
+//   second order (R-form)  S += k k^T;  C += q v^T;  m += q;  z = S q;  R += z v^T;  r += z;
+//                          o = q^T R  (ratio-normalised: / (q . r + eps))
+//   decayed                w = g (k^T C), s = g (k . m);  S = g S + k k^T;  C = g C + q v^T;
+//                          G = g G + k w^T;  m = g m + q;  h = g h + s k;  Khat += k k^T;
+//                          rho *= g;  x = q^T S;  o = x^T C - q^T G  (/ (x . m - q . h + eps))
+//   AHLA                   P += k v^T;  Dm += k q^T;  y = q^T P;  E += k y^T;  o = q^T E
+//   third order            S += k k^T;  P += k v^T;  Q2 += q q^T;  a = S q;  b = q^T P;
+//                          F += a b^T;  X += q b^T;  Z += a q^T;  o = q^T F
+// S is symmetric, so every product with a vector reads matrix columns: thread j of a group
+// walks rows i, and four groups of D threads split the rows (partial sums in shared memory).
+// The head's state is staged in shared memory (every load in flight at once), updated there
+// and written back once: one read and one write of the state per step.
+template <int D>
+__device__ __forceinline__ void col_dot(const float* __restrict__ M, const float* x, float* part, float* out) {
+    const int j = threadIdx.x % D, g = threadIdx.x / D;       // NT / D groups
+    constexpr int G = NT / D, RPG = D / G;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int i = g * RPG; i < (g + 1) * RPG; ++i) acc = fmaf(x[i], M[i * D + j], acc);
+    part[g * D + j] = acc;
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float t = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) t += part[h * D + threadIdx.x];
+        out[threadIdx.x] = t;
+    }
+    __syncthreads();
+}
+
+template <int OP, bool NORM, int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TIn* __restrict__ q,
+                                             const TIn* __restrict__ k, const TIn* __restrict__ v,
+                                             const float* __restrict__ gamma, float eps, int H, float* __restrict__ o) {
+    using S = Sum<OP, D>;
+    constexpr int DD = D * D;
+    constexpr int N4 = S::SIZE / 4, PER = (N4 + NT - 1) / NT;
+    __shared__ float qs[D], ks[D], vs[D], a[D], b[D], part[NT];
+    __shared__ float scal[2];
+    extern __shared__ float4 st4[];
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    float4* gst = reinterpret_cast<float4*>(state + (size_t)bh * S::SIZE);
+    // asynchronous 16-byte copies (no registers held): all of them in flight, then one wait
+    for (int i = 0; i < PER; ++i) {
+        const int e = tid + i * NT;
+        if (e < N4) {
+            const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(st4 + e));
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gst + e) : "memory");
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    float* st = reinterpret_cast<float*>(st4);
+    if (tid < D) {
+        qs[tid] = to_f32(q[(size_t)bh * D + tid]);
+        ks[tid] = to_f32(k[(size_t)bh * D + tid]);
+        vs[tid] = to_f32(v[(size_t)bh * D + tid]);
+    }
+    __syncthreads();
+    if (OP == OP_HLA2) {
+        float* Sm = st + S::mat(0); float* Cm = st + S::mat(1); float* Rm = st + S::mat(2);
+        float* m = st + S::vec(0); float* r = st + S::vec(1);
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            Sm[e] = fmaf(ks[i], ks[j], Sm[e]);
+            Cm[e] = fmaf(qs[i], vs[j], Cm[e]);
+        }
+        if (tid < D) m[tid] += qs[tid];
+        __syncthreads();
+        col_dot<D>(Sm, qs, part, a);                            // a = z = S q
+        for (int e = tid; e < DD; e += NT) Rm[e] = fmaf(a[e / D], vs[e % D], Rm[e]);
+        if (tid < D) r[tid] += a[tid];
+        __syncthreads();
+        col_dot<D>(Rm, qs, part, b);                            // b = q^T R
+        if (tid < D) {
+            float den = 1.f;
+            if (NORM) {
+                float t = 0.f;
+                for (int i = 0; i < D; ++i) t = fmaf(qs[i], r[i], t);
+                den = t + eps;
+            }
+            o[(size_t)bh * D + tid] = NORM ? b[tid] / den : b[tid];
+        }
+    } else if (OP == OP_HLA2D) {
+        const float g = gamma[bh % H];
+        float* Sm = st + S::mat(0); float* Cm = st + S::mat(1); float* Gm = st + S::mat(2); float* Kh = st + S::mat(3);
+        float* m = st + S::vec(0); float* h = st + S::vec(1);
+        col_dot<D>(Cm, ks, part, a);                            // a = k^T C (before the update)
+        if (tid == 0) {
+            float t = 0.f;
+            for (int i = 0; i < D; ++i) t = fmaf(ks[i], m[i], t);
+            scal[0] = g * t;                                    // s = g (k . m)
+        }
+        __syncthreads();
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            const float kk = ks[i] * ks[j];
+            Sm[e] = fmaf(g, Sm[e], kk);
+            Cm[e] = fmaf(g, Cm[e], qs[i] * vs[j]);
+            Gm[e] = fmaf(g, Gm[e], ks[i] * (g * a[j]));
+            Kh[e] += kk;
+        }
+        if (tid < D) {
+            m[tid] = fmaf(g, m[tid], qs[tid]);
+            h[tid] = fmaf(g, h[tid], scal[0] * ks[tid]);
+        }
+        if (tid == 0) st[S::SCAL] *= g;
+        __syncthreads();
+        col_dot<D>(Sm, qs, part, b);                            // b = x = q^T S
+        // o_j = sum_i x_i C[i][j] - q_i G[i][j]
+        {
+            const int j = tid % D, gi = tid / D;
+            constexpr int G = NT / D, RPG = D / G;
+            float acc = 0.f;
+            for (int i = gi * RPG; i < (gi + 1) * RPG; ++i) acc += b[i] * Cm[i * D + j] - qs[i] * Gm[i * D + j];
+            part[gi * D + j] = acc;
+        }
+        __syncthreads();
+        if (tid < D) {
+            float t = 0.f;
+            for (int hh = 0; hh < NT / D; ++hh) t += part[hh * D + tid];
+            float den = 1.f;
+            if (NORM) {
+                float x = 0.f;
+                for (int i = 0; i < D; ++i) x += b[i] * m[i] - qs[i] * h[i];
+                den = x + eps;
+            }
+            o[(size_t)bh * D + tid] = NORM ? t / den : t;
+        }
+    } else if (OP == OP_AHLA) {
+        float* P = st + S::mat(0); float* E = st + S::mat(1); float* Dm = st + S::mat(2);
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            P[e] = fmaf(ks[i], vs[j], P[e]);
+            Dm[e] = fmaf(ks[i], qs[j], Dm[e]);
+        }
+        __syncthreads();
+        col_dot<D>(P, qs, part, a);                             // a = y = q^T P
+        for (int e = tid; e < DD; e += NT) E[e] = fmaf(ks[e / D], a[e % D], E[e]);
+        __syncthreads();
+        col_dot<D>(E, qs, part, b);                             // b = q^T E
+        if (tid < D) o[(size_t)bh * D + tid] = b[tid];
+    } else {                                                    // OP_HLA3
+        float* Sm = st + S::mat(0); float* Q2 = st + S::mat(1); float* P = st + S::mat(2);
+        float* F = st + S::mat(3); float* X = st + S::mat(4); float* Z = st + S::mat(5);
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            Sm[e] = fmaf(ks[i], ks[j], Sm[e]);
+            P[e] = fmaf(ks[i], vs[j], P[e]);
+            Q2[e] = fmaf(qs[i], qs[j], Q2[e]);
+        }
+        __syncthreads();
+        col_dot<D>(Sm, qs, part, a);                            // a = S q
+        col_dot<D>(P, qs, part, b);                             // b = q^T P
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            F[e] = fmaf(a[i], b[j], F[e]);
+            X[e] = fmaf(qs[i], b[j], X[e]);
+            Z[e] = fmaf(a[i], qs[j], Z[e]);
+        }
+        __syncthreads();
+        col_dot<D>(F, qs, part, a);                             // a = q^T F
+        if (tid < D) o[(size_t)bh * D + tid] = a[tid];
+    }
+    __syncthreads();
+    for (int e = tid; e < N4; e += NT) gst[e] = st4[e];
+}
+
+template <int OP, bool NORM, int D, typename TIn>
+static cudaError_t step_launch(float* st_, const void* q, const void* k, const void* v, const float* gamma,
+                               float eps, int BH, int H, float* o, cudaStream_t st) {
+    auto kf = k_step<OP, NORM, D, TIn>;
+    const int smem = Sum<OP, D>::SIZE * (int)sizeof(float);     // the head's state
+    cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kf<<<BH, NT, smem, st>>>(st_, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H, o);
+    return cudaGetLastError();
+}
+
+template <typename TIn, int D>
+static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const void* k, const void* v,
+                           const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st) {
+    switch (op) {
+    case OP_HLA2:
+        return norm ? step_launch<OP_HLA2, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_HLA2, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA2D:
+        return norm ? step_launch<OP_HLA2D, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_HLA2D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_AHLA: return step_launch<OP_AHLA, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA3: return step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const void* q, const void* k, const void* v,
+                 const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st) {
+    if (bf16) {
+        if (d == 32) return step_op<__nv_bfloat16, 32>(op, norm, state_io, q, k, v, gamma, eps, BH, H, o, st);
+        return step_op<__nv_bfloat16, 64>(op, norm, state_io, q, k, v, gamma, eps, BH, H, o, st);
+    }
+    if (d == 32) return step_op<float, 32>(op, norm, state_io, q, k, v, gamma, eps, BH, H, o, st);
+    return step_op<float, 64>(op, norm, state_io, q, k, v, gamma, eps, BH, H, o, st);
+}
+
 
 }  // namespace simt
 }  // namespace hla

@@ -26,5 +26,16 @@ cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const vo
                     const float* gamma, float eps, float* o, int BH, int H, int T, float* sums,
                     cudaStream_t st, cudaEvent_t* ev);
 
+// Streaming state: one summary (summary_floats(op, d) floats) per head.
+// state(): the state of each head after its T tokens (chunk kernel, up-sweep, copy of the
+// root) into state_out[BH][summary_floats]; sums is workspace_floats(op, d, BH, T) floats.
+cudaError_t state(int op, bool bf16, int d, const void* q, const void* k, const void* v, const float* gamma, int BH,
+                  int H, int T, float* sums, float* state_out, cudaStream_t st);
+// kernels state() enqueues
+int state_launches(int T);
+// step(): one token per head ([BH][d] q, k, v): state advanced in place, o [BH][d] written.
+cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const void* q, const void* k, const void* v,
+                 const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st);
+
 }  // namespace simt
 }  // namespace hla

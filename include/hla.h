@@ -146,6 +146,61 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
 
 /*
+ * Streaming state (decoding one token at a time after a prefill).
+ *
+ * The pages give every operator both as a masked sum and as a streaming
+ * recurrence with an O(1)-per-token state (Metodología 1-3), and build the
+ * chunked scan on segment summaries that concatenate (Metodología 4).  A head's
+ * state after t tokens is the summary of those t tokens: the recurrence's state
+ * reached from zero, plus the maps the combine needs.  Layout, per head, fp32,
+ * hla_state_floats() floats: n matrices of d x d (row-major), then vectors of
+ * d, then one scalar, padded to a multiple of 32 floats:
+ *   second order          S = sum k k^T, C = sum q v^T, R = S C - G;  m = sum q,
+ *                         r = S m - h          (o_t = q_t^T R_t, den = q_t^T r_t)
+ *   second order, decayed S, C, G, Khat = sum k k^T (undecayed);  m, h;  rho =
+ *                         gamma^t              (o_t = q_t^T (S_t C_t - G_t))
+ *   AHLA                  P = sum k v^T, E, D = sum k q^T      (o_t = q_t^T E_t)
+ *   third order           S, Q2 = sum q q^T, P, F, X, Z        (o_t = q_t^T F_t)
+ * A state of zero tokens is all zeros, except rho = 1 for the decayed form.
+ * The state of HLA_OP_HLA2_NORM is that of HLA_OP_HLA2.
+ */
+
+/* Floats of one head's state, or 0 when (op, decayed, d, dv) is invalid or unsupported
+ * (decayed: hla2 / hla2_normalized with gamma). */
+size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv);
+
+/* Workspace bytes hla_state() needs, or 0 when the request is invalid or unsupported.
+ * Same arguments as hla_workspace_bytes(). */
+size_t hla_state_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
+
+/* Kernels one hla_state() call enqueues (chunk kernel, up-sweep levels, copy), or 0. */
+int hla_state_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
+
+/*
+ * Prefill: the state of every head after its T tokens, written to state
+ * [B*H][hla_state_floats] (device, fp32, 16-byte aligned, caller-owned).
+ * q, k, v, gamma, shapes and dtypes as for the forward calls.  Runs the
+ * CUDA-core chunk-summary kernel and the up-sweep half of the Blelloch scan,
+ * whose root is the summary of the whole sequence.  Workspace: at least
+ * hla_state_workspace_bytes().  Errors as for the forward calls.
+ */
+hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v, float* state,
+                       int B, int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decode: one token per head.  q, k, v: [B][H][d] (device, HLA_F32 or HLA_BF16,
+ * 16-byte aligned); o: [B][H][dv] fp32.  Advances state [B*H][hla_state_floats]
+ * in place by the recurrence's update and writes each head's o_t (divided by
+ * den_t + eps for HLA_OP_HLA2_NORM).  gamma: as for the forward calls; the state
+ * must be of the matching (decayed or not) form.  One kernel launch, no
+ * workspace.  Argument errors as for the forward calls (T is 1).
+ */
+hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, const void* v, float* o,
+                      int B, int H, int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
+                      void* stream);
+
+/*
  * Tuning knob of the tensor-core path: chunks of 128 tokens per segment (the
  * unit one CTA walks).  0 restores the automatic choice.  Values outside
  * {0, 1, 2, 4, 8, 16} return HLA_ERR_SHAPE.  Process-wide setting: it changes

@@ -152,6 +152,43 @@ def test_selftest_argument_errors(lib):
     assert wt(vp(16), 256, 2000000, vp(0)) == 2
 
 
+def test_streaming_state_sizes_and_argument_errors(lib):
+    """State sizes follow the summary layout; bad calls are refused before any launch."""
+    vp, f = ctypes.c_void_p, ctypes.c_float
+    d = 64
+    pad = lambda n: (n + 31) // 32 * 32                       # noqa: E731
+    assert lib.hla_state_floats(0, 0, d, d) == pad(3 * d * d + 2 * d + 4)     # S, C, R ; m, r
+    assert lib.hla_state_floats(1, 1, d, d) == pad(4 * d * d + 2 * d + 4)     # decayed: + Khat, rho
+    assert lib.hla_state_floats(2, 0, d, d) == pad(3 * d * d + 4)             # P, E, D
+    assert lib.hla_state_floats(3, 0, 32, 32) == pad(6 * 32 * 32 + 4)        # S, Q2, P, F, X, Z
+    assert lib.hla_state_floats(2, 1, d, d) == 0                              # no decayed AHLA
+    assert lib.hla_state_floats(0, 0, 48, 48) == 0
+    assert lib.hla_state_floats(0, 0, 64, 32) == 0
+    # workspace: status block + the CUDA-core chunk summaries (64-token chunks, padded to 2^k)
+    n = lib.hla_state_workspace_bytes(0, 1, 0, 4, 16, 4096, d, d)
+    assert n == 256 + 4 * 64 * 64 * lib.hla_state_floats(0, 0, d, d)
+    assert lib.hla_state_workspace_bytes(2, 1, 1, 4, 16, 4096, d, d) == 0
+    assert lib.hla_state_kernel_launches(0, 1, 0, 4, 16, 4096, d, d) == 2 + 6     # 64 chunks: 6 levels
+    assert lib.hla_state_kernel_launches(0, 0, 0, 1, 1, 64, 32, 32) == 2
+    st = lib.hla_state
+    a = [vp(16), vp(16), vp(16), vp(16)]
+    assert st(0, vp(0), *a[1:], 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 1      # NULL q
+    assert st(4, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
+    assert st(0, *a, 0, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 2                # B = 0
+    assert st(0, *a, 1, 1, 64, d, d, 7, vp(0), vp(16), 1 << 20, vp(0)) == 4                # dtype
+    assert st(2, *a, 1, 1, 64, d, d, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5               # gamma + AHLA
+    assert st(0, vp(8), *a[1:], 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 3     # alignment
+    assert st(0, *a, 1, 1, 64, d, d, 0, vp(0), vp(0), 1 << 20, vp(0)) == 6                 # no workspace
+    assert st(0, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 64, vp(0)) == 6                     # too small
+    sp = lib.hla_step
+    b = [vp(16)] * 5
+    assert sp(0, vp(0), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 1                 # NULL state
+    assert sp(0, *b, 1, 1, 48, 48, 0, vp(0), f(1e-6), vp(0)) == 5                          # d = 48
+    assert sp(0, *b, 1, 0, d, d, 0, vp(0), f(1e-6), vp(0)) == 2                            # H = 0
+    assert sp(3, *b, 1, 1, 32, 32, 0, vp(16), f(1e-6), vp(0)) == 5                         # gamma + HLA-3
+    assert sp(0, vp(24), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 3                # alignment
+
+
 def test_product_path_never_touches_the_oracle():
     """The package (binding + CUDA sources) must not import, call or link oracle/."""
     pkg = os.path.join(ROOT, "higher_order_linear_chunked_b200")

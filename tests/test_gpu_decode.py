@@ -1,0 +1,143 @@
+"""Streaming state (prefill export) and one-token decode steps, through the C ABI, against
+the fp64 oracle's state-carrying recurrences.
+
+"Higher-order Linear Attention" summary (gist.science 2510.27258): every operator has a
+streaming form with an O(1)-per-token state (Metodología 1-3), and the chunked scan is built
+on segment summaries that concatenate (Metodología 4).  The state a head carries after t
+tokens is the summary of those t tokens, so:
+* the exported state must equal the oracle's summary of the prefix;
+* prefill then decode must reproduce the masked forward over the whole sequence, and end
+  in the state of the whole sequence;
+* decoding from the empty state must reproduce the forward from the first token.
+"""
+import numpy as np
+import pytest
+
+import hla_inputs
+import oracle
+import oracle.segments as seg
+
+torch = pytest.importorskip("torch")
+import higher_order_linear_chunked_b200 as hla  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+STATE_TOL = 1e-4          # fp32 state against fp64, relative to each matrix's largest entry
+OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3"]
+DEV = torch.device("cuda:0")
+
+
+def recipe(op, dtype, B, H, T, d, seed):
+    qk = "softplus" if op == "hla2n" else "scaled"
+    v = "unit" if op == "hla2n" else "scaled"
+    g = (0.9, 0.999) if op == "hla2d" else None
+    return hla_inputs.Workload(f"{op}_{dtype}_{B}x{H}x{T}x{d}", op, dtype, B, H, T, d, d, qk, v,
+                               gamma_range=g, seed=seed)
+
+
+def oracle_state(op, q, k, v, gamma):
+    """Summary-layout state of one head ([T,d] fp64 arrays) as a list of arrays in slot order."""
+    if op in ("hla2", "hla2n"):
+        s = seg.hla2_summary(q, k, v)
+        return [s["S"], s["C"], s["S"] @ s["C"] - s["G"], s["m"], s["S"] @ s["m"] - s["h"]]
+    if op == "hla2d":
+        s = seg.hla2_summary(q, k, v, gamma=gamma)
+        return [s["S"], s["C"], s["G"], s["Khat"], s["m"], s["h"], np.array([float(s["rho"])])]
+    if op == "ahla":
+        s = seg.ahla_summary(q, k, v)
+        return [s["P"], s["E"], s["D"]]
+    s = seg.hla3_summary(q, k, v)
+    return [s["S"], s["Q2"], s["P"], s["F"], s["X"], s["Z"]]
+
+
+def split_state(op, x, d):
+    """The GPU state vector of one head, cut into the same slots."""
+    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6}[op]
+    nvec = 2 if op in ("hla2", "hla2n", "hla2d") else 0
+    out = [x[i * d * d:(i + 1) * d * d].reshape(d, d) for i in range(nmat)]
+    base = nmat * d * d
+    out += [x[base + i * d: base + (i + 1) * d] for i in range(nvec)]
+    if op == "hla2d":
+        out.append(x[base + 2 * d: base + 2 * d + 1])
+    return out
+
+
+def assert_state_close(op, got, want, d):
+    for a, b in zip(split_state(op, got, d), want):
+        scale = max(np.abs(b).max(), 1e-30)
+        assert np.abs(np.asarray(a, np.float64) - b).max() / scale < STATE_TOL
+
+
+def gpu(x):
+    return x.to(DEV) if x is not None else None
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 200])
+def test_exported_state_is_the_prefix_summary(op, dtype, d, T):
+    w = recipe(op, dtype, 1, 2, T, d, seed=T + d)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    st = hla.state(op, gpu(q), gpu(k), gpu(v), gamma=gpu(g)).cpu().numpy()
+    for h in range(2):
+        want = oracle_state(op, q[0, h].double().numpy(), k[0, h].double().numpy(), v[0, h].double().numpy(),
+                            float(g[h]) if g is not None else None)
+        assert_state_close(op, st[0, h], want, d)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T0,T1", [(64, 5), (130, 17), (1, 3)])
+def test_prefill_then_decode_equals_the_forward(op, dtype, T0, T1):
+    d = 64 if dtype == "bf16" else 32
+    w = recipe(op, dtype, 2, 3, T0 + T1, d, seed=T0 * 3 + T1)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    st = hla.state(op, gpu(q[:, :, :T0].contiguous()), gpu(k[:, :, :T0].contiguous()),
+                   gpu(v[:, :, :T0].contiguous()), gamma=gpu(g))
+    outs = []
+    for t in range(T0, T0 + T1):
+        outs.append(hla.step(op, st, gpu(q[:, :, t].contiguous()), gpu(k[:, :, t].contiguous()),
+                             gpu(v[:, :, t].contiguous()), gamma=gpu(g), eps=w.eps))
+    torch.cuda.synchronize()
+    o = torch.stack(outs, dim=2).cpu()
+    ref = oracle.recur(op, q, k, v, gamma=g, eps=w.eps)[:, :, T0:]
+    assert oracle.max_row_rel_err(o, ref) <= TOL[dtype]
+    whole = hla.state(op, gpu(q), gpu(k), gpu(v), gamma=gpu(g)).cpu().numpy()
+    got = st.cpu().numpy()
+    for b in range(2):
+        for h in range(3):
+            want = split_state(op, whole[b, h], d)
+            assert_state_close(op, got[b, h], [np.asarray(x, np.float64) for x in want], d)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_decode_from_the_empty_state(op):
+    d, T = 32, 40
+    w = recipe(op, "f32", 1, 2, T, d, seed=11)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    st = hla.new_state(op, 1, 2, d)
+    outs = [hla.step(op, st, gpu(q[:, :, t].contiguous()), gpu(k[:, :, t].contiguous()),
+                     gpu(v[:, :, t].contiguous()), gamma=gpu(g), eps=w.eps) for t in range(T)]
+    torch.cuda.synchronize()
+    o = torch.stack(outs, dim=2).cpu()
+    assert oracle.max_row_rel_err(o, oracle.recur(op, q, k, v, gamma=g, eps=w.eps)) <= TOL["f32"]
+
+
+def test_normalised_decay_state_and_steps():
+    """hla2n with gamma: the decayed state form and the ratio-normalised output."""
+    d, T0, T1 = 32, 70, 6
+    w = hla_inputs.Workload("x", "hla2n", "f32", 1, 2, T0 + T1, d, d, "softplus", "unit",
+                            gamma_range=(0.9, 0.999), seed=5)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    st = hla.state("hla2n", gpu(q[:, :, :T0].contiguous()), gpu(k[:, :, :T0].contiguous()),
+                   gpu(v[:, :, :T0].contiguous()), gamma=gpu(g))
+    assert st.shape[-1] == hla.state_floats("hla2n", d, d, decayed=True)
+    outs = [hla.step("hla2n", st, gpu(q[:, :, t].contiguous()), gpu(k[:, :, t].contiguous()),
+                     gpu(v[:, :, t].contiguous()), gamma=gpu(g), eps=w.eps) for t in range(T0, T0 + T1)]
+    torch.cuda.synchronize()
+    o = torch.stack(outs, dim=2).cpu()
+    ref = np.stack([oracle.hla2_run(q[0, h], k[0, h], v[0, h], gamma=float(g[h]), normalized=True,
+                                    eps=w.eps)[0] for h in range(2)])[None, :, T0:]
+    assert oracle.max_row_rel_err(o, ref) <= TOL["f32"]
