@@ -34,7 +34,7 @@ _SRC = os.path.join(_HERE, "hla_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4}
+OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4, "hla2u": 5}
 
 
 def build(force: bool = False) -> str:
@@ -61,6 +61,8 @@ def _load():
         lib.oracle_ahla_head.restype = None
         lib.oracle_hla3_head.argtypes = [dp, dp, dp, i, i, i, dp, dp, dp, dp]
         lib.oracle_hla3_head.restype = None
+        lib.oracle_hla2u_head.argtypes = [dp, dp, dp, i, i, i, dp, dp, dp]
+        lib.oracle_hla2u_head.restype = None
         _lib = lib
     return _lib
 
@@ -85,7 +87,8 @@ def recur(op: str, q, k, v, gamma=None, eps: float = 1e-6, nthreads: Optional[in
 
     op: "hla2" (Metodología 1 output), "hla2n" (ratio-normalised, Metodología 1
     "Normalización"), "hla2d" (decayed, Contribuciones 2; gamma [H]), "ahla"
-    (Metodología 2), "hla3" (Metodología 3).
+    (Metodología 2), "hla3" (Metodología 3), "hla2u" (the unmasked configuration of
+    Contribuciones 2: o_t = q_t^T S_t C_t).
     """
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -158,6 +161,21 @@ def hla3_run(q, k, v, state=None, want_output: bool = True):
     o = np.zeros((T, dv)) if want_output else None
     lib.oracle_hla3_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, _ptr(st["S"]), _ptr(st["P"]),
                          _ptr(st["F"]), _ptr(o))
+    return o, st
+
+
+def hla2u_run(q, k, v, state=None, want_output: bool = True):
+    """Unmasked second-order recurrence over one head from ``state`` = dict(S, C) or None."""
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, d = q.shape
+    dv = v.shape[1]
+    if state is None:
+        st = dict(S=np.zeros((d, d)), C=np.zeros((d, dv)))
+    else:
+        st = {key: np.array(val, dtype=np.float64, copy=True, order="C") for key, val in state.items()}
+    o = np.zeros((T, dv)) if want_output else None
+    lib.oracle_hla2u_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, _ptr(st["S"]), _ptr(st["C"]), _ptr(o))
     return o, st
 
 

@@ -82,6 +82,16 @@ def hla2_decay(q, k, v, gamma, normalized: bool = False, eps: float = 1e-6):
     return out
 
 
+def hla2u(q, k, v):
+    """Second order without the inner mask (Contribuciones 2, unmasked configuration):
+    o_t = q_t^T S_t C_t = sum_{j<=t} sum_{i<=t} (q_t.k_i)(q_j.k_i) v_j.  In matrix form
+    W = L (.) (A A*^T) with A = L (.) Q K^T and A* = Q K^T (j's scores unmasked), O = W V."""
+    A = scores(q, k)
+    Astar = _f64(q) @ np.swapaxes(_f64(k), -1, -2)
+    W = _tril(A @ np.swapaxes(Astar, -1, -2))
+    return W @ _f64(v)
+
+
 def ahla(q, k, v):
     """AHLA (Metodología 2): o_t = sum_{j<=t} (q_t.k_j) sum_{i<=j} (q_j.k_i) v_i, i.e. O = A (A V)."""
     A = scores(q, k)
@@ -107,4 +117,6 @@ def forward(op: str, q, k, v, gamma=None, eps: float = 1e-6):
         return ahla(q, k, v)
     if op == "hla3":
         return hla3(q, k, v)
+    if op == "hla2u":
+        return hla2u(q, k, v)
     raise ValueError(op)

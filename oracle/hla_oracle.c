@@ -18,6 +18,9 @@
  *     page gives no decayed formula; the reading used is: before each token's
  *     update, every state (S, C, G, m, h) is multiplied by the head's gamma,
  *     then the undecayed updates run on the scaled values.
+ *   - Contribuciones 2, the unmasked configuration: the naive product that
+ *     the masked form corrects, o_t = q_t^T S^K_t C^QV_t (Metodología 1 names
+ *     G_t as the correction of the future terms it includes).
  *   - Metodología 2 (AHLA): operator Q (K^T Q)(K^T V); streaming state
  *     P^KV_t = sum k v^T and E_t, with o_t = q_t^T E_t.
  *   - Metodología 3 (third order): A A^T A with A = Q K^T, masked, i.e.
@@ -111,6 +114,42 @@ void oracle_hla2_head(const double* q, const double* k, const double* v,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Second order, unmasked inside the prefix.                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One head.  State in/out: S[d][d] = sum k k^T and C[d][dv] = sum q v^T, both
+ * inclusive of t.  o_t = q_t^T S_t C_t, evaluated as (q_t^T S_t) C_t.
+ */
+void oracle_hla2u_head(const double* q, const double* k, const double* v,
+                       int T, int d, int dv, double* S, double* C, double* o)
+{
+    double* qS = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int t = 0; t < T; ++t) {
+        const double* qt = q + (size_t)t * d;
+        const double* kt = k + (size_t)t * d;
+        const double* vt = v + (size_t)t * dv;
+        for (int a = 0; a < d; ++a) {
+            for (int b = 0; b < d; ++b) S[(size_t)a * d + b] += kt[a] * kt[b];
+            for (int c = 0; c < dv; ++c) C[(size_t)a * dv + c] += qt[a] * vt[c];
+        }
+        if (!o) continue;
+        for (int b = 0; b < d; ++b) {
+            double s = 0.0;
+            for (int a = 0; a < d; ++a) s += qt[a] * S[(size_t)a * d + b];
+            qS[b] = s;
+        }
+        double* ot = o + (size_t)t * dv;
+        for (int c = 0; c < dv; ++c) {
+            double s = 0.0;
+            for (int a = 0; a < d; ++a) s += qS[a] * C[(size_t)a * dv + c];
+            ot[c] = s;
+        }
+    }
+    free(qS);
+}
+
+/* ------------------------------------------------------------------------ */
 /* AHLA.                                                                     */
 /* ------------------------------------------------------------------------ */
 
@@ -197,7 +236,7 @@ void oracle_hla3_head(const double* q, const double* k, const double* v,
 /* Many heads on host threads (full-size workloads, CPU baseline).           */
 /* ------------------------------------------------------------------------ */
 
-enum { OP_HLA2 = 0, OP_HLA2N = 1, OP_HLA2D = 2, OP_AHLA = 3, OP_HLA3 = 4 };
+enum { OP_HLA2 = 0, OP_HLA2N = 1, OP_HLA2D = 2, OP_AHLA = 3, OP_HLA3 = 4, OP_HLA2U = 5 };
 
 typedef struct {
     int op, BH, H, T, d, dv;
@@ -236,6 +275,9 @@ static void run_head(job_t* J, int bh)
     case OP_HLA3:
         oracle_hla3_head(q, k, v, T, d, dv, a, b, c, o);
         break;
+    case OP_HLA2U:
+        oracle_hla2u_head(q, k, v, T, d, dv, a, b, o);
+        break;
     }
     free(a); free(b); free(c); free(m); free(h);
 }
@@ -264,7 +306,7 @@ int oracle_forward(int op, int B, int H, int T, int d, int dv,
 {
     if (B < 1 || H < 1 || T < 0 || d < 1 || dv < 1 || !q || !k || !v || !o) return -1;
     if (op == OP_HLA2D && !gamma) return -1;
-    if (op < OP_HLA2 || op > OP_HLA3) return -1;
+    if (op < OP_HLA2 || op > OP_HLA2U) return -1;
     job_t J;
     J.op = op; J.BH = B * H; J.H = H; J.T = T; J.d = d; J.dv = dv;
     J.q = q; J.k = k; J.v = v; J.gamma = gamma; J.eps = eps; J.o = o; J.next = 0;

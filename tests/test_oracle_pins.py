@@ -171,7 +171,7 @@ def test_literal_sums(seed):
 # recurrence vs masked-matrix definition (exactness claim)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u"])
 @pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (1, 2, 17, 3, 2), (2, 2, 64, 4, 4), (1, 1, 40, 1, 3)])
 def test_recur_equals_brute(op, shape):
     B, H, T, d, dv = shape
@@ -393,3 +393,47 @@ def test_metric():
     ref = np.array([[[[3.0, 4.0], [1.0, 0.0]]]])
     o = np.array([[[[3.0, 4.5], [1.0, 0.0]]]])
     assert abs(oracle.max_row_rel_err(o, ref) - 0.1) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# the unmasked configuration (Contribuciones 2): o_t = q_t^T S_t C_t
+# ---------------------------------------------------------------------------
+
+def test_unmasked_literal_double_sum():
+    rng = np.random.default_rng(21)
+    T, d, dv = 9, 3, 2
+    q, k, v = rng.standard_normal((T, d)), rng.standard_normal((T, d)), rng.standard_normal((T, dv))
+    want = np.zeros((T, dv))
+    for t in range(T):
+        for i in range(t + 1):
+            for j in range(t + 1):
+                want[t] += _dot(q[t], k[i]) * _dot(q[j], k[i]) * v[j]
+    got = oracle.recur("hla2u", one_head(q), one_head(k), one_head(v))[0, 0]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(brute.hla2u(q, k, v), want, rtol=1e-12, atol=1e-12)
+
+
+def test_unmasked_minus_masked_is_the_cross_summary():
+    """Metodología 1: G_t corrects the future terms of the naive product, so the unmasked
+    output minus the masked one is q_t^T G_t, with G from the masked recurrence's own state."""
+    rng = np.random.default_rng(22)
+    T, d, dv = 30, 4, 3
+    q, k, v = rng.standard_normal((T, d)), rng.standard_normal((T, d)), rng.standard_normal((T, dv))
+    ou = oracle.recur("hla2u", one_head(q), one_head(k), one_head(v))[0, 0]
+    om = oracle.recur("hla2", one_head(q), one_head(k), one_head(v))[0, 0]
+    st = None
+    for t in range(T):
+        _, st = oracle.hla2_run(q[t:t + 1], k[t:t + 1], v[t:t + 1], st, want_output=False)
+        np.testing.assert_allclose(ou[t] - om[t], q[t] @ st["G"], rtol=1e-10, atol=1e-12)
+
+
+def test_unmasked_single_token_and_planted_mask():
+    rng = np.random.default_rng(23)
+    q, k, v = rng.standard_normal((1, 5)), rng.standard_normal((1, 5)), rng.standard_normal((1, 2))
+    o = oracle.recur("hla2u", one_head(q), one_head(k), one_head(v))[0, 0]
+    np.testing.assert_allclose(o[0], (q[0] @ k[0]) ** 2 * v[0], rtol=1e-13)
+    # a planted mistake: masking the j side too gives the masked operator, which the pins reject
+    T = 12
+    q, k, v = rng.standard_normal((T, 3)), rng.standard_normal((T, 3)), rng.standard_normal((T, 2))
+    assert oracle.max_row_rel_err(brute.hla2(q, k, v), oracle.recur("hla2u", one_head(q), one_head(k),
+                                                                    one_head(v))[0, 0]) > 1e-3
