@@ -170,6 +170,10 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     if w.op == "ahla":
         # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
         flops = 6 * c * D + 4 * D * D
+    elif w.op == "hla2u":
+        # per token: A* = Q K^T, P Q^T, A K, W V (2cD each); A A*^T (2c^2); Q S0, Q (S0 C0),
+        # (A K) C0 (2D^2 each); S0 C0 once per chunk (2D^3 / c)
+        flops = 8 * c * D + 2 * c * c + 6 * D * D + 2 * D ** 3 // c
     elif w.op == "hla2d" and path == "tc":
         # per token: A* = Q K^T, Gam P Q^T, H K, W V (2cD each); Q S0, Q G0, Q M0, (Gam H K) C0
         # (2D^2 each); H A*^T and A A^T (2c^2 each)

@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(_HERE, "libhla.so")
 
 HLA_OK = 0
 HLA_F32, HLA_BF16 = 0, 1
-OP_HLA2, OP_HLA2_NORM, OP_AHLA, OP_HLA3 = 0, 1, 2, 3
+OP_HLA2, OP_HLA2_NORM, OP_AHLA, OP_HLA3, OP_HLA2_UNMASKED = 0, 1, 2, 3, 4
 
 STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_ALIGN", 4: "HLA_ERR_DTYPE",
                 5: "HLA_ERR_UNSUPPORTED", 6: "HLA_ERR_WORKSPACE", 7: "HLA_ERR_CUDA", 8: "HLA_ERR_TIMEOUT"}
@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_
 EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
            "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
            "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
-           "hla_state_kernel_launches", "hla_state", "hla_step")
+           "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked")
 
 
 class HLAError(RuntimeError):
@@ -65,7 +65,7 @@ def load_library(path: Optional[str] = None):
     lib.hla_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
     lib.hla_workspace_bytes.restype = sz
     common = [vp, vp, vp, vp, i, i, i, i, i, i, vp]
-    for name in ("hla2_forward", "ahla_forward", "hla3_forward"):
+    for name in ("hla2_forward", "ahla_forward", "hla3_forward", "hla2_forward_unmasked"):
         fn = getattr(lib, name)
         fn.argtypes = common + [vp, sz, vp]
         fn.restype = i
@@ -185,6 +185,8 @@ def _call(op: int, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=N
         rc = lib.ahla_forward(*args, *ws)
     elif op == OP_HLA3:
         rc = lib.hla3_forward(*args, *ws)
+    elif op == OP_HLA2_UNMASKED:
+        rc = lib.hla2_forward_unmasked(*args, *ws)
     else:
         raise ValueError(op)
     if rc != HLA_OK:
@@ -212,8 +214,13 @@ def hla3(q, k, v, out=None, workspace=None, stream=None):
     return _call(OP_HLA3, q, k, v, out=out, workspace=workspace, stream=stream)
 
 
+def hla2_unmasked(q, k, v, out=None, workspace=None, stream=None):
+    """Unmasked second-order forward, o_t = q_t^T S_t C_t."""
+    return _call(OP_HLA2_UNMASKED, q, k, v, out=out, workspace=workspace, stream=stream)
+
+
 def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):
-    """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3"."""
+    """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3", "hla2u"."""
     if op_name == "hla2":
         return hla2(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "hla2n":
@@ -226,10 +233,13 @@ def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, work
         return ahla(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "hla3":
         return hla3(q, k, v, out=out, workspace=workspace, stream=stream)
+    if op_name == "hla2u":
+        return hla2_unmasked(q, k, v, out=out, workspace=workspace, stream=stream)
     raise ValueError(op_name)
 
 
-OP_CODES = {"hla2": OP_HLA2, "hla2n": OP_HLA2_NORM, "hla2d": OP_HLA2, "ahla": OP_AHLA, "hla3": OP_HLA3}
+OP_CODES = {"hla2": OP_HLA2, "hla2n": OP_HLA2_NORM, "hla2d": OP_HLA2, "ahla": OP_AHLA, "hla3": OP_HLA3,
+            "hla2u": OP_HLA2_UNMASKED}
 
 
 def read_device_status(workspace, stream=None) -> int:

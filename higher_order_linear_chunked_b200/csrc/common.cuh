@@ -13,6 +13,7 @@ enum Op : int {
     OP_HLA2D = 1,  // second order with per-head decay
     OP_AHLA = 2,
     OP_HLA3 = 3,
+    OP_HLA2U = 4,  // second order without the inner mask (o_t = q_t^T S_t C_t)
 };
 
 // Device status word values (first int of every workspace).

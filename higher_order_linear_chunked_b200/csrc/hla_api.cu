@@ -37,12 +37,17 @@ Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H,
     r.bf16 = (dtype == HLA_BF16);
     if (op == HLA_OP_HLA2 || op == HLA_OP_HLA2_NORM) r.op = decayed ? hla::OP_HLA2D : hla::OP_HLA2;
     else if (op == HLA_OP_AHLA) r.op = hla::OP_AHLA;
+    else if (op == HLA_OP_HLA2_UNMASKED) r.op = hla::OP_HLA2U;
     else r.op = hla::OP_HLA3;
     r.B = B; r.H = H; r.T = T; r.d = d; r.dv = dv;
     return r;
 }
 
 bool use_tc(const Request& r) { return hla::tc::supported(r.op, r.norm, r.bf16, r.d); }
+
+// Ops with no decayed form.
+bool undecayed_only(hla_op_t op) { return op == HLA_OP_AHLA || op == HLA_OP_HLA3 || op == HLA_OP_HLA2_UNMASKED; }
+bool valid_op(hla_op_t op) { return op >= HLA_OP_HLA2 && op <= HLA_OP_HLA2_UNMASKED; }
 
 size_t workspace_for(const Request& r) {
     const int BH = r.B * r.H;
@@ -53,11 +58,11 @@ size_t workspace_for(const Request& r) {
 hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, float* o, int B, int H, int T,
                      int d, int dv, hla_dtype_t dtype, const float* gamma, float eps, void* workspace,
                      size_t workspace_bytes, void* stream, void* const* phase_events = nullptr) {
-    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!valid_op(op)) return HLA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, T, d, dv);
     if (s != HLA_OK) return s;
-    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (gamma && undecayed_only(op)) return HLA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HLA_ERR_ALIGN;
     if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
     const Request r = make_request(op, gamma != nullptr, dtype, B, H, T, d, dv);
@@ -107,9 +112,9 @@ const char* hla_status_str(hla_status_t s) {
 }
 
 size_t hla_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
-    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return 0;
+    if (!valid_op(op)) return 0;
     if (check_shape(dtype, B, H, T, d, dv) != HLA_OK) return 0;
-    if (decayed && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return 0;
+    if (decayed && undecayed_only(op)) return 0;
     return workspace_for(make_request(op, decayed != 0, dtype, B, H, T, d, dv));
 }
 
@@ -150,6 +155,13 @@ hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
     return forward(HLA_OP_HLA3, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace, workspace_bytes, stream);
 }
 
+hla_status_t hla2_forward_unmasked(const void* q, const void* k, const void* v, float* o, int B, int H, int T,
+                                   int d, int dv, hla_dtype_t dtype, const float* gamma, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+    return forward(HLA_OP_HLA2_UNMASKED, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace,
+                   workspace_bytes, stream);
+}
+
 hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, const void* v, float* o, int B,
                                   int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
                                   void* workspace, size_t workspace_bytes, void* stream,
@@ -159,9 +171,9 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
 }
 
 size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv) {
-    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return 0;
+    if (!valid_op(op)) return 0;
     if (d != dv || (d != 32 && d != 64)) return 0;
-    if (decayed && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return 0;
+    if (decayed && undecayed_only(op)) return 0;
     return hla::simt::summary_floats(make_request(op, decayed != 0, HLA_F32, 1, 1, 1, d, dv).op, d);
 }
 
@@ -178,11 +190,11 @@ int hla_state_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B
 hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v, float* state, int B, int H, int T,
                        int d, int dv, hla_dtype_t dtype, const float* gamma, void* workspace,
                        size_t workspace_bytes, void* stream) {
-    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!valid_op(op)) return HLA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !state) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, T, d, dv);
     if (s != HLA_OK) return s;
-    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (gamma && undecayed_only(op)) return HLA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state)) return HLA_ERR_ALIGN;
     if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
     const Request r = make_request(op, gamma != nullptr, dtype, B, H, T, d, dv);
@@ -198,11 +210,11 @@ hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v,
 
 hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, const void* v, float* o, int B, int H,
                       int d, int dv, hla_dtype_t dtype, const float* gamma, float eps, void* stream) {
-    if (op < HLA_OP_HLA2 || op > HLA_OP_HLA3) return HLA_ERR_UNSUPPORTED;
+    if (!valid_op(op)) return HLA_ERR_UNSUPPORTED;
     if (!state || !q || !k || !v || !o) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, 1, d, dv);
     if (s != HLA_OK) return s;
-    if (gamma && (op == HLA_OP_AHLA || op == HLA_OP_HLA3)) return HLA_ERR_UNSUPPORTED;
+    if (gamma && undecayed_only(op)) return HLA_ERR_UNSUPPORTED;
     if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HLA_ERR_ALIGN;
     if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
     const Request r = make_request(op, gamma != nullptr, dtype, B, H, 1, d, dv);

@@ -21,6 +21,8 @@
 //   third order    summary  S, Q2 = Q^T Q, P, X = Q^T (A V), Z = K^T (A^T Q),
 //                           F = K^T (A^T (A V));
 //                  output   W as above, O = Q F0 + W (Q P0 + A V)
+//   unmasked       summary  S = K^T K, C = Q^T V;  combine S, C add;
+//   second order   output   W = L (.) (Q S0 Q^T + A A*^T), O = Q (S0 C0) + W V + (A K) C0
 #include "common.cuh"
 #include "simt.h"
 
@@ -42,7 +44,7 @@ struct Dim {
 template <int OP, int D>
 struct Sum {
     static constexpr int DD = D * D;
-    static constexpr int NMAT = OP == OP_HLA3 ? 6 : OP == OP_HLA2D ? 4 : 3;
+    static constexpr int NMAT = OP == OP_HLA3 ? 6 : OP == OP_HLA2D ? 4 : OP == OP_HLA2U ? 2 : 3;
     static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D) ? 2 : 0;
     static constexpr int VEC0 = NMAT * DD;
     static constexpr int SCAL = VEC0 + NVEC * D;
@@ -55,6 +57,7 @@ struct Sum {
 //   OP_HLA2D: S=0 C=1 G=2 Khat=3 ; m=0 h=1 ; scalar rho
 //   OP_AHLA : P=0 E=1 Dm=2
 //   OP_HLA3 : S=0 Q2=1 P=2 F=3 X=4 Z=5
+//   OP_HLA2U: S=0 C=1
 
 size_t summary_floats(int op, int d) {
     switch (op) {
@@ -62,6 +65,7 @@ size_t summary_floats(int op, int d) {
     case OP_HLA2D: return d == 32 ? Sum<OP_HLA2D, 32>::SIZE : Sum<OP_HLA2D, 64>::SIZE;
     case OP_AHLA: return d == 32 ? Sum<OP_AHLA, 32>::SIZE : Sum<OP_AHLA, 64>::SIZE;
     case OP_HLA3: return d == 32 ? Sum<OP_HLA3, 32>::SIZE : Sum<OP_HLA3, 64>::SIZE;
+    case OP_HLA2U: return d == 32 ? Sum<OP_HLA2U, 32>::SIZE : Sum<OP_HLA2U, 64>::SIZE;
     }
     return 0;
 }
@@ -227,9 +231,10 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     }
     __syncthreads();
     // A* = Q K^T (masked to A = L (.) A* except for the decayed op, which needs both parts)
-    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
-        As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
-    });
+    if (OP != OP_HLA2U)
+        mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
+            As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
+        });
     __syncthreads();
 
     auto store_mat = [&](int slot) {
@@ -281,6 +286,9 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
             out[S::vec(1) + a] = sh;                                     // h = K^T u
         }
         if (threadIdx.x == 0) out[S::SCAL] = gpow(g, len);               // rho = gamma^len
+    } else if (OP == OP_HLA2U) {
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(0));        // S = K^T K
+        mm<D, D, C>(TileT{Qs, LD}, Tile{Vs, LD}, Zero{}, store_mat(1));        // C = Q^T V
     } else if (OP == OP_AHLA) {
         mm<D, D, C>(TileT{Ks, LD}, Tile{Vs, LD}, Zero{}, store_mat(0));        // P = K^T V
         mm<D, D, C>(TileT{Ks, LD}, Tile{Qs, LD}, Zero{}, store_mat(2));        // Dm = K^T Q
@@ -348,6 +356,9 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
             out[S::vec(1) + a] = rb * A[S::vec(1) + a] + B[S::vec(1) + a] + rb * s;
         }
         if (threadIdx.x == 0) out[S::SCAL] = A[S::SCAL] * rb;
+    } else if (OP == OP_HLA2U) {
+        add2(0);
+        add2(1);
     } else if (OP == OP_AHLA) {
         add2(0);
         add2(2);
@@ -452,6 +463,9 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
         }
         g = gamma[bh % H];
         for (int j = threadIdx.x; j <= C; j += blockDim.x) gp[j] = gpow(g, j);
+    } else if (OP == OP_HLA2U) {
+        load_mat<D>(M0, pre + S::mat(0));   // S0
+        load_mat<D>(M1, pre + S::mat(1));   // C0
     } else if (OP == OP_AHLA) {
         load_mat<D>(M0, pre + S::mat(0));   // P0
         load_mat<D>(M1, pre + S::mat(1));   // E0
@@ -462,10 +476,12 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     }
     __syncthreads();
     mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
-        As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
+        As[r * LDC + c] = (OP == OP_HLA2D || OP == OP_HLA2U || c <= r) ? x : 0.f;
     });
-    if (OP == OP_HLA2 || OP == OP_HLA3)
+    if (OP == OP_HLA2 || OP == OP_HLA3 || OP == OP_HLA2U)
         mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, Put{Ps, LD});                      // P = Q S0
+    if (OP == OP_HLA2U)
+        mm<D, D, D>(Tile{M0, LD}, Tile{M1, LD}, Zero{}, Put{M2, LD});                      // S0 C0
     if (OP == OP_HLA2D)
         mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, [&](int r, int c, float x) {         // P~ = Gamma Q S0
             Ps[r * LD + c] = gp[r + 1] * x;
@@ -520,6 +536,17 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
         mm3<C, D, C, D, D>(Tile{Ws, LDC}, Tile{Vs, LD},
                            [&](int r, int c) { return gp[r + 1] * Ys[r * LD + c]; }, Tile{M1, LD},
                            [&](int r, int c) { return -gp[r + 1] * Qs[r * LD + c]; }, Tile{M2, LD}, Zero{}, emit);
+    } else if (OP == OP_HLA2U) {
+        // As holds A* = Q K^T unmasked; A = L (.) A*.
+        auto Am = [&](int r, int c) { return c <= r ? As[r * LDC + c] : 0.f; };
+        // W = L (.) (P Q^T + A A*^T): the pair weight summed over every key up to the query's token
+        mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Am, TileT{As, LDC}, Zero{},
+                        [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
+        mm<C, D, C>(Am, Tile{Ks, LD}, Zero{}, Put{Ys, LD});                                    // Y = A K
+        __syncthreads();
+        // O = Q (S0 C0) + W V + Y C0
+        mm3<C, D, D, C, D>(Tile{Qs, LD}, Tile{M2, LD}, Tile{Ws, LDC}, Tile{Vs, LD}, Tile{Ys, LD}, Tile{M1, LD},
+                           Zero{}, emit);
     } else if (OP == OP_AHLA) {
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M0, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y = Q P0 + A V
         __syncthreads();
@@ -593,6 +620,7 @@ cudaError_t scan(int op, int d, float* sums, int NCp, int BH, cudaStream_t st) {
     case OP_HLA2D: return d == 32 ? scan_levels<OP_HLA2D, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA2D, 64>(sums, NCp, BH, st);
     case OP_AHLA: return d == 32 ? scan_levels<OP_AHLA, 32>(sums, NCp, BH, st) : scan_levels<OP_AHLA, 64>(sums, NCp, BH, st);
     case OP_HLA3: return d == 32 ? scan_levels<OP_HLA3, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA3, 64>(sums, NCp, BH, st);
+    case OP_HLA2U: return d == 32 ? scan_levels<OP_HLA2U, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA2U, 64>(sums, NCp, BH, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -639,6 +667,7 @@ static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, 
                     : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     case OP_AHLA: return run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     case OP_HLA3: return run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     }
     return cudaErrorInvalidValue;
 }
@@ -701,6 +730,7 @@ static cudaError_t state_op(int op, const void* q, const void* k, const void* v,
     case OP_HLA2D: return state_run<OP_HLA2D, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_AHLA: return state_run<OP_AHLA, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_HLA3: return state_run<OP_HLA3, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_HLA2U: return state_run<OP_HLA2U, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -730,6 +760,7 @@ int state_launches(int T) {
 //   AHLA                   P += k v^T;  Dm += k q^T;  y = q^T P;  E += k y^T;  o = q^T E
 //   third order            S += k k^T;  P += k v^T;  Q2 += q q^T;  a = S q;  b = q^T P;
 //                          F += a b^T;  X += q b^T;  Z += a q^T;  o = q^T F
+//   unmasked               S += k k^T;  C += q v^T;  o = (q^T S) C
 // S is symmetric, so every product with a vector reads matrix columns: thread j of a group
 // walks rows i, and four groups of D threads split the rows (partial sums in shared memory).
 // The head's state is staged in shared memory (every load in flight at once), updated there
@@ -850,6 +881,17 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
             }
             o[(size_t)bh * D + tid] = NORM ? t / den : t;
         }
+    } else if (OP == OP_HLA2U) {
+        float* Sm = st + S::mat(0); float* Cm = st + S::mat(1);
+        for (int e = tid; e < DD; e += NT) {
+            const int i = e / D, j = e % D;
+            Sm[e] = fmaf(ks[i], ks[j], Sm[e]);
+            Cm[e] = fmaf(qs[i], vs[j], Cm[e]);
+        }
+        __syncthreads();
+        col_dot<D>(Sm, qs, part, a);                            // a = q^T S
+        col_dot<D>(Cm, a, part, b);                             // b = (q^T S) C
+        if (tid < D) o[(size_t)bh * D + tid] = b[tid];
     } else if (OP == OP_AHLA) {
         float* P = st + S::mat(0); float* E = st + S::mat(1); float* Dm = st + S::mat(2);
         for (int e = tid; e < DD; e += NT) {
@@ -912,6 +954,7 @@ static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const v
                     : step_launch<OP_HLA2D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_AHLA: return step_launch<OP_AHLA, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA3: return step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA2U: return step_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -17,6 +17,10 @@
  *                           o_t = sum_{j<=t} (q_t.k_j) sum_{i<=j} (q_j.k_i) v_i.
  *   hla3_forward            Metodología 3: third order A A^T A, masked:
  *                           O = (M A) V, M = L (.) (A A^T), A = L (.) Q K^T.
+ *   hla2_forward_unmasked   Contribuciones 2, the unmasked configuration: the
+ *                           naive product the cross summary G_t corrects,
+ *                           o_t = q_t^T S^K_t C^QV_t
+ *                               = sum_{j<=t} sum_{i<=t} (q_t.k_i)(q_j.k_i) v_j.
  *
  * The mask L includes the diagonal (j <= t).  All four are computed with the
  * chunk-parallel scheme of Metodología 4: per-segment summaries, a Blelloch
@@ -76,7 +80,8 @@ typedef enum {
     HLA_OP_HLA2 = 0,       /* hla2_forward */
     HLA_OP_HLA2_NORM = 1,  /* hla2_forward_normalized */
     HLA_OP_AHLA = 2,       /* ahla_forward */
-    HLA_OP_HLA3 = 3        /* hla3_forward */
+    HLA_OP_HLA3 = 3,       /* hla3_forward */
+    HLA_OP_HLA2_UNMASKED = 4  /* hla2_forward_unmasked */
 } hla_op_t;
 
 /* Version of this ABI (bumped on any signature change). */
@@ -117,6 +122,13 @@ hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
                           int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                           const float* gamma, void* workspace, size_t workspace_bytes,
                           void* stream);
+
+/* Unmasked second-order forward, o_t = q_t^T S^K_t C^QV_t (Contribuciones 2, the unmasked
+ * configuration).  gamma must be NULL.  CUDA-core kernels for every dtype and d. */
+hla_status_t hla2_forward_unmasked(const void* q, const void* k, const void* v, float* o,
+                                   int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                   const float* gamma, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /*
  * Same computation as the four entry points above, selected by `op`, with
@@ -161,6 +173,7 @@ int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, in
  *                         gamma^t              (o_t = q_t^T (S_t C_t - G_t))
  *   AHLA                  P = sum k v^T, E, D = sum k q^T      (o_t = q_t^T E_t)
  *   third order           S, Q2 = sum q q^T, P, F, X, Z        (o_t = q_t^T F_t)
+ *   unmasked second order S, C                                 (o_t = q_t^T S_t C_t)
  * A state of zero tokens is all zeros, except rho = 1 for the decayed form.
  * The state of HLA_OP_HLA2_NORM is that of HLA_OP_HLA2.
  */

@@ -173,7 +173,7 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     st = lib.hla_state
     a = [vp(16), vp(16), vp(16), vp(16)]
     assert st(0, vp(0), *a[1:], 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 1      # NULL q
-    assert st(4, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
+    assert st(5, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
     assert st(0, *a, 0, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 2                # B = 0
     assert st(0, *a, 1, 1, 64, d, d, 7, vp(0), vp(16), 1 << 20, vp(0)) == 4                # dtype
     assert st(2, *a, 1, 1, 64, d, d, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5               # gamma + AHLA
@@ -187,6 +187,22 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert sp(0, *b, 1, 0, d, d, 0, vp(0), f(1e-6), vp(0)) == 2                            # H = 0
     assert sp(3, *b, 1, 1, 32, 32, 0, vp(16), f(1e-6), vp(0)) == 5                         # gamma + HLA-3
     assert sp(0, vp(24), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 3                # alignment
+
+
+def test_unmasked_op_sizes_and_errors(lib):
+    """The unmasked second-order op: CUDA-core kernels only, no decayed form, state (S, C)."""
+    vp = ctypes.c_void_p
+    op = hla.OP_HLA2_UNMASKED
+    assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) > 0
+    assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0          # no decay
+    assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
+    assert lib.hla_state_floats(op, 0, 64, 64) == (2 * 64 * 64 + 4 + 31) // 32 * 32
+    f = lib.hla2_forward_unmasked
+    a = [vp(16)] * 4
+    assert f(*a, 1, 1, 64, 64, 64, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5                  # gamma given
+    assert f(vp(0), *a[1:], 1, 1, 64, 64, 64, 0, vp(0), vp(16), 1 << 20, vp(0)) == 1        # NULL q
+    assert f(*a, 1, 1, 64, 48, 48, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                  # d = 48
+    assert f(*a, 1, 1, 64, 64, 64, 0, vp(0), vp(16), 64, vp(0)) == 6                       # workspace
 
 
 def test_product_path_never_touches_the_oracle():

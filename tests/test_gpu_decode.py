@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 STATE_TOL = 1e-4          # fp32 state against fp64, relative to each matrix's largest entry
-OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3"]
+OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u"]
 DEV = torch.device("cuda:0")
 
 
@@ -47,13 +47,16 @@ def oracle_state(op, q, k, v, gamma):
     if op == "ahla":
         s = seg.ahla_summary(q, k, v)
         return [s["P"], s["E"], s["D"]]
+    if op == "hla2u":
+        _, s = oracle.hla2u_run(q, k, v, want_output=False)
+        return [s["S"], s["C"]]
     s = seg.hla3_summary(q, k, v)
     return [s["S"], s["Q2"], s["P"], s["F"], s["X"], s["Z"]]
 
 
 def split_state(op, x, d):
     """The GPU state vector of one head, cut into the same slots."""
-    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6}[op]
+    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6, "hla2u": 2}[op]
     nvec = 2 if op in ("hla2", "hla2n", "hla2d") else 0
     out = [x[i * d * d:(i + 1) * d * d].reshape(d, d) for i in range(nmat)]
     base = nmat * d * d

@@ -250,3 +250,24 @@ def test_full_size_workloads(name):
         ref = oracle.recur(w.op, q[sl], k[sl], v[sl], gamma=gh, eps=w.eps)
         err = oracle.max_row_rel_err(o[sl], ref)
         assert err <= TOL[w.dtype], (name, bh, err)
+
+
+# ---------------------------------------------------------------------------
+# the unmasked configuration (CUDA-core kernels): o_t = q_t^T S_t C_t
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 333, 1000])
+def test_unmasked_parity(dtype, d, T):
+    w = recipe("hla2u", dtype, 1, 2, T, d, seed=T + 5)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    o = gpu_forward("hla2u", q, k, v, None)
+    assert oracle.max_row_rel_err(o.cpu(), reference("hla2u", q, k, v, None)) <= TOL[dtype]
+
+
+def test_unmasked_many_heads():
+    w = recipe("hla2u", "bf16", 3, 5, 97, 64, seed=4)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    o = gpu_forward("hla2u", q, k, v, None)
+    assert oracle.max_row_rel_err(o.cpu(), reference("hla2u", q, k, v, None)) <= TOL["bf16"]
