@@ -34,7 +34,7 @@ _SRC = os.path.join(_HERE, "hla_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4, "hla2u": 5}
+OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4, "hla2u": 5, "ahlan": 6, "hla3n": 7}
 
 
 def build(force: bool = False) -> str:
@@ -88,7 +88,8 @@ def recur(op: str, q, k, v, gamma=None, eps: float = 1e-6, nthreads: Optional[in
     op: "hla2" (Metodología 1 output), "hla2n" (ratio-normalised, Metodología 1
     "Normalización"), "hla2d" (decayed, Contribuciones 2; gamma [H]), "ahla"
     (Metodología 2), "hla3" (Metodología 3), "hla2u" (the unmasked configuration of
-    Contribuciones 2: o_t = q_t^T S_t C_t).
+    Contribuciones 2: o_t = q_t^T S_t C_t), "ahlan" / "hla3n" (ratio-normalised: divided by
+    the same operator on a ones value column, plus eps).
     """
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)

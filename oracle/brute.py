@@ -119,4 +119,8 @@ def forward(op: str, q, k, v, gamma=None, eps: float = 1e-6):
         return hla3(q, k, v)
     if op == "hla2u":
         return hla2u(q, k, v)
+    if op in ("ahlan", "hla3n"):
+        f = ahla if op == "ahlan" else hla3
+        ones = np.ones(_f64(q).shape[:-1] + (1,))
+        return f(q, k, v) / (f(q, k, ones) + eps)
     raise ValueError(op)

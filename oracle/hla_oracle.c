@@ -23,6 +23,11 @@
  *     G_t as the correction of the future terms it includes).
  *   - Metodología 2 (AHLA): operator Q (K^T Q)(K^T V); streaming state
  *     P^KV_t = sum k v^T and E_t, with o_t = q_t^T E_t.
+ *   - Metodología 2 also lists the AHLA streaming summaries (P^KV, m^K, E, n):
+ *     with the value column replaced by ones, P^KV becomes m^K and E becomes n.
+ *     The ratio-normalised AHLA read from that (and the ratio-normalised third
+ *     order, the same way) divides the output by the same masked operator
+ *     applied to a ones column, plus eps, as the second order does.
  *   - Metodología 3 (third order): A A^T A with A = Q K^T, masked, i.e.
  *     O = (M A) V with M = L (.) (A A^T), A = L (.) Q K^T; streaming with the
  *     prefix moments S^K_t, P^KV_t and the running sum F_t.
@@ -236,7 +241,9 @@ void oracle_hla3_head(const double* q, const double* k, const double* v,
 /* Many heads on host threads (full-size workloads, CPU baseline).           */
 /* ------------------------------------------------------------------------ */
 
-enum { OP_HLA2 = 0, OP_HLA2N = 1, OP_HLA2D = 2, OP_AHLA = 3, OP_HLA3 = 4, OP_HLA2U = 5 };
+enum { OP_HLA2 = 0, OP_HLA2N = 1, OP_HLA2D = 2, OP_AHLA = 3, OP_HLA3 = 4, OP_HLA2U = 5, OP_AHLAN = 6,
+       OP_HLA3N = 7 };
+
 
 typedef struct {
     int op, BH, H, T, d, dv;
@@ -246,6 +253,9 @@ typedef struct {
     int next;                /* next head to take (under lock) */
     pthread_mutex_t lock;
 } job_t;
+
+/* o = num / (den + eps), den the same operator run on a ones value column (one column). */
+static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, double* o);
 
 static void run_head(job_t* J, int bh)
 {
@@ -278,8 +288,31 @@ static void run_head(job_t* J, int bh)
     case OP_HLA2U:
         oracle_hla2u_head(q, k, v, T, d, dv, a, b, o);
         break;
+    case OP_AHLAN:
+        oracle_ahla_head(q, k, v, T, d, dv, b, c, o);
+        divide_by_ones_run(J, q, k, T, d, dv, o);
+        break;
+    case OP_HLA3N:
+        oracle_hla3_head(q, k, v, T, d, dv, a, b, c, o);
+        divide_by_ones_run(J, q, k, T, d, dv, o);
+        break;
     }
     free(a); free(b); free(c); free(m); free(h);
+}
+
+static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, double* o)
+{
+    double* ones = (double*)malloc(sizeof(double) * (size_t)T);
+    double* den = (double*)malloc(sizeof(double) * (size_t)T);
+    double* s1 = (double*)calloc((size_t)d * d, sizeof(double));
+    double* s2 = (double*)calloc((size_t)d, sizeof(double));
+    double* s3 = (double*)calloc((size_t)d, sizeof(double));
+    for (int t = 0; t < T; ++t) ones[t] = 1.0;
+    if (J->op == OP_AHLAN) oracle_ahla_head(q, k, ones, T, d, 1, s2, s3, den);
+    else oracle_hla3_head(q, k, ones, T, d, 1, s1, s2, s3, den);
+    for (int t = 0; t < T; ++t)
+        for (int c = 0; c < dv; ++c) o[(size_t)t * dv + c] /= den[t] + J->eps;
+    free(ones); free(den); free(s1); free(s2); free(s3);
 }
 
 static void* worker(void* arg)
@@ -306,7 +339,7 @@ int oracle_forward(int op, int B, int H, int T, int d, int dv,
 {
     if (B < 1 || H < 1 || T < 0 || d < 1 || dv < 1 || !q || !k || !v || !o) return -1;
     if (op == OP_HLA2D && !gamma) return -1;
-    if (op < OP_HLA2 || op > OP_HLA2U) return -1;
+    if (op < OP_HLA2 || op > OP_HLA3N) return -1;
     job_t J;
     J.op = op; J.BH = B * H; J.H = H; J.T = T; J.d = d; J.dv = dv;
     J.q = q; J.k = k; J.v = v; J.gamma = gamma; J.eps = eps; J.o = o; J.next = 0;

@@ -171,7 +171,7 @@ def test_literal_sums(seed):
 # recurrence vs masked-matrix definition (exactness claim)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n"])
 @pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (1, 2, 17, 3, 2), (2, 2, 64, 4, 4), (1, 1, 40, 1, 3)])
 def test_recur_equals_brute(op, shape):
     B, H, T, d, dv = shape
@@ -179,7 +179,7 @@ def test_recur_equals_brute(op, shape):
     q = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
     k = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
     v = rng.standard_normal((B, H, T, dv))
-    if op == "hla2n":
+    if op in ("hla2n", "ahlan", "hla3n"):
         q, k = np.abs(q), np.abs(k)
     g = rng.uniform(0.9, 0.999, size=H)
     r = oracle.recur(op, q, k, v, gamma=g, eps=EPS)
@@ -437,3 +437,60 @@ def test_unmasked_single_token_and_planted_mask():
     q, k, v = rng.standard_normal((T, 3)), rng.standard_normal((T, 3)), rng.standard_normal((T, 2))
     assert oracle.max_row_rel_err(brute.hla2(q, k, v), oracle.recur("hla2u", one_head(q), one_head(k),
                                                                     one_head(v))[0, 0]) > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# ratio-normalised AHLA and third order: the same operator on a ones value column
+# ---------------------------------------------------------------------------
+
+def test_normalised_ahla_literal_and_named_summaries():
+    """Metodología 2 names the AHLA summaries (P^KV, m^K, E, n).  With m^K = sum k and
+    n_t = sum_{j<=t} k_j (q_j . m^K_j), the denominator is q_t . n_t: the literal masked sum
+    of the operator with every v replaced by 1."""
+    rng = np.random.default_rng(31)
+    T, d, dv = 11, 3, 2
+    q, k = np.abs(rng.standard_normal((T, d))), np.abs(rng.standard_normal((T, d)))
+    v = rng.standard_normal((T, dv))
+    num = np.zeros((T, dv))
+    den = np.zeros(T)
+    mK = np.zeros(d)
+    n = np.zeros(d)
+    for t in range(T):
+        for j in range(t + 1):
+            for i in range(j + 1):
+                w = _dot(q[t], k[j]) * _dot(q[j], k[i])
+                num[t] += w * v[i]
+                den[t] += w
+        mK += k[t]
+        n += k[t] * _dot(q[t], mK)
+        assert abs(_dot(q[t], n) - den[t]) < 1e-12 * max(1.0, den[t])
+    got = oracle.recur("ahlan", one_head(q), one_head(k), one_head(v), eps=EPS)[0, 0]
+    np.testing.assert_allclose(got, num / (den[:, None] + EPS), rtol=1e-12)
+
+
+def test_normalised_third_order_literal():
+    rng = np.random.default_rng(32)
+    T, d, dv = 8, 3, 2
+    q, k = np.abs(rng.standard_normal((T, d))), np.abs(rng.standard_normal((T, d)))
+    v = rng.standard_normal((T, dv))
+    A = np.tril(q @ k.T)
+    M = np.tril(A @ A.T)
+    W = M @ A                                 # o = W v: the masked A A^T A weights
+    num = W @ v
+    den = W.sum(axis=1)
+    got = oracle.recur("hla3n", one_head(q), one_head(k), one_head(v), eps=EPS)[0, 0]
+    np.testing.assert_allclose(got, num / (den[:, None] + EPS), rtol=1e-12)
+
+
+@pytest.mark.parametrize("op", ["ahlan", "hla3n"])
+def test_normalised_constant_v_and_homogeneity(op):
+    rng = np.random.default_rng(33)
+    T, d = 20, 4
+    q, k = np.abs(rng.standard_normal((T, d))), np.abs(rng.standard_normal((T, d)))
+    v = np.full((T, 3), 2.5)
+    o = oracle.recur(op, one_head(q), one_head(k), one_head(v), eps=1e-12)[0, 0]
+    np.testing.assert_allclose(o, 2.5, rtol=1e-9)
+    v = rng.standard_normal((T, 3))
+    o1 = oracle.recur(op, one_head(q), one_head(k), one_head(v), eps=0.0)[0, 0]
+    o2 = oracle.recur(op, one_head(3.0 * q), one_head(k), one_head(v), eps=0.0)[0, 0]
+    np.testing.assert_allclose(o1, o2, rtol=1e-10)     # degree 0 in q (ratio of equal degrees)
