@@ -167,7 +167,7 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     """Algorithmic work of the output kernel per token ('Roofline')."""
     D = w.d
     c = 128 if path == "tc" else 64
-    if w.op == "ahla":
+    if w.op in ("ahla", "ahlan"):
         # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
         flops = 6 * c * D + 4 * D * D
     elif w.op == "hla2u":

@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(_HERE, "libhla.so")
 
 HLA_OK = 0
 HLA_F32, HLA_BF16 = 0, 1
-OP_HLA2, OP_HLA2_NORM, OP_AHLA, OP_HLA3, OP_HLA2_UNMASKED = 0, 1, 2, 3, 4
+OP_HLA2, OP_HLA2_NORM, OP_AHLA, OP_HLA3, OP_HLA2_UNMASKED, OP_AHLA_NORM, OP_HLA3_NORM = 0, 1, 2, 3, 4, 5, 6
 
 STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_ALIGN", 4: "HLA_ERR_DTYPE",
                 5: "HLA_ERR_UNSUPPORTED", 6: "HLA_ERR_WORKSPACE", 7: "HLA_ERR_CUDA", 8: "HLA_ERR_TIMEOUT"}
@@ -38,7 +38,8 @@ STATUS_NAMES = {0: "HLA_OK", 1: "HLA_ERR_NULL", 2: "HLA_ERR_SHAPE", 3: "HLA_ERR_
 EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_forward", "hla2_forward_normalized",
            "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
            "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
-           "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked")
+           "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked",
+           "ahla_forward_normalized", "hla3_forward_normalized")
 
 
 class HLAError(RuntimeError):
@@ -69,8 +70,10 @@ def load_library(path: Optional[str] = None):
         fn = getattr(lib, name)
         fn.argtypes = common + [vp, sz, vp]
         fn.restype = i
-    lib.hla2_forward_normalized.argtypes = common + [f, vp, sz, vp]
-    lib.hla2_forward_normalized.restype = i
+    for name in ("hla2_forward_normalized", "ahla_forward_normalized", "hla3_forward_normalized"):
+        fn = getattr(lib, name)
+        fn.argtypes = common + [f, vp, sz, vp]
+        fn.restype = i
     lib.hla_forward_profiled.argtypes = [i] + common + [f, vp, sz, vp, vp]
     lib.hla_forward_profiled.restype = i
     lib.hla_kernel_launches.argtypes = [i, i, i, i, i, i, i, i]
@@ -187,6 +190,10 @@ def _call(op: int, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=N
         rc = lib.hla3_forward(*args, *ws)
     elif op == OP_HLA2_UNMASKED:
         rc = lib.hla2_forward_unmasked(*args, *ws)
+    elif op == OP_AHLA_NORM:
+        rc = lib.ahla_forward_normalized(*args, ctypes.c_float(eps), *ws)
+    elif op == OP_HLA3_NORM:
+        rc = lib.hla3_forward_normalized(*args, ctypes.c_float(eps), *ws)
     else:
         raise ValueError(op)
     if rc != HLA_OK:
@@ -220,7 +227,8 @@ def hla2_unmasked(q, k, v, out=None, workspace=None, stream=None):
 
 
 def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):
-    """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3", "hla2u"."""
+    """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3", "hla2u",
+    "ahlan", "hla3n" (ratio-normalised AHLA / third order)."""
     if op_name == "hla2":
         return hla2(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "hla2n":
@@ -235,11 +243,15 @@ def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, work
         return hla3(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "hla2u":
         return hla2_unmasked(q, k, v, out=out, workspace=workspace, stream=stream)
+    if op_name == "ahlan":
+        return _call(OP_AHLA_NORM, q, k, v, eps=eps, out=out, workspace=workspace, stream=stream)
+    if op_name == "hla3n":
+        return _call(OP_HLA3_NORM, q, k, v, eps=eps, out=out, workspace=workspace, stream=stream)
     raise ValueError(op_name)
 
 
 OP_CODES = {"hla2": OP_HLA2, "hla2n": OP_HLA2_NORM, "hla2d": OP_HLA2, "ahla": OP_AHLA, "hla3": OP_HLA3,
-            "hla2u": OP_HLA2_UNMASKED}
+            "hla2u": OP_HLA2_UNMASKED, "ahlan": OP_AHLA_NORM, "hla3n": OP_HLA3_NORM}
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -33,21 +33,28 @@ hla_status_t check_shape(hla_dtype_t dtype, int B, int H, int T, int d, int dv) 
 
 Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
     Request r{};
-    r.norm = (op == HLA_OP_HLA2_NORM);
+    r.norm = (op == HLA_OP_HLA2_NORM || op == HLA_OP_AHLA_NORM || op == HLA_OP_HLA3_NORM);
     r.bf16 = (dtype == HLA_BF16);
     if (op == HLA_OP_HLA2 || op == HLA_OP_HLA2_NORM) r.op = decayed ? hla::OP_HLA2D : hla::OP_HLA2;
-    else if (op == HLA_OP_AHLA) r.op = hla::OP_AHLA;
+    else if (op == HLA_OP_AHLA || op == HLA_OP_AHLA_NORM) r.op = hla::OP_AHLA;
     else if (op == HLA_OP_HLA2_UNMASKED) r.op = hla::OP_HLA2U;
     else r.op = hla::OP_HLA3;
     r.B = B; r.H = H; r.T = T; r.d = d; r.dv = dv;
     return r;
 }
 
-bool use_tc(const Request& r) { return hla::tc::supported(r.op, r.norm, r.bf16, r.d); }
+// The tensor-core AHLA walkers carry no normaliser: ratio-normalised AHLA runs on the CUDA cores.
+bool use_tc(const Request& r) {
+    if (r.op == hla::OP_AHLA && r.norm) return false;
+    return hla::tc::supported(r.op, r.norm, r.bf16, r.d);
+}
 
 // Ops with no decayed form.
-bool undecayed_only(hla_op_t op) { return op == HLA_OP_AHLA || op == HLA_OP_HLA3 || op == HLA_OP_HLA2_UNMASKED; }
-bool valid_op(hla_op_t op) { return op >= HLA_OP_HLA2 && op <= HLA_OP_HLA2_UNMASKED; }
+bool undecayed_only(hla_op_t op) {
+    return op == HLA_OP_AHLA || op == HLA_OP_HLA3 || op == HLA_OP_HLA2_UNMASKED || op == HLA_OP_AHLA_NORM ||
+           op == HLA_OP_HLA3_NORM;
+}
+bool valid_op(hla_op_t op) { return op >= HLA_OP_HLA2 && op <= HLA_OP_HLA3_NORM; }
 
 size_t workspace_for(const Request& r) {
     const int BH = r.B * r.H;
@@ -153,6 +160,20 @@ hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
                           int dv, hla_dtype_t dtype, const float* gamma, void* workspace, size_t workspace_bytes,
                           void* stream) {
     return forward(HLA_OP_HLA3, q, k, v, o, B, H, T, d, dv, dtype, gamma, 0.f, workspace, workspace_bytes, stream);
+}
+
+hla_status_t ahla_forward_normalized(const void* q, const void* k, const void* v, float* o, int B, int H, int T,
+                                    int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return forward(HLA_OP_AHLA_NORM, q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, workspace, workspace_bytes,
+                   stream);
+}
+
+hla_status_t hla3_forward_normalized(const void* q, const void* k, const void* v, float* o, int B, int H, int T,
+                                    int d, int dv, hla_dtype_t dtype, const float* gamma, float eps,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+    return forward(HLA_OP_HLA3_NORM, q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, workspace, workspace_bytes,
+                   stream);
 }
 
 hla_status_t hla2_forward_unmasked(const void* q, const void* k, const void* v, float* o, int B, int H, int T,

@@ -16,11 +16,13 @@
 //                           den = Q r0 + W 1 (ratio-normalised)
 //   decayed        state (S, C, G, Khat, m, h, rho), rho = gamma^len, Khat = K^T K;
 //                  combine and output formulas in combine_into / k_output below
-//   AHLA           summary  P = K^T V, Dm = K^T Q, E = K^T (A V);
-//                  combine  E_AB = E_A + E_B + Dm_B P_A; output O = Q E0 + A (Q P0 + A V)
+//   AHLA           summary  P = K^T V, Dm = K^T Q, E = K^T (A V);  mK = K^T 1, n = K^T (A 1)
+//                  combine  E_AB = E_A + E_B + Dm_B P_A (n likewise, with mK for P);
+//                  output   O = Q E0 + A (Q P0 + A V);  ratio-normalised: den = Q n0 + A (Q mK0 + A 1)
 //   third order    summary  S, Q2 = Q^T Q, P, X = Q^T (A V), Z = K^T (A^T Q),
 //                           F = K^T (A^T (A V));
-//                  output   W as above, O = Q F0 + W (Q P0 + A V)
+//                  output   W as above, O = Q F0 + W (Q P0 + A V);  with V replaced by a ones
+//                           column: vectors mK, X1, F1 and den = Q F1_0 + W (Q mK0 + A 1)
 //   unmasked       summary  S = K^T K, C = Q^T V;  combine S, C add;
 //   second order   output   W = L (.) (Q S0 Q^T + A A*^T), O = Q (S0 C0) + W V + (A K) C0
 #include "common.cuh"
@@ -45,7 +47,7 @@ template <int OP, int D>
 struct Sum {
     static constexpr int DD = D * D;
     static constexpr int NMAT = OP == OP_HLA3 ? 6 : OP == OP_HLA2D ? 4 : OP == OP_HLA2U ? 2 : 3;
-    static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D) ? 2 : 0;
+    static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D || OP == OP_AHLA) ? 2 : OP == OP_HLA3 ? 3 : 0;
     static constexpr int VEC0 = NMAT * DD;
     static constexpr int SCAL = VEC0 + NVEC * D;
     static constexpr int SIZE = (SCAL + 4 + 31) / 32 * 32;
@@ -55,8 +57,8 @@ struct Sum {
 // Matrix / vector slots.
 //   OP_HLA2 : S=0 C=1 R=2 ; m=0 r=1
 //   OP_HLA2D: S=0 C=1 G=2 Khat=3 ; m=0 h=1 ; scalar rho
-//   OP_AHLA : P=0 E=1 Dm=2
-//   OP_HLA3 : S=0 Q2=1 P=2 F=3 X=4 Z=5
+//   OP_AHLA : P=0 E=1 Dm=2 ; mK=0 n=1            (the ratio-normaliser's P and E: V -> ones)
+//   OP_HLA3 : S=0 Q2=1 P=2 F=3 X=4 Z=5 ; mK=0 X1=1 F1=2   (likewise for P, X, F)
 //   OP_HLA2U: S=0 C=1
 
 size_t summary_floats(int op, int d) {
@@ -295,6 +297,21 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
         mm<C, D, C>(Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});         // Y = A V
         __syncthreads();
         mm<D, D, C>(TileT{Ks, LD}, Tile{Ys, LD}, Zero{}, store_mat(1));        // E = K^T Y
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {              // u = A 1
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s += As[i * LDC + j];
+            us[i] = s;
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sn = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Ks[i * LD + a];
+                sn += Ks[i * LD + a] * us[i];
+            }
+            out[S::vec(0) + a] = sm_;                                    // mK = K^T 1
+            out[S::vec(1) + a] = sn;                                     // n = K^T (A 1)
+        }
     } else {  // OP_HLA3
         mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(0));        // S
         mm<D, D, C>(TileT{Qs, LD}, Tile{Qs, LD}, Zero{}, store_mat(1));        // Q2
@@ -308,6 +325,31 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
         mm<C, D, C>(TileT{As, LDC}, Tile{Ys, LD}, Zero{}, Put{Y2, LD});        // A^T Yl
         __syncthreads();
         mm<D, D, C>(TileT{Ks, LD}, Tile{Y2, LD}, Zero{}, store_mat(3));        // F = K^T (A^T Yl)
+        // the same with V replaced by ones: u = A 1, w = A^T u
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s += As[i * LDC + j];
+            us[i] = s;
+        }
+        __syncthreads();
+        float* ws_ = lam;                                                 // C floats, unused here
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+            float s = 0.f;
+            for (int r = i; r < C; ++r) s += As[r * LDC + i] * us[r];
+            ws_[i] = s;
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sx = 0.f, sf = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Ks[i * LD + a];
+                sx += Qs[i * LD + a] * us[i];
+                sf += Ks[i * LD + a] * ws_[i];
+            }
+            out[S::vec(0) + a] = sm_;                                    // mK = K^T 1
+            out[S::vec(1) + a] = sx;                                     // X1 = Q^T (A 1)
+            out[S::vec(2) + a] = sf;                                     // F1 = K^T (A^T (A 1))
+        }
     }
 }
 
@@ -364,6 +406,12 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
         add2(2);
         mm<D, D, D>(G(B, 2), G(A, 0),
                     [&](int r, int c) { return A[S::mat(1) + r * D + c] + B[S::mat(1) + r * D + c]; }, dst(1));
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {          // n_AB = n_A + n_B + Dm_B mK_A
+            float s = 0.f;
+            for (int b = 0; b < D; ++b) s += B[S::mat(2) + a * D + b] * A[S::vec(0) + b];
+            out[S::vec(0) + a] = A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = A[S::vec(1) + a] + B[S::vec(1) + a] + s;
+        }
     } else {  // OP_HLA3
         // tmp = S_A Q2_B
         mm<D, D, D>(G(A, 0), G(B, 1), Zero{}, [&](int r, int c, float x) { tmp[r * D + c] = x; });
@@ -377,6 +425,19 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
         mm3<D, D, D, D, D>(Tile{tmp, D}, G(A, 2), G(A, 0), G(B, 4), G(B, 5), G(A, 2),
                            [&](int r, int c) { return A[S::mat(3) + r * D + c] + B[S::mat(3) + r * D + c]; },
                            dst(3));
+        // vectors (P -> mK, X -> X1, F -> F1): X1_AB = X1_A + X1_B + Q2_B mK_A,
+        // F1_AB = F1_A + F1_B + (S_A Q2_B) mK_A + S_A X1_B + Z_B mK_A
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sx = 0.f, sf = 0.f;
+            for (int b = 0; b < D; ++b) {
+                const float mk = A[S::vec(0) + b];
+                sx += B[S::mat(1) + a * D + b] * mk;
+                sf += tmp[a * D + b] * mk + A[S::mat(0) + a * D + b] * B[S::vec(1) + b] + B[S::mat(5) + a * D + b] * mk;
+            }
+            out[S::vec(0) + a] = A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = A[S::vec(1) + a] + B[S::vec(1) + a] + sx;
+            out[S::vec(2) + a] = A[S::vec(2) + a] + B[S::vec(2) + a] + sf;
+        }
     }
 }
 
@@ -469,10 +530,18 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     } else if (OP == OP_AHLA) {
         load_mat<D>(M0, pre + S::mat(0));   // P0
         load_mat<D>(M1, pre + S::mat(1));   // E0
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            vec[a] = pre[S::vec(0) + a];      // mK0
+            vec[D + a] = pre[S::vec(1) + a];  // n0
+        }
     } else {
         load_mat<D>(M0, pre + S::mat(0));   // S0
         load_mat<D>(M1, pre + S::mat(2));   // P0
         load_mat<D>(M2, pre + S::mat(3));   // F0
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            vec[a] = pre[S::vec(0) + a];      // mK0
+            vec[D + a] = pre[S::vec(2) + a];  // F1_0
+        }
     }
     __syncthreads();
     mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
@@ -550,12 +619,44 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     } else if (OP == OP_AHLA) {
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M0, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y = Q P0 + A V
         __syncthreads();
+        if (NORM) {     // y1 = Q mK0 + A 1 (in gp), den = Q n0 + A y1
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[a];
+                for (int j = 0; j <= r; ++j) s += As[r * LDC + j];
+                gp[r] = s;
+            }
+            __syncthreads();
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[D + a];
+                for (int j = 0; j <= r; ++j) s += As[r * LDC + j] * gp[j];
+                den[r] = s;
+            }
+            __syncthreads();
+        }
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{As, LDC}, Tile{Ys, LD}, Zero{}, emit);          // O = Q E0 + A Y
     } else {  // OP_HLA3
         mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Tile{As, LDC}, TileT{As, LDC}, Zero{},
                         [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y = Q P0 + A V
         __syncthreads();
+        if (NORM) {     // y1 = Q mK0 + A 1 (in gp), den = Q F1_0 + W y1
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[a];
+                for (int j = 0; j <= r; ++j) s += As[r * LDC + j];
+                gp[r] = s;
+            }
+            __syncthreads();
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[D + a];
+                for (int j = 0; j <= r; ++j) s += Ws[r * LDC + j] * gp[j];
+                den[r] = s;
+            }
+            __syncthreads();
+        }
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M2, LD}, Tile{Ws, LDC}, Tile{Ys, LD}, Zero{}, emit);          // O = Q F0 + W Y
     }
 }
@@ -665,8 +766,12 @@ static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, 
     case OP_HLA2D:
         return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
                     : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
-    case OP_AHLA: return run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
-    case OP_HLA3: return run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_AHLA:
+        return norm ? run<OP_AHLA, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_HLA3:
+        return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     }
     return cudaErrorInvalidValue;
@@ -757,9 +862,11 @@ int state_launches(int T) {
 //   decayed                w = g (k^T C), s = g (k . m);  S = g S + k k^T;  C = g C + q v^T;
 //                          G = g G + k w^T;  m = g m + q;  h = g h + s k;  Khat += k k^T;
 //                          rho *= g;  x = q^T S;  o = x^T C - q^T G  (/ (x . m - q . h + eps))
-//   AHLA                   P += k v^T;  Dm += k q^T;  y = q^T P;  E += k y^T;  o = q^T E
+//   AHLA                   P += k v^T;  Dm += k q^T;  y = q^T P;  E += k y^T;  o = q^T E;
+//                          mK += k;  n += (q . mK) k;  ratio-normalised: o / (q . n + eps)
 //   third order            S += k k^T;  P += k v^T;  Q2 += q q^T;  a = S q;  b = q^T P;
-//                          F += a b^T;  X += q b^T;  Z += a q^T;  o = q^T F
+//                          F += a b^T;  X += q b^T;  Z += a q^T;  o = q^T F;  mK += k;
+//                          F1 += (q . mK) a;  X1 += (q . mK) q;  ratio-normalised: / (q . F1 + eps)
 //   unmasked               S += k k^T;  C += q v^T;  o = (q^T S) C
 // S is symmetric, so every product with a vector reads matrix columns: thread j of a group
 // walks rows i, and four groups of D threads split the rows (partial sums in shared memory).
@@ -899,12 +1006,29 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
             P[e] = fmaf(ks[i], vs[j], P[e]);
             Dm[e] = fmaf(ks[i], qs[j], Dm[e]);
         }
+        float* mK = st + S::vec(0); float* n = st + S::vec(1);
+        if (tid < D) mK[tid] += ks[tid];
         __syncthreads();
         col_dot<D>(P, qs, part, a);                             // a = y = q^T P
+        if (tid == 0) {
+            float t = 0.f;
+            for (int i = 0; i < D; ++i) t = fmaf(qs[i], mK[i], t);
+            scal[0] = t;                                        // y1 = q . mK
+        }
         for (int e = tid; e < DD; e += NT) E[e] = fmaf(ks[e / D], a[e % D], E[e]);
         __syncthreads();
+        if (tid < D) n[tid] = fmaf(ks[tid], scal[0], n[tid]);
+        __syncthreads();
         col_dot<D>(E, qs, part, b);                             // b = q^T E
-        if (tid < D) o[(size_t)bh * D + tid] = b[tid];
+        if (tid < D) {
+            float den = 1.f;
+            if (NORM) {
+                float t = 0.f;
+                for (int i = 0; i < D; ++i) t = fmaf(qs[i], n[i], t);
+                den = t + eps;
+            }
+            o[(size_t)bh * D + tid] = NORM ? b[tid] / den : b[tid];
+        }
     } else {                                                    // OP_HLA3
         float* Sm = st + S::mat(0); float* Q2 = st + S::mat(1); float* P = st + S::mat(2);
         float* F = st + S::mat(3); float* X = st + S::mat(4); float* Z = st + S::mat(5);
@@ -914,9 +1038,16 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
             P[e] = fmaf(ks[i], vs[j], P[e]);
             Q2[e] = fmaf(qs[i], qs[j], Q2[e]);
         }
+        float* mK = st + S::vec(0); float* X1 = st + S::vec(1); float* F1 = st + S::vec(2);
+        if (tid < D) mK[tid] += ks[tid];
         __syncthreads();
         col_dot<D>(Sm, qs, part, a);                            // a = S q
         col_dot<D>(P, qs, part, b);                             // b = q^T P
+        if (tid == 0) {
+            float t = 0.f;
+            for (int i = 0; i < D; ++i) t = fmaf(qs[i], mK[i], t);
+            scal[0] = t;                                        // b1 = q . mK
+        }
         for (int e = tid; e < DD; e += NT) {
             const int i = e / D, j = e % D;
             F[e] = fmaf(a[i], b[j], F[e]);
@@ -924,8 +1055,21 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
             Z[e] = fmaf(a[i], qs[j], Z[e]);
         }
         __syncthreads();
+        if (tid < D) {
+            F1[tid] = fmaf(a[tid], scal[0], F1[tid]);
+            X1[tid] = fmaf(qs[tid], scal[0], X1[tid]);
+        }
+        __syncthreads();
         col_dot<D>(F, qs, part, a);                             // a = q^T F
-        if (tid < D) o[(size_t)bh * D + tid] = a[tid];
+        if (tid < D) {
+            float den = 1.f;
+            if (NORM) {
+                float t = 0.f;
+                for (int i = 0; i < D; ++i) t = fmaf(qs[i], F1[i], t);
+                den = t + eps;
+            }
+            o[(size_t)bh * D + tid] = NORM ? a[tid] / den : a[tid];
+        }
     }
     __syncthreads();
     for (int e = tid; e < N4; e += NT) gst[e] = st4[e];
@@ -952,8 +1096,12 @@ static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const v
     case OP_HLA2D:
         return norm ? step_launch<OP_HLA2D, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
                     : step_launch<OP_HLA2D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
-    case OP_AHLA: return step_launch<OP_AHLA, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
-    case OP_HLA3: return step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_AHLA:
+        return norm ? step_launch<OP_AHLA, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_AHLA, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA3:
+        return norm ? step_launch<OP_HLA3, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA2U: return step_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     }
     return cudaErrorInvalidValue;

@@ -60,8 +60,8 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads of the problem list (sizes, distributions, dtypes), plus the
-# unmasked configuration at the headline's shape; the names say what each one is.
+# The five workloads of the problem list (sizes, distributions, dtypes), plus three for the
+# widened operators; the names say what each one is.
 WORKLOADS = {
     "hla2_f32_1x2x256x32": Workload(
         "hla2_f32_1x2x256x32", "hla2", "f32", 1, 2, 256, 32, 32, "scaled", "scaled"),
@@ -75,9 +75,14 @@ WORKLOADS = {
         "ahla_bf16_4x16x8192x64", "ahla", "bf16", 4, 16, 8192, 64, 64, "scaled", "scaled"),
     "hla3_f32_2x8x4096x32": Workload(
         "hla3_f32_2x8x4096x32", "hla3", "f32", 2, 8, 4096, 32, 32, "scaled", "scaled"),
-    # not one of the five: the unmasked second-order configuration at the headline's shape
+    # not among the five: the unmasked second order at the headline's shape, and the
+    # ratio-normalised AHLA / third order at the shapes of their plain workloads
     "hla2u_bf16_4x16x4096x64": Workload(
         "hla2u_bf16_4x16x4096x64", "hla2u", "bf16", 4, 16, 4096, 64, 64, "scaled", "scaled"),
+    "ahlan_bf16_4x16x8192x64": Workload(
+        "ahlan_bf16_4x16x8192x64", "ahlan", "bf16", 4, 16, 8192, 64, 64, "softplus", "unit"),
+    "hla3n_f32_2x8x4096x32": Workload(
+        "hla3n_f32_2x8x4096x32", "hla3n", "f32", 2, 8, 4096, 32, 32, "softplus", "unit"),
 }
 
 

@@ -17,6 +17,10 @@
  *                           o_t = sum_{j<=t} (q_t.k_j) sum_{i<=j} (q_j.k_i) v_i.
  *   hla3_forward            Metodología 3: third order A A^T A, masked:
  *                           O = (M A) V, M = L (.) (A A^T), A = L (.) Q K^T.
+ *   ahla_forward_normalized Metodología 2 lists the AHLA summaries (P^KV, m^K,
+ *   hla3_forward_normalized E, n): the ratio-normalised AHLA divides by the same
+ *                           masked operator on a ones value column,
+ *                           q_t^T n_t + eps; the third order likewise.
  *   hla2_forward_unmasked   Contribuciones 2, the unmasked configuration: the
  *                           naive product the cross summary G_t corrects,
  *                           o_t = q_t^T S^K_t C^QV_t
@@ -81,7 +85,9 @@ typedef enum {
     HLA_OP_HLA2_NORM = 1,  /* hla2_forward_normalized */
     HLA_OP_AHLA = 2,       /* ahla_forward */
     HLA_OP_HLA3 = 3,       /* hla3_forward */
-    HLA_OP_HLA2_UNMASKED = 4  /* hla2_forward_unmasked */
+    HLA_OP_HLA2_UNMASKED = 4, /* hla2_forward_unmasked */
+    HLA_OP_AHLA_NORM = 5,  /* ahla_forward_normalized */
+    HLA_OP_HLA3_NORM = 6   /* hla3_forward_normalized */
 } hla_op_t;
 
 /* Version of this ABI (bumped on any signature change). */
@@ -122,6 +128,19 @@ hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
                           int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                           const float* gamma, void* workspace, size_t workspace_bytes,
                           void* stream);
+
+/* Ratio-normalised AHLA and third-order forwards: the output divided by the same masked
+ * operator applied to a ones value column, plus eps (for AHLA, q_t^T n_t with the named
+ * summaries m^K = sum k and n_t = sum_j k_j (q_j^T m^K_j)).  gamma must be NULL.  CUDA-core
+ * kernels for every dtype and d. */
+hla_status_t ahla_forward_normalized(const void* q, const void* k, const void* v, float* o,
+                                     int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                     const float* gamma, float eps,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+hla_status_t hla3_forward_normalized(const void* q, const void* k, const void* v, float* o,
+                                     int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                     const float* gamma, float eps,
+                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Unmasked second-order forward, o_t = q_t^T S^K_t C^QV_t (Contribuciones 2, the unmasked
  * configuration).  gamma must be NULL.  CUDA-core kernels for every dtype and d. */
@@ -171,11 +190,13 @@ int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, in
  *                         r = S m - h          (o_t = q_t^T R_t, den = q_t^T r_t)
  *   second order, decayed S, C, G, Khat = sum k k^T (undecayed);  m, h;  rho =
  *                         gamma^t              (o_t = q_t^T (S_t C_t - G_t))
- *   AHLA                  P = sum k v^T, E, D = sum k q^T      (o_t = q_t^T E_t)
- *   third order           S, Q2 = sum q q^T, P, F, X, Z        (o_t = q_t^T F_t)
+ *   AHLA                  P = sum k v^T, E, D = sum k q^T;  m^K = sum k, n
+ *                         (o_t = q_t^T E_t, den_t = q_t^T n_t)
+ *   third order           S, Q2 = sum q q^T, P, F, X, Z;  m^K, X1, F1 (X and F with v
+ *                         replaced by 1)     (o_t = q_t^T F_t, den_t = q_t^T F1_t)
  *   unmasked second order S, C                                 (o_t = q_t^T S_t C_t)
  * A state of zero tokens is all zeros, except rho = 1 for the decayed form.
- * The state of HLA_OP_HLA2_NORM is that of HLA_OP_HLA2.
+ * The state of a ratio-normalised op is that of its plain op.
  */
 
 /* Floats of one head's state, or 0 when (op, decayed, d, dv) is invalid or unsupported

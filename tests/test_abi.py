@@ -159,8 +159,10 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     pad = lambda n: (n + 31) // 32 * 32                       # noqa: E731
     assert lib.hla_state_floats(0, 0, d, d) == pad(3 * d * d + 2 * d + 4)     # S, C, R ; m, r
     assert lib.hla_state_floats(1, 1, d, d) == pad(4 * d * d + 2 * d + 4)     # decayed: + Khat, rho
-    assert lib.hla_state_floats(2, 0, d, d) == pad(3 * d * d + 4)             # P, E, D
-    assert lib.hla_state_floats(3, 0, 32, 32) == pad(6 * 32 * 32 + 4)        # S, Q2, P, F, X, Z
+    assert lib.hla_state_floats(2, 0, d, d) == pad(3 * d * d + 2 * d + 4)     # P, E, D ; mK, n
+    assert lib.hla_state_floats(3, 0, 32, 32) == pad(6 * 32 * 32 + 3 * 32 + 4)   # S Q2 P F X Z ; mK X1 F1
+    assert lib.hla_state_floats(5, 0, d, d) == lib.hla_state_floats(2, 0, d, d)   # normalised: same state
+    assert lib.hla_state_floats(6, 0, 32, 32) == lib.hla_state_floats(3, 0, 32, 32)
     assert lib.hla_state_floats(2, 1, d, d) == 0                              # no decayed AHLA
     assert lib.hla_state_floats(0, 0, 48, 48) == 0
     assert lib.hla_state_floats(0, 0, 64, 32) == 0
@@ -173,7 +175,7 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     st = lib.hla_state
     a = [vp(16), vp(16), vp(16), vp(16)]
     assert st(0, vp(0), *a[1:], 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 1      # NULL q
-    assert st(5, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
+    assert st(7, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
     assert st(0, *a, 0, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 2                # B = 0
     assert st(0, *a, 1, 1, 64, d, d, 7, vp(0), vp(16), 1 << 20, vp(0)) == 4                # dtype
     assert st(2, *a, 1, 1, 64, d, d, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5               # gamma + AHLA
@@ -187,6 +189,23 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert sp(0, *b, 1, 0, d, d, 0, vp(0), f(1e-6), vp(0)) == 2                            # H = 0
     assert sp(3, *b, 1, 1, 32, 32, 0, vp(16), f(1e-6), vp(0)) == 5                         # gamma + HLA-3
     assert sp(0, vp(24), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 3                # alignment
+
+
+def test_normalised_ahla_hla3_routing_and_errors(lib):
+    """Ratio-normalised AHLA / third order: CUDA-core kernels (the tensor-core AHLA walker
+    carries no normaliser), no decayed form, the plain op's workspace."""
+    vp, f = ctypes.c_void_p, ctypes.c_float
+    for op, plain in ((hla.OP_AHLA_NORM, hla.OP_AHLA), (hla.OP_HLA3_NORM, hla.OP_HLA3)):
+        assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
+        assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0           # no decay
+        assert lib.hla_workspace_bytes(op, hla.HLA_F32, 0, 2, 8, 4096, 32, 32) == \
+            lib.hla_workspace_bytes(plain, hla.HLA_F32, 0, 2, 8, 4096, 32, 32)
+    assert lib.hla_uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 1
+    a = [vp(16)] * 4
+    for fn in (lib.ahla_forward_normalized, lib.hla3_forward_normalized):
+        assert fn(*a, 1, 1, 64, 64, 64, 0, vp(16), f(1e-6), vp(16), 1 << 20, vp(0)) == 5     # gamma given
+        assert fn(vp(0), *a[1:], 1, 1, 64, 64, 64, 0, vp(0), f(1e-6), vp(16), 1 << 20, vp(0)) == 1
+        assert fn(*a, 1, 1, 64, 64, 64, 0, vp(0), f(1e-6), vp(16), 64, vp(0)) == 6           # workspace
 
 
 def test_unmasked_op_sizes_and_errors(lib):

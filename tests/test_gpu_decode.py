@@ -24,13 +24,14 @@ pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 STATE_TOL = 1e-4          # fp32 state against fp64, relative to each matrix's largest entry
-OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u"]
+OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n"]
+NORMALISED = ("hla2n", "ahlan", "hla3n")
 DEV = torch.device("cuda:0")
 
 
 def recipe(op, dtype, B, H, T, d, seed):
-    qk = "softplus" if op == "hla2n" else "scaled"
-    v = "unit" if op == "hla2n" else "scaled"
+    qk = "softplus" if op in NORMALISED else "scaled"
+    v = "unit" if op in NORMALISED else "scaled"
     g = (0.9, 0.999) if op == "hla2d" else None
     return hla_inputs.Workload(f"{op}_{dtype}_{B}x{H}x{T}x{d}", op, dtype, B, H, T, d, d, qk, v,
                                gamma_range=g, seed=seed)
@@ -44,20 +45,23 @@ def oracle_state(op, q, k, v, gamma):
     if op == "hla2d":
         s = seg.hla2_summary(q, k, v, gamma=gamma)
         return [s["S"], s["C"], s["G"], s["Khat"], s["m"], s["h"], np.array([float(s["rho"])])]
-    if op == "ahla":
+    ones = np.ones((q.shape[0], 1))
+    if op in ("ahla", "ahlan"):
         s = seg.ahla_summary(q, k, v)
-        return [s["P"], s["E"], s["D"]]
+        _, s1 = oracle.ahla_run(q, k, ones, want_output=False)     # v -> 1: P -> mK, E -> n
+        return [s["P"], s["E"], s["D"], s1["P"][:, 0], s1["E"][:, 0]]
     if op == "hla2u":
         _, s = oracle.hla2u_run(q, k, v, want_output=False)
         return [s["S"], s["C"]]
     s = seg.hla3_summary(q, k, v)
-    return [s["S"], s["Q2"], s["P"], s["F"], s["X"], s["Z"]]
+    s1 = seg.hla3_summary(q, k, ones)                              # v -> 1: P, X, F -> mK, X1, F1
+    return [s["S"], s["Q2"], s["P"], s["F"], s["X"], s["Z"], s1["P"][:, 0], s1["X"][:, 0], s1["F"][:, 0]]
 
 
 def split_state(op, x, d):
     """The GPU state vector of one head, cut into the same slots."""
-    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6, "hla2u": 2}[op]
-    nvec = 2 if op in ("hla2", "hla2n", "hla2d") else 0
+    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6, "hla2u": 2, "ahlan": 3, "hla3n": 6}[op]
+    nvec = {"hla2": 2, "hla2n": 2, "hla2d": 2, "ahla": 2, "ahlan": 2, "hla3": 3, "hla3n": 3, "hla2u": 0}[op]
     out = [x[i * d * d:(i + 1) * d * d].reshape(d, d) for i in range(nmat)]
     base = nmat * d * d
     out += [x[base + i * d: base + (i + 1) * d] for i in range(nvec)]

@@ -271,3 +271,19 @@ def test_unmasked_many_heads():
     q, k, v, _ = hla_inputs.make_inputs(w)
     o = gpu_forward("hla2u", q, k, v, None)
     assert oracle.max_row_rel_err(o.cpu(), reference("hla2u", q, k, v, None)) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# ratio-normalised AHLA and third order (CUDA-core kernels)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("op", ["ahlan", "hla3n"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 65, 200, 1000])
+def test_normalised_ahla_hla3_parity(op, dtype, d, T):
+    w = hla_inputs.Workload(f"{op}_{dtype}_1x2x{T}x{d}", op, dtype, 1, 2, T, d, d, "softplus", "unit", seed=T + 9)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    o = gpu_forward(op, q, k, v, None, eps=w.eps)
+    ref = reference(op, q, k, v, None, eps=w.eps)
+    assert oracle.max_row_rel_err(o.cpu(), ref) <= TOL[dtype]
