@@ -83,6 +83,9 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     using S = simt_layout;
     float* slot = MODE == OUTPUT ? p.pre + ((size_t)bh * p.NSp + seg * p.ratio) * S::size
                                  : p.sums + ((size_t)bh * p.NSp + seg) * S::size;
+    // Programmatic dependent launch: the output walk may be scheduled once every summary CTA
+    // has started; its CTAs that fold summaries wait for this grid's completion first.
+    if (MODE == SUMMARY && tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (seg >= p.NS) {                                    // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
@@ -120,6 +123,9 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // the carried-in prefix (P^T, E^T) through shared memory: coalesced loads, rows
         // swizzled by 16-byte chunk, then every thread takes its row
         float* stage = reinterpret_cast<float*>(sm + AS_A);   // P^T [64][64] | E^T [64][64]
+        // the summaries are read below: wait for the summary walk (a no-op without a
+        // programmatic dependency); segment 0 reads none
+        if (p.fold && seg > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         if (p.fold) {
             // n = seg * ratio slots: P0^T = sum_l P^T_l and
             // E0^T = sum_l E^T_l + sum_{m < n-1} P^T_m Dsuf^T(m+1), Dsuf^T(m) = sum_{m <= l < n} D^T_l
@@ -458,8 +464,23 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (prm.fold) {
+        // a programmatic dependent of the summary walk (see the second-order forward)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pl.NS, BH);
+        cfg.blockDim = dim3(ANT);
+        cfg.dynamicSmemBytes = ASMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, k_ahla_walk<OUTPUT>, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
+    } else {
+        k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }

@@ -118,6 +118,9 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     using S = simt_layout;
     float* slot = MODE == OUTPUT ? p.pre + ((size_t)bh * p.NSp + seg * p.ratio) * S::size
                                  : p.sums + ((size_t)bh * p.NSp + seg) * S::size;
+    // Programmatic dependent launch: the output walk may be scheduled once every summary CTA
+    // has started; its CTAs that fold summaries wait for this grid's completion first.
+    if (MODE == SUMMARY && tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (seg >= p.NS) {                       // padding slots: identity (zeros)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
@@ -170,6 +173,9 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     float* stage = reinterpret_cast<float*>(sm + SM_A);                   // S [64][64] | R [64][64]
     float* stage_r = reinterpret_cast<float*>(sm + SM_Z);                 // r [64]
     auto sw = [](int i, int j) { return i * D + ((((j >> 2) ^ (i & 7)) << 2) | (j & 3)); };
+    // The summaries are read below: wait for the summary walk (a no-op without a programmatic
+    // dependency).  Segment 0 reads none and does not wait.
+    if (MODE == OUTPUT && p.fold && seg > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     if (MODE == OUTPUT && epi && p.fold) {
         // n = seg * ratio slots: S0 = sum_l S_l, R0 = sum_l R_l + sum_{m < n-1} S_m Csuf(m+1),
         // r0 = sum_l r_l + sum_{m < n-1} S_m msuf(m+1), with Csuf(m) = sum_{m <= l < n} C_l (the
@@ -946,8 +952,25 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    k_walk<OUTPUT><<<dim3(pl.NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (prm.fold) {
+        // launched as a programmatic dependent of the summary walk: its set-up and first loads
+        // overlap the summary walk's end (nothing stands between the two launches unless the
+        // caller asked for phase events, which then serialise them)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pl.NS, BH);
+        cfg.blockDim = dim3(NTH);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&cfg, k_walk<OUTPUT>, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
+    } else {
+        k_walk<OUTPUT><<<dim3(pl.NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }
