@@ -164,7 +164,9 @@ def load_peaks():
 
 
 def output_kernel_model(path: str, w: hla_inputs.Workload):
-    """Algorithmic work of the output kernel per token ('Roofline')."""
+    """Algorithmic work of the output kernel per token: the products the method needs per
+    chunk of c tokens, each 2 flop per multiply-add, divided by c (no discarded halves of
+    stacked products, no state walk)."""
     D = w.d
     c = 128 if path == "tc" else 64
     if w.op in ("ahla", "ahlan"):
