@@ -19,6 +19,13 @@ Contents
 All formulas come from "Resumen Técnico: Atención Lineal de Orden Superior
 (HLA)" (gist.science, paper 2510.27258), sections Metodología 1-4 and
 Contribuciones 1-3; each function cites its passage.
+
+Pinning.  Every op is pinned to literal sums, brute force, closed forms and
+invariants of the operator as read from the page.  Three readings have no
+printed counterpart to pin against (parity unpinned against the page's own
+algebra): the decay rule (the page gives no decayed formula), the third-order
+nine-summary algebra (named, not printed), and the AHLA / third-order
+normalisers (named, not printed; read as the operator on a ones value column).
 """
 from __future__ import annotations
 
