@@ -327,3 +327,62 @@ def test_decay_every_term_is_needed(term):
     q, k, v = rand_head(48, 4, 3, seed=9)
     ref = recur("hla2d", q, k, v, gamma=0.9)
     assert rel(decay_forward(q, k, v, 0.9, 16, drop=term), ref) > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# ratio-normalised AHLA / third order: the combine of the normaliser vectors
+# ---------------------------------------------------------------------------
+
+def _vec_summaries(q, k, n):
+    """Oracle summaries of two segments and of their concatenation, with v a ones column."""
+    ones = np.ones((q.shape[0], 1))
+    A = dict(q=q[:n], k=k[:n], v=ones[:n])
+    B = dict(q=q[n:], k=k[n:], v=ones[n:])
+    return A, B, dict(q=q, k=k, v=ones)
+
+
+@pytest.mark.parametrize("n", [1, 7, 20])
+def test_ahla_normaliser_vectors_combine(n):
+    """mK and n are P and E with v a ones column: n_AB = n_A + n_B + D_B mK_A."""
+    rng = np.random.default_rng(n)
+    q, k = rng.standard_normal((31, 4)), rng.standard_normal((31, 4))
+    A, B, AB = _vec_summaries(q, k, n)
+    sa, sb, sab = (seg.ahla_summary(x["q"], x["k"], x["v"]) for x in (A, B, AB))
+    mk_a, mk_b = sa["P"][:, 0], sb["P"][:, 0]
+    n_a, n_b = sa["E"][:, 0], sb["E"][:, 0]
+    np.testing.assert_allclose(mk_a + mk_b, sab["P"][:, 0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(n_a + n_b + sb["D"] @ mk_a, sab["E"][:, 0], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [1, 9, 22])
+def test_third_order_normaliser_vectors_combine(n):
+    """mK, X1, F1 are P, X, F with v a ones column: X1_AB = X1_A + X1_B + Q2_B mK_A and
+    F1_AB = F1_A + F1_B + S_A Q2_B mK_A + S_A X1_B + Z_B mK_A."""
+    rng = np.random.default_rng(40 + n)
+    q, k = rng.standard_normal((29, 3)), rng.standard_normal((29, 3))
+    A, B, AB = _vec_summaries(q, k, n)
+    sa, sb, sab = (seg.hla3_summary(x["q"], x["k"], x["v"]) for x in (A, B, AB))
+    mk_a, x1_a, f1_a = sa["P"][:, 0], sa["X"][:, 0], sa["F"][:, 0]
+    mk_b, x1_b, f1_b = sb["P"][:, 0], sb["X"][:, 0], sb["F"][:, 0]
+    np.testing.assert_allclose(x1_a + x1_b + sb["Q2"] @ mk_a, sab["X"][:, 0], rtol=1e-11, atol=1e-11)
+    f1 = f1_a + f1_b + sa["S"] @ sb["Q2"] @ mk_a + sa["S"] @ x1_b + sb["Z"] @ mk_a
+    np.testing.assert_allclose(f1, sab["F"][:, 0], rtol=1e-11, atol=1e-11)
+
+
+def test_normaliser_vectors_give_the_literal_denominator():
+    """q_t . n_t (AHLA) and q_t . F1_t (third order) from the running vectors equal the masked
+    operators applied to a ones column, token by token."""
+    rng = np.random.default_rng(44)
+    T, d = 17, 3
+    q, k = np.abs(rng.standard_normal((T, d))), np.abs(rng.standard_normal((T, d)))
+    ones = np.ones((T, 1))
+    den_a = oracle.recur("ahla", q[None, None], k[None, None], ones[None, None])[0, 0, :, 0]
+    den_3 = oracle.recur("hla3", q[None, None], k[None, None], ones[None, None])[0, 0, :, 0]
+    mk, nv, S, F1 = np.zeros(d), np.zeros(d), np.zeros((d, d)), np.zeros(d)
+    for t in range(T):
+        mk = mk + k[t]
+        nv = nv + k[t] * (q[t] @ mk)
+        S = S + np.outer(k[t], k[t])
+        F1 = F1 + (S @ q[t]) * (q[t] @ mk)
+        assert abs(q[t] @ nv - den_a[t]) < 1e-12 * max(1.0, den_a[t])
+        assert abs(q[t] @ F1 - den_3[t]) < 1e-12 * max(1.0, den_3[t])
