@@ -37,8 +37,9 @@
  * each value in (0, 1].  Base addresses must be 16-byte aligned.
  *
  * Supported shapes.  d == dv.  HLA_F32: d in {32, 64}, every op (fp32 CUDA-core
- * path).  HLA_BF16: d in {32, 64}, every op; d == 64 without decay runs the
- * tcgen05 tensor-core path for hla2 / hla2_normalized / ahla.  T >= 1 (any
+ * path).  HLA_BF16: d in {32, 64}, every op; with d == 64 the tcgen05
+ * tensor-core path runs hla2 (with or without decay), hla2_normalized (without
+ * decay) and ahla, and every other op runs on the CUDA cores.  T >= 1 (any
  * value; the tail chunk is padded), B, H >= 1, B*H*T < 2^31.  Anything else
  * returns HLA_ERR_UNSUPPORTED or HLA_ERR_SHAPE before any launch.
  *
@@ -90,7 +91,8 @@ typedef enum {
     HLA_OP_HLA3_NORM = 6   /* hla3_forward_normalized */
 } hla_op_t;
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped on any signature change or addition; 2 added the unmasked and
+ * ratio-normalised AHLA / third-order ops and the streaming-state calls). */
 int hla_abi_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.hla_abi_version() == 1
+    assert lib.hla_abi_version() == 2
     for code in range(9):
         s = lib.hla_status_str(code).decode()
         assert s.startswith(hla.STATUS_NAMES[code])
