@@ -129,7 +129,7 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
     const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
     if (use_tc(r)) return hla::tc::kernel_launches(r.op, r.norm, B * H, T);
-    return hla::simt::kernel_launches(T);
+    return hla::simt::kernel_launches(r.op, r.d, T);
 }
 
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {

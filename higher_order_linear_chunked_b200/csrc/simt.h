@@ -8,8 +8,9 @@ namespace simt {
 
 // floats in one chunk summary for internal op id `op` at head dim d
 size_t summary_floats(int op, int d);
-// kernels one forward enqueues (chunk kernel, scan levels, output kernel)
-int kernel_launches(int T);
+// kernels one forward enqueues (chunk kernel, the scan: one fold launch, or one launch per
+// tree level when three summaries do not fit in shared memory, output kernel)
+int kernel_launches(int op, int d, int T);
 // floats of workspace the path needs after the status block
 size_t workspace_floats(int op, int d, int BH, int T);
 // summary layout helpers for other paths: offsets (in floats) of matrix / vector slots
