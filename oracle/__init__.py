@@ -14,6 +14,8 @@ Contents
 * :mod:`oracle.brute` - the O(T^3) masked-matrix definitions (numpy, fp64).
 * :mod:`oracle.segments` - segment summaries, the semidirect-product combine
   maps and a Blelloch exclusive scan over them, on the host in fp64.
+* :mod:`oracle.backward` - gradients of the second-order forward (reverse-mode
+  differentiation of the masked-matrix definition, torch CPU float64).
 * :func:`max_row_rel_err` - the parity metric.
 
 All formulas come from "Resumen Técnico: Atención Lineal de Orden Superior

@@ -1,0 +1,34 @@
+"""Gradients of the second-order masked forward, fp64, for the backward pass.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+"Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 4 and
+Contribuciones 2: the scan reproduces the serial activations exactly, which the page offers as
+the basis of exact parallel training; it prints no gradient.  The reference here is therefore
+the plain one: reverse-mode differentiation (torch autograd, CPU, float64) of the masked-matrix
+definition O = (L (.) (A A^T)) V with A = L (.) Q K^T, for a given output gradient dO.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import _f64
+
+
+def hla2_forward_matrix(q, k, v):
+    """The masked second-order output as torch float64 ops (differentiable)."""
+    import torch
+    T = q.shape[-2]
+    L = torch.tril(torch.ones(T, T, dtype=torch.float64))
+    A = L * (q @ k.transpose(-1, -2))
+    W = L * (A @ A.transpose(-1, -2))
+    return W @ v
+
+
+def hla2_grads(q, k, v, do):
+    """(dQ, dK, dV) of sum(O * dO) for O = hla2(q, k, v), fp64 numpy arrays of q's shape."""
+    import torch
+    tq, tk, tv = (torch.tensor(_f64(x), requires_grad=True) for x in (q, k, v))
+    o = hla2_forward_matrix(tq, tk, tv)
+    o.backward(torch.tensor(_f64(do)))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()

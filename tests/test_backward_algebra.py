@@ -1,0 +1,122 @@
+"""Groundwork for the backward pass (CPU, fp64): the gradient reference and the chunked
+reverse walk a kernel would run.
+
+"Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 4 and
+Contribuciones 2 claim exact scan-based training but print no gradient.  The reference,
+``oracle.backward.hla2_grads``, is reverse-mode differentiation of the masked-matrix definition.
+It is pinned here by central finite differences of the independent numpy definition and by the
+single-token closed form.  The chunked reverse walk is then checked against it: the forward
+walk over chunks carries (S0, R0); the backward walk runs over the chunks in reverse order,
+carrying their adjoints (dS0, dR0), and forms the chunk's dQ, dK, dV with the same masked
+chunk-local products as the forward.
+"""
+import numpy as np
+import pytest
+
+import oracle.brute as brute
+from oracle.backward import hla2_grads
+
+
+def rand(T, d, dv, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((T, d)) / np.sqrt(d), rng.standard_normal((T, d)) / np.sqrt(d),
+            rng.standard_normal((T, dv)), rng.standard_normal((T, dv)))
+
+
+def test_reference_matches_finite_differences():
+    q, k, v, do = rand(6, 3, 2, 1)
+    gq, gk, gv = hla2_grads(q, k, v, do)
+    f = lambda q_, k_, v_: float(np.sum(brute.hla2(q_, k_, v_) * do))   # noqa: E731
+    h = 1e-6
+    for x, g, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+def test_reference_single_token_closed_form():
+    q, k, v, do = rand(1, 4, 3, 2)
+    gq, gk, gv = hla2_grads(q, k, v, do)
+    s, w = float(q[0] @ k[0]), float(v[0] @ do[0])
+    np.testing.assert_allclose(gq[0], 2 * s * w * k[0], rtol=1e-12)
+    np.testing.assert_allclose(gk[0], 2 * s * w * q[0], rtol=1e-12)
+    np.testing.assert_allclose(gv[0], s * s * do[0], rtol=1e-12)
+
+
+def chunks(x, c):
+    T = x.shape[0]
+    n = -(-T // c)
+    return [np.vstack([x, np.zeros((n * c - T, x.shape[1]))])[i * c:(i + 1) * c] for i in range(n)]
+
+
+def chunked_backward(q, k, v, do, c, drop=None):
+    """Reverse walk over chunks.  Forward per chunk (S0, R0 carried in):
+        A = L (.) Q K^T,  P = Q S0,  W = L (.) (P Q^T + A A^T),  O = Q R0 + W V,
+        Z = P + A K,  S0' = S0 + K^T K,  R0' = R0 + Z^T V.
+    Backward per chunk, given dO and the adjoints (dS0', dR0') of the states it hands on:
+        dV = W^T dO + Z dR0';  dZ = V dR0'^T;  dW = L (.) dO V^T;
+        dP = dZ + dW Q;  dA = L (.) (dZ K^T + (dW + dW^T) A);
+        dQ = dO R0^T + dW^T P + dP S0^T + dA K;  dK = K (dS0' + dS0'^T) + A^T dZ + dA^T Q;
+        dS0 = dS0' + Q^T dP;  dR0 = dR0' + Q^T dO.
+    ``drop`` ("dS" or "dR") withholds one carried adjoint, only to show that it is needed."""
+    d, dv = q.shape[1], v.shape[1]
+    Qs, Ks, Vs, Gs = chunks(q, c), chunks(k, c), chunks(v, c), chunks(do, c)
+    L = np.tril(np.ones((c, c)))
+    S0, R0 = np.zeros((d, d)), np.zeros((d, dv))
+    saved = []
+    for Q, K, V in zip(Qs, Ks, Vs):                     # forward walk: keep the carried states
+        saved.append((S0, R0))
+        A = L * (Q @ K.T)
+        Z = Q @ S0 + A @ K
+        S0, R0 = S0 + K.T @ K, R0 + Z.T @ V
+    dS, dR = np.zeros((d, d)), np.zeros((d, dv))
+    gq, gk, gv = [], [], []
+    for (Q, K, V, dO), (S0, R0) in zip(reversed(list(zip(Qs, Ks, Vs, Gs))), reversed(saved)):
+        A = L * (Q @ K.T)
+        P = Q @ S0
+        W = L * (P @ Q.T + A @ A.T)
+        Z = P + A @ K
+        dV = W.T @ dO + Z @ dR
+        dZ = V @ dR.T
+        dW = L * (dO @ V.T)
+        dP = dZ + dW @ Q
+        dA = L * (dZ @ K.T + (dW + dW.T) @ A)
+        dQ = dO @ R0.T + dW.T @ P + dP @ S0.T + dA @ K
+        dK = K @ (dS + dS.T) + A.T @ dZ + dA.T @ Q
+        dS, dR = dS + Q.T @ dP, dR + Q.T @ dO
+        if drop == "dS":
+            dS = np.zeros_like(dS)
+        if drop == "dR":
+            dR = np.zeros_like(dR)
+        gq.append(dQ); gk.append(dK); gv.append(dV)
+    T = q.shape[0]
+    return (np.vstack(gq[::-1])[:T], np.vstack(gk[::-1])[:T], np.vstack(gv[::-1])[:T])
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (7, 4), (16, 4), (37, 8), (64, 16), (100, 32)])
+def test_chunked_reverse_walk_matches_the_reference(T, c):
+    q, k, v, do = rand(T, 5, 3, T + c)
+    want = hla2_grads(q, k, v, do)
+    got = chunked_backward(q, k, v, do, c)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("drop", ["dS", "dR"])
+def test_reverse_walk_needs_both_carried_adjoints(drop):
+    """Withholding either carried adjoint breaks the gradients once there are several chunks
+    (and changes nothing with one chunk): the match above covers the cross-chunk terms."""
+    q, k, v, do = rand(40, 4, 3, 5)
+    want = hla2_grads(q, k, v, do)
+    one = chunked_backward(q, k, v, do, 40, drop=drop)
+    for a, b in zip(one, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+    many = chunked_backward(q, k, v, do, 8, drop=drop)
+    assert max(np.abs(a - b).max() / np.abs(b).max() for a, b in zip(many, want)) > 1e-3
