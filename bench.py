@@ -3,7 +3,7 @@
 
 Default workload: ratio-normalised second-order HLA, bf16 inputs, fp32 output,
 B=4, H=16, T=4096, d=dv=64 (262,144 tokens per step), synthetic seeded inputs.
-One step = one full forward (segment summaries, Blelloch scan, output pass).
+One step = one full forward (segment summaries, exclusive scan of the summaries, output pass).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 

@@ -26,10 +26,12 @@
  *                           o_t = q_t^T S^K_t C^QV_t
  *                               = sum_{j<=t} sum_{i<=t} (q_t.k_i)(q_j.k_i) v_j.
  *
- * The mask L includes the diagonal (j <= t).  All four are computed with the
- * chunk-parallel scheme of Metodología 4: per-segment summaries, a Blelloch
+ * The mask L includes the diagonal (j <= t).  Every operator is computed with
+ * the chunk-parallel scheme of Metodología 4: per-segment summaries, an
  * exclusive scan with the semidirect-product combine, and a per-chunk output
- * pass that applies each chunk's carried-in prefix.
+ * pass that applies each chunk's carried-in prefix.  The scan is a factored
+ * segment prefix on the tensor-core path, and a per-head fold or the Blelloch
+ * tree (the page's form) on the CUDA-core path; all give the same prefixes.
  *
  * Layout.  q, k: [B][H][T][d]; v: [B][H][T][dv]; o: [B][H][T][dv], contiguous
  * row-major.  q, k, v are fp32 (HLA_F32) or bf16 (HLA_BF16), all three the same
