@@ -32,3 +32,15 @@ def hla2_grads(q, k, v, do):
     o = hla2_forward_matrix(tq, tk, tv)
     o.backward(torch.tensor(_f64(do)))
     return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def hla2n_grads(q, k, v, do, eps: float = 1e-6):
+    """(dQ, dK, dV) for the ratio-normalised output O = num / (den + eps), den the masked
+    operator on a ones value column (Metodología 1, Normalización)."""
+    import torch
+    tq, tk, tv = (torch.tensor(_f64(x), requires_grad=True) for x in (q, k, v))
+    num = hla2_forward_matrix(tq, tk, tv)
+    den = hla2_forward_matrix(tq, tk, torch.ones(tv.shape[:-1] + (1,), dtype=torch.float64))
+    o = num / (den + eps)
+    o.backward(torch.tensor(_f64(do)))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()

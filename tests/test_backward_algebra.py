@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle.brute as brute
-from oracle.backward import hla2_grads
+from oracle.backward import hla2_grads, hla2n_grads
 
 
 def rand(T, d, dv, seed):
@@ -39,6 +39,25 @@ def test_reference_matches_finite_differences():
             args_p[which], args_m[which] = xp, xm
             num[idx] = (f(*args_p) - f(*args_m)) / (2 * h)
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+def test_normalised_reference_matches_finite_differences():
+    rng = np.random.default_rng(3)
+    T, d, dv = 5, 3, 2
+    q, k = np.abs(rng.standard_normal((T, d))), np.abs(rng.standard_normal((T, d)))
+    v, do = rng.standard_normal((T, dv)), rng.standard_normal((T, dv))
+    gq, gk, gv = hla2n_grads(q, k, v, do, 1e-6)
+    f = lambda q_, k_, v_: float(np.sum(brute.hla2(q_, k_, v_, normalized=True, eps=1e-6) * do))  # noqa: E731
+    h = 1e-6
+    for x, g, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p, args_m = [q, k, v], [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num = (f(*args_p) - f(*args_m)) / (2 * h)
+            assert abs(g[idx] - num) <= 1e-6 * max(1.0, abs(num))
 
 
 def test_reference_single_token_closed_form():
@@ -120,3 +139,23 @@ def test_reverse_walk_needs_both_carried_adjoints(drop):
         np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
     many = chunked_backward(q, k, v, do, 8, drop=drop)
     assert max(np.abs(a - b).max() / np.abs(b).max() for a, b in zip(many, want)) > 1e-3
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (23, 8), (64, 16)])
+def test_normalised_backward_is_the_walk_on_ones_augmented_values(T, c):
+    """The ratio-normalised output is num / (den + eps) with den the operator on a ones column,
+    so its backward is the same reverse walk on [V | 1] with the output gradient
+    [dO / (den + eps) | -sum_c dO num / (den + eps)^2], the last dV column discarded."""
+    rng = np.random.default_rng(T)
+    q, k = np.abs(rng.standard_normal((T, 4))) / 2, np.abs(rng.standard_normal((T, 4))) / 2
+    v, do = rng.standard_normal((T, 3)), rng.standard_normal((T, 3))
+    eps = 1e-6
+    v1 = np.hstack([v, np.ones((T, 1))])
+    out = brute.hla2(q, k, v1)
+    num, den = out[:, :3], out[:, 3:]
+    g = np.hstack([do / (den + eps), -(do * num).sum(axis=1, keepdims=True) / (den + eps) ** 2])
+    gq, gk, gv = chunked_backward(q, k, v1, g, c)
+    want = hla2n_grads(q, k, v, do, eps)
+    np.testing.assert_allclose(gq, want[0], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(gk, want[1], rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(gv[:, :3], want[2], rtol=1e-9, atol=1e-10)
