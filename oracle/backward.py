@@ -6,7 +6,8 @@ TEST INFRASTRUCTURE ONLY (see the package docstring).
 Contribuciones 2: the scan reproduces the serial activations exactly, which the page offers as
 the basis of exact parallel training; it prints no gradient.  The reference here is therefore
 the plain one: reverse-mode differentiation (torch autograd, CPU, float64) of the masked-matrix
-definition O = (L (.) (A A^T)) V with A = L (.) Q K^T, for a given output gradient dO.
+definitions, for a given output gradient dO: O = (L (.) (A A^T)) V for the second order and
+O = A (A V) for AHLA (Metodología 2), with A = L (.) Q K^T.
 """
 from __future__ import annotations
 
@@ -42,5 +43,17 @@ def hla2n_grads(q, k, v, do, eps: float = 1e-6):
     num = hla2_forward_matrix(tq, tk, tv)
     den = hla2_forward_matrix(tq, tk, torch.ones(tv.shape[:-1] + (1,), dtype=torch.float64))
     o = num / (den + eps)
+    o.backward(torch.tensor(_f64(do)))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def ahla_grads(q, k, v, do):
+    """(dQ, dK, dV) for the AHLA output O = A (A V), A = L (.) Q K^T."""
+    import torch
+    tq, tk, tv = (torch.tensor(_f64(x), requires_grad=True) for x in (q, k, v))
+    T = tq.shape[-2]
+    L = torch.tril(torch.ones(T, T, dtype=torch.float64))
+    A = L * (tq @ tk.transpose(-1, -2))
+    o = A @ (A @ tv)
     o.backward(torch.tensor(_f64(do)))
     return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()

@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle.brute as brute
-from oracle.backward import hla2_grads, hla2n_grads
+from oracle.backward import ahla_grads, hla2_grads, hla2n_grads
 
 
 def rand(T, d, dv, seed):
@@ -159,3 +159,64 @@ def test_normalised_backward_is_the_walk_on_ones_augmented_values(T, c):
     np.testing.assert_allclose(gq, want[0], rtol=1e-9, atol=1e-10)
     np.testing.assert_allclose(gk, want[1], rtol=1e-9, atol=1e-10)
     np.testing.assert_allclose(gv[:, :3], want[2], rtol=1e-9, atol=1e-10)
+
+
+# ---------------------------------------------------------------------------
+# AHLA (Metodología 2): O = A (A V)
+# ---------------------------------------------------------------------------
+
+def test_ahla_reference_matches_finite_differences():
+    q, k, v, do = rand(6, 3, 2, 11)
+    gq, gk, gv = ahla_grads(q, k, v, do)
+    f = lambda q_, k_, v_: float(np.sum(brute.ahla(q_, k_, v_) * do))   # noqa: E731
+    h = 1e-6
+    for x, g, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p, args_m = [q, k, v], [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num = (f(*args_p) - f(*args_m)) / (2 * h)
+            assert abs(g[idx] - num) <= 1e-6 * max(1.0, abs(num))
+
+
+def ahla_chunked_backward(q, k, v, do, c):
+    """Reverse walk for AHLA.  Forward per chunk (P0, E0 carried in):
+        A = L (.) Q K^T,  Y = Q P0 + A V,  O = Q E0 + A Y,  P0' = P0 + K^T V,  E0' = E0 + K^T Y.
+    Backward per chunk, given dO and the adjoints (dP0', dE0') of the states it hands on:
+        dY = A^T dO + K dE0';  dA = L (.) (dO Y^T + dY V^T);
+        dQ = dO E0^T + dY P0^T + dA K;  dK = Y dE0'^T + V dP0'^T + dA^T Q;  dV = K dP0' + A^T dY;
+        dE0 = dE0' + Q^T dO;  dP0 = dP0' + Q^T dY."""
+    d, dv = q.shape[1], v.shape[1]
+    Qs, Ks, Vs, Gs = chunks(q, c), chunks(k, c), chunks(v, c), chunks(do, c)
+    L = np.tril(np.ones((c, c)))
+    P0, E0 = np.zeros((d, dv)), np.zeros((d, dv))
+    saved = []
+    for Q, K, V in zip(Qs, Ks, Vs):
+        saved.append((P0, E0))
+        A = L * (Q @ K.T)
+        Y = Q @ P0 + A @ V
+        P0, E0 = P0 + K.T @ V, E0 + K.T @ Y
+    dP, dE = np.zeros((d, dv)), np.zeros((d, dv))
+    gq, gk, gv = [], [], []
+    for (Q, K, V, dO), (P0, E0) in zip(reversed(list(zip(Qs, Ks, Vs, Gs))), reversed(saved)):
+        A = L * (Q @ K.T)
+        Y = Q @ P0 + A @ V
+        dY = A.T @ dO + K @ dE
+        dA = L * (dO @ Y.T + dY @ V.T)
+        gq.append(dO @ E0.T + dY @ P0.T + dA @ K)
+        gk.append(Y @ dE.T + V @ dP.T + dA.T @ Q)
+        gv.append(K @ dP + A.T @ dY)
+        dE, dP = dE + Q.T @ dO, dP + Q.T @ dY
+    T = q.shape[0]
+    return tuple(np.vstack(g[::-1])[:T] for g in (gq, gk, gv))
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (9, 4), (37, 8), (64, 16), (100, 32)])
+def test_ahla_chunked_reverse_walk_matches_the_reference(T, c):
+    q, k, v, do = rand(T, 5, 3, T + 2 * c)
+    want = ahla_grads(q, k, v, do)
+    got = ahla_chunked_backward(q, k, v, do, c)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
