@@ -7,7 +7,8 @@ Contribuciones 2: the scan reproduces the serial activations exactly, which the 
 the basis of exact parallel training; it prints no gradient.  The reference here is therefore
 the plain one: reverse-mode differentiation (torch autograd, CPU, float64) of the masked-matrix
 definitions, for a given output gradient dO: O = (L (.) (A A^T)) V for the second order and
-O = A (A V) for AHLA (Metodología 2), with A = L (.) Q K^T.
+O = A (A V) for AHLA (Metodología 2) and O = (M A) V, M = L (.) (A A^T), for the third order
+(Metodología 3), with A = L (.) Q K^T.
 """
 from __future__ import annotations
 
@@ -55,5 +56,18 @@ def ahla_grads(q, k, v, do):
     L = torch.tril(torch.ones(T, T, dtype=torch.float64))
     A = L * (tq @ tk.transpose(-1, -2))
     o = A @ (A @ tv)
+    o.backward(torch.tensor(_f64(do)))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def hla3_grads(q, k, v, do):
+    """(dQ, dK, dV) for the third-order output O = (M A) V, M = L (.) (A A^T), A = L (.) Q K^T."""
+    import torch
+    tq, tk, tv = (torch.tensor(_f64(x), requires_grad=True) for x in (q, k, v))
+    T = tq.shape[-2]
+    L = torch.tril(torch.ones(T, T, dtype=torch.float64))
+    A = L * (tq @ tk.transpose(-1, -2))
+    M = L * (A @ A.transpose(-1, -2))
+    o = (M @ A) @ tv
     o.backward(torch.tensor(_f64(do)))
     return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()

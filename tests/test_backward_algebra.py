@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle.brute as brute
-from oracle.backward import ahla_grads, hla2_grads, hla2n_grads
+from oracle.backward import ahla_grads, hla2_grads, hla2n_grads, hla3_grads
 
 
 def rand(T, d, dv, seed):
@@ -220,3 +220,74 @@ def test_ahla_chunked_reverse_walk_matches_the_reference(T, c):
     got = ahla_chunked_backward(q, k, v, do, c)
     for a, b in zip(got, want):
         np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+
+
+# ---------------------------------------------------------------------------
+# third order (Metodología 3): O = (M A) V, M = L (.) (A A^T)
+# ---------------------------------------------------------------------------
+
+def test_hla3_reference_matches_finite_differences():
+    q, k, v, do = rand(6, 3, 2, 12)
+    gq, gk, gv = hla3_grads(q, k, v, do)
+    f = lambda q_, k_, v_: float(np.sum(brute.hla3(q_, k_, v_) * do))   # noqa: E731
+    h = 1e-6
+    for x, g, which in ((q, gq, 0), (k, gk, 1), (v, gv, 2)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p, args_m = [q, k, v], [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            num = (f(*args_p) - f(*args_m)) / (2 * h)
+            assert abs(g[idx] - num) <= 1e-6 * max(1.0, abs(num))
+
+
+def hla3_chunked_backward(q, k, v, do, c):
+    """Reverse walk for the third order.  Forward per chunk (S0, P0, F0 carried in):
+        A = L (.) Q K^T,  P = Q S0,  W = L (.) (P Q^T + A A^T),  Y = Q P0 + A V,  Z = P + A K,
+        O = Q F0 + W Y,   S0' = S0 + K^T K,  P0' = P0 + K^T V,  F0' = F0 + Z^T Y.
+    Backward per chunk, given dO and the adjoints (dS0', dP0', dF0'):
+        dY = W^T dO + Z dF0';  dW = L (.) dO Y^T;  dZ = Y dF0'^T;  dP = dZ + dW Q;
+        dA = L (.) (dZ K^T + dY V^T + (dW + dW^T) A);
+        dQ = dO F0^T + dW^T P + dY P0^T + dP S0^T + dA K;
+        dK = K (dS0' + dS0'^T) + V dP0'^T + A^T dZ + dA^T Q;  dV = K dP0' + A^T dY;
+        dS0 = dS0' + Q^T dP;  dP0 = dP0' + Q^T dY;  dF0 = dF0' + Q^T dO."""
+    d, dv = q.shape[1], v.shape[1]
+    Qs, Ks, Vs, Gs = chunks(q, c), chunks(k, c), chunks(v, c), chunks(do, c)
+    L = np.tril(np.ones((c, c)))
+    S0, P0, F0 = np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv))
+    saved = []
+    for Q, K, V in zip(Qs, Ks, Vs):
+        saved.append((S0, P0, F0))
+        A = L * (Q @ K.T)
+        Y = Q @ P0 + A @ V
+        Z = Q @ S0 + A @ K
+        S0, P0, F0 = S0 + K.T @ K, P0 + K.T @ V, F0 + Z.T @ Y
+    dS, dP0a, dF = np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv))
+    gq, gk, gv = [], [], []
+    for (Q, K, V, dO), (S0, P0, F0) in zip(reversed(list(zip(Qs, Ks, Vs, Gs))), reversed(saved)):
+        A = L * (Q @ K.T)
+        P = Q @ S0
+        W = L * (P @ Q.T + A @ A.T)
+        Y = Q @ P0 + A @ V
+        Z = P + A @ K
+        dY = W.T @ dO + Z @ dF
+        dW = L * (dO @ Y.T)
+        dZ = Y @ dF.T
+        dP = dZ + dW @ Q
+        dA = L * (dZ @ K.T + dY @ V.T + (dW + dW.T) @ A)
+        gq.append(dO @ F0.T + dW.T @ P + dY @ P0.T + dP @ S0.T + dA @ K)
+        gk.append(K @ (dS + dS.T) + V @ dP0a.T + A.T @ dZ + dA.T @ Q)
+        gv.append(K @ dP0a + A.T @ dY)
+        dS, dP0a, dF = dS + Q.T @ dP, dP0a + Q.T @ dY, dF + Q.T @ dO
+    T = q.shape[0]
+    return tuple(np.vstack(g[::-1])[:T] for g in (gq, gk, gv))
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (9, 4), (37, 8), (64, 16), (100, 32)])
+def test_hla3_chunked_reverse_walk_matches_the_reference(T, c):
+    q, k, v, do = rand(T, 4, 3, T + 3 * c)
+    want = hla3_grads(q, k, v, do)
+    got = hla3_chunked_backward(q, k, v, do, c)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-10)
