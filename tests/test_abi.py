@@ -231,6 +231,21 @@ def test_unmasked_op_sizes_and_errors(lib):
     assert f(*a, 1, 1, 64, 64, 64, 0, vp(0), vp(16), 64, vp(0)) == 6                       # workspace
 
 
+def test_header_is_plain_c(tmp_path):
+    """include/hla.h is a C ABI: it compiles as strict C99 (and as C++) with no CUDA header."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    src = tmp_path / "use_hla.c"
+    src.write_text('#include "hla.h"\nint main(void) { return hla_abi_version() > 0 ? 0 : 1; }\n')
+    inc = os.path.join(ROOT, "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-I", inc,
+                    str(src)], check=True)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", "c++", "-I", inc,
+                    str(src)], check=True)
+
+
 def test_product_path_never_touches_the_oracle():
     """The package (binding + CUDA sources) must not import, call or link oracle/."""
     pkg = os.path.join(ROOT, "higher_order_linear_chunked_b200")
