@@ -54,6 +54,8 @@ def parse_args(argv=None):
                    help="streaming decode steps timed after the forward (0: skip)")
     p.add_argument("--segment-chunks", type=int, default=0,
                    help="tensor-core path: 128-token chunks per segment (0 = the library's choice)")
+    p.add_argument("--workload-steps", type=int, default=10,
+                   help="timed steps per workload of the 'workloads' object (0: skip it)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -321,26 +323,29 @@ def run_ours(args):
     clk = clocks.summary()
     model = output_kernel_model(path, w)
     out_avg_ms = statistics.mean(out_ms)
-    achieved = model["flops_per_token"] * tokens / (out_avg_ms / 1e3) / 1e12
-    if model["bound"] == "tensor":
-        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-        peak_note = f"bf16 dense burst ({peak_kind})"
-    else:
-        smax = float(peaks.get("sm_max_mhz", 1965.0))
-        peak = alu_peak_tflops(smax)
-        peak_note = f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"
-    roofline = {"kernel": "output", "bound": model["bound"], "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
-                "flops_per_token": model["flops_per_token"], "kernel_ms": out_avg_ms,
-                "phase_ms": {"note": "separate loop with events between the kernels (serialised)",
-                             "step": statistics.mean([ev[0].elapsed_time(ev[3]) for ev in events]),
-                             "summary": statistics.mean(sum_ms), "scan": statistics.mean(scan_ms),
-                             "output": out_avg_ms}}
+    roofline = roofline_of(path, w, out_avg_ms, tokens, peaks, peak_kind)
     roofline["traffic"] = _traffic_from_profiles(path, w)
+    roofline["phase_ms"] = {"note": "separate loop with events between the kernels (serialised)",
+                            "step": statistics.mean([ev[0].elapsed_time(ev[3]) for ev in events]),
+                            "summary": statistics.mean(sum_ms), "scan": statistics.mean(scan_ms),
+                            "output": out_avg_ms}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, q, k, v, g)
+
+    # parity of the timed output itself: the fp64 oracle on every head and token (rank 0)
+    parity = None
+    if rank == 0 and not args.no_cpu_baseline:
+        parity = parity_against_oracle(w, out, q, k, v, g)
+
+    # the problem's five workloads at full size: throughput, the output kernel against its roofline,
+    # and the full-output parity error against the oracle (rank 0, one GPU)
+    workloads = None
+    if rank == 0 and world == 1 and args.workload_steps > 0:
+        del flush
+        workloads = measure_workloads(dev, args, peaks, peak_kind, {w.name: (value, ms_per_step, roofline,
+                                                                             parity)})
 
     if rank == 0:
         line = {
@@ -352,13 +357,104 @@ def run_ours(args):
                        "segment_chunks": args.segment_chunks or "auto",
                        "l2": "flushed before every step (512 MiB write, outside the timed events)",
                        "parallelism": f"dp{world} (independent heads per rank, no collective)"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "clocks": clk,
+            "roofline": roofline, "parity": parity, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+            "workloads": workloads, "clocks": clk,
             "gpu_launches": launches_per_step * args.steps, "device_status": status,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+TOLERANCE = {"f32": 1e-4, "bf16": 2e-2}     # max row-wise relative L2 error against the fp64 oracle
+FIVE = ("hla2_f32_1x2x256x32", "hla2n_bf16_4x16x4096x64", "hla2d_bf16_2x16x16384x64", "ahla_bf16_4x16x8192x64",
+        "hla3_f32_2x8x4096x32")
+
+
+def parity_against_oracle(w, out, q, k, v, g):
+    """Max row-wise relative L2 error of a GPU output against the fp64 oracle over every head and
+    token of the workload (the oracle runs on all host cores, one thread per head)."""
+    import oracle
+    ref = oracle.recur(w.op, q, k, v, gamma=g, eps=w.eps)
+    err = oracle.max_row_rel_err(out.detach().cpu(), ref)
+    return {"max_row_rel_err": err, "tol": TOLERANCE[w.dtype], "pass": err <= TOLERANCE[w.dtype],
+            "rows": int(w.B * w.H * w.T), "against": "fp64 oracle (serial recurrence), every head and token"}
+
+
+def roofline_of(path, w, out_ms, tokens, peaks, peak_kind):
+    model = output_kernel_model(path, w)
+    achieved = model["flops_per_token"] * tokens / (out_ms / 1e3) / 1e12
+    if model["bound"] == "tensor":
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        note = f"bf16 dense burst ({peak_kind})"
+    else:
+        smax = float(peaks.get("sm_max_mhz", 1965.0))
+        peak = alu_peak_tflops(smax)
+        note = f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"
+    return {"kernel": "output", "bound": model["bound"], "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "peak_source": note, "flops_per_token": model["flops_per_token"],
+            "kernel_ms": out_ms}
+
+
+def measure_workloads(dev, args, peaks, peak_kind, done):
+    """Every one of the five workloads at its full size, one after the other on this GPU: forward
+    throughput (CUDA events around each step, L2 flushed before it), the output kernel against its
+    roofline (phase events), and the full-output parity error against the fp64 oracle."""
+    import torch
+
+    import higher_order_linear_chunked_b200 as hla
+    res = {}
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for name in FIVE:
+        w = hla_inputs.workload(name)
+        if name in done:
+            value, ms, roof, par = done[name]
+            res[name] = {"tokens_per_s": value, "ms_per_step": ms, "roofline_frac": roof["frac"],
+                         "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "kernel_ms")},
+                         "parity": par, "note": "the headline line above"}
+            continue
+        q, k, v, g = hla_inputs.make_inputs(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        gd = g.to(dev) if g is not None else None
+        out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
+        op = hla.OP_CODES[w.op]
+        ws = hla.make_workspace(op, qd, vd, decayed=gd is not None)
+        dcode = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
+        path = "tc" if hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv) else "simt"
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            hla.forward(w.op, qd, kd, vd, gamma=gd, eps=w.eps, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.workload_steps)]
+        for a, b in bounds:
+            flush.zero_()
+            a.record()
+            hla.forward(w.op, qd, kd, vd, gamma=gd, eps=w.eps, out=out, workspace=ws)
+            b.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in bounds)
+        status = hla.read_device_status(ws)
+        par = parity_against_oracle(w, out, q, k, v, g)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.workload_steps)]
+        for ev in evs:
+            for e in ev:
+                e.record()
+        torch.cuda.synchronize()
+        for ev in evs:
+            flush.zero_()
+            hla.forward_profiled(w.op, qd, kd, vd, ev, gamma=gd, eps=w.eps, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        out_ms = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in evs)
+        roof = roofline_of(path, w, out_ms, w.tokens, peaks, peak_kind)
+        res[name] = {"tokens_per_s": w.tokens / (ms / 1e3), "ms_per_step": ms, "roofline_frac": roof["frac"],
+                     "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "kernel_ms")},
+                     "parity": par, "path": path, "dtype": w.dtype, "steps": args.workload_steps,
+                     "device_status": status,
+                     "config": {"op": w.op, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "dv": w.dv}}
+        del qd, kd, vd, out, ws
+    return res
 
 
 def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
@@ -371,9 +467,10 @@ def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
     B, H, T, d = qd.shape
     dev = qd.device
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    st = hla.state(w.op, qd, kd, vd, gamma=gd)                      # warm-up prefill (not timed)
     flush.zero_()
     ev[0].record()
-    st = hla.state(w.op, qd, kd, vd, gamma=gd)
+    st = hla.state(w.op, qd, kd, vd, gamma=gd, out=st)
     ev[1].record()
     torch.cuda.synchronize()
     prefill_ms = ev[0].elapsed_time(ev[1])
@@ -395,7 +492,8 @@ def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
     nbytes = B * H * (2 * st.shape[-1] * 4 + 3 * d * esz + vd.shape[-1] * 4)   # state in and out, q k v, o
     gbs = nbytes / (step_ms / 1e3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    return {"prefill_ms": prefill_ms, "prefill_tokens": B * H * T, "steps": steps, "us_per_step": step_ms * 1e3,
+    return {"prefill_ms": prefill_ms, "prefill_note": "second call (the first is a warm-up), L2 flushed before it",
+            "prefill_tokens": B * H * T, "steps": steps, "us_per_step": step_ms * 1e3,
             "tokens_per_s": B * H / (step_ms / 1e3), "gpu_launches_per_step": 1,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "bytes_per_step": nbytes, "peak_source": f"HBM copy ({peak_kind})"},

@@ -39,7 +39,7 @@ EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_for
            "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
            "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
            "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked",
-           "ahla_forward_normalized", "hla3_forward_normalized")
+           "ahla_forward_normalized", "hla3_forward_normalized", "hla_noalloc_read_device_status")
 
 
 class HLAError(RuntimeError):
@@ -86,6 +86,8 @@ def load_library(path: Optional[str] = None):
     lib.hla_read_device_status.restype = i
     lib.hla2_forward_normalized_noalloc.argtypes = common + [f, vp]
     lib.hla2_forward_normalized_noalloc.restype = i
+    lib.hla_noalloc_read_device_status.argtypes = [vp, ctypes.POINTER(i)]
+    lib.hla_noalloc_read_device_status.restype = i
     lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
     lib.hla_selftest_umma.restype = i
     lib.hla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]

@@ -19,6 +19,7 @@ struct Request {
     bool norm;     // ratio-normalised
     bool bf16;
     int B, H, T, d, dv;
+    int seg;       // tensor-core path: chunks per output segment (0 = automatic), read once per call
 };
 
 // Shape / dtype checks shared by the size query and the forward calls.
@@ -40,6 +41,7 @@ Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H,
     else if (op == HLA_OP_HLA2_UNMASKED) r.op = hla::OP_HLA2U;
     else r.op = hla::OP_HLA3;
     r.B = B; r.H = H; r.T = T; r.d = d; r.dv = dv;
+    r.seg = hla::tc::segment_chunks();
     return r;
 }
 
@@ -58,7 +60,7 @@ bool valid_op(hla_op_t op) { return op >= HLA_OP_HLA2 && op <= HLA_OP_HLA3_NORM;
 
 size_t workspace_for(const Request& r) {
     const int BH = r.B * r.H;
-    if (use_tc(r)) return hla::kStatusBytes + hla::tc::workspace_bytes(r.op, r.norm, BH, r.T);
+    if (use_tc(r)) return hla::kStatusBytes + hla::tc::workspace_bytes(r.op, r.norm, BH, r.T, r.seg);
     return hla::kStatusBytes + sizeof(float) * hla::simt::workspace_floats(r.op, r.d, BH, r.T);
 }
 
@@ -84,7 +86,7 @@ hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, f
     cudaEvent_t* ev = phase_events ? reinterpret_cast<cudaEvent_t*>(const_cast<void**>(phase_events)) : nullptr;
     cudaError_t e;
     if (use_tc(r)) {
-        e = hla::tc::forward(r.op, r.norm, q, k, v, gamma, eps, o, B * H, H, T, body, status, st, ev);
+        e = hla::tc::forward(r.op, r.norm, q, k, v, gamma, eps, o, B * H, H, T, body, status, st, ev, r.seg);
     } else {
         e = hla::simt::forward(r.op, r.norm, r.bf16, r.d, q, k, v, gamma, eps, o, B * H, H, T,
                                reinterpret_cast<float*>(body), st, ev);
@@ -128,7 +130,7 @@ size_t hla_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, i
 int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
     const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
-    if (use_tc(r)) return hla::tc::kernel_launches(r.op, r.norm, B * H, T);
+    if (use_tc(r)) return hla::tc::kernel_launches(r.op, r.norm, B * H, T, r.seg);
     return hla::simt::kernel_launches(r.op, r.d, T);
 }
 

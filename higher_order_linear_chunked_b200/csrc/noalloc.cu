@@ -62,3 +62,14 @@ extern "C" hla_status_t hla2_forward_normalized_noalloc(const void* q, const voi
     return hla2_forward_normalized(q, k, v, o, B, H, T, d, dv, dtype, gamma, eps, scratch,
                                    (size_t)HLA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// The status word of the last no-alloc call on this device sits at the start of the scratch
+// array (where every forward keeps it in its workspace); the regular hla_read_device_status
+// reads it from there.
+extern "C" hla_status_t hla_noalloc_read_device_status(void* stream, int* device_status) {
+    if (!device_status) return HLA_ERR_NULL;
+    void* scratch = nullptr;
+    const hla_status_t s = scratch_address(&scratch);
+    if (s != HLA_OK) return s;
+    return hla_read_device_status(scratch, stream, device_status);
+}

@@ -8,15 +8,19 @@ namespace tc {
 
 // true when (internal op, normalised, bf16, d) runs on the tcgen05 kernels
 bool supported(int op, bool norm, bool bf16, int d);
-// process-wide segment length (chunks); 0 = automatic; false if invalid
+// process-wide default segment length (chunks); 0 = automatic; false if invalid
 bool set_segment_chunks(int chunks);
-// kernels one forward enqueues
-int kernel_launches(int op, bool norm, int BH, int T);
+// the default, read once by every request (the size query and the forward each take their own
+// reading, and each call plans with the value it read)
+int segment_chunks();
+// kernels one forward enqueues (seg_chunks: the request's segment length)
+int kernel_launches(int op, bool norm, int BH, int T, int seg_chunks);
 // workspace bytes the path needs after the status block
-size_t workspace_bytes(int op, bool norm, int BH, int T);
+size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks);
 // enqueue the forward (summaries, prefixes, output); gamma: device [H] decay factors or null
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
-                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
+                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                    int seg_chunks);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

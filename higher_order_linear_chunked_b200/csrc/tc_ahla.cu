@@ -429,18 +429,18 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
 int ahla_ctas_per_sm() { return kCtasPerSM; }
 
-size_t ahla_workspace_bytes(int BH, int T) {
-    const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
+size_t ahla_workspace_bytes(int BH, int T, int seg_chunks) {
+    const Plan pl = plan(BH, T, kCtasPerSM * kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
 cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
-                         int* status, cudaStream_t st, cudaEvent_t* ev) {
+                         int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
-    const Plan pl = plan(BH, T, kCtasPerSM * kSMs);
+    const Plan pl = plan(BH, T, kCtasPerSM * kSMs, seg_chunks);
     Params prm;                              // the output walk
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = 0.f; prm.norm = 0;

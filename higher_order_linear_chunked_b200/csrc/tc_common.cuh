@@ -115,7 +115,8 @@ struct Plan {
 // Segment lengths for BH heads of T tokens when `slots` walker CTAs can run at once.  The
 // last output segment's summary is never needed, so summaries cover (NS - 1) NCH chunks per
 // head, in segments short enough to fill the machine.
-Plan plan(int BH, int T, int slots);
+// seg_chunks: chunks per output segment (0 = automatic).
+Plan plan(int BH, int T, int slots, int seg_chunks);
 
 // Up to this many summary slots per head, an output walker folds its prefix itself.
 constexpr int PH_MAX = 9;
@@ -131,10 +132,10 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
                           int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
 
 // The AHLA forward on the tcgen05 walkers (tc_ahla.cu).
-size_t ahla_workspace_bytes(int BH, int T);
+size_t ahla_workspace_bytes(int BH, int T, int seg_chunks);
 int ahla_ctas_per_sm();
 cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
-                         int* status, cudaStream_t st, cudaEvent_t* ev);
+                         int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks);
 
 }  // namespace tc
 }  // namespace hla

@@ -32,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "ptx.cuh"
 #include "simt.h"
@@ -812,7 +814,7 @@ int next_pow2(int n) {
     return p;
 }
 
-int g_segment_chunks = 0;   // 0 = automatic
+std::atomic<int> g_segment_chunks{0};   // 0 = automatic
 
 }  // namespace
 
@@ -840,7 +842,7 @@ bool make_map_out(CUtensorMap* map, float* base, int T, int BH) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-Plan plan(int BH, int T, int slots) {
+Plan plan(int BH, int T, int slots, int seg_chunks) {
     Plan pl;
     pl.NC = (T + C - 1) / C;
     // Costs in chunk-times.  One walk over CTAs of `len` chunks takes (waves of CTAs) x (len +
@@ -862,8 +864,8 @@ Plan plan(int BH, int T, int slots) {
         }
         return best;
     };
-    if (g_segment_chunks > 0) {
-        pl.NCH = g_segment_chunks;
+    if (seg_chunks > 0) {
+        pl.NCH = seg_chunks;
     } else {
         long long best = -1;                 // ties: the longer output segment
         for (int nch = 1; nch <= 16; nch *= 2) {
@@ -894,33 +896,36 @@ cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH
 
 bool set_segment_chunks(int chunks) {
     if (chunks != 0 && chunks != 1 && chunks != 2 && chunks != 4 && chunks != 8 && chunks != 16) return false;
-    g_segment_chunks = chunks;
+    g_segment_chunks.store(chunks);
     return true;
 }
+
+int segment_chunks() { return g_segment_chunks.load(); }
 
 bool supported(int op, bool norm, bool bf16, int d) {
     if (!bf16 || d != D) return false;
     return op == OP_HLA2 || op == OP_AHLA || (op == OP_HLA2D && !norm);
 }
 
-size_t workspace_bytes(int op, bool /*norm*/, int BH, int T) {
-    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T);
+size_t workspace_bytes(int op, bool /*norm*/, int BH, int T, int seg_chunks) {
+    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T, seg_chunks);
     if (op == OP_HLA2D) return decay_workspace_bytes(BH, T);
-    const Plan pl = plan(BH, T, kSMs);
+    const Plan pl = plan(BH, T, kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-int kernel_launches(int op, bool /*norm*/, int BH, int T) {
+int kernel_launches(int op, bool /*norm*/, int BH, int T, int seg_chunks) {
     if (op == OP_HLA2D) return decay_kernel_launches();
     // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
     // two launches), output walk
-    const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm() * kSMs : kSMs);
+    const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm() * kSMs : kSMs, seg_chunks);
     return pl.NSf + 1 > PH_MAX ? 4 : 2;     // else the output walker folds the prefix itself
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
-                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
-    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev);
+                    float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                    int seg_chunks) {
+    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev, seg_chunks);
     if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
@@ -928,7 +933,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
-    const Plan pl = plan(BH, T, kSMs);
+    const Plan pl = plan(BH, T, kSMs, seg_chunks);
     Params prm;                              // the output walk
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = eps; prm.norm = norm ? 1 : 0;

@@ -241,9 +241,12 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
 /*
  * Tuning knob of the tensor-core path: chunks of 128 tokens per segment (the
  * unit one CTA walks).  0 restores the automatic choice.  Values outside
- * {0, 1, 2, 4, 8, 16} return HLA_ERR_SHAPE.  Process-wide setting: it changes
- * hla_workspace_bytes() and must not be changed while calls are being made
- * from other threads.  Results do not depend on it beyond rounding.
+ * {0, 1, 2, 4, 8, 16} return HLA_ERR_SHAPE.  A process-wide default held in
+ * an atomic: every call (the size query and each forward) reads it once and
+ * plans with that one value, so a call never mixes two settings.  It changes
+ * hla_workspace_bytes(): a forward whose own reading needs more workspace
+ * than the caller passed returns HLA_ERR_WORKSPACE before any launch.
+ * Results do not depend on it beyond rounding.
  */
 hla_status_t hla_set_segment_chunks(int chunks);
 
@@ -285,6 +288,18 @@ hla_status_t hla_read_device_status(const void* workspace, void* stream, int* de
 hla_status_t hla2_forward_normalized_noalloc(const void* q, const void* k, const void* v, float* o,
                                              int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                                              const float* gamma, float eps, void* stream);
+
+/*
+ * Device status word of the last hla2_forward_normalized_noalloc() call on the
+ * current device (the paper has no counterpart).  That call keeps its status
+ * word inside the built-in scratch array, whose address callers never see, so
+ * this is how they learn whether one of its kernels gave up a bounded wait.
+ * Synchronises `stream`, then copies the word into *device_status: HLA_OK, or
+ * HLA_ERR_TIMEOUT when a bounded wait ran out (the output is then undefined).
+ * Returns HLA_ERR_NULL for a NULL device_status, HLA_ERR_CUDA if a CUDA call
+ * fails; before the first no-alloc call on the device it reports HLA_OK.
+ */
+hla_status_t hla_noalloc_read_device_status(void* stream, int* device_status);
 
 /*
  * Tensor-core layout self-check (diagnostic; no counterpart on the pages).

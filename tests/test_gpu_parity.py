@@ -233,7 +233,7 @@ def test_decay_strong_and_weak_tensor_cores(gam):
 
 
 # ---------------------------------------------------------------------------
-# the five full-size workloads: whole GPU forward, oracle on sampled heads
+# the full-size workloads: whole GPU forward against the oracle on every head and token
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("name", list(hla_inputs.WORKLOADS))
@@ -242,14 +242,12 @@ def test_full_size_workloads(name):
     q, k, v, g = hla_inputs.make_inputs(w)
     o = gpu_forward(w.op, q, k, v, g, eps=w.eps).cpu()
     assert torch.isfinite(o).all()
+    ref = oracle.recur(w.op, q, k, v, gamma=g, eps=w.eps)         # every head (host threads)
     BH = w.B * w.H
-    for bh in sorted({0, BH // 2, BH - 1}):
-        b, h = divmod(bh, w.H)
-        sl = (slice(b, b + 1), slice(h, h + 1))
-        gh = g[h:h + 1] if g is not None else None
-        ref = oracle.recur(w.op, q[sl], k[sl], v[sl], gamma=gh, eps=w.eps)
-        err = oracle.max_row_rel_err(o[sl], ref)
-        assert err <= TOL[w.dtype], (name, bh, err)
+    per_head = [oracle.max_row_rel_err(o.reshape(BH, w.T, w.dv)[bh], ref.reshape(BH, w.T, w.dv)[bh])
+                for bh in range(BH)]
+    worst = max(range(BH), key=lambda bh: per_head[bh])
+    assert per_head[worst] <= TOL[w.dtype], (name, worst, per_head[worst])
 
 
 # ---------------------------------------------------------------------------
