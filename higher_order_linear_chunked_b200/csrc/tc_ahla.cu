@@ -452,11 +452,9 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
     sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_ahla_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  ASMEM_BYTES)) != cudaSuccess)
+    if ((e = set_smem(k_ahla_walk<SUMMARY>, ASMEM_BYTES)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_ahla_walk<OUTPUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  ASMEM_BYTES)) != cudaSuccess)
+    if ((e = set_smem(k_ahla_walk<OUTPUT>, ASMEM_BYTES)) != cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
     k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);

@@ -98,6 +98,16 @@ __device__ __forceinline__ void st_row32_zero(uint8_t* tile, int row, int c0) {
 }
 
 // ---------------------------------------------------------------- host side
+// Dynamic shared memory of a kernel, with the whole unified L1 / shared array preferred as shared
+// memory: the default carveout can leave room for only one CTA of ~100 KB on an SM, which would
+// halve the walkers that are sized to run two per SM.
+template <typename K>
+inline cudaError_t set_smem(K* kernel, int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                static_cast<int>(cudaSharedmemCarveoutMaxShared));
+}
 // [BH][T][64] bf16 tensor, box = one 128-token chunk, 128-byte swizzle, zero fill past T.
 bool make_map(CUtensorMap* map, const void* base, int T, int BH);
 // [BH][T][64] fp32 output, box = 32 columns x one chunk, 128-byte swizzle (TMA stores).

@@ -654,9 +654,9 @@ cudaError_t decay_forward(const void* q, const void* k, const void* v, const flo
     prm.status = status;
     const int NC = prm.NC;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_dec_summary, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_BYTES)) != cudaSuccess)
+    if ((e = set_smem(k_dec_summary, S1_BYTES)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_dec_output, cudaFuncAttributeMaxDynamicSharedMemorySize, S3_BYTES)) != cudaSuccess)
+    if ((e = set_smem(k_dec_output, S3_BYTES)) != cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
     k_dec_summary<<<dim3(NC, BH), DNT, S1_BYTES, st>>>(mq, mk, mv, prm);

@@ -945,10 +945,10 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
     sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_walk<SUMMARY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+    if ((e = set_smem(k_walk<SUMMARY>, SMEM_BYTES)) !=
         cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(k_walk<OUTPUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+    if ((e = set_smem(k_walk<OUTPUT>, SMEM_BYTES)) !=
         cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
