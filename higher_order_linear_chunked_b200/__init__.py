@@ -39,7 +39,8 @@ EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_for
            "ahla_forward", "hla3_forward", "hla_forward_profiled", "hla_kernel_launches", "hla_uses_tensor_cores", "hla_set_segment_chunks", "hla_read_device_status", "hla_selftest_umma", "hla_selftest_wait_timeout",
            "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
            "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked",
-           "ahla_forward_normalized", "hla3_forward_normalized", "hla_noalloc_read_device_status")
+           "ahla_forward_normalized", "hla3_forward_normalized", "hla_noalloc_read_device_status",
+           "hla_backward_workspace_bytes", "hla_backward_kernel_launches", "hla2_backward")
 
 
 class HLAError(RuntimeError):
@@ -86,6 +87,12 @@ def load_library(path: Optional[str] = None):
     lib.hla_read_device_status.restype = i
     lib.hla2_forward_normalized_noalloc.argtypes = common + [f, vp]
     lib.hla2_forward_normalized_noalloc.restype = i
+    lib.hla_backward_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+    lib.hla_backward_workspace_bytes.restype = sz
+    lib.hla_backward_kernel_launches.argtypes = [i, i, i, i, i, i, i]
+    lib.hla_backward_kernel_launches.restype = i
+    lib.hla2_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, sz, vp]
+    lib.hla2_backward.restype = i
     lib.hla_noalloc_read_device_status.argtypes = [vp, ctypes.POINTER(i)]
     lib.hla_noalloc_read_device_status.restype = i
     lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
@@ -226,6 +233,34 @@ def hla3(q, k, v, out=None, workspace=None, stream=None):
 def hla2_unmasked(q, k, v, out=None, workspace=None, stream=None):
     """Unmasked second-order forward, o_t = q_t^T S_t C_t."""
     return _call(OP_HLA2_UNMASKED, q, k, v, out=out, workspace=workspace, stream=stream)
+
+
+def hla2_backward(q, k, v, dout, workspace=None, stream=None):
+    """Gradients (dq, dk, dv), fp32, of sum(O * dout) for O = hla2(q, k, v) (masked second order,
+    no decay).  dout: fp32 [B, H, T, dv] on q's device."""
+    torch = _torch()
+    _check(q, k, v)
+    if not dout.is_cuda or dout.dtype != torch.float32 or not dout.is_contiguous() or dout.shape != v.shape:
+        raise ValueError("dout must be a contiguous CUDA float32 tensor shaped like v")
+    lib = load_library()
+    B, H, T, d = q.shape
+    dvd = v.shape[-1]
+    n = int(lib.hla_backward_workspace_bytes(OP_HLA2, _dtype_code(q), B, H, T, d, dvd))
+    if n == 0:
+        raise HLAError(5, "no backward kernel for this shape/dtype")
+    if workspace is None:
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    dq = torch.empty((B, H, T, d), dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((B, H, T, dvd), dtype=torch.float32, device=q.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    vp = ctypes.c_void_p
+    rc = lib.hla2_backward(vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()), vp(dout.data_ptr()),
+                           vp(dq.data_ptr()), vp(dk.data_ptr()), vp(dv.data_ptr()), B, H, T, d, dvd, _dtype_code(q),
+                           vp(0), vp(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()), vp(st.cuda_stream))
+    if rc != HLA_OK:
+        raise HLAError(rc, "hla2_backward rejected the call")
+    return dq, dk, dv
 
 
 def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):

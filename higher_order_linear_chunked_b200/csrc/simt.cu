@@ -1198,5 +1198,256 @@ cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const voi
 }
 
 
+
+// ===========================================================================
+// Backward pass of the masked second-order output (no decay, not normalised).
+//
+// "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 4 and
+// Contribuciones 2: the page offers the exact scan as the basis of exact parallel training but
+// prints no gradient.  These kernels differentiate the chunk algebra of the forward: for chunk c
+// (Q, K, V, dO: its 64-row tiles; S0, R0: the state carried in, the forward scan's exclusive
+// prefix; dS', dR': the adjoints of the state it hands on)
+//     A = L (.) Q K^T,  P = Q S0,  W = L (.) (P Q^T + A A^T),  Z = P + A K,
+//     O = Q R0 + W V,   S0' = S0 + K^T K,   R0' = R0 + Z^T V,
+// reverse mode gives
+//     dW = L (.) dO V^T,   dV = W^T dO + Z dR',   dZ = V dR'^T,   dP = dZ + dW Q,
+//     dA = L (.) (dZ K^T + (dW + dW^T) A),
+//     dQ = dO R0^T + dW^T P + dP S0^T + dA K,   dK = K (dS' + dS'^T) + A^T dZ + dA^T Q,
+// and the adjoints handed back, dR = dR' + Q^T dO and dS = dS' + Q^T dP.  Unrolled over the
+// chunks after c they are suffix sums:
+//     dR'(c) = sum_{m > c} Q_m^T dO_m,
+//     dS'(c) = sum_{m > c} (U_m + C_m dR'(m)^T),   U_m = Q_m^T (dW_m Q_m),  C_m = Q_m^T V_m,
+// so every chunk runs in parallel apart from two element-wise suffix sums:
+//   the forward's chunk summaries and scan (S0, R0 per chunk);
+//   k_bwd_chunk: Y = Q^T dO, U, C per chunk;  k_bwd_suffix: dR' in place of Y;
+//   k_bwd_cross: X = U + C dR'^T in place of U;  k_bwd_suffix: dS' in place of X;
+//   k_bwd_out: dQ, dK, dV of every chunk.
+// Everything in fp32 on the CUDA cores; bf16 inputs are widened on load.
+// ===========================================================================
+template <int D>
+struct Bwd {
+    static constexpr int DD = D * D;
+    static constexpr int SIZE = 3 * DD;       // per chunk: [Y | dR'], [U | X | dS'], C
+};
+
+// The (dW + dW^T) view of a masked c x c tile.
+struct SymTile {
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[r * ld + c] + p[c * ld + r]; }
+};
+// Global row-major D x D matrix views.
+struct GMat {
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[r * ld + c]; }
+};
+struct GMatT {
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[c * ld + r]; }
+};
+// Store into a tile with the causal mask (column > row written as 0).
+struct PutMasked {
+    float* p;
+    int ld;
+    __device__ void operator()(int r, int c, float x) const { p[r * ld + c] = c <= r ? x : 0.f; }
+};
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_bwd_chunk(const TIn* __restrict__ q, const TIn* __restrict__ v,
+                                                  const float* __restrict__ dout, int T, int NCp,
+                                                  float* __restrict__ bw) {
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Vs = Qs + C * LD;
+    float* Os = Vs + C * LD;                  // dO
+    float* dWs = Os + C * LD;                 // C x LDC
+    float* Gs = dWs + C * LDC;                // dW Q
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Vs, v + head, t0, T);
+    load_rows<D>(Os, dout + head, t0, T);
+    __syncthreads();
+    float* out = bw + ((size_t)bh * NCp + chunk) * Bwd<D>::SIZE;
+    // Y = Q^T dO, C = Q^T V, dW = L (.) dO V^T
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Os, LD}, Zero{}, [&](int r, int c, float x) { out[r * D + c] = x; });
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Vs, LD}, Zero{}, [&](int r, int c, float x) { out[2 * D * D + r * D + c] = x; });
+    mm<C, C, D>(Tile{Os, LD}, TileT{Vs, LD}, Zero{}, PutMasked{dWs, LDC});
+    __syncthreads();
+    mm<C, D, C>(Tile{dWs, LDC}, Tile{Qs, LD}, Zero{}, Put{Gs, LD});          // dW Q
+    __syncthreads();
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Gs, LD}, Zero{}, [&](int r, int c, float x) { out[D * D + r * D + c] = x; });
+}
+
+// Exclusive suffix sum over a head's NC chunks of matrix slot `slot`, element-wise and in place.
+template <int D>
+__global__ void __launch_bounds__(NT) k_bwd_suffix(float* __restrict__ bw, int NC, int NCp, int slot) {
+    const int e = blockIdx.x * NT + threadIdx.x;
+    if (e >= D * D) return;
+    float* p = bw + (size_t)blockIdx.y * NCp * Bwd<D>::SIZE + slot * D * D + e;
+    float run = 0.f;
+    for (int c = NC - 1; c >= 0; --c) {
+        const float y = p[(size_t)c * Bwd<D>::SIZE];
+        p[(size_t)c * Bwd<D>::SIZE] = run;
+        run += y;
+    }
+}
+
+// X = U + C dR'^T per chunk, in place of U.
+template <int D>
+__global__ void __launch_bounds__(NT) k_bwd_cross(float* __restrict__ bw, int NCp) {
+    constexpr int LD = Dim<D>::LD;
+    __shared__ float Cs[D * LD], Rs[D * LD];
+    float* slot = bw + ((size_t)blockIdx.y * NCp + blockIdx.x) * Bwd<D>::SIZE;
+    load_mat<D>(Cs, slot + 2 * D * D);
+    load_mat<D>(Rs, slot);
+    __syncthreads();
+    float* U = slot + D * D;
+    mm<D, D, D>(Tile{Cs, LD}, TileT{Rs, LD}, [&](int r, int c) { return U[r * D + c]; },
+                [&](int r, int c, float x) { U[r * D + c] = x; });
+}
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_bwd_out(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                                const TIn* __restrict__ v, const float* __restrict__ dout,
+                                                int T, int NCp, const float* __restrict__ sums,
+                                                const float* __restrict__ bw, float* __restrict__ dq,
+                                                float* __restrict__ dk, float* __restrict__ dv) {
+    using S = Sum<OP_HLA2, D>;
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const float* pre = sums + ((size_t)bh * NCp + chunk) * S::SIZE;          // S0 = mat(0), R0 = mat(2)
+    const float* adj = bw + ((size_t)bh * NCp + chunk) * Bwd<D>::SIZE;       // dR' = 0, dS' = 1
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Ks = Qs + C * LD;
+    float* Vs = Ks + C * LD;                  // V, later the first three terms of dQ
+    float* Os = Vs + C * LD;                  // dO
+    float* Ps = Os + C * LD;                  // P
+    float* Zs = Ps + C * LD;                  // Z, later dP
+    float* As = Zs + C * LD;                  // C x LDC: A
+    float* Ws = As + C * LDC;                 // W, later dZ
+    float* dWs = Ws + C * LDC;                // dW
+    float* dAs = dWs + C * LDC;               // dA
+    float* M0 = dAs + C * LDC;                // D x LD: S0, later dS' + dS'^T
+    float* M1 = M0 + D * LD;                  // dR', later R0
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Ks, k + head, t0, T);
+    load_rows<D>(Vs, v + head, t0, T);
+    load_rows<D>(Os, dout + head, t0, T);
+    load_mat<D>(M0, pre + S::mat(0));
+    load_mat<D>(M1, adj);
+    __syncthreads();
+    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, PutMasked{As, LDC});     // A
+    mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, Put{Ps, LD});              // P = Q S0
+    mm<C, C, D>(Tile{Os, LD}, TileT{Vs, LD}, Zero{}, PutMasked{dWs, LDC});    // dW
+    __syncthreads();
+    mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Tile{As, LDC}, TileT{As, LDC}, Zero{}, PutMasked{Ws, LDC});  // W
+    mm<C, D, C>(Tile{As, LDC}, Tile{Ks, LD}, [&](int r, int c) { return Ps[r * LD + c]; }, Put{Zs, LD});   // Z
+    __syncthreads();
+    // dV = W^T dO + Z dR'
+    mm2<C, D, C, D>(TileT{Ws, LDC}, Tile{Os, LD}, Tile{Zs, LD}, Tile{M1, LD}, Zero{},
+                    [&](int r, int c, float x) { if (t0 + r < T) dv[head + (size_t)(t0 + r) * D + c] = x; });
+    __syncthreads();
+    mm<C, D, D>(Tile{Vs, LD}, TileT{M1, LD}, Zero{}, Put{Ws, LD});            // dZ = V dR'^T (over W)
+    __syncthreads();
+    mm<C, D, C>(Tile{dWs, LDC}, Tile{Qs, LD}, [&](int r, int c) { return Ws[r * LD + c]; }, Put{Zs, LD});  // dP
+    mm2<C, C, D, C>(Tile{Ws, LD}, TileT{Ks, LD}, SymTile{dWs, LDC}, Tile{As, LDC}, Zero{}, PutMasked{dAs, LDC});  // dA
+    load_mat<D>(M1, pre + S::mat(2));                                         // R0
+    __syncthreads();
+    // dQ = dO R0^T + dW^T P + dA K (+ dP S0^T below)
+    mm3<C, D, D, C, C>(Tile{Os, LD}, TileT{M1, LD}, TileT{dWs, LDC}, Tile{Ps, LD}, Tile{dAs, LDC}, Tile{Ks, LD},
+                       Zero{}, Put{Vs, LD});
+    __syncthreads();
+    mm<C, D, D>(Tile{Zs, LD}, TileT{M0, LD}, [&](int r, int c) { return Vs[r * LD + c]; },
+                [&](int r, int c, float x) { if (t0 + r < T) dq[head + (size_t)(t0 + r) * D + c] = x; });
+    __syncthreads();
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {                   // dS' + dS'^T
+        const int r = e / D, c = e % D;
+        M0[r * LD + c] = adj[D * D + r * D + c] + adj[D * D + c * D + r];
+    }
+    __syncthreads();
+    // dK = K (dS' + dS'^T) + A^T dZ + dA^T Q
+    mm3<C, D, D, C, C>(Tile{Ks, LD}, Tile{M0, LD}, TileT{As, LDC}, Tile{Ws, LD}, TileT{dAs, LDC}, Tile{Qs, LD},
+                       Zero{}, [&](int r, int c, float x) { if (t0 + r < T) dk[head + (size_t)(t0 + r) * D + c] = x; });
+}
+
+template <int D>
+static size_t bwd_chunk_smem() {
+    return sizeof(float) * (size_t)(4 * C * Dim<D>::LD + C * LDC);
+}
+template <int D>
+static size_t bwd_out_smem() {
+    return sizeof(float) * (size_t)(6 * C * Dim<D>::LD + 4 * C * LDC + 2 * D * Dim<D>::LD);
+}
+
+size_t backward_workspace_floats(int d, int BH, int T) {
+    const int NCp = next_pow2((T + C - 1) / C);
+    return workspace_floats(OP_HLA2, d, BH, T) + (size_t)BH * NCp * 3 * d * d;
+}
+
+int backward_launches(int d, int T) {
+    // summaries, scan, chunk terms, two suffix sums, cross term, gradients
+    return kernel_launches(OP_HLA2, d, T) - 1 + 5;
+}
+
+template <int D, typename TIn>
+static cudaError_t backward_run(const void* q, const void* k, const void* v, const float* dout, float* dq, float* dk,
+                                float* dv, int BH, int T, float* ws, cudaStream_t st) {
+    const int NC = (T + C - 1) / C;
+    const int NCp = next_pow2(NC);
+    float* sums = ws;
+    float* bw = ws + workspace_floats(OP_HLA2, D, BH, T);
+    auto ks = k_summary<OP_HLA2, D, TIn>;
+    auto kc = k_bwd_chunk<D, TIn>;
+    auto ko = k_bwd_out<D, TIn>;
+    const size_t s1 = summary_smem<D>(), s2 = bwd_chunk_smem<D>(), s3 = bwd_out_smem<D>();
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
+    // the forward's carried states: chunk summaries, then their exclusive scan
+    ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, nullptr, 1, T, NC, NCp, sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (fold_fits<OP_HLA2, D>()) {
+        auto kf = k_scan_fold<OP_HLA2, D>;
+        if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)fold_smem<OP_HLA2, D>())) != cudaSuccess)
+            return e;
+        kf<<<BH, NT, fold_smem<OP_HLA2, D>(), st>>>(sums, NC, NCp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else if ((e = scan_levels<OP_HLA2, D>(sums, NCp, BH, st)) != cudaSuccess) {
+        return e;
+    }
+    kc<<<dim3(NC, BH), NT, s2, st>>>((const TIn*)q, (const TIn*)v, dout, T, NCp, bw);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 sg((D * D + NT - 1) / NT, BH);
+    k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 0);                       // dR'
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_cross<D><<<dim3(NC, BH), NT, 0, st>>>(bw, NCp);                      // X = U + C dR'^T
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dS'
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
+                                     dv);
+    return cudaGetLastError();
+}
+
+cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st) {
+    if (bf16) {
+        if (d == 32) return backward_run<32, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+        return backward_run<64, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+    }
+    if (d == 32) return backward_run<32, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+    return backward_run<64, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+}
+
 }  // namespace simt
 }  // namespace hla

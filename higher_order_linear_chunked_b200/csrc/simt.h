@@ -38,5 +38,12 @@ int state_launches(int T);
 cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const void* q, const void* k, const void* v,
                  const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st);
 
+// Backward pass of the masked second-order output (no decay, not normalised): dq, dk, dv fp32
+// [BH][T][d] for the output gradient dout fp32 [BH][T][d]; ws: backward_workspace_floats floats.
+size_t backward_workspace_floats(int d, int BH, int T);
+int backward_launches(int d, int T);
+cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
+
 }  // namespace simt
 }  // namespace hla

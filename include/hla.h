@@ -239,6 +239,33 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
                       void* stream);
 
 /*
+ * Backward pass (gradients) of the masked second-order output, plain form
+ * ("Higher-order Linear Attention" summary, gist.science 2510.27258: Metodología 4
+ * and Contribuciones 2 present the exact chunked scan as the basis of exact
+ * parallel training; the page prints no gradient, these are reverse-mode
+ * derivatives of O = (L (.) (A A^T)) V, A = L (.) Q K^T).
+ *
+ * hla_backward_workspace_bytes: device workspace bytes hla2_backward needs for
+ * (op, dtype, B, H, T, d, dv); 0 when the request is invalid or has no backward
+ * kernel (only HLA_OP_HLA2, undecayed, d = dv in {32, 64}).
+ *
+ * hla2_backward: given the output gradient dout [B][H][T][dv] (fp32, device),
+ * writes dq, dk [B][H][T][d] and dv_out [B][H][T][dv] (fp32, device, caller-
+ * owned, 16-byte aligned) for the forward hla2_forward(q, k, v) of the same
+ * inputs (HLA_F32 or HLA_BF16; bf16 values are widened, all arithmetic is
+ * fp32).  The forward's carried chunk states are recomputed from q, k, v (no
+ * saved activations).  Kernels: the forward's chunk summaries and scan, then
+ * per-chunk adjoint terms, two suffix sums and the per-chunk gradients (see
+ * hla_backward_kernel_launches).  Errors as for the forward calls; a non-NULL
+ * gamma is HLA_ERR_UNSUPPORTED.  Enqueued on `stream`, asynchronous.
+ */
+size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
+int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
+hla_status_t hla2_backward(const void* q, const void* k, const void* v, const float* dout, float* dq,
+                           float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                           const float* gamma, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Tuning knob of the tensor-core path: chunks of 128 tokens per segment (the
  * unit one CTA walks).  0 restores the automatic choice.  Values outside
  * {0, 1, 2, 4, 8, 16} return HLA_ERR_SHAPE.  A process-wide default held in
