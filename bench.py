@@ -54,6 +54,8 @@ def parse_args(argv=None):
                    help="streaming decode steps timed after the forward (0: skip)")
     p.add_argument("--segment-chunks", type=int, default=0,
                    help="tensor-core path: 128-token chunks per segment (0 = the library's choice)")
+    p.add_argument("--backward-steps", type=int, default=10,
+                   help="timed steps of the second-order backward at the workload's shape (0: skip)")
     p.add_argument("--workload-steps", type=int, default=10,
                    help="timed steps per workload of the 'workloads' object (0: skip it)")
     args = p.parse_args(argv)
@@ -320,6 +322,9 @@ def run_ours(args):
     decode = None
     if args.decode_steps > 0:
         decode = decode_measure(w, qd, kd, vd, gd, flush, args.decode_steps, peaks, peak_kind)
+    backward = None
+    if args.backward_steps > 0 and w.op in ("hla2", "hla2n") and gd is None:
+        backward = backward_measure(w, qd, kd, vd, flush, args.backward_steps, peaks, q, k, v, rank)
     clk = clocks.summary()
     model = output_kernel_model(path, w)
     out_avg_ms = statistics.mean(out_ms)
@@ -358,7 +363,7 @@ def run_ours(args):
                        "l2": "flushed before every step (512 MiB write, outside the timed events)",
                        "parallelism": f"dp{world} (independent heads per rank, no collective)"},
             "roofline": roofline, "parity": parity, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
-            "workloads": workloads, "clocks": clk,
+            "backward": backward, "workloads": workloads, "clocks": clk,
             "gpu_launches": launches_per_step * args.steps, "device_status": status,
         }
         print(json.dumps(line), flush=True)
@@ -455,6 +460,70 @@ def measure_workloads(dev, args, peaks, peak_kind, done):
                      "config": {"op": w.op, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "dv": w.dv}}
         del qd, kd, vd, out, ws
     return res
+
+
+def backward_measure(w, qd, kd, vd, flush, steps, peaks, q, k, v, rank):
+    """The masked second-order backward (hla2_backward) on the workload's inputs with a seeded fp32
+    output gradient: time per call (CUDA events, L2 flushed before each), tokens/s, the gradient
+    kernels against the FP32 FFMA peak, and a directional-derivative check of the result against
+    the fp64 oracle's forward on one head (rank 0)."""
+    import numpy as np
+    import torch
+
+    import higher_order_linear_chunked_b200 as hla
+    dev = qd.device
+    g = torch.Generator("cpu").manual_seed(w.seed + 1234)
+    do = torch.randn(tuple(qd.shape[:3]) + (vd.shape[-1],), generator=g, dtype=torch.float32)
+    dod = do.to(dev)
+    ws = torch.empty(hla.load_library().hla_backward_workspace_bytes(hla.OP_HLA2, hla.HLA_BF16 if w.dtype == "bf16"
+                                                                      else hla.HLA_F32, w.B, w.H, w.T, w.d, w.dv),
+                     dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        grads = hla.hla2_backward(qd, kd, vd, dod, workspace=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        grads = hla.hla2_backward(qd, kd, vd, dod, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    c, D = 64, w.d
+    # gradient products per 64-token chunk, in multiply-adds: chunk terms (Q^T dO, Q^T V, dO V^T,
+    # dW Q, Q^T (dW Q)), the cross term C dR'^T, and the chunk gradients (A, P, dW, W, Z, dV, dZ,
+    # dP, dA, dQ, dK); the forward summaries it recomputes are not counted
+    macs = (3 * c * D * D + 2 * c * c * D) + D ** 3 + (8 * c * c * D + 6 * c * D * D + 2 * c ** 3 + 3 * c * c * D)
+    flops_per_token = 2 * macs / c
+    achieved = flops_per_token * w.tokens / (ms / 1e3) / 1e12
+    smax = float(peaks.get("sm_max_mhz", 1965.0))
+    peak = alu_peak_tflops(smax)
+    check = None
+    if rank == 0:
+        b_, h_ = 0, 0
+        rng = np.random.default_rng(0)
+        import oracle
+        qh, kh, vh, doh = (x[b_, h_].double().numpy() for x in (q, k, v, do))
+        dirs = [rng.standard_normal(x.shape) for x in (qh, kh, vh)]
+        eps = 1e-4
+
+        def f(s):
+            o = oracle.recur("hla2", (qh + s * dirs[0])[None, None], (kh + s * dirs[1])[None, None],
+                             (vh + s * dirs[2])[None, None])[0, 0]
+            return float(np.sum(o * doh))
+        num = (f(eps) - f(-eps)) / (2 * eps)
+        ana = sum(float(np.sum(gr[b_, h_].double().cpu().numpy() * dr)) for gr, dr in zip(grads, dirs))
+        check = {"directional_derivative_rel_err": abs(ana - num) / max(1.0, abs(num)), "head": [b_, h_],
+                 "against": "central difference of the fp64 oracle forward"}
+    return {"op": "hla2 (plain masked second order)", "ms": ms, "tokens_per_s": w.tokens / (ms / 1e3),
+            "gpu_launches_per_step": hla.load_library().hla_backward_kernel_launches(
+                hla.OP_HLA2, hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32, w.B, w.H, w.T, w.d, w.dv),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "flops_per_token": flops_per_token,
+                         "peak_source": f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"},
+            "check": check, "l2": "flushed before every call (outside the events)"}
 
 
 def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):

@@ -43,7 +43,11 @@ _SRC = os.path.join(_HERE, "hla_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4, "hla2u": 5, "ahlan": 6, "hla3n": 7}
+OPS = {"hla2": 0, "hla2n": 1, "hla2d": 2, "ahla": 3, "hla3": 4, "hla2u": 5, "ahlan": 6, "hla3n": 7,
+       "ahlad": 3, "hla3d": 4}
+# op names that require a gamma (the decayed forms); every other op except "hla2u" takes an
+# optional gamma that selects its decayed form
+DECAYED = ("hla2d", "ahlad", "hla3d")
 
 
 def build(force: bool = False) -> str:
@@ -66,9 +70,9 @@ def _load():
         lib.oracle_hla2_head.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double, i, ctypes.c_double,
                                          dp, dp, dp, dp, dp, dp]
         lib.oracle_hla2_head.restype = None
-        lib.oracle_ahla_head.argtypes = [dp, dp, dp, i, i, i, dp, dp, dp]
+        lib.oracle_ahla_head.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double, dp, dp, dp]
         lib.oracle_ahla_head.restype = None
-        lib.oracle_hla3_head.argtypes = [dp, dp, dp, i, i, i, dp, dp, dp, dp]
+        lib.oracle_hla3_head.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double, dp, dp, dp, dp]
         lib.oracle_hla3_head.restype = None
         lib.oracle_hla2u_head.argtypes = [dp, dp, dp, i, i, i, dp, dp, dp]
         lib.oracle_hla2u_head.restype = None
@@ -98,8 +102,13 @@ def recur(op: str, q, k, v, gamma=None, eps: float = 1e-6, nthreads: Optional[in
     "Normalización"), "hla2d" (decayed, Contribuciones 2; gamma [H]), "ahla"
     (Metodología 2), "hla3" (Metodología 3), "hla2u" (the unmasked configuration of
     Contribuciones 2: o_t = q_t^T S_t C_t), "ahlan" / "hla3n" (ratio-normalised: divided by
-    the same operator on a ones value column, plus eps).
+    the same operator on a ones value column, plus eps), "ahlad" / "hla3d" (AHLA / third order
+    with per-head decay, gamma [H]: every state scaled by gamma before each update, the reading
+    Contribuciones 2's decayed operators get for the second order).  A gamma passed with "hla2",
+    "hla2n", "ahla", "hla3", "ahlan" or "hla3n" selects the decayed form of that op.
     """
+    if op in DECAYED and gamma is None:
+        raise ValueError(f"op {op} needs gamma")
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, T, d = q.shape
@@ -143,8 +152,9 @@ def hla2_run(q, k, v, state=None, gamma: Optional[float] = None, normalized: boo
     return o, st
 
 
-def ahla_run(q, k, v, state=None, want_output: bool = True):
-    """AHLA recurrence over one head from ``state`` = dict(P, E) or None."""
+def ahla_run(q, k, v, state=None, want_output: bool = True, gamma: Optional[float] = None):
+    """AHLA recurrence over one head from ``state`` = dict(P, E) or None; decayed (P, E scaled
+    by gamma before every update) when ``gamma`` is not None."""
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     T, d = q.shape
@@ -154,12 +164,14 @@ def ahla_run(q, k, v, state=None, want_output: bool = True):
     else:
         st = {key: np.array(val, dtype=np.float64, copy=True, order="C") for key, val in state.items()}
     o = np.zeros((T, dv)) if want_output else None
-    lib.oracle_ahla_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, _ptr(st["P"]), _ptr(st["E"]), _ptr(o))
+    lib.oracle_ahla_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, 1 if gamma is not None else 0,
+                         float(gamma if gamma is not None else 1.0), _ptr(st["P"]), _ptr(st["E"]), _ptr(o))
     return o, st
 
 
-def hla3_run(q, k, v, state=None, want_output: bool = True):
-    """Third-order recurrence over one head from ``state`` = dict(S, P, F) or None."""
+def hla3_run(q, k, v, state=None, want_output: bool = True, gamma: Optional[float] = None):
+    """Third-order recurrence over one head from ``state`` = dict(S, P, F) or None; decayed (S, P,
+    F scaled by gamma before every update) when ``gamma`` is not None."""
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     T, d = q.shape
@@ -169,7 +181,8 @@ def hla3_run(q, k, v, state=None, want_output: bool = True):
     else:
         st = {key: np.array(val, dtype=np.float64, copy=True, order="C") for key, val in state.items()}
     o = np.zeros((T, dv)) if want_output else None
-    lib.oracle_hla3_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, _ptr(st["S"]), _ptr(st["P"]),
+    lib.oracle_hla3_head(_ptr(q), _ptr(k), _ptr(v), T, d, dv, 1 if gamma is not None else 0,
+                         float(gamma if gamma is not None else 1.0), _ptr(st["S"]), _ptr(st["P"]),
                          _ptr(st["F"]), _ptr(o))
     return o, st
 

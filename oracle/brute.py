@@ -105,22 +105,61 @@ def hla3(q, k, v):
     return (M @ A) @ _f64(v)
 
 
+def _decay_weights(gamma, lead, T):
+    """Gamma[..., t, j] = gamma^(t - j) for j <= t, else 0; gamma per head ([H] for [B,H,T,d]
+    inputs) or a scalar."""
+    g = np.asarray(gamma, dtype=np.float64)
+    if g.ndim == 1 and len(lead) == 2:
+        g = g[None, :, None, None]
+    else:
+        g = g.reshape((1,) * (len(lead) + 2))
+    idx = np.arange(T, dtype=np.float64)
+    diff = idx[:, None] - idx[None, :]
+    return np.where(diff >= 0, g ** np.maximum(diff, 0.0), 0.0)
+
+
+def ahla_decay(q, k, v, gamma):
+    """AHLA with per-head decay under the reading "scale every state by gamma, then update":
+    P_t = gamma P + k v^T, E_t = gamma E + k (q^T P_t), o_t = q_t^T E_t, which unrolls to
+        o_t = sum_{j<=t} sum_{i<=j} gamma^(t-i) (q_t.k_j)(q_j.k_i) v_i,
+    i.e. O = At (At V) with At = G (.) A, G_tj = gamma^(t-j): gamma^(t-i) = gamma^(t-j) gamma^(j-i)."""
+    q, k = _f64(q), _f64(k)
+    At = scores(q, k) * _decay_weights(gamma, q.shape[:-2], q.shape[-2])
+    return At @ (At @ _f64(v))
+
+
+def hla3_decay(q, k, v, gamma):
+    """Third order with per-head decay under the same reading (S, P, F scaled before each update):
+        o_t = sum_{s<=t} sum_{a<=s} sum_{b<=s} gamma^(t-a) gamma^(s-b) (q_t.k_a)(q_s.k_a)(q_s.k_b) v_b,
+    i.e. O = (L (.) (At A^T)) (At V) with At = G (.) A."""
+    q, k = _f64(q), _f64(k)
+    A = scores(q, k)
+    At = A * _decay_weights(gamma, q.shape[:-2], q.shape[-2])
+    M = _tril(At @ np.swapaxes(A, -1, -2))
+    return M @ (At @ _f64(v))
+
+
 def forward(op: str, q, k, v, gamma=None, eps: float = 1e-6):
     """Dispatch by op name, same names as :func:`oracle.recur`."""
     if op == "hla2":
-        return hla2(q, k, v)
+        return hla2(q, k, v) if gamma is None else hla2_decay(q, k, v, gamma)
     if op == "hla2n":
-        return hla2(q, k, v, normalized=True, eps=eps)
+        return hla2(q, k, v, normalized=True, eps=eps) if gamma is None else \
+            hla2_decay(q, k, v, gamma, normalized=True, eps=eps)
     if op == "hla2d":
         return hla2_decay(q, k, v, gamma)
-    if op == "ahla":
-        return ahla(q, k, v)
-    if op == "hla3":
-        return hla3(q, k, v)
+    if op in ("ahla", "ahlad"):
+        return ahla(q, k, v) if gamma is None else ahla_decay(q, k, v, gamma)
+    if op in ("hla3", "hla3d"):
+        return hla3(q, k, v) if gamma is None else hla3_decay(q, k, v, gamma)
     if op == "hla2u":
         return hla2u(q, k, v)
     if op in ("ahlan", "hla3n"):
-        f = ahla if op == "ahlan" else hla3
+        if gamma is None:
+            f = ahla if op == "ahlan" else hla3
+        else:
+            base = ahla_decay if op == "ahlan" else hla3_decay
+            f = lambda q_, k_, v_: base(q_, k_, v_, gamma)   # noqa: E731
         ones = np.ones(_f64(q).shape[:-1] + (1,))
         return f(q, k, v) / (f(q, k, ones) + eps)
     raise ValueError(op)

@@ -31,6 +31,10 @@
  *   - Metodología 3 (third order): A A^T A with A = Q K^T, masked, i.e.
  *     O = (M A) V with M = L (.) (A A^T), A = L (.) Q K^T; streaming with the
  *     prefix moments S^K_t, P^KV_t and the running sum F_t.
+ *   - Contribuciones 2 names masked operators with exponential decay for the
+ *     family, with no formula for AHLA or the third order either.  The reading
+ *     is the second order's: before each token's update every state of the
+ *     recurrence (AHLA: P, E; third order: S, P, F) is multiplied by gamma.
  *
  * Everything is the serial token-by-token recurrence, evaluated in double, with
  * the products written as the plain loops they are.  q_t^T (S C - G) is
@@ -161,15 +165,18 @@ void oracle_hla2u_head(const double* q, const double* k, const double* v,
 /*
  * One head.  State in/out: P[d][dv] (= sum k v^T, inclusive of t) and
  * E[d][dv] (= sum_j k_j (q_j^T P_j)).  o_t = q_t^T E_t.
+ * decay != 0: P and E are multiplied by gamma before every token's update.
  */
 void oracle_ahla_head(const double* q, const double* k, const double* v,
-                      int T, int d, int dv, double* P, double* E, double* o)
+                      int T, int d, int dv, int decay, double gamma, double* P, double* E, double* o)
 {
     double* qP = (double*)malloc(sizeof(double) * (size_t)dv);
     for (int t = 0; t < T; ++t) {
         const double* qt = q + (size_t)t * d;
         const double* kt = k + (size_t)t * d;
         const double* vt = v + (size_t)t * dv;
+        if (decay)
+            for (int a = 0; a < d * dv; ++a) { P[a] *= gamma; E[a] *= gamma; }
         for (int a = 0; a < d; ++a)
             for (int c = 0; c < dv; ++c) P[(size_t)a * dv + c] += kt[a] * vt[c];
         for (int c = 0; c < dv; ++c) {
@@ -199,9 +206,10 @@ void oracle_ahla_head(const double* q, const double* k, const double* v,
  * (= sum k v^T, inclusive), F[d][dv] (= sum_s (S_s q_s)(q_s^T P_s)).
  * o_t = q_t^T F_t.  Term by term: q_t^T S_s q_s is the masked (A A^T)_{ts}
  * and q_s^T P_s is row s of A V, so o = (M A) V with M = L (.) (A A^T).
+ * decay != 0: S, P and F are multiplied by gamma before every token's update.
  */
 void oracle_hla3_head(const double* q, const double* k, const double* v,
-                      int T, int d, int dv, double* S, double* P, double* F, double* o)
+                      int T, int d, int dv, int decay, double gamma, double* S, double* P, double* F, double* o)
 {
     double* Sq = (double*)malloc(sizeof(double) * (size_t)d);
     double* qP = (double*)malloc(sizeof(double) * (size_t)dv);
@@ -209,6 +217,10 @@ void oracle_hla3_head(const double* q, const double* k, const double* v,
         const double* qt = q + (size_t)t * d;
         const double* kt = k + (size_t)t * d;
         const double* vt = v + (size_t)t * dv;
+        if (decay) {
+            for (int a = 0; a < d * d; ++a) S[a] *= gamma;
+            for (int a = 0; a < d * dv; ++a) { P[a] *= gamma; F[a] *= gamma; }
+        }
         for (int a = 0; a < d; ++a) {
             for (int b = 0; b < d; ++b) S[(size_t)a * d + b] += kt[a] * kt[b];
             for (int c = 0; c < dv; ++c) P[(size_t)a * dv + c] += kt[a] * vt[c];
@@ -255,7 +267,8 @@ typedef struct {
 } job_t;
 
 /* o = num / (den + eps), den the same operator run on a ones value column (one column). */
-static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, double* o);
+static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, int dec, double g,
+                               double* o);
 
 static void run_head(job_t* J, int bh)
 {
@@ -269,38 +282,42 @@ static void run_head(job_t* J, int bh)
     double* c = (double*)calloc((size_t)d * dv, sizeof(double));
     double* m = (double*)calloc((size_t)d, sizeof(double));
     double* h = (double*)calloc((size_t)d, sizeof(double));
+    /* a gamma array decays every op that has a decayed form (the unmasked one has none) */
+    const int dec = J->gamma != NULL;
+    const double g = dec ? J->gamma[bh % J->H] : 1.0;
     switch (J->op) {
     case OP_HLA2:
-        oracle_hla2_head(q, k, v, T, d, dv, 0, 1.0, 0, 0.0, a, b, c, m, h, o);
+        oracle_hla2_head(q, k, v, T, d, dv, dec, g, 0, 0.0, a, b, c, m, h, o);
         break;
     case OP_HLA2N:
-        oracle_hla2_head(q, k, v, T, d, dv, 0, 1.0, 1, J->eps, a, b, c, m, h, o);
+        oracle_hla2_head(q, k, v, T, d, dv, dec, g, 1, J->eps, a, b, c, m, h, o);
         break;
     case OP_HLA2D:
-        oracle_hla2_head(q, k, v, T, d, dv, 1, J->gamma[bh % J->H], 0, 0.0, a, b, c, m, h, o);
+        oracle_hla2_head(q, k, v, T, d, dv, 1, g, 0, 0.0, a, b, c, m, h, o);
         break;
     case OP_AHLA:
-        oracle_ahla_head(q, k, v, T, d, dv, b, c, o);
+        oracle_ahla_head(q, k, v, T, d, dv, dec, g, b, c, o);
         break;
     case OP_HLA3:
-        oracle_hla3_head(q, k, v, T, d, dv, a, b, c, o);
+        oracle_hla3_head(q, k, v, T, d, dv, dec, g, a, b, c, o);
         break;
     case OP_HLA2U:
         oracle_hla2u_head(q, k, v, T, d, dv, a, b, o);
         break;
     case OP_AHLAN:
-        oracle_ahla_head(q, k, v, T, d, dv, b, c, o);
-        divide_by_ones_run(J, q, k, T, d, dv, o);
+        oracle_ahla_head(q, k, v, T, d, dv, dec, g, b, c, o);
+        divide_by_ones_run(J, q, k, T, d, dv, dec, g, o);
         break;
     case OP_HLA3N:
-        oracle_hla3_head(q, k, v, T, d, dv, a, b, c, o);
-        divide_by_ones_run(J, q, k, T, d, dv, o);
+        oracle_hla3_head(q, k, v, T, d, dv, dec, g, a, b, c, o);
+        divide_by_ones_run(J, q, k, T, d, dv, dec, g, o);
         break;
     }
     free(a); free(b); free(c); free(m); free(h);
 }
 
-static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, double* o)
+static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T, int d, int dv, int dec, double g,
+                               double* o)
 {
     double* ones = (double*)malloc(sizeof(double) * (size_t)T);
     double* den = (double*)malloc(sizeof(double) * (size_t)T);
@@ -308,8 +325,8 @@ static void divide_by_ones_run(job_t* J, const double* q, const double* k, int T
     double* s2 = (double*)calloc((size_t)d, sizeof(double));
     double* s3 = (double*)calloc((size_t)d, sizeof(double));
     for (int t = 0; t < T; ++t) ones[t] = 1.0;
-    if (J->op == OP_AHLAN) oracle_ahla_head(q, k, ones, T, d, 1, s2, s3, den);
-    else oracle_hla3_head(q, k, ones, T, d, 1, s1, s2, s3, den);
+    if (J->op == OP_AHLAN) oracle_ahla_head(q, k, ones, T, d, 1, dec, g, s2, s3, den);
+    else oracle_hla3_head(q, k, ones, T, d, 1, dec, g, s1, s2, s3, den);
     for (int t = 0; t < T; ++t)
         for (int c = 0; c < dv; ++c) o[(size_t)t * dv + c] /= den[t] + J->eps;
     free(ones); free(den); free(s1); free(s2); free(s3);
@@ -330,7 +347,9 @@ static void* worker(void* arg)
 
 /*
  * All B*H heads of one workload.  q, k: [B*H][T][d]; v, o: [B*H][T][dv];
- * gamma: [H] (decayed op only, else NULL).  nthreads <= 0 means one.
+ * gamma: [H] or NULL.  Required by OP_HLA2D; with any other op except
+ * OP_HLA2U a non-NULL gamma selects that op's decayed form.  nthreads <= 0
+ * means one.
  * Returns 0, or -1 on bad arguments.
  */
 int oracle_forward(int op, int B, int H, int T, int d, int dv,
@@ -339,6 +358,7 @@ int oracle_forward(int op, int B, int H, int T, int d, int dv,
 {
     if (B < 1 || H < 1 || T < 0 || d < 1 || dv < 1 || !q || !k || !v || !o) return -1;
     if (op == OP_HLA2D && !gamma) return -1;
+    if (op == OP_HLA2U && gamma) return -1;
     if (op < OP_HLA2 || op > OP_HLA3N) return -1;
     job_t J;
     J.op = op; J.BH = B * H; J.H = H; J.T = T; J.d = d; J.dv = dv;

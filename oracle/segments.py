@@ -20,14 +20,20 @@ second order (optionally decayed, gamma = 1 for none)
                G = rho_B G_A + G_B + rho_B Khat_B C_A,
                h = rho_B h_A + h_B + rho_B Khat_B m_A,
                Khat = Khat_A + Khat_B,  rho = rho_A rho_B.
-AHLA
-    state P, E; map D = sum k q^T.
-    A then B:  P = P_A + P_B,  D = D_A + D_B,  E = E_A + E_B + D_B P_A.
-third order
-    state S, P, F; maps Q2 = sum q q^T, X = sum_s q_s q_s^T P_s, Z = sum_s S_s q_s q_s^T
-    (P_s, S_s local to the segment, inclusive of s).
-    A then B:  S, P, Q2 add;  Z = Z_A + Z_B + S_A Q2_B;  X = X_A + X_B + Q2_B P_A;
-               F = F_A + F_B + S_A Q2_B P_A + S_A X_B + Z_B P_A.
+AHLA (optionally decayed: P, E scaled by gamma before every update)
+    state P, E; maps D = sum k q^T (undecayed), rho = gamma^len.
+    A then B:  P = rho_B P_A + P_B,  D = D_A + D_B,  E = rho_B E_A + E_B + rho_B D_B P_A,
+               rho = rho_A rho_B.
+third order (optionally decayed: S, P, F scaled by gamma before every update)
+    state S, P, F; maps Q2 = sum_s gamma^tau_s q_s q_s^T (tau_s = 1-based position in the
+    segment), X = sum_s q_s q_s^T P_s, Z = sum_s S_s q_s q_s^T (P_s, S_s local to the segment,
+    inclusive of s), rho = gamma^len.
+    A then B:  S = rho_B S_A + S_B,  P = rho_B P_A + P_B,  Q2 = Q2_A + rho_A Q2_B,
+               Z = Z_A + Z_B + S_A Q2_B,  X = X_A + X_B + Q2_B P_A,
+               F = rho_B F_A + F_B + rho_B (S_A Q2_B P_A + S_A X_B + Z_B P_A),  rho = rho_A rho_B.
+    (A token s of B sees S_s = gamma^tau_s S_A + S^B_s and P_s = gamma^tau_s P_A + P^B_s; its F term
+    decays by gamma^(len_B - tau_s) to the end of B.)  With gamma = 1 every rho is 1 and Q2 the
+    plain sum of q q^T.
 """
 from __future__ import annotations
 
@@ -53,31 +59,36 @@ def hla2_summary(q, k, v, gamma: Optional[float] = None) -> Summary:
     return st
 
 
-def ahla_summary(q, k, v) -> Summary:
+def ahla_summary(q, k, v, gamma: Optional[float] = None) -> Summary:
     q, k, v = _f64(q), _f64(k), _f64(v)
-    _, st = ahla_run(q, k, v, None, want_output=False)
+    _, st = ahla_run(q, k, v, None, want_output=False, gamma=gamma)
     st["D"] = k.T @ q
+    st["rho"] = np.array((1.0 if gamma is None else float(gamma)) ** q.shape[0])
     return st
 
 
-def hla3_summary(q, k, v) -> Summary:
+def hla3_summary(q, k, v, gamma: Optional[float] = None) -> Summary:
     q, k, v = _f64(q), _f64(k), _f64(v)
     T, d = q.shape
     dv = v.shape[1]
-    _, st = hla3_run(q, k, v, None, want_output=False)
+    g = 1.0 if gamma is None else float(gamma)
+    _, st = hla3_run(q, k, v, None, want_output=False, gamma=gamma)
     S = np.zeros((d, d))
     P = np.zeros((d, dv))
+    Q2 = np.zeros((d, d))
     X = np.zeros((d, dv))
     Z = np.zeros((d, d))
     for s in range(T):
-        S += np.outer(k[s], k[s])
-        P += np.outer(k[s], v[s])
+        S = g * S + np.outer(k[s], k[s])
+        P = g * P + np.outer(k[s], v[s])
         qq = np.outer(q[s], q[s])
+        Q2 += g ** (s + 1) * qq
         X += qq @ P
         Z += S @ qq
-    st["Q2"] = q.T @ q
+    st["Q2"] = Q2
     st["X"] = X
     st["Z"] = Z
+    st["rho"] = np.array(g ** T)
     return st
 
 
@@ -91,12 +102,12 @@ def hla2_identity(d: int, dv: int) -> Summary:
 
 
 def ahla_identity(d: int, dv: int) -> Summary:
-    return dict(P=np.zeros((d, dv)), E=np.zeros((d, dv)), D=np.zeros((d, d)))
+    return dict(P=np.zeros((d, dv)), E=np.zeros((d, dv)), D=np.zeros((d, d)), rho=np.array(1.0))
 
 
 def hla3_identity(d: int, dv: int) -> Summary:
     return dict(S=np.zeros((d, d)), P=np.zeros((d, dv)), F=np.zeros((d, dv)), Q2=np.zeros((d, d)),
-                X=np.zeros((d, dv)), Z=np.zeros((d, d)))
+                X=np.zeros((d, dv)), Z=np.zeros((d, d)), rho=np.array(1.0))
 
 
 # --------------------------------------------------------------------------
@@ -117,18 +128,22 @@ def hla2_combine(A: Summary, B: Summary) -> Summary:
 
 
 def ahla_combine(A: Summary, B: Summary) -> Summary:
-    return dict(P=A["P"] + B["P"], E=A["E"] + B["E"] + B["D"] @ A["P"], D=A["D"] + B["D"])
+    r = B["rho"]
+    return dict(P=r * A["P"] + B["P"], E=r * A["E"] + B["E"] + r * (B["D"] @ A["P"]), D=A["D"] + B["D"],
+                rho=A["rho"] * B["rho"])
 
 
 def hla3_combine(A: Summary, B: Summary) -> Summary:
+    r = B["rho"]
     SQ = A["S"] @ B["Q2"]
     return dict(
-        S=A["S"] + B["S"],
-        P=A["P"] + B["P"],
-        Q2=A["Q2"] + B["Q2"],
+        S=r * A["S"] + B["S"],
+        P=r * A["P"] + B["P"],
+        Q2=A["Q2"] + A["rho"] * B["Q2"],
         Z=A["Z"] + B["Z"] + SQ,
         X=A["X"] + B["X"] + B["Q2"] @ A["P"],
-        F=A["F"] + B["F"] + SQ @ A["P"] + A["S"] @ B["X"] + B["Z"] @ A["P"],
+        F=r * A["F"] + B["F"] + r * (SQ @ A["P"] + A["S"] @ B["X"] + B["Z"] @ A["P"]),
+        rho=A["rho"] * B["rho"],
     )
 
 
@@ -200,29 +215,29 @@ def hla2_scan_forward(q, k, v, lengths: List[int], gamma: Optional[float] = None
     return np.concatenate(outs, axis=0)
 
 
-def ahla_scan_forward(q, k, v, lengths: List[int], scan=blelloch_exclusive):
+def ahla_scan_forward(q, k, v, lengths: List[int], scan=blelloch_exclusive, gamma: Optional[float] = None):
     q, k, v = _f64(q), _f64(k), _f64(v)
     b = split_points(q.shape[0], lengths)
-    sums = [ahla_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]])
+    sums = [ahla_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], gamma)
             for i in range(len(lengths))]
     pre = scan(sums, ahla_combine, ahla_identity(q.shape[1], v.shape[1]))
     outs = []
     for i in range(len(lengths)):
         st = {key: pre[i][key] for key in ("P", "E")}
-        o, _ = ahla_run(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], st)
+        o, _ = ahla_run(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], st, gamma=gamma)
         outs.append(o)
     return np.concatenate(outs, axis=0)
 
 
-def hla3_scan_forward(q, k, v, lengths: List[int], scan=blelloch_exclusive):
+def hla3_scan_forward(q, k, v, lengths: List[int], scan=blelloch_exclusive, gamma: Optional[float] = None):
     q, k, v = _f64(q), _f64(k), _f64(v)
     b = split_points(q.shape[0], lengths)
-    sums = [hla3_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]])
+    sums = [hla3_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], gamma)
             for i in range(len(lengths))]
     pre = scan(sums, hla3_combine, hla3_identity(q.shape[1], v.shape[1]))
     outs = []
     for i in range(len(lengths)):
         st = {key: pre[i][key] for key in ("S", "P", "F")}
-        o, _ = hla3_run(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], st)
+        o, _ = hla3_run(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], st, gamma=gamma)
         outs.append(o)
     return np.concatenate(outs, axis=0)

@@ -62,6 +62,12 @@ def test_golden_hand_examples(case):
         exp = np.asarray(case["hla2d"], dtype=np.float64)
         np.testing.assert_allclose(oracle.recur("hla2d", q, k, v, gamma=g)[0, 0], exp, rtol=0, atol=1e-12)
         np.testing.assert_allclose(brute.hla2_decay(q, k, v, g)[0, 0], exp, rtol=0, atol=1e-12)
+    for op in ("ahlad", "hla3d"):
+        if op in case:
+            g = np.array([case["hla2d_gamma"]])
+            exp = np.asarray(case[op], dtype=np.float64)
+            np.testing.assert_allclose(oracle.recur(op, q, k, v, gamma=g)[0, 0], exp, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(brute.forward(op, q, k, v, gamma=g)[0, 0], exp, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------------------
@@ -171,17 +177,22 @@ def test_literal_sums(seed):
 # recurrence vs masked-matrix definition (exactness claim)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n", "ahlad",
+                                "hla3d", "hla2n+g", "ahlan+g", "hla3n+g"])
 @pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (1, 2, 17, 3, 2), (2, 2, 64, 4, 4), (1, 1, 40, 1, 3)])
 def test_recur_equals_brute(op, shape):
+    """The serial recurrence equals the masked-matrix definition for every op; "op+g" is the
+    ratio-normalised op with per-head decay (the gamma argument selects the decayed form)."""
     B, H, T, d, dv = shape
     rng = np.random.default_rng(T * 31 + d)
     q = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
     k = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
     v = rng.standard_normal((B, H, T, dv))
-    if op in ("hla2n", "ahlan", "hla3n"):
+    name = op.split("+")[0]
+    if name in ("hla2n", "ahlan", "hla3n"):
         q, k = np.abs(q), np.abs(k)
-    g = rng.uniform(0.9, 0.999, size=H)
+    g = rng.uniform(0.9, 0.999, size=H) if (op.endswith("+g") or name in oracle.DECAYED) else None
+    op = name
     r = oracle.recur(op, q, k, v, gamma=g, eps=EPS)
     b = brute.forward(op, q, k, v, gamma=g, eps=EPS)
     assert oracle.max_row_rel_err(r, b) < 1e-11
@@ -494,3 +505,147 @@ def test_normalised_constant_v_and_homogeneity(op):
     o1 = oracle.recur(op, one_head(q), one_head(k), one_head(v), eps=0.0)[0, 0]
     o2 = oracle.recur(op, one_head(3.0 * q), one_head(k), one_head(v), eps=0.0)[0, 0]
     np.testing.assert_allclose(o1, o2, rtol=1e-10)     # degree 0 in q (ratio of equal degrees)
+
+
+# ---------------------------------------------------------------------------
+# decayed AHLA and third order (Contribuciones 2 with Metodología 2 and 3; reading: every state
+# of the recurrence scaled by gamma before each token's update)
+# ---------------------------------------------------------------------------
+
+def literal_ahla_decay(q, k, v, g):
+    """o_t = sum_{j<=t} sum_{i<=j} g^(t-i) (q_t.k_j)(q_j.k_i) v_i, as plain loops."""
+    T, dv = len(q), len(v[0])
+    out = []
+    for t in range(T):
+        o = [0.0] * dv
+        for j in range(t + 1):
+            for i in range(j + 1):
+                w = g ** (t - i) * _dot(q[t], k[j]) * _dot(q[j], k[i])
+                for c in range(dv):
+                    o[c] += w * v[i][c]
+        out.append(o)
+    return np.asarray(out)
+
+
+def literal_hla3_decay(q, k, v, g):
+    """o_t = sum_{s<=t} sum_{a<=s} sum_{b<=s} g^(t-a) g^(s-b) (q_t.k_a)(q_s.k_a)(q_s.k_b) v_b."""
+    T, dv = len(q), len(v[0])
+    out = []
+    for t in range(T):
+        o = [0.0] * dv
+        for s in range(t + 1):
+            for a in range(s + 1):
+                for b in range(s + 1):
+                    w = g ** (t - a) * g ** (s - b) * _dot(q[t], k[a]) * _dot(q[s], k[a]) * _dot(q[s], k[b])
+                    for c in range(dv):
+                        o[c] += w * v[b][c]
+        out.append(o)
+    return np.asarray(out)
+
+
+@pytest.mark.parametrize("g", [0.5, 0.9, 1.0])
+def test_decayed_ahla_hla3_literal_sums(g):
+    rng = np.random.default_rng(int(g * 100))
+    T, d, dv = 9, 3, 2
+    q, k, v = rng.standard_normal((T, d)), rng.standard_normal((T, d)), rng.standard_normal((T, dv))
+    gam = np.array([g])
+    np.testing.assert_allclose(oracle.recur("ahlad", one_head(q), one_head(k), one_head(v), gamma=gam)[0, 0],
+                               literal_ahla_decay(q.tolist(), k.tolist(), v.tolist(), g), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.recur("hla3d", one_head(q), one_head(k), one_head(v), gamma=gam)[0, 0],
+                               literal_hla3_decay(q.tolist(), k.tolist(), v.tolist(), g), rtol=1e-12, atol=1e-12)
+
+
+def test_decayed_ahla_hla3_all_ones_closed_forms():
+    """d = 1, all ones: AHLA o_t = sum_{m=0}^{t} (m+1) g^m (the pairs i <= j <= t with t - i = m
+    number m + 1); third order o_t = sum_{s<=t} g^(t-s) ((1 - g^(s+1)) / (1 - g))^2."""
+    T, g = 40, 0.8
+    one = np.ones((1, 1, T, 1))
+    a = oracle.recur("ahlad", one, one, one, gamma=np.array([g]))[0, 0, :, 0]
+    h = oracle.recur("hla3d", one, one, one, gamma=np.array([g]))[0, 0, :, 0]
+    for t in range(T):
+        assert abs(a[t] - sum((m + 1) * g ** m for m in range(t + 1))) < 1e-12 * max(1.0, a[t])
+        ref = sum(g ** (t - s) * ((1 - g ** (s + 1)) / (1 - g)) ** 2 for s in range(t + 1))
+        assert abs(h[t] - ref) < 1e-12 * max(1.0, ref)
+
+
+def test_decayed_ahla_hla3_gamma_one_is_undecayed_bitwise():
+    q, k, v = _rand()
+    qp, kp = np.abs(q), np.abs(k)
+    ones = np.array([1.0, 1.0])
+    for op, base in (("ahlad", "ahla"), ("hla3d", "hla3")):
+        assert np.array_equal(oracle.recur(op, q, k, v, gamma=ones), oracle.recur(base, q, k, v))
+    for op in ("ahlan", "hla3n"):
+        assert np.array_equal(oracle.recur(op, qp, kp, v, gamma=ones, eps=EPS), oracle.recur(op, qp, kp, v, eps=EPS))
+
+
+def test_decayed_ahla_hla3_homogeneity_and_causality():
+    q, k, v = _rand()
+    g = np.array([0.9, 0.7])
+    a, b, c = 1.5, 0.5, -2.0
+    for op, p in (("ahlad", 2), ("hla3d", 3)):
+        base = oracle.recur(op, q, k, v, gamma=g)
+        np.testing.assert_allclose(oracle.recur(op, a * q, b * k, c * v, gamma=g), a ** p * b ** p * c * base,
+                                   rtol=1e-11, atol=1e-12)
+        s = 11
+        q2, k2, v2 = q.copy(), k.copy(), v.copy()
+        q2[..., s:, :] += 2.0
+        v2[..., s:, :] *= -3.0
+        pert = oracle.recur(op, q2, k2, v2, gamma=g)
+        assert np.array_equal(base[..., :s, :], pert[..., :s, :])
+        assert not np.allclose(base[..., s:, :], pert[..., s:, :])
+
+
+@pytest.mark.parametrize("lengths", SEGMENTATIONS)
+@pytest.mark.parametrize("scan", [seg.blelloch_exclusive, seg.fold_exclusive])
+def test_decayed_ahla_hla3_scan_matches_recurrence(lengths, scan):
+    q, k, v = _rand(T=40, d=3, dv=2, seed=5)
+    g = np.array([0.93, 0.8])
+    for op, fwd in (("ahlad", seg.ahla_scan_forward), ("hla3d", seg.hla3_scan_forward)):
+        ref = oracle.recur(op, q, k, v, gamma=g)[0, 1]
+        assert rel(fwd(q[0, 1], k[0, 1], v[0, 1], lengths, scan=scan, gamma=0.8), ref) < 1e-10
+
+
+@pytest.mark.parametrize("kind", ["ahla", "hla3"])
+def test_decayed_combine_is_concatenation_and_associative(kind):
+    q, k, v = (x[0, 0] for x in _rand(T=30, d=3, dv=2, seed=9))
+    b = [0, 9, 17, 30]
+    g = 0.85
+    if kind == "ahla":
+        summ = lambda s, e: seg.ahla_summary(q[s:e], k[s:e], v[s:e], g)   # noqa: E731
+        comb, ident = seg.ahla_combine, seg.ahla_identity(3, 2)
+    else:
+        summ = lambda s, e: seg.hla3_summary(q[s:e], k[s:e], v[s:e], g)   # noqa: E731
+        comb, ident = seg.hla3_combine, seg.hla3_identity(3, 2)
+    A, B, C = summ(b[0], b[1]), summ(b[1], b[2]), summ(b[2], b[3])
+    _close_summary(comb(A, B), summ(b[0], b[2]))
+    _close_summary(comb(comb(A, B), C), comb(A, comb(B, C)))
+    _close_summary(comb(ident, A), A)
+    _close_summary(comb(A, ident), A)
+
+
+def test_decayed_ahla_hla3_planted_mistakes_are_caught():
+    """Mistakes a decayed implementation could make, planted in copies of the oracle's maps: the
+    pins above must tell each apart from the real thing."""
+    q, k, v = (x[0, 0] for x in _rand(T=24, d=3, dv=2, seed=4))
+    g = 0.8
+    # (1) AHLA with only P decayed (E accumulated undecayed) disagrees with the literal sum
+    P = np.zeros((3, 2))
+    E = np.zeros((3, 2))
+    wrong = []
+    for t in range(24):
+        P = g * P + np.outer(k[t], v[t])
+        E = E + np.outer(k[t], q[t] @ P)
+        wrong.append(q[t] @ E)
+    lit = literal_ahla_decay(q.tolist(), k.tolist(), v.tolist(), g)
+    assert rel(np.asarray(wrong), lit) > 1e-3
+    # (2) the third-order combine with an undecayed Q2 map breaks concatenation
+    summ = lambda s, e: seg.hla3_summary(q[s:e], k[s:e], v[s:e], g)   # noqa: E731
+    A, B = summ(0, 10), summ(10, 24)
+    B_plain = dict(B)
+    B_plain["Q2"] = q[10:24].T @ q[10:24]
+    bad = seg.hla3_combine(A, B_plain)
+    assert rel(bad["F"], summ(0, 24)["F"]) > 1e-3
+    # (3) the AHLA combine without rho on the cross term breaks concatenation
+    sA, sB = seg.ahla_summary(q[:10], k[:10], v[:10], g), seg.ahla_summary(q[10:], k[10:], v[10:], g)
+    E_bad = sB["rho"] * sA["E"] + sB["E"] + sB["D"] @ sA["P"]
+    assert rel(E_bad, seg.ahla_summary(q, k, v, g)["E"]) > 1e-3
