@@ -173,7 +173,7 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     stacked products, no state walk)."""
     D = w.d
     c = 128 if path == "tc" else 64
-    if w.op in ("ahla", "ahlan"):
+    if w.op in ("ahla", "ahlan", "ahlad"):
         # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
         flops = 6 * c * D + 4 * D * D
     elif w.op == "hla2u":
@@ -187,6 +187,8 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     else:
         # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
         flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
+        if w.op in ("hla3", "hla3n", "hla3d"):
+            flops += 2 * D * (D + c)      # the third order also forms Y = [Q|A][P0;V] before O = [Q|W][F0;Y]
     return {"bound": "tensor" if path == "tc" else "alu", "flops_per_token": flops, "chunk": c}
 
 

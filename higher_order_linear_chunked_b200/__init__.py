@@ -220,14 +220,14 @@ def hla2_normalized(q, k, v, eps: float = 1e-6, gamma=None, out=None, workspace=
     return _call(OP_HLA2_NORM, q, k, v, gamma=gamma, eps=eps, out=out, workspace=workspace, stream=stream)
 
 
-def ahla(q, k, v, out=None, workspace=None, stream=None):
-    """AHLA masked forward."""
-    return _call(OP_AHLA, q, k, v, out=out, workspace=workspace, stream=stream)
+def ahla(q, k, v, gamma=None, out=None, workspace=None, stream=None):
+    """AHLA masked forward (optional per-head decay gamma [H])."""
+    return _call(OP_AHLA, q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
 
 
-def hla3(q, k, v, out=None, workspace=None, stream=None):
-    """Third-order masked HLA forward."""
-    return _call(OP_HLA3, q, k, v, out=out, workspace=workspace, stream=stream)
+def hla3(q, k, v, gamma=None, out=None, workspace=None, stream=None):
+    """Third-order masked HLA forward (optional per-head decay gamma [H])."""
+    return _call(OP_HLA3, q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
 
 
 def hla2_unmasked(q, k, v, out=None, workspace=None, stream=None):
@@ -265,7 +265,8 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None):
 
 def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, workspace=None, stream=None):
     """Dispatch by name: "hla2", "hla2n", "hla2d" (needs gamma), "ahla", "hla3", "hla2u",
-    "ahlan", "hla3n" (ratio-normalised AHLA / third order)."""
+    "ahlan", "hla3n" (ratio-normalised AHLA / third order), "ahlad", "hla3d" (AHLA / third order
+    with decay: need gamma).  gamma, when given, selects the decayed form of any op but "hla2u"."""
     if op_name == "hla2":
         return hla2(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "hla2n":
@@ -274,21 +275,24 @@ def forward(op_name: str, q, k, v, gamma=None, eps: float = 1e-6, out=None, work
         if gamma is None:
             raise ValueError("hla2d needs gamma")
         return hla2(q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
-    if op_name == "ahla":
-        return ahla(q, k, v, out=out, workspace=workspace, stream=stream)
-    if op_name == "hla3":
-        return hla3(q, k, v, out=out, workspace=workspace, stream=stream)
+    if op_name in ("ahlad", "hla3d") and gamma is None:
+        raise ValueError(f"{op_name} needs gamma")
+    if op_name in ("ahla", "ahlad"):
+        return ahla(q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
+    if op_name in ("hla3", "hla3d"):
+        return hla3(q, k, v, gamma=gamma, out=out, workspace=workspace, stream=stream)
     if op_name == "hla2u":
         return hla2_unmasked(q, k, v, out=out, workspace=workspace, stream=stream)
     if op_name == "ahlan":
-        return _call(OP_AHLA_NORM, q, k, v, eps=eps, out=out, workspace=workspace, stream=stream)
+        return _call(OP_AHLA_NORM, q, k, v, gamma=gamma, eps=eps, out=out, workspace=workspace, stream=stream)
     if op_name == "hla3n":
-        return _call(OP_HLA3_NORM, q, k, v, eps=eps, out=out, workspace=workspace, stream=stream)
+        return _call(OP_HLA3_NORM, q, k, v, gamma=gamma, eps=eps, out=out, workspace=workspace, stream=stream)
     raise ValueError(op_name)
 
 
 OP_CODES = {"hla2": OP_HLA2, "hla2n": OP_HLA2_NORM, "hla2d": OP_HLA2, "ahla": OP_AHLA, "hla3": OP_HLA3,
-            "hla2u": OP_HLA2_UNMASKED, "ahlan": OP_AHLA_NORM, "hla3n": OP_HLA3_NORM}
+            "hla2u": OP_HLA2_UNMASKED, "ahlan": OP_AHLA_NORM, "hla3n": OP_HLA3_NORM, "ahlad": OP_AHLA,
+            "hla3d": OP_HLA3}
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -14,6 +14,8 @@ enum Op : int {
     OP_AHLA = 2,
     OP_HLA3 = 3,
     OP_HLA2U = 4,  // second order without the inner mask (o_t = q_t^T S_t C_t)
+    OP_AHLAD = 5,  // AHLA with per-head decay
+    OP_HLA3D = 6,  // third order with per-head decay
 };
 
 // Device status word values (first int of every workspace).

@@ -48,8 +48,9 @@ struct Dim {
 template <int OP, int D>
 struct Sum {
     static constexpr int DD = D * D;
-    static constexpr int NMAT = OP == OP_HLA3 ? 6 : OP == OP_HLA2D ? 4 : OP == OP_HLA2U ? 2 : 3;
-    static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D || OP == OP_AHLA) ? 2 : OP == OP_HLA3 ? 3 : 0;
+    static constexpr int NMAT = (OP == OP_HLA3 || OP == OP_HLA3D) ? 6 : OP == OP_HLA2D ? 4 : OP == OP_HLA2U ? 2 : 3;
+    static constexpr int NVEC = (OP == OP_HLA2 || OP == OP_HLA2D || OP == OP_AHLA || OP == OP_AHLAD) ? 2
+                                : (OP == OP_HLA3 || OP == OP_HLA3D) ? 3 : 0;
     static constexpr int VEC0 = NMAT * DD;
     static constexpr int SCAL = VEC0 + NVEC * D;
     static constexpr int SIZE = (SCAL + 4 + 31) / 32 * 32;
@@ -62,6 +63,8 @@ struct Sum {
 //   OP_AHLA : P=0 E=1 Dm=2 ; mK=0 n=1            (the ratio-normaliser's P and E: V -> ones)
 //   OP_HLA3 : S=0 Q2=1 P=2 F=3 X=4 Z=5 ; mK=0 X1=1 F1=2   (likewise for P, X, F)
 //   OP_HLA2U: S=0 C=1
+//   OP_AHLAD: as OP_AHLA (Dm undecayed) ; scalar rho
+//   OP_HLA3D: as OP_HLA3 (Q2 weighted by gamma^position, X and Z undecayed sums) ; scalar rho
 
 size_t summary_floats(int op, int d) {
     switch (op) {
@@ -70,9 +73,14 @@ size_t summary_floats(int op, int d) {
     case OP_AHLA: return d == 32 ? Sum<OP_AHLA, 32>::SIZE : Sum<OP_AHLA, 64>::SIZE;
     case OP_HLA3: return d == 32 ? Sum<OP_HLA3, 32>::SIZE : Sum<OP_HLA3, 64>::SIZE;
     case OP_HLA2U: return d == 32 ? Sum<OP_HLA2U, 32>::SIZE : Sum<OP_HLA2U, 64>::SIZE;
+    case OP_AHLAD: return d == 32 ? Sum<OP_AHLAD, 32>::SIZE : Sum<OP_AHLAD, 64>::SIZE;
+    case OP_HLA3D: return d == 32 ? Sum<OP_HLA3D, 32>::SIZE : Sum<OP_HLA3D, 64>::SIZE;
     }
     return 0;
 }
+
+// the ops whose summaries carry rho = gamma^length (identity: 1)
+__host__ __device__ constexpr bool decayed_op(int op) { return op == OP_HLA2D || op == OP_AHLAD || op == OP_HLA3D; }
 
 // ---------------------------------------------------------------------------
 // Block-cooperative small matrix products in shared/global memory.
@@ -192,7 +200,7 @@ __device__ __forceinline__ float gpow(float g, int n) {  // gamma^n, n >= 0
 template <int OP, int D>
 __device__ void write_identity(float* out) {
     using S = Sum<OP, D>;
-    for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) out[e] = (OP == OP_HLA2D && e == S::SCAL) ? 1.f : 0.f;
+    for (int e = threadIdx.x; e < S::SIZE; e += blockDim.x) out[e] = (decayed_op(OP) && e == S::SCAL) ? 1.f : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -220,6 +228,7 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     float* Y2 = Ys + C * LD;      // C x LD
     float* us = Y2 + C * LD;      // C
     float* lam = us + C;          // C  (decay weights)
+    float* gpw = lam + C;         // C + 1: gamma^j
     const size_t head = (size_t)bh * T * D;
     const int t0 = chunk * C;
     load_rows<D>(Qs, q + head, t0, T);
@@ -227,17 +236,20 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     load_rows<D>(Vs, v + head, t0, T);
     float g = 1.f;
     const int len = min(C, T - t0);      // tokens in this chunk (the last one may be short)
-    if (OP == OP_HLA2D) {
+    if (decayed_op(OP)) {
         // gamma^(len - 1 - tau): decayed to the chunk's own last token, so that the summary of
         // a short last chunk is the state after the sequence's last token (the streaming state)
         g = gamma[bh % H];
         for (int j = threadIdx.x; j < C; j += blockDim.x) lam[j] = j < len ? gpow(g, len - 1 - j) : 0.f;
+        for (int j = threadIdx.x; j <= C; j += blockDim.x) gpw[j] = gpow(g, j);
     }
     __syncthreads();
-    // A* = Q K^T (masked to A = L (.) A* except for the decayed op, which needs both parts)
+    // A* = Q K^T (masked to A = L (.) A* except for the decayed second order, which needs both
+    // parts; the decayed AHLA / third order keep At = gamma^(t-j) A_tj)
     if (OP != OP_HLA2U)
         mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
-            As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
+            if (OP == OP_AHLAD || OP == OP_HLA3D) As[r * LDC + c] = c <= r ? gpw[r - c] * x : 0.f;
+            else As[r * LDC + c] = (OP == OP_HLA2D || c <= r) ? x : 0.f;
         });
     __syncthreads();
 
@@ -293,6 +305,71 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     } else if (OP == OP_HLA2U) {
         mm<D, D, C>(TileT{Ks, LD}, Tile{Ks, LD}, Zero{}, store_mat(0));        // S = K^T K
         mm<D, D, C>(TileT{Qs, LD}, Tile{Vs, LD}, Zero{}, store_mat(1));        // C = Q^T V
+    } else if (OP == OP_AHLAD) {
+        // As = At.  P = K^T Lam V, Dm = K^T Q, Y = At V, E = K^T Lam Y; mK = K^T Lam 1, n = K^T Lam (At 1)
+        auto kl = [&](int r, int c) { return Ks[c * LD + r] * lam[c]; };               // (K^T Lam)[r][c]
+        mm<D, D, C>(kl, Tile{Vs, LD}, Zero{}, store_mat(0));
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Qs, LD}, Zero{}, store_mat(2));
+        mm<C, D, C>(Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});
+        __syncthreads();
+        mm<D, D, C>(kl, Tile{Ys, LD}, Zero{}, store_mat(1));
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s += As[i * LDC + j];
+            us[i] = s;
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sn = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Ks[i * LD + a] * lam[i];
+                sn += Ks[i * LD + a] * lam[i] * us[i];
+            }
+            out[S::vec(0) + a] = sm_;
+            out[S::vec(1) + a] = sn;
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = gpow(g, len);
+    } else if (OP == OP_HLA3D) {
+        // As = At.  S = K^T Lam K, Q2 = Q^T Gam Q (Gam = gamma^(tau+1)), P = K^T Lam V, Y = At V,
+        // X = Q^T Y, Z = K^T (At^T Q), F = K^T (At^T Lam Y); vectors with V -> 1
+        auto kl = [&](int r, int c) { return Ks[c * LD + r] * lam[c]; };
+        mm<D, D, C>(kl, Tile{Ks, LD}, Zero{}, store_mat(0));
+        mm<D, D, C>([&](int r, int c) { return Qs[c * LD + r] * gpw[c + 1]; }, Tile{Qs, LD}, Zero{}, store_mat(1));
+        mm<D, D, C>(kl, Tile{Vs, LD}, Zero{}, store_mat(2));
+        mm<C, D, C>(Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});
+        mm<C, D, C>(TileT{As, LDC}, Tile{Qs, LD}, Zero{}, Put{Y2, LD});
+        __syncthreads();
+        mm<D, D, C>(TileT{Qs, LD}, Tile{Ys, LD}, Zero{}, store_mat(4));
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Y2, LD}, Zero{}, store_mat(5));
+        __syncthreads();
+        mm<C, D, C>(TileT{As, LDC}, [&](int r, int c) { return lam[r] * Ys[r * LD + c]; }, Zero{}, Put{Y2, LD});
+        __syncthreads();
+        mm<D, D, C>(TileT{Ks, LD}, Tile{Y2, LD}, Zero{}, store_mat(3));
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {              // u = At 1
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s += As[i * LDC + j];
+            us[i] = s;
+        }
+        __syncthreads();
+        float* ws_ = Y2;                                                  // w = At^T Lam u (C floats)
+        for (int i = threadIdx.x; i < C; i += blockDim.x) {
+            float s = 0.f;
+            for (int r = i; r < C; ++r) s += As[r * LDC + i] * lam[r] * us[r];
+            ws_[i] = s;
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sm_ = 0.f, sx = 0.f, sf = 0.f;
+            for (int i = 0; i < C; ++i) {
+                sm_ += Ks[i * LD + a] * lam[i];
+                sx += Qs[i * LD + a] * us[i];
+                sf += Ks[i * LD + a] * ws_[i];
+            }
+            out[S::vec(0) + a] = sm_;                                    // mK = K^T Lam 1
+            out[S::vec(1) + a] = sx;                                     // X1 = Q^T (At 1)
+            out[S::vec(2) + a] = sf;                                     // F1 = K^T (At^T Lam At 1)
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = gpow(g, len);
     } else if (OP == OP_AHLA) {
         mm<D, D, C>(TileT{Ks, LD}, Tile{Vs, LD}, Zero{}, store_mat(0));        // P = K^T V
         mm<D, D, C>(TileT{Ks, LD}, Tile{Qs, LD}, Zero{}, store_mat(2));        // Dm = K^T Q
@@ -403,6 +480,55 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
     } else if (OP == OP_HLA2U) {
         add2(0);
         add2(1);
+    } else if (OP == OP_AHLAD) {
+        // P = rb P_A + P_B, E = rb E_A + E_B + rb Dm_B P_A, Dm adds; vectors alike (n gets rb Dm_B mK_A)
+        const float rb = B[S::SCAL];
+        for (int e = threadIdx.x; e < DD; e += blockDim.x) {
+            out[S::mat(0) + e] = rb * A[S::mat(0) + e] + B[S::mat(0) + e];
+            out[S::mat(2) + e] = A[S::mat(2) + e] + B[S::mat(2) + e];
+        }
+        mm<D, D, D>([&](int r, int c) { return rb * B[S::mat(2) + r * D + c]; }, G(A, 0),
+                    [&](int r, int c) { return rb * A[S::mat(1) + r * D + c] + B[S::mat(1) + r * D + c]; }, dst(1));
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float s = 0.f;
+            for (int b = 0; b < D; ++b) s += B[S::mat(2) + a * D + b] * A[S::vec(0) + b];
+            out[S::vec(0) + a] = rb * A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = rb * A[S::vec(1) + a] + B[S::vec(1) + a] + rb * s;
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = A[S::SCAL] * rb;
+    } else if (OP == OP_HLA3D) {
+        // S = rb S_A + S_B, P = rb P_A + P_B, Q2 = Q2_A + ra Q2_B, Z = Z_A + Z_B + S_A Q2_B,
+        // X = X_A + X_B + Q2_B P_A, F = rb F_A + F_B + rb (S_A Q2_B P_A + S_A X_B + Z_B P_A)
+        const float ra = A[S::SCAL], rb = B[S::SCAL];
+        mm<D, D, D>(G(A, 0), G(B, 1), Zero{}, [&](int r, int c, float x) { tmp[r * D + c] = x; });   // S_A Q2_B
+        __syncthreads();
+        for (int e = threadIdx.x; e < DD; e += blockDim.x) {
+            out[S::mat(0) + e] = rb * A[S::mat(0) + e] + B[S::mat(0) + e];
+            out[S::mat(1) + e] = A[S::mat(1) + e] + ra * B[S::mat(1) + e];
+            out[S::mat(2) + e] = rb * A[S::mat(2) + e] + B[S::mat(2) + e];
+            out[S::mat(5) + e] = A[S::mat(5) + e] + B[S::mat(5) + e] + tmp[e];
+        }
+        mm<D, D, D>(G(B, 1), G(A, 2),
+                    [&](int r, int c) { return A[S::mat(4) + r * D + c] + B[S::mat(4) + r * D + c]; }, dst(4));
+        auto rbt = [&](const float* p, int slot) {
+            return [=](int r, int c) { return rb * p[S::mat(slot) + r * D + c]; };
+        };
+        mm3<D, D, D, D, D>([&](int r, int c) { return rb * tmp[r * D + c]; }, G(A, 2), rbt(A, 0), G(B, 4), rbt(B, 5),
+                           G(A, 2),
+                           [&](int r, int c) { return rb * A[S::mat(3) + r * D + c] + B[S::mat(3) + r * D + c]; },
+                           dst(3));
+        for (int a = threadIdx.x; a < D; a += blockDim.x) {
+            float sx = 0.f, sf = 0.f;
+            for (int b = 0; b < D; ++b) {
+                const float mk = A[S::vec(0) + b];
+                sx += B[S::mat(1) + a * D + b] * mk;
+                sf += tmp[a * D + b] * mk + A[S::mat(0) + a * D + b] * B[S::vec(1) + b] + B[S::mat(5) + a * D + b] * mk;
+            }
+            out[S::vec(0) + a] = rb * A[S::vec(0) + a] + B[S::vec(0) + a];
+            out[S::vec(1) + a] = A[S::vec(1) + a] + B[S::vec(1) + a] + sx;
+            out[S::vec(2) + a] = rb * A[S::vec(2) + a] + B[S::vec(2) + a] + rb * sf;
+        }
+        if (threadIdx.x == 0) out[S::SCAL] = ra * rb;
     } else if (OP == OP_AHLA) {
         add2(0);
         add2(2);
@@ -493,7 +619,7 @@ __global__ void k_identity(float* sums, int NCp) {
 template <int OP, int D>
 constexpr size_t fold_smem() { return sizeof(float) * (3 * (size_t)Sum<OP, D>::SIZE + (size_t)D * D); }
 template <int OP, int D>
-constexpr bool fold_fits() { return OP != OP_HLA3 && fold_smem<OP, D>() <= 227 * 1024; }
+constexpr bool fold_fits() { return OP != OP_HLA3 && OP != OP_HLA3D && fold_smem<OP, D>() <= 227 * 1024; }
 
 template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int NC, int NCp) {
@@ -585,7 +711,7 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     } else if (OP == OP_HLA2U) {
         load_mat<D>(M0, pre + S::mat(0));   // S0
         load_mat<D>(M1, pre + S::mat(1));   // C0
-    } else if (OP == OP_AHLA) {
+    } else if (OP == OP_AHLA || OP == OP_AHLAD) {
         load_mat<D>(M0, pre + S::mat(0));   // P0
         load_mat<D>(M1, pre + S::mat(1));   // E0
         for (int a = threadIdx.x; a < D; a += blockDim.x) {
@@ -601,11 +727,15 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
             vec[D + a] = pre[S::vec(2) + a];  // F1_0
         }
     }
+    if (OP == OP_AHLAD || OP == OP_HLA3D) {
+        g = gamma[bh % H];
+        for (int j = threadIdx.x; j <= C; j += blockDim.x) gp[j] = gpow(g, j);
+    }
     __syncthreads();
     mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, [&](int r, int c, float x) {
         As[r * LDC + c] = (OP == OP_HLA2D || OP == OP_HLA2U || c <= r) ? x : 0.f;
     });
-    if (OP == OP_HLA2 || OP == OP_HLA3 || OP == OP_HLA2U)
+    if (OP == OP_HLA2 || OP == OP_HLA3 || OP == OP_HLA3D || OP == OP_HLA2U)
         mm<C, D, D>(Tile{Qs, LD}, Tile{M0, LD}, Zero{}, Put{Ps, LD});                      // P = Q S0
     if (OP == OP_HLA2U)
         mm<D, D, D>(Tile{M0, LD}, Tile{M1, LD}, Zero{}, Put{M2, LD});                      // S0 C0
@@ -694,6 +824,44 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
             __syncthreads();
         }
         mm2<C, D, D, C>(Tile{Qs, LD}, Tile{M1, LD}, Tile{As, LDC}, Tile{Ys, LD}, Zero{}, emit);          // O = Q E0 + A Y
+    } else if (OP == OP_AHLAD || OP == OP_HLA3D) {
+        // Gam = diag(gamma^(tau+1)) (the carried state decays by one step per token of the chunk
+        // up to and including tau), At_tj = gamma^(t-j) A_tj:
+        //   AHLA:  Y = Gam Q P0 + At V,  O = Gam Q E0 + At Y
+        //   third: Y = Gam Q P0 + At V,  W = L (.) (Gam P Q^T + At A^T),  O = Gam Q F0 + W Y
+        auto At = [&](int r, int c) { return c <= r ? gp[r - c] * As[r * LDC + c] : 0.f; };
+        auto GQ = [&](int r, int c) { return gp[r + 1] * Qs[r * LD + c]; };
+        const float* Pm = OP == OP_AHLAD ? M0 : M1;                                            // P0
+        const float* Em = OP == OP_AHLAD ? M1 : M2;                                            // E0 / F0
+        mm2<C, D, D, C>(GQ, Tile{Pm, LD}, At, Tile{Vs, LD}, Zero{}, Put{Ys, LD});
+        if (OP == OP_HLA3D)
+            mm2<C, C, D, C>([&](int r, int c) { return gp[r + 1] * Ps[r * LD + c]; }, TileT{Qs, LD}, At,
+                            TileT{As, LDC}, Zero{}, [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
+        __syncthreads();
+        if (NORM) {     // y1 = Gam Q mK0 + At 1 (in Ps column 0), den = Gam Q n0 + At y1 (F1_0, W y1)
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[a];
+                s *= gp[r + 1];
+                for (int j = 0; j <= r; ++j) s += gp[r - j] * As[r * LDC + j];
+                den[r] = s;                                  // y1, for now
+            }
+            __syncthreads();
+            float* y1 = Ps;                                  // P is not read again
+            for (int r = threadIdx.x; r < C; r += blockDim.x) y1[r * LD] = den[r];
+            __syncthreads();
+            for (int r = threadIdx.x; r < C; r += blockDim.x) {
+                float s = 0.f;
+                for (int a = 0; a < D; ++a) s += Qs[r * LD + a] * vec[D + a];
+                s *= gp[r + 1];
+                for (int j = 0; j <= r; ++j)
+                    s += (OP == OP_AHLAD ? gp[r - j] * As[r * LDC + j] : Ws[r * LDC + j]) * y1[j * LD];
+                den[r] = s;
+            }
+            __syncthreads();
+        }
+        if (OP == OP_AHLAD) mm2<C, D, D, C>(GQ, Tile{Em, LD}, At, Tile{Ys, LD}, Zero{}, emit);
+        else mm2<C, D, D, C>(GQ, Tile{Em, LD}, Tile{Ws, LDC}, Tile{Ys, LD}, Zero{}, emit);
     } else {  // OP_HLA3
         mm2<C, C, D, C>(Tile{Ps, LD}, TileT{Qs, LD}, Tile{As, LDC}, TileT{As, LDC}, Zero{},
                         [&](int r, int c, float x) { Ws[r * LDC + c] = c <= r ? x : 0.f; });
@@ -731,7 +899,7 @@ static int next_pow2(int n) {
 template <int D>
 static size_t summary_smem() {
     constexpr int LD = Dim<D>::LD;
-    return sizeof(float) * (size_t)(3 * C * LD + C * LDC + 2 * C * LD + 2 * C);
+    return sizeof(float) * (size_t)(3 * C * LD + C * LDC + 2 * C * LD + 3 * C + 1);
 }
 template <int D>
 static size_t output_smem() {
@@ -780,6 +948,8 @@ cudaError_t scan(int op, int d, float* sums, int NCp, int BH, cudaStream_t st) {
     case OP_AHLA: return d == 32 ? scan_levels<OP_AHLA, 32>(sums, NCp, BH, st) : scan_levels<OP_AHLA, 64>(sums, NCp, BH, st);
     case OP_HLA3: return d == 32 ? scan_levels<OP_HLA3, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA3, 64>(sums, NCp, BH, st);
     case OP_HLA2U: return d == 32 ? scan_levels<OP_HLA2U, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA2U, 64>(sums, NCp, BH, st);
+    case OP_AHLAD: return d == 32 ? scan_levels<OP_AHLAD, 32>(sums, NCp, BH, st) : scan_levels<OP_AHLAD, 64>(sums, NCp, BH, st);
+    case OP_HLA3D: return d == 32 ? scan_levels<OP_HLA3D, 32>(sums, NCp, BH, st) : scan_levels<OP_HLA3D, 64>(sums, NCp, BH, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -840,6 +1010,12 @@ static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, 
         return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
                     : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_AHLAD:
+        return norm ? run<OP_AHLAD, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_AHLAD, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    case OP_HLA3D:
+        return norm ? run<OP_HLA3D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
+                    : run<OP_HLA3D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
     }
     return cudaErrorInvalidValue;
 }
@@ -862,6 +1038,8 @@ static bool uses_fold(int op, int d) {
     case OP_AHLA: return d == 32 ? fold_fits<OP_AHLA, 32>() : fold_fits<OP_AHLA, 64>();
     case OP_HLA3: return d == 32 ? fold_fits<OP_HLA3, 32>() : fold_fits<OP_HLA3, 64>();
     case OP_HLA2U: return d == 32 ? fold_fits<OP_HLA2U, 32>() : fold_fits<OP_HLA2U, 64>();
+    case OP_AHLAD: return d == 32 ? fold_fits<OP_AHLAD, 32>() : fold_fits<OP_AHLAD, 64>();
+    case OP_HLA3D: return d == 32 ? fold_fits<OP_HLA3D, 32>() : fold_fits<OP_HLA3D, 64>();
     }
     return false;
 }
@@ -916,6 +1094,8 @@ static cudaError_t state_op(int op, const void* q, const void* k, const void* v,
     case OP_AHLA: return state_run<OP_AHLA, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_HLA3: return state_run<OP_HLA3, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_HLA2U: return state_run<OP_HLA2U, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_AHLAD:
+    case OP_HLA3D: return cudaErrorNotSupported;   // no streaming form for the decayed AHLA / third order
     }
     return cudaErrorInvalidValue;
 }
@@ -1183,6 +1363,8 @@ static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const v
         return norm ? step_launch<OP_HLA3, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
                     : step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA2U: return step_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_AHLAD:
+    case OP_HLA3D: return cudaErrorNotSupported;   // no streaming form for the decayed AHLA / third order
     }
     return cudaErrorInvalidValue;
 }

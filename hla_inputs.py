@@ -83,6 +83,14 @@ WORKLOADS = {
         "ahlan_bf16_4x16x8192x64", "ahlan", "bf16", 4, 16, 8192, 64, 64, "softplus", "unit"),
     "hla3n_f32_2x8x4096x32": Workload(
         "hla3n_f32_2x8x4096x32", "hla3n", "f32", 2, 8, 4096, 32, 32, "softplus", "unit"),
+    # the decayed AHLA and third order at the shapes of their plain workloads, gamma as for the
+    # decayed second order
+    "ahlad_bf16_4x16x8192x64": Workload(
+        "ahlad_bf16_4x16x8192x64", "ahlad", "bf16", 4, 16, 8192, 64, 64, "scaled", "scaled",
+        gamma_range=(0.95, 0.999)),
+    "hla3d_f32_2x8x4096x32": Workload(
+        "hla3d_f32_2x8x4096x32", "hla3d", "f32", 2, 8, 4096, 32, 32, "scaled", "scaled",
+        gamma_range=(0.95, 0.999)),
 }
 
 

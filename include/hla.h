@@ -102,7 +102,7 @@ const char* hla_status_str(hla_status_t status);
 
 /*
  * Bytes of device workspace one call needs, or 0 when the request is invalid
- * or unsupported.  decayed: nonzero when gamma will be passed (hla2 only).
+ * or unsupported.  decayed: nonzero when gamma will be passed (every op but the unmasked one).
  */
 size_t hla_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed,
                            int B, int H, int T, int d, int dv);
@@ -121,13 +121,18 @@ hla_status_t hla2_forward_normalized(const void* q, const void* k, const void* v
                                      const float* gamma, float eps,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
-/* AHLA masked forward (Metodología 2).  gamma must be NULL (no decayed AHLA). */
+/* AHLA masked forward (Metodología 2).  gamma: device fp32 [H] or NULL.  With gamma
+ * (Contribuciones 2's decayed operators; the page gives no formula, the reading is the second
+ * order's: P and E scaled by gamma_h before each token's update), the output is
+ * o_t = sum_{j<=t} sum_{i<=j} gamma^(t-i) (q_t.k_j)(q_j.k_i) v_i, on CUDA-core kernels. */
 hla_status_t ahla_forward(const void* q, const void* k, const void* v, float* o,
                           int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                           const float* gamma, void* workspace, size_t workspace_bytes,
                           void* stream);
 
-/* Third-order masked forward (Metodología 3).  gamma must be NULL. */
+/* Third-order masked forward (Metodología 3).  gamma: device fp32 [H] or NULL.  With gamma
+ * (same reading: S, P and F scaled by gamma_h before each token's update) the output is
+ * O = (L (.) (At A^T)) (At V) with At_tj = gamma^(t-j) A_tj, on CUDA-core kernels. */
 hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
                           int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                           const float* gamma, void* workspace, size_t workspace_bytes,
@@ -135,8 +140,9 @@ hla_status_t hla3_forward(const void* q, const void* k, const void* v, float* o,
 
 /* Ratio-normalised AHLA and third-order forwards: the output divided by the same masked
  * operator applied to a ones value column, plus eps (for AHLA, q_t^T n_t with the named
- * summaries m^K = sum k and n_t = sum_j k_j (q_j^T m^K_j)).  gamma must be NULL.  CUDA-core
- * kernels for every dtype and d. */
+ * summaries m^K = sum k and n_t = sum_j k_j (q_j^T m^K_j)).  gamma: NULL, or device fp32 [H] for
+ * the decayed operator (divided by the decayed operator on ones).  CUDA-core kernels for every
+ * dtype and d. */
 hla_status_t ahla_forward_normalized(const void* q, const void* k, const void* v, float* o,
                                      int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                                      const float* gamma, float eps,
@@ -158,8 +164,8 @@ hla_status_t hla2_forward_unmasked(const void* q, const void* k, const void* v, 
  * timing hooks: when `phase_events` is non-NULL it points to four cudaEvent_t
  * handles (created by the caller, timing enabled) that are recorded on
  * `stream` before the segment-summary kernel, after it, after the scan, and
- * after the output kernel.  gamma is accepted for HLA_OP_HLA2 and
- * HLA_OP_HLA2_NORM only; eps is used by HLA_OP_HLA2_NORM only.
+ * after the output kernel.  gamma as for the op's own entry point; eps is used
+ * by the ratio-normalised ops only.
  */
 hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, const void* v, float* o,
                                   int B, int H, int T, int d, int dv, hla_dtype_t dtype,
@@ -204,7 +210,9 @@ int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, in
  */
 
 /* Floats of one head's state, or 0 when (op, decayed, d, dv) is invalid or unsupported
- * (decayed: hla2 / hla2_normalized with gamma). */
+ * (decayed: hla2 / hla2_normalized with gamma; the decayed AHLA and third order have a
+ * forward but no streaming state, and hla_state / hla_step refuse them with
+ * HLA_ERR_UNSUPPORTED). */
 size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv);
 
 /* Workspace bytes hla_state() needs, or 0 when the request is invalid or unsupported.

@@ -60,7 +60,9 @@ def test_workspace_sizes(lib):
     assert ws(hla.OP_HLA2, hla.HLA_F32, 0, 1, 1, 10, 64, 32) == 0          # d != dv
     assert ws(hla.OP_HLA2, hla.HLA_F32, 0, 0, 1, 10, 64, 64) == 0          # B = 0
     assert ws(hla.OP_HLA2, 7, 0, 1, 1, 10, 64, 64) == 0                    # bad dtype
-    assert ws(hla.OP_AHLA, hla.HLA_F32, 1, 1, 1, 10, 64, 64) == 0          # no decayed AHLA
+    assert ws(hla.OP_AHLA, hla.HLA_F32, 1, 1, 1, 10, 64, 64) > 0           # decayed AHLA
+    assert ws(hla.OP_HLA3, hla.HLA_F32, 1, 1, 1, 10, 32, 32) > 0           # decayed third order
+    assert ws(hla.OP_HLA2_UNMASKED, hla.HLA_F32, 1, 1, 1, 10, 64, 64) == 0  # no decayed unmasked op
     assert ws(9, hla.HLA_F32, 0, 1, 1, 10, 64, 64) == 0                    # bad op
 
 
@@ -124,10 +126,7 @@ def test_argument_errors_are_reported_before_any_launch(lib, name):
     assert _call(lib, name, ws=0) == 6                     # HLA_ERR_WORKSPACE
     assert _call(lib, name, wsb=64) == 6
     assert _call(lib, name, ws=32 + 8) == 3
-    if name in ("ahla_forward", "hla3_forward"):
-        assert _call(lib, name, gamma=64) == 5             # gamma only for second order
-    else:
-        assert _call(lib, name, gamma=66) == 3             # misaligned gamma
+    assert _call(lib, name, gamma=66) == 3                 # misaligned gamma
 
 
 def test_segment_chunks_knob(lib):
@@ -200,17 +199,19 @@ def test_streaming_state_sizes_and_argument_errors(lib):
 
 def test_normalised_ahla_hla3_routing_and_errors(lib):
     """Ratio-normalised AHLA / third order: CUDA-core kernels (the tensor-core AHLA walker
-    carries no normaliser), no decayed form, the plain op's workspace."""
+    carries no normaliser), a decayed form on the CUDA cores, the plain op's workspace."""
     vp, f = ctypes.c_void_p, ctypes.c_float
     for op, plain in ((hla.OP_AHLA_NORM, hla.OP_AHLA), (hla.OP_HLA3_NORM, hla.OP_HLA3)):
         assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
-        assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0           # no decay
+        assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) > 0            # decayed form
+        assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0
         assert lib.hla_workspace_bytes(op, hla.HLA_F32, 0, 2, 8, 4096, 32, 32) == \
             lib.hla_workspace_bytes(plain, hla.HLA_F32, 0, 2, 8, 4096, 32, 32)
     assert lib.hla_uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 1
     a = [vp(16)] * 4
     for fn in (lib.ahla_forward_normalized, lib.hla3_forward_normalized):
-        assert fn(*a, 1, 1, 64, 64, 64, 0, vp(16), f(1e-6), vp(16), 1 << 20, vp(0)) == 5     # gamma given
+        assert fn(*a, 1, 1, 64, 64, 64, 0, vp(16), f(1e-6), vp(16), 64, vp(0)) == 6          # gamma: decayed,
+        assert fn(*a, 1, 1, 64, 64, 64, 0, vp(18), f(1e-6), vp(16), 1 << 20, vp(0)) == 3     # sized, aligned
         assert fn(vp(0), *a[1:], 1, 1, 64, 64, 64, 0, vp(0), f(1e-6), vp(16), 1 << 20, vp(0)) == 1
         assert fn(*a, 1, 1, 64, 64, 64, 0, vp(0), f(1e-6), vp(16), 64, vp(0)) == 6           # workspace
 

@@ -285,3 +285,45 @@ def test_normalised_ahla_hla3_parity(op, dtype, d, T):
     o = gpu_forward(op, q, k, v, None, eps=w.eps)
     ref = reference(op, q, k, v, None, eps=w.eps)
     assert oracle.max_row_rel_err(o.cpu(), ref) <= TOL[dtype]
+
+
+# ---------------------------------------------------------------------------
+# decayed AHLA and third order, plain and ratio-normalised (CUDA-core kernels)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("op", ["ahlad", "hla3d", "ahlan", "hla3n"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 65, 200, 1000])
+def test_decayed_ahla_hla3_parity(op, dtype, d, T):
+    norm = op.endswith("n")
+    w = hla_inputs.Workload(f"{op}_{dtype}_1x2x{T}x{d}", op, dtype, 1, 2, T, d, d,
+                            "softplus" if norm else "scaled", "unit" if norm else "scaled", seed=T + 17,
+                            gamma_range=(0.9, 0.999))
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(op, q, k, v, g, eps=w.eps)
+    ref = reference(op, q, k, v, g, eps=w.eps)
+    assert oracle.max_row_rel_err(o.cpu(), ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("op", ["ahlad", "hla3d"])
+@pytest.mark.parametrize("gam", [0.5, 0.95, 0.999])
+def test_decayed_ahla_hla3_strong_and_weak(op, gam):
+    """One gamma per run, from strong to weak decay, several chunks and a ragged tail."""
+    d = 64 if op == "ahlad" else 32
+    dtype = "bf16" if op == "ahlad" else "f32"
+    w = hla_inputs.Workload(f"{op}_{gam}", op, dtype, 1, 2, 777, d, d, "scaled", "scaled", seed=int(gam * 1000))
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    g = torch.full((2,), gam)
+    o = gpu_forward(op, q, k, v, g)
+    assert oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g)) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("op", ["ahla", "hla3"])
+def test_decayed_gamma_one_matches_undecayed(op):
+    d, dtype = (64, "bf16") if op == "ahla" else (32, "f32")
+    w = hla_inputs.Workload(f"{op}_g1", op, dtype, 1, 2, 300, d, d, "scaled", "scaled", seed=3)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    a = gpu_forward(op + "d", q, k, v, torch.ones(2))
+    b = gpu_forward(op, q, k, v, None)
+    assert oracle.max_row_rel_err(a.cpu(), b.cpu()) <= TOL[dtype]
