@@ -168,6 +168,11 @@ struct TileT {                     // transposed view: element (r, c) = tile[c][
     int ld;
     __device__ float operator()(int r, int c) const { return p[c * ld + r]; }
 };
+struct GTile {                  // element (r, c) of a row-major matrix in global memory
+    const float* p;
+    int ld;
+    __device__ float operator()(int r, int c) const { return p[r * ld + c]; }
+};
 struct Put {                    // plain store into a tile
     float* p;
     int ld;
@@ -663,6 +668,85 @@ __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int 
 }
 
 // ---------------------------------------------------------------------------
+// Third order: the exclusive prefix in factored form.  The combine's cross terms depend on the
+// earlier operand only through S, P and m^K, which add plainly, so unrolled over the chunks
+//     S0(n) = sum_{l<n} S_l,   P0(n) = sum_{l<n} P_l,   mK0(n) = sum_{l<n} mK_l,
+//     F0(n) = sum_{l<n} (F_l + S0(l) Q2_l P0(l) + S0(l) X_l + Z_l P0(l)),
+//     F1_0(n) = sum_{l<n} (F1_l + S0(l) Q2_l mK0(l) + S0(l) X1_l + Z_l mK0(l)),
+// which are all the output kernel reads.  Three launches, each parallel over chunks or elements:
+// plain exclusive sums of S, P, mK in place; the corrected F_l, F1_l per chunk; their exclusive
+// sums in place.  The result equals the Blelloch tree's up to the order of fp32 additions.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ sums, int NC, int NCp, int which) {
+    using S = Sum<OP_HLA3, D>;
+    const int e = blockIdx.x * NT + threadIdx.x;
+    int off;
+    if (which == 0) {                        // S, P and mK
+        if (e >= 2 * D * D + D) return;
+        off = e < D * D ? S::mat(0) + e : e < 2 * D * D ? S::mat(2) + (e - D * D) : S::vec(0) + (e - 2 * D * D);
+    } else {                                 // the corrected F and F1
+        if (e >= D * D + D) return;
+        off = e < D * D ? S::mat(3) + e : S::vec(2) + (e - D * D);
+    }
+    float* p = sums + (size_t)blockIdx.y * NCp * S::SIZE + off;
+    float run = 0.f;
+    for (int l = 0; l < NC; ++l) {
+        const float y = p[(size_t)l * S::SIZE];
+        p[(size_t)l * S::SIZE] = run;
+        run += y;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ sums, int NCp) {
+    using S = Sum<OP_HLA3, D>;
+    constexpr int LD = Dim<D>::LD;
+    extern __shared__ float smx[];
+    float* S0 = smx;
+    float* P0 = S0 + D * LD;
+    float* SQ = P0 + D * LD;
+    float* mk = SQ + D * LD;
+    float* sq_m = mk + D;
+    float* slot = sums + ((size_t)blockIdx.y * NCp + blockIdx.x) * S::SIZE;
+    load_mat<D>(S0, slot + S::mat(0));       // S0(l) (the plain prefix, in place)
+    load_mat<D>(P0, slot + S::mat(2));       // P0(l)
+    for (int a = threadIdx.x; a < D; a += blockDim.x) mk[a] = slot[S::vec(0) + a];
+    __syncthreads();
+    const float* Q2 = slot + S::mat(1);
+    mm<D, D, D>(Tile{S0, LD}, GTile{Q2, D}, Zero{}, Put{SQ, LD});                  // S0 Q2
+    __syncthreads();
+    float* F = slot + S::mat(3);
+    // F += (S0 Q2) P0 + S0 X + Z P0
+    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, GTile{slot + S::mat(4), D},
+                       GTile{slot + S::mat(5), D}, Tile{P0, LD}, [&](int r, int c) { return F[r * D + c]; },
+                       [&](int r, int c, float x) { F[r * D + c] = x; });
+    for (int a = threadIdx.x; a < D; a += blockDim.x) {
+        float s = 0.f;
+        for (int b = 0; b < D; ++b)
+            s += SQ[a * LD + b] * mk[b] + S0[a * LD + b] * slot[S::vec(1) + b] + slot[S::mat(5) + a * D + b] * mk[b];
+        sq_m[a] = s;
+    }
+    __syncthreads();
+    for (int a = threadIdx.x; a < D; a += blockDim.x) slot[S::vec(2) + a] += sq_m[a];
+}
+
+template <int D>
+static cudaError_t hla3_factored_prefix(float* sums, int NC, int NCp, int BH, cudaStream_t st) {
+    k_hla3_prefix_plain<D><<<dim3((2 * D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 0);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int smem = (int)(sizeof(float) * (3 * D * Dim<D>::LD + 2 * D));
+    if ((e = cudaFuncSetAttribute(k_hla3_prefix_cross<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    k_hla3_prefix_cross<D><<<dim3(NC, BH), NT, smem, st>>>(sums, NCp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_hla3_prefix_plain<D><<<dim3((D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 1);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Output kernel: one block per (chunk, head); applies the chunk's prefix.
 // ---------------------------------------------------------------------------
 template <int OP, bool NORM, int D, typename TIn>
@@ -975,7 +1059,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, H, T, NC, NCp, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if (fold_fits<OP, D>()) {
+    if (OP == OP_HLA3) {
+        if ((e = hla3_factored_prefix<D>(sums, NC, NCp, BH, st)) != cudaSuccess) return e;
+    } else if (fold_fits<OP, D>()) {
         auto kf = k_scan_fold<OP, D>;
         if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fold_smem<OP, D>())) !=
             cudaSuccess)
@@ -1045,6 +1131,7 @@ static bool uses_fold(int op, int d) {
 }
 
 int kernel_launches(int op, int d, int T) {
+    if (op == OP_HLA3) return 2 + 3;          // the factored prefix
     return 2 + (uses_fold(op, d) ? 1 : scan_launches(next_pow2((T + C - 1) / C)));
 }
 

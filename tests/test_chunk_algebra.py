@@ -386,3 +386,32 @@ def test_normaliser_vectors_give_the_literal_denominator():
         F1 = F1 + (S @ q[t]) * (q[t] @ mk)
         assert abs(q[t] @ nv - den_a[t]) < 1e-12 * max(1.0, den_a[t])
         assert abs(q[t] @ F1 - den_3[t]) < 1e-12 * max(1.0, den_3[t])
+
+
+def third_order_factored_prefix(sums):
+    """The third-order exclusive prefix as the CUDA-core path runs it (three launches): plain
+    exclusive sums S0, P0, then per chunk the corrected F_l + S0(l) Q2_l P0(l) + S0(l) X_l +
+    Z_l P0(l), then its plain exclusive sum F0."""
+    S0 = [0.0 * sums[0]["S"]]
+    P0 = [0.0 * sums[0]["P"]]
+    for s in sums[:-1]:
+        S0.append(S0[-1] + s["S"])
+        P0.append(P0[-1] + s["P"])
+    Y = [s["F"] + S0[l] @ s["Q2"] @ P0[l] + S0[l] @ s["X"] + s["Z"] @ P0[l] for l, s in enumerate(sums)]
+    F0 = [0.0 * Y[0]]
+    for y in Y[:-1]:
+        F0.append(F0[-1] + y)
+    return [dict(S=S0[l], P=P0[l], F=F0[l]) for l in range(len(sums))]
+
+
+@pytest.mark.parametrize("lengths", [[6], [3, 9, 1], [8, 8, 8, 8, 8], [1, 2, 3, 4, 5, 6, 7]])
+def test_third_order_factored_prefix_equals_the_combine_fold(lengths):
+    T, d, dv = sum(lengths), 4, 3
+    q, k, v = rand_head(T, d, dv, seed=7 + len(lengths))
+    b = seg.split_points(T, lengths)
+    sums = [seg.hla3_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]]) for i in range(len(lengths))]
+    ref = seg.fold_exclusive(sums, seg.hla3_combine, seg.hla3_identity(d, dv))
+    got = third_order_factored_prefix(sums)
+    for n in range(len(lengths)):
+        for key in ("S", "P", "F"):
+            np.testing.assert_allclose(got[n][key], ref[n][key], rtol=0, atol=1e-11)
