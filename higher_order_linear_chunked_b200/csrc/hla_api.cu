@@ -95,8 +95,12 @@ hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, f
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 
-// Streaming-state requests run on the CUDA-core kernels (fp32 state, any supported dtype).
+// Streaming-state requests: the undecayed second order with bf16 inputs and d = 64 runs on the
+// tensor-core summary walker; everything else on the CUDA-core kernels (fp32 state either way).
+bool state_on_tc(const Request& r) { return r.op == hla::OP_HLA2 && use_tc(r); }
+
 size_t state_workspace_for(const Request& r) {
+    if (state_on_tc(r)) return hla::kStatusBytes + hla::tc::state_workspace_bytes(r.B * r.H, r.T);
     return hla::kStatusBytes + sizeof(float) * hla::simt::workspace_floats(r.op, r.d, r.B * r.H, r.T);
 }
 
@@ -209,6 +213,7 @@ size_t hla_state_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, in
 
 int hla_state_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
     if (hla_state_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
+    if (state_on_tc(make_request(op, decayed != 0, dtype, B, H, T, d, dv))) return 2;
     return hla::simt::state_launches(T);
 }
 
@@ -229,7 +234,9 @@ hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
     float* sums = reinterpret_cast<float*>(static_cast<char*>(workspace) + hla::kStatusBytes);
-    const cudaError_t e = hla::simt::state(r.op, r.bf16, d, q, k, v, gamma, B * H, H, T, sums, state, st);
+    const cudaError_t e = state_on_tc(r)
+                              ? hla::tc::state(q, k, v, B * H, T, sums, static_cast<int*>(workspace), state, st)
+                              : hla::simt::state(r.op, r.bf16, d, q, k, v, gamma, B * H, H, T, sums, state, st);
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 

@@ -706,29 +706,33 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ su
     float* S0 = smx;
     float* P0 = S0 + D * LD;
     float* SQ = P0 + D * LD;
-    float* mk = SQ + D * LD;
-    float* sq_m = mk + D;
+    float* Q2 = SQ + D * LD;
+    float* Xs = Q2 + D * LD;
+    float* Zs = Xs + D * LD;
+    float* mk = Zs + D * LD;
+    float* x1 = mk + D;
     float* slot = sums + ((size_t)blockIdx.y * NCp + blockIdx.x) * S::SIZE;
     load_mat<D>(S0, slot + S::mat(0));       // S0(l) (the plain prefix, in place)
+    load_mat<D>(Q2, slot + S::mat(1));
     load_mat<D>(P0, slot + S::mat(2));       // P0(l)
-    for (int a = threadIdx.x; a < D; a += blockDim.x) mk[a] = slot[S::vec(0) + a];
+    load_mat<D>(Xs, slot + S::mat(4));
+    load_mat<D>(Zs, slot + S::mat(5));
+    for (int a = threadIdx.x; a < D; a += blockDim.x) {
+        mk[a] = slot[S::vec(0) + a];
+        x1[a] = slot[S::vec(1) + a];
+    }
     __syncthreads();
-    const float* Q2 = slot + S::mat(1);
-    mm<D, D, D>(Tile{S0, LD}, GTile{Q2, D}, Zero{}, Put{SQ, LD});                  // S0 Q2
+    mm<D, D, D>(Tile{S0, LD}, Tile{Q2, LD}, Zero{}, Put{SQ, LD});                  // S0 Q2
     __syncthreads();
     float* F = slot + S::mat(3);
     // F += (S0 Q2) P0 + S0 X + Z P0
-    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, GTile{slot + S::mat(4), D},
-                       GTile{slot + S::mat(5), D}, Tile{P0, LD}, [&](int r, int c) { return F[r * D + c]; },
-                       [&](int r, int c, float x) { F[r * D + c] = x; });
+    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, Tile{Xs, LD}, Tile{Zs, LD}, Tile{P0, LD},
+                       [&](int r, int c) { return F[r * D + c]; }, [&](int r, int c, float x) { F[r * D + c] = x; });
     for (int a = threadIdx.x; a < D; a += blockDim.x) {
         float s = 0.f;
-        for (int b = 0; b < D; ++b)
-            s += SQ[a * LD + b] * mk[b] + S0[a * LD + b] * slot[S::vec(1) + b] + slot[S::mat(5) + a * D + b] * mk[b];
-        sq_m[a] = s;
+        for (int b = 0; b < D; ++b) s += SQ[a * LD + b] * mk[b] + S0[a * LD + b] * x1[b] + Zs[a * LD + b] * mk[b];
+        slot[S::vec(2) + a] += s;
     }
-    __syncthreads();
-    for (int a = threadIdx.x; a < D; a += blockDim.x) slot[S::vec(2) + a] += sq_m[a];
 }
 
 template <int D>
@@ -736,7 +740,7 @@ static cudaError_t hla3_factored_prefix(float* sums, int NC, int NCp, int BH, cu
     k_hla3_prefix_plain<D><<<dim3((2 * D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int smem = (int)(sizeof(float) * (3 * D * Dim<D>::LD + 2 * D));
+    const int smem = (int)(sizeof(float) * (6 * D * Dim<D>::LD + 2 * D));
     if ((e = cudaFuncSetAttribute(k_hla3_prefix_cross<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
         return e;
@@ -1559,10 +1563,17 @@ __global__ void __launch_bounds__(NT) k_bwd_suffix(float* __restrict__ bw, int N
     if (e >= D * D) return;
     float* p = bw + (size_t)blockIdx.y * NCp * Bwd<D>::SIZE + slot * D * D + e;
     float run = 0.f;
-    for (int c = NC - 1; c >= 0; --c) {
-        const float y = p[(size_t)c * Bwd<D>::SIZE];
-        p[(size_t)c * Bwd<D>::SIZE] = run;
-        run += y;
+    for (int c0 = NC - 1; c0 >= 0; c0 -= 8) {      // eight independent loads in flight
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (c0 - i >= 0) y[i] = p[(size_t)(c0 - i) * Bwd<D>::SIZE];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (c0 - i >= 0) {
+                p[(size_t)(c0 - i) * Bwd<D>::SIZE] = run;
+                run += y[i];
+            }
     }
 }
 

@@ -21,6 +21,11 @@ size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks);
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
                     float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
                     int seg_chunks);
+// streaming state (second order, bf16, d = 64): the summary walker over every chunk of every
+// head, then each head's segments combined into state_out [BH][summary floats]; two launches
+size_t state_workspace_bytes(int BH, int T);
+cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, void* ws, int* status, float* state_out,
+                  cudaStream_t st);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

@@ -789,6 +789,78 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_sum(float* __restrict__ pre, i
     }
 }
 
+// ---------------------------------------------------------------- streaming state
+// The state after a head's T tokens is the combine of its segment summaries in order:
+//   S = sum_l S_l,  C = sum_l C_l,  m = sum_l m_l,
+//   R = sum_l R_l + sum_{j < NS-1} S_j Csuf(j+1),  r = sum_l r_l + sum_{j < NS-1} S_j msuf(j+1),
+// with Csuf(j) = sum_{l >= j} C_l (the combine's cross terms grouped by their S factor).  One
+// CTA per head; the result is written in the slot layout, which is also the state layout.
+__global__ void __launch_bounds__(PX_NT) k_state_total(const float* __restrict__ sums, int NS, int NSp,
+                                                       float* __restrict__ state) {
+    using S = simt_layout;
+    __shared__ __align__(16) float Sj[D * (D + 4)];
+    __shared__ __align__(16) float Cs[D * D];
+    __shared__ float ms[D];
+    const int bh = blockIdx.x, tid = threadIdx.x;
+    const float* sb = sums + (size_t)bh * NSp * S::size;
+    float* out = state + (size_t)bh * S::size;
+    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);      // this thread's 4 x 4 of R
+    float racc[4][4];
+    for (int a = 0; a < 4; ++a)
+        for (int b = 0; b < 4; ++b) racc[a][b] = 0.f;
+    float rv = 0.f;
+    // plain sums of S, C, m, R, r
+    for (int f = tid; f < 2 * D * D / 4; f += PX_NT) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int l = 0; l < NS; ++l) {
+            const float4 x = reinterpret_cast<const float4*>(sb + (size_t)l * S::size)[f];
+            acc = make_float4(acc.x + x.x, acc.y + x.y, acc.z + x.z, acc.w + x.w);
+        }
+        reinterpret_cast<float4*>(out)[f] = acc;               // S, then C
+    }
+    if (tid < D) {
+        float mv = 0.f;
+        for (int l = 0; l < NS; ++l) {
+            mv += sb[(size_t)l * S::size + S::vec(0) + tid];
+            rv += sb[(size_t)l * S::size + S::vec(1) + tid];
+        }
+        out[S::vec(0) + tid] = mv;
+    }
+    for (int l = 0; l < NS; ++l)
+        for (int a = 0; a < 4; ++a) {
+            const float4 x = *reinterpret_cast<const float4*>(sb + (size_t)l * S::size + S::mat(2) + (r + a) * D + c);
+            racc[a][0] += x.x; racc[a][1] += x.y; racc[a][2] += x.z; racc[a][3] += x.w;
+        }
+    // cross terms, from the last segment backwards
+    for (int j = NS - 2; j >= 0; --j) {
+        const float* cl = sb + (size_t)(j + 1) * S::size;
+        const float* sj = sb + (size_t)j * S::size;
+        for (int f = tid; f < D * D; f += PX_NT) {
+            Cs[f] = (j == NS - 2 ? 0.f : Cs[f]) + cl[S::mat(1) + f];
+            Sj[(f / D) * (D + 4) + f % D] = sj[S::mat(0) + f];
+        }
+        if (tid < D) ms[tid] = (j == NS - 2 ? 0.f : ms[tid]) + cl[S::vec(0) + tid];
+        __syncthreads();
+        for (int k = 0; k < D; ++k) {
+            const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
+            for (int a = 0; a < 4; ++a) {
+                const float sv = Sj[(r + a) * (D + 4) + k];
+                racc[a][0] = fmaf(sv, cv.x, racc[a][0]);
+                racc[a][1] = fmaf(sv, cv.y, racc[a][1]);
+                racc[a][2] = fmaf(sv, cv.z, racc[a][2]);
+                racc[a][3] = fmaf(sv, cv.w, racc[a][3]);
+            }
+        }
+        if (tid < D)
+            for (int k = 0; k < D; ++k) rv = fmaf(Sj[tid * (D + 4) + k], ms[k], rv);
+        __syncthreads();
+    }
+    for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4*>(out + S::mat(2) + (r + a) * D + c) = make_float4(racc[a][0], racc[a][1], racc[a][2], racc[a][3]);
+    if (tid < D) out[S::vec(1) + tid] = rv;
+    for (int e = S::vec(0) + 2 * D + tid; e < S::size; e += PX_NT) out[e] = 0.f;
+}
+
 // ---------------------------------------------------------------- host side
 namespace {
 
@@ -891,6 +963,54 @@ cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(pre, NS, NSp);
+    return cudaGetLastError();
+}
+
+// Segment length of the state walk: every chunk of every head is summarised, in segments of
+// `len` chunks, one CTA each; the same makespan model as plan(): waves x (len + 1) chunk-times,
+// plus about one per segment for the per-head combine.
+static int state_segment_chunks(int BH, int T) {
+    const int NC = (T + C - 1) / C;
+    int best_len = 1;
+    long long best = -1;
+    for (int len = 1; len <= 16; len *= 2) {
+        const long long ns = (NC + len - 1) / len;
+        const long long c = ((BH * ns + kSMs - 1) / kSMs) * (len + 1) + ns;
+        if (best < 0 || c < best) {
+            best = c;
+            best_len = len;
+        }
+        if (len >= NC) break;
+    }
+    return best_len;
+}
+
+size_t state_workspace_bytes(int BH, int T) {
+    const int len = state_segment_chunks(BH, T);
+    const int NS = ((T + C - 1) / C + len - 1) / len;
+    return sizeof(float) * (size_t)BH * next_pow2(NS) * simt_layout::size;
+}
+
+cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, void* ws, int* status, float* state_out,
+                  cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
+        !make_map_out(&mo, state_out, 1, 1))
+        return cudaErrorInvalidValue;
+    const int len = state_segment_chunks(BH, T);
+    const int NS = ((T + C - 1) / C + len - 1) / len;
+    Params sprm{};
+    sprm.T = T; sprm.BH = BH; sprm.NCH = len; sprm.NS = NS; sprm.NSp = next_pow2(NS); sprm.ratio = 1;
+    sprm.fold = 0; sprm.eps = 0.f; sprm.norm = 0;
+    sprm.sums = static_cast<float*>(ws);
+    sprm.pre = nullptr;
+    sprm.o = nullptr;
+    sprm.status = status;
+    cudaError_t e;
+    if ((e = set_smem(k_walk<SUMMARY>, SMEM_BYTES)) != cudaSuccess) return e;
+    k_walk<SUMMARY><<<dim3(NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_state_total<<<BH, PX_NT, 0, st>>>(sprm.sums, NS, sprm.NSp, state_out);
     return cudaGetLastError();
 }
 

@@ -225,7 +225,10 @@ int hla_state_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B
 /*
  * Prefill: the state of every head after its T tokens, written to state
  * [B*H][hla_state_floats] (device, fp32, 16-byte aligned, caller-owned).
- * q, k, v, gamma, shapes and dtypes as for the forward calls.  Runs the
+ * q, k, v, gamma, shapes and dtypes as for the forward calls.  The undecayed
+ * second order (plain or ratio-normalised) with bf16 inputs and d = dv = 64 runs
+ * the tensor-core summary walker over segments of every head, then one CTA per
+ * head combines the segment summaries (two launches).  Everything else runs the
  * CUDA-core chunk-summary kernel and the up-sweep half of the Blelloch scan,
  * whose root is the summary of the whole sequence.  Workspace: at least
  * hla_state_workspace_bytes().  Errors as for the forward calls.

@@ -175,10 +175,17 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert lib.hla_state_floats(0, 0, 48, 48) == 0
     assert lib.hla_state_floats(0, 0, 64, 32) == 0
     # workspace: status block + the CUDA-core chunk summaries (64-token chunks, padded to 2^k)
-    n = lib.hla_state_workspace_bytes(0, 1, 0, 4, 16, 4096, d, d)
+    n = lib.hla_state_workspace_bytes(0, 0, 0, 4, 16, 4096, d, d)
     assert n == 256 + 4 * 64 * 64 * lib.hla_state_floats(0, 0, d, d)
     assert lib.hla_state_workspace_bytes(2, 1, 1, 4, 16, 4096, d, d) == 0
-    assert lib.hla_state_kernel_launches(0, 1, 0, 4, 16, 4096, d, d) == 2 + 6     # 64 chunks: 6 levels
+    assert lib.hla_state_kernel_launches(0, 0, 0, 4, 16, 4096, d, d) == 2 + 6     # 64 chunks: 6 levels
+    # bf16, d = 64, undecayed second order: the tensor-core summary walker over 16-chunk segments
+    # (two per head at T = 4096), then one combine per head
+    n = lib.hla_state_workspace_bytes(0, 1, 0, 4, 16, 4096, d, d)
+    assert n == 256 + 64 * 2 * 4 * lib.hla_state_floats(0, 0, d, d)
+    assert lib.hla_state_kernel_launches(0, 1, 0, 4, 16, 4096, d, d) == 2
+    assert lib.hla_state_kernel_launches(1, 1, 0, 4, 16, 4096, d, d) == 2
+    assert lib.hla_state_kernel_launches(0, 1, 1, 4, 16, 4096, d, d) == 2 + 6     # decayed: CUDA cores
     assert lib.hla_state_kernel_launches(0, 0, 0, 1, 1, 64, 32, 32) == 2
     st = lib.hla_state
     a = [vp(16), vp(16), vp(16), vp(16)]

@@ -24,6 +24,15 @@ pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 STATE_TOL = 1e-4          # fp32 state against fp64, relative to each matrix's largest entry
+# The undecayed second order with bf16 inputs and d = 64 exports its state from the tensor-core
+# summary walker, whose MMA operands (A, S0, Z) are rounded to bf16 (unit roundoff 2^-9, about
+# 2e-3): its matrices carry that rounding, a few units of 2e-3 of the matrix scale, bounded here
+# by 1e-2.  The outputs decoded from it still meet the bf16 output gate (2e-2), checked below.
+STATE_TOL_TC = 1e-2
+
+
+def state_tol(op, dtype, d):
+    return STATE_TOL_TC if (op in ("hla2", "hla2n") and dtype == "bf16" and d == 64) else STATE_TOL
 OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n"]
 NORMALISED = ("hla2n", "ahlan", "hla3n")
 DEV = torch.device("cuda:0")
@@ -70,10 +79,10 @@ def split_state(op, x, d):
     return out
 
 
-def assert_state_close(op, got, want, d):
+def assert_state_close(op, got, want, d, tol=STATE_TOL):
     for a, b in zip(split_state(op, got, d), want):
         scale = max(np.abs(b).max(), 1e-30)
-        assert np.abs(np.asarray(a, np.float64) - b).max() / scale < STATE_TOL
+        assert np.abs(np.asarray(a, np.float64) - b).max() / scale < tol
 
 
 def gpu(x):
@@ -91,7 +100,7 @@ def test_exported_state_is_the_prefix_summary(op, dtype, d, T):
     for h in range(2):
         want = oracle_state(op, q[0, h].double().numpy(), k[0, h].double().numpy(), v[0, h].double().numpy(),
                             float(g[h]) if g is not None else None)
-        assert_state_close(op, st[0, h], want, d)
+        assert_state_close(op, st[0, h], want, d, state_tol(op, dtype, d))
 
 
 @pytest.mark.parametrize("op", OPS)
@@ -116,7 +125,7 @@ def test_prefill_then_decode_equals_the_forward(op, dtype, T0, T1):
     for b in range(2):
         for h in range(3):
             want = split_state(op, whole[b, h], d)
-            assert_state_close(op, got[b, h], [np.asarray(x, np.float64) for x in want], d)
+            assert_state_close(op, got[b, h], [np.asarray(x, np.float64) for x in want], d, state_tol(op, dtype, d))
 
 
 @pytest.mark.parametrize("op", OPS)
