@@ -40,7 +40,8 @@ EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_for
            "hla2_forward_normalized_noalloc", "hla_state_floats", "hla_state_workspace_bytes",
            "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked",
            "ahla_forward_normalized", "hla3_forward_normalized", "hla_noalloc_read_device_status",
-           "hla_backward_workspace_bytes", "hla_backward_kernel_launches", "hla2_backward")
+           "hla_backward_workspace_bytes", "hla_backward_kernel_launches", "hla2_backward",
+           "hla2_backward_normalized")
 
 
 class HLAError(RuntimeError):
@@ -93,6 +94,8 @@ def load_library(path: Optional[str] = None):
     lib.hla_backward_kernel_launches.restype = i
     lib.hla2_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, sz, vp]
     lib.hla2_backward.restype = i
+    lib.hla2_backward_normalized.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]
+    lib.hla2_backward_normalized.restype = i
     lib.hla_noalloc_read_device_status.argtypes = [vp, ctypes.POINTER(i)]
     lib.hla_noalloc_read_device_status.restype = i
     lib.hla_selftest_umma.argtypes = [i, vp, vp, vp, i, i, vp]
@@ -235,9 +238,10 @@ def hla2_unmasked(q, k, v, out=None, workspace=None, stream=None):
     return _call(OP_HLA2_UNMASKED, q, k, v, out=out, workspace=workspace, stream=stream)
 
 
-def hla2_backward(q, k, v, dout, workspace=None, stream=None):
+def hla2_backward(q, k, v, dout, workspace=None, stream=None, normalized: bool = False, eps: float = 1e-6):
     """Gradients (dq, dk, dv), fp32, of sum(O * dout) for O = hla2(q, k, v) (masked second order,
-    no decay).  dout: fp32 [B, H, T, dv] on q's device."""
+    no decay), or O = hla2_normalized(q, k, v, eps) with ``normalized``.  dout: fp32 [B, H, T, dv]
+    on q's device."""
     torch = _torch()
     _check(q, k, v)
     if not dout.is_cuda or dout.dtype != torch.float32 or not dout.is_contiguous() or dout.shape != v.shape:
@@ -245,7 +249,8 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None):
     lib = load_library()
     B, H, T, d = q.shape
     dvd = v.shape[-1]
-    n = int(lib.hla_backward_workspace_bytes(OP_HLA2, _dtype_code(q), B, H, T, d, dvd))
+    op = OP_HLA2_NORM if normalized else OP_HLA2
+    n = int(lib.hla_backward_workspace_bytes(op, _dtype_code(q), B, H, T, d, dvd))
     if n == 0:
         raise HLAError(5, "no backward kernel for this shape/dtype")
     if workspace is None:
@@ -255,9 +260,13 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None):
     dv = torch.empty((B, H, T, dvd), dtype=torch.float32, device=q.device)
     st = stream if stream is not None else torch.cuda.current_stream(q.device)
     vp = ctypes.c_void_p
-    rc = lib.hla2_backward(vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()), vp(dout.data_ptr()),
-                           vp(dq.data_ptr()), vp(dk.data_ptr()), vp(dv.data_ptr()), B, H, T, d, dvd, _dtype_code(q),
-                           vp(0), vp(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()), vp(st.cuda_stream))
+    head = [vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()), vp(dout.data_ptr()), vp(dq.data_ptr()),
+            vp(dk.data_ptr()), vp(dv.data_ptr()), B, H, T, d, dvd, _dtype_code(q), vp(0)]
+    tail = [vp(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()), vp(st.cuda_stream)]
+    if normalized:
+        rc = lib.hla2_backward_normalized(*head, ctypes.c_float(eps), *tail)
+    else:
+        rc = lib.hla2_backward(*head, *tail)
     if rc != HLA_OK:
         raise HLAError(rc, "hla2_backward rejected the call")
     return dq, dk, dv

@@ -256,19 +256,22 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
 }
 
 size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
-    if (op != HLA_OP_HLA2) return 0;
+    if (op != HLA_OP_HLA2 && op != HLA_OP_HLA2_NORM) return 0;
     if (check_shape(dtype, B, H, T, d, dv) != HLA_OK) return 0;
+    if (op == HLA_OP_HLA2_NORM)
+        return hla::kStatusBytes + sizeof(float) * hla::simt::backward_normalized_workspace_floats(d, B * H, T);
     return hla::kStatusBytes + sizeof(float) * hla::simt::backward_workspace_floats(d, B * H, T);
 }
 
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
     if (hla_backward_workspace_bytes(op, dtype, B, H, T, d, dv) == 0) return 0;
-    return hla::simt::backward_launches(d, T);
+    return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(d, T) : hla::simt::backward_launches(d, T);
 }
 
-hla_status_t hla2_backward(const void* q, const void* k, const void* v, const float* dout, float* dq, float* dk,
-                           float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+hla_status_t backward_call(hla_op_t op, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                           float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                           const float* gamma, float eps, void* workspace, size_t workspace_bytes, void* stream) {
     if (!q || !k || !v || !dout || !dq || !dk || !dv_out) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, T, d, dv);
     if (s != HLA_OK) return s;
@@ -278,12 +281,32 @@ hla_status_t hla2_backward(const void* q, const void* k, const void* v, const fl
         return HLA_ERR_ALIGN;
     if (!workspace) return HLA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return HLA_ERR_ALIGN;
-    if (workspace_bytes < hla_backward_workspace_bytes(HLA_OP_HLA2, dtype, B, H, T, d, dv)) return HLA_ERR_WORKSPACE;
+    if (workspace_bytes < hla_backward_workspace_bytes(op, dtype, B, H, T, d, dv)) return HLA_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
     float* body = reinterpret_cast<float*>(static_cast<char*>(workspace) + hla::kStatusBytes);
-    const cudaError_t e = hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, st);
+    const cudaError_t e =
+        op == HLA_OP_HLA2_NORM
+            ? hla::simt::backward_normalized(dtype == HLA_BF16, d, q, k, v, dout, eps, dq, dk, dv_out, B * H, T, body,
+                                             st)
+            : hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, st);
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
+}
+}  // namespace
+
+hla_status_t hla2_backward(const void* q, const void* k, const void* v, const float* dout, float* dq, float* dk,
+                           float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_call(HLA_OP_HLA2, q, k, v, dout, dq, dk, dv_out, B, H, T, d, dv, dtype, gamma, 0.f, workspace,
+                         workspace_bytes, stream);
+}
+
+hla_status_t hla2_backward_normalized(const void* q, const void* k, const void* v, const float* dout, float* dq,
+                                      float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                                      const float* gamma, float eps, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+    return backward_call(HLA_OP_HLA2_NORM, q, k, v, dout, dq, dk, dv_out, B, H, T, d, dv, dtype, gamma, eps, workspace,
+                         workspace_bytes, stream);
 }
 
 hla_status_t hla_set_segment_chunks(int chunks) {

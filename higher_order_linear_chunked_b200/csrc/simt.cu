@@ -27,6 +27,8 @@
 //                           column: vectors mK, X1, F1 and den = Q F1_0 + W (Q mK0 + A 1)
 //   unmasked       summary  S = K^T K, C = Q^T V;  combine S, C add;
 //   second order   output   W = L (.) (Q S0 Q^T + A A*^T), O = Q (S0 C0) + W V + (A K) C0
+#include <algorithm>
+
 #include "common.cuh"
 #include "simt.h"
 
@@ -1716,6 +1718,94 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
                                      dv);
+    return cudaGetLastError();
+}
+
+cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
+// Ratio-normalised second order: o = num / (den + eps), num = W V and den = W 1 (the same operator
+// on a ones value column).  With dO given,
+//     dnum = dO / (den + eps),   dden_t = -sum_f dO_tf num_tf / (den_t + eps)^2,
+// and den_t is column 0 of the operator on an all-ones value tensor, whose gradient with respect
+// to q and k, for an output gradient that is dden in column 0 and zero elsewhere, is the ones
+// term.  So (dq, dk, dv) = backward(q, k, v; dnum) + (the dq, dk of backward(q, k, 1; [dden, 0..])).
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void k_fill_ones(TIn* __restrict__ x, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        x[i] = TIn(1.f);
+}
+
+// One thread per (token, head) row: dnum and the ones term's output gradient (dden in column 0).
+template <int D>
+__global__ void k_norm_grads(const float* __restrict__ num, const float* __restrict__ den, const float* __restrict__ dout,
+                             float eps, size_t rows, float* __restrict__ dnum, float* __restrict__ g1) {
+    const size_t r = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const float s = 1.f / (den[r * D] + eps);
+    float acc = 0.f;
+    for (int f = 0; f < D; ++f) {
+        const float g = dout[r * D + f];
+        dnum[r * D + f] = g * s;
+        acc = fmaf(g, num[r * D + f], acc);
+        g1[r * D + f] = 0.f;
+    }
+    g1[r * D] = -acc * s * s;
+}
+
+__global__ void k_add_into(float* __restrict__ a, const float* __restrict__ b, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        a[i] += b[i];
+}
+
+size_t backward_normalized_workspace_floats(int d, int BH, int T) {
+    const size_t n = (size_t)BH * T * d;
+    const size_t inner = std::max(backward_workspace_floats(d, BH, T), workspace_floats(OP_HLA2, d, BH, T));
+    // num, the ones operator, the ones (as fp32: big enough for either dtype), dnum, its ones term's
+    // output gradient, dq2, dk2, dv2
+    return 8 * n + inner;
+}
+
+int backward_normalized_launches(int d, int T) {
+    // two plain forwards, the ones, the gradient split, two plain backwards, two additions
+    return 2 * kernel_launches(OP_HLA2, d, T) + 1 + 1 + 2 * backward_launches(d, T) + 2;
+}
+
+cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
+                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws,
+                                cudaStream_t st) {
+    const size_t n = (size_t)BH * T * d;
+    float* num = ws;
+    float* den = num + n;
+    float* ones = den + n;
+    float* dnum = ones + n;
+    float* g1 = dnum + n;
+    float* dq2 = g1 + n;
+    float* dk2 = dq2 + n;
+    float* dv2 = dk2 + n;
+    float* inner = dv2 + n;
+    const int blocks = 4 * 148;
+    cudaError_t e;
+    if (bf16) k_fill_ones<__nv_bfloat16><<<blocks, NT, 0, st>>>(reinterpret_cast<__nv_bfloat16*>(ones), n);
+    else k_fill_ones<float><<<blocks, NT, 0, st>>>(ones, n);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, v, nullptr, 0.f, num, BH, 1, T, inner, st, nullptr)) !=
+        cudaSuccess)
+        return e;
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, ones, nullptr, 0.f, den, BH, 1, T, inner, st, nullptr)) !=
+        cudaSuccess)
+        return e;
+    const size_t rows = (size_t)BH * T;
+    if (d == 32) k_norm_grads<32><<<(unsigned)((rows + NT - 1) / NT), NT, 0, st>>>(num, den, dout, eps, rows, dnum, g1);
+    else k_norm_grads<64><<<(unsigned)((rows + NT - 1) / NT), NT, 0, st>>>(num, den, dout, eps, rows, dnum, g1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = backward(bf16, d, q, k, v, dnum, dq, dk, dv, BH, T, inner, st)) != cudaSuccess) return e;
+    if ((e = backward(bf16, d, q, k, ones, g1, dq2, dk2, dv2, BH, T, inner, st)) != cudaSuccess) return e;
+    k_add_into<<<blocks, NT, 0, st>>>(dq, dq2, n);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_add_into<<<blocks, NT, 0, st>>>(dk, dk2, n);
     return cudaGetLastError();
 }
 

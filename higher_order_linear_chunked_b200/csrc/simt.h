@@ -44,6 +44,13 @@ size_t backward_workspace_floats(int d, int BH, int T);
 int backward_launches(int d, int T);
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
                      float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
+// The same for the ratio-normalised output (two plain forwards, two plain backwards, element-wise
+// glue); ws: backward_normalized_workspace_floats floats.
+size_t backward_normalized_workspace_floats(int d, int BH, int T);
+int backward_normalized_launches(int d, int T);
+cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
+                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws,
+                                cudaStream_t st);
 
 }  // namespace simt
 }  // namespace hla

@@ -256,9 +256,9 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
  * parallel training; the page prints no gradient, these are reverse-mode
  * derivatives of O = (L (.) (A A^T)) V, A = L (.) Q K^T).
  *
- * hla_backward_workspace_bytes: device workspace bytes hla2_backward needs for
- * (op, dtype, B, H, T, d, dv); 0 when the request is invalid or has no backward
- * kernel (only HLA_OP_HLA2, undecayed, d = dv in {32, 64}).
+ * hla_backward_workspace_bytes: device workspace bytes the backward call of op
+ * needs for (dtype, B, H, T, d, dv); 0 when the request is invalid or has no
+ * backward kernel (HLA_OP_HLA2 and HLA_OP_HLA2_NORM, undecayed, d = dv in {32, 64}).
  *
  * hla2_backward: given the output gradient dout [B][H][T][dv] (fp32, device),
  * writes dq, dk [B][H][T][d] and dv_out [B][H][T][dv] (fp32, device, caller-
@@ -275,6 +275,20 @@ int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, i
 hla_status_t hla2_backward(const void* q, const void* k, const void* v, const float* dout, float* dq,
                            float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                            const float* gamma, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass of the ratio-normalised second order, o = num / (den + eps) (Metodología 1,
+ * Normalización), same arguments as hla2_backward plus eps (as passed to the forward).  The
+ * denominator is the same masked operator on a ones value column, so the gradient is the plain
+ * backward with dout / (den + eps), plus the plain backward on the ones column with the per-row
+ * output gradient -sum_f dout_f num_f / (den + eps)^2 (its dq and dk).  num and den are
+ * recomputed by two plain fp32 forwards.  Workspace: hla_backward_workspace_bytes(
+ * HLA_OP_HLA2_NORM, ...), about 8 B*H*T*d floats more than the plain backward's.
+ */
+hla_status_t hla2_backward_normalized(const void* q, const void* k, const void* v, const float* dout, float* dq,
+                                      float* dk, float* dv_out, int B, int H, int T, int d, int dv,
+                                      hla_dtype_t dtype, const float* gamma, float eps, void* workspace,
+                                      size_t workspace_bytes, void* stream);
 
 /*
  * Tuning knob of the tensor-core path: chunks of 128 tokens per segment (the

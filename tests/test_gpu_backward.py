@@ -81,3 +81,45 @@ def test_backward_matches_autograd_of_the_gpu_forward_at_the_headline_shape():
         num = (f(eps) - f(-eps)) / (2 * eps)
         ana = float(np.sum(dq[b, h] * dirs[0]) + np.sum(dk[b, h] * dirs[1]) + np.sum(dv[b, h] * dirs[2]))
         assert abs(ana - num) <= 1e-3 * max(1.0, abs(num)), (bh, ana, num)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [2, 65, 200])
+def test_normalised_backward_parity(dtype, d, T):
+    """The ratio-normalised output's gradient (hla2_backward_normalized) against
+    ``oracle.backward.hla2n_grads`` (reverse-mode through num / (den + eps), pinned by finite
+    differences), on the normalised workload's input distribution (positive q and k).  A single
+    token is the degenerate case, tested below: there o = v s^2 / (s^2 + eps) with s = q.k does
+    not depend on q or k up to eps."""
+    from oracle.backward import hla2n_grads
+    w = hla_inputs.Workload(f"bwdn_{T}", "hla2n", dtype, 1, 2, T, d, d, "softplus", "unit", seed=T + 3 * d)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    do = torch.randn((1, 2, T, d), generator=torch.Generator("cpu").manual_seed(T), dtype=torch.float32)
+    dev = torch.device("cuda:0")
+    got = hla.hla2_backward(q.to(dev), k.to(dev), v.to(dev), do.to(dev), normalized=True, eps=w.eps)
+    torch.cuda.synchronize()
+    for h in range(2):
+        want = hla2n_grads(q[0, h], k[0, h], v[0, h], do[0, h], w.eps)
+        for name, gt, wt in zip(("dq", "dk", "dv"), got, want):
+            err = oracle.max_row_rel_err(gt[0, h].cpu(), wt)
+            assert err <= TOL[dtype], (name, h, err)
+
+
+def test_normalised_backward_single_token():
+    """T = 1: dv = s^2 / (s^2 + eps) dO exactly; dq and dk are of order eps, the difference of the
+    numerator's and the denominator's terms, each of size 2 |v.dO| |k| / |s|.  The GPU result must
+    be small against those terms (fp32 cancellation leaves a few units of 1e-7 of them)."""
+    w = hla_inputs.Workload("bwdn_1", "hla2n", "f32", 1, 2, 1, 32, 32, "softplus", "unit", seed=5)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    do = torch.randn((1, 2, 1, 32), generator=torch.Generator("cpu").manual_seed(1), dtype=torch.float32)
+    dev = torch.device("cuda:0")
+    dq, dk, dv = (x.cpu().double() for x in hla.hla2_backward(q.to(dev), k.to(dev), v.to(dev), do.to(dev),
+                                                              normalized=True, eps=w.eps))
+    for h in range(2):
+        qh, kh, vh, dh = (x[0, h, 0].double() for x in (q, k, v, do))
+        s = float(qh @ kh)
+        np.testing.assert_allclose(dv[0, h, 0].numpy(), (s * s / (s * s + w.eps) * dh).numpy(), rtol=1e-6)
+        scale = 2 * abs(float(vh @ dh)) / abs(s)
+        assert float(dq[0, h, 0].norm()) <= 1e-5 * scale * float(kh.norm())
+        assert float(dk[0, h, 0].norm()) <= 1e-5 * scale * float(qh.norm())
