@@ -45,11 +45,7 @@ Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H,
     return r;
 }
 
-// The tensor-core AHLA walkers carry no normaliser: ratio-normalised AHLA runs on the CUDA cores.
-bool use_tc(const Request& r) {
-    if (r.op == hla::OP_AHLA && r.norm) return false;
-    return hla::tc::supported(r.op, r.norm, r.bf16, r.d);
-}
+bool use_tc(const Request& r) { return hla::tc::supported(r.op, r.norm, r.bf16, r.d); }
 
 // Ops with no decayed form.
 bool undecayed_only(hla_op_t op) { return op == HLA_OP_HLA2_UNMASKED; }

@@ -29,6 +29,8 @@
 //   second order   output   W = L (.) (Q S0 Q^T + A A*^T), O = Q (S0 C0) + W V + (A K) C0
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "simt.h"
 
@@ -1428,6 +1430,166 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
     for (int e = tid; e < N4; e += NT) gst[e] = st4[e];
 }
 
+// The same step for the second-order family (R-form, decayed, unmasked) with a head's state
+// split by rows over a cluster of STEP_CL CTAs, so that a step's DRAM round trip is spread over
+// STEP_CL times more SMs.  Every row-local part of the update stays in its CTA:
+//   S_i += k_i k,  C_i += q_i v,  z_i = S_i . q  (S symmetric: S q reads row i),  R_i += z_i v;
+// only sums over the rows cross CTAs: the output o_j = sum_i q_i R_ij (second order),
+// sum_i x_i C_ij - q_i G_ij (decayed), sum_i x_i C_ij (unmasked), their denominators, and the
+// decayed form's a = k^T C and k . m taken before its update.  Each such sum is one partial
+// vector per CTA in shared memory, read by every CTA of the cluster through distributed shared
+// memory after a cluster barrier (two buffers, so a second sum never overwrites a partial that
+// another CTA may still be reading).
+constexpr int STEP_CL = 8;    // CTAs per head
+constexpr int STEP_NT = 128;  // threads per CTA: a float4 of each owned matrix row slice per thread
+
+template <int OP, bool NORM, int D, typename TIn>
+__global__ void __cluster_dims__(STEP_CL, 1, 1) __launch_bounds__(STEP_NT)
+    k_step_rows(float* __restrict__ state, const TIn* __restrict__ q, const TIn* __restrict__ k,
+                const TIn* __restrict__ v, const float* __restrict__ gamma, float eps, int H, float* __restrict__ o) {
+    using S = Sum<OP, D>;
+    constexpr int ROWS = D / STEP_CL;        // rows of every matrix this CTA owns
+    constexpr int LPR = D / 4;               // threads per row, one float4 each
+    constexpr int ACT = ROWS * LPR;          // threads that own a float4 of every matrix
+    constexpr int NM = S::NMAT;
+    static_assert(ACT <= STEP_NT && 32 % LPR == 0, "row slice layout");
+    __shared__ float qs[D], ks[D], vs[D], full[D + 1];
+    __shared__ float prod[ROWS][D + 1];      // per-row terms of a sum over rows
+    __shared__ float red[2][D + 1];          // this CTA's partial sums, read by the whole cluster
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    const int rank = static_cast<int>(cl.block_rank());
+    const int bh = blockIdx.x / STEP_CL, tid = threadIdx.x;
+    const int rl = tid / LPR, j0 = 4 * (tid % LPR), i = rank * ROWS + rl;
+    const bool act = tid < ACT, lead = act && (tid % LPR) == 0;
+    float* st = state + (size_t)bh * S::SIZE;
+
+    float4 M[NM];
+    float vec0 = 0.f, vec1 = 0.f;
+    if (act) {
+#pragma unroll
+        for (int m = 0; m < NM; ++m) M[m] = *reinterpret_cast<const float4*>(st + S::mat(m) + i * D + j0);
+        if (S::NVEC > 0 && lead) {
+            vec0 = st[S::vec(0) + i];
+            vec1 = st[S::vec(1) + i];
+        }
+    }
+    if (tid < D) {
+        qs[tid] = to_f32(q[(size_t)bh * D + tid]);
+        ks[tid] = to_f32(k[(size_t)bh * D + tid]);
+        vs[tid] = to_f32(v[(size_t)bh * D + tid]);
+    }
+    __syncthreads();
+
+    // Sum over the cluster's rows of prod[.][0 .. n): this CTA's rows into red[buf], then every
+    // CTA's partial through distributed shared memory into full[0 .. n).
+    auto cluster_sum = [&](int buf, int n) {
+        __syncthreads();
+        for (int t = tid; t < n; t += STEP_NT) {
+            float a = 0.f;
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) a += prod[r][t];
+            red[buf][t] = a;
+        }
+        cl.sync();
+        for (int t = tid; t < n; t += STEP_NT) {
+            float a = 0.f;
+#pragma unroll
+            for (int r = 0; r < STEP_CL; ++r) a += cl.map_shared_rank(&red[buf][0], r)[t];
+            full[t] = a;
+        }
+        __syncthreads();
+    };
+    auto row_dot = [&](const float4& x) {          // row i of a matrix . q, over the row's LPR threads
+        float a = x.x * qs[j0] + x.y * qs[j0 + 1] + x.z * qs[j0 + 2] + x.w * qs[j0 + 3];
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+        return a;
+    };
+    const float4 k4 = make_float4(ks[j0], ks[j0 + 1], ks[j0 + 2], ks[j0 + 3]);
+    const float4 v4 = make_float4(vs[j0], vs[j0 + 1], vs[j0 + 2], vs[j0 + 3]);
+    auto axpy = [](float4& y, float a, const float4& x) {
+        y.x = fmaf(a, x.x, y.x); y.y = fmaf(a, x.y, y.y); y.z = fmaf(a, x.z, y.z); y.w = fmaf(a, x.w, y.w);
+    };
+    auto put = [&](float4 x) {
+        prod[rl][j0] = x.x; prod[rl][j0 + 1] = x.y; prod[rl][j0 + 2] = x.z; prod[rl][j0 + 3] = x.w;
+    };
+    float qi = 0.f, ki = 0.f;
+    if (act) { qi = qs[i]; ki = ks[i]; }
+    int nred = D;                                   // length of the final sum (D + 1 with a denominator)
+
+    if (OP == OP_HLA2) {                            // S=0 C=1 R=2 ; m r
+        float z = 0.f;
+        if (act) {
+            axpy(M[0], ki, k4);
+            axpy(M[1], qi, v4);
+            z = row_dot(M[0]);
+            axpy(M[2], z, v4);
+            vec0 += qi;
+            vec1 += z;
+            put(make_float4(qi * M[2].x, qi * M[2].y, qi * M[2].z, qi * M[2].w));
+            if (NORM && lead) prod[rl][D] = qi * vec1;
+        }
+        nred = NORM ? D + 1 : D;
+    } else if (OP == OP_HLA2U) {                    // S=0 C=1
+        if (act) {
+            axpy(M[0], ki, k4);
+            axpy(M[1], qi, v4);
+            const float x = row_dot(M[0]);
+            put(make_float4(x * M[1].x, x * M[1].y, x * M[1].z, x * M[1].w));
+        }
+    } else {                                        // OP_HLA2D: S=0 C=1 G=2 Khat=3 ; m h ; rho
+        const float g = gamma[bh % H];
+        if (act) {                                  // a = k^T C and k . m, before the update
+            put(make_float4(ki * M[1].x, ki * M[1].y, ki * M[1].z, ki * M[1].w));
+            if (lead) prod[rl][D] = ki * vec0;
+        }
+        cluster_sum(0, D + 1);
+        if (act) {
+            const float4 a4 = make_float4(g * full[j0], g * full[j0 + 1], g * full[j0 + 2], g * full[j0 + 3]);
+            const float sg = g * full[D];
+            M[0] = make_float4(fmaf(g, M[0].x, ki * k4.x), fmaf(g, M[0].y, ki * k4.y), fmaf(g, M[0].z, ki * k4.z),
+                               fmaf(g, M[0].w, ki * k4.w));
+            M[1] = make_float4(fmaf(g, M[1].x, qi * v4.x), fmaf(g, M[1].y, qi * v4.y), fmaf(g, M[1].z, qi * v4.z),
+                               fmaf(g, M[1].w, qi * v4.w));
+            M[2] = make_float4(fmaf(g, M[2].x, ki * a4.x), fmaf(g, M[2].y, ki * a4.y), fmaf(g, M[2].z, ki * a4.z),
+                               fmaf(g, M[2].w, ki * a4.w));
+            M[3].x += ki * k4.x; M[3].y += ki * k4.y; M[3].z += ki * k4.z; M[3].w += ki * k4.w;
+            vec0 = fmaf(g, vec0, qi);
+            vec1 = fmaf(g, vec1, sg * ki);
+            const float x = row_dot(M[0]);
+            put(make_float4(x * M[1].x - qi * M[2].x, x * M[1].y - qi * M[2].y, x * M[1].z - qi * M[2].z,
+                            x * M[1].w - qi * M[2].w));
+            if (NORM && lead) prod[rl][D] = x * vec0 - qi * vec1;
+        }
+        if (rank == 0 && tid == 0) st[S::SCAL] *= g;
+        nred = NORM ? D + 1 : D;
+    }
+    if (act) {
+#pragma unroll
+        for (int m = 0; m < NM; ++m) *reinterpret_cast<float4*>(st + S::mat(m) + i * D + j0) = M[m];
+        if (S::NVEC > 0 && lead) {
+            st[S::vec(0) + i] = vec0;
+            st[S::vec(1) + i] = vec1;
+        }
+    }
+    cluster_sum(1, nred);
+    constexpr int OC = D / STEP_CL;                 // output columns written by this CTA
+    if (tid < OC) {
+        const int j = rank * OC + tid;
+        o[(size_t)bh * D + j] = NORM ? full[j] / (full[D] + eps) : full[j];
+    }
+    cl.sync();                                      // no CTA leaves while another reads its partials
+}
+
+template <int OP, bool NORM, int D, typename TIn>
+static cudaError_t step_rows_launch(float* st_, const void* q, const void* k, const void* v, const float* gamma,
+                                    float eps, int BH, int H, float* o, cudaStream_t st) {
+    k_step_rows<OP, NORM, D, TIn><<<BH * STEP_CL, STEP_NT, 0, st>>>(st_, (const TIn*)q, (const TIn*)k,
+                                                                    (const TIn*)v, gamma, eps, H, o);
+    return cudaGetLastError();
+}
+
 template <int OP, bool NORM, int D, typename TIn>
 static cudaError_t step_launch(float* st_, const void* q, const void* k, const void* v, const float* gamma,
                                float eps, int BH, int H, float* o, cudaStream_t st) {
@@ -1444,18 +1606,18 @@ static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const v
                            const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st) {
     switch (op) {
     case OP_HLA2:
-        return norm ? step_launch<OP_HLA2, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
-                    : step_launch<OP_HLA2, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+        return norm ? step_rows_launch<OP_HLA2, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_rows_launch<OP_HLA2, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA2D:
-        return norm ? step_launch<OP_HLA2D, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
-                    : step_launch<OP_HLA2D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+        return norm ? step_rows_launch<OP_HLA2D, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_rows_launch<OP_HLA2D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_AHLA:
         return norm ? step_launch<OP_AHLA, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
                     : step_launch<OP_AHLA, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA3:
         return norm ? step_launch<OP_HLA3, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
                     : step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
-    case OP_HLA2U: return step_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA2U: return step_rows_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_AHLAD:
     case OP_HLA3D: return cudaErrorNotSupported;   // no streaming form for the decayed AHLA / third order
     }

@@ -19,6 +19,20 @@
 // its columns) and its bf16 copy in shared memory right after the K tile, so one MMA of
 // N = 256 gives [A | Q P0 | Q E0] at once.  96 KB of shared memory and 256 TMEM columns
 // per CTA: two CTAs share an SM, and one's epilogues overlap the other's MMAs.
+//
+// Ratio-normalised AHLA (the denominator is the same operator with V replaced by a ones
+// column: o_t = q_t^T E_t / (q_t^T n_t + eps), n_t = sum_{s<=t} k_s (q_s . mK_s), mK_t =
+// sum_{s<=t} k_s) runs the same walk on [V | 1]:
+//     [Y | y1] = Q [P0 | mK0] + A [V | 1],   [O | den] = Q [E0 | n0] + A [Y | y1],
+//     mK0 += K^T 1,   n0 += K^T y1.
+// The ones column and y1 are column 0 of two extra [tok][64] tiles that sit at a fixed
+// distance from V and from Y, so the N = 80 products read [V | 1] and [Y | y1] as one
+// operand; the state increments (1^T K ; y1^T K) come from one M = 128 product over the two
+// extra tiles stacked (rows 0 and 64 used).  The fp32 vectors mK0, n0 live in the registers
+// of the threads of TMEM lanes 0 and 64, their bf16 copies in row 0 of two 16-row K-major
+// tiles that give Q mK0 and Q n0 from N = 16 products.  The segment summary carries (mK, n)
+// in its two vector slots; two segments combine as (mK_A + mK_B, n_A + n_B + D_B mK_A).
+// The wider accumulators take 512 TMEM columns: one CTA per SM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -44,6 +58,15 @@ constexpr uint32_t AS_A = AS_ST + TILE;  // O staging (output walk); set-up: the
 constexpr uint32_t AS_BAR = AS_A + 2 * TILE;
 constexpr uint32_t AS_TOTAL = AS_BAR + 64;
 constexpr uint32_t ASMEM_BYTES = AS_TOTAL + 1024;   // + alignment slack
+// ratio-normalised only
+constexpr uint32_t AS_ONES = AS_A + 2 * TILE;   // [tok][64], column 0 = 1 (the rest 0)
+constexpr uint32_t AS_Y1 = AS_ONES + TILE;      // [tok][64], column 0 = y1 (the rest 0)
+constexpr uint32_t AS_NM = AS_Y1 + TILE;        // K-major [16][64]: row 0 = mK0^T (the rest 0)
+constexpr uint32_t AS_NN = AS_NM + 2048;        // K-major [16][64]: row 0 = n0^T (the rest 0)
+constexpr uint32_t AS_VEC = AS_NN + 2048;       // set-up: the carried-in mK0, n0 (fp32)
+constexpr uint32_t AS_BAR_N = AS_VEC + 512;
+constexpr uint32_t ASMEM_BYTES_N = AS_BAR_N + 64 + 1024;
+template <bool NORM> constexpr uint32_t asmem_bytes() { return NORM ? ASMEM_BYTES_N : ASMEM_BYTES; }
 
 // TMEM columns (fp32, 128 lanes).
 constexpr uint32_t TA_A = 0;      // A (128); then the masked A as bf16 pairs at columns 0-31
@@ -54,6 +77,11 @@ constexpr uint32_t TA_Y = 128;    // Q P0, then Y (64)
 constexpr uint32_t TA_O = 192;    // output walk: Q E0, then O (64)
 constexpr uint32_t TA_D = 192;    // summary walk: lanes 0-63 D^T of the segment (64)
 constexpr uint32_t TA_COLS = 256;
+// ratio-normalised: A and the increment as above
+constexpr uint32_t TN_Y = 128;    // [Q P0 | Q mK0], then [Y | y1] (80)
+constexpr uint32_t TN_O = 224;    // output walk: [Q E0 | Q n0], then [O | den] (80); summary: lanes 0-63 D^T
+constexpr uint32_t TN_V = 320;    // [1^T K ; y1^T K]: lanes 0 and 64 (64)
+constexpr uint32_t TN_COLS = 512;
 
 enum Mode { SUMMARY = 0, OUTPUT = 1 };
 
@@ -67,13 +95,15 @@ enum Mode { SUMMARY = 0, OUTPUT = 1 };
 //                                                      -> E3: state += increment, to bf16;
 //                                                             O staged over A; next loads
 // The staged O goes to HBM by TMA bulk stores while the next chunk's R1 runs.
-template <int MODE>
-__global__ void __launch_bounds__(ANT, kCtasPerSM)
+template <int MODE, bool NORM>
+__global__ void __launch_bounds__(ANT, NORM ? 1 : kCtasPerSM)
 k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + AS_BAR);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + (NORM ? AS_BAR_N : AS_BAR));
+    constexpr uint32_t TY = NORM ? TN_Y : TA_Y, TO = NORM ? TN_O : TA_O, TD = NORM ? TN_O : TA_D;
+    constexpr uint32_t TCOLS = NORM ? TN_COLS : TA_COLS;
     uint64_t* bar_mma = bar_load + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -113,10 +143,28 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     };
     if (tid == 0) issue_load(0);
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, TA_COLS);
+        ptx::tmem_alloc(tmem_slot, TCOLS);
         ptx::tmem_relinquish();
     }
 
+    // Ratio-normalised: the ones tile (column 0 = 1), the y1 tile and the two vector tiles start
+    // as zeros; only column 0 / row 0 of them is written later.  The threads of TMEM lanes 0
+    // and 64 (vrow) hold half of the fp32 vectors mK0 and n0 each.
+    const bool vrow = NORM && lane == 0 && (quad & 1) == 0;
+    float st2[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) st2[i] = 0.f;
+    float* vecs = reinterpret_cast<float*>(sm + AS_VEC);    // set-up: carried-in mK0 | n0
+    if (NORM) {
+        uint4* z = reinterpret_cast<uint4*>(sm + AS_ONES);
+        for (int e = tid; e < (int)(2 * TILE + 4096) / 16; e += ANT) {
+            // ones tile: 16-byte chunk e is token e / 8, physical chunk e % 8, which holds the
+            // columns of logical chunk (e % 8) ^ (token % 8); logical chunk 0 starts at column 0
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+            if (e < (int)TILE / 16 && ((e ^ (e >> 3)) & 7) == 0) u.x = 0x3F80u;   // bf16 1.0
+            z[e] = u;
+        }
+    }
     // This thread's part of the fp32 state: row `row` of [P^T ; E^T], columns half*32 .. +31.
     float st[32];
     if (MODE == OUTPUT) {
@@ -144,8 +192,13 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                 for (int b = 0; b < 4; ++b) racc[a][b] = 0.f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) sacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            float macc = 0.f, nacc = 0.f;                      // normalised: mK0, n0 (column tid)
             for (int l = 0; l < n; ++l) {
                 const float* sl = sb + (size_t)l * S::size;
+                if (NORM && tid < D) {
+                    macc += sl[S::vec(0) + tid];
+                    nacc += sl[S::vec(1) + tid];
+                }
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
                     const float4 x = *reinterpret_cast<const float4*>(sl + S::mat(2) + (r + a) * D + c);
@@ -167,6 +220,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     reinterpret_cast<float4*>(Sm)[f] = reinterpret_cast<const float4*>(smp + S::mat(0))[f];
                 }
                 __syncthreads();
+                if (NORM && tid < D) {                         // n0 += D_suf(m+1) mK_m
+                    const float* mk = smp + S::vec(0);
+                    for (int k = 0; k < D; ++k) nacc = fmaf(mk[k], Cs[k * D + tid], nacc);
+                }
 #pragma unroll 8
                 for (int k = 0; k < D; ++k) {
                     const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
@@ -180,6 +237,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     }
                 }
                 __syncthreads();
+            }
+            if (NORM && tid < D) {
+                vecs[tid] = macc;
+                vecs[D + tid] = nacc;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -196,6 +257,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         } else {
             const float4* p4 = reinterpret_cast<const float4*>(slot + S::mat(0));
             const float4* e4 = reinterpret_cast<const float4*>(slot + S::mat(2));
+            if (NORM && tid < D) {
+                vecs[tid] = slot[S::vec(0) + tid];
+                vecs[D + tid] = slot[S::vec(1) + tid];
+            }
             float4 xp[4], xe[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -217,6 +282,11 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             const float4 x = src[(half * 8 + j) ^ (r & 7)];
             st[4 * j] = x.x; st[4 * j + 1] = x.y; st[4 * j + 2] = x.z; st[4 * j + 3] = x.w;
         }
+        if (vrow) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) st2[i] = vecs[(quad >> 1) * D + half * 32 + i];
+            st_row32(sm + (quad ? AS_NN : AS_NM), 0, half * 32, st2);
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[i] = 0.f;
@@ -230,8 +300,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
 
     const uint32_t sbase = ptx::smem_u32(sm);
-    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, MODE == OUTPUT ? 256 : 192, false, false);
-    constexpr uint32_t I_N64_KM = ptx::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, (MODE == OUTPUT && !NORM) ? 256 : 192, false, false);
+    constexpr uint32_t I_N64_KK = ptx::idesc_bf16(128, 64, false, false);
+    constexpr uint32_t I_N16_KK = ptx::idesc_bf16(128, 16, false, false);
+    constexpr uint32_t I_NV_KM = ptx::idesc_bf16(128, NORM ? 80 : 64, false, true);   // [V | 1], [Y | y1]
     constexpr uint32_t I_N64_MM = ptx::idesc_bf16(128, 64, true, true);
     auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };                         // +32 B
     auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };                       // +2048 B
@@ -242,26 +314,39 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     auto issue_r1 = [&]() {
         const uint64_t dQ = kdesc(sbase + AS_Q, 0), dKS = kdesc(sbase + AS_K, 0);
         for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TA_A, k1(dQ, s), k1(dKS, s), I_R1, s > 0);
+        if (NORM) {                          // Q mK0 -> y1 column; output: Q E0, Q n0 -> den column
+            const uint64_t dNM = kdesc(sbase + AS_NM, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TY + 64, k1(dQ, s), k1(dNM, s), I_N16_KK, s > 0);
+            if (MODE == OUTPUT) {
+                const uint64_t dE = kdesc(sbase + AS_ST + 64 * 128, 0), dNN = kdesc(sbase + AS_NN, 0);
+                for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TO, k1(dQ, s), k1(dE, s), I_N64_KK, s > 0);
+                for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TO + 64, k1(dQ, s), k1(dNN, s), I_N16_KK, s > 0);
+            }
+        }
     };
     // masked A as bf16 pairs: K-step s (tokens 16 s .. 16 s + 15)
     auto a_pairs = [&](int s) { return tmem + TA_A + (s < 4 ? 8 * s : 96 + 8 * (s - 4)); };
     auto issue_r2 = [&](int n) {
-        const uint64_t dVm = mdesc(sbase + AS_V, TILE, 0);
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TA_Y, a_pairs(s), mn(dVm, s), I_N64_KM, 1);
+        const uint64_t dVm = mdesc(sbase + AS_V, NORM ? AS_ONES - AS_V : TILE, 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TY, a_pairs(s), mn(dVm, s), I_NV_KM, 1);
         if (MODE == SUMMARY) {   // lanes 0-63: D^T += Q^T K (lanes 64-127 take K^T K, unused)
             const uint64_t dQK = mdesc(sbase + AS_Q, AS_K - AS_Q, 0), dKm = mdesc(sbase + AS_K, TILE, 0);
             for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + TA_D, mn(dQK, s), mn(dKm, s), I_N64_MM, (n > 0 || s > 0) ? 1u : 0u);
+                ptx::umma_bf16(tmem + TD, mn(dQK, s), mn(dKm, s), I_N64_MM, (n > 0 || s > 0) ? 1u : 0u);
         }
     };
     auto issue_r3 = [&]() {
         const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
         if (MODE == OUTPUT) {
-            const uint64_t dYm = mdesc(sbase + AS_Q, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TA_O, a_pairs(s), mn(dYm, s), I_N64_KM, 1);
+            const uint64_t dYm = mdesc(sbase + AS_Q, NORM ? AS_Y1 - AS_Q : TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TO, a_pairs(s), mn(dYm, s), I_NV_KM, 1);
         }
         const uint64_t dVY = mdesc(sbase + AS_V, AS_Q - AS_V, 0);
         for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TA_INC, mn(dVY, s), mn(dKm, s), I_N64_MM, s > 0);
+        if (NORM) {                          // [1^T K ; y1^T K] at lanes 0 and 64
+            const uint64_t dOY = mdesc(sbase + AS_ONES, AS_Y1 - AS_ONES, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TN_V, mn(dOY, s), mn(dKm, s), I_N64_MM, s > 0);
+        }
     };
 
     uint32_t mma_phase = 0;
@@ -330,8 +415,13 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // E2: Y -> AS_Q (the Q tile is no longer read)
     auto epi2 = [&]() {
         float v[32];
-        ptx::tmem_ld32(tmem + lane_base + TA_Y + half * 32, v);
+        ptx::tmem_ld32(tmem + lane_base + TY + half * 32, v);
         st_row32(sm + AS_Q, row, half * 32, v);
+        if (NORM && half == 0) {             // y1 -> column 0 of the y1 tile
+            float w[16];
+            ptx::tmem_ld16(tmem + lane_base + TY + 64, w);
+            *reinterpret_cast<bf16*>(sm + AS_Y1 + row * 128 + ((row & 7) << 4)) = __float2bfloat16_rn(w[0]);
+        }
     };
     // E3: state += increment, its bf16 copy -> AS_ST; O of the chunk (fp32) staged over the
     // A tile as two [128 rows][32 cols] boxes in the 128B-swizzled TMA layout
@@ -341,8 +431,23 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[i] += v[i];
         if (MODE == OUTPUT || row < 64) st_row32(sm + AS_ST, row, half * 32, st);
+        if (NORM && (quad & 1) == 0) {       // lanes 0 and 64: mK0 += K^T 1, n0 += K^T y1
+            ptx::tmem_ld32(tmem + lane_base + TN_V + half * 32, v);
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) st2[i] += v[i];
+                if (quad == 0 || MODE == OUTPUT) st_row32(sm + (quad ? AS_NN : AS_NM), 0, half * 32, st2);
+            }
+        }
         if (MODE == OUTPUT) {
-            ptx::tmem_ld32(tmem + lane_base + TA_O + half * 32, v);
+            ptx::tmem_ld32(tmem + lane_base + TO + half * 32, v);
+            if (NORM) {
+                float w[16];
+                ptx::tmem_ld16(tmem + lane_base + TO + 64, w);
+                const float scale = 1.f / (w[0] + p.eps);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= scale;
+            }
             float4* box = reinterpret_cast<float4*>(sm + AS_A + half * (C * 128) + row * 128);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -398,7 +503,7 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if (quad < 2) {
             float v[32];
             put_row(0, row, st);                                   // P^T
-            ptx::tmem_ld32(tmem + lane_base + TA_D + half * 32, v);
+            ptx::tmem_ld32(tmem + lane_base + TD + half * 32, v);
             put_row(1, row, v);                                    // D^T
         } else {
             put_row(2, row - 64, st);                              // E^T
@@ -410,7 +515,12 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             const int rr = (f >> 4) & (D - 1);
             out4[f] = st4[(f & ~15) | ((f & 15) ^ (rr & 7))];
         }
-        for (int f = 3 * D * D / 4 + tid; f < S::size / 4; f += ANT) out4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int f = (NORM ? S::vec(2) : S::vec(0)) / 4 + tid; f < S::size / 4; f += ANT)
+            out4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (vrow) {                          // (mK, n) of the segment
+#pragma unroll
+            for (int i = 0; i < 32; ++i) slot[S::vec(quad >> 1) + half * 32 + i] = st2[i];
+        }
     }
     if (MODE == OUTPUT && tid == 0) ptx::bulk_wait_all();  // O stores done before the CTA exits
     if (!ok && tid == 0) {
@@ -422,28 +532,29 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) ptx::tmem_dealloc(tmem, TA_COLS);
+    if (warp == 1) ptx::tmem_dealloc(tmem, TCOLS);
 }
 
 }  // namespace
 
-int ahla_ctas_per_sm() { return kCtasPerSM; }
+int ahla_ctas_per_sm(bool norm) { return norm ? 1 : kCtasPerSM; }
 
-size_t ahla_workspace_bytes(int BH, int T, int seg_chunks) {
-    const Plan pl = plan(BH, T, kCtasPerSM * kSMs, seg_chunks);
+size_t ahla_workspace_bytes(int BH, int T, int seg_chunks, bool norm) {
+    const Plan pl = plan(BH, T, ahla_ctas_per_sm(norm) * kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
-                         int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
+template <bool NORM>
+static cudaError_t ahla_run(const void* q, const void* k, const void* v, float* o, int BH, int T, float eps,
+                            void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
-    const Plan pl = plan(BH, T, kCtasPerSM * kSMs, seg_chunks);
+    const Plan pl = plan(BH, T, ahla_ctas_per_sm(NORM) * kSMs, seg_chunks);
     Params prm;                              // the output walk
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
-    prm.eps = 0.f; prm.norm = 0;
+    prm.eps = eps; prm.norm = NORM ? 1 : 0;
     prm.sums = static_cast<float*>(ws);
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
@@ -451,36 +562,42 @@ cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, 
     prm.fold = pl.NSf + 1 <= PH_MAX ? 1 : 0;  // few slots: each output CTA folds its own prefix
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
     sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
+    constexpr int SMEM = (int)asmem_bytes<NORM>();
     cudaError_t e;
-    if ((e = set_smem(k_ahla_walk<SUMMARY>, ASMEM_BYTES)) != cudaSuccess)
-        return e;
-    if ((e = set_smem(k_ahla_walk<OUTPUT>, ASMEM_BYTES)) != cudaSuccess)
-        return e;
+    if ((e = set_smem(k_ahla_walk<SUMMARY, NORM>, SMEM)) != cudaSuccess) return e;
+    if ((e = set_smem(k_ahla_walk<OUTPUT, NORM>, SMEM)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_ahla_walk<SUMMARY><<<dim3(pl.NSp, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
+    k_ahla_walk<SUMMARY, NORM><<<dim3(pl.NSp, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
+    if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st, NORM)) != cudaSuccess)
+        return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
     if (prm.fold) {
         // a programmatic dependent of the summary walk (see the second-order forward)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(pl.NS, BH);
         cfg.blockDim = dim3(ANT);
-        cfg.dynamicSmemBytes = ASMEM_BYTES;
+        cfg.dynamicSmemBytes = SMEM;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&cfg, k_ahla_walk<OUTPUT>, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
+        if ((e = cudaLaunchKernelEx(&cfg, k_ahla_walk<OUTPUT, NORM>, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
     } else {
-        k_ahla_walk<OUTPUT><<<dim3(pl.NS, BH), ANT, ASMEM_BYTES, st>>>(mq, mk, mv, mo, prm);
+        k_ahla_walk<OUTPUT, NORM><<<dim3(pl.NS, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, prm);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
+}
+
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, bool norm, float eps,
+                         void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
+    if (norm) return ahla_run<true>(q, k, v, o, BH, T, eps, ws, status, st, ev, seg_chunks);
+    return ahla_run<false>(q, k, v, o, BH, T, 0.f, ws, status, st, ev, seg_chunks);
 }
 
 }  // namespace tc

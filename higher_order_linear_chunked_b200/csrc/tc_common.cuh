@@ -133,7 +133,11 @@ constexpr int PH_MAX = 9;
 
 // Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for
 // every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
-cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st);
+// left_vec: the vector of the second slot is a row on the left of the first factor's
+// partner (ratio-normalised AHLA: n_AB = n_A + n_B + D_B mK_A, D^T in the C place) instead of
+// the second order's r_AB = r_A + r_B + S_A m_B.
+cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st,
+                          bool left_vec = false);
 
 // The decayed second-order forward, chunk-parallel (tc_decay.cu).
 size_t decay_workspace_bytes(int BH, int T);
@@ -141,11 +145,11 @@ int decay_kernel_launches();
 cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
                           int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
 
-// The AHLA forward on the tcgen05 walkers (tc_ahla.cu).
-size_t ahla_workspace_bytes(int BH, int T, int seg_chunks);
-int ahla_ctas_per_sm();
-cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, void* ws,
-                         int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks);
+// The AHLA forward on the tcgen05 walkers, plain or ratio-normalised (tc_ahla.cu).
+size_t ahla_workspace_bytes(int BH, int T, int seg_chunks, bool norm);
+int ahla_ctas_per_sm(bool norm);
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, bool norm, float eps,
+                         void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks);
 
 }  // namespace tc
 }  // namespace hla

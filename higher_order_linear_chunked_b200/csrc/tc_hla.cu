@@ -691,11 +691,11 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
 constexpr int PX_NT = 256;
 
 __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict__ sums, float* __restrict__ pre,
-                                                        int NSp) {
+                                                        int NSp, int left_vec) {
     using S = simt_layout;
     __shared__ __align__(16) float S0s[D * (D + 4)];   // padded rows: conflict-free column walks
     __shared__ __align__(16) float Cs[D * D];
-    __shared__ float ms[D];
+    __shared__ float ms[D], m0s[D];
     const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const float* sb = sums + (size_t)bh * NSp * S::size;
     float* out = pre + ((size_t)bh * NSp + l) * S::size;
@@ -730,6 +730,7 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict_
         }
         if (tid < D) {
             ms[tid] = mv;
+            m0s[tid] = m0;
             out[S::vec(0) + tid] = m0;                                       // m0(l)
         }
     }
@@ -761,8 +762,11 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict_
             *reinterpret_cast<float4*>(out + S::mat(2) + (r + a) * D + c) = make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
         if (tid < D) {
             float yv = sb[(size_t)l * S::size + S::vec(1) + tid];
-            for (int k = 0; k < D; ++k) yv = fmaf(S0s[tid * (D + 4) + k], ms[k], yv);
-            out[S::vec(1) + tid] = yv;                                       // y_l
+            if (left_vec)                                                    // y_l = n_l + m0(l)^T C_l
+                for (int k = 0; k < D; ++k) yv = fmaf(m0s[k], Cs[k * D + tid], yv);
+            else                                                             // y_l = r_l + S0(l) m_l
+                for (int k = 0; k < D; ++k) yv = fmaf(S0s[tid * (D + 4) + k], ms[k], yv);
+            out[S::vec(1) + tid] = yv;
         }
     }
 }
@@ -958,8 +962,8 @@ Plan plan(int BH, int T, int slots, int seg_chunks) {
     return pl;
 }
 
-cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st) {
-    k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp);
+cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st, bool left_vec) {
+    k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp, left_vec ? 1 : 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(pre, NS, NSp);
@@ -1027,25 +1031,25 @@ bool supported(int op, bool norm, bool bf16, int d) {
     return op == OP_HLA2 || op == OP_AHLA || (op == OP_HLA2D && !norm);
 }
 
-size_t workspace_bytes(int op, bool /*norm*/, int BH, int T, int seg_chunks) {
-    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T, seg_chunks);
+size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks) {
+    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T, seg_chunks, norm);
     if (op == OP_HLA2D) return decay_workspace_bytes(BH, T);
     const Plan pl = plan(BH, T, kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-int kernel_launches(int op, bool /*norm*/, int BH, int T, int seg_chunks) {
+int kernel_launches(int op, bool norm, int BH, int T, int seg_chunks) {
     if (op == OP_HLA2D) return decay_kernel_launches();
     // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
     // two launches), output walk
-    const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm() * kSMs : kSMs, seg_chunks);
+    const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm(norm) * kSMs : kSMs, seg_chunks);
     return pl.NSf + 1 > PH_MAX ? 4 : 2;     // else the output walker folds the prefix itself
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
                     float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
                     int seg_chunks) {
-    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, ws, status, st, ev, seg_chunks);
+    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, norm, eps, ws, status, st, ev, seg_chunks);
     if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;

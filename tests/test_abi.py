@@ -72,8 +72,10 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     use = lambda op, dt, dec, T=4096, d=64: lib.hla_uses_tensor_cores(op, dt, dec, 4, 16, T, d, d)
     launches = lambda op, dt, dec, T=4096, d=64: lib.hla_kernel_launches(op, dt, dec, 4, 16, T, d, d)
     bf16, f32 = hla.HLA_BF16, hla.HLA_F32
-    # bf16, d = 64: second order (plain, normalised, decayed) and AHLA run on the tensor cores
-    for op, dec in ((hla.OP_HLA2, 0), (hla.OP_HLA2_NORM, 0), (hla.OP_HLA2, 1), (hla.OP_AHLA, 0)):
+    # bf16, d = 64: second order (plain, normalised, decayed) and AHLA (plain, normalised) run on
+    # the tensor cores
+    for op, dec in ((hla.OP_HLA2, 0), (hla.OP_HLA2_NORM, 0), (hla.OP_HLA2, 1), (hla.OP_AHLA, 0),
+                    (hla.OP_AHLA_NORM, 0)):
         assert use(op, bf16, dec) == 1, (op, dec)
     # the rest on CUDA cores: fp32 inputs, d = 32, third order, normalised with decay
     assert use(hla.OP_HLA2, f32, 0) == 0
@@ -85,13 +87,19 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     # chunk summaries, three prefix kernels and the output kernel
     assert launches(hla.OP_HLA2_NORM, bf16, 0) == 2   # the output walker folds the prefix
     assert launches(hla.OP_AHLA, bf16, 0) == 2
+    assert launches(hla.OP_AHLA_NORM, bf16, 0) == 2
+    # the normalised AHLA walker runs one CTA per SM (512 TMEM columns): its segment plan, and
+    # so its workspace, differs from the plain walker's (two per SM) at the same shape
+    ws_tc = lambda op, B, H, T: lib.hla_workspace_bytes(op, bf16, 0, B, H, T, 64, 64)
+    assert ws_tc(hla.OP_AHLA_NORM, 4, 16, 8192) > 0 and ws_tc(hla.OP_AHLA, 4, 16, 8192) > 0
+    assert lib.hla_kernel_launches(hla.OP_AHLA_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 4   # many slots
     assert lib.hla_kernel_launches(hla.OP_HLA2_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 4   # many slots
     assert launches(hla.OP_HLA2, bf16, 1) == 5
     # CUDA-core path: chunk kernel, one scan launch (a per-head fold) and the output kernel;
     # the third order takes the factored prefix (three launches); its decayed form keeps the
     # per-level Blelloch tree: 64 chunks of 64 tokens, 2 x 6 levels
     assert launches(hla.OP_HLA2, f32, 0) == 3
-    assert launches(hla.OP_AHLA_NORM, bf16, 0) == 3
+    assert launches(hla.OP_AHLA_NORM, f32, 0) == 3
     assert launches(hla.OP_HLA2_UNMASKED, bf16, 0) == 3
     assert launches(hla.OP_HLA3, f32, 0, d=32) == 2 + 3      # the factored third-order prefix
     assert launches(hla.OP_HLA3, f32, 0) == 2 + 3
@@ -207,11 +215,13 @@ def test_streaming_state_sizes_and_argument_errors(lib):
 
 
 def test_normalised_ahla_hla3_routing_and_errors(lib):
-    """Ratio-normalised AHLA / third order: CUDA-core kernels (the tensor-core AHLA walker
-    carries no normaliser), a decayed form on the CUDA cores, the plain op's workspace."""
+    """Ratio-normalised AHLA / third order: the tensor-core walker for bf16 AHLA at d = 64 (a
+    ones column beside V), CUDA-core kernels otherwise (the third order, fp32, d = 32, decay)
+    with the plain op's workspace."""
     vp, f = ctypes.c_void_p, ctypes.c_float
+    assert lib.hla_uses_tensor_cores(hla.OP_AHLA_NORM, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 1
+    assert lib.hla_uses_tensor_cores(hla.OP_HLA3_NORM, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
     for op, plain in ((hla.OP_AHLA_NORM, hla.OP_AHLA), (hla.OP_HLA3_NORM, hla.OP_HLA3)):
-        assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
         assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) > 0            # decayed form
         assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0
         assert lib.hla_workspace_bytes(op, hla.HLA_F32, 0, 2, 8, 4096, 32, 32) == \
