@@ -552,6 +552,9 @@ def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
     times = []
     for t in range(steps):
         flush.zero_()
+        # a spin kernel keeps the stream busy while the host enqueues the step (the Python call
+        # takes longer than the kernel), so the events time the device, not the host
+        torch.cuda._sleep(200000)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         hla.step(w.op, st, *toks[t], gamma=gd, eps=w.eps, out=o)
@@ -559,12 +562,21 @@ def decode_measure(w, qd, kd, vd, gd, flush, steps, peaks, peak_kind):
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     step_ms = statistics.mean(times)
+    host = []                                                       # host time of one call
+    for t in range(steps):
+        h0 = time.perf_counter()
+        hla.step(w.op, st, *toks[t], gamma=gd, eps=w.eps, out=o)
+        host.append(time.perf_counter() - h0)
+        torch.cuda.synchronize()
     esz = qd.element_size()
     nbytes = B * H * (2 * st.shape[-1] * 4 + 3 * d * esz + vd.shape[-1] * 4)   # state in and out, q k v, o
     gbs = nbytes / (step_ms / 1e3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     return {"prefill_ms": prefill_ms, "prefill_note": "second call (the first is a warm-up), L2 flushed before it",
             "prefill_tokens": B * H * T, "steps": steps, "us_per_step": step_ms * 1e3,
+            "host_us_per_call": statistics.median(host) * 1e6,
+            "timing": "events around each step with the stream kept busy before it (device time, the "
+                      "event pair included); the host time of the Python call is reported apart",
             "tokens_per_s": B * H / (step_ms / 1e3), "gpu_launches_per_step": 1,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "bytes_per_step": nbytes, "peak_source": f"HBM copy ({peak_kind})"},

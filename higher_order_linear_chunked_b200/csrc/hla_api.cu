@@ -45,7 +45,9 @@ Request make_request(hla_op_t op, bool decayed, hla_dtype_t dtype, int B, int H,
     return r;
 }
 
-bool use_tc(const Request& r) { return hla::tc::supported(r.op, r.norm, r.bf16, r.d); }
+bool use_tc(const Request& r) {
+    return hla::tc::supported(r.op, r.norm, r.bf16, r.d) && hla::tc::fits(r.op, r.norm, r.B * r.H, r.T, r.seg);
+}
 
 // Ops with no decayed form.
 bool undecayed_only(hla_op_t op) { return op == HLA_OP_HLA2_UNMASKED; }

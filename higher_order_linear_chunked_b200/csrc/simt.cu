@@ -1437,9 +1437,9 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
 // only sums over the rows cross CTAs: the output o_j = sum_i q_i R_ij (second order),
 // sum_i x_i C_ij - q_i G_ij (decayed), sum_i x_i C_ij (unmasked), their denominators, and the
 // decayed form's a = k^T C and k . m taken before its update.  Each such sum is one partial
-// vector per CTA in shared memory, read by every CTA of the cluster through distributed shared
-// memory after a cluster barrier (two buffers, so a second sum never overwrites a partial that
-// another CTA may still be reading).
+// vector per CTA, which the CTA writes into slot `rank` of every CTA's shared memory (distributed
+// shared memory stores); after one cluster barrier each CTA adds its slots locally.  No CTA
+// touches another's shared memory after the last barrier, so none waits for the others to leave.
 constexpr int STEP_CL = 8;    // CTAs per head
 constexpr int STEP_NT = 128;  // threads per CTA: a float4 of each owned matrix row slice per thread
 
@@ -1455,7 +1455,7 @@ __global__ void __cluster_dims__(STEP_CL, 1, 1) __launch_bounds__(STEP_NT)
     static_assert(ACT <= STEP_NT && 32 % LPR == 0, "row slice layout");
     __shared__ float qs[D], ks[D], vs[D], full[D + 1];
     __shared__ float prod[ROWS][D + 1];      // per-row terms of a sum over rows
-    __shared__ float red[2][D + 1];          // this CTA's partial sums, read by the whole cluster
+    __shared__ float red[2][STEP_CL][D + 1]; // every CTA's partial sums, two rounds
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     const int rank = static_cast<int>(cl.block_rank());
@@ -1481,21 +1481,22 @@ __global__ void __cluster_dims__(STEP_CL, 1, 1) __launch_bounds__(STEP_NT)
     }
     __syncthreads();
 
-    // Sum over the cluster's rows of prod[.][0 .. n): this CTA's rows into red[buf], then every
-    // CTA's partial through distributed shared memory into full[0 .. n).
+    // Sum over the cluster's rows of prod[.][0 .. n): this CTA's rows, stored into slot `rank` of
+    // red[buf] in every CTA of the cluster; one cluster barrier; the slots added into full[0 .. n).
     auto cluster_sum = [&](int buf, int n) {
         __syncthreads();
         for (int t = tid; t < n; t += STEP_NT) {
             float a = 0.f;
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) a += prod[r][t];
-            red[buf][t] = a;
+#pragma unroll
+            for (int r = 0; r < STEP_CL; ++r) cl.map_shared_rank(&red[buf][rank][0], r)[t] = a;
         }
         cl.sync();
         for (int t = tid; t < n; t += STEP_NT) {
             float a = 0.f;
 #pragma unroll
-            for (int r = 0; r < STEP_CL; ++r) a += cl.map_shared_rank(&red[buf][0], r)[t];
+            for (int r = 0; r < STEP_CL; ++r) a += red[buf][r][t];
             full[t] = a;
         }
         __syncthreads();
@@ -1579,7 +1580,6 @@ __global__ void __cluster_dims__(STEP_CL, 1, 1) __launch_bounds__(STEP_NT)
         const int j = rank * OC + tid;
         o[(size_t)bh * D + j] = NORM ? full[j] / (full[D] + eps) : full[j];
     }
-    cl.sync();                                      // no CTA leaves while another reads its partials
 }
 
 template <int OP, bool NORM, int D, typename TIn>

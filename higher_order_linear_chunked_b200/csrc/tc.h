@@ -8,6 +8,8 @@ namespace tc {
 
 // true when (internal op, normalised, bf16, d) runs on the tcgen05 kernels
 bool supported(int op, bool norm, bool bf16, int d);
+// and for this shape: the decayed AHLA walk needs its prefix folded into the output walker
+bool fits(int op, bool norm, int BH, int T, int seg_chunks);
 // process-wide default segment length (chunks); 0 = automatic; false if invalid
 bool set_segment_chunks(int chunks);
 // the default, read once by every request (the size query and the forward each take their own

@@ -33,6 +33,16 @@
 // tiles that give Q mK0 and Q n0 from N = 16 products.  The segment summary carries (mK, n)
 // in its two vector slots; two segments combine as (mK_A + mK_B, n_A + n_B + D_B mK_A).
 // The wider accumulators take 512 TMEM columns: one CTA per SM.
+//
+// With per-head decay (every state multiplied by gamma before each token's update) the chunk
+// algebra takes the decayed masked scores At[tau][j] = g^(tau-j) A[tau][j], the row weights
+// Gam = diag(g^(tau+1)) and Lam = diag(g^(len-1-tau)), and rho = g^len:
+//     Y = Gam Q P0 + At V,   O = Gam Q E0 + At Y,   P0 = rho P0 + K^T Lam V,   E0 = rho E0 + K^T Lam Y
+// (the normaliser's vectors likewise).  The weights are applied in fp32 before each operand's
+// one rounding to bf16: At in the A epilogue, Gam on the fp32 accumulators Q P0 and Q E0 in
+// TMEM, Lam on a copy of K that takes the state tile's place while the state is not read.
+// A segment summary carries rho = g^length in its scalar slot; the fold weights summary l
+// by the product of the later summaries' rho (the decayed combine, unrolled).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -95,7 +105,7 @@ enum Mode { SUMMARY = 0, OUTPUT = 1 };
 //                                                      -> E3: state += increment, to bf16;
 //                                                             O staged over A; next loads
 // The staged O goes to HBM by TMA bulk stores while the next chunk's R1 runs.
-template <int MODE, bool NORM>
+template <int MODE, bool NORM, bool DECAY>
 __global__ void __launch_bounds__(ANT, NORM ? 1 : kCtasPerSM)
 k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, Params p) {
@@ -116,13 +126,17 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // Programmatic dependent launch: the output walk may be scheduled once every summary CTA
     // has started; its CTAs that fold summaries wait for this grid's completion first.
     if (MODE == SUMMARY && tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (seg >= p.NS) {                                    // padding slots: identity (zeros)
+    if (seg >= p.NS) {                                    // padding slots: identity (zeros, rho = 1)
         if (MODE == SUMMARY) {
             float4* s4 = reinterpret_cast<float4*>(slot);
-            for (int e = tid; e < S::size / 4; e += ANT) s4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = tid; e < S::size / 4; e += ANT)
+                s4[e] = make_float4(DECAY && e == S::vec(2) / 4 ? 1.f : 0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
+    // decay: g = gamma of the head, lg = log2(g) (g = 1: every weight is 1)
+    const float g = DECAY ? p.gamma[bh % p.H] : 1.f;
+    const float lg = DECAY ? log2f(g) : 0.f;
     const int chunk0 = seg * p.NCH;
     const int nch = min(p.NCH, (p.T + C - 1) / C - chunk0);
 
@@ -193,23 +207,29 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 #pragma unroll
             for (int i = 0; i < 4; ++i) sacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             float macc = 0.f, nacc = 0.f;                      // normalised: mK0, n0 (column tid)
-            for (int l = 0; l < n; ++l) {
+            // decay: summary l enters with weight w_l = prod_{l < m < n} rho_m
+            float wl = 1.f;
+            for (int l = n - 1; l >= 0; --l) {
                 const float* sl = sb + (size_t)l * S::size;
                 if (NORM && tid < D) {
-                    macc += sl[S::vec(0) + tid];
-                    nacc += sl[S::vec(1) + tid];
+                    macc = fmaf(wl, sl[S::vec(0) + tid], macc);
+                    nacc = fmaf(wl, sl[S::vec(1) + tid], nacc);
                 }
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
                     const float4 x = *reinterpret_cast<const float4*>(sl + S::mat(2) + (r + a) * D + c);
-                    racc[a][0] += x.x; racc[a][1] += x.y; racc[a][2] += x.z; racc[a][3] += x.w;
+                    racc[a][0] = fmaf(wl, x.x, racc[a][0]); racc[a][1] = fmaf(wl, x.y, racc[a][1]);
+                    racc[a][2] = fmaf(wl, x.z, racc[a][2]); racc[a][3] = fmaf(wl, x.w, racc[a][3]);
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float4 x = reinterpret_cast<const float4*>(sl + S::mat(0))[tid + ANT * i];
-                    sacc[i] = make_float4(sacc[i].x + x.x, sacc[i].y + x.y, sacc[i].z + x.z, sacc[i].w + x.w);
+                    sacc[i] = make_float4(fmaf(wl, x.x, sacc[i].x), fmaf(wl, x.y, sacc[i].y), fmaf(wl, x.z, sacc[i].z),
+                                          fmaf(wl, x.w, sacc[i].w));
                 }
+                if (DECAY) wl *= sl[S::vec(2)];
             }
+            float wm = DECAY && n >= 1 ? sb[(size_t)(n - 1) * S::size + S::vec(2)] : 1.f;   // w_{n-2}
             for (int m = n - 2; m >= 0; --m) {
                 const float* cl = sb + (size_t)(m + 1) * S::size;
                 const float* smp = sb + (size_t)m * S::size;
@@ -217,13 +237,18 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
                     const float4 x = reinterpret_cast<const float4*>(cl + S::mat(1))[f];
                     const float4 o = m == n - 2 ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<float4*>(Cs)[f];
                     reinterpret_cast<float4*>(Cs)[f] = make_float4(o.x + x.x, o.y + x.y, o.z + x.z, o.w + x.w);
-                    reinterpret_cast<float4*>(Sm)[f] = reinterpret_cast<const float4*>(smp + S::mat(0))[f];
+                    float4 pm = reinterpret_cast<const float4*>(smp + S::mat(0))[f];
+                    if (DECAY) pm = make_float4(wm * pm.x, wm * pm.y, wm * pm.z, wm * pm.w);
+                    reinterpret_cast<float4*>(Sm)[f] = pm;     // w_m P^T_m
                 }
                 __syncthreads();
-                if (NORM && tid < D) {                         // n0 += D_suf(m+1) mK_m
+                if (NORM && tid < D) {                         // n0 += w_m D_suf(m+1) mK_m
                     const float* mk = smp + S::vec(0);
-                    for (int k = 0; k < D; ++k) nacc = fmaf(mk[k], Cs[k * D + tid], nacc);
+                    float t = 0.f;
+                    for (int k = 0; k < D; ++k) t = fmaf(mk[k], Cs[k * D + tid], t);
+                    nacc = fmaf(wm, t, nacc);
                 }
+                if (DECAY) wm *= smp[S::vec(2)];
 #pragma unroll 8
                 for (int k = 0; k < D; ++k) {
                     const float4 cv = *reinterpret_cast<const float4*>(Cs + k * D + c);
@@ -336,7 +361,8 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
     };
     auto issue_r3 = [&]() {
-        const uint64_t dKm = mdesc(sbase + AS_K, TILE, 0);
+        // the increments' B operand: K, or with decay Lam K (staged over the state tile)
+        const uint64_t dKm = mdesc(sbase + (DECAY ? AS_ST : AS_K), TILE, 0);
         if (MODE == OUTPUT) {
             const uint64_t dYm = mdesc(sbase + AS_Q, NORM ? AS_Y1 - AS_Q : TILE, 0);
             for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + TO, a_pairs(s), mn(dYm, s), I_NV_KM, 1);
@@ -394,21 +420,95 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // blocks b0 = 2 half and b0 + 1 (columns 64 half .. +63) and writes their pairs to columns
     // 96 half .. +31, which it has read itself.  Blocks above the diagonal (b > quad) become
     // zeros (the A of every chunk overwrites them).
-    auto epi1 = [&]() {
+    // decay weights g^(tau - j) on this lane's token block b (tau = row): below the diagonal
+    // g^(tau - j1) g^(j1 - j) with j1 the block's last token (both exponents >= 0); on it
+    // g^(lane - i) for i <= lane (the rest is masked)
+    auto weigh = [&](float (&x)[32], int b) {
+        if (b < quad) {
+            float w = exp2f((float)(row - 32 * b - 31) * lg);
+#pragma unroll
+            for (int i = 31; i >= 0; --i) {
+                x[i] *= w;
+                w *= g;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] *= exp2f((float)max(lane - i, 0) * lg);
+        }
+    };
+    // fp32 TMEM columns [col, col + 16) of this lane times sc, in place
+    auto scale16 = [&](uint32_t col, float sc) {
+        float v[16];
+        ptx::tmem_ld16(tmem + lane_base + col, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] *= sc;
+        ptx::tmem_st16(tmem + lane_base + col, v);
+    };
+    auto epi1 = [&](int n) {
         const int b0 = 2 * half;
         const uint32_t pc = TA_A + 96 * half;
         float v0[32], v1[32];
         if (b0 + 1 <= quad) {
-            ptx::tmem_ld32x2(tmem + lane_base + TA_A + 32 * b0, tmem + lane_base + TA_A + 32 * (b0 + 1), v0, v1);
-            st_pairs(pc, v0, false);
-            st_pairs(pc + 16, v1, b0 + 1 == quad);
+            if (DECAY) {
+                // one block at a time (registers), in an order in which no pair store lands on
+                // fp32 columns not yet read: half 0 stores to columns 0-31 (block 0 first), half 1
+                // to columns 96-127 (block 3 first)
+                if (half == 0) {
+                    ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * b0, v0);
+                    weigh(v0, b0);
+                    st_pairs(pc, v0, false);
+                    ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * (b0 + 1), v1);
+                    weigh(v1, b0 + 1);
+                    st_pairs(pc + 16, v1, b0 + 1 == quad);
+                } else {
+                    ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * (b0 + 1), v1);
+                    weigh(v1, b0 + 1);
+                    st_pairs(pc + 16, v1, b0 + 1 == quad);
+                    ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * b0, v0);
+                    weigh(v0, b0);
+                    st_pairs(pc, v0, false);
+                }
+            } else {
+                ptx::tmem_ld32x2(tmem + lane_base + TA_A + 32 * b0, tmem + lane_base + TA_A + 32 * (b0 + 1), v0, v1);
+                st_pairs(pc, v0, false);
+                st_pairs(pc + 16, v1, b0 + 1 == quad);
+            }
         } else if (b0 == quad) {
             ptx::tmem_ld32(tmem + lane_base + TA_A + 32 * b0, v0);
+            if (DECAY) weigh(v0, b0);
             st_pairs(pc, v0, true);
             st_pairs(pc + 16, nullptr, false);
         } else {
             st_pairs(pc, nullptr, false);
             st_pairs(pc + 16, nullptr, false);
+        }
+        if (DECAY) {
+            // Gam on Q P0 (and Q mK0), and in the output walk on Q E0 (and Q n0)
+            const float gr = exp2f((float)(row + 1) * lg);
+            scale16(TY + half * 32, gr);
+            scale16(TY + half * 32 + 16, gr);
+            if (NORM && half == 0) scale16(TY + 64, gr);
+            if (MODE == OUTPUT) {
+                scale16(TO + half * 32, gr);
+                scale16(TO + half * 32 + 16, gr);
+                if (NORM && half == 0) scale16(TO + 64, gr);
+            }
+            // Lam K over the state tile (R1 has read the state; E3 rewrites it): this lane's row,
+            // half of its 16-byte chunks; rows past the sequence are zero
+            const int len = min(C, p.T - (chunk0 + n) * C);
+            const float lam = row < len ? exp2f((float)(len - 1 - row) * lg) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t off = row * 128 + ((((half * 4 + j) ^ row) & 7) << 4);
+                uint4 u = *reinterpret_cast<const uint4*>(sm + AS_K + off);
+                uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                    w[e] = ptx::pack_bf16(lam * f.x, lam * f.y);
+                }
+                *reinterpret_cast<uint4*>(sm + AS_ST + off) = u;
+            }
         }
         ptx::tmem_st_wait();
     };
@@ -425,17 +525,18 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     };
     // E3: state += increment, its bf16 copy -> AS_ST; O of the chunk (fp32) staged over the
     // A tile as two [128 rows][32 cols] boxes in the 128B-swizzled TMA layout
-    auto epi3 = [&]() {
+    auto epi3 = [&](int n) {
         float v[32];
+        const float rho = DECAY ? exp2f((float)min(C, p.T - (chunk0 + n) * C) * lg) : 1.f;
         ptx::tmem_ld32(tmem + lane_base + TA_INC + half * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) st[i] += v[i];
+        for (int i = 0; i < 32; ++i) st[i] = fmaf(rho, st[i], v[i]);
         if (MODE == OUTPUT || row < 64) st_row32(sm + AS_ST, row, half * 32, st);
         if (NORM && (quad & 1) == 0) {       // lanes 0 and 64: mK0 += K^T 1, n0 += K^T y1
             ptx::tmem_ld32(tmem + lane_base + TN_V + half * 32, v);
             if (lane == 0) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) st2[i] += v[i];
+                for (int i = 0; i < 32; ++i) st2[i] = fmaf(rho, st2[i], v[i]);
                 if (quad == 0 || MODE == OUTPUT) st_row32(sm + (quad ? AS_NN : AS_NM), 0, half * 32, st2);
             }
         }
@@ -474,7 +575,7 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             }
         }
         if (!commit_wait()) { ok = false; break; }          // loads and R1 done
-        epi1();
+        epi1(n);
         sync_for_mma();
         if (tid == 0) issue_r2(n);
         if (!commit_wait()) { ok = false; break; }          // R2 done
@@ -486,7 +587,7 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         if (!commit_wait()) { ok = false; break; }          // R3 done: Q/Y, K, V free
         if (tid == 0 && n + 1 < nch) issue_load(n + 1);
-        epi3();
+        epi3(n);
         sync_for_mma();
     }
     if (MODE == OUTPUT && ok && tid == 0) store_o(nch - 1);
@@ -515,8 +616,10 @@ k_ahla_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             const int rr = (f >> 4) & (D - 1);
             out4[f] = st4[(f & ~15) | ((f & 15) ^ (rr & 7))];
         }
+        // decay: rho of the segment = g^(its length)
+        const float rho_seg = DECAY ? exp2f((float)min(nch * C, p.T - chunk0 * C) * lg) : 0.f;
         for (int f = (NORM ? S::vec(2) : S::vec(0)) / 4 + tid; f < S::size / 4; f += ANT)
-            out4[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+            out4[f] = make_float4(DECAY && f == S::vec(2) / 4 ? rho_seg : 0.f, 0.f, 0.f, 0.f);
         if (vrow) {                          // (mK, n) of the segment
 #pragma unroll
             for (int i = 0; i < 32; ++i) slot[S::vec(quad >> 1) + half * 32 + i] = st2[i];
@@ -544,30 +647,42 @@ size_t ahla_workspace_bytes(int BH, int T, int seg_chunks, bool norm) {
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
-template <bool NORM>
-static cudaError_t ahla_run(const void* q, const void* k, const void* v, float* o, int BH, int T, float eps,
-                            void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
+bool ahla_folds(int BH, int T, int seg_chunks, bool norm) {
+    const Plan pl = plan(BH, T, ahla_ctas_per_sm(norm) * kSMs, seg_chunks);
+    return pl.NSf + 1 <= PH_MAX;
+}
+
+template <bool NORM, bool DECAY>
+static cudaError_t ahla_run(const void* q, const void* k, const void* v, float* o, int BH, int H, int T, float eps,
+                            const float* gamma, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                            int seg_chunks) {
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, ahla_ctas_per_sm(NORM) * kSMs, seg_chunks);
-    Params prm;                              // the output walk
+    Params prm = {};                         // the output walk
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = eps; prm.norm = NORM ? 1 : 0;
     prm.sums = static_cast<float*>(ws);
     prm.pre = prm.sums + (size_t)BH * pl.NSp * simt_layout::size;
     prm.o = o;
     prm.status = status;
+    prm.gamma = gamma;
+    prm.H = H;
     prm.fold = pl.NSf + 1 <= PH_MAX ? 1 : 0;  // few slots: each output CTA folds its own prefix
+    // the decayed walk folds its prefix only (the prefix kernels carry no decay)
+    if (DECAY && !prm.fold) return cudaErrorNotSupported;
     Params sprm = prm;                       // the summary walk: shorter segments, slots 0 .. NSf - 1
     sprm.NCH = pl.NCHs; sprm.NS = pl.NSf; sprm.ratio = 1; sprm.fold = 0;
     constexpr int SMEM = (int)asmem_bytes<NORM>();
+    auto ksum = k_ahla_walk<SUMMARY, NORM, DECAY>;
+    auto kout = k_ahla_walk<OUTPUT, NORM, DECAY>;
     cudaError_t e;
-    if ((e = set_smem(k_ahla_walk<SUMMARY, NORM>, SMEM)) != cudaSuccess) return e;
-    if ((e = set_smem(k_ahla_walk<OUTPUT, NORM>, SMEM)) != cudaSuccess) return e;
+    if ((e = set_smem(ksum, SMEM)) != cudaSuccess) return e;
+    if ((e = set_smem(kout, SMEM)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_ahla_walk<SUMMARY, NORM><<<dim3(pl.NSp, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, sprm);
+    ksum<<<dim3(pl.NSp, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st, NORM)) != cudaSuccess)
@@ -585,19 +700,24 @@ static cudaError_t ahla_run(const void* q, const void* k, const void* v, float* 
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&cfg, k_ahla_walk<OUTPUT, NORM>, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
+        if ((e = cudaLaunchKernelEx(&cfg, kout, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
     } else {
-        k_ahla_walk<OUTPUT, NORM><<<dim3(pl.NS, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, prm);
+        kout<<<dim3(pl.NS, BH), ANT, SMEM, st>>>(mq, mk, mv, mo, prm);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }
 
-cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, bool norm, float eps,
-                         void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks) {
-    if (norm) return ahla_run<true>(q, k, v, o, BH, T, eps, ws, status, st, ev, seg_chunks);
-    return ahla_run<false>(q, k, v, o, BH, T, 0.f, ws, status, st, ev, seg_chunks);
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int H, int T, bool norm,
+                         float eps, const float* gamma, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                         int seg_chunks) {
+    if (gamma) {
+        if (norm) return ahla_run<true, true>(q, k, v, o, BH, H, T, eps, gamma, ws, status, st, ev, seg_chunks);
+        return ahla_run<false, true>(q, k, v, o, BH, H, T, 0.f, gamma, ws, status, st, ev, seg_chunks);
+    }
+    if (norm) return ahla_run<true, false>(q, k, v, o, BH, H, T, eps, nullptr, ws, status, st, ev, seg_chunks);
+    return ahla_run<false, false>(q, k, v, o, BH, H, T, 0.f, nullptr, ws, status, st, ev, seg_chunks);
 }
 
 }  // namespace tc

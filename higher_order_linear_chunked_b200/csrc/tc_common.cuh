@@ -38,6 +38,8 @@ struct Params {
     float* pre;      // [BH][NSp][summary floats]: carried-in prefixes
     float* o;        // [BH][T][64]
     int* status;
+    const float* gamma;  // AHLA with decay: per-head gamma (else nullptr)
+    int H;               // heads per batch (gamma index = bh % H)
 };
 
 // ---------------------------------------------------------------- descriptors
@@ -145,11 +147,15 @@ int decay_kernel_launches();
 cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
                           int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
 
-// The AHLA forward on the tcgen05 walkers, plain or ratio-normalised (tc_ahla.cu).
+// The AHLA forward on the tcgen05 walkers, plain or ratio-normalised, with per-head decay when
+// gamma is given (tc_ahla.cu).  The decayed walk needs the prefix folded into the output walker
+// (ahla_folds).
 size_t ahla_workspace_bytes(int BH, int T, int seg_chunks, bool norm);
 int ahla_ctas_per_sm(bool norm);
-cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int T, bool norm, float eps,
-                         void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks);
+bool ahla_folds(int BH, int T, int seg_chunks, bool norm);
+cudaError_t ahla_forward(const void* q, const void* k, const void* v, float* o, int BH, int H, int T, bool norm,
+                         float eps, const float* gamma, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                         int seg_chunks);
 
 }  // namespace tc
 }  // namespace hla

@@ -1028,11 +1028,15 @@ int segment_chunks() { return g_segment_chunks.load(); }
 
 bool supported(int op, bool norm, bool bf16, int d) {
     if (!bf16 || d != D) return false;
-    return op == OP_HLA2 || op == OP_AHLA || (op == OP_HLA2D && !norm);
+    return op == OP_HLA2 || op == OP_AHLA || op == OP_AHLAD || (op == OP_HLA2D && !norm);
+}
+
+bool fits(int op, bool norm, int BH, int T, int seg_chunks) {
+    return op != OP_AHLAD || ahla_folds(BH, T, seg_chunks, norm);
 }
 
 size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks) {
-    if (op == OP_AHLA) return ahla_workspace_bytes(BH, T, seg_chunks, norm);
+    if (op == OP_AHLA || op == OP_AHLAD) return ahla_workspace_bytes(BH, T, seg_chunks, norm);
     if (op == OP_HLA2D) return decay_workspace_bytes(BH, T);
     const Plan pl = plan(BH, T, kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
@@ -1042,14 +1046,19 @@ int kernel_launches(int op, bool norm, int BH, int T, int seg_chunks) {
     if (op == OP_HLA2D) return decay_kernel_launches();
     // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
     // two launches), output walk
-    const Plan pl = plan(BH, T, op == OP_AHLA ? ahla_ctas_per_sm(norm) * kSMs : kSMs, seg_chunks);
+    const bool ahla = op == OP_AHLA || op == OP_AHLAD;
+    const Plan pl = plan(BH, T, ahla ? ahla_ctas_per_sm(norm) * kSMs : kSMs, seg_chunks);
     return pl.NSf + 1 > PH_MAX ? 4 : 2;     // else the output walker folds the prefix itself
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
                     float* o, int BH, int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
                     int seg_chunks) {
-    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, T, norm, eps, ws, status, st, ev, seg_chunks);
+    if (op == OP_AHLA) return ahla_forward(q, k, v, o, BH, H, T, norm, eps, nullptr, ws, status, st, ev, seg_chunks);
+    if (op == OP_AHLAD) {
+        if (!gamma) return cudaErrorInvalidValue;
+        return ahla_forward(q, k, v, o, BH, H, T, norm, eps, gamma, ws, status, st, ev, seg_chunks);
+    }
     if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
@@ -1058,7 +1067,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
     const Plan pl = plan(BH, T, kSMs, seg_chunks);
-    Params prm;                              // the output walk
+    Params prm = {};                         // the output walk
     prm.T = T; prm.BH = BH; prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NSp = pl.NSp; prm.ratio = pl.ratio;
     prm.eps = eps; prm.norm = norm ? 1 : 0;
     prm.sums = static_cast<float*>(ws);

@@ -75,7 +75,7 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     # bf16, d = 64: second order (plain, normalised, decayed) and AHLA (plain, normalised) run on
     # the tensor cores
     for op, dec in ((hla.OP_HLA2, 0), (hla.OP_HLA2_NORM, 0), (hla.OP_HLA2, 1), (hla.OP_AHLA, 0),
-                    (hla.OP_AHLA_NORM, 0)):
+                    (hla.OP_AHLA_NORM, 0), (hla.OP_AHLA, 1), (hla.OP_AHLA_NORM, 1)):
         assert use(op, bf16, dec) == 1, (op, dec)
     # the rest on CUDA cores: fp32 inputs, d = 32, third order, normalised with decay
     assert use(hla.OP_HLA2, f32, 0) == 0
@@ -88,6 +88,11 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert launches(hla.OP_HLA2_NORM, bf16, 0) == 2   # the output walker folds the prefix
     assert launches(hla.OP_AHLA, bf16, 0) == 2
     assert launches(hla.OP_AHLA_NORM, bf16, 0) == 2
+    assert launches(hla.OP_AHLA, bf16, 1) == 2                                          # decayed AHLA
+    # the decayed AHLA walk folds its prefix in the output walker: a plan with more summary slots
+    # than that (one long head) runs on the CUDA cores
+    assert lib.hla_uses_tensor_cores(hla.OP_AHLA, bf16, 1, 1, 1, 65536, 64, 64) == 0
+    assert lib.hla_uses_tensor_cores(hla.OP_AHLA, bf16, 0, 1, 1, 65536, 64, 64) == 1
     # the normalised AHLA walker runs one CTA per SM (512 TMEM columns): its segment plan, and
     # so its workspace, differs from the plain walker's (two per SM) at the same shape
     ws_tc = lambda op, B, H, T: lib.hla_workspace_bytes(op, bf16, 0, B, H, T, 64, 64)
@@ -221,9 +226,10 @@ def test_normalised_ahla_hla3_routing_and_errors(lib):
     vp, f = ctypes.c_void_p, ctypes.c_float
     assert lib.hla_uses_tensor_cores(hla.OP_AHLA_NORM, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 1
     assert lib.hla_uses_tensor_cores(hla.OP_HLA3_NORM, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 0
+    assert lib.hla_uses_tensor_cores(hla.OP_AHLA_NORM, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 1   # + decay
+    assert lib.hla_uses_tensor_cores(hla.OP_HLA3_NORM, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0
     for op, plain in ((hla.OP_AHLA_NORM, hla.OP_AHLA), (hla.OP_HLA3_NORM, hla.OP_HLA3)):
         assert lib.hla_workspace_bytes(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) > 0            # decayed form
-        assert lib.hla_uses_tensor_cores(op, hla.HLA_BF16, 1, 4, 16, 4096, 64, 64) == 0
         assert lib.hla_workspace_bytes(op, hla.HLA_F32, 0, 2, 8, 4096, 32, 32) == \
             lib.hla_workspace_bytes(plain, hla.HLA_F32, 0, 2, 8, 4096, 32, 32)
     assert lib.hla_uses_tensor_cores(hla.OP_AHLA, hla.HLA_BF16, 0, 4, 16, 4096, 64, 64) == 1

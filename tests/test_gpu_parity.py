@@ -24,9 +24,12 @@ OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3"]
 
 
 def recipe(op, dtype, B, H, T, d, seed=0):
-    qk = "softplus" if op == "hla2n" else "scaled"
-    v = "unit" if op == "hla2n" else "scaled"
-    g = (0.95, 0.999) if op == "hla2d" else None
+    """Workload of an op name; "ahlan_g" is the ratio-normalised AHLA with per-head decay."""
+    decayed = op in ("hla2d", "ahlad", "ahlan_g")
+    op = "ahlan" if op == "ahlan_g" else op
+    qk = "softplus" if op in ("hla2n", "ahlan") else "scaled"
+    v = "unit" if op in ("hla2n", "ahlan") else "scaled"
+    g = ((0.95, 0.999) if op == "hla2d" else (0.9, 0.999)) if decayed else None
     return hla_inputs.Workload(f"{op}_{dtype}_{B}x{H}x{T}x{d}", op, dtype, B, H, T, d, d, qk, v,
                                gamma_range=g, seed=seed)
 
@@ -109,19 +112,37 @@ def test_bf16_d64_parity_across_segments(op, T):
     assert err <= TOL["bf16"], err
 
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla", "ahlan", "ahlad", "ahlan_g"])
 @pytest.mark.parametrize("nch", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T", [129, 1000, 2049])
 def test_segment_length_invariance(op, nch, T):
-    """Tensor-core walk over 1..16 chunks per segment: same result (to rounding) as the oracle."""
+    """Tensor-core walk over 1..16 chunks per segment: same result (to rounding) as the oracle.
+    (The decayed AHLA walk folds its prefix in the output walker; a plan with more summary slots
+    than that fold takes runs on the CUDA cores, which the oracle checks the same way.)"""
     w = recipe(op, "bf16", 2, 2, T, 64, seed=nch + T)
     q, k, v, g = hla_inputs.make_inputs(w)
     hla.set_segment_chunks(nch)
     try:
-        o = gpu_forward(op, q, k, v, g)
+        o = gpu_forward(w.op, q, k, v, g, eps=w.eps)
     finally:
         hla.set_segment_chunks(0)
-    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(op, q, k, v, gamma=g))
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(w.op, q, k, v, gamma=g, eps=w.eps))
+    assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("op", ["ahlad", "ahlan_g"])
+@pytest.mark.parametrize("gam", [0.3, 0.9, 0.999, 1.0])
+def test_decayed_ahla_tensor_cores_gamma_range(op, gam):
+    """Decayed AHLA on the tensor-core walker from strong to no decay: many output segments per
+    head (the decayed fold), a ragged tail, one gamma per head pair."""
+    w = recipe(op, "bf16", 1, 2, 1500, 64, seed=int(gam * 100) + 5)
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    g = torch.full((2,), gam)
+    lib_uses = hla.uses_tensor_cores(hla.OP_AHLA_NORM if w.op == "ahlan" else hla.OP_AHLA, hla.HLA_BF16, True,
+                                     1, 2, 1500, 64, 64)
+    assert lib_uses
+    o = gpu_forward(w.op, q, k, v, g, eps=w.eps)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(w.op, q, k, v, gamma=g, eps=w.eps))
     assert err <= TOL["bf16"], err
 
 
