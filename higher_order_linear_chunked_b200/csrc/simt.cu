@@ -680,10 +680,14 @@ __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int 
 // which are all the output kernel reads.  Three launches, each parallel over chunks or elements:
 // plain exclusive sums of S, P, mK in place; the corrected F_l, F1_l per chunk; their exclusive
 // sums in place.  The result equals the Blelloch tree's up to the order of fp32 additions.
+// With decay (OP_HLA3D) the combine scales the earlier operand's S, P, mK, F, F1 by the later
+// one's rho and its cross terms by rho too, while Q2, X, Z enter only as the chunk's own; so
+// the sums become decayed running sums (run = rho_l run + y_l) and the corrected terms
+// F_l + rho_l (...), with the same three launches.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ sums, int NC, int NCp, int which) {
-    using S = Sum<OP_HLA3, D>;
+    using S = Sum<OP, D>;
     const int e = blockIdx.x * NT + threadIdx.x;
     int off;
     if (which == 0) {                        // S, P and mK
@@ -694,17 +698,28 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ su
         off = e < D * D ? S::mat(3) + e : S::vec(2) + (e - D * D);
     }
     float* p = sums + (size_t)blockIdx.y * NCp * S::SIZE + off;
+    const float* rho = sums + (size_t)blockIdx.y * NCp * S::SIZE + S::SCAL;
     float run = 0.f;
-    for (int l = 0; l < NC; ++l) {
-        const float y = p[(size_t)l * S::SIZE];
-        p[(size_t)l * S::SIZE] = run;
-        run += y;
+    for (int l0 = 0; l0 < NC; l0 += 8) {     // eight loads in flight, then the dependent adds
+        float y[8], r[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NC) {
+                y[i] = p[(size_t)(l0 + i) * S::SIZE];
+                r[i] = OP == OP_HLA3D ? rho[(size_t)(l0 + i) * S::SIZE] : 1.f;
+            }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NC) {
+                p[(size_t)(l0 + i) * S::SIZE] = run;
+                run = OP == OP_HLA3D ? fmaf(r[i], run, y[i]) : run + y[i];
+            }
     }
 }
 
-template <int D>
+template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ sums, int NCp) {
-    using S = Sum<OP_HLA3, D>;
+    using S = Sum<OP, D>;
     constexpr int LD = Dim<D>::LD;
     extern __shared__ float smx[];
     float* S0 = smx;
@@ -729,28 +744,28 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ su
     mm<D, D, D>(Tile{S0, LD}, Tile{Q2, LD}, Zero{}, Put{SQ, LD});                  // S0 Q2
     __syncthreads();
     float* F = slot + S::mat(3);
-    // F += (S0 Q2) P0 + S0 X + Z P0
-    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, Tile{Xs, LD}, Tile{Zs, LD}, Tile{P0, LD},
-                       [&](int r, int c) { return F[r * D + c]; }, [&](int r, int c, float x) { F[r * D + c] = x; });
+    const float rho = OP == OP_HLA3D ? slot[S::SCAL] : 1.f;
+    // F += rho ((S0 Q2) P0 + S0 X + Z P0)
+    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, Tile{Xs, LD}, Tile{Zs, LD}, Tile{P0, LD}, Zero{},
+                       [&](int r, int c, float x) { F[r * D + c] = fmaf(rho, x, F[r * D + c]); });
     for (int a = threadIdx.x; a < D; a += blockDim.x) {
         float s = 0.f;
         for (int b = 0; b < D; ++b) s += SQ[a * LD + b] * mk[b] + S0[a * LD + b] * x1[b] + Zs[a * LD + b] * mk[b];
-        slot[S::vec(2) + a] += s;
+        slot[S::vec(2) + a] = fmaf(rho, s, slot[S::vec(2) + a]);
     }
 }
 
-template <int D>
+template <int OP, int D>
 static cudaError_t hla3_factored_prefix(float* sums, int NC, int NCp, int BH, cudaStream_t st) {
-    k_hla3_prefix_plain<D><<<dim3((2 * D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 0);
+    k_hla3_prefix_plain<OP, D><<<dim3((2 * D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem = (int)(sizeof(float) * (6 * D * Dim<D>::LD + 2 * D));
-    if ((e = cudaFuncSetAttribute(k_hla3_prefix_cross<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-        cudaSuccess)
-        return e;
-    k_hla3_prefix_cross<D><<<dim3(NC, BH), NT, smem, st>>>(sums, NCp);
+    auto kc = k_hla3_prefix_cross<OP, D>;
+    if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    kc<<<dim3(NC, BH), NT, smem, st>>>(sums, NCp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_hla3_prefix_plain<D><<<dim3((D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 1);
+    k_hla3_prefix_plain<OP, D><<<dim3((D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 1);
     return cudaGetLastError();
 }
 
@@ -1067,8 +1082,8 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
     ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, H, T, NC, NCp, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    if (OP == OP_HLA3) {
-        if ((e = hla3_factored_prefix<D>(sums, NC, NCp, BH, st)) != cudaSuccess) return e;
+    if (OP == OP_HLA3 || OP == OP_HLA3D) {
+        if ((e = hla3_factored_prefix<OP, D>(sums, NC, NCp, BH, st)) != cudaSuccess) return e;
     } else if (fold_fits<OP, D>()) {
         auto kf = k_scan_fold<OP, D>;
         if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fold_smem<OP, D>())) !=
@@ -1139,7 +1154,7 @@ static bool uses_fold(int op, int d) {
 }
 
 int kernel_launches(int op, int d, int T) {
-    if (op == OP_HLA3) return 2 + 3;          // the factored prefix
+    if (op == OP_HLA3 || op == OP_HLA3D) return 2 + 3;   // the factored prefix (decayed or not)
     return 2 + (uses_fold(op, d) ? 1 : scan_launches(next_pow2((T + C - 1) / C)));
 }
 

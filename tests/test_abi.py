@@ -101,14 +101,13 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert lib.hla_kernel_launches(hla.OP_HLA2_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 4   # many slots
     assert launches(hla.OP_HLA2, bf16, 1) == 5
     # CUDA-core path: chunk kernel, one scan launch (a per-head fold) and the output kernel;
-    # the third order takes the factored prefix (three launches); its decayed form keeps the
-    # per-level Blelloch tree: 64 chunks of 64 tokens, 2 x 6 levels
+    # the third order, decayed or not, takes the factored prefix (three launches)
     assert launches(hla.OP_HLA2, f32, 0) == 3
     assert launches(hla.OP_AHLA_NORM, f32, 0) == 3
     assert launches(hla.OP_HLA2_UNMASKED, bf16, 0) == 3
     assert launches(hla.OP_HLA3, f32, 0, d=32) == 2 + 3      # the factored third-order prefix
     assert launches(hla.OP_HLA3, f32, 0) == 2 + 3
-    assert launches(hla.OP_HLA3, f32, 1, d=32) == 2 + 12     # decayed: the per-level tree
+    assert launches(hla.OP_HLA3, f32, 1, d=32) == 2 + 3      # decayed: the same three prefix launches
     # decayed workspace: 256 B status block + one 4 x 64 x 64 fp32 slot per 128-token chunk
     T = 16384
     assert lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, T, 64, 64) == 256 + 32 * (T // 128) * 4 * 64 * 64 * 4

@@ -264,6 +264,74 @@ def test_ahla_segment_plan_matches_recurrence():
     assert rel(np.vstack(outs), recur("ahla", q, k, v)) < 1e-12
 
 
+def ahla_walk_decayed(q, k, v, c, g, P0=None, E0=None):
+    """The tensor-core AHLA walker with decay: At = g^(tau - j) A on the masked scores,
+    Gam = diag(g^(tau+1)), Lam = diag(g^(len-1-tau)), rho = g^len per chunk:
+        Y = Gam Q P0 + At V,  O = Gam Q E0 + At Y,  P0 = rho P0 + K^T Lam V,  E0 = rho E0 + K^T Lam Y.
+    Chunks are the sequence's own (the last one may be short)."""
+    d, dv = q.shape[1], v.shape[1]
+    P0 = np.zeros((d, dv)) if P0 is None else P0
+    E0 = np.zeros((d, dv)) if E0 is None else E0
+    outs = []
+    for t0 in range(0, q.shape[0], c):
+        Q, K, V = q[t0:t0 + c], k[t0:t0 + c], v[t0:t0 + c]
+        n = Q.shape[0]
+        tau = np.arange(n)
+        At = np.tril(Q @ K.T) * np.tril(g ** (tau[:, None] - tau[None, :]).clip(min=0))
+        Gam = (g ** (tau + 1))[:, None]
+        Lam = (g ** (n - 1 - tau))[:, None]
+        Y = Gam * (Q @ P0) + At @ V
+        outs.append(Gam * (Q @ E0) + At @ Y)
+        P0 = g ** n * P0 + K.T @ (Lam * V)
+        E0 = g ** n * E0 + K.T @ (Lam * Y)
+    return np.vstack(outs), P0, E0
+
+
+@pytest.mark.parametrize("gamma", [1.0, 0.97, 0.6])
+@pytest.mark.parametrize("T,c", [(1, 8), (13, 8), (64, 16), (99, 32)])
+def test_ahla_decayed_chunk_step_matches_recurrence(T, c, gamma):
+    q, k, v = rand_head(T, 5, 3, seed=T + 2000)
+    O, _, _ = ahla_walk_decayed(q, k, v, c, gamma)
+    assert rel(O, recur("ahlad", q, k, v, gamma=gamma)) < 1e-12
+
+
+@pytest.mark.parametrize("normalized", [False, True])
+@pytest.mark.parametrize("gamma", [0.97, 0.6])
+def test_ahla_decayed_segment_plan_matches_recurrence(gamma, normalized):
+    """Decayed summary segments walked from zero (rho = g^length), the fold of their prefix with
+    summary l weighted by the product of the later summaries' rho (P0, E0, and the cross term
+    P^T_m D_suf^T(m+1) by the weight of m), then decayed output walks; on [V | 1] for the
+    ratio-normalised form (its vectors mK, n are the ones column's P and E)."""
+    T, c, NCH, d, dv = 150, 8, 3, 4, 3
+    q, k, v = rand_head(T, d, dv, seed=9)
+    if normalized:
+        q, k = np.abs(q), np.abs(k)
+    v1 = np.hstack([v, np.ones((T, 1))]) if normalized else v
+    seg_tok = NCH * c
+    n_out = -(-T // seg_tok)
+    slots = []
+    for i in range(n_out - 1):
+        sl = slice(i * seg_tok, (i + 1) * seg_tok)
+        _, P, E = ahla_walk_decayed(q[sl], k[sl], v1[sl], c, gamma)
+        slots.append(dict(P=P, E=E, D=k[sl].T @ q[sl], rho=gamma ** seg_tok))
+    outs = []
+    for n in range(n_out):
+        P0, E0 = np.zeros((d, v1.shape[1])), np.zeros((d, v1.shape[1]))
+        w = [np.prod([s["rho"] for s in slots[l + 1:n]]) for l in range(n)]
+        for l in range(n):
+            P0 = P0 + w[l] * slots[l]["P"]
+            E0 = E0 + w[l] * slots[l]["E"]
+        for m in range(n - 1):
+            Dsuf = sum(slots[l]["D"] for l in range(m + 1, n))
+            E0 = E0 + w[m] * (Dsuf @ slots[m]["P"])
+        sl = slice(n * seg_tok, min((n + 1) * seg_tok, T))
+        outs.append(ahla_walk_decayed(q[sl], k[sl], v1[sl], c, gamma, P0=P0, E0=E0)[0])
+    O = np.vstack(outs)
+    if normalized:
+        O = O[:, :-1] / (O[:, -1:] + EPS)
+    assert rel(O, recur("ahlan" if normalized else "ahlad", q, k, v, gamma=gamma)) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # decayed second order: chunk summaries, prefix recurrences and the output split
 # ---------------------------------------------------------------------------
@@ -388,19 +456,22 @@ def test_normaliser_vectors_give_the_literal_denominator():
         assert abs(q[t] @ F1 - den_3[t]) < 1e-12 * max(1.0, den_3[t])
 
 
-def third_order_factored_prefix(sums):
+def third_order_factored_prefix(sums, decayed=False):
     """The third-order exclusive prefix as the CUDA-core path runs it (three launches): plain
     exclusive sums S0, P0, then per chunk the corrected F_l + S0(l) Q2_l P0(l) + S0(l) X_l +
-    Z_l P0(l), then its plain exclusive sum F0."""
+    Z_l P0(l), then its plain exclusive sum F0.  Decayed: running sums run = rho_l run + y_l
+    and the cross term scaled by rho_l."""
+    rho = [float(s["rho"]) if decayed else 1.0 for s in sums]
     S0 = [0.0 * sums[0]["S"]]
     P0 = [0.0 * sums[0]["P"]]
-    for s in sums[:-1]:
-        S0.append(S0[-1] + s["S"])
-        P0.append(P0[-1] + s["P"])
-    Y = [s["F"] + S0[l] @ s["Q2"] @ P0[l] + S0[l] @ s["X"] + s["Z"] @ P0[l] for l, s in enumerate(sums)]
+    for l, s in enumerate(sums[:-1]):
+        S0.append(rho[l] * S0[-1] + s["S"])
+        P0.append(rho[l] * P0[-1] + s["P"])
+    Y = [s["F"] + rho[l] * (S0[l] @ s["Q2"] @ P0[l] + S0[l] @ s["X"] + s["Z"] @ P0[l])
+         for l, s in enumerate(sums)]
     F0 = [0.0 * Y[0]]
-    for y in Y[:-1]:
-        F0.append(F0[-1] + y)
+    for l, y in enumerate(Y[:-1]):
+        F0.append(rho[l] * F0[-1] + y)
     return [dict(S=S0[l], P=P0[l], F=F0[l]) for l in range(len(sums))]
 
 
@@ -415,3 +486,25 @@ def test_third_order_factored_prefix_equals_the_combine_fold(lengths):
     for n in range(len(lengths)):
         for key in ("S", "P", "F"):
             np.testing.assert_allclose(got[n][key], ref[n][key], rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("lengths", [[6], [3, 9, 1], [8, 8, 8, 8, 8], [1, 2, 3, 4, 5, 6, 7]])
+@pytest.mark.parametrize("gamma", [0.5, 0.9, 1.0])
+def test_decayed_third_order_factored_prefix_equals_the_combine_fold(lengths, gamma):
+    """The decayed third-order prefix in factored form (decayed running sums of S, P and of the
+    rho-scaled corrected F) against the fold of the decayed combine."""
+    T, d, dv = sum(lengths), 4, 3
+    q, k, v = rand_head(T, d, dv, seed=11 + len(lengths))
+    b = seg.split_points(T, lengths)
+    sums = [seg.hla3_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], gamma=gamma)
+            for i in range(len(lengths))]
+    ref = seg.fold_exclusive(sums, seg.hla3_combine, seg.hla3_identity(d, dv))
+    got = third_order_factored_prefix(sums, decayed=True)
+    for n in range(len(lengths)):
+        for key in ("S", "P", "F"):
+            np.testing.assert_allclose(got[n][key], ref[n][key], rtol=0, atol=1e-11)
+    # a planted mistake: the cross term without its rho differs once there is decay
+    if gamma < 1.0 and len(lengths) > 2:
+        wrong = third_order_factored_prefix([dict(s, rho=np.array(1.0)) if i else s for i, s in enumerate(sums)],
+                                            decayed=True)
+        assert max(np.abs(wrong[n]["F"] - ref[n]["F"]).max() for n in range(len(lengths))) > 1e-6
