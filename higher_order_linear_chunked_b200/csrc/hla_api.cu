@@ -283,11 +283,12 @@ hla_status_t backward_call(hla_op_t op, const void* q, const void* k, const void
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
     float* body = reinterpret_cast<float*>(static_cast<char*>(workspace) + hla::kStatusBytes);
+    int* status = static_cast<int*>(workspace);
     const cudaError_t e =
         op == HLA_OP_HLA2_NORM
             ? hla::simt::backward_normalized(dtype == HLA_BF16, d, q, k, v, dout, eps, dq, dk, dv_out, B * H, T, body,
-                                             st)
-            : hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, st);
+                                             status, st)
+            : hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, status, st);
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 }  // namespace

@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "simt.h"
+#include "tc.h"
 
 namespace hla {
 namespace simt {
@@ -1858,7 +1859,7 @@ int backward_launches(int d, int T) {
 
 template <int D, typename TIn>
 static cudaError_t backward_run(const void* q, const void* k, const void* v, const float* dout, float* dq, float* dk,
-                                float* dv, int BH, int T, float* ws, cudaStream_t st) {
+                                float* dv, int BH, int T, float* ws, int* status, bool fp32_only, cudaStream_t st) {
     const int NC = (T + C - 1) / C;
     const int NCp = next_pow2(NC);
     float* sums = ws;
@@ -1893,13 +1894,18 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dS'
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the gradients: on the tensor cores for bf16 at d = 64 (128-token chunks, reading every other
+    // carried state and adjoint of the 64-token stages), else on the CUDA cores
+    if (D == 64 && sizeof(TIn) == 2 && !fp32_only)
+        return tc::bwd_out(q, k, v, dout, sums, bw, NC, NCp, dq, dk, dv, BH, T, status, st);
     ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
                                      dv);
     return cudaGetLastError();
 }
 
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
-                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
+                     float* dk, float* dv, int BH, int T, float* ws, int* status, cudaStream_t st,
+                     bool fp32_only);
 
 // ---------------------------------------------------------------------------
 // Ratio-normalised second order: o = num / (den + eps), num = W V and den = W 1 (the same operator
@@ -1951,7 +1957,7 @@ int backward_normalized_launches(int d, int T) {
 }
 
 cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
-                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws,
+                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws, int* status,
                                 cudaStream_t st) {
     const size_t n = (size_t)BH * T * d;
     float* num = ws;
@@ -1978,8 +1984,12 @@ cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, 
     if (d == 32) k_norm_grads<32><<<(unsigned)((rows + NT - 1) / NT), NT, 0, st>>>(num, den, dout, eps, rows, dnum, g1);
     else k_norm_grads<64><<<(unsigned)((rows + NT - 1) / NT), NT, 0, st>>>(num, den, dout, eps, rows, dnum, g1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = backward(bf16, d, q, k, v, dnum, dq, dk, dv, BH, T, inner, st)) != cudaSuccess) return e;
-    if ((e = backward(bf16, d, q, k, ones, g1, dq2, dk2, dv2, BH, T, inner, st)) != cudaSuccess) return e;
+    // The two terms of dq and dk nearly cancel where o barely depends on q and k (o = v for a
+    // constant v), so both passes keep the fp32 gradient kernel: bf16 operands would leave an
+    // error of the size of each term, not of their difference.
+    if ((e = backward(bf16, d, q, k, v, dnum, dq, dk, dv, BH, T, inner, status, st, true)) != cudaSuccess) return e;
+    if ((e = backward(bf16, d, q, k, ones, g1, dq2, dk2, dv2, BH, T, inner, status, st, true)) != cudaSuccess)
+        return e;
     k_add_into<<<blocks, NT, 0, st>>>(dq, dq2, n);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_add_into<<<blocks, NT, 0, st>>>(dk, dk2, n);
@@ -1987,13 +1997,13 @@ cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, 
 }
 
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
-                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st) {
+                     float* dk, float* dv, int BH, int T, float* ws, int* status, cudaStream_t st, bool fp32_only) {
     if (bf16) {
-        if (d == 32) return backward_run<32, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
-        return backward_run<64, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+        if (d == 32) return backward_run<32, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, status, true, st);
+        return backward_run<64, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, status, fp32_only, st);
     }
-    if (d == 32) return backward_run<32, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
-    return backward_run<64, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+    if (d == 32) return backward_run<32, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, status, true, st);
+    return backward_run<64, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, status, true, st);
 }
 
 }  // namespace simt

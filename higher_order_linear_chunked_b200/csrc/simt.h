@@ -39,17 +39,20 @@ cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const voi
                  const float* gamma, float eps, int BH, int H, float* o, cudaStream_t st);
 
 // Backward pass of the masked second-order output (no decay, not normalised): dq, dk, dv fp32
-// [BH][T][d] for the output gradient dout fp32 [BH][T][d]; ws: backward_workspace_floats floats.
+// [BH][T][d] for the output gradient dout fp32 [BH][T][d]; ws: backward_workspace_floats floats;
+// status: the device status word (a bounded wait that gave up sets it).  bf16 at d = 64 takes
+// the tensor-core gradient kernel for its last stage unless fp32_only.
 size_t backward_workspace_floats(int d, int BH, int T);
 int backward_launches(int d, int T);
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
-                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
+                     float* dk, float* dv, int BH, int T, float* ws, int* status, cudaStream_t st,
+                     bool fp32_only = false);
 // The same for the ratio-normalised output (two plain forwards, two plain backwards, element-wise
 // glue); ws: backward_normalized_workspace_floats floats.
 size_t backward_normalized_workspace_floats(int d, int BH, int T);
 int backward_normalized_launches(int d, int T);
 cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
-                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws,
+                                float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws, int* status,
                                 cudaStream_t st);
 
 }  // namespace simt

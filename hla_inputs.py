@@ -91,6 +91,10 @@ WORKLOADS = {
     "hla3d_f32_2x8x4096x32": Workload(
         "hla3d_f32_2x8x4096x32", "hla3d", "f32", 2, 8, 4096, 32, 32, "scaled", "scaled",
         gamma_range=(0.95, 0.999)),
+    # the ratio-normalised AHLA with decay (op "ahlan" with a gamma per head)
+    "ahlan_decayed_bf16_4x16x8192x64": Workload(
+        "ahlan_decayed_bf16_4x16x8192x64", "ahlan", "bf16", 4, 16, 8192, 64, 64, "softplus", "unit",
+        gamma_range=(0.95, 0.999)),
 }
 
 

@@ -4,9 +4,9 @@
 Contribuciones 2: exact scan-based training.  The reference is ``oracle.backward.hla2_grads``
 (reverse-mode differentiation of the masked-matrix definition, pinned by finite differences in
 ``tests/test_backward_algebra.py``).  The library's hla2_backward runs the chunk-parallel reverse
-walk in fp32 on the GPU.  Metric and gates as for the forward: max row-wise relative L2 error,
-1e-4 for fp32 inputs, 2e-2 for bf16 inputs (the bf16 values are widened exactly, so the bf16 gate
-is loose here).
+walk on the GPU: fp32 on the CUDA cores, except the last stage (the gradients of every chunk) for
+bf16 inputs at d = 64, which runs on the tensor cores with bf16 operands.  Metric and gates as for
+the forward: max row-wise relative L2 error, 1e-4 for fp32 inputs, 2e-2 for bf16 inputs.
 """
 import numpy as np
 import pytest
@@ -61,7 +61,14 @@ def test_backward_matches_autograd_of_the_gpu_forward_at_the_headline_shape():
     """At B=4, H=16, T=4096, d=64 the fp64 reference is too large to run per head in the test, so
     the gradient is checked by a property that holds at any size: for a random direction (dQ, dK,
     dV)-weighted sum, <grad, delta> equals the directional derivative of <O, dO> computed from the
-    oracle's forward by central differences on two heads."""
+    oracle's forward by central differences on two heads.
+
+    Gate: for delta with independent standard normal entries, <grad, delta> and <err, delta> are
+    centred with standard deviations ||grad|| and ||err||, so the error is measured in units of
+    ||grad|| (the gradient of the heads checked): |ana - num| <= 2e-2 ||grad||, the bf16 parity
+    gate.  bf16 inputs at d = 64 take the tensor-core gradient kernel, whose bf16 operands leave
+    about 2e-3 of ||grad|| (checked chunk by chunk against the fp64 reference in
+    test_backward_full_length_head); |num| itself has no fixed relation to ||grad||."""
     B, H, T, d = 4, 16, 4096, 64
     q, k, v, do = _case("bf16", B, H, T, d, seed=11)
     dev = torch.device("cuda:0")
@@ -80,7 +87,15 @@ def test_backward_matches_autograd_of_the_gpu_forward_at_the_headline_shape():
             return float(np.sum(o * doh))
         num = (f(eps) - f(-eps)) / (2 * eps)
         ana = float(np.sum(dq[b, h] * dirs[0]) + np.sum(dk[b, h] * dirs[1]) + np.sum(dv[b, h] * dirs[2]))
-        assert abs(ana - num) <= 1e-3 * max(1.0, abs(num)), (bh, ana, num)
+        gnorm = float(np.sqrt(np.sum(dq[b, h] ** 2) + np.sum(dk[b, h] ** 2) + np.sum(dv[b, h] ** 2)))
+        assert abs(ana - num) <= TOL["bf16"] * gnorm, (bh, ana, num, gnorm)
+
+
+def test_backward_full_length_head():
+    """One head at the headline's length (T = 4096, 32 tensor-core chunks, the carried state and
+    adjoints at their largest) against the fp64 reference gradient, row by row."""
+    q, k, v, do = _case("bf16", 1, 1, 4096, 64, seed=11)
+    _check("bf16", q, k, v, do)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
