@@ -263,7 +263,8 @@ size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H
 
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
     if (hla_backward_workspace_bytes(op, dtype, B, H, T, d, dv) == 0) return 0;
-    return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(d, T) : hla::simt::backward_launches(d, T);
+    return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(d, T)
+                                  : hla::simt::backward_launches(dtype == HLA_BF16, d, T);
 }
 
 namespace {

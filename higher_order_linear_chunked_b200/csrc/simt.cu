@@ -1849,11 +1849,15 @@ static size_t bwd_out_smem() {
 
 size_t backward_workspace_floats(int d, int BH, int T) {
     const int NCp = next_pow2((T + C - 1) / C);
-    return workspace_floats(OP_HLA2, d, BH, T) + (size_t)BH * NCp * 3 * d * d;
+    // forward summaries, adjoint slots, and at d = 64 the 128-token prefixes of the tensor-core path
+    return workspace_floats(OP_HLA2, d, BH, T) + (size_t)BH * NCp * 3 * d * d +
+           (d == 64 ? tc::chunk_prefix_floats(BH, T) : 0);
 }
 
-int backward_launches(int d, int T) {
-    // summaries, scan, chunk terms, two suffix sums, cross term, gradients
+int backward_launches(bool bf16, int d, int T) {
+    // bf16 at d = 64: summary walker, two prefix kernels, chunk terms, two suffix sums, cross term,
+    // tensor-core gradients; otherwise summaries, the scan, the same adjoint stages, gradients
+    if (bf16 && d == 64) return 3 + 5;
     return kernel_launches(OP_HLA2, d, T) - 1 + 5;
 }
 
@@ -1864,6 +1868,8 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     const int NCp = next_pow2(NC);
     float* sums = ws;
     float* bw = ws + workspace_floats(OP_HLA2, D, BH, T);
+    float* pre128 = bw + (size_t)BH * NCp * Bwd<D>::SIZE;      // tensor-core path only
+    const bool tc_path = D == 64 && sizeof(TIn) == 2 && !fp32_only;
     auto ks = k_summary<OP_HLA2, D, TIn>;
     auto kc = k_bwd_chunk<D, TIn>;
     auto ko = k_bwd_out<D, TIn>;
@@ -1872,7 +1878,12 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
-    // the forward's carried states: chunk summaries, then their exclusive scan
+    // the forward's carried states.  Tensor-core path: the state entering every 128-token chunk,
+    // from the summary walker over one-chunk segments and the segment-prefix kernels.  Otherwise
+    // the CUDA-core chunk summaries (64 tokens) and their exclusive scan.
+    if (tc_path) {
+        if ((e = tc::chunk_prefixes(q, k, v, BH, T, sums, pre128, status, st)) != cudaSuccess) return e;
+    } else {
     ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, nullptr, 1, T, NC, NCp, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (fold_fits<OP_HLA2, D>()) {
@@ -1885,6 +1896,7 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     } else if ((e = scan_levels<OP_HLA2, D>(sums, NCp, BH, st)) != cudaSuccess) {
         return e;
     }
+    }
     kc<<<dim3(NC, BH), NT, s2, st>>>((const TIn*)q, (const TIn*)v, dout, T, NCp, bw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 sg((D * D + NT - 1) / NT, BH);
@@ -1894,10 +1906,9 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dS'
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the gradients: on the tensor cores for bf16 at d = 64 (128-token chunks, reading every other
-    // carried state and adjoint of the 64-token stages), else on the CUDA cores
-    if (D == 64 && sizeof(TIn) == 2 && !fp32_only)
-        return tc::bwd_out(q, k, v, dout, sums, bw, NC, NCp, dq, dk, dv, BH, T, status, st);
+    // the gradients: on the tensor cores for bf16 at d = 64 (128-token chunks: the adjoints of
+    // every other 64-token stage), else on the CUDA cores
+    if (tc_path) return tc::bwd_out(q, k, v, dout, pre128, bw, NC, NCp, dq, dk, dv, BH, T, status, st);
     ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
                                      dv);
     return cudaGetLastError();
@@ -1953,7 +1964,7 @@ size_t backward_normalized_workspace_floats(int d, int BH, int T) {
 
 int backward_normalized_launches(int d, int T) {
     // two plain forwards, the ones, the gradient split, two plain backwards, two additions
-    return 2 * kernel_launches(OP_HLA2, d, T) + 1 + 1 + 2 * backward_launches(d, T) + 2;
+    return 2 * kernel_launches(OP_HLA2, d, T) + 1 + 1 + 2 * backward_launches(false, d, T) + 2;
 }
 
 cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,

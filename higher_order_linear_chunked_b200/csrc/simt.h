@@ -43,7 +43,7 @@ cudaError_t step(int op, bool norm, bool bf16, int d, float* state_io, const voi
 // status: the device status word (a bounded wait that gave up sets it).  bf16 at d = 64 takes
 // the tensor-core gradient kernel for its last stage unless fp32_only.
 size_t backward_workspace_floats(int d, int BH, int T);
-int backward_launches(int d, int T);
+int backward_launches(bool bf16, int d, int T);
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
                      float* dk, float* dv, int BH, int T, float* ws, int* status, cudaStream_t st,
                      bool fp32_only = false);

@@ -28,13 +28,18 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
 size_t state_workspace_bytes(int BH, int T);
 cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, void* ws, int* status, float* state_out,
                   cudaStream_t st);
+// the carried state at every 128-token chunk (second order, bf16, d = 64): the summary walker
+// over one-chunk segments into sums, then the segment-prefix kernels into pre; both
+// [BH][next_pow2(chunks)][summary floats] (chunk_prefix_floats each); three launches
+size_t chunk_prefix_floats(int BH, int T);
+cudaError_t chunk_prefixes(const void* q, const void* k, const void* v, int BH, int T, float* sums, float* pre,
+                           int* status, cudaStream_t st);
 // backward of the masked second order, last stage (bf16, d = 64): dq, dk, dv of every 128-token
-// chunk on tcgen05, from the forward's exclusive prefix slots (sums: 64-token chunks, the
-// CUDA-core summary layout) and the adjoint slots (bw: dR', dS', C per 64-token chunk); NC64
-// 64-token chunks per head, NCp slots per head in both arrays
-cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* sums,
-                    const float* bw, int NC64, int NCp, float* dq, float* dk, float* dv, int BH, int T, int* status,
-                    cudaStream_t st);
+// chunk on tcgen05, from the exclusive prefixes of chunk_prefixes (pre) and the adjoint slots (bw:
+// dR', dS', C per 64-token chunk, NCp64 slots per head); NC64 64-token chunks per head
+cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
+                    const float* bw, int NC64, int NCp64, float* dq, float* dk, float* dv, int BH, int T,
+                    int* status, cudaStream_t st);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

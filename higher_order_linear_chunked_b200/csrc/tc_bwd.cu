@@ -75,9 +75,9 @@ constexpr uint32_t TB_A = 0, TB_DW = 128, TB_Z = 256, TB_DZ = 320, TB_DK = 384, 
 constexpr uint32_t TB_W = TB_A, TB_DA = TB_DW, TB_DV = TB_Z;
 
 struct BwdParams {
-    int T, NC64, NCp;
-    const float* sums;   // forward prefix slots (64-token chunks): S0 = mat 0, R0 = mat 2
-    const float* bw;     // adjoint slots (64-token chunks): dR' = 0, dS' = 1
+    int T, NC64, NCp64, NSp;
+    const float* pre;    // exclusive prefixes per 128-token chunk (NSp slots per head): S0 = mat 0, R0 = mat 2
+    const float* bw;     // adjoint slots per 64-token chunk (NCp64 per head): dR' = 0, dS' = 1
     int* status;
 };
 
@@ -137,13 +137,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
         ptx::tmem_alloc(tmem_slot, TB_COLS);
         ptx::tmem_relinquish();
     }
-    // carried state (64-token chunk 2c) and adjoints leaving the chunk (64-token chunk 2c + 1, or
-    // none after the sequence's last chunk) as bf16 tiles, while the loads are in flight
+    // carried state (prefix of the chunk) and adjoints leaving the chunk (64-token chunk 2c + 1,
+    // or none after the sequence's last chunk) as bf16 tiles, while the loads are in flight
     {
-        const float* pre = p.sums + ((size_t)bh * p.NCp + 2 * chunk) * simt_layout::size;
+        const float* pre = p.pre + ((size_t)bh * p.NSp + chunk) * simt_layout::size;
         const int ca = 2 * chunk + 1;
         const bool has_adj = ca < p.NC64;
-        const float* adj = p.bw + ((size_t)bh * p.NCp + (has_adj ? ca : 0)) * BW_SIZE;
+        const float* adj = p.bw + ((size_t)bh * p.NCp64 + (has_adj ? ca : 0)) * BW_SIZE;
         mat_tile(sm + SB_S0, pre + simt_layout::mat(0), false, false);
         mat_tile(sm + SB_R0, pre + simt_layout::mat(2), false, false);
         mat_tile(sm + SB_GR, adj, false, !has_adj);
@@ -355,9 +355,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
 
 }  // namespace
 
-cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* sums,
-                    const float* bw, int NC64, int NCp, float* dq, float* dk, float* dv, int BH, int T, int* status,
-                    cudaStream_t st) {
+cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
+                    const float* bw, int NC64, int NCp64, float* dq, float* dk, float* dv, int BH, int T,
+                    int* status, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mdo, const_cast<float*>(dout), T, BH) || !make_map_out(&mdq, dq, T, BH) ||
@@ -366,8 +366,11 @@ cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* do
     BwdParams prm;
     prm.T = T;
     prm.NC64 = NC64;
-    prm.NCp = NCp;
-    prm.sums = sums;
+    prm.NCp64 = NCp64;
+    int nsp = 1;
+    while (nsp < (T + C - 1) / C) nsp *= 2;
+    prm.NSp = nsp;
+    prm.pre = pre;
     prm.bw = bw;
     prm.status = status;
     cudaError_t e = set_smem(k_bwd_tc, (int)BSMEM_BYTES);

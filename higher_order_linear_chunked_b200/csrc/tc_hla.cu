@@ -1018,6 +1018,28 @@ cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, vo
     return cudaGetLastError();
 }
 
+size_t chunk_prefix_floats(int BH, int T) {
+    return (size_t)BH * next_pow2((T + C - 1) / C) * simt_layout::size;
+}
+
+cudaError_t chunk_prefixes(const void* q, const void* k, const void* v, int BH, int T, float* sums, float* pre,
+                           int* status, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
+        !make_map_out(&mo, pre, 1, 1))
+        return cudaErrorInvalidValue;
+    const int NS = (T + C - 1) / C;          // one chunk per summary segment
+    Params sprm{};
+    sprm.T = T; sprm.BH = BH; sprm.NCH = 1; sprm.NS = NS; sprm.NSp = next_pow2(NS); sprm.ratio = 1;
+    sprm.sums = sums;
+    sprm.status = status;
+    cudaError_t e;
+    if ((e = set_smem(k_walk<SUMMARY>, SMEM_BYTES)) != cudaSuccess) return e;
+    k_walk<SUMMARY><<<dim3(NS, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_prefix(sums, pre, NS, sprm.NSp, BH, st);
+}
+
 bool set_segment_chunks(int chunks) {
     if (chunks != 0 && chunks != 1 && chunks != 2 && chunks != 4 && chunks != 8 && chunks != 16) return false;
     g_segment_chunks.store(chunks);

@@ -263,12 +263,16 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
  * hla2_backward: given the output gradient dout [B][H][T][dv] (fp32, device),
  * writes dq, dk [B][H][T][d] and dv_out [B][H][T][dv] (fp32, device, caller-
  * owned, 16-byte aligned) for the forward hla2_forward(q, k, v) of the same
- * inputs (HLA_F32 or HLA_BF16; bf16 values are widened, all arithmetic is
- * fp32).  The forward's carried chunk states are recomputed from q, k, v (no
- * saved activations).  Kernels: the forward's chunk summaries and scan, then
+ * inputs (HLA_F32 or HLA_BF16).  The forward's carried chunk states are
+ * recomputed from q, k, v (no saved activations).  Kernels: the carried states,
  * per-chunk adjoint terms, two suffix sums and the per-chunk gradients (see
- * hla_backward_kernel_launches).  Errors as for the forward calls; a non-NULL
- * gamma is HLA_ERR_UNSUPPORTED.  Enqueued on `stream`, asynchronous.
+ * hla_backward_kernel_launches).  Arithmetic: fp32 on the CUDA cores, except
+ * for HLA_BF16 at d = 64, where the carried states come from the tensor-core
+ * summary walker and the per-chunk gradients from a tensor-core kernel with
+ * bf16 operands and fp32 accumulation (dout and the intermediate dZ enter as
+ * two bf16 terms each); its gradient carries about 2e-3 of the gradient's norm
+ * as rounding.  Errors as for the forward calls; a non-NULL gamma is
+ * HLA_ERR_UNSUPPORTED.  Enqueued on `stream`, asynchronous.
  */
 size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
@@ -282,7 +286,8 @@ hla_status_t hla2_backward(const void* q, const void* k, const void* v, const fl
  * denominator is the same masked operator on a ones value column, so the gradient is the plain
  * backward with dout / (den + eps), plus the plain backward on the ones column with the per-row
  * output gradient -sum_f dout_f num_f / (den + eps)^2 (its dq and dk).  num and den are
- * recomputed by two plain fp32 forwards.  Workspace: hla_backward_workspace_bytes(
+ * recomputed by two plain forwards; both backward passes keep the fp32 gradient kernel (their
+ * dq and dk terms nearly cancel where o barely depends on q, k).  Workspace: hla_backward_workspace_bytes(
  * HLA_OP_HLA2_NORM, ...), about 8 B*H*T*d floats more than the plain backward's.
  */
 hla_status_t hla2_backward_normalized(const void* q, const void* k, const void* v, const float* dout, float* dq,
