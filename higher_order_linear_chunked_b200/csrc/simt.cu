@@ -1856,7 +1856,8 @@ size_t backward_workspace_floats(int d, int BH, int T) {
 
 int backward_launches(bool bf16, int d, int T) {
     // bf16 at d = 64: summary walker, two prefix kernels, chunk terms, two suffix sums, cross term,
-    // tensor-core gradients; otherwise summaries, the scan, the same adjoint stages, gradients
+    // gradients (128-token chunks); otherwise summaries, the scan, the same adjoint stages (64-token
+    // chunks), gradients
     if (bf16 && d == 64) return 3 + 5;
     return kernel_launches(OP_HLA2, d, T) - 1 + 5;
 }
@@ -1868,22 +1869,32 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     const int NCp = next_pow2(NC);
     float* sums = ws;
     float* bw = ws + workspace_floats(OP_HLA2, D, BH, T);
-    float* pre128 = bw + (size_t)BH * NCp * Bwd<D>::SIZE;      // tensor-core path only
-    const bool tc_path = D == 64 && sizeof(TIn) == 2 && !fp32_only;
+    cudaError_t e;
+    if (D == 64 && sizeof(TIn) == 2 && !fp32_only) {
+        // tensor-core path, 128-token chunks throughout: the state entering every chunk (summary
+        // walker over one-chunk segments, segment-prefix kernels), the adjoint terms, their
+        // suffix sums and cross term (CUDA cores), the gradients
+        float* pre = bw + (size_t)BH * NCp * Bwd<D>::SIZE;
+        const int NC2 = (T + 127) / 128, NSp2 = next_pow2(NC2);
+        if ((e = tc::chunk_prefixes(q, k, v, BH, T, sums, pre, status, st)) != cudaSuccess) return e;
+        if ((e = tc::bwd_terms(q, v, dout, bw, BH, T, status, st)) != cudaSuccess) return e;
+        const dim3 sg2((D * D + NT - 1) / NT, BH);
+        k_bwd_suffix<D><<<sg2, NT, 0, st>>>(bw, NC2, NSp2, 0);                // dR'
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_bwd_cross<D><<<dim3(NC2, BH), NT, 0, st>>>(bw, NSp2);                // X = U + C dR'^T
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_bwd_suffix<D><<<sg2, NT, 0, st>>>(bw, NC2, NSp2, 1);                // dS'
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        return tc::bwd_out(q, k, v, dout, pre, bw, dq, dk, dv, BH, T, status, st);
+    }
     auto ks = k_summary<OP_HLA2, D, TIn>;
     auto kc = k_bwd_chunk<D, TIn>;
     auto ko = k_bwd_out<D, TIn>;
     const size_t s1 = summary_smem<D>(), s2 = bwd_chunk_smem<D>(), s3 = bwd_out_smem<D>();
-    cudaError_t e;
     if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
-    // the forward's carried states.  Tensor-core path: the state entering every 128-token chunk,
-    // from the summary walker over one-chunk segments and the segment-prefix kernels.  Otherwise
-    // the CUDA-core chunk summaries (64 tokens) and their exclusive scan.
-    if (tc_path) {
-        if ((e = tc::chunk_prefixes(q, k, v, BH, T, sums, pre128, status, st)) != cudaSuccess) return e;
-    } else {
+    // the forward's carried states: chunk summaries, then their exclusive scan
     ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, nullptr, 1, T, NC, NCp, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (fold_fits<OP_HLA2, D>()) {
@@ -1896,7 +1907,6 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     } else if ((e = scan_levels<OP_HLA2, D>(sums, NCp, BH, st)) != cudaSuccess) {
         return e;
     }
-    }
     kc<<<dim3(NC, BH), NT, s2, st>>>((const TIn*)q, (const TIn*)v, dout, T, NCp, bw);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 sg((D * D + NT - 1) / NT, BH);
@@ -1906,9 +1916,6 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dS'
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the gradients: on the tensor cores for bf16 at d = 64 (128-token chunks: the adjoints of
-    // every other 64-token stage), else on the CUDA cores
-    if (tc_path) return tc::bwd_out(q, k, v, dout, pre128, bw, NC, NCp, dq, dk, dv, BH, T, status, st);
     ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
                                      dv);
     return cudaGetLastError();

@@ -34,12 +34,16 @@ cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, vo
 size_t chunk_prefix_floats(int BH, int T);
 cudaError_t chunk_prefixes(const void* q, const void* k, const void* v, int BH, int T, float* sums, float* pre,
                            int* status, cudaStream_t st);
-// backward of the masked second order, last stage (bf16, d = 64): dq, dk, dv of every 128-token
-// chunk on tcgen05, from the exclusive prefixes of chunk_prefixes (pre) and the adjoint slots (bw:
-// dR', dS', C per 64-token chunk, NCp64 slots per head); NC64 64-token chunks per head
+// backward of the masked second order (bf16, d = 64), 128-token chunks, slots
+// [BH][next_pow2(chunks)][3 d d] (fp32):
+//   bwd_terms: Y = Q^T dO, U = Q^T (dW Q), C = Q^T V of every chunk into its slot [Y | U | C];
+//   bwd_out:   dq, dk, dv of every chunk from the exclusive prefixes of chunk_prefixes (pre) and
+//              the slots after the suffix sums (bw: dR', dS')
+cudaError_t bwd_terms(const void* q, const void* v, const float* dout, float* terms, int BH, int T, int* status,
+                      cudaStream_t st);
 cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
-                    const float* bw, int NC64, int NCp64, float* dq, float* dk, float* dv, int BH, int T,
-                    int* status, cudaStream_t st);
+                    const float* bw, float* dq, float* dk, float* dv, int BH, int T, int* status,
+                    cudaStream_t st);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

@@ -75,9 +75,10 @@ constexpr uint32_t TB_A = 0, TB_DW = 128, TB_Z = 256, TB_DZ = 320, TB_DK = 384, 
 constexpr uint32_t TB_W = TB_A, TB_DA = TB_DW, TB_DV = TB_Z;
 
 struct BwdParams {
-    int T, NC64, NCp64, NSp;
-    const float* pre;    // exclusive prefixes per 128-token chunk (NSp slots per head): S0 = mat 0, R0 = mat 2
-    const float* bw;     // adjoint slots per 64-token chunk (NCp64 per head): dR' = 0, dS' = 1
+    int T, NSp;
+    const float* pre;    // exclusive prefixes per chunk (NSp slots per head): S0 = mat 0, R0 = mat 2
+    const float* bw;     // adjoint slots per chunk (NSp per head): dR' = 0, dS' = 1 (exclusive suffixes)
+    float* terms;        // k_bwd_terms: the slots [Y | U | C] it writes
     int* status;
 };
 
@@ -137,17 +138,15 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
         ptx::tmem_alloc(tmem_slot, TB_COLS);
         ptx::tmem_relinquish();
     }
-    // carried state (prefix of the chunk) and adjoints leaving the chunk (64-token chunk 2c + 1,
-    // or none after the sequence's last chunk) as bf16 tiles, while the loads are in flight
+    // carried state (the chunk's exclusive prefix) and the adjoints leaving the chunk (the
+    // exclusive suffixes) as bf16 tiles, while the loads are in flight
     {
         const float* pre = p.pre + ((size_t)bh * p.NSp + chunk) * simt_layout::size;
-        const int ca = 2 * chunk + 1;
-        const bool has_adj = ca < p.NC64;
-        const float* adj = p.bw + ((size_t)bh * p.NCp64 + (has_adj ? ca : 0)) * BW_SIZE;
+        const float* adj = p.bw + ((size_t)bh * p.NSp + chunk) * BW_SIZE;
         mat_tile(sm + SB_S0, pre + simt_layout::mat(0), false, false);
         mat_tile(sm + SB_R0, pre + simt_layout::mat(2), false, false);
-        mat_tile(sm + SB_GR, adj, false, !has_adj);
-        mat_tile(sm + SB_GS, adj + D * D, true, !has_adj);
+        mat_tile(sm + SB_GR, adj, false, false);
+        mat_tile(sm + SB_GS, adj + D * D, true, false);
     }
     // the loads: every thread waits (bounded), then dO (fp32 boxes) -> bf16 tile
     bool ok = ptx::mbar_wait(bar_load, 0);
@@ -353,23 +352,217 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
     if (warp == 1) ptx::tmem_dealloc(tmem, TB_COLS);
 }
 
+// ---------------------------------------------------------------- adjoint terms
+// Per 128-token chunk, the terms of the adjoint recurrences of the state (exclusive suffix sums
+// of them, taken by the CUDA-core kernels, give dR' and dS'):
+//     Y = Q^T dO,   C = Q^T V,   U = Q^T (dW Q),   dW = L (.) dO V^T,
+// as fp32 64 x 64 matrices into the chunk's slot [Y | U | C].  The Q^T products are one M = 128
+// product each over the Q and V tiles stacked ([Q^T ; V^T] X; rows 0-63 kept).  Three rounds:
+// dO enters as two bf16 terms (hi + lo), as in the gradient kernel: Y feeds dR' and every dq.
+//   R1: dW* = dO V^T, [Y ; .] = [Q^T ; V^T] dO, [C ; .] = [Q^T ; V^T] V  -> E1: dW masked to bf16
+//   R2: G = dW Q                                                           -> E2: G to bf16
+//   R3: [U ; .] = [Q^T ; V^T] G                                             -> E3: Y, U, C stored
+constexpr uint32_t SA_Q = 0, SA_V = TILE, SA_O = 2 * TILE, SA_OL = 3 * TILE, SA_DW = 4 * TILE;
+constexpr uint32_t SA_BAR = 6 * TILE;
+constexpr uint32_t TSMEM_BYTES = SA_BAR + 64 + 1024;
+constexpr uint32_t SA_OF = SA_DW;               // dO (fp32 boxes) before dW is written
+constexpr uint32_t SA_G = SA_O;                 // G over dO (read by R1 only)
+constexpr uint32_t TT_DW = 0, TT_G = 0, TT_U = 64, TT_Y = 128, TT_C = 192, TT_COLS = 256;
+
+__global__ void __launch_bounds__(BNT, 2)
+k_bwd_terms(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tv,
+            const __grid_constant__ CUtensorMap tdo, BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + SA_BAR);
+    uint64_t* bar_mma = bar_load + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int t0 = chunk * C;
+    if (tid == 0) {
+        ptx::mbar_init(bar_load, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(bar_load, 4 * TILE);
+        ptx::tma_load_3d(sm + SA_Q, &tq, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + SA_V, &tv, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + SA_OF, &tdo, bar_load, 0, t0, bh);
+        ptx::tma_load_3d(sm + SA_OF + C * 128, &tdo, bar_load, 32, t0, bh);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, TT_COLS);
+        ptx::tmem_relinquish();
+    }
+    bool ok = ptx::mbar_wait(bar_load, 0);
+    {
+        const float4* box = reinterpret_cast<const float4*>(sm + SA_OF + half * (C * 128) + row * 128);
+        float x[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 f = box[j ^ (row & 7)];
+            x[4 * j] = f.x; x[4 * j + 1] = f.y; x[4 * j + 2] = f.z; x[4 * j + 3] = f.w;
+        }
+        split_row(sm + SA_O, sm + SA_OL, row, half * 32, x);
+    }
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    ok = __syncthreads_and(ok) != 0;
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    constexpr uint32_t I_128_KK = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t I_64_KM = ptx::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t I_64_MM = ptx::idesc_bf16(128, 64, true, true);
+    auto k1 = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 2); };
+    auto k2 = [](uint64_t d0, int s) { return d0 + (uint64_t)(((s >> 2) * TILE + (s & 3) * 32) >> 4); };
+    auto mn = [](uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); };
+    const uint64_t dQV = mdesc(sb + SA_Q, SA_V - SA_Q, 0);      // [Q^T ; V^T], MN-major, M = 128
+    auto stacked = [&](uint32_t d, uint32_t b, bool acc) {        // [Q^T ; V^T] X, X a [tok][64] tile
+        const uint64_t db = mdesc(sb + b, TILE, 0);
+        for (int s = 0; s < 8; ++s)
+            ptx::umma_bf16(tmem + d, mn(dQV, s), mn(db, s), I_64_MM, (acc || s > 0) ? 1u : 0u);
+    };
+    uint32_t mma_phase = 0;
+    auto commit_wait = [&]() -> bool {
+        bool good = true;
+        ptx::tc_fence_before();
+        if (tid == 0) {
+            ptx::umma_commit(bar_mma);
+            good = ptx::mbar_wait(bar_mma, mma_phase);
+        }
+        mma_phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
+    auto sync_for_mma = [&]() {
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+    };
+    int round = 0;
+    if (ok) {
+        if (tid == 0) {                      // R1
+            const uint64_t dO = kdesc(sb + SA_O, 0), dOL = kdesc(sb + SA_OL, 0), dV = kdesc(sb + SA_V, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TT_DW, k1(dO, s), k1(dV, s), I_128_KK, s > 0 ? 1u : 0u);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + TT_DW, k1(dOL, s), k1(dV, s), I_128_KK, 1u);
+            stacked(TT_Y, SA_O, false);
+            stacked(TT_Y, SA_OL, true);
+            stacked(TT_C, SA_V, false);
+        }
+        round = 1;
+        ok = commit_wait();
+    }
+    if (ok) {
+        // E1: dW masked (j <= t) to the K-major [t][j] tile
+        const int b0 = 2 * half;
+        float v0[32], v1[32];
+        if (b0 + 1 <= quad) {
+            ptx::tmem_ld32x2(tmem + lane_base + TT_DW + 32 * b0, tmem + lane_base + TT_DW + 32 * (b0 + 1), v0, v1);
+            if (b0 + 1 == quad) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i > lane) v1[i] = 0.f;
+            }
+            st_row32(sm + SA_DW, row, 32 * b0, v0);
+            st_row32(sm + SA_DW, row, 32 * (b0 + 1), v1);
+        } else if (b0 == quad) {
+            ptx::tmem_ld32(tmem + lane_base + TT_DW + 32 * b0, v0);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (i > lane) v0[i] = 0.f;
+            st_row32(sm + SA_DW, row, 32 * b0, v0);
+            st_row32_zero(sm + SA_DW, row, 32 * (b0 + 1));
+        } else {
+            st_row32_zero(sm + SA_DW, row, 32 * b0);
+            st_row32_zero(sm + SA_DW, row, 32 * (b0 + 1));
+        }
+        sync_for_mma();
+        if (tid == 0) {                      // R2: G = dW Q
+            const uint64_t dA = kdesc2(sb + SA_DW, 0), dB = mdesc(sb + SA_Q, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + TT_G, k2(dA, s), mn(dB, s), I_64_KM, s > 0 ? 1u : 0u);
+        }
+        round = 2;
+        ok = commit_wait();
+    }
+    if (ok) {
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + TT_G + 32 * half, v);
+        st_row32(sm + SA_G, row, 32 * half, v);
+        sync_for_mma();
+        if (tid == 0) stacked(TT_U, SA_G, false);   // R3
+        round = 3;
+        ok = commit_wait();
+    }
+    if (ok && quad < 2) {
+        // E3: rows 0-63 (Q features) of Y, U, C into the slot, this thread's half row of each
+        float* slot = p.terms + ((size_t)bh * p.NSp + chunk) * BW_SIZE;
+        const uint32_t cols[3] = {TT_Y, TT_U, TT_C};
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+            float v[32];
+            ptx::tmem_ld32(tmem + lane_base + cols[m] + 32 * half, v);
+            float4* dst = reinterpret_cast<float4*>(slot + m * D * D + row * D + 32 * half);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+    }
+    if (!ok && tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        ptx::mbar_wait(bar_load, 0, 100000000ull);
+        if (round > 0) {
+            ptx::umma_commit(bar_mma);
+            ptx::mbar_wait(bar_mma, mma_phase, 100000000ull);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, TT_COLS);
+}
+
 }  // namespace
 
+static int slots_per_head(int T) {
+    int n = 1;
+    while (n < (T + C - 1) / C) n *= 2;
+    return n;
+}
+
+cudaError_t bwd_terms(const void* q, const void* v, const float* dout, float* terms, int BH, int T, int* status,
+                      cudaStream_t st) {
+    CUtensorMap mq, mv, mdo;
+    if (!make_map(&mq, q, T, BH) || !make_map(&mv, v, T, BH) || !make_map_out(&mdo, const_cast<float*>(dout), T, BH))
+        return cudaErrorInvalidValue;
+    BwdParams prm{};
+    prm.T = T;
+    prm.NSp = slots_per_head(T);
+    prm.terms = terms;
+    prm.status = status;
+    cudaError_t e = set_smem(k_bwd_terms, (int)TSMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    k_bwd_terms<<<dim3((T + C - 1) / C, BH), BNT, TSMEM_BYTES, st>>>(mq, mv, mdo, prm);
+    return cudaGetLastError();
+}
+
 cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
-                    const float* bw, int NC64, int NCp64, float* dq, float* dk, float* dv, int BH, int T,
-                    int* status, cudaStream_t st) {
+                    const float* bw, float* dq, float* dk, float* dv, int BH, int T, int* status,
+                    cudaStream_t st) {
     CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mdo, const_cast<float*>(dout), T, BH) || !make_map_out(&mdq, dq, T, BH) ||
         !make_map_out(&mdk, dk, T, BH) || !make_map_out(&mdv, dv, T, BH))
         return cudaErrorInvalidValue;
-    BwdParams prm;
+    BwdParams prm{};
     prm.T = T;
-    prm.NC64 = NC64;
-    prm.NCp64 = NCp64;
-    int nsp = 1;
-    while (nsp < (T + C - 1) / C) nsp *= 2;
-    prm.NSp = nsp;
+    prm.NSp = slots_per_head(T);
     prm.pre = pre;
     prm.bw = bw;
     prm.status = status;
