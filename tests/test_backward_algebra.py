@@ -128,6 +128,54 @@ def test_chunked_reverse_walk_matches_the_reference(T, c):
         np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
 
 
+def z_form_backward(q, k, v, do, c):
+    """The tensor-core gradient stage's algebra, chunk-parallel: carried (S0, R0) by the forward's
+    exclusive prefixes; the adjoints leaving each chunk by exclusive suffix sums of its terms
+        Y = Q^T dO,  U = Q^T (dW Q),  C = Q^T V:   dR'(c) = sum_{m>c} Y_m,
+        dS'(c) = sum_{m>c} (U_m + C_m dR'(m)^T);
+    then per chunk, in the Z form (Z = Q S0 + A K, W = L (.) Q Z^T):
+        dW = L (.) dO V^T,  dZ = dW^T Q + V dR'^T,  dA = L (.) dZ K^T,
+        dQ = dO R0^T + dZ S0 + dW Z + dA K,  dK = K (dS' + dS'^T) + A^T dZ + dA^T Q,
+        dV = W^T dO + Z dR'."""
+    d, dv = q.shape[1], v.shape[1]
+    Qs, Ks, Vs, Gs = chunks(q, c), chunks(k, c), chunks(v, c), chunks(do, c)
+    n = len(Qs)
+    L = np.tril(np.ones((c, c)))
+    S0s, R0s = [], []
+    S0, R0 = np.zeros((d, d)), np.zeros((d, dv))
+    for Q, K, V in zip(Qs, Ks, Vs):
+        S0s.append(S0); R0s.append(R0)
+        Z = Q @ S0 + (L * (Q @ K.T)) @ K
+        S0, R0 = S0 + K.T @ K, R0 + Z.T @ V
+    Y = [Q.T @ dO for Q, dO in zip(Qs, Gs)]
+    U = [Q.T @ ((L * (dO @ V.T)) @ Q) for Q, V, dO in zip(Qs, Vs, Gs)]
+    Cm = [Q.T @ V for Q, V in zip(Qs, Vs)]
+    dR = [sum((Y[m] for m in range(i + 1, n)), np.zeros((d, dv))) for i in range(n)]
+    dS = [sum((U[m] + Cm[m] @ dR[m].T for m in range(i + 1, n)), np.zeros((d, d))) for i in range(n)]
+    gq, gk, gv = [], [], []
+    for i, (Q, K, V, dO) in enumerate(zip(Qs, Ks, Vs, Gs)):
+        A = L * (Q @ K.T)
+        Z = Q @ S0s[i] + A @ K
+        W = L * (Q @ Z.T)
+        dW = L * (dO @ V.T)
+        dZ = dW.T @ Q + V @ dR[i].T
+        dA = L * (dZ @ K.T)
+        gq.append(dO @ R0s[i].T + dZ @ S0s[i] + dW @ Z + dA @ K)
+        gk.append(K @ (dS[i] + dS[i].T) + A.T @ dZ + dA.T @ Q)
+        gv.append(W.T @ dO + Z @ dR[i])
+    T = q.shape[0]
+    return (np.vstack(gq)[:T], np.vstack(gk)[:T], np.vstack(gv)[:T])
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (7, 4), (16, 4), (37, 8), (64, 16), (100, 32), (300, 128)])
+def test_z_form_chunk_parallel_gradients_match_the_reference(T, c):
+    q, k, v, do = rand(T, 5, 3, T + 3 * c)
+    want = hla2_grads(q, k, v, do)
+    got = z_form_backward(q, k, v, do, c)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+
+
 @pytest.mark.parametrize("drop", ["dS", "dR"])
 def test_reverse_walk_needs_both_carried_adjoints(drop):
     """Withholding either carried adjoint breaks the gradients once there are several chunks
