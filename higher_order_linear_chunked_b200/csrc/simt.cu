@@ -1855,10 +1855,10 @@ size_t backward_workspace_floats(int d, int BH, int T) {
 }
 
 int backward_launches(bool bf16, int d, int T) {
-    // bf16 at d = 64: summary walker, two prefix kernels, chunk terms, two suffix sums, cross term,
-    // gradients (128-token chunks); otherwise summaries, the scan, the same adjoint stages (64-token
-    // chunks), gradients
-    if (bf16 && d == 64) return 3 + 5;
+    // bf16 at d = 64: summary walker, three prefix kernels, chunk terms, two suffix sums, cross
+    // term, gradients (128-token chunks); otherwise summaries, the scan, the same adjoint stages
+    // (64-token chunks), gradients
+    if (bf16 && d == 64) return 4 + 5;
     return kernel_launches(OP_HLA2, d, T) - 1 + 5;
 }
 

@@ -30,7 +30,7 @@ cudaError_t state(const void* q, const void* k, const void* v, int BH, int T, vo
                   cudaStream_t st);
 // the carried state at every 128-token chunk (second order, bf16, d = 64): the summary walker
 // over one-chunk segments into sums, then the segment-prefix kernels into pre; both
-// [BH][next_pow2(chunks)][summary floats] (chunk_prefix_floats each); three launches
+// [BH][next_pow2(chunks)][summary floats] (chunk_prefix_floats each); four launches
 size_t chunk_prefix_floats(int BH, int T);
 cudaError_t chunk_prefixes(const void* q, const void* k, const void* v, int BH, int T, float* sums, float* pre,
                            int* status, cudaStream_t st);

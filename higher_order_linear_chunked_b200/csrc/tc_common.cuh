@@ -134,7 +134,8 @@ Plan plan(int BH, int T, int slots, int seg_chunks);
 constexpr int PH_MAX = 9;
 
 // Exclusive segment prefixes of the summaries (slot layout simt_layout): `pre` gets, for
-// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Two launches.
+// every segment l, (S0(l), m0(l)) and the corrected (R0(l), r0(l)).  Three launches: running
+// sums of S and m, the cross term per segment, running sums of the corrected R and r.
 // left_vec: the vector of the second slot is a row on the left of the first factor's
 // partner (ratio-normalised AHLA: n_AB = n_A + n_B + D_B mK_A, D^T in the C place) instead of
 // the second order's r_AB = r_A + r_B + S_A m_B.

@@ -685,10 +685,35 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
 // prefix of the corrected R.  Both prefixes are plain sums, so every segment and every
 // matrix element runs in parallel; the result equals the Blelloch tree's (up to the
 // order of fp32 additions).
-//   k_prefix_cross (one CTA per segment x head): S0(l), m0(l) by summation, then
-//       Y_l = R_l + S0(l) C_l and y_l = r_l + S0(l) m_l, written to the prefix slot l;
+//   k_prefix_run (one thread per element of S and m): S0(l), m0(l) as running sums into the
+//       prefix slots;
+//   k_prefix_cross (one CTA per segment x head): Y_l = R_l + S0(l) C_l and
+//       y_l = r_l + S0(l) m_l, written to the prefix slot l;
 //   k_prefix_sum (one thread per matrix element): R0(n) = sum_{l<n} Y_l in place.
 constexpr int PX_NT = 256;
+
+// S0(l) = sum_{m<l} S_m and m0(l) likewise, element-wise running sums (eight loads in flight).
+__global__ void __launch_bounds__(PX_NT) k_prefix_run(const float* __restrict__ sums, float* __restrict__ pre, int NS,
+                                                      int NSp) {
+    using S = simt_layout;
+    const int e = blockIdx.x * PX_NT + threadIdx.x;     // element of the S | m region
+    if (e >= D * D + D) return;
+    const int off = e < D * D ? S::mat(0) + e : S::vec(0) + (e - D * D);
+    const size_t base = (size_t)blockIdx.y * NSp * S::size + off;
+    float run = 0.f;
+    for (int l0 = 0; l0 < NS; l0 += 8) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NS) y[i] = sums[base + (size_t)(l0 + i) * S::size];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (l0 + i < NS) {
+                pre[base + (size_t)(l0 + i) * S::size] = run;
+                run += y[i];
+            }
+    }
+}
 
 __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict__ sums, float* __restrict__ pre,
                                                         int NSp, int left_vec) {
@@ -699,22 +724,11 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict_
     const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const float* sb = sums + (size_t)bh * NSp * S::size;
     float* out = pre + ((size_t)bh * NSp + l) * S::size;
-    // S0(l) = sum_{m<l} S_m : this thread owns float4 items tid + 256 i (i < 4)
+    // S0(l), m0(l): from k_prefix_run, this thread's float4 items tid + 256 i (i < 4)
     float4 acc[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int m = 0; m < l; ++m) {
-        const float4* src = reinterpret_cast<const float4*>(sb + (size_t)m * S::size + S::mat(0));
-        float4 x[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = src[tid + PX_NT * i];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = make_float4(acc[i].x + x[i].x, acc[i].y + x[i].y, acc[i].z + x[i].z,
-                                                         acc[i].w + x[i].w);
-    }
-    float m0 = 0.f;
-    if (tid < D)
-        for (int m = 0; m < l; ++m) m0 += sb[(size_t)m * S::size + S::vec(0) + tid];
+    for (int i = 0; i < 4; ++i) acc[i] = reinterpret_cast<const float4*>(out + S::mat(0))[tid + PX_NT * i];
+    const float m0 = tid < D ? out[S::vec(0) + tid] : 0.f;
     {
         const float* cl = sb + (size_t)l * S::size;
         float4 c[4];
@@ -726,12 +740,10 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_cross(const float* __restrict_
             const int f = tid + PX_NT * i, r = f >> 4, c4 = f & 15;
             *reinterpret_cast<float4*>(S0s + r * (D + 4) + 4 * c4) = acc[i];
             reinterpret_cast<float4*>(Cs)[f] = c[i];
-            reinterpret_cast<float4*>(out + S::mat(0))[f] = acc[i];          // S0(l)
         }
         if (tid < D) {
             ms[tid] = mv;
             m0s[tid] = m0;
-            out[S::vec(0) + tid] = m0;                                       // m0(l)
         }
     }
     __syncthreads();
@@ -963,8 +975,11 @@ Plan plan(int BH, int T, int slots, int seg_chunks) {
 }
 
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st, bool left_vec) {
-    k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp, left_vec ? 1 : 0);
+    k_prefix_run<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(sums, pre, NS, NSp);
     cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_prefix_cross<<<dim3(NS, BH), PX_NT, 0, st>>>(sums, pre, NSp, left_vec ? 1 : 0);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_prefix_sum<<<dim3((D * D + D + PX_NT - 1) / PX_NT, BH), PX_NT, 0, st>>>(pre, NS, NSp);
     return cudaGetLastError();
@@ -1067,10 +1082,10 @@ size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks) {
 int kernel_launches(int op, bool norm, int BH, int T, int seg_chunks) {
     if (op == OP_HLA2D) return decay_kernel_launches();
     // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
-    // two launches), output walk
+    // three launches), output walk
     const bool ahla = op == OP_AHLA || op == OP_AHLAD;
     const Plan pl = plan(BH, T, ahla ? ahla_ctas_per_sm(norm) * kSMs : kSMs, seg_chunks);
-    return pl.NSf + 1 > PH_MAX ? 4 : 2;     // else the output walker folds the prefix itself
+    return pl.NSf + 1 > PH_MAX ? 5 : 2;     // else the output walker folds the prefix itself
 }
 
 cudaError_t forward(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma, float eps,
