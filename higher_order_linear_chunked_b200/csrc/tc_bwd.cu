@@ -22,7 +22,8 @@
 //       (dO: the two-term split below; dZ likewise)
 //   R2: Z += A K, dZ = dW^T Q + V G_R^T               -> E2: Z, dZ to bf16 tiles
 //   R3: W* = Q Z^T, dA* = dZ K^T,
-//       dK = K G_Ssym + A^T dZ, dQ = dO R0^T + dZ S0  -> E3: W (over A), dA (over dZ, S0, G_Ssym)
+//       dK = K (G_S^T + G_S) + A^T dZ,                -> E3: W (over A), dA (over dZ, S0, G_S)
+//       dQ = dO R0^T + dZ S0   (G_S read K-major and MN-major: no transposed copy)
 //   R4: dV = W^T dO + Z G_R, dQ += dW Z + dA K, dK += dA^T Q
 //                                                     -> E4: dQ, dK, dV staged, TMA stores
 // TMEM (512 columns): A* / W* 0-127, dW* / dA* 128-255, Z / dV 256-319, dZ 320-383, dK 384-447,
@@ -60,7 +61,7 @@ constexpr uint32_t SB_DW = SB_A + 2 * TILE;     // dW masked
 constexpr uint32_t SB_Z = SB_DW + 2 * TILE;     // Z   [tok][64]
 constexpr uint32_t SB_DZ = SB_Z + TILE;         // dZ  [tok][64]      } after R3: dA (two atoms)
 constexpr uint32_t SB_S0 = SB_DZ + TILE;        // S0  [64][64]       }
-constexpr uint32_t SB_GS = SB_S0 + MAT;         // G_S + G_S^T        }
+constexpr uint32_t SB_GS = SB_S0 + MAT;         // G_S                }
 constexpr uint32_t SB_DZL = SB_GS + MAT;        // dZ - hi (lo)
 constexpr uint32_t SB_R0 = SB_DZL + TILE;       // R0  [64][64]
 constexpr uint32_t SB_GR = SB_R0 + MAT;         // G_R [64][64]
@@ -82,17 +83,25 @@ struct BwdParams {
     int* status;
 };
 
-// 64 x 64 fp32 row-major matrix (global) -> bf16 K-major tile (row r, 128-byte swizzle); sym:
-// the matrix plus its transpose.  Thread t converts row t / 4, columns 16 (t % 4) .. + 15.
-__device__ __forceinline__ void mat_tile(uint8_t* tile, const float* m, bool sym, bool zero) {
+// Four 64 x 64 fp32 row-major matrices (global) -> bf16 K-major tiles (128-byte swizzle).  Thread
+// t converts row t / 4, columns 16 (t % 4) .. + 15 of each; all sixteen 16-byte loads are issued
+// before the first conversion.
+__device__ __forceinline__ void mat_tiles4(uint8_t* const (&tiles)[4], const float* const (&m)[4]) {
     const int r = threadIdx.x >> 2, c0 = 16 * (threadIdx.x & 3);
-    float v[16];
+    float4 x[4][4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        v[i] = zero ? 0.f : m[r * D + c0 + i];
-        if (sym && !zero) v[i] += m[(c0 + i) * D + r];
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[j][i] = reinterpret_cast<const float4*>(m[j] + r * D + c0)[i];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[4 * i] = x[j][i].x; v[4 * i + 1] = x[j][i].y; v[4 * i + 2] = x[j][i].z; v[4 * i + 3] = x[j][i].w;
+        }
+        st_row16(tiles[j], TILE, r, c0, v);
     }
-    st_row16(tile, TILE, r, c0, v);
 }
 
 // 32 fp32 columns c0 .. c0 + 31 of row `row` as two bf16 terms: hi into one [tok][64] tile, the
@@ -143,10 +152,9 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
     {
         const float* pre = p.pre + ((size_t)bh * p.NSp + chunk) * simt_layout::size;
         const float* adj = p.bw + ((size_t)bh * p.NSp + chunk) * BW_SIZE;
-        mat_tile(sm + SB_S0, pre + simt_layout::mat(0), false, false);
-        mat_tile(sm + SB_R0, pre + simt_layout::mat(2), false, false);
-        mat_tile(sm + SB_GR, adj, false, false);
-        mat_tile(sm + SB_GS, adj + D * D, true, false);
+        uint8_t* const tiles[4] = {sm + SB_S0, sm + SB_R0, sm + SB_GR, sm + SB_GS};
+        const float* const mats[4] = {pre + simt_layout::mat(0), pre + simt_layout::mat(2), adj, adj + D * D};
+        mat_tiles4(tiles, mats);
     }
     // the loads: every thread waits (bounded), then dO (fp32 boxes) -> bf16 tile
     bool ok = ptx::mbar_wait(bar_load, 0);
@@ -289,12 +297,13 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
         half_tile(TB_Z, SB_Z, 0);
         half_tile(TB_DZ, SB_DZ, SB_DZL);
         sync_for_mma();
-        // R3: W* = Q Z^T, dA* = dZ K^T, dK = K G_Ssym + A^T dZ, dQ = dO R0^T + dZ S0
+        // R3: W* = Q Z^T, dA* = dZ K^T, dK = K (G_S^T + G_S) + A^T dZ, dQ = dO R0^T + dZ S0
         if (tid == 0) {
             mm_kk(TB_W, SB_Q, SB_Z, I_128_KK, false);
             mm_kk(TB_DA, SB_DZ, SB_K, I_128_KK, false);
             mm_kk(TB_DA, SB_DZL, SB_K, I_128_KK, true);
-            mm_kk(TB_DK, SB_K, SB_GS, I_64_KK, false);
+            mm_kk(TB_DK, SB_K, SB_GS, I_64_KK, false);            // K G_S^T
+            mm_km(TB_DK, SB_K, SB_GS, true);                      // K G_S
             mm_mm(TB_DK, SB_A, SB_DZ, true);
             mm_mm(TB_DK, SB_A, SB_DZL, true);
             mm_kk(TB_DQ, SB_O, SB_R0, I_64_KK, false);
@@ -307,7 +316,7 @@ k_bwd_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtenso
     }
     if (ok) {
         mask_tile(TB_W, SB_A);               // W over A (A^T dZ is done)
-        mask_tile(TB_DA, SB_DA);             // dA over dZ, S0, G_Ssym (their products are done)
+        mask_tile(TB_DA, SB_DA);             // dA over dZ, S0, G_S (their products are done)
         sync_for_mma();
         // R4: dV = W^T dO + Z G_R, dQ += dW Z + dA K, dK += dA^T Q
         if (tid == 0) {
