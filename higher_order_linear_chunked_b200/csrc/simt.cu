@@ -47,6 +47,29 @@ struct Dim {
     static constexpr int LD = D + 1;  // padded row stride of c x D / D x D tiles
 };
 
+// Programmatic dependent launch between the kernels of one forward: a kernel lets the next one
+// launch as soon as all of its CTAs have started (pdl_release), and the next one waits for its
+// completion (pdl_wait) before it reads what that kernel wrote; loads of the forward's inputs go
+// before the wait.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_dep(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // Summary layout: NMAT matrices D x D, then NVEC vectors D, then one scalar.
 // ---------------------------------------------------------------------------
@@ -224,6 +247,7 @@ __global__ void __launch_bounds__(NT) k_summary(const TIn* __restrict__ q, const
     using S = Sum<OP, D>;
     constexpr int LD = Dim<D>::LD;
     const int chunk = blockIdx.x, bh = blockIdx.y;
+    pdl_release();
     float* out = sums + ((size_t)bh * NCp + chunk) * S::SIZE;
     if (chunk >= NC) {
         write_identity<OP, D>(out);
@@ -582,6 +606,8 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
 template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_scan_level(float* __restrict__ sums, int NCp, int step, int down, int root) {
     using S = Sum<OP, D>;
+    pdl_release();
+    pdl_wait();
     extern __shared__ float sm[];
     float* As = sm;
     float* Bs = As + S::SIZE;
@@ -613,6 +639,8 @@ __global__ void __launch_bounds__(NT) k_scan_level(float* __restrict__ sums, int
 template <int OP, int D>
 __global__ void k_identity(float* sums, int NCp) {
     using S = Sum<OP, D>;
+    pdl_release();
+    pdl_wait();
     write_identity<OP, D>(sums + (size_t)blockIdx.x * NCp * S::SIZE);
 }
 
@@ -635,6 +663,8 @@ template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int NC, int NCp) {
     using S = Sum<OP, D>;
     constexpr int N4 = S::SIZE / 4, PER = (N4 + NT - 1) / NT;
+    pdl_release();
+    pdl_wait();
     extern __shared__ float4 sm4[];
     float* acc = reinterpret_cast<float*>(sm4);          // prefix of slots 0 .. l-1
     float* other = acc + S::SIZE;
@@ -689,6 +719,8 @@ __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int 
 template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ sums, int NC, int NCp, int which) {
     using S = Sum<OP, D>;
+    pdl_release();
+    pdl_wait();
     const int e = blockIdx.x * NT + threadIdx.x;
     int off;
     if (which == 0) {                        // S, P and mK
@@ -721,6 +753,8 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ su
 template <int OP, int D>
 __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ sums, int NCp) {
     using S = Sum<OP, D>;
+    pdl_release();
+    pdl_wait();
     constexpr int LD = Dim<D>::LD;
     extern __shared__ float smx[];
     float* S0 = smx;
@@ -758,16 +792,14 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ su
 
 template <int OP, int D>
 static cudaError_t hla3_factored_prefix(float* sums, int NC, int NCp, int BH, cudaStream_t st) {
-    k_hla3_prefix_plain<OP, D><<<dim3((2 * D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 0);
-    cudaError_t e = cudaGetLastError();
+    auto kp = k_hla3_prefix_plain<OP, D>;
+    cudaError_t e = launch_dep(kp, dim3((2 * D * D + D + NT - 1) / NT, BH), dim3(NT), 0, st, sums, NC, NCp, 0);
     if (e != cudaSuccess) return e;
     const int smem = (int)(sizeof(float) * (6 * D * Dim<D>::LD + 2 * D));
     auto kc = k_hla3_prefix_cross<OP, D>;
     if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    kc<<<dim3(NC, BH), NT, smem, st>>>(sums, NCp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_hla3_prefix_plain<OP, D><<<dim3((D * D + D + NT - 1) / NT, BH), NT, 0, st>>>(sums, NC, NCp, 1);
-    return cudaGetLastError();
+    if ((e = launch_dep(kc, dim3(NC, BH), dim3(NT), (size_t)smem, st, sums, NCp)) != cudaSuccess) return e;
+    return launch_dep(kp, dim3((D * D + D + NT - 1) / NT, BH), dim3(NT), 0, st, sums, NC, NCp, 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -801,6 +833,7 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     load_rows<D>(Qs, q + head, t0, T);
     load_rows<D>(Ks, k + head, t0, T);
     load_rows<D>(Vs, v + head, t0, T);
+    pdl_wait();                              // the prefixes below come from the scan
     float g = 1.f;
     if (OP == OP_HLA2) {
         load_mat<D>(M0, pre + S::mat(0));   // S0
@@ -1034,18 +1067,14 @@ static cudaError_t scan_levels(float* sums, int NCp, int BH, cudaStream_t st) {
     const size_t s2 = scan_smem<OP, D>();
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
-    if (NCp == 1) {
-        k_identity<OP, D><<<BH, NT, 0, st>>>(sums, NCp);
-        return cudaGetLastError();
-    }
-    for (int step = 1; step < NCp; step *= 2) {
-        kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 0, 0);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    for (int step = NCp / 2; step >= 1; step /= 2) {
-        kl<<<dim3(NCp / (2 * step), BH), NT, s2, st>>>(sums, NCp, step, 1, step == NCp / 2);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+    if (NCp == 1) return launch_dep(k_identity<OP, D>, dim3(BH), dim3(NT), 0, st, sums, NCp);
+    for (int step = 1; step < NCp; step *= 2)
+        if ((e = launch_dep(kl, dim3(NCp / (2 * step), BH), dim3(NT), s2, st, sums, NCp, step, 0, 0)) != cudaSuccess)
+            return e;
+    for (int step = NCp / 2; step >= 1; step /= 2)
+        if ((e = launch_dep(kl, dim3(NCp / (2 * step), BH), dim3(NT), s2, st, sums, NCp, step, 1,
+                            step == NCp / 2 ? 1 : 0)) != cudaSuccess)
+            return e;
     return cudaSuccess;
 }
 
@@ -1090,14 +1119,14 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fold_smem<OP, D>())) !=
             cudaSuccess)
             return e;
-        kf<<<BH, NT, fold_smem<OP, D>(), st>>>(sums, NC, NCp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_dep(kf, dim3(BH), dim3(NT), fold_smem<OP, D>(), st, sums, NC, NCp)) != cudaSuccess) return e;
     } else if ((e = scan_levels<OP, D>(sums, NCp, BH, st)) != cudaSuccess) {
         return e;
     }
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H, T, NCp, sums, o);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_dep(ko, dim3(NC, BH), dim3(NT), s3, st, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H,
+                        T, NCp, (const float*)sums, o)) != cudaSuccess)
+        return e;
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }
