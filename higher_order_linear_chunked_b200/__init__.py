@@ -348,23 +348,36 @@ def forward_profiled(op_name: str, q, k, v, events, gamma=None, eps: float = 1e-
 # streaming state: prefill (state after T tokens) and one-token decode steps
 # ---------------------------------------------------------------------------
 
+DECAYED_OPS = ("hla2d", "ahlad", "hla3d")
+
+
+def _rho_offset(op_name: str, d: int) -> int:
+    """Float offset of rho in a decayed state: after the op family's matrices and vectors."""
+    if op_name in ("hla2", "hla2n", "hla2d"):
+        return 4 * d * d + 2 * d
+    if op_name in ("ahla", "ahlan", "ahlad"):
+        return 3 * d * d + 2 * d
+    return 6 * d * d + 3 * d
+
+
 def state_floats(op_name: str, d: int, dv: int, decayed=None) -> int:
     """Floats of one head's streaming state for ``op_name`` (see ``hla_state_floats``);
-    ``decayed`` defaults to ``op_name == "hla2d"`` (pass True for "hla2n" with gamma)."""
-    dec = op_name == "hla2d" if decayed is None else bool(decayed)
+    ``decayed`` defaults to the op name's own ("hla2d", "ahlad", "hla3d"); pass True for a
+    plain or ratio-normalised op used with gamma."""
+    dec = op_name in DECAYED_OPS if decayed is None else bool(decayed)
     return int(load_library().hla_state_floats(OP_CODES[op_name], int(dec), d, dv))
 
 
 def new_state(op_name: str, B: int, H: int, d: int, device="cuda", decayed=None):
     """The state of zero tokens: zeros, with rho = 1 for the decayed form."""
     torch = _torch()
-    dec = op_name == "hla2d" if decayed is None else bool(decayed)
+    dec = op_name in DECAYED_OPS if decayed is None else bool(decayed)
     n = state_floats(op_name, d, d, decayed=dec)
     if n == 0:
         raise HLAError(5, "no streaming state for this op / d")
     st = torch.zeros((B, H, n), dtype=torch.float32, device=device)
     if dec:
-        st[..., 4 * d * d + 2 * d] = 1.0       # rho, after four d x d matrices and two vectors
+        st[..., _rho_offset(op_name, d)] = 1.0
     return st
 
 
@@ -376,9 +389,9 @@ def state(op_name: str, q, k, v, gamma=None, out=None, workspace=None, stream=No
     B, H, T, d = q.shape
     dv = v.shape[-1]
     op = OP_CODES[op_name]
-    decayed = op_name == "hla2d" or (op_name == "hla2n" and gamma is not None)
-    if op_name == "hla2d" and gamma is None:
-        raise ValueError("hla2d needs gamma")
+    decayed = op_name in DECAYED_OPS or (gamma is not None and op_name != "hla2u")
+    if op_name in DECAYED_OPS and gamma is None:
+        raise ValueError(f"{op_name} needs gamma")
     n = int(lib.hla_state_floats(op, int(decayed), d, dv))
     if out is None:
         out = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
@@ -401,6 +414,8 @@ def state(op_name: str, q, k, v, gamma=None, out=None, workspace=None, stream=No
 def step(op_name: str, state_io, q, k, v, gamma=None, eps: float = 1e-6, out=None, stream=None):
     """Decode one token per head: q, k, v [B, H, d]; advances ``state_io`` in place; returns o [B, H, dv]."""
     torch = _torch()
+    if op_name in DECAYED_OPS and gamma is None:
+        raise ValueError(f"{op_name} needs gamma")
     for name, t in (("q", q), ("k", k), ("v", v), ("state", state_io)):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor")

@@ -51,10 +51,6 @@ bool use_tc(const Request& r) {
 
 // Ops with no decayed form.
 bool undecayed_only(hla_op_t op) { return op == HLA_OP_HLA2_UNMASKED; }
-// Ops with a decayed forward but no decayed streaming state (hla_state / hla_step).
-bool no_decayed_state(hla_op_t op) {
-    return op == HLA_OP_AHLA || op == HLA_OP_HLA3 || op == HLA_OP_AHLA_NORM || op == HLA_OP_HLA3_NORM;
-}
 bool valid_op(hla_op_t op) { return op >= HLA_OP_HLA2 && op <= HLA_OP_HLA3_NORM; }
 
 size_t workspace_for(const Request& r) {
@@ -199,13 +195,12 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
 size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv) {
     if (!valid_op(op)) return 0;
     if (d != dv || (d != 32 && d != 64)) return 0;
-    if (decayed && (undecayed_only(op) || no_decayed_state(op))) return 0;
+    if (decayed && undecayed_only(op)) return 0;
     return hla::simt::summary_floats(make_request(op, decayed != 0, HLA_F32, 1, 1, 1, d, dv).op, d);
 }
 
 size_t hla_state_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
-    if (decayed && no_decayed_state(op)) return 0;
     return state_workspace_for(make_request(op, decayed != 0, dtype, B, H, T, d, dv));
 }
 
@@ -222,7 +217,7 @@ hla_status_t hla_state(hla_op_t op, const void* q, const void* k, const void* v,
     if (!q || !k || !v || !state) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, T, d, dv);
     if (s != HLA_OK) return s;
-    if (gamma && (undecayed_only(op) || no_decayed_state(op))) return HLA_ERR_UNSUPPORTED;
+    if (gamma && undecayed_only(op)) return HLA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state)) return HLA_ERR_ALIGN;
     if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
     const Request r = make_request(op, gamma != nullptr, dtype, B, H, T, d, dv);
@@ -244,7 +239,7 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
     if (!state || !q || !k || !v || !o) return HLA_ERR_NULL;
     hla_status_t s = check_shape(dtype, B, H, 1, d, dv);
     if (s != HLA_OK) return s;
-    if (gamma && (undecayed_only(op) || no_decayed_state(op))) return HLA_ERR_UNSUPPORTED;
+    if (gamma && undecayed_only(op)) return HLA_ERR_UNSUPPORTED;
     if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HLA_ERR_ALIGN;
     if (gamma && (reinterpret_cast<uintptr_t>(gamma) & 3u)) return HLA_ERR_ALIGN;
     const Request r = make_request(op, gamma != nullptr, dtype, B, H, 1, d, dv);

@@ -1234,8 +1234,8 @@ static cudaError_t state_op(int op, const void* q, const void* k, const void* v,
     case OP_AHLA: return state_run<OP_AHLA, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_HLA3: return state_run<OP_HLA3, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     case OP_HLA2U: return state_run<OP_HLA2U, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
-    case OP_AHLAD:
-    case OP_HLA3D: return cudaErrorNotSupported;   // no streaming form for the decayed AHLA / third order
+    case OP_AHLAD: return state_run<OP_AHLAD, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
+    case OP_HLA3D: return state_run<OP_HLA3D, D, TIn>(q, k, v, gamma, BH, H, T, sums, state, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -1264,9 +1264,12 @@ int state_launches(int T) {
 //                          rho *= g;  x = q^T S;  o = x^T C - q^T G  (/ (x . m - q . h + eps))
 //   AHLA                   P += k v^T;  Dm += k q^T;  y = q^T P;  E += k y^T;  o = q^T E;
 //                          mK += k;  n += (q . mK) k;  ratio-normalised: o / (q . n + eps)
+//                          (decayed: P, E, mK, n scaled by g first, Dm not; rho *= g)
 //   third order            S += k k^T;  P += k v^T;  Q2 += q q^T;  a = S q;  b = q^T P;
 //                          F += a b^T;  X += q b^T;  Z += a q^T;  o = q^T F;  mK += k;
 //                          F1 += (q . mK) a;  X1 += (q . mK) q;  ratio-normalised: / (q . F1 + eps)
+//                          (decayed: S, P, F, mK, F1 scaled by g first; Q2 += rho g q q^T;
+//                          X, Z, X1 not; rho *= g: the combine with the token's own summary)
 //   unmasked               S += k k^T;  C += q v^T;  o = (q^T S) C
 // S is symmetric, so every product with a vector reads matrix columns: thread j of a group
 // walks rows i, and four groups of D threads split the rows (partial sums in shared memory).
@@ -1399,15 +1402,22 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
         col_dot<D>(Sm, qs, part, a);                            // a = q^T S
         col_dot<D>(Cm, a, part, b);                             // b = (q^T S) C
         if (tid < D) o[(size_t)bh * D + tid] = b[tid];
-    } else if (OP == OP_AHLA) {
+    } else if (OP == OP_AHLA || OP == OP_AHLAD) {
+        // decayed: P, E, mK, n scaled by g before the update, D undecayed, rho *= g
+        const float g = OP == OP_AHLAD ? gamma[bh % H] : 1.f;
         float* P = st + S::mat(0); float* E = st + S::mat(1); float* Dm = st + S::mat(2);
         for (int e = tid; e < DD; e += NT) {
             const int i = e / D, j = e % D;
-            P[e] = fmaf(ks[i], vs[j], P[e]);
+            P[e] = fmaf(ks[i], vs[j], g * P[e]);
             Dm[e] = fmaf(ks[i], qs[j], Dm[e]);
+            E[e] *= g;
         }
         float* mK = st + S::vec(0); float* n = st + S::vec(1);
-        if (tid < D) mK[tid] += ks[tid];
+        if (tid < D) {
+            mK[tid] = fmaf(g, mK[tid], ks[tid]);
+            n[tid] *= g;
+        }
+        if (OP == OP_AHLAD && tid == 0) st[S::SCAL] *= g;
         __syncthreads();
         col_dot<D>(P, qs, part, a);                             // a = y = q^T P
         if (tid == 0) {
@@ -1429,17 +1439,27 @@ __global__ void __launch_bounds__(NT) k_step(float* __restrict__ state, const TI
             }
             o[(size_t)bh * D + tid] = NORM ? b[tid] / den : b[tid];
         }
-    } else {                                                    // OP_HLA3
+    } else {                                                    // OP_HLA3, OP_HLA3D
+        // decayed: S, P, F, mK, F1 scaled by g before the update; Q2 gains the token with weight
+        // rho g (its position's), X, Z, X1 undecayed; rho *= g
+        const float g = OP == OP_HLA3D ? gamma[bh % H] : 1.f;
+        const float wq = OP == OP_HLA3D ? st[S::SCAL] * g : 1.f;
         float* Sm = st + S::mat(0); float* Q2 = st + S::mat(1); float* P = st + S::mat(2);
         float* F = st + S::mat(3); float* X = st + S::mat(4); float* Z = st + S::mat(5);
+        __syncthreads();                                        // every thread has read rho
         for (int e = tid; e < DD; e += NT) {
             const int i = e / D, j = e % D;
-            Sm[e] = fmaf(ks[i], ks[j], Sm[e]);
-            P[e] = fmaf(ks[i], vs[j], P[e]);
-            Q2[e] = fmaf(qs[i], qs[j], Q2[e]);
+            Sm[e] = fmaf(ks[i], ks[j], g * Sm[e]);
+            P[e] = fmaf(ks[i], vs[j], g * P[e]);
+            Q2[e] = fmaf(wq * qs[i], qs[j], Q2[e]);
+            F[e] *= g;
         }
         float* mK = st + S::vec(0); float* X1 = st + S::vec(1); float* F1 = st + S::vec(2);
-        if (tid < D) mK[tid] += ks[tid];
+        if (tid < D) {
+            mK[tid] = fmaf(g, mK[tid], ks[tid]);
+            F1[tid] *= g;
+        }
+        if (OP == OP_HLA3D && tid == 0) st[S::SCAL] = wq;
         __syncthreads();
         col_dot<D>(Sm, qs, part, a);                            // a = S q
         col_dot<D>(P, qs, part, b);                             // b = q^T P
@@ -1664,7 +1684,11 @@ static cudaError_t step_op(int op, bool norm, float* st_, const void* q, const v
                     : step_launch<OP_HLA3, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_HLA2U: return step_rows_launch<OP_HLA2U, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     case OP_AHLAD:
-    case OP_HLA3D: return cudaErrorNotSupported;   // no streaming form for the decayed AHLA / third order
+        return norm ? step_launch<OP_AHLAD, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_AHLAD, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
+    case OP_HLA3D:
+        return norm ? step_launch<OP_HLA3D, true, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st)
+                    : step_launch<OP_HLA3D, false, D, TIn>(st_, q, k, v, gamma, eps, BH, H, o, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -201,18 +201,19 @@ int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, in
  *   second order, decayed S, C, G, Khat = sum k k^T (undecayed);  m, h;  rho =
  *                         gamma^t              (o_t = q_t^T (S_t C_t - G_t))
  *   AHLA                  P = sum k v^T, E, D = sum k q^T;  m^K = sum k, n
- *                         (o_t = q_t^T E_t, den_t = q_t^T n_t)
+ *                         (o_t = q_t^T E_t, den_t = q_t^T n_t); decayed: P, E, m^K, n
+ *                         decay, D does not; then rho = gamma^t
  *   third order           S, Q2 = sum q q^T, P, F, X, Z;  m^K, X1, F1 (X and F with v
- *                         replaced by 1)     (o_t = q_t^T F_t, den_t = q_t^T F1_t)
+ *                         replaced by 1)     (o_t = q_t^T F_t, den_t = q_t^T F1_t);
+ *                         decayed: S, P, F, m^K, F1 decay, Q2 weights token s by
+ *                         gamma^(s+1), X, Z, X1 do not; then rho = gamma^t
  *   unmasked second order S, C                                 (o_t = q_t^T S_t C_t)
  * A state of zero tokens is all zeros, except rho = 1 for the decayed form.
  * The state of a ratio-normalised op is that of its plain op.
  */
 
 /* Floats of one head's state, or 0 when (op, decayed, d, dv) is invalid or unsupported
- * (decayed: hla2 / hla2_normalized with gamma; the decayed AHLA and third order have a
- * forward but no streaming state, and hla_state / hla_step refuse them with
- * HLA_ERR_UNSUPPORTED). */
+ * (the unmasked second order has no decayed form). */
 size_t hla_state_floats(hla_op_t op, int decayed, int d, int dv);
 
 /* Workspace bytes hla_state() needs, or 0 when the request is invalid or unsupported.

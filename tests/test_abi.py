@@ -183,13 +183,16 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert lib.hla_state_floats(3, 0, 32, 32) == pad(6 * 32 * 32 + 3 * 32 + 4)   # S Q2 P F X Z ; mK X1 F1
     assert lib.hla_state_floats(5, 0, d, d) == lib.hla_state_floats(2, 0, d, d)   # normalised: same state
     assert lib.hla_state_floats(6, 0, 32, 32) == lib.hla_state_floats(3, 0, 32, 32)
-    assert lib.hla_state_floats(2, 1, d, d) == 0                              # no decayed AHLA
+    assert lib.hla_state_floats(2, 1, d, d) == lib.hla_state_floats(2, 0, d, d)   # decayed AHLA: + rho
+    assert lib.hla_state_floats(3, 1, 32, 32) == lib.hla_state_floats(3, 0, 32, 32)
+    assert lib.hla_state_floats(4, 1, d, d) == 0                              # no decayed unmasked op
     assert lib.hla_state_floats(0, 0, 48, 48) == 0
     assert lib.hla_state_floats(0, 0, 64, 32) == 0
     # workspace: status block + the CUDA-core chunk summaries (64-token chunks, padded to 2^k)
     n = lib.hla_state_workspace_bytes(0, 0, 0, 4, 16, 4096, d, d)
     assert n == 256 + 4 * 64 * 64 * lib.hla_state_floats(0, 0, d, d)
-    assert lib.hla_state_workspace_bytes(2, 1, 1, 4, 16, 4096, d, d) == 0
+    assert lib.hla_state_workspace_bytes(2, 1, 1, 4, 16, 4096, d, d) > 0       # decayed AHLA (CUDA cores)
+    assert lib.hla_state_workspace_bytes(4, 1, 1, 4, 16, 4096, d, d) == 0
     assert lib.hla_state_kernel_launches(0, 0, 0, 4, 16, 4096, d, d) == 2 + 6     # 64 chunks: 6 levels
     # bf16, d = 64, undecayed second order: the tensor-core summary walker over 16-chunk segments
     # (two per head at T = 4096), then one combine per head
@@ -205,7 +208,7 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert st(7, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 5                # bad op
     assert st(0, *a, 0, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 2                # B = 0
     assert st(0, *a, 1, 1, 64, d, d, 7, vp(0), vp(16), 1 << 20, vp(0)) == 4                # dtype
-    assert st(2, *a, 1, 1, 64, d, d, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5               # gamma + AHLA
+    assert st(4, *a, 1, 1, 64, d, d, 0, vp(16), vp(16), 1 << 20, vp(0)) == 5               # gamma + unmasked
     assert st(0, vp(8), *a[1:], 1, 1, 64, d, d, 0, vp(0), vp(16), 1 << 20, vp(0)) == 3     # alignment
     assert st(0, *a, 1, 1, 64, d, d, 0, vp(0), vp(0), 1 << 20, vp(0)) == 6                 # no workspace
     assert st(0, *a, 1, 1, 64, d, d, 0, vp(0), vp(16), 64, vp(0)) == 6                     # too small
@@ -214,7 +217,7 @@ def test_streaming_state_sizes_and_argument_errors(lib):
     assert sp(0, vp(0), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 1                 # NULL state
     assert sp(0, *b, 1, 1, 48, 48, 0, vp(0), f(1e-6), vp(0)) == 5                          # d = 48
     assert sp(0, *b, 1, 0, d, d, 0, vp(0), f(1e-6), vp(0)) == 2                            # H = 0
-    assert sp(3, *b, 1, 1, 32, 32, 0, vp(16), f(1e-6), vp(0)) == 5                         # gamma + HLA-3
+    assert sp(4, *b, 1, 1, 32, 32, 0, vp(16), f(1e-6), vp(0)) == 5                         # gamma + unmasked
     assert sp(0, vp(24), *b[1:], 1, 1, d, d, 0, vp(0), f(1e-6), vp(0)) == 3                # alignment
 
 

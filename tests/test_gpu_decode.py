@@ -33,7 +33,7 @@ STATE_TOL_TC = 1e-2
 
 def state_tol(op, dtype, d):
     return STATE_TOL_TC if (op in ("hla2", "hla2n") and dtype == "bf16" and d == 64) else STATE_TOL
-OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n"]
+OPS = ["hla2", "hla2n", "hla2d", "ahla", "hla3", "hla2u", "ahlan", "hla3n", "ahlad", "hla3d"]
 NORMALISED = ("hla2n", "ahlan", "hla3n")
 DEV = torch.device("cuda:0")
 
@@ -41,7 +41,7 @@ DEV = torch.device("cuda:0")
 def recipe(op, dtype, B, H, T, d, seed):
     qk = "softplus" if op in NORMALISED else "scaled"
     v = "unit" if op in NORMALISED else "scaled"
-    g = (0.9, 0.999) if op == "hla2d" else None
+    g = (0.9, 0.999) if op in ("hla2d", "ahlad", "hla3d") else None
     return hla_inputs.Workload(f"{op}_{dtype}_{B}x{H}x{T}x{d}", op, dtype, B, H, T, d, d, qk, v,
                                gamma_range=g, seed=seed)
 
@@ -59,6 +59,15 @@ def oracle_state(op, q, k, v, gamma):
         s = seg.ahla_summary(q, k, v)
         _, s1 = oracle.ahla_run(q, k, ones, want_output=False)     # v -> 1: P -> mK, E -> n
         return [s["P"], s["E"], s["D"], s1["P"][:, 0], s1["E"][:, 0]]
+    if op == "ahlad":
+        s = seg.ahla_summary(q, k, v, gamma=gamma)
+        s1 = seg.ahla_summary(q, k, ones, gamma=gamma)
+        return [s["P"], s["E"], s["D"], s1["P"][:, 0], s1["E"][:, 0], np.array([float(s["rho"])])]
+    if op == "hla3d":
+        s = seg.hla3_summary(q, k, v, gamma=gamma)
+        s1 = seg.hla3_summary(q, k, ones, gamma=gamma)
+        return [s["S"], s["Q2"], s["P"], s["F"], s["X"], s["Z"], s1["P"][:, 0], s1["X"][:, 0], s1["F"][:, 0],
+                np.array([float(s["rho"])])]
     if op == "hla2u":
         _, s = oracle.hla2u_run(q, k, v, want_output=False)
         return [s["S"], s["C"]]
@@ -69,13 +78,15 @@ def oracle_state(op, q, k, v, gamma):
 
 def split_state(op, x, d):
     """The GPU state vector of one head, cut into the same slots."""
-    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6, "hla2u": 2, "ahlan": 3, "hla3n": 6}[op]
-    nvec = {"hla2": 2, "hla2n": 2, "hla2d": 2, "ahla": 2, "ahlan": 2, "hla3": 3, "hla3n": 3, "hla2u": 0}[op]
+    nmat = {"hla2": 3, "hla2n": 3, "hla2d": 4, "ahla": 3, "hla3": 6, "hla2u": 2, "ahlan": 3, "hla3n": 6,
+            "ahlad": 3, "hla3d": 6}[op]
+    nvec = {"hla2": 2, "hla2n": 2, "hla2d": 2, "ahla": 2, "ahlan": 2, "hla3": 3, "hla3n": 3, "hla2u": 0,
+            "ahlad": 2, "hla3d": 3}[op]
     out = [x[i * d * d:(i + 1) * d * d].reshape(d, d) for i in range(nmat)]
     base = nmat * d * d
     out += [x[base + i * d: base + (i + 1) * d] for i in range(nvec)]
-    if op == "hla2d":
-        out.append(x[base + 2 * d: base + 2 * d + 1])
+    if op in ("hla2d", "ahlad", "hla3d"):
+        out.append(x[base + nvec * d: base + nvec * d + 1])
     return out
 
 
@@ -156,4 +167,22 @@ def test_normalised_decay_state_and_steps():
     o = torch.stack(outs, dim=2).cpu()
     ref = np.stack([oracle.hla2_run(q[0, h], k[0, h], v[0, h], gamma=float(g[h]), normalized=True,
                                     eps=w.eps)[0] for h in range(2)])[None, :, T0:]
+    assert oracle.max_row_rel_err(o, ref) <= TOL["f32"]
+
+
+@pytest.mark.parametrize("op", ["ahlan", "hla3n"])
+def test_normalised_decayed_ahla_hla3_state_and_steps(op):
+    """Ratio-normalised AHLA / third order with gamma: the decayed state form (its vectors decay
+    with the matrices) and the ratio-normalised output, prefill then decode against the oracle."""
+    d, T0, T1 = 32, 70, 6
+    w = hla_inputs.Workload("x", op, "f32", 1, 2, T0 + T1, d, d, "softplus", "unit", gamma_range=(0.9, 0.999), seed=6)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    st = hla.state(op, gpu(q[:, :, :T0].contiguous()), gpu(k[:, :, :T0].contiguous()),
+                   gpu(v[:, :, :T0].contiguous()), gamma=gpu(g))
+    assert st.shape[-1] == hla.state_floats(op, d, d, decayed=True)
+    outs = [hla.step(op, st, gpu(q[:, :, t].contiguous()), gpu(k[:, :, t].contiguous()),
+                     gpu(v[:, :, t].contiguous()), gamma=gpu(g), eps=w.eps) for t in range(T0, T0 + T1)]
+    torch.cuda.synchronize()
+    o = torch.stack(outs, dim=2).cpu()
+    ref = oracle.recur(op, q, k, v, gamma=g, eps=w.eps)[:, :, T0:]
     assert oracle.max_row_rel_err(o, ref) <= TOL["f32"]
