@@ -325,8 +325,8 @@ def run_ours(args):
     if args.decode_steps > 0:
         decode = decode_measure(w, qd, kd, vd, gd, flush, args.decode_steps, peaks, peak_kind)
     backward = None
-    if args.backward_steps > 0 and w.op in ("hla2", "hla2n") and gd is None:
-        backward = backward_measure(w, qd, kd, vd, flush, args.backward_steps, peaks, q, k, v, rank)
+    if args.backward_steps > 0 and w.op in ("hla2", "hla2n", "ahla") and gd is None:
+        backward = backward_measure(w, qd, kd, vd, flush, args.backward_steps, peaks, q, k, v, rank, peak_kind)
     clk = clocks.summary()
     model = output_kernel_model(path, w)
     out_avg_ms = statistics.mean(out_ms)
@@ -464,11 +464,12 @@ def measure_workloads(dev, args, peaks, peak_kind, done):
     return res
 
 
-def backward_measure(w, qd, kd, vd, flush, steps, peaks, q, k, v, rank):
-    """The masked second-order backward (hla2_backward) on the workload's inputs with a seeded fp32
-    output gradient: time per call (CUDA events, L2 flushed before each), tokens/s, the gradient
-    kernels against the FP32 FFMA peak, and a directional-derivative check of the result against
-    the fp64 oracle's forward on one head (rank 0)."""
+def backward_measure(w, qd, kd, vd, flush, steps, peaks, q, k, v, rank, peak_kind="fallback"):
+    """The backward pass of the workload's operator (the plain masked second order for hla2 and
+    hla2n workloads, hla2_backward; AHLA for ahla workloads, ahla_backward) on its inputs with a
+    seeded fp32 output gradient: time per call (CUDA events, L2 flushed before each), tokens/s,
+    the gradient products against the peak of the units they run on, and a directional-derivative
+    check of the result against the fp64 oracle's forward on one head (rank 0)."""
     import numpy as np
     import torch
 
@@ -477,31 +478,55 @@ def backward_measure(w, qd, kd, vd, flush, steps, peaks, q, k, v, rank):
     g = torch.Generator("cpu").manual_seed(w.seed + 1234)
     do = torch.randn(tuple(qd.shape[:3]) + (vd.shape[-1],), generator=g, dtype=torch.float32)
     dod = do.to(dev)
-    ws = torch.empty(hla.load_library().hla_backward_workspace_bytes(hla.OP_HLA2, hla.HLA_BF16 if w.dtype == "bf16"
-                                                                      else hla.HLA_F32, w.B, w.H, w.T, w.d, w.dv),
+    ahla = w.op == "ahla"
+    opc = hla.OP_AHLA if ahla else hla.OP_HLA2
+    dtc = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
+    run = hla.ahla_backward if ahla else hla.hla2_backward
+    ws = torch.empty(hla.load_library().hla_backward_workspace_bytes(opc, dtc, w.B, w.H, w.T, w.d, w.dv),
                      dtype=torch.uint8, device=dev)
     for _ in range(3):
-        grads = hla.hla2_backward(qd, kd, vd, dod, workspace=ws)
+        grads = run(qd, kd, vd, dod, workspace=ws)
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        grads = hla.hla2_backward(qd, kd, vd, dod, workspace=ws)
+        grads = run(qd, kd, vd, dod, workspace=ws)
         b.record()
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     ms = statistics.mean(times)
-    c, D = 64, w.d
-    # gradient products per 64-token chunk, in multiply-adds: chunk terms (Q^T dO, Q^T V, dO V^T,
-    # dW Q, Q^T (dW Q)), the cross term C dR'^T, and the chunk gradients (A, P, dW, W, Z, dV, dZ,
-    # dP, dA, dQ, dK); the forward summaries it recomputes are not counted
-    macs = (3 * c * D * D + 2 * c * c * D) + D ** 3 + (8 * c * c * D + 6 * c * D * D + 2 * c ** 3 + 3 * c * c * D)
+    D = w.d
+    smax = float(peaks.get("sm_max_mhz", 1965.0))
+    tensor = not ahla and w.dtype == "bf16" and D == 64
+    if tensor:
+        # tensor-core path, 128-token chunks, in multiply-adds per chunk (the two-term splits of dO
+        # and dZ are precision work, not counted): adjoint terms (dO V^T, Q^T dO, Q^T V, dW Q,
+        # Q^T (dW Q)), the cross term C dR'^T, and the gradients in the Z form (A, Q S0, A K, dO V^T,
+        # dW^T Q, V dR'^T, Q Z^T, dZ K^T, K dS', A^T dZ, dO R0^T, dZ S0, W^T dO, Z dR', dW Z, dA K,
+        # dA^T Q); the carried states it recomputes are not counted
+        c = 128
+        macs = (2 * c * c * D + 3 * c * D * D) + D ** 3 + (11 * c * c * D + 6 * c * D * D)
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        bound, peak_source = "tensor", f"bf16 dense burst ({peak_kind})"
+    elif ahla:
+        # AHLA, CUDA cores, 64-token chunks: chunk terms (A, Q^T dO, Q^T K, A^T dO, Q^T (A^T dO)), the
+        # cross term M dE', and the gradients (A, Y, dY, dA, dV, dQ, dK)
+        c = 64
+        macs = (2 * c * c * D + 3 * c * D * D) + D ** 3 + (8 * c * c * D + 7 * c * D * D)
+        peak, bound = alu_peak_tflops(smax), "alu"
+        peak_source = f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"
+    else:
+        # second order, CUDA cores, 64-token chunks: chunk terms (Q^T dO, Q^T V, dO V^T, dW Q,
+        # Q^T (dW Q)), the cross term C dR'^T, and the chunk gradients (A, P, dW, W, Z, dV, dZ, dP,
+        # dA, dQ, dK); the forward summaries it recomputes are not counted
+        c = 64
+        macs = (3 * c * D * D + 2 * c * c * D) + D ** 3 + (8 * c * c * D + 6 * c * D * D + 2 * c ** 3 + 3 * c * c * D)
+        peak, bound = alu_peak_tflops(smax), "alu"
+        peak_source = f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"
     flops_per_token = 2 * macs / c
     achieved = flops_per_token * w.tokens / (ms / 1e3) / 1e12
-    smax = float(peaks.get("sm_max_mhz", 1965.0))
-    peak = alu_peak_tflops(smax)
     check = None
     if rank == 0:
         b_, h_ = 0, 0
@@ -512,19 +537,20 @@ def backward_measure(w, qd, kd, vd, flush, steps, peaks, q, k, v, rank):
         eps = 1e-4
 
         def f(s):
-            o = oracle.recur("hla2", (qh + s * dirs[0])[None, None], (kh + s * dirs[1])[None, None],
-                             (vh + s * dirs[2])[None, None])[0, 0]
+            o = oracle.recur("ahla" if ahla else "hla2", (qh + s * dirs[0])[None, None],
+                             (kh + s * dirs[1])[None, None], (vh + s * dirs[2])[None, None])[0, 0]
             return float(np.sum(o * doh))
         num = (f(eps) - f(-eps)) / (2 * eps)
         ana = sum(float(np.sum(gr[b_, h_].double().cpu().numpy() * dr)) for gr, dr in zip(grads, dirs))
         check = {"directional_derivative_rel_err": abs(ana - num) / max(1.0, abs(num)), "head": [b_, h_],
                  "against": "central difference of the fp64 oracle forward"}
-    return {"op": "hla2 (plain masked second order)", "ms": ms, "tokens_per_s": w.tokens / (ms / 1e3),
-            "gpu_launches_per_step": hla.load_library().hla_backward_kernel_launches(
-                hla.OP_HLA2, hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32, w.B, w.H, w.T, w.d, w.dv),
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "flops_per_token": flops_per_token,
-                         "peak_source": f"FP32 FFMA 148x128x2 flop at {smax:.0f} MHz (derived)"},
+    return {"op": "ahla" if ahla else "hla2 (plain masked second order)", "ms": ms,
+            "tokens_per_s": w.tokens / (ms / 1e3),
+            "gpu_launches_per_step": hla.load_library().hla_backward_kernel_launches(opc, dtc, w.B, w.H, w.T, w.d,
+                                                                                     w.dv),
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "flops_per_token": flops_per_token, "scope": "whole call",
+                         "peak_source": peak_source},
             "check": check, "l2": "flushed before every call (outside the events)"}
 
 

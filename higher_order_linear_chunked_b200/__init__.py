@@ -41,7 +41,7 @@ EXPORTS = ("hla_abi_version", "hla_status_str", "hla_workspace_bytes", "hla2_for
            "hla_state_kernel_launches", "hla_state", "hla_step", "hla2_forward_unmasked",
            "ahla_forward_normalized", "hla3_forward_normalized", "hla_noalloc_read_device_status",
            "hla_backward_workspace_bytes", "hla_backward_kernel_launches", "hla2_backward",
-           "hla2_backward_normalized")
+           "hla2_backward_normalized", "ahla_backward")
 
 
 class HLAError(RuntimeError):
@@ -94,6 +94,8 @@ def load_library(path: Optional[str] = None):
     lib.hla_backward_kernel_launches.restype = i
     lib.hla2_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, sz, vp]
     lib.hla2_backward.restype = i
+    lib.ahla_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, sz, vp]
+    lib.ahla_backward.restype = i
     lib.hla2_backward_normalized.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, f, vp, sz, vp]
     lib.hla2_backward_normalized.restype = i
     lib.hla_noalloc_read_device_status.argtypes = [vp, ctypes.POINTER(i)]
@@ -242,6 +244,15 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None, normalized: bool =
     """Gradients (dq, dk, dv), fp32, of sum(O * dout) for O = hla2(q, k, v) (masked second order,
     no decay), or O = hla2_normalized(q, k, v, eps) with ``normalized``.  dout: fp32 [B, H, T, dv]
     on q's device."""
+    return _backward(OP_HLA2_NORM if normalized else OP_HLA2, q, k, v, dout, workspace, stream, eps)
+
+
+def ahla_backward(q, k, v, dout, workspace=None, stream=None):
+    """Gradients (dq, dk, dv), fp32, of sum(O * dout) for O = ahla(q, k, v) (no decay)."""
+    return _backward(OP_AHLA, q, k, v, dout, workspace, stream, 0.0)
+
+
+def _backward(op, q, k, v, dout, workspace, stream, eps):
     torch = _torch()
     _check(q, k, v)
     if not dout.is_cuda or dout.dtype != torch.float32 or not dout.is_contiguous() or dout.shape != v.shape:
@@ -249,7 +260,6 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None, normalized: bool =
     lib = load_library()
     B, H, T, d = q.shape
     dvd = v.shape[-1]
-    op = OP_HLA2_NORM if normalized else OP_HLA2
     n = int(lib.hla_backward_workspace_bytes(op, _dtype_code(q), B, H, T, d, dvd))
     if n == 0:
         raise HLAError(5, "no backward kernel for this shape/dtype")
@@ -263,12 +273,14 @@ def hla2_backward(q, k, v, dout, workspace=None, stream=None, normalized: bool =
     head = [vp(q.data_ptr()), vp(k.data_ptr()), vp(v.data_ptr()), vp(dout.data_ptr()), vp(dq.data_ptr()),
             vp(dk.data_ptr()), vp(dv.data_ptr()), B, H, T, d, dvd, _dtype_code(q), vp(0)]
     tail = [vp(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()), vp(st.cuda_stream)]
-    if normalized:
+    if op == OP_HLA2_NORM:
         rc = lib.hla2_backward_normalized(*head, ctypes.c_float(eps), *tail)
+    elif op == OP_AHLA:
+        rc = lib.ahla_backward(*head, *tail)
     else:
         rc = lib.hla2_backward(*head, *tail)
     if rc != HLA_OK:
-        raise HLAError(rc, "hla2_backward rejected the call")
+        raise HLAError(rc, "the backward call rejected it")
     return dq, dk, dv
 
 

@@ -249,8 +249,9 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
 }
 
 size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
-    if (op != HLA_OP_HLA2 && op != HLA_OP_HLA2_NORM) return 0;
+    if (op != HLA_OP_HLA2 && op != HLA_OP_HLA2_NORM && op != HLA_OP_AHLA) return 0;
     if (check_shape(dtype, B, H, T, d, dv) != HLA_OK) return 0;
+    if (op == HLA_OP_AHLA) return hla::kStatusBytes + sizeof(float) * hla::simt::ahla_backward_workspace_floats(d, B * H, T);
     if (op == HLA_OP_HLA2_NORM)
         return hla::kStatusBytes + sizeof(float) * hla::simt::backward_normalized_workspace_floats(d, B * H, T);
     return hla::kStatusBytes + sizeof(float) * hla::simt::backward_workspace_floats(d, B * H, T);
@@ -258,6 +259,7 @@ size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H
 
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
     if (hla_backward_workspace_bytes(op, dtype, B, H, T, d, dv) == 0) return 0;
+    if (op == HLA_OP_AHLA) return hla::simt::ahla_backward_launches(d, T);
     return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(d, T)
                                   : hla::simt::backward_launches(dtype == HLA_BF16, d, T);
 }
@@ -280,11 +282,14 @@ hla_status_t backward_call(hla_op_t op, const void* q, const void* k, const void
     if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return HLA_ERR_CUDA;
     float* body = reinterpret_cast<float*>(static_cast<char*>(workspace) + hla::kStatusBytes);
     int* status = static_cast<int*>(workspace);
-    const cudaError_t e =
-        op == HLA_OP_HLA2_NORM
-            ? hla::simt::backward_normalized(dtype == HLA_BF16, d, q, k, v, dout, eps, dq, dk, dv_out, B * H, T, body,
-                                             status, st)
-            : hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, status, st);
+    cudaError_t e;
+    if (op == HLA_OP_AHLA)
+        e = hla::simt::ahla_backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, st);
+    else if (op == HLA_OP_HLA2_NORM)
+        e = hla::simt::backward_normalized(dtype == HLA_BF16, d, q, k, v, dout, eps, dq, dk, dv_out, B * H, T, body,
+                                           status, st);
+    else
+        e = hla::simt::backward(dtype == HLA_BF16, d, q, k, v, dout, dq, dk, dv_out, B * H, T, body, status, st);
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
 }  // namespace
@@ -293,6 +298,13 @@ hla_status_t hla2_backward(const void* q, const void* k, const void* v, const fl
                            float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma,
                            void* workspace, size_t workspace_bytes, void* stream) {
     return backward_call(HLA_OP_HLA2, q, k, v, dout, dq, dk, dv_out, B, H, T, d, dv, dtype, gamma, 0.f, workspace,
+                         workspace_bytes, stream);
+}
+
+hla_status_t ahla_backward(const void* q, const void* k, const void* v, const float* dout, float* dq, float* dk,
+                           float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype, const float* gamma,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_call(HLA_OP_AHLA, q, k, v, dout, dq, dk, dv_out, B, H, T, d, dv, dtype, gamma, 0.f, workspace,
                          workspace_bytes, stream);
 }
 

@@ -1812,7 +1812,7 @@ __global__ void __launch_bounds__(NT) k_bwd_suffix(float* __restrict__ bw, int N
 
 // X = U + C dR'^T per chunk, in place of U.
 template <int D>
-__global__ void __launch_bounds__(NT) k_bwd_cross(float* __restrict__ bw, int NCp) {
+__global__ void __launch_bounds__(NT) k_bwd_cross(float* __restrict__ bw, int NCp, int trans) {
     constexpr int LD = Dim<D>::LD;
     __shared__ float Cs[D * LD], Rs[D * LD];
     float* slot = bw + ((size_t)blockIdx.y * NCp + blockIdx.x) * Bwd<D>::SIZE;
@@ -1820,8 +1820,10 @@ __global__ void __launch_bounds__(NT) k_bwd_cross(float* __restrict__ bw, int NC
     load_mat<D>(Rs, slot);
     __syncthreads();
     float* U = slot + D * D;
-    mm<D, D, D>(Tile{Cs, LD}, TileT{Rs, LD}, [&](int r, int c) { return U[r * D + c]; },
-                [&](int r, int c, float x) { U[r * D + c] = x; });
+    auto acc = [&](int r, int c) { return U[r * D + c]; };
+    auto put = [&](int r, int c, float x) { U[r * D + c] = x; };
+    if (trans) mm<D, D, D>(Tile{Cs, LD}, TileT{Rs, LD}, acc, put);     // second order: U + C dR'^T
+    else mm<D, D, D>(Tile{Cs, LD}, Tile{Rs, LD}, acc, put);            // AHLA: U + M dE'
 }
 
 template <int D, typename TIn>
@@ -1934,7 +1936,7 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
         const dim3 sg2((D * D + NT - 1) / NT, BH);
         k_bwd_suffix<D><<<sg2, NT, 0, st>>>(bw, NC2, NSp2, 0);                // dR'
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        k_bwd_cross<D><<<dim3(NC2, BH), NT, 0, st>>>(bw, NSp2);                // X = U + C dR'^T
+        k_bwd_cross<D><<<dim3(NC2, BH), NT, 0, st>>>(bw, NSp2, 1);             // X = U + C dR'^T
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         k_bwd_suffix<D><<<sg2, NT, 0, st>>>(bw, NC2, NSp2, 1);                // dS'
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1965,7 +1967,7 @@ static cudaError_t backward_run(const void* q, const void* k, const void* v, con
     const dim3 sg((D * D + NT - 1) / NT, BH);
     k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 0);                       // dR'
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_bwd_cross<D><<<dim3(NC, BH), NT, 0, st>>>(bw, NCp);                      // X = U + C dR'^T
+    k_bwd_cross<D><<<dim3(NC, BH), NT, 0, st>>>(bw, NCp, 1);                   // X = U + C dR'^T
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dS'
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -2065,6 +2067,171 @@ cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_add_into<<<blocks, NT, 0, st>>>(dk, dk2, n);
     return cudaGetLastError();
+}
+
+// ===========================================================================
+// Backward pass of the AHLA output (no decay, not normalised).  The forward's chunk algebra:
+//     A = L (.) Q K^T,  Y = Q P0 + A V,  O = Q E0 + A Y,  P0' = P0 + K^T V,  E0' = E0 + K^T Y.
+// Reverse mode, with dO given and (dP', dE') the adjoints of the state the chunk hands on:
+//     dY = A^T dO + K dE',   dA = L (.) (dO Y^T + dY V^T),
+//     dQ = dO E0^T + dY P0^T + dA K,   dK = Y dE'^T + V dP'^T + dA^T Q,   dV = K dP' + A^T dY,
+// and the adjoints handed back dE = dE' + Q^T dO, dP = dP' + Q^T dY.  Unrolled over the chunks
+// after c they are suffix sums, of the same shape as the second order's:
+//     dE'(c) = sum_{m>c} Q_m^T dO_m,   dP'(c) = sum_{m>c} (U_m + M_m dE'(m)),
+//     U_m = Q_m^T (A_m^T dO_m),   M_m = Q_m^T K_m
+// (slot layout [Y = Q^T dO | U | M]; the cross term without the transpose).
+// ===========================================================================
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_abwd_chunk(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                                   const float* __restrict__ dout, int T, int NCp,
+                                                   float* __restrict__ bw) {
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Ks = Qs + C * LD;
+    float* Os = Ks + C * LD;                  // dO
+    float* Gs = Os + C * LD;                  // A^T dO
+    float* As = Gs + C * LD;                  // C x LDC
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Ks, k + head, t0, T);
+    load_rows<D>(Os, dout + head, t0, T);
+    __syncthreads();
+    float* out = bw + ((size_t)bh * NCp + chunk) * Bwd<D>::SIZE;
+    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, PutMasked{As, LDC});                          // A
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Os, LD}, Zero{}, [&](int r, int c, float x) { out[r * D + c] = x; });      // Y
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Ks, LD}, Zero{},
+                [&](int r, int c, float x) { out[2 * D * D + r * D + c] = x; });                   // M
+    __syncthreads();
+    mm<C, D, C>(TileT{As, LDC}, Tile{Os, LD}, Zero{}, Put{Gs, LD});                                 // A^T dO
+    __syncthreads();
+    mm<D, D, C>(TileT{Qs, LD}, Tile{Gs, LD}, Zero{},
+                [&](int r, int c, float x) { out[D * D + r * D + c] = x; });                       // U
+}
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NT) k_abwd_out(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                                                 const TIn* __restrict__ v, const float* __restrict__ dout,
+                                                 int T, int NCp, const float* __restrict__ sums,
+                                                 const float* __restrict__ bw, float* __restrict__ dq,
+                                                 float* __restrict__ dk, float* __restrict__ dv) {
+    using S = Sum<OP_AHLA, D>;
+    constexpr int LD = Dim<D>::LD;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const float* pre = sums + ((size_t)bh * NCp + chunk) * S::SIZE;          // P0 = mat(0), E0 = mat(1)
+    const float* adj = bw + ((size_t)bh * NCp + chunk) * Bwd<D>::SIZE;       // dE' = 0, dP' = 1
+    extern __shared__ float sm[];
+    float* Qs = sm;
+    float* Ks = Qs + C * LD;
+    float* Vs = Ks + C * LD;
+    float* Os = Vs + C * LD;                  // dO
+    float* Ys = Os + C * LD;                  // Y
+    float* dYs = Ys + C * LD;                 // dY
+    float* As = dYs + C * LD;                 // C x LDC: A
+    float* dAs = As + C * LDC;                // dA
+    float* P0 = dAs + C * LDC;                // D x LD
+    float* E0 = P0 + D * LD;
+    float* dP = E0 + D * LD;
+    float* dE = dP + D * LD;
+    const size_t head = (size_t)bh * T * D;
+    const int t0 = chunk * C;
+    load_rows<D>(Qs, q + head, t0, T);
+    load_rows<D>(Ks, k + head, t0, T);
+    load_rows<D>(Vs, v + head, t0, T);
+    load_rows<D>(Os, dout + head, t0, T);
+    load_mat<D>(P0, pre + S::mat(0));
+    load_mat<D>(E0, pre + S::mat(1));
+    load_mat<D>(dE, adj);
+    load_mat<D>(dP, adj + D * D);
+    __syncthreads();
+    mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, PutMasked{As, LDC});                          // A
+    __syncthreads();
+    mm2<C, D, D, C>(Tile{Qs, LD}, Tile{P0, LD}, Tile{As, LDC}, Tile{Vs, LD}, Zero{}, Put{Ys, LD});   // Y
+    mm2<C, D, C, D>(TileT{As, LDC}, Tile{Os, LD}, Tile{Ks, LD}, Tile{dE, LD}, Zero{}, Put{dYs, LD}); // dY
+    __syncthreads();
+    // dA = L (.) (dO Y^T + dY V^T);  dV = K dP' + A^T dY
+    mm2<C, C, D, D>(Tile{Os, LD}, TileT{Ys, LD}, Tile{dYs, LD}, TileT{Vs, LD}, Zero{}, PutMasked{dAs, LDC});
+    mm2<C, D, D, C>(Tile{Ks, LD}, Tile{dP, LD}, TileT{As, LDC}, Tile{dYs, LD}, Zero{},
+                    [&](int r, int c, float x) { if (t0 + r < T) dv[head + (size_t)(t0 + r) * D + c] = x; });
+    __syncthreads();
+    // dQ = dO E0^T + dY P0^T + dA K;  dK = Y dE'^T + V dP'^T + dA^T Q
+    mm3<C, D, D, D, C>(Tile{Os, LD}, TileT{E0, LD}, Tile{dYs, LD}, TileT{P0, LD}, Tile{dAs, LDC}, Tile{Ks, LD},
+                       Zero{}, [&](int r, int c, float x) { if (t0 + r < T) dq[head + (size_t)(t0 + r) * D + c] = x; });
+    mm3<C, D, D, D, C>(Tile{Ys, LD}, TileT{dE, LD}, Tile{Vs, LD}, TileT{dP, LD}, TileT{dAs, LDC}, Tile{Qs, LD},
+                       Zero{}, [&](int r, int c, float x) { if (t0 + r < T) dk[head + (size_t)(t0 + r) * D + c] = x; });
+}
+
+template <int D>
+static size_t abwd_chunk_smem() {
+    return sizeof(float) * (size_t)(4 * C * Dim<D>::LD + C * LDC);
+}
+template <int D>
+static size_t abwd_out_smem() {
+    return sizeof(float) * (size_t)(6 * C * Dim<D>::LD + 2 * C * LDC + 4 * D * Dim<D>::LD);
+}
+
+size_t ahla_backward_workspace_floats(int d, int BH, int T) {
+    const int NCp = next_pow2((T + C - 1) / C);
+    return workspace_floats(OP_AHLA, d, BH, T) + (size_t)BH * NCp * 3 * d * d;
+}
+
+int ahla_backward_launches(int d, int T) {
+    // summaries, the scan, chunk terms, two suffix sums, cross term, gradients
+    return kernel_launches(OP_AHLA, d, T) - 1 + 5;
+}
+
+template <int D, typename TIn>
+static cudaError_t ahla_backward_run(const void* q, const void* k, const void* v, const float* dout, float* dq,
+                                     float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st) {
+    const int NC = (T + C - 1) / C;
+    const int NCp = next_pow2(NC);
+    float* sums = ws;
+    float* bw = ws + workspace_floats(OP_AHLA, D, BH, T);
+    auto ks = k_summary<OP_AHLA, D, TIn>;
+    auto kc = k_abwd_chunk<D, TIn>;
+    auto ko = k_abwd_out<D, TIn>;
+    const size_t s1 = summary_smem<D>(), s2 = abwd_chunk_smem<D>(), s3 = abwd_out_smem<D>();
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess) return e;
+    // the forward's carried states: chunk summaries, then their exclusive scan
+    ks<<<dim3(NCp, BH), NT, s1, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, nullptr, 1, T, NC, NCp, sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (fold_fits<OP_AHLA, D>()) {
+        auto kf = k_scan_fold<OP_AHLA, D>;
+        if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)fold_smem<OP_AHLA, D>())) != cudaSuccess)
+            return e;
+        kf<<<BH, NT, fold_smem<OP_AHLA, D>(), st>>>(sums, NC, NCp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else if ((e = scan_levels<OP_AHLA, D>(sums, NCp, BH, st)) != cudaSuccess) {
+        return e;
+    }
+    kc<<<dim3(NC, BH), NT, s2, st>>>((const TIn*)q, (const TIn*)k, dout, T, NCp, bw);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 sg((D * D + NT - 1) / NT, BH);
+    k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 0);                       // dE'
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_cross<D><<<dim3(NC, BH), NT, 0, st>>>(bw, NCp, 0);                   // X = U + M dE'
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    k_bwd_suffix<D><<<sg, NT, 0, st>>>(bw, NC, NCp, 1);                       // dP'
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ko<<<dim3(NC, BH), NT, s3, st>>>((const TIn*)q, (const TIn*)k, (const TIn*)v, dout, T, NCp, sums, bw, dq, dk,
+                                     dv);
+    return cudaGetLastError();
+}
+
+cudaError_t ahla_backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                          float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st) {
+    if (bf16) {
+        if (d == 32) return ahla_backward_run<32, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+        return ahla_backward_run<64, __nv_bfloat16>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+    }
+    if (d == 32) return ahla_backward_run<32, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
+    return ahla_backward_run<64, float>(q, k, v, dout, dq, dk, dv, BH, T, ws, st);
 }
 
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,

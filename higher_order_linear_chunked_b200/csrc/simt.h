@@ -47,6 +47,12 @@ int backward_launches(bool bf16, int d, int T);
 cudaError_t backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
                      float* dk, float* dv, int BH, int T, float* ws, int* status, cudaStream_t st,
                      bool fp32_only = false);
+// Backward pass of the AHLA output (no decay, not normalised), fp32 on the CUDA cores;
+// ws: ahla_backward_workspace_floats floats.
+size_t ahla_backward_workspace_floats(int d, int BH, int T);
+int ahla_backward_launches(int d, int T);
+cudaError_t ahla_backward(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout, float* dq,
+                          float* dk, float* dv, int BH, int T, float* ws, cudaStream_t st);
 // The same for the ratio-normalised output (two plain forwards, two plain backwards, element-wise
 // glue); ws: backward_normalized_workspace_floats floats.
 size_t backward_normalized_workspace_floats(int d, int BH, int T);

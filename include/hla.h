@@ -259,7 +259,8 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
  *
  * hla_backward_workspace_bytes: device workspace bytes the backward call of op
  * needs for (dtype, B, H, T, d, dv); 0 when the request is invalid or has no
- * backward kernel (HLA_OP_HLA2 and HLA_OP_HLA2_NORM, undecayed, d = dv in {32, 64}).
+ * backward kernel (HLA_OP_HLA2, HLA_OP_HLA2_NORM and HLA_OP_AHLA, undecayed, d = dv in
+ * {32, 64}).
  *
  * hla2_backward: given the output gradient dout [B][H][T][dv] (fp32, device),
  * writes dq, dk [B][H][T][d] and dv_out [B][H][T][dv] (fp32, device, caller-
@@ -278,6 +279,18 @@ hla_status_t hla_step(hla_op_t op, float* state, const void* q, const void* k, c
 size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv);
 hla_status_t hla2_backward(const void* q, const void* k, const void* v, const float* dout, float* dq,
+                           float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
+                           const float* gamma, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass of the AHLA output, O = A (A V), A = L (.) Q K^T (Metodología 2; reverse-mode
+ * derivatives of the masked form).  Same arguments, layouts, workspace query
+ * (hla_backward_workspace_bytes(HLA_OP_AHLA, ...)), errors and stream semantics as
+ * hla2_backward.  fp32 on the CUDA cores for every dtype and d: the forward's carried (P0, E0)
+ * per 64-token chunk, the adjoint terms Q^T dO, Q^T (A^T dO), Q^T K per chunk, two suffix sums
+ * (dE', dP') with their cross term, and the per-chunk gradients.
+ */
+hla_status_t ahla_backward(const void* q, const void* k, const void* v, const float* dout, float* dq,
                            float* dk, float* dv_out, int B, int H, int T, int d, int dv, hla_dtype_t dtype,
                            const float* gamma, void* workspace, size_t workspace_bytes, void* stream);
 

@@ -261,6 +261,51 @@ def ahla_chunked_backward(q, k, v, do, c):
     return tuple(np.vstack(g[::-1])[:T] for g in (gq, gk, gv))
 
 
+def ahla_chunk_parallel_backward(q, k, v, do, c):
+    """The AHLA GPU backward's algebra, chunk-parallel: carried (P0, E0) from the forward's
+    prefixes; adjoints leaving each chunk as suffix sums of its terms
+        Y = Q^T dO,  U = Q^T (A^T dO),  M = Q^T K:   dE'(c) = sum_{m>c} Y_m,
+        dP'(c) = sum_{m>c} (U_m + M_m dE'(m));
+    then per chunk dY = A^T dO + K dE', dA = L (.) (dO Y^T + dY V^T),
+        dQ = dO E0^T + dY P0^T + dA K,  dK = Y dE'^T + V dP'^T + dA^T Q,  dV = K dP' + A^T dY."""
+    d, dv = q.shape[1], v.shape[1]
+    Qs, Ks, Vs, Gs = chunks(q, c), chunks(k, c), chunks(v, c), chunks(do, c)
+    n = len(Qs)
+    L = np.tril(np.ones((c, c)))
+    P0s, E0s = [], []
+    P0, E0 = np.zeros((d, dv)), np.zeros((d, dv))
+    for Q, K, V in zip(Qs, Ks, Vs):
+        P0s.append(P0); E0s.append(E0)
+        A = L * (Q @ K.T)
+        Y = Q @ P0 + A @ V
+        P0, E0 = P0 + K.T @ V, E0 + K.T @ Y
+    Yt = [Q.T @ dO for Q, dO in zip(Qs, Gs)]
+    U = [Q.T @ ((L * (Q @ K.T)).T @ dO) for Q, K, dO in zip(Qs, Ks, Gs)]
+    M = [Q.T @ K for Q, K in zip(Qs, Ks)]
+    dE = [sum((Yt[m] for m in range(i + 1, n)), np.zeros((d, dv))) for i in range(n)]
+    dP = [sum((U[m] + M[m] @ dE[m] for m in range(i + 1, n)), np.zeros((d, dv))) for i in range(n)]
+    gq, gk, gv = [], [], []
+    for i, (Q, K, V, dO) in enumerate(zip(Qs, Ks, Vs, Gs)):
+        A = L * (Q @ K.T)
+        Y = Q @ P0s[i] + A @ V
+        dY = A.T @ dO + K @ dE[i]
+        dA = L * (dO @ Y.T + dY @ V.T)
+        gq.append(dO @ E0s[i].T + dY @ P0s[i].T + dA @ K)
+        gk.append(Y @ dE[i].T + V @ dP[i].T + dA.T @ Q)
+        gv.append(K @ dP[i] + A.T @ dY)
+    T = q.shape[0]
+    return tuple(np.vstack(g)[:T] for g in (gq, gk, gv))
+
+
+@pytest.mark.parametrize("T,c", [(1, 4), (9, 4), (37, 8), (64, 16), (100, 32)])
+def test_ahla_chunk_parallel_gradients_match_the_reference(T, c):
+    q, k, v, do = rand(T, 5, 3, T + 5 * c)
+    want = ahla_grads(q, k, v, do)
+    got = ahla_chunk_parallel_backward(q, k, v, do, c)
+    for a, b in zip(got, want):
+        np.testing.assert_allclose(a, b, rtol=1e-10, atol=1e-10)
+
+
 @pytest.mark.parametrize("T,c", [(1, 4), (9, 4), (37, 8), (64, 16), (100, 32)])
 def test_ahla_chunked_reverse_walk_matches_the_reference(T, c):
     q, k, v, do = rand(T, 5, 3, T + 2 * c)

@@ -138,3 +138,34 @@ def test_normalised_backward_single_token():
         scale = 2 * abs(float(vh @ dh)) / abs(s)
         assert float(dq[0, h, 0].norm()) <= 1e-5 * scale * float(kh.norm())
         assert float(dk[0, h, 0].norm()) <= 1e-5 * scale * float(qh.norm())
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [32, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 333])
+def test_ahla_backward_parity(dtype, d, T):
+    """AHLA's gradient (ahla_backward, fp32 on the CUDA cores) against ``oracle.backward.ahla_grads``
+    (reverse-mode through O = A (A V), pinned by finite differences)."""
+    from oracle.backward import ahla_grads
+    q, k, v, do = _case(dtype, 1, 2, T, d, seed=T + 2 * d)
+    dev = torch.device("cuda:0")
+    got = hla.ahla_backward(q.to(dev), k.to(dev), v.to(dev), do.to(dev))
+    torch.cuda.synchronize()
+    for h in range(2):
+        want = ahla_grads(q[0, h], k[0, h], v[0, h], do[0, h])
+        for name, gt, wt in zip(("dq", "dk", "dv"), got, want):
+            err = oracle.max_row_rel_err(gt[0, h].cpu(), wt)
+            assert err <= TOL[dtype], (name, h, err)
+
+
+def test_ahla_backward_many_heads_and_chunks():
+    from oracle.backward import ahla_grads
+    q, k, v, do = _case("bf16", 2, 3, 1000, 64, seed=8)
+    dev = torch.device("cuda:0")
+    got = hla.ahla_backward(q.to(dev), k.to(dev), v.to(dev), do.to(dev))
+    torch.cuda.synchronize()
+    for bh in range(6):
+        b, h = divmod(bh, 3)
+        want = ahla_grads(q[b, h], k[b, h], v[b, h], do[b, h])
+        for name, gt, wt in zip(("dq", "dk", "dv"), got, want):
+            assert oracle.max_row_rel_err(gt[b, h].cpu(), wt) <= TOL["bf16"], (name, bh)
