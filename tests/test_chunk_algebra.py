@@ -397,6 +397,143 @@ def test_decay_every_term_is_needed(term):
     assert rel(decay_forward(q, k, v, 0.9, 16, drop=term), ref) > 1e-3
 
 
+def decay_walk_chunk(Q, K, V, g, S0, C0, G0, drop=None):
+    """One chunk of the decayed second-order walker, state (S0, C0, G0) carried in.
+
+    Returns O and the state after the chunk:
+        S0' = rho S0 + K^T Lam K,  C0' = rho C0 + Q^T Lam V,  G0' = rho G0 + K^T Y,
+        Y = U^T Lam V + rho K C0,
+        O = W V + Gam (Z C0 - Q G0),  Z = Gam P + H K,  P = Q S0,
+        W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T).
+    ``drop`` zeroes one named term (used only to show that each term is needed)."""
+    c = Q.shape[0]
+    tau = np.arange(c)
+    lam, rho, Gam = g ** (c - 1 - tau), g ** c, g ** (tau + 1)
+    Dl = tau[:, None] - tau[None, :]
+    Dg = np.where(Dl >= 0, g ** np.maximum(Dl, 0), 0.0)
+    keep = lambda name, x: 0.0 * x if drop == name else x
+    As = Q @ K.T
+    A, U = np.tril(As), np.triu(As, 1)
+    At = Dg * As
+    H = np.where(Dl > 0, (Dg - 1.0) * As, 0.0)
+    P = Q @ S0
+    W = Dg * (Gam[:, None] * (P @ Q.T) + At @ A.T + H @ U.T)
+    Z = Gam[:, None] * P + H @ K
+    O = W @ V + Gam[:, None] * (Z @ C0 - Q @ G0)
+    Y = U.T @ (lam[:, None] * V) + keep("rhoKC0", rho * (K @ C0))
+    return O, (rho * S0 + K.T @ (lam[:, None] * K), rho * C0 + Q.T @ (lam[:, None] * V), rho * G0 + K.T @ Y)
+
+
+def decay_walk_summary(q, k, v, g, c):
+    """A summary walk over whole chunks from the zero state: S and the chunk contributions
+    to G enter with their weight rho^(N-1-l) (applied to Lam K and to Y), C is carried chunk
+    to chunk (Y needs it), Khat = K^T K is summed unweighted; rho_seg = g^(cN)."""
+    d, dv = q.shape[1], v.shape[1]
+    N = q.shape[0] // c
+    tau = np.arange(c)
+    rho = g ** c
+    S, G, Kh = np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, d))
+    C0 = np.zeros((d, dv))
+    for l in range(N):
+        Q, K, V = (x[l * c:(l + 1) * c] for x in (q, k, v))
+        lam = g ** (c - 1 - tau)
+        w = g ** (c * (N - l) - 1 - tau)                       # lam rho^(N-1-l)
+        U = np.triu(Q @ K.T, 1)
+        Y = U.T @ (lam[:, None] * V) + rho * (K @ C0)
+        S = S + K.T @ (w[:, None] * K)
+        G = G + K.T @ (rho ** (N - 1 - l) * Y)
+        Kh = Kh + K.T @ K
+        C0 = rho * C0 + Q.T @ (lam[:, None] * V)
+    return dict(S=S, C=C0, G=G, Khat=Kh, rho=g ** (c * N))
+
+
+def decay_fold(slots, n):
+    """The output walker's prologue fold of slots 0..n-1 (exclusive prefix of slot n):
+    S0 = sum w_m S_m, C0 = sum w_m C_m, G0 = sum w_m (G_m + Ksuf(m+1) C_m), with
+    w_m = prod_{m<p<n} rho_p and Ksuf(m+1) = sum_{m<l<n} Khat_l (unweighted)."""
+    S0, C0, G0 = (0.0 * slots[0][x] for x in ("S", "C", "G"))
+    w, Ksuf = 1.0, 0.0 * slots[0]["Khat"]
+    for m in range(n - 1, -1, -1):
+        s = slots[m]
+        S0 = S0 + w * s["S"]
+        C0 = C0 + w * s["C"]
+        G0 = G0 + w * (s["G"] + Ksuf @ s["C"])
+        Ksuf = Ksuf + s["Khat"]
+        w = w * s["rho"]
+    return S0, C0, G0
+
+
+@pytest.mark.parametrize("gamma", [1.0, 0.999, 0.95, 0.5])
+@pytest.mark.parametrize("T,c", [(5, 8), (37, 8), (64, 16), (100, 16)])
+def test_decay_walk_chunk_step_matches_recurrence(T, c, gamma):
+    q, k, v = rand_head(T, 4, 3, seed=T + int(gamma * 1000))
+    S0, C0, G0 = np.zeros((4, 4)), np.zeros((4, 3)), np.zeros((4, 3))
+    outs = []
+    for Q, K, V in zip(chunks(q, c), chunks(k, c), chunks(v, c)):
+        O, (S0, C0, G0) = decay_walk_chunk(Q, K, V, gamma, S0, C0, G0)
+        outs.append(O)
+    assert rel(np.vstack(outs)[:T], recur("hla2d", q, k, v, gamma=gamma)) < 1e-12
+
+
+def test_decay_walk_needs_the_rho_k_c0_term():
+    """Without the carried C0 in Y the state walk drifts from the recurrence."""
+    q, k, v = rand_head(64, 4, 3, seed=5)
+    S0, C0, G0 = np.zeros((4, 4)), np.zeros((4, 3)), np.zeros((4, 3))
+    outs = []
+    for Q, K, V in zip(chunks(q, 16), chunks(k, 16), chunks(v, 16)):
+        O, (S0, C0, G0) = decay_walk_chunk(Q, K, V, 0.9, S0, C0, G0, drop="rhoKC0")
+        outs.append(O)
+    assert rel(np.vstack(outs), recur("hla2d", q, k, v, gamma=0.9)) > 1e-3
+
+
+@pytest.mark.parametrize("gamma", [0.999, 0.9, 0.5])
+@pytest.mark.parametrize("lengths", [[2], [1, 3, 2], [2, 2, 2, 2, 2]])
+def test_decay_segment_summaries_and_fold_equal_the_combine(gamma, lengths):
+    """Walked segment summaries against the decayed combine of per-token summaries, and the
+    prologue fold against the exclusive fold of that combine."""
+    c, d, dv = 8, 4, 3
+    T = c * sum(lengths)
+    q, k, v = rand_head(T, d, dv, seed=sum(lengths) + int(gamma * 100))
+    b = [0]
+    for n in lengths:
+        b.append(b[-1] + n * c)
+    slots = [decay_walk_summary(q[b[i]:b[i + 1]], k[b[i]:b[i + 1]], v[b[i]:b[i + 1]], gamma, c)
+             for i in range(len(lengths))]
+    # reference: walk the recurrence's state over each segment and across them
+    for n in range(len(lengths) + 1):
+        S0, C0, G0 = decay_fold(slots, n) if n else (np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv)))
+        S, C, G = np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv))
+        for t in range(b[n]):
+            S, C, G = gamma * S, gamma * C, gamma * G
+            G = G + np.outer(k[t], k[t]) @ C
+            S = S + np.outer(k[t], k[t])
+            C = C + np.outer(q[t], v[t])
+        for x, y in ((S0, S), (C0, C), (G0, G)):
+            np.testing.assert_allclose(x, y, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("gamma", [0.97, 0.5])
+@pytest.mark.parametrize("T,c,NCH,ratio", [(200, 8, 5, 1), (200, 8, 6, 3), (129, 16, 2, 2), (70, 8, 4, 4)])
+def test_decay_walk_segment_plan_matches_recurrence(T, c, NCH, ratio, gamma):
+    """Summary segments of NCH/ratio chunks walked from zero, each output segment folding
+    the slots before it, then walking its chunks: the decayed walker's stages end to end."""
+    d, dv = 4, 3
+    q, k, v = rand_head(T, d, dv, seed=T + NCH + ratio)
+    nchunks = -(-T // c)
+    NCHs = NCH // ratio
+    n_out = -(-nchunks // NCH)
+    slots = [decay_walk_summary(*(x[i * NCHs * c:(i + 1) * NCHs * c] for x in (q, k, v)), gamma, c)
+             for i in range((n_out - 1) * ratio)]
+    outs = []
+    for n in range(n_out):
+        state = decay_fold(slots, n * ratio) if n else (np.zeros((d, d)), np.zeros((d, dv)), np.zeros((d, dv)))
+        lo, hi = n * NCH * c, min((n + 1) * NCH * c, T)
+        for Q, K, V in zip(chunks(q[lo:hi], c), chunks(k[lo:hi], c), chunks(v[lo:hi], c)):
+            O, state = decay_walk_chunk(Q, K, V, gamma, *state)
+            outs.append(O)
+    assert rel(np.vstack(outs)[:T], recur("hla2d", q, k, v, gamma=gamma)) < 1e-11
+
+
 # ---------------------------------------------------------------------------
 # ratio-normalised AHLA / third order: the combine of the normaliser vectors
 # ---------------------------------------------------------------------------
