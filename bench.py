@@ -181,9 +181,10 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
         # (A K) C0 (2D^2 each); S0 C0 once per chunk (2D^3 / c)
         flops = 8 * c * D + 2 * c * c + 6 * D * D + 2 * D ** 3 // c
     elif w.op == "hla2d" and path == "tc":
-        # per token: A* = Q K^T, Gam P Q^T, H K, W V (2cD each); Q S0, Q G0, Q M0, (Gam H K) C0
-        # (2D^2 each); H A*^T and A A^T (2c^2 each)
-        flops = 8 * c * D + 8 * D * D + 4 * c * c
+        # the decayed output walker forms O and carries the state. Per token: A* = Q K^T,
+        # Gam P Q^T, H K, W V (2cD each), At A^T and H U^T (2c^2 each), P = Q S0, Z C0, Q G0
+        # (2D^2 each); the state: K^T Lam K, Q^T Lam V, K C0, K^T Y (2D^2 each), U^T Lam V (2cD)
+        flops = 10 * c * D + 14 * D * D + 4 * c * c
     else:
         # per token: A = Q K^T (2cD), P = Q S0 (2D^2), W = [P|A][Q|A]^T (2c(D+c)), O = [Q|W][R0;V] (2D(D+c))
         flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)

@@ -142,11 +142,12 @@ constexpr int PH_MAX = 9;
 cudaError_t launch_prefix(const float* sums, float* pre, int NS, int NSp, int BH, cudaStream_t st,
                           bool left_vec = false);
 
-// The decayed second-order forward, chunk-parallel (tc_decay.cu).
-size_t decay_workspace_bytes(int BH, int T);
-int decay_kernel_launches();
+// The decayed second-order forward as a segment walk (tc_decay.cu): the summary walk, then the
+// output walk with the prefix of the summaries folded into each output CTA.
+size_t decay_workspace_bytes(int BH, int T, int seg_chunks);
+int decay_kernel_launches(int BH, int T, int seg_chunks);
 cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
-                          int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev);
+                          int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev, int seg_chunks);
 
 // The AHLA forward on the tcgen05 walkers, plain or ratio-normalised, with per-head decay when
 // gamma is given (tc_ahla.cu).  The decayed walk needs the prefix folded into the output walker

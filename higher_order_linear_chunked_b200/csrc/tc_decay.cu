@@ -10,15 +10,11 @@
 // Chunk algebra.  c = 128 tokens, local index tau.  Gam_tau = g^(tau+1), lam_tau = g^(c-1-tau),
 // rho = g^c.  A* = Q K^T (no mask), A = L (.) A*, U = strict upper part of A*,
 // At[tau][i] = g^(tau-i) A*[tau][i] for i <= tau, H[tau][i] = (g^(tau-i) - 1) A*[tau][i] for
-// i < tau (0 elsewhere).
-//   summary of a chunk from the zero state:
-//     S = K^T Lam K,   C = Q^T Lam V,   Khat = K^T K,   G = K^T (U^T Lam V)
-//   state entering chunk l (every earlier chunk is full):
-//     S0(l+1) = rho S0(l) + S_l,   C0(l+1) = rho C0(l) + C_l,
-//     G0(l+1) = rho G0(l) + G_l + rho Khat_l C0(l)
-//   output of a chunk with carried-in (S0, C0, G0), P = Q S0:
-//     W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T),   Dg[tau][j] = g^(tau-j)
-//     O = W V + Gam (Gam P + H K) C0 - Gam (Q G0)
+// i < tau (0 elsewhere).  With (S0, C0, G0) carried into a chunk (every earlier chunk full):
+//     S0' = rho S0 + K^T Lam K,   C0' = rho C0 + Q^T Lam V,   G0' = rho G0 + K^T Y,
+//     Y = U^T Lam V + rho K C0        (the chunk's G plus rho Khat C0, Khat = K^T K)
+//     O = W V + Gam (Z C0 - Q G0),    Z = Gam P + H K,   P = Q S0,
+//     W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T),   Dg[tau][j] = g^(tau-j).
 // The cross terms are the carried-in S0 times the chunk's C (through P Q^T), the chunk's
 // decayed-minus-undecayed key moment times C0 (through H K), and the carried-in
 // Gam S0 C0 - G0 (through Gam P C0 and Q G0).
@@ -27,14 +23,12 @@
 // writing it as a difference of separately rounded products would lose the weight to bf16
 // rounding at strong decay (H A*^T + A A^T) or at weak decay (At A*^T - A U^T).
 //
-// Kernels (every chunk independent):
-//   k_dec_summary (tcgen05, two CTAs per SM)   chunk summaries (S, C, Khat, G^T), fp32
-//   k_dec_prefix_sc, k_dec_cross, k_dec_prefix_g (CUDA cores)
-//                                               in place: S0, C0; Y^T = G^T + rho C0^T Khat;
-//                                               G0^T (Khat is symmetric)
-//   k_dec_output (tcgen05, persistent: one CTA per SM over the chunks)
-//                                               turns (S0, C0, G0^T) into bf16 operand tiles
-//                                               and forms O, written by TMA bulk tensor stores
+// Kernels (a segment walk, as for the undecayed second order; only segment summaries reach HBM):
+//   k_dsum  (tcgen05, one CTA per summary segment x head)  walks its chunks from the zero state
+//                                                         and writes the segment summary
+//   k_dwalk (tcgen05, one CTA per output segment x head)   folds the summaries before its
+//                                                         segment, then walks its chunks with
+//                                                         the state in TMEM, writing O by TMA
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -49,24 +43,7 @@ namespace tc {
 namespace {
 
 constexpr int DNT = 256;                  // 8 warps, two per TMEM lane quadrant
-constexpr int DSUM = 4 * D * D;           // chunk state: S, C, Khat, G^T (then Y^T, then G0^T)
 constexpr uint32_t QTILE = D * D * 2;     // one 64 x 64 bf16 tile = 8 KB
-
-struct DParams {
-    int T, BH, H, NC;
-    const float* gamma;
-    float* sums;      // per head NC x DSUM fp32, in the blocked layout of dsum()
-    int* status;
-};
-
-// Chunk states of a head are stored in blocks of 32 consecutive elements of one matrix,
-// chunk-major inside a block: element e (0 .. DSUM) of chunk l sits at
-//     sums + bh NC DSUM + (e / 32) NC 32 + l 32 + e % 32.
-// A warp that follows one block across the chunks reads one contiguous run, and one chunk's
-// state is 512 whole 128-byte lines.
-__device__ __forceinline__ float* dsum(const DParams& p, int bh, int l, int e) {
-    return p.sums + (size_t)bh * p.NC * DSUM + (size_t)(e >> 5) * p.NC * 32 + l * 32 + (e & 31);
-}
 
 // g^n for n >= 0 (binary powering).
 __device__ __forceinline__ float gpow_n(float g, int n) {
@@ -109,353 +86,148 @@ __device__ __forceinline__ auto k2s(uint64_t d0, int s) {
 }
 __device__ __forceinline__ auto mns(uint64_t d0, int s) { return d0 + (uint64_t)(s * 128); }
 
-// ---------------------------------------------------------------- chunk summaries
-// Shared memory (offsets from the dynamic base, which is 1024-byte aligned):
-constexpr uint32_t S1_U = 0;                // U: [128 j][128 i] K-major, two atoms
-constexpr uint32_t S1_LK = S1_U + 2 * TILE; // Lam K  [tok][feat]   } equally spaced: the
-constexpr uint32_t S1_LV = S1_LK + TILE;    // Lam V  [tok][feat]   } N = 192 MN-major operand
-constexpr uint32_t S1_K = S1_LV + TILE;     // K      [tok][feat]   } [Lam K | Lam V | K]
-constexpr uint32_t S1_Q = S1_K + TILE;      // Q, then Y = U^T Lam V
-constexpr uint32_t S1_V = S1_Q + TILE;      // V
-constexpr uint32_t S1_TAB = S1_V + TILE;    // lam[128]
-constexpr uint32_t S1_BAR = S1_TAB + C * 4;
-constexpr uint32_t S1_BYTES = S1_BAR + 64;  // no slack: checked at run time
-// The summary is staged (fp32, rows swizzled by 16-byte chunk) over U, Lam K, Lam V.
-
-// Threads: warp w reads TMEM lane quadrant (w & 3) and half (w >> 2) of the columns.
-// Rounds: R1 A* = Q K^T                                -> E1: U to bf16; Lam K, Lam V
-//         R2 Y = U^T Lam V; [K^T ; Q^T][Lam K | Lam V | K]  (S, -, Khat ; -, C, -)
-//                                                      -> E2: Y to bf16; S, C, Khat staged
-//         R3 [Y^T ; V^T] K   (lanes 0-63: G^T)          -> E3: G^T staged; summary stored
-__global__ void __launch_bounds__(DNT, 2)
-k_dec_summary(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-              const __grid_constant__ CUtensorMap tv, DParams p) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* sm = smem_raw;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;
-    const int chunk = blockIdx.x, bh = blockIdx.y;
-    if (ptx::smem_u32(sm) & 1023) {            // the swizzled tiles need a 1024-byte base
-        if (tid == 0) set_status(p.status, DEV_ALIGN);
-        return;
-    }
-    float* lam = reinterpret_cast<float*>(sm + S1_TAB);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S1_BAR);
-    MmaSync ms{bar_load + 1, 0};
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 2);
-    const float g = p.gamma[bh % p.H];
-    if (tid == 0) {
-        ptx::mbar_init(bar_load, 1);
-        ptx::mbar_init(ms.bar, 1);
-        ptx::fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-        const int t0 = chunk * C;
-        ptx::mbar_arrive_expect_tx(bar_load, 3 * TILE);
-        ptx::tma_load_3d(sm + S1_Q, &tq, bar_load, 0, t0, bh);
-        ptx::tma_load_3d(sm + S1_K, &tk, bar_load, 0, t0, bh);
-        ptx::tma_load_3d(sm + S1_V, &tv, bar_load, 0, t0, bh);
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 256);
-        ptx::tmem_relinquish();
-    }
-    if (tid < C) lam[tid] = gpow_n(g, C - 1 - tid);
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t sb = ptx::smem_u32(sm);
-    bool ok = ptx::mbar_wait(bar_load, 0);     // every thread: the tiles are read below
-    if (ok && tid == 0) {
-        ptx::tc_fence_after();
-        const uint64_t dQ = kdesc(sb + S1_Q, 0), dK = kdesc(sb + S1_K, 0);
-        constexpr uint32_t I_QK = ptx::idesc_bf16(128, 128, false, false);
-        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem, k1s(dQ, s), k1s(dK, s), I_QK, s > 0);
-    }
-    // Lam K and Lam V: scale each token row by lam; the swizzle moves 16-byte chunks within a
-    // row, so a chunk keeps its place.
-    if (ok) {
-        const float l = lam[row];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint32_t off = row * 128 + (half * 4 + c) * 16;
-            const uint4 kx = *reinterpret_cast<const uint4*>(sm + S1_K + off);
-            const uint4 vx = *reinterpret_cast<const uint4*>(sm + S1_V + off);
-            auto scale = [&](uint32_t w) {
-                __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w);
-                const float2 f = __bfloat1622float2(h);
-                return ptx::pack_bf16(f.x * l, f.y * l);
-            };
-            *reinterpret_cast<uint4*>(sm + S1_LK + off) = make_uint4(scale(kx.x), scale(kx.y), scale(kx.z), scale(kx.w));
-            *reinterpret_cast<uint4*>(sm + S1_LV + off) = make_uint4(scale(vx.x), scale(vx.y), scale(vx.z), scale(vx.w));
-        }
-    }
-    ok = __syncthreads_and(ok) != 0;
-    if (ok) ok = ms.commit_wait(tid == 0);      // R1 done
-    if (ok) {
-        // E1: U = strict upper part of A*, row `row` (this thread: columns half*64 .. +63)
-        float v[32];
-#pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 + 31 < quad * 32) {                                 // wholly below the diagonal
-                st_row32_zero(sm + S1_U, row, c0);
-                continue;
-            }
-            ptx::tmem_ld32(tmem + lane_base + c0, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i <= row) v[i] = 0.f;
-            st_row32(sm + S1_U, row, c0, v);
-        }
-        sync_for_mma();
-        if (tid == 0) {
-            constexpr uint32_t I_Y = ptx::idesc_bf16(128, 64, true, true);
-            constexpr uint32_t I_ST = ptx::idesc_bf16(128, 192, true, true);
-            const uint64_t dU = mdesc(sb + S1_U, TILE, 0), dLV = mdesc(sb + S1_LV, TILE, 0);
-            const uint64_t dKQ = mdesc(sb + S1_K, S1_Q - S1_K, 0), dB3 = mdesc(sb + S1_LK, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 192, mns(dU, s), mns(dLV, s), I_Y, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dKQ, s), mns(dB3, s), I_ST, s > 0);
-        }
-        ok = ms.commit_wait(tid == 0);          // R2 done
-    }
-    float* stg = reinterpret_cast<float*>(sm + S1_U);   // [4][64][64] fp32, rows chunk-swizzled
-    auto put_row = [&](int m, int r, int c0, const float (&x)[32]) {
-        float4* dst = reinterpret_cast<float4*>(stg + m * D * D + r * D);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            dst[(c0 / 4 + j) ^ (r & 7)] = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
-    };
-    if (ok) {
-        // E2: Y -> bf16 over Q; S (lanes 0-63, cols 0-63), Khat (lanes 0-63, cols 128-191),
-        // C (lanes 64-127, cols 64-127) staged
-        float v[32];
-        ptx::tmem_ld32(tmem + lane_base + 192 + half * 32, v);
-        st_row32(sm + S1_Q, row, half * 32, v);
-        if (quad < 2) {
-            ptx::tmem_ld32(tmem + lane_base + half * 32, v);
-            put_row(0, row, half * 32, v);
-            ptx::tmem_ld32(tmem + lane_base + 128 + half * 32, v);
-            put_row(2, row, half * 32, v);
-        } else {
-            ptx::tmem_ld32(tmem + lane_base + 64 + half * 32, v);
-            put_row(1, row - 64, half * 32, v);
-        }
-        sync_for_mma();
-        if (tid == 0) {
-            constexpr uint32_t I_G = ptx::idesc_bf16(128, 64, true, true);
-            const uint64_t dYV = mdesc(sb + S1_Q, S1_V - S1_Q, 0), dK = mdesc(sb + S1_K, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem, mns(dYV, s), mns(dK, s), I_G, s > 0);
-        }
-        ok = ms.commit_wait(tid == 0);          // R3 done
-    }
-    if (ok) {
-        if (quad < 2) {
-            float v[32];
-            ptx::tmem_ld32(tmem + lane_base + half * 32, v);
-            put_row(3, row, half * 32, v);
-        }
-        __syncthreads();
-        const float4* st4 = reinterpret_cast<const float4*>(stg);
-        for (int f = tid; f < DSUM / 4; f += DNT) {
-            const int r = (f >> 4) & (D - 1);
-            *reinterpret_cast<float4*>(dsum(p, bh, chunk, 4 * f)) = st4[(f & ~15) | ((f & 15) ^ (r & 7))];
-        }
-    } else if (tid == 0) {
-        set_status(p.status, DEV_TIMEOUT);
-        ptx::mbar_wait(bar_load, 0, 100000000ull);
-        ptx::umma_commit(ms.bar);
-        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == 1) ptx::tmem_dealloc(tmem, 256);
-}
-
-// ---------------------------------------------------------------- prefixes (CUDA cores)
-constexpr int PNT = 256;
-
-// Exclusive decayed prefix over chunks of S (slot matrix 0) and C (matrix 1), in place:
-// X0(0) = 0, X0(l+1) = rho X0(l) + X_l.  One thread per matrix element.
-__global__ void __launch_bounds__(PNT) k_dec_prefix_sc(DParams p) {
-    const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
-    if (e >= 2 * D * D) return;
-    const float rho = gpow_n(p.gamma[bh % p.H], C);
-    float* x = dsum(p, bh, 0, e);             // chunk l at x + 32 l
-    float run = 0.f;
-    for (int l0 = 0; l0 < p.NC; l0 += 16) {
-        float y[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) y[i] = x[(l0 + i) * 32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) {
-                x[(l0 + i) * 32] = run;
-                run = fmaf(rho, run, y[i]);
-            }
-    }
-}
-
-// Per chunk: Y^T = G^T + rho C0^T Khat, in place of G^T (matrix 3).  (Y = G + rho Khat C0 and
-// Khat is symmetric.)
-__global__ void __launch_bounds__(PNT) k_dec_cross(DParams p) {
-    __shared__ __align__(16) float Kh[D * D];
-    __shared__ __align__(16) float C0[D * D];
-    const int l = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const float rho = gpow_n(p.gamma[bh % p.H], C);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int f = tid + PNT * i;
-        const float4 c = *reinterpret_cast<const float4*>(dsum(p, bh, l, D * D + 4 * f));
-        const float4 k = *reinterpret_cast<const float4*>(dsum(p, bh, l, 2 * D * D + 4 * f));
-        reinterpret_cast<float4*>(C0)[f] = c;
-        reinterpret_cast<float4*>(Kh)[f] = make_float4(rho * k.x, rho * k.y, rho * k.z, rho * k.w);
-    }
-    __syncthreads();
-    const int r = 4 * (tid >> 4), c = 4 * (tid & 15);   // rows r.. of Y^T (columns of C0), columns c..
-    float y[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const float4 gx = *reinterpret_cast<const float4*>(dsum(p, bh, l, 3 * D * D + (r + a) * D + c));
-        y[a][0] = gx.x; y[a][1] = gx.y; y[a][2] = gx.z; y[a][3] = gx.w;
-    }
-#pragma unroll 8
-    for (int k = 0; k < D; ++k) {
-        const float4 cv = *reinterpret_cast<const float4*>(C0 + k * D + r);
-        const float4 kv = *reinterpret_cast<const float4*>(Kh + k * D + c);
-        const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            y[a][0] = fmaf(cc[a], kv.x, y[a][0]); y[a][1] = fmaf(cc[a], kv.y, y[a][1]);
-            y[a][2] = fmaf(cc[a], kv.z, y[a][2]); y[a][3] = fmaf(cc[a], kv.w, y[a][3]);
-        }
-    }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4*>(dsum(p, bh, l, 3 * D * D + (r + a) * D + c)) =
-            make_float4(y[a][0], y[a][1], y[a][2], y[a][3]);
-}
-
-// Exclusive decayed prefix of Y^T (matrix 3) into G0^T, in place.
-__global__ void __launch_bounds__(PNT) k_dec_prefix_g(DParams p) {
-    const int e = blockIdx.x * PNT + threadIdx.x, bh = blockIdx.y;
-    if (e >= D * D) return;
-    const float rho = gpow_n(p.gamma[bh % p.H], C);
-    float* x = dsum(p, bh, 0, 3 * D * D + e);
-    float run = 0.f;
-    for (int l0 = 0; l0 < p.NC; l0 += 16) {
-        float y[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) y[i] = x[(l0 + i) * 32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (l0 + i < p.NC) {
-                x[(l0 + i) * 32] = run;
-                run = fmaf(rho, run, y[i]);
-            }
-    }
-}
-
-// ---------------------------------------------------------------- output (persistent)
-// One CTA per SM takes the (chunk, head) items w = blockIdx.x, blockIdx.x + gridDim.x, ...;
-// items are independent.  Q, K, V and the carried-in state tiles are double buffered: the
-// next item's TMA loads are issued as an item starts, and the epilogue warps turn the next
-// item's fp32 state into bf16 tiles while the current item's second MMA round runs.  At, H,
-// W and Gam Z are MMA A operands read from tensor memory.
+// ================================================================ segment walkers
+// The decayed second order as a walk (the state carried chunk to chunk inside one CTA, only
+// segment summaries in HBM).  Per chunk, with the carried-in (S0, C0, G0):
+//     S0' = rho S0 + K^T Lam K,   C0' = rho C0 + Q^T Lam V,   G0' = rho G0 + K^T Y,
+//     Y = U^T Lam V + rho K C0                       (G_l + rho Khat_l C0 of the chunk algebra)
+//     O = W V + Gam (Z C0 - Q G0),   Z = Gam P + H K,   P = Q S0,
+//     W = Dg (.) L (.) (Gam P Q^T + At A^T + H U^T).
+// The fp32 state stays in TMEM as MMA accumulators.  The epilogue that turns it into the next
+// chunk's bf16 operand tiles writes it back multiplied by rho; the chunk's products then
+// accumulate onto it.  S and G occupy TMEM lanes 0-63, C lanes 64-127: their products are
+// M = 128 with a stacked MN-major A operand whose other 64-row half is a 2 KB zero block
+// ([K^T ; 0], [0 ; Q^T]), so they add nothing to the other half's lanes.  The zero block lies
+// after every K tile and before every Q tile, so both stackings have a positive block offset.
 //
-// Shared memory: two stages of [Q | K | S0, G0^T | C0 | V] (72 KB each; K sits directly
-// before S0, G0^T so that [K ; S0^T ; G0^T] is one B operand), then A, U (B operands), Gam P,
-// the table of gamma powers and the barriers.
-constexpr uint32_t SQ_ = 0, SK_ = TILE, SSG_ = 2 * TILE, SC0_ = 2 * TILE + 2 * QTILE;
-constexpr uint32_t SV_ = 2 * TILE + 3 * QTILE;
-constexpr uint32_t STAGE3 = 3 * TILE + 3 * QTILE;   // 72 KB
-constexpr uint32_t S3_A = 2 * STAGE3;               // A, later the O staging boxes
-constexpr uint32_t S3_U = S3_A + 2 * TILE;          // U
-constexpr uint32_t S3_P = S3_U + 2 * TILE;          // Gam P
-constexpr uint32_t S3_TAB = S3_P + TILE;            // g^n, n = 0..256
-constexpr uint32_t S3_BAR = S3_TAB + 260 * 4;       // 2 load barriers, the MMA barrier, TMEM slot
-constexpr uint32_t S3_BYTES = S3_BAR + 64 + 1024;   // + alignment slack
+// Summary slot of a segment of N chunks (fp32): S, C, G, Khat (row-major 64 x 64 each), then
+// rho_seg = g^(cN).  Walked from the zero state; S and the G increments enter with the weight
+// rho^(N-1-l) of chunk l (on Lam K and on Y), so only C is rescaled chunk by chunk (Y needs
+// the running C0); Khat = sum K^T K is unweighted.  An output CTA of segment s folds the slots
+// before it (exclusive prefix, m from the last slot back, w the product of the later rho):
+//     S0 = sum w_m S_m,   C0 = sum w_m C_m,   G0 = sum w_m (G_m + Ksuf(m+1) C_m),
+//     Ksuf(m+1) = sum_{m<l} Khat_l.
+constexpr int WSLOT = 4 * D * D + 32;
 
-// TMEM columns
-constexpr uint32_t T3_AS = 0;     // A*, then W (fp32)        (128)
-constexpr uint32_t T3_P = 128;    // P                        (64)
-constexpr uint32_t T3_QG = 192;   // Q G0                     (64)
-constexpr uint32_t T3_HK = 256;   // H K                      (64)
-constexpr uint32_t T3_O = 320;    // O                        (64)
-constexpr uint32_t T3_AT = 384;   // At, then W (bf16 pairs)  (64)
-constexpr uint32_t T3_H = 448;    // H, then Gam Z (bf16)     (64)
+struct WParams {
+    int T, BH, H;
+    int NCH, NS;        // output walk: chunks per segment, segments per head
+    int NCHs, NSf;      // summary walk: chunks per segment, segments per head
+    int ratio;          // summary segments per output segment
+    const float* gamma;
+    float* sums;        // [BH][NSf][WSLOT]
+    int* status;
+};
 
-// Rounds per item: R1 [A* | P | Q G0] = Q [K ; S0^T ; G0^T]^T  -> E1: At, H to TMEM; A, U,
-//                                                                  Gam P to shared memory
-//                  R2 W = Gam P Q^T + At A^T + H U^T; H K      -> E2: W (masked, Dg) and
-//                                                                  Gam Z = Gam (Gam P + H K) to TMEM
-//                  R3 O = W V + (Gam Z) C0                     -> E3: O - Gam Q G0, TMA store
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+// Stacked MN-major A operand of K-step s: the 64-row block at `top` (advancing with s) over
+// the zero block `zero` (fixed), or the zero block over the block at `bottom`.
+__device__ __forceinline__ uint64_t top_over_zero(uint32_t top, uint32_t zero, int s) {
+    const uint32_t a = top + s * 2048;
+    return ptx::desc_sw128(a, zero - a, 1024);
+}
+__device__ __forceinline__ uint64_t zero_over_bottom(uint32_t zero, uint32_t bottom, int s) {
+    return ptx::desc_sw128(zero, bottom + s * 2048 - zero, 1024);
+}
+// Half the 16-byte chunks of row `row` of a [128][64] bf16 tile scaled by x into the same
+// place of another tile (the swizzle moves chunks only within a row, so any chunk keeps its
+// place).  Half h takes the physical chunks (4h + c) ^ (row mod 8): the lanes of a warp, on
+// consecutive rows, then touch eight different chunk columns instead of one.
+__device__ __forceinline__ void scale_row_half(const uint8_t* src, uint8_t* dst, int row, int half, float x) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t off = row * 128 + (((half * 4 + c) ^ (row & 7)) << 4);
+        const uint4 u = *reinterpret_cast<const uint4*>(src + off);
+        auto sc = [&](uint32_t w) {
+            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w);
+            const float2 f = __bfloat1622float2(h);
+            return ptx::pack_bf16(f.x * x, f.y * x);
+        };
+        *reinterpret_cast<uint4*>(dst + off) = make_uint4(sc(u.x), sc(u.y), sc(u.z), sc(u.w));
+    }
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    float a[16], b[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = v[i];
+        b[i] = v[16 + i];
+    }
+    ptx::tmem_st16(taddr, a);
+    ptx::tmem_st16(taddr + 16, b);
+}
+
+// ---------------------------------------------------------------- summary walk
+// Shared memory: K tiles, the zero block, Q tiles (this order), V tiles, then the scaled and
+// derived tiles.  TMEM columns: A* 0, Y 128, S 192 (lanes 0-63), G|C 256, Khat 320 (lanes 0-63).
+constexpr uint32_t W1_K0 = 0, W1_K1 = TILE, W1_Z = 2 * TILE;
+constexpr uint32_t W1_Q0 = 2 * TILE + 2048, W1_Q1 = W1_Q0 + TILE;
+constexpr uint32_t W1_V0 = W1_Q1 + TILE, W1_V1 = W1_V0 + TILE;
+constexpr uint32_t W1_WK = W1_V1 + TILE;    // rho^(N-1-l) Lam K
+constexpr uint32_t W1_LV = W1_WK + TILE;    // Lam V
+constexpr uint32_t W1_U = W1_LV + TILE;     // U [128 tau][128 i] K-major, two atoms
+constexpr uint32_t W1_Y = W1_U + 2 * TILE;  // rho^(N-1-l) Y, bf16 [tau][v]
+constexpr uint32_t W1_C0 = W1_Y + TILE;     // C0, bf16 [f][v]
+constexpr uint32_t W1_BAR = W1_C0 + QTILE;
+constexpr uint32_t W1_BYTES = W1_BAR + 64 + 1024;
+constexpr uint32_t T1_X = 0, T1_Y = 128, T1_S = 192, T1_GC = 256, T1_KH = 320;
+
+// Rounds per chunk n: [G += [K^T;0] Y of chunk n-1; A* = Q K^T; Y = K C0]  -> E1: U, rho Y,
+//                     Lam-scaled K and V tiles
+//                     [C += [0;Q^T] Lam V; Y += U^T Lam V] (then S, Khat in the background)
+//                                                            -> E2: Y tile; C0' tile, rho C0'
 __global__ void __launch_bounds__(DNT, 1)
-k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-             const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, DParams p) {
+k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+       const __grid_constant__ CUtensorMap tv, WParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int items = p.NC * p.BH;
-    const int w0 = blockIdx.x;
-    if (w0 >= items) return;
-    float* gp = reinterpret_cast<float*>(sm + S3_TAB);
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(sm + S3_BAR);   // [2]
-    MmaSync ms{bar_load + 2, 0};
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_load + 3);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    // the output walk may be scheduled once every summary CTA has started
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int N = p.NCHs;                     // summary segments are whole chunks
+    const int chunk0 = seg * N;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + W1_BAR);   // loads [2], MMA
+    MmaSync ms{bar + 2, 0};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 3);
+    const float g = p.gamma[bh % p.H];
+    const float rho = gpow_n(g, C);
+    const float lam = gpow_n(g, C - 1 - row);
     if (tid == 0) {
-        ptx::mbar_init(&bar_load[0], 1);
-        ptx::mbar_init(&bar_load[1], 1);
+        ptx::mbar_init(&bar[0], 1);
+        ptx::mbar_init(&bar[1], 1);
         ptx::mbar_init(ms.bar, 1);
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    int issued[2] = {0, 0}, waited[2] = {0, 0};       // thread 0's load bookkeeping
-    auto issue_loads = [&](int w, int b) {
-        uint8_t* st = sm + b * STAGE3;
-        const int bh = w / p.NC, t0 = (w % p.NC) * C;
-        ptx::mbar_arrive_expect_tx(&bar_load[b], 3 * TILE);
-        ptx::tma_load_3d(st + SQ_, &tq, &bar_load[b], 0, t0, bh);
-        ptx::tma_load_3d(st + SK_, &tk, &bar_load[b], 0, t0, bh);
-        ptx::tma_load_3d(st + SV_, &tv, &bar_load[b], 0, t0, bh);
+    int issued[2] = {0, 0};
+    auto issue = [&](int n) {
+        const int b = n & 1;
+        const int t0 = (chunk0 + n) * C;
+        ptx::mbar_arrive_expect_tx(&bar[b], 3 * TILE);
+        ptx::tma_load_3d(sm + (b ? W1_Q1 : W1_Q0), &tq, &bar[b], 0, t0, bh);
+        ptx::tma_load_3d(sm + (b ? W1_K1 : W1_K0), &tk, &bar[b], 0, t0, bh);
+        ptx::tma_load_3d(sm + (b ? W1_V1 : W1_V0), &tv, &bar[b], 0, t0, bh);
         ++issued[b];
     };
-    // carried-in S0, C0 and G0^T of item w -> bf16 operand tiles of stage b, row for row (row r,
-    // 16-byte chunk j at j ^ (r & 7)); S0 is symmetric, so its rows serve as the K-major S0^T
-    auto convert_state = [&](int w, int b) {
-        uint8_t* st = sm + b * STAGE3;
-        const int bh = w / p.NC, l = w % p.NC;
-        constexpr int NI = 3 * D * 8 / DNT;
-        float4 x[NI][2];
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
-            const float4* src = reinterpret_cast<const float4*>(dsum(p, bh, l, (t == 2 ? 3 : t) * D * D + r * D + 8 * j));
-            x[i][0] = src[0];
-            x[i][1] = src[1];
-        }
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            const int f = tid + DNT * i, t = f >> 9, r = (f >> 3) & 63, j = f & 7;
-            const uint32_t tile = t == 0 ? SSG_ : t == 1 ? SC0_ : SSG_ + QTILE;
-            *reinterpret_cast<uint4*>(st + tile + r * 128 + ((j ^ (r & 7)) << 4)) =
-                make_uint4(ptx::pack_bf16(x[i][0].x, x[i][0].y), ptx::pack_bf16(x[i][0].z, x[i][0].w),
-                           ptx::pack_bf16(x[i][1].x, x[i][1].y), ptx::pack_bf16(x[i][1].z, x[i][1].w));
-        }
-    };
-    if (tid == 0) issue_loads(w0, 0);
+    if (tid == 0) {
+        issue(0);
+        if (N > 1) issue(1);
+    }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
-    convert_state(w0, 0);
+    // the zero block and C0 = 0; U's blocks wholly below the diagonal are zero in every chunk
+    for (int i = tid; i < 2048 / 16; i += DNT) reinterpret_cast<uint4*>(sm + W1_Z)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < QTILE / 16; i += DNT) reinterpret_cast<uint4*>(sm + W1_C0)[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+        if (c0 + 31 < quad * 32) st_row32_zero(sm + W1_U, row, c0);
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
     __syncthreads();
@@ -463,10 +235,382 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t sb = ptx::smem_u32(sm);
-    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 256, false, false);
+    {
+        // S, G|C and Khat start at zero.  Their products always accumulate: one that cleared
+        // its accumulator would clear the lanes the other half of G|C holds.
+        float z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+        tmem_st32(tmem + lane_base + T1_S + half * 32, z);
+        tmem_st32(tmem + lane_base + T1_GC + half * 32, z);
+        tmem_st32(tmem + lane_base + T1_KH + half * 32, z);
+        ptx::tmem_st_wait();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    constexpr uint32_t I_QK = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
+    constexpr uint32_t I_MN = ptx::idesc_bf16(128, 64, true, true);
+    bool ok = true;
+    int waited[2] = {0, 0};
+    for (int n = 0; n < N; ++n) {
+        const int b = n & 1;
+        const uint32_t Qb = b ? W1_Q1 : W1_Q0, Kb = b ? W1_K1 : W1_K0, Vb = b ? W1_V1 : W1_V0;
+        ok = ptx::mbar_wait(&bar[b], (n >> 1) & 1);           // every thread reads K, V below
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        ++waited[b];
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            if (n > 0) {                                        // G of chunk n-1
+                const uint32_t Kp = b ? W1_K0 : W1_K1;
+                const uint64_t dY = mdesc(sb + W1_Y, TILE, 0);
+                for (int s = 0; s < 8; ++s)
+                    ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z, s), mns(dY, s), I_MN, 1);
+            }
+            const uint64_t dQ = kdesc(sb + Qb, 0), dK = kdesc(sb + Kb, 0), dC0 = mdesc(sb + W1_C0, TILE, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_X, k1s(dQ, s), k1s(dK, s), I_QK, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_Y, k1s(dK, s), mns(dC0, s), I_KM, s > 0);
+        }
+        if (!ms.commit_wait(tid == 0)) { ok = false; break; }
+        if (tid == 0 && n >= 1 && n + 1 < N) issue(n + 1);      // stage b^1: chunk n-1 is consumed
+        {
+            // E1: U (strict upper part of A*, row `row`, columns half*64 .. +63); rho Y; the
+            // weighted Lam K and Lam V tiles of this chunk
+            float v[32];
+#pragma unroll
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 + 31 < quad * 32) continue;               // zero since set-up
+                ptx::tmem_ld32(tmem + lane_base + T1_X + c0, v);
+                if (c0 <= quad * 32 + 31 && c0 + 31 >= quad * 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i <= row) v[i] = 0.f;
+                }
+                st_row32(sm + W1_U, row, c0, v);
+            }
+            ptx::tmem_ld32(tmem + lane_base + T1_Y + half * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rho;
+            tmem_st32(tmem + lane_base + T1_Y + half * 32, v);
+            scale_row_half(sm + Kb, sm + W1_WK, row, half, lam * gpow_n(rho, N - 1 - n));
+            scale_row_half(sm + Vb, sm + W1_LV, row, half, lam);
+            ptx::tmem_st_wait();
+        }
+        sync_for_mma();
+        if (tid == 0) {
+            const uint64_t dLV = mdesc(sb + W1_LV, TILE, 0), dU = mdesc(sb + W1_U, TILE, 0);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T1_GC, zero_over_bottom(sb + W1_Z, sb + Qb, s), mns(dLV, s), I_MN, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T1_Y, mns(dU, s), mns(dLV, s), I_MN, 1);
+        }
+        if (!ms.commit_wait(tid == 0)) { ok = false; break; }
+        if (tid == 0) {                                         // S and Khat run during E2
+            const uint64_t dWK = mdesc(sb + W1_WK, TILE, 0), dKm = mdesc(sb + Kb, TILE, 0);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T1_S, top_over_zero(sb + Kb, sb + W1_Z, s), mns(dWK, s), I_MN, 1);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T1_KH, top_over_zero(sb + Kb, sb + W1_Z, s), mns(dKm, s), I_MN, 1);
+        }
+        {
+            // E2: the weighted Y to bf16; C0' (lanes 64-127) to its tile and back as rho C0'
+            float v[32];
+            ptx::tmem_ld32(tmem + lane_base + T1_Y + half * 32, v);
+            const float wy = gpow_n(rho, N - 1 - n);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= wy;
+            st_row32(sm + W1_Y, row, half * 32, v);
+            if (quad >= 2 && n + 1 < N) {
+                ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
+                st_row32(sm + W1_C0, row - 64, half * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= rho;
+                tmem_st32(tmem + lane_base + T1_GC + half * 32, v);
+                ptx::tmem_st_wait();
+            }
+        }
+        sync_for_mma();
+    }
+    if (ok) {
+        if (tid == 0) {
+            const uint32_t Kp = ((N - 1) & 1) ? W1_K1 : W1_K0;
+            const uint64_t dY = mdesc(sb + W1_Y, TILE, 0);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z, s), mns(dY, s), I_MN, 1);
+        }
+        ok = ms.commit_wait(tid == 0);
+    }
+    if (ok) {
+        // the slot: lanes 0-63 hold rows of S, G, Khat; lanes 64-127 rows of C
+        float* slot = p.sums + ((size_t)bh * p.NSf + seg) * WSLOT;
+        float v[32];
+        auto put = [&](int m, int r) {
+            float4* dst = reinterpret_cast<float4*>(slot + m * D * D + r * D + half * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        };
+        if (quad < 2) {
+            ptx::tmem_ld32(tmem + lane_base + T1_S + half * 32, v);
+            put(0, row);
+            ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
+            put(2, row);
+            ptx::tmem_ld32(tmem + lane_base + T1_KH + half * 32, v);
+            put(3, row);
+        } else {
+            ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
+            put(1, row - 64);
+        }
+        if (tid == 0) slot[4 * D * D] = gpow_n(g, C * N);
+    } else if (tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        for (int b = 0; b < 2; ++b)
+            if (issued[b] > waited[b]) ptx::mbar_wait(&bar[b], (issued[b] - 1) & 1, 100000000ull);
+        ptx::umma_commit(ms.bar);
+        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- output walk
+// Shared memory: stage b holds K_b directly followed by S0_b (one K-major B operand [K ; S0]
+// of N = 192) and Q_b.  The A tile's second atom begins with 64 rows that the causal mask
+// keeps zero; its first 2 KB are the zero block of the stacked operands (after both K tiles,
+// before both Q tiles).  V(n) sits in V slot n&1 and Lam V(n) in the other; V(n+1) is loaded
+// over Lam V(n) once R2(n) has read it.
+constexpr uint32_t W3_K0 = 0, W3_S00 = TILE, W3_K1 = TILE + QTILE, W3_S01 = 2 * TILE + QTILE;
+constexpr uint32_t W3_A = 2 * TILE + 2 * QTILE;   // A [128 tau][128 j] K-major, two atoms
+constexpr uint32_t W3_Z = W3_A + TILE;
+constexpr uint32_t W3_Q0 = W3_A + 2 * TILE, W3_Q1 = W3_Q0 + TILE;
+constexpr uint32_t W3_V0 = W3_Q1 + TILE, W3_V1 = W3_V0 + TILE;
+constexpr uint32_t W3_LK = W3_V1 + TILE;          // Lam K
+constexpr uint32_t W3_M1 = W3_LK + TILE;          // Gam P (E1 -> R2), then Y (E2 -> R3)
+constexpr uint32_t W3_C0 = W3_M1 + TILE;          // C0, bf16 [f][v]
+constexpr uint32_t W3_G0 = W3_C0 + QTILE;         // -G0, bf16 [f][v]
+constexpr uint32_t W3_U = W3_G0 + QTILE;          // U [128][128] K-major, two atoms
+constexpr uint32_t W3_TAB = W3_U + 2 * TILE;      // g^n, n = 0 .. 256
+constexpr uint32_t W3_BAR = W3_TAB + 260 * 4;
+constexpr uint32_t W3_BYTES = W3_BAR + 128 + 1024;
+// TMEM columns
+constexpr uint32_t T3W_X = 0;     // A*, then W; O2 = Z C0 - Q G0 (columns 0-63) in R3
+constexpr uint32_t T3W_P = 128;   // P, Gam P, then Z; O1 = W V in R3
+constexpr uint32_t T3W_Y = 192;   // K C0, rho K C0, then Y
+constexpr uint32_t T3W_AT = 256;  // At, then W (bf16 pairs)
+constexpr uint32_t T3W_H = 320;   // H (bf16 pairs), then Z (pairs, 320-351)
+constexpr uint32_t T3W_S = 384;   // S (lanes 0-63)
+constexpr uint32_t T3W_GC = 448;  // G (lanes 0-63) | C (lanes 64-127)
+
+// Rounds per chunk: R1 [A* | P] = Q [K ; S0]^T (issued during the last chunk's E3), K C0;
+//                     then S += [K^T;0] Lam K, C += [0;Q^T] Lam V
+//                     -> E1: At, H pairs; A, U tiles; Gam P (tile and TMEM); rho K C0
+//                   R2 W = Gam P Q^T + At A^T + H U^T; Z = Gam P + H K; Y = rho K C0 + U^T Lam V
+//                     -> E2: W pairs (Dg, mask); Z pairs; Y tile; S0' tile, rho S0'
+//                   R3 O1 = W V; O2 = Z C0 - Q G0; G += [K^T;0] Y
+//                     -> E3: O = O1 + Gam O2 (TMA store from the chunk's Q, K tiles); C0', -G0'
+//                        tiles, rho C0', rho G0';
+//                        Lam K, Lam V of the next chunk
+__global__ void __launch_bounds__(DNT, 1)
+k_dwalk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to, WParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = align1024(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int NC = (p.T + C - 1) / C;
+    const int chunk0 = seg * p.NCH;
+    const int nch = min(p.NCH, NC - chunk0);
+    float* gp = reinterpret_cast<float*>(sm + W3_TAB);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + W3_BAR);
+    uint64_t* bar_qk = bar;          // [2] Q, K of a stage
+    uint64_t* bar_v = bar + 2;       // [2] V of a slot
+    uint64_t* bar_m1 = bar + 4;      // MMA rounds (first commit)
+    uint64_t* bar_m2 = bar + 5;      // MMA rounds (second commit: products an epilogue reads last)
+    uint64_t* bar_f = bar + 6;       // [2] prologue fold, one per operand buffer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 8);
+    const float g = p.gamma[bh % p.H];
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) ptx::mbar_init(&bar[i], 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    int iq[2] = {0, 0}, wq[2] = {0, 0}, iv[2] = {0, 0}, wv[2] = {0, 0};   // loads issued / waited
+    auto issue_qk = [&](int n) {
+        const int b = n & 1, t0 = (chunk0 + n) * C;
+        ptx::mbar_arrive_expect_tx(&bar_qk[b], 2 * TILE);
+        ptx::tma_load_3d(sm + (b ? W3_Q1 : W3_Q0), &tq, &bar_qk[b], 0, t0, bh);
+        ptx::tma_load_3d(sm + (b ? W3_K1 : W3_K0), &tk, &bar_qk[b], 0, t0, bh);
+        ++iq[b];
+    };
+    auto issue_v = [&](int n) {
+        const int b = n & 1, t0 = (chunk0 + n) * C;
+        ptx::mbar_arrive_expect_tx(&bar_v[b], TILE);
+        ptx::tma_load_3d(sm + (b ? W3_V1 : W3_V0), &tv, &bar_v[b], 0, t0, bh);
+        ++iv[b];
+    };
+    if (tid == 0) {
+        issue_qk(0);
+        issue_v(0);
+        if (nch > 1) issue_qk(1);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
+    const float rho = gpow_n(g, C), lam = gpow_n(g, C - 1 - row), gam = gpow_n(g, row + 1);
+    // A's blocks above the diagonal are zero in every chunk (the zero block among them)
+#pragma unroll
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+        if (c0 > quad * 32 + 31) st_row32_zero(sm + W3_A, row, c0);
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 192, false, false);
     constexpr uint32_t I_W = ptx::idesc_bf16(128, 128, false, false);
     constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
-    // packed bf16 pairs of 32 values (columns c0 .. c0+31) into 16 TMEM columns of this lane
+    constexpr uint32_t I_MN = ptx::idesc_bf16(128, 64, true, true);
+    uint32_t ph1 = 0, ph2 = 0, phf[2] = {0, 0};
+    int fold_pending[2] = {0, 0};
+    auto mwait = [&](uint64_t* b, uint32_t& ph) {   // thread 0 has committed to b; the block agrees
+        bool good = true;
+        if (tid == 0) good = ptx::mbar_wait(b, ph);
+        ph ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
+
+    // ---- carried-in state: fold the slots m < ns of this head (the exclusive prefix of segment
+    // seg), from the last slot back with w = the product of the later rho and Ksuf = the sum of
+    // the later Khat: S0 = sum w S_m, C0 = sum w C_m, G0 = sum w G_m + X, X = sum Ksuf (w C_m).
+    // Each thread keeps a 4 x 4 block of S0, C0, sum w G and Ksuf in fp32.  X runs on the tensor
+    // core from two-term bf16 splits: A = [Ksuf_hi ; Ksuf_lo] (M = 128) times B = (w C_m)_hi and
+    // (w C_m)_lo, so X = D(lanes 0-63) + D(lanes 64-127) carries about 16 bits of each factor
+    // (TMEM columns T3W_Y; operand buffers over U and over Lam K + M1, alternately).
+    float* FS = reinterpret_cast<float*>(sm + W3_LK);    // fp32 staging (rows swizzled by
+    float* FC = reinterpret_cast<float*>(sm + W3_M1);    // 16-byte chunk), free until E0(0)
+    float* FG = reinterpret_cast<float*>(sm + W3_V1);
+    float* FX = reinterpret_cast<float*>(sm + W3_U);     // the lanes 64-127 half of X
+    auto sw = [](int i, int j) { return i * D + ((((j >> 2) ^ (i & 7)) << 2) | (j & 3)); };
+    const int ns = seg * p.ratio;
+    bool ok = true;
+    {
+        const int r = 4 * (tid >> 4), c = 4 * (tid & 15);   // this thread's 4 x 4 block
+        float aS[4][4], aC[4][4], aG[4][4], ks[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) aS[a][e] = aC[a][e] = aG[a][e] = ks[a][e] = 0.f;
+        if (ns > 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");       // the summary walk's slots
+            const float* s0 = p.sums + (size_t)bh * p.NSf * WSLOT;
+            const uint32_t buf[2] = {W3_U, W3_LK};                    // A2 16 KB, B hi 8 KB, B lo 8 KB
+            auto put4 = [&](uint32_t tile, int rr, int cc, float x0, float x1, float x2, float x3) {
+                *reinterpret_cast<uint2*>(sm + tile + ptx::sw128_offset(rr, cc)) =
+                    make_uint2(ptx::pack_bf16(x0, x1), ptx::pack_bf16(x2, x3));
+            };
+            auto lo_of = [](float x) { return x - __bfloat162float(__float2bfloat16_rn(x)); };
+            float4 xs[4], xc[4], xg[4], xk[4];
+            float rho_m = 1.f;
+            auto load = [&](int m) {
+                const float* sl = s0 + (size_t)m * WSLOT;
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    xs[a] = *reinterpret_cast<const float4*>(sl + (r + a) * D + c);
+                    xc[a] = *reinterpret_cast<const float4*>(sl + D * D + (r + a) * D + c);
+                    xg[a] = *reinterpret_cast<const float4*>(sl + 2 * D * D + (r + a) * D + c);
+                    xk[a] = *reinterpret_cast<const float4*>(sl + 3 * D * D + (r + a) * D + c);
+                }
+                rho_m = sl[4 * D * D];
+            };
+            load(ns - 1);
+            float w = 1.f;
+            for (int m = ns - 1; m >= 0 && ok; --m) {
+                float wc[4][4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    wc[a][0] = w * xc[a].x; wc[a][1] = w * xc[a].y; wc[a][2] = w * xc[a].z; wc[a][3] = w * xc[a].w;
+                }
+                if (m < ns - 1) {                                     // X += Ksuf (w C_m)
+                    const int j = m & 1;
+                    if (fold_pending[j]) {                            // the MMAs that read buffer j
+                        bool good = true;
+                        if (tid == 0) good = ptx::mbar_wait(&bar_f[j], phf[j]);
+                        phf[j] ^= 1;
+                        fold_pending[j] = 0;
+                        if (!__syncthreads_and(good)) { ok = false; break; }
+                    }
+                    const uint32_t A2 = buf[j], Bh = buf[j] + TILE, Bl = Bh + QTILE;
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        put4(A2, r + a, c, ks[a][0], ks[a][1], ks[a][2], ks[a][3]);
+                        put4(A2, 64 + r + a, c, lo_of(ks[a][0]), lo_of(ks[a][1]), lo_of(ks[a][2]), lo_of(ks[a][3]));
+                        put4(Bh, r + a, c, wc[a][0], wc[a][1], wc[a][2], wc[a][3]);
+                        put4(Bl, r + a, c, lo_of(wc[a][0]), lo_of(wc[a][1]), lo_of(wc[a][2]), lo_of(wc[a][3]));
+                    }
+                    ptx::fence_proxy_async();
+                    __syncthreads();
+                    if (tid == 0) {
+                        ptx::tc_fence_after();
+                        const uint64_t dA = kdesc(sb + A2, 0), dBh = mdesc(sb + Bh, TILE, 0), dBl = mdesc(sb + Bl, TILE, 0);
+                        for (int s = 0; s < 4; ++s)
+                            ptx::umma_bf16(tmem + T3W_Y, k1s(dA, s), mns(dBh, s), I_KM, m < ns - 2 || s > 0);
+                        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3W_Y, k1s(dA, s), mns(dBl, s), I_KM, 1);
+                        ptx::umma_commit(&bar_f[j]);
+                    }
+                    fold_pending[j] = 1;
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const float sx[4] = {xs[a].x, xs[a].y, xs[a].z, xs[a].w};
+                    const float gx[4] = {xg[a].x, xg[a].y, xg[a].z, xg[a].w};
+                    const float kx[4] = {xk[a].x, xk[a].y, xk[a].z, xk[a].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        aS[a][e] = fmaf(w, sx[e], aS[a][e]);
+                        aC[a][e] += wc[a][e];
+                        aG[a][e] = fmaf(w, gx[e], aG[a][e]);
+                        ks[a][e] += kx[e];
+                    }
+                }
+                w *= rho_m;
+                if (m > 0) load(m - 1);
+            }
+            for (int j = 0; j < 2; ++j)
+                if (fold_pending[j]) {
+                    bool good = true;
+                    if (tid == 0) good = ptx::mbar_wait(&bar_f[j], phf[j], ok ? 1000000000ull : 100000000ull);
+                    phf[j] ^= 1;
+                    fold_pending[j] = 0;
+                    if (!__syncthreads_and(good)) ok = false;
+                }
+            ptx::tc_fence_after();
+        }
+        if (ns > 1 && ok && quad >= 2) {                              // X, lanes 64-127 half
+            float v[32];
+            ptx::tmem_ld32(tmem + lane_base + T3W_Y + half * 32, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(FX + sw(row - 64, half * 32 + 4 * j)) =
+                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            *reinterpret_cast<float4*>(FS + sw(r + a, c)) = make_float4(aS[a][0], aS[a][1], aS[a][2], aS[a][3]);
+            *reinterpret_cast<float4*>(FC + sw(r + a, c)) = make_float4(aC[a][0], aC[a][1], aC[a][2], aC[a][3]);
+            *reinterpret_cast<float4*>(FG + sw(r + a, c)) = make_float4(aG[a][0], aG[a][1], aG[a][2], aG[a][3]);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
     auto st_pairs = [&](uint32_t tcol, const float (&x)[32]) {
         uint32_t r[16];
 #pragma unroll
@@ -479,139 +623,272 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
         for (int i = 0; i < 16; ++i) r[i] = 0u;
         ptx::tmem_st16u(tmem + lane_base + tcol, r);
     };
+    auto frow = [&](const float* F, int i, float (&v)[32]) {     // row i, columns half*32 .. +31
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = *reinterpret_cast<const float4*>(F + sw(i, half * 32 + 4 * j));
+            v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+        }
+    };
+    if (ok) {
+        // the state to its operand tiles (S0 by rows: S is symmetric) and, times rho, to TMEM;
+        // the At / W and H pairs above the diagonal (those that nothing overwrites) to zero
+        float v[32];
+        if (quad < 2) {
+            frow(FS, row, v);
+            st_row32(sm + W3_S00, row, half * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rho;
+            tmem_st32(tmem + lane_base + T3W_S + half * 32, v);
+            frow(FG, row, v);
+            if (ns > 1) {
+                float x[32], y[32];
+                ptx::tmem_ld32(tmem + lane_base + T3W_Y + half * 32, x);
+                frow(FX, row, y);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] += x[i] + y[i];
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = -v[i];
+            st_row32(sm + W3_G0, row, half * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= -rho;
+            tmem_st32(tmem + lane_base + T3W_GC + half * 32, v);
+        } else {
+            frow(FC, row - 64, v);
+            st_row32(sm + W3_C0, row - 64, half * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rho;
+            tmem_st32(tmem + lane_base + T3W_GC + half * 32, v);
+        }
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+            if (c0 > quad * 32 + 31) {
+                st_pairs_zero(T3W_AT + c0 / 2);
+                st_pairs_zero(T3W_H + c0 / 2);
+            }
+        ptx::tmem_st_wait();
+    }
+    __syncthreads();                                                  // FS, FC, FG, FX read
+    if (ok) {
+        ok = ptx::mbar_wait(&bar_qk[0], 0) && ptx::mbar_wait(&bar_v[0], 0);
+        if (ok) {                                                     // E0 of chunk 0
+            ++wq[0];
+            ++wv[0];
+            scale_row_half(sm + W3_K0, sm + W3_LK, row, half, lam);
+            scale_row_half(sm + W3_V0, sm + W3_V1, row, half, lam);
+        }
+    }
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    ok = __syncthreads_and(ok) != 0;
+    ptx::tc_fence_after();
+    // [A* | P] = Q [K ; S0]^T of a chunk is issued as soon as its tiles are in place: for chunk 0
+    // here, for chunk n+1 while E3 of chunk n runs
+    auto issue_qks = [&](int n) {
+        const uint32_t Qb = (n & 1) ? W3_Q1 : W3_Q0, Kb = (n & 1) ? W3_K1 : W3_K0;
+        const uint64_t dQ = kdesc(sb + Qb, 0), dKS = kdesc(sb + Kb, 0);
+        for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3W_X, k1s(dQ, s), k1s(dKS, s), I_R1, s > 0);
+    };
+    if (ok && tid == 0) issue_qks(0);
 
-    bool ok = true;
-    int cur_bh = -1;
-    int it = 0;
-    for (int w = w0; w < items && ok; w += gridDim.x, ++it) {
-        const int b = it & 1;
-        const uint32_t st = b * STAGE3;
-        const int bh = w / p.NC, chunk = w % p.NC;
-        const int wn = w + gridDim.x;
-        if (bh != cur_bh) {                  // gamma powers of this item's head (block-uniform)
-            cur_bh = bh;
-            const float g = p.gamma[bh % p.H];
-            for (int n = tid; n <= 2 * C; n += DNT) gp[n] = gpow_n(g, n);
-        }
+    for (int n = 0; n < nch && ok; ++n) {
+        const int b = n & 1;
+        const bool more = n + 1 < nch;
+        const uint32_t Qb = b ? W3_Q1 : W3_Q0, Kb = b ? W3_K1 : W3_K0;
+        const uint32_t Vn = b ? W3_V1 : W3_V0, LVn = b ? W3_V0 : W3_V1;
         if (tid == 0) {
-            if (wn < items) issue_loads(wn, b ^ 1);        // stage b^1 was freed by the last item
-            ok = ptx::mbar_wait(&bar_load[b], (it >> 1) & 1);
-            if (ok) {
-                ++waited[b];
-                ptx::tc_fence_after();
-                const uint64_t dQ = kdesc(sb + st + SQ_, 0), dKSG = kdesc(sb + st + SK_, 0);
-                for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dQ, s), k1s(dKSG, s), I_R1, s > 0);
-            }
-            ptx::bulk_wait_read();                          // the last item's O boxes (over A) are read
+            ptx::tc_fence_after();
+            const uint64_t dKS = kdesc(sb + Kb, 0), dC = mdesc(sb + W3_C0, TILE, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3W_Y, k1s(dKS, s), mns(dC, s), I_KM, s > 0);
+            ptx::umma_commit(bar_m1);
+            // the state products run during E1
+            const uint64_t dLK = mdesc(sb + W3_LK, TILE, 0), dLV = mdesc(sb + LVn, TILE, 0);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T3W_S, top_over_zero(sb + Kb, sb + W3_Z, s), mns(dLK, s), I_MN, 1);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T3W_GC, zero_over_bottom(sb + W3_Z, sb + Qb, s), mns(dLV, s), I_MN, 1);
         }
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R1 done
+        if (!mwait(bar_m1, ph1)) { ok = false; break; }              // R1 done
+        if (tid == 0 && n >= 1 && more) {
+            // stage b^1: chunk n-1 is consumed and its O boxes (over its Q, K tiles) are read
+            ptx::bulk_wait_read();
+            issue_qk(n + 1);
+        }
         {
-            // E1: from A* row `row`, columns half*64 .. +63 in two blocks of 32: At, H (TMEM, bf16
-            // pairs), A, U (shared memory); Gam P (columns half*32 .. +31).  Blocks wholly above
-            // the diagonal are zero in At, H and A, blocks wholly below it zero in U.
-            float v[32], w32[32];
+            // E1: row `row` of A*, columns half*64 .. +63 in two blocks of 32.  With the weight
+            // g^d, d = row - column: At = g^d x (d >= 0), H = At - x (d > 0), A = x (d >= 0),
+            // U = x (d < 0).
+            float vb[2][32], w32[32];
+            ptx::tmem_ld32x2(tmem + lane_base + T3W_X + half * 64, tmem + lane_base + T3W_X + half * 64 + 32,
+                             vb[0], vb[1]);
 #pragma unroll
-            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-                ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
-                if (c0 > quad * 32 + 31) {
-                    st_pairs_zero(T3_AT + c0 / 2);
-                    st_pairs_zero(T3_H + c0 / 2);
-                    st_row32_zero(sm + S3_A, row, c0);
-                    st_row32(sm + S3_U, row, c0, v);
+            for (int blk = 0; blk < 2; ++blk) {
+                const int c0 = half * 64 + 32 * blk;
+                float (&v)[32] = vb[blk];
+                if (c0 > quad * 32 + 31) {                              // above the diagonal
+                    st_row32(sm + W3_U, row, c0, v);
+                    if (c0 < 64) st_pairs_zero(T3W_H + c0 / 2);        // Z pairs were here
+                    continue;
+                }
+                if (c0 + 31 < quad * 32) {                              // below the diagonal
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w32[i] = gp[row - c0 - i] * v[i];
+                    st_pairs(T3W_AT + c0 / 2, w32);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w32[i] -= v[i];
+                    st_pairs(T3W_H + c0 / 2, w32);
+                    st_row32(sm + W3_A, row, c0, v);
+                    st_row32_zero(sm + W3_U, row, c0);
                     continue;
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int d = row - (c0 + i);                      // tau - i
-                    w32[i] = d >= 0 ? gp[d] * v[i] : 0.f;              // At
-                }
-                st_pairs(T3_AT + c0 / 2, w32);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
                     const int d = row - (c0 + i);
-                    w32[i] = d > 0 ? (gp[d] - 1.f) * v[i] : 0.f;      // H
+                    w32[i] = d >= 0 ? gp[d] * v[i] : 0.f;
                 }
-                st_pairs(T3_H + c0 / 2, w32);
+                st_pairs(T3W_AT + c0 / 2, w32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i < row) ? w32[i] - v[i] : 0.f;
+                st_pairs(T3W_H + c0 / 2, w32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i <= row) ? v[i] : 0.f;
+                st_row32(sm + W3_A, row, c0, w32);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i > row) ? v[i] : 0.f;
+                st_row32(sm + W3_U, row, c0, w32);
+            }
+            ptx::tmem_ld32x2(tmem + lane_base + T3W_P + half * 32, tmem + lane_base + T3W_Y + half * 32, vb[0], w32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                vb[0][i] *= gam;
+                w32[i] *= rho;
+            }
+            st_row32(sm + W3_M1, row, half * 32, vb[0]);
+            tmem_st32(tmem + lane_base + T3W_P + half * 32, vb[0]);
+            tmem_st32(tmem + lane_base + T3W_Y + half * 32, w32);
+            ptx::tmem_st_wait();
+        }
+        sync_for_mma();
+        if (tid == 0) {
+            const uint64_t dGP = kdesc(sb + W3_M1, 0), dQ = kdesc(sb + Qb, 0);
+            const uint64_t dA = kdesc2(sb + W3_A, 0), dU = kdesc2(sb + W3_U, 0);
+            const uint64_t dKm = mdesc(sb + Kb, TILE, 0), dUm = mdesc(sb + W3_U, TILE, 0);
+            const uint64_t dLV = mdesc(sb + LVn, TILE, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3W_X, k1s(dGP, s), k1s(dQ, s), I_W, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3W_X, tmem + T3W_AT + 8 * s, k2s(dA, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3W_X, tmem + T3W_H + 8 * s, k2s(dU, s), I_W, 1);
+            ptx::umma_commit(bar_m1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3W_P, tmem + T3W_H + 8 * s, mns(dKm, s), I_KM, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T3W_Y, mns(dUm, s), mns(dLV, s), I_MN, 1);
+            ptx::umma_commit(bar_m2);
+        }
+        if (!mwait(bar_m1, ph1)) { ok = false; break; }              // W done
+        {
+            // E2a: W = Dg (.) L (.) x to pairs
+            float v[32];
+#pragma unroll
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) continue;                      // zero since set-up
+                ptx::tmem_ld32(tmem + lane_base + T3W_X + c0, v);
                 if (c0 + 31 < quad * 32) {
-                    st_row32(sm + S3_A, row, c0, v);
-                    st_row32_zero(sm + S3_U, row, c0);
-                    continue;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= gp[row - c0 - i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int d = row - (c0 + i);
+                        v[i] = d >= 0 ? gp[d] * v[i] : 0.f;
+                    }
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i <= row) ? v[i] : 0.f;   // A
-                st_row32(sm + S3_A, row, c0, w32);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) w32[i] = (c0 + i > row) ? v[i] : 0.f;    // U
-                st_row32(sm + S3_U, row, c0, w32);
+                st_pairs(T3W_AT + c0 / 2, v);
             }
-            ptx::tmem_ld32(tmem + lane_base + T3_P + half * 32, v);
-            const float gam = gp[row + 1];
+        }
+        if (!mwait(bar_m2, ph2)) { ok = false; break; }              // Z, Y and the state products done
+        if (tid == 0 && more) issue_v(n + 1);                         // over Lam V(n)
+        {
+            // E2b: Z to pairs; Y to its tile; S0' to the next stage's tile, rho S0' back
+            float v[32], y[32];
+            ptx::tmem_ld32x2(tmem + lane_base + T3W_P + half * 32, tmem + lane_base + T3W_Y + half * 32, v, y);
+            st_pairs(T3W_H + half * 16, v);
+            st_row32(sm + W3_M1, row, half * 32, y);
+            if (quad < 2 && more) {
+                ptx::tmem_ld32(tmem + lane_base + T3W_S + half * 32, v);
+                st_row32(sm + (b ? W3_S00 : W3_S01), row, half * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= gam;
-            st_row32(sm + S3_P, row, half * 32, v);
+                for (int i = 0; i < 32; ++i) v[i] *= rho;
+                tmem_st32(tmem + lane_base + T3W_S + half * 32, v);
+            }
             ptx::tmem_st_wait();
         }
         sync_for_mma();
         if (tid == 0) {
-            const uint64_t dP = kdesc(sb + S3_P, 0), dQ = kdesc(sb + st + SQ_, 0);
-            const uint64_t dA = kdesc2(sb + S3_A, 0), dU = kdesc2(sb + S3_U, 0);
-            const uint64_t dKm = mdesc(sb + st + SK_, TILE, 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3_AS, k1s(dP, s), k1s(dQ, s), I_W, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_AS, tmem + T3_AT + 8 * s, k2s(dA, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_AS, tmem + T3_H + 8 * s, k2s(dU, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_HK, tmem + T3_H + 8 * s, mns(dKm, s), I_KM, s > 0);
+            const uint64_t dV = mdesc(sb + Vn, TILE, 0), dC = mdesc(sb + W3_C0, TILE, 0);
+            const uint64_t dG = mdesc(sb + W3_G0, TILE, 0), dQ = kdesc(sb + Qb, 0);
+            const uint64_t dY = mdesc(sb + W3_M1, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3W_P, tmem + T3W_AT + 8 * s, mns(dV, s), I_KM, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16_ts(tmem + T3W_X, tmem + T3W_H + 8 * s, mns(dC, s), I_KM, s > 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T3W_X, k1s(dQ, s), mns(dG, s), I_KM, 1);
+            ptx::umma_commit(bar_m1);
+            for (int s = 0; s < 8; ++s)
+                ptx::umma_bf16(tmem + T3W_GC, top_over_zero(sb + Kb, sb + W3_Z, s), mns(dY, s), I_MN, 1);
+            ptx::umma_commit(bar_m2);
         }
-        if (wn < items) convert_state(wn, b ^ 1);                  // overlaps R2
-        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R2 done
+        if (!mwait(bar_m1, ph1)) { ok = false; break; }              // O1, O2 done
+        // E3: O = O1 + Gam O2, staged as two [128][32] fp32 boxes over this chunk's Q and K
+        // tiles: Q is read for the last time by R3's first products, K by the G product, so the
+        // second box waits for it.  Then the next chunk's C0, -G0 tiles and rho C0, rho G0 back;
+        // Lam K, Lam V of the next chunk.
+        float o[32];
         {
-            // E2: W[tau][j] = g^(tau-j) x for j <= tau -> TMEM over At; Gam (Gam P + H K) -> over H
-            float v[32], w32[32];
+            float m[32];
+            ptx::tmem_ld32x2(tmem + lane_base + T3W_P + half * 32, tmem + lane_base + T3W_X + half * 32, o, m);
 #pragma unroll
-            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-                if (c0 > quad * 32 + 31) {
-                    st_pairs_zero(T3_AT + c0 / 2);
-                    continue;
-                }
-                ptx::tmem_ld32(tmem + lane_base + T3_AS + c0, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int d = row - (c0 + i);
-                    v[i] = d >= 0 ? gp[d] * v[i] : 0.f;
-                }
-                st_pairs(T3_AT + c0 / 2, v);
-            }
-            ptx::tmem_ld32x2(tmem + lane_base + T3_P + half * 32, tmem + lane_base + T3_HK + half * 32, v, w32);
-            const float gam = gp[row + 1];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = gam * fmaf(gam, v[i], w32[i]);
-            st_pairs(T3_H + half * 16, v);
-            ptx::tmem_st_wait();
+            for (int i = 0; i < 32; ++i) o[i] = fmaf(gam, m[i], o[i]);
         }
-        sync_for_mma();
-        if (tid == 0) {
-            const uint64_t dVm = mdesc(sb + st + SV_, TILE, 0), dC = mdesc(sb + st + SC0_, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T3_O, tmem + T3_AT + 8 * s, mns(dVm, s), I_KM, s > 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16_ts(tmem + T3_O, tmem + T3_H + 8 * s, mns(dC, s), I_KM, 1);
-        }
-        if (!ms.commit_wait(tid == 0)) { ok = false; break; }   // R3 done
-        {
-            // E3: O - Gam (Q G0), staged as two [128][32] fp32 boxes over A, then TMA stores
-            float o[32], m[32];
-            ptx::tmem_ld32x2(tmem + lane_base + T3_O + half * 32, tmem + lane_base + T3_QG + half * 32, o, m);
-            const float gam = gp[row + 1];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = fmaf(-gam, m[i], o[i]);
-            float4* box = reinterpret_cast<float4*>(sm + S3_A + half * (C * 128) + row * 128);
+        auto put_box = [&]() {
+            float4* box = reinterpret_cast<float4*>(sm + (half ? Kb : Qb) + row * 128);
 #pragma unroll
             for (int j = 0; j < 8; ++j) box[j ^ (row & 7)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-            ptx::fence_proxy_async();
+        };
+        if (half == 0) put_box();
+        ptx::tc_fence_before();
+        if (!mwait(bar_m2, ph2)) { ok = false; break; }              // G done; O1, O2 read
+        if (tid == 0 && more && ptx::mbar_wait(&bar_qk[b ^ 1], ((n + 1) >> 1) & 1))
+            issue_qks(n + 1);                                         // over O2, O1: runs during E3b
+        if (half == 1) put_box();
+        bool good = true;
+        if (more) {
+            float m[32];
+            ptx::tmem_ld32(tmem + lane_base + T3W_GC + half * 32, m);
+            if (quad < 2) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = -m[i];
+                st_row32(sm + W3_G0, row, half * 32, o);
+            } else {
+                st_row32(sm + W3_C0, row - 64, half * 32, m);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m[i] *= rho;
+            tmem_st32(tmem + lane_base + T3W_GC + half * 32, m);
+            ptx::tmem_st_wait();
+            const int nb = b ^ 1, par = ((n + 1) >> 1) & 1;
+            good = ptx::mbar_wait(&bar_qk[nb], par) && ptx::mbar_wait(&bar_v[nb], par);
+            if (good) {
+                ++wq[nb];
+                ++wv[nb];
+                scale_row_half(sm + (nb ? W3_K1 : W3_K0), sm + W3_LK, row, half, lam);
+                scale_row_half(sm + LVn, sm + Vn, row, half, lam);   // V(n+1) -> Lam V(n+1)
+            }
         }
-        __syncthreads();
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        ok = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
         if (tid == 0) {
-            ptx::tma_store_3d(&to, sm + S3_A, 0, chunk * C, bh);
-            ptx::tma_store_3d(&to, sm + S3_A + C * 128, 32, chunk * C, bh);
+            const int t0 = (chunk0 + n) * C;
+            ptx::tma_store_3d(&to, sm + Qb, 0, t0, bh);
+            ptx::tma_store_3d(&to, sm + Kb, 32, t0, bh);
             ptx::bulk_commit();
         }
     }
@@ -620,10 +897,12 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
         if (!ok) {
             set_status(p.status, DEV_TIMEOUT);
             // let loads and MMAs already in flight land before TMEM and shared memory are released
-            for (int b = 0; b < 2; ++b)
-                if (issued[b] > waited[b]) ptx::mbar_wait(&bar_load[b], (issued[b] - 1) & 1, 100000000ull);
-            ptx::umma_commit(ms.bar);
-            ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+            for (int b = 0; b < 2; ++b) {
+                if (iq[b] > wq[b]) ptx::mbar_wait(&bar_qk[b], (iq[b] - 1) & 1, 100000000ull);
+                if (iv[b] > wv[b]) ptx::mbar_wait(&bar_v[b], (iv[b] - 1) & 1, 100000000ull);
+            }
+            ptx::umma_commit(bar_m1);
+            ptx::mbar_wait(bar_m1, ph1, 100000000ull);
         }
     }
     ptx::tc_fence_before();
@@ -633,45 +912,90 @@ k_dec_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUt
 
 }  // namespace
 
-size_t decay_workspace_bytes(int BH, int T) {
-    const size_t NC = (size_t)(T + C - 1) / C;
-    return (size_t)BH * NC * DSUM * sizeof(float);
+namespace {
+// Segment plan of the decayed walk, from a makespan model in microseconds per CTA wave:
+// an output chunk ~7, a summary chunk ~3.5, set-up ~3 per walk, ~0.6 per folded slot.
+// Summaries cover the chunks before the last output segment.
+struct DPlan {
+    int NC, NCH, NS, NCHs, NSf, ratio;
+};
+DPlan dwalk_plan(int BH, int T, int seg_chunks) {
+    DPlan pl;
+    pl.NC = (T + C - 1) / C;
+    auto waves = [](long long ctas) { return (double)((ctas + kSMs - 1) / kSMs); };
+    double best = -1.0;
+    pl.NCH = 1;
+    pl.NCHs = 1;
+    for (int nch = 1; nch <= 128; nch *= 2) {
+        if (seg_chunks > 0 && nch != seg_chunks) continue;
+        const int NS = (pl.NC + nch - 1) / nch;
+        const int ncsum = (NS - 1) * nch;
+        for (int len = nch; len >= 1; len /= 2) {
+            const double out = waves((long long)BH * NS) * (nch * 7.0 + 3.0 + 0.6 * (NS - 1) * (nch / len));
+            const double sum = ncsum ? waves((long long)BH * (ncsum / len)) * (len * 3.5 + 3.0) : 0.0;
+            if (best < 0.0 || out + sum < best) {
+                best = out + sum;
+                pl.NCH = nch;
+                pl.NCHs = len;
+            }
+            if (ncsum == 0) break;
+        }
+        if (seg_chunks <= 0 && nch >= pl.NC) break;
+    }
+    pl.NS = (pl.NC + pl.NCH - 1) / pl.NCH;
+    pl.ratio = pl.NCH / pl.NCHs;
+    pl.NSf = (pl.NS - 1) * pl.ratio;
+    return pl;
+}
+}  // namespace
+
+size_t decay_workspace_bytes(int BH, int T, int seg_chunks) {
+    const DPlan pl = dwalk_plan(BH, T, seg_chunks);
+    return (size_t)BH * (pl.NSf > 0 ? pl.NSf : 1) * WSLOT * sizeof(float);
 }
 
-int decay_kernel_launches() { return 5; }
+int decay_kernel_launches(int BH, int T, int seg_chunks) {
+    return dwalk_plan(BH, T, seg_chunks).NSf > 0 ? 2 : 1;
+}
 
 cudaError_t decay_forward(const void* q, const void* k, const void* v, const float* gamma, float* o, int BH,
-                          int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev) {
+                               int H, int T, void* ws, int* status, cudaStream_t st, cudaEvent_t* ev,
+                               int seg_chunks) {
     if (!gamma || H < 1) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, q, T, BH) || !make_map(&mk, k, T, BH) || !make_map(&mv, v, T, BH) ||
         !make_map_out(&mo, o, T, BH))
         return cudaErrorInvalidValue;
-    DParams prm;
-    prm.T = T; prm.BH = BH; prm.H = H; prm.NC = (T + C - 1) / C;
+    const DPlan pl = dwalk_plan(BH, T, seg_chunks);
+    WParams prm;
+    prm.T = T; prm.BH = BH; prm.H = H;
+    prm.NCH = pl.NCH; prm.NS = pl.NS; prm.NCHs = pl.NCHs; prm.NSf = pl.NSf; prm.ratio = pl.ratio;
     prm.gamma = gamma;
     prm.sums = static_cast<float*>(ws);
     prm.status = status;
-    const int NC = prm.NC;
     cudaError_t e;
-    if ((e = set_smem(k_dec_summary, S1_BYTES)) != cudaSuccess)
-        return e;
-    if ((e = set_smem(k_dec_output, S3_BYTES)) != cudaSuccess)
-        return e;
+    if ((e = set_smem(k_dsum, W1_BYTES)) != cudaSuccess) return e;
+    if ((e = set_smem(k_dwalk, W3_BYTES)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_dec_summary<<<dim3(NC, BH), DNT, S1_BYTES, st>>>(mq, mk, mv, prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (pl.NSf > 0) {
+        k_dsum<<<dim3(pl.NSf, BH), DNT, W1_BYTES, st>>>(mq, mk, mv, prm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
-    k_dec_prefix_sc<<<dim3((2 * D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_dec_cross<<<dim3(NC, BH), PNT, 0, st>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_dec_prefix_g<<<dim3((D * D + PNT - 1) / PNT, BH), PNT, 0, st>>>(prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    const int items = NC * BH;
-    k_dec_output<<<items < kSMs ? items : kSMs, DNT, S3_BYTES, st>>>(mq, mk, mv, mo, prm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the output walk is a programmatic dependent of the summary walk: CTAs of segment 0 (and
+    // every CTA's set-up and first loads) overlap the summary walk; the folding CTAs wait for it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.NS, BH);
+    cfg.blockDim = dim3(DNT);
+    cfg.dynamicSmemBytes = W3_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.NSf > 0 ? 1 : 0;
+    if ((e = cudaLaunchKernelEx(&cfg, k_dwalk, mq, mk, mv, mo, prm)) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }

@@ -1074,13 +1074,13 @@ bool fits(int op, bool norm, int BH, int T, int seg_chunks) {
 
 size_t workspace_bytes(int op, bool norm, int BH, int T, int seg_chunks) {
     if (op == OP_AHLA || op == OP_AHLAD) return ahla_workspace_bytes(BH, T, seg_chunks, norm);
-    if (op == OP_HLA2D) return decay_workspace_bytes(BH, T);
+    if (op == OP_HLA2D) return decay_workspace_bytes(BH, T, seg_chunks);
     const Plan pl = plan(BH, T, kSMs, seg_chunks);
     return 2 * sizeof(float) * (size_t)BH * pl.NSp * simt_layout::size;
 }
 
 int kernel_launches(int op, bool norm, int BH, int T, int seg_chunks) {
-    if (op == OP_HLA2D) return decay_kernel_launches();
+    if (op == OP_HLA2D) return decay_kernel_launches(BH, T, seg_chunks);
     // summary walk, the prefix (up to PH_MAX slots per head: folded into the output walk; else
     // three launches), output walk
     const bool ahla = op == OP_AHLA || op == OP_AHLAD;
@@ -1096,7 +1096,7 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         if (!gamma) return cudaErrorInvalidValue;
         return ahla_forward(q, k, v, o, BH, H, T, norm, eps, gamma, ws, status, st, ev, seg_chunks);
     }
-    if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev);
+    if (op == OP_HLA2D) return decay_forward(q, k, v, gamma, o, BH, H, T, ws, status, st, ev, seg_chunks);
     if (op != OP_HLA2) return cudaErrorNotSupported;
     if (simt::summary_floats(OP_HLA2, D) != (size_t)simt_layout::size) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;

@@ -83,8 +83,8 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert use(hla.OP_HLA3, bf16, 0) == 0
     assert use(hla.OP_HLA2_NORM, bf16, 1) == 0
     # launches per forward: summary walker, the prefix (with up to nine summary slots per head
-    # folded into the output walker; else three kernels), output walker; the decayed path has
-    # chunk summaries, three prefix kernels and the output kernel
+    # folded into the output walker; else three kernels), output walker; the decayed second
+    # order folds its prefix in the output walker at every plan
     assert launches(hla.OP_HLA2_NORM, bf16, 0) == 2   # the output walker folds the prefix
     assert launches(hla.OP_AHLA, bf16, 0) == 2
     assert launches(hla.OP_AHLA_NORM, bf16, 0) == 2
@@ -99,7 +99,8 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert ws_tc(hla.OP_AHLA_NORM, 4, 16, 8192) > 0 and ws_tc(hla.OP_AHLA, 4, 16, 8192) > 0
     assert lib.hla_kernel_launches(hla.OP_AHLA_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 5   # many slots
     assert lib.hla_kernel_launches(hla.OP_HLA2_NORM, bf16, 0, 1, 1, 65536, 64, 64) == 5   # many slots
-    assert launches(hla.OP_HLA2, bf16, 1) == 5
+    assert launches(hla.OP_HLA2, bf16, 1) == 2
+    assert lib.hla_kernel_launches(hla.OP_HLA2, bf16, 1, 1, 2, 200, 64, 64) == 1   # one segment per head
     # CUDA-core path: chunk kernel, one scan launch (a per-head fold) and the output kernel;
     # the third order, decayed or not, takes the factored prefix (three launches)
     assert launches(hla.OP_HLA2, f32, 0) == 3
@@ -108,11 +109,13 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert launches(hla.OP_HLA3, f32, 0, d=32) == 2 + 3      # the factored third-order prefix
     assert launches(hla.OP_HLA3, f32, 0) == 2 + 3
     assert launches(hla.OP_HLA3, f32, 1, d=32) == 2 + 3      # decayed: the same three prefix launches
-    # decayed workspace: 256 B status block + one 4 x 64 x 64 fp32 slot per 128-token chunk
-    T = 16384
-    assert lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, T, 64, 64) == 256 + 32 * (T // 128) * 4 * 64 * 64 * 4
-    assert lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, T + 1, 64, 64) == \
-        256 + 32 * (T // 128 + 1) * 4 * 64 * 64 * 4
+    # decayed workspace: 256 B status block + segment summaries only, each slot S, C, G, Khat
+    # (4 x 64 x 64 fp32) and rho, a whole number of slots per head and fewer than one per four
+    # 128-token chunks at this shape
+    T, slot = 16384, (4 * 64 * 64 + 32) * 4
+    for t in (T, T + 1):
+        body = lib.hla_workspace_bytes(hla.OP_HLA2, bf16, 1, 2, 16, t, 64, 64) - 256
+        assert body > 0 and body % (32 * slot) == 0 and body // (32 * slot) <= T // 128 // 4
 
 
 def _call(lib, name, q=16, k=16, v=16, o=16, B=1, H=1, T=8, d=32, dv=32, dtype=0, gamma=0, ws=16,

@@ -112,7 +112,7 @@ def test_bf16_d64_parity_across_segments(op, T):
     assert err <= TOL["bf16"], err
 
 
-@pytest.mark.parametrize("op", ["hla2", "hla2n", "ahla", "ahlan", "ahlad", "ahlan_g"])
+@pytest.mark.parametrize("op", ["hla2", "hla2n", "hla2d", "ahla", "ahlan", "ahlad", "ahlan_g"])
 @pytest.mark.parametrize("nch", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("T", [129, 1000, 2049])
 def test_segment_length_invariance(op, nch, T):
@@ -240,6 +240,23 @@ def test_decay_gamma_one_matches_undecayed_tensor_cores(T):
     ref = oracle.recur("hla2", q, k, v)
     assert oracle.max_row_rel_err(a.cpu(), ref) <= TOL["bf16"]
     assert oracle.max_row_rel_err(a.cpu(), b.cpu()) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("gam", [0.3, 0.5, 0.95, 0.999, 1.0])
+@pytest.mark.parametrize("nch,T", [(1, 2049), (2, 4097), (4, 1500), (16, 5000)])
+def test_decayed_walk_segment_plans(gam, nch, T):
+    """The decayed second-order walk from strong to no decay over forced segment plans: up to
+    32 summary slots folded by one output CTA, ragged tails, one gamma per head pair."""
+    w = recipe("hla2d", "bf16", 1, 2, T, 64, seed=nch * 31 + int(gam * 100))
+    q, k, v, _ = hla_inputs.make_inputs(w)
+    g = torch.full((2,), gam)
+    hla.set_segment_chunks(nch)
+    try:
+        o = gpu_forward("hla2d", q, k, v, g)
+    finally:
+        hla.set_segment_chunks(0)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2d", q, k, v, gamma=g))
+    assert err <= TOL["bf16"], err
 
 
 @pytest.mark.parametrize("gam", [0.5, 0.95, 0.999])
