@@ -160,74 +160,85 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 }
 
 // ---------------------------------------------------------------- summary walk
-// Shared memory: K tiles, the zero block, Q tiles (this order), V tiles, then the scaled and
-// derived tiles.  TMEM columns: A* 0, Y 128, S 192 (lanes 0-63), G|C 256, Khat 320 (lanes 0-63).
-constexpr uint32_t W1_K0 = 0, W1_K1 = TILE, W1_Z = 2 * TILE;
-constexpr uint32_t W1_Q0 = 2 * TILE + 2048, W1_Q1 = W1_Q0 + TILE;
-constexpr uint32_t W1_V0 = W1_Q1 + TILE, W1_V1 = W1_V0 + TILE;
-constexpr uint32_t W1_WK = W1_V1 + TILE;    // rho^(N-1-l) Lam K
-constexpr uint32_t W1_LV = W1_WK + TILE;    // Lam V
-constexpr uint32_t W1_U = W1_LV + TILE;     // U [128 tau][128 i] K-major, two atoms
-constexpr uint32_t W1_Y = W1_U + 2 * TILE;  // rho^(N-1-l) Y, bf16 [tau][v]
-constexpr uint32_t W1_C0 = W1_Y + TILE;     // C0, bf16 [f][v]
-constexpr uint32_t W1_BAR = W1_C0 + QTILE;
-constexpr uint32_t W1_BYTES = W1_BAR + 64 + 1024;
-constexpr uint32_t T1_X = 0, T1_Y = 128, T1_S = 192, T1_GC = 256, T1_KH = 320;
+// Two CTAs per SM (108 KB of shared memory, 256 TMEM columns, at most 128 registers a thread),
+// so one CTA's epilogues overlap the other's MMAs.  Shared memory: the zero block Z1, the two
+// K tiles, the Q tile, the V tile (V, then Lam V in place), the weighted Lam K tile, the Y tile,
+// the rho C0 tile, the zero block Z2 (Z1 lies before every K and Q tile, Z2 after every K tile).
+// TMEM columns: X 0-127 (A*^T = K Q^T; then U^T as bf16 pairs in 0-31 and 96-127 and Y in
+// 32-95), S | Khat 128-191 (lanes 0-63 | 64-127), G | C 192-255 (lanes 0-63 | 64-127).
+constexpr uint32_t W1_Z1 = 0, W1_K0 = 2048, W1_K1 = W1_K0 + TILE, W1_Q = W1_K1 + TILE;
+constexpr uint32_t W1_V = W1_Q + TILE;      // V, then Lam V
+constexpr uint32_t W1_WK = W1_V + TILE;     // rho^(N-1-l) Lam K
+constexpr uint32_t W1_Y = W1_WK + TILE;     // rho^(N-1-l) Y, bf16 [tau][v]
+constexpr uint32_t W1_C0 = W1_Y + TILE;     // rho C0, bf16 [f][v]
+constexpr uint32_t W1_Z2 = W1_C0 + QTILE;
+constexpr uint32_t W1_BAR = W1_Z2 + 2048;
+constexpr uint32_t W1_BYTES = W1_BAR + 64;  // the dynamic base must be 1024-aligned (checked)
+constexpr uint32_t T1_X = 0, T1_Y = 32, T1_SK = 128, T1_GC = 192;
 
-// Rounds per chunk n: [G += [K^T;0] Y of chunk n-1; A* = Q K^T; Y = K C0]  -> E1: U, rho Y,
-//                     Lam-scaled K and V tiles
-//                     [C += [0;Q^T] Lam V; Y += U^T Lam V] (then S, Khat in the background)
-//                                                            -> E2: Y tile; C0' tile, rho C0'
-__global__ void __launch_bounds__(DNT, 1)
+// Rounds per chunk n: [G += [K^T;0] Y of chunk n-1; A*^T = K Q^T]       -> E1: U^T pairs, Lam V
+//                     in place, weighted Lam K
+//                     [C += [0;Q^T] Lam V; Y = K (rho C0) + U^T Lam V] (then S += [K^T;0] w Lam K,
+//                     Khat += [0;K^T] K in the background)            -> E2: Y tile; rho C0' tile
+//                                                                        and back to TMEM
+__global__ void __launch_bounds__(DNT, 2)
 k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
        const __grid_constant__ CUtensorMap tv, WParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = align1024(smem_raw);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = smem_raw;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
     const int seg = blockIdx.x, bh = blockIdx.y;
     // the output walk may be scheduled once every summary CTA has started
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (ptx::smem_u32(sm) & 1023) {            // the swizzled tiles need a 1024-byte base
+        if (tid == 0) set_status(p.status, DEV_ALIGN);
+        return;
+    }
     const int N = p.NCHs;                     // summary segments are whole chunks
     const int chunk0 = seg * N;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + W1_BAR);   // loads [2], MMA
-    MmaSync ms{bar + 2, 0};
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 3);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + W1_BAR);
+    uint64_t* bar_k = bar;                    // [2] K of a stage
+    uint64_t* bar_qv = bar + 2;               // Q and V
+    uint64_t* bar_m = bar + 3;                // MMA rounds
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
     const float g = p.gamma[bh % p.H];
     const float rho = gpow_n(g, C);
     const float lam = gpow_n(g, C - 1 - row);
     if (tid == 0) {
-        ptx::mbar_init(&bar[0], 1);
-        ptx::mbar_init(&bar[1], 1);
-        ptx::mbar_init(ms.bar, 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&bar[i], 1);
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    int issued[2] = {0, 0};
-    auto issue = [&](int n) {
+    int ik[2] = {0, 0}, wk[2] = {0, 0}, iqv = 0, wqv = 0;
+    auto issue_k = [&](int n) {
         const int b = n & 1;
-        const int t0 = (chunk0 + n) * C;
-        ptx::mbar_arrive_expect_tx(&bar[b], 3 * TILE);
-        ptx::tma_load_3d(sm + (b ? W1_Q1 : W1_Q0), &tq, &bar[b], 0, t0, bh);
-        ptx::tma_load_3d(sm + (b ? W1_K1 : W1_K0), &tk, &bar[b], 0, t0, bh);
-        ptx::tma_load_3d(sm + (b ? W1_V1 : W1_V0), &tv, &bar[b], 0, t0, bh);
-        ++issued[b];
+        ptx::mbar_arrive_expect_tx(&bar_k[b], TILE);
+        ptx::tma_load_3d(sm + (b ? W1_K1 : W1_K0), &tk, &bar_k[b], 0, (chunk0 + n) * C, bh);
+        ++ik[b];
+    };
+    auto issue_qv = [&](int n) {
+        ptx::mbar_arrive_expect_tx(bar_qv, 2 * TILE);
+        ptx::tma_load_3d(sm + W1_Q, &tq, bar_qv, 0, (chunk0 + n) * C, bh);
+        ptx::tma_load_3d(sm + W1_V, &tv, bar_qv, 0, (chunk0 + n) * C, bh);
+        ++iqv;
     };
     if (tid == 0) {
-        issue(0);
-        if (N > 1) issue(1);
+        issue_k(0);
+        issue_qv(0);
+        if (N > 1) issue_k(1);
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_alloc(tmem_slot, 256);
         ptx::tmem_relinquish();
     }
-    // the zero block and C0 = 0; U's blocks wholly below the diagonal are zero in every chunk
-    for (int i = tid; i < 2048 / 16; i += DNT) reinterpret_cast<uint4*>(sm + W1_Z)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // the zero blocks and rho C0 = 0
+    for (int i = tid; i < 2048 / 16; i += DNT) {
+        reinterpret_cast<uint4*>(sm + W1_Z1)[i] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(sm + W1_Z2)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int i = tid; i < QTILE / 16; i += DNT) reinterpret_cast<uint4*>(sm + W1_C0)[i] = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
-        if (c0 + 31 < quad * 32) st_row32_zero(sm + W1_U, row, c0);
     ptx::fence_proxy_async();
     ptx::tc_fence_before();
     __syncthreads();
@@ -236,14 +247,13 @@ k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t sb = ptx::smem_u32(sm);
     {
-        // S, G|C and Khat start at zero.  Their products always accumulate: one that cleared
-        // its accumulator would clear the lanes the other half of G|C holds.
+        // S | Khat and G | C start at zero.  Their products always accumulate: one that cleared
+        // its accumulator would clear the lanes that the other half holds.
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.f;
-        tmem_st32(tmem + lane_base + T1_S + half * 32, z);
+        tmem_st32(tmem + lane_base + T1_SK + half * 32, z);
         tmem_st32(tmem + lane_base + T1_GC + half * 32, z);
-        tmem_st32(tmem + lane_base + T1_KH + half * 32, z);
         ptx::tmem_st_wait();
     }
     ptx::tc_fence_before();
@@ -252,69 +262,83 @@ k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
     constexpr uint32_t I_QK = ptx::idesc_bf16(128, 128, false, false);
     constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
     constexpr uint32_t I_MN = ptx::idesc_bf16(128, 64, true, true);
+    uint32_t phase = 0;
+    auto mma_wait = [&]() {                   // thread 0 has committed; the block agrees
+        bool good = true;
+        if (tid == 0) good = ptx::mbar_wait(bar_m, phase);
+        phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
     bool ok = true;
-    int waited[2] = {0, 0};
     for (int n = 0; n < N; ++n) {
         const int b = n & 1;
-        const uint32_t Qb = b ? W1_Q1 : W1_Q0, Kb = b ? W1_K1 : W1_K0, Vb = b ? W1_V1 : W1_V0;
-        ok = ptx::mbar_wait(&bar[b], (n >> 1) & 1);           // every thread reads K, V below
+        const uint32_t Kb = b ? W1_K1 : W1_K0;
+        // every thread: this chunk's K, Q, V (K and V are read below)
+        ok = ptx::mbar_wait(&bar_k[b], (n >> 1) & 1) && ptx::mbar_wait(bar_qv, n & 1);
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
-        ++waited[b];
+        ++wk[b];
+        ++wqv;
         if (tid == 0) {
             ptx::tc_fence_after();
             if (n > 0) {                                        // G of chunk n-1
                 const uint32_t Kp = b ? W1_K0 : W1_K1;
                 const uint64_t dY = mdesc(sb + W1_Y, TILE, 0);
                 for (int s = 0; s < 8; ++s)
-                    ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z, s), mns(dY, s), I_MN, 1);
+                    ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z2, s), mns(dY, s), I_MN, 1);
             }
-            const uint64_t dQ = kdesc(sb + Qb, 0), dK = kdesc(sb + Kb, 0), dC0 = mdesc(sb + W1_C0, TILE, 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_X, k1s(dQ, s), k1s(dK, s), I_QK, s > 0);
-            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_Y, k1s(dK, s), mns(dC0, s), I_KM, s > 0);
+            const uint64_t dK = kdesc(sb + Kb, 0), dQ = kdesc(sb + W1_Q, 0);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_X, k1s(dK, s), k1s(dQ, s), I_QK, s > 0);
+            ptx::umma_commit(bar_m);
         }
-        if (!ms.commit_wait(tid == 0)) { ok = false; break; }
-        if (tid == 0 && n >= 1 && n + 1 < N) issue(n + 1);      // stage b^1: chunk n-1 is consumed
+        if (!mma_wait()) { ok = false; break; }
+        if (tid == 0 && n + 1 < N && n >= 1) issue_k(n + 1);   // stage b^1: chunk n-1's G is done
         {
-            // E1: U (strict upper part of A*, row `row`, columns half*64 .. +63); rho Y; the
-            // weighted Lam K and Lam V tiles of this chunk
-            float v[32];
+            // E1: row `row` = key token i of A*^T; U^T keeps the query columns tau < i.  Each half
+            // packs its 64 columns into the 32 columns it read first (0-31, 96-127), leaving
+            // 32-95 for Y.
+            float v0[32], v1[32];
+            ptx::tmem_ld32x2(tmem + lane_base + T1_X + half * 64, tmem + lane_base + T1_X + half * 64 + 32, v0, v1);
+            uint32_t pr[16];
 #pragma unroll
-            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-                if (c0 + 31 < quad * 32) continue;               // zero since set-up
-                ptx::tmem_ld32(tmem + lane_base + T1_X + c0, v);
-                if (c0 <= quad * 32 + 31 && c0 + 31 >= quad * 32) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c0 + i <= row) v[i] = 0.f;
-                }
-                st_row32(sm + W1_U, row, c0, v);
+            for (int i = 0; i < 16; ++i) {
+                const int t0 = half * 64 + 2 * i;
+                pr[i] = ptx::pack_bf16(t0 < row ? v0[2 * i] : 0.f, t0 + 1 < row ? v0[2 * i + 1] : 0.f);
             }
-            ptx::tmem_ld32(tmem + lane_base + T1_Y + half * 32, v);
+            const uint32_t pcol = T1_X + half * 96;
+            ptx::tmem_st16u(tmem + lane_base + pcol, pr);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= rho;
-            tmem_st32(tmem + lane_base + T1_Y + half * 32, v);
+            for (int i = 0; i < 16; ++i) {
+                const int t0 = half * 64 + 32 + 2 * i;
+                pr[i] = ptx::pack_bf16(t0 < row ? v1[2 * i] : 0.f, t0 + 1 < row ? v1[2 * i + 1] : 0.f);
+            }
+            ptx::tmem_st16u(tmem + lane_base + pcol + 16, pr);
             scale_row_half(sm + Kb, sm + W1_WK, row, half, lam * gpow_n(rho, N - 1 - n));
-            scale_row_half(sm + Vb, sm + W1_LV, row, half, lam);
+            scale_row_half(sm + W1_V, sm + W1_V, row, half, lam);
             ptx::tmem_st_wait();
         }
         sync_for_mma();
         if (tid == 0) {
-            const uint64_t dLV = mdesc(sb + W1_LV, TILE, 0), dU = mdesc(sb + W1_U, TILE, 0);
+            const uint64_t dLV = mdesc(sb + W1_V, TILE, 0), dC0 = mdesc(sb + W1_C0, TILE, 0);
+            const uint64_t dK = kdesc(sb + Kb, 0);
             for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + T1_GC, zero_over_bottom(sb + W1_Z, sb + Qb, s), mns(dLV, s), I_MN, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + T1_Y, mns(dU, s), mns(dLV, s), I_MN, 1);
-        }
-        if (!ms.commit_wait(tid == 0)) { ok = false; break; }
-        if (tid == 0) {                                         // S and Khat run during E2
+                ptx::umma_bf16(tmem + T1_GC, zero_over_bottom(sb + W1_Z1, sb + W1_Q, s), mns(dLV, s), I_MN, 1);
+            for (int s = 0; s < 4; ++s) ptx::umma_bf16(tmem + T1_Y, k1s(dK, s), mns(dC0, s), I_KM, s > 0);
+            for (int s = 0; s < 8; ++s)         // U^T pairs: K-steps 0-3 in columns 0-31, 4-7 in 96-127
+                ptx::umma_bf16_ts(tmem + T1_Y, tmem + T1_X + (s < 4 ? 8 * s : 96 + 8 * (s - 4)), mns(dLV, s), I_KM, 1);
+            ptx::umma_commit(bar_m);
             const uint64_t dWK = mdesc(sb + W1_WK, TILE, 0), dKm = mdesc(sb + Kb, TILE, 0);
+            for (int s = 0; s < 8; ++s)         // S (lanes 0-63) and Khat (lanes 64-127) in the background
+                ptx::umma_bf16(tmem + T1_SK, top_over_zero(sb + Kb, sb + W1_Z2, s), mns(dWK, s), I_MN, 1);
             for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + T1_S, top_over_zero(sb + Kb, sb + W1_Z, s), mns(dWK, s), I_MN, 1);
-            for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + T1_KH, top_over_zero(sb + Kb, sb + W1_Z, s), mns(dKm, s), I_MN, 1);
+                ptx::umma_bf16(tmem + T1_SK, zero_over_bottom(sb + W1_Z1, sb + Kb, s), mns(dKm, s), I_MN, 1);
         }
+        if (!mma_wait()) { ok = false; break; }
+        if (tid == 0 && n + 1 < N) issue_qv(n + 1);             // Q and Lam V are read
         {
-            // E2: the weighted Y to bf16; C0' (lanes 64-127) to its tile and back as rho C0'
+            // E2: the weighted Y to bf16; rho C0' (lanes 64-127) to its tile and back to TMEM
             float v[32];
             ptx::tmem_ld32(tmem + lane_base + T1_Y + half * 32, v);
             const float wy = gpow_n(rho, N - 1 - n);
@@ -323,9 +347,9 @@ k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             st_row32(sm + W1_Y, row, half * 32, v);
             if (quad >= 2 && n + 1 < N) {
                 ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
-                st_row32(sm + W1_C0, row - 64, half * 32, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] *= rho;
+                st_row32(sm + W1_C0, row - 64, half * 32, v);
                 tmem_st32(tmem + lane_base + T1_GC + half * 32, v);
                 ptx::tmem_st_wait();
             }
@@ -337,41 +361,37 @@ k_dsum(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
             const uint32_t Kp = ((N - 1) & 1) ? W1_K1 : W1_K0;
             const uint64_t dY = mdesc(sb + W1_Y, TILE, 0);
             for (int s = 0; s < 8; ++s)
-                ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z, s), mns(dY, s), I_MN, 1);
+                ptx::umma_bf16(tmem + T1_GC, top_over_zero(sb + Kp, sb + W1_Z2, s), mns(dY, s), I_MN, 1);
+            ptx::umma_commit(bar_m);
         }
-        ok = ms.commit_wait(tid == 0);
+        ok = mma_wait();
     }
     if (ok) {
-        // the slot: lanes 0-63 hold rows of S, G, Khat; lanes 64-127 rows of C
+        // the slot: lanes 0-63 hold rows of S and G, lanes 64-127 rows of Khat and C
         float* slot = p.sums + ((size_t)bh * p.NSf + seg) * WSLOT;
+        const int r = row & 63;
         float v[32];
-        auto put = [&](int m, int r) {
+        auto put = [&](int m) {
             float4* dst = reinterpret_cast<float4*>(slot + m * D * D + r * D + half * 32);
 #pragma unroll
             for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         };
-        if (quad < 2) {
-            ptx::tmem_ld32(tmem + lane_base + T1_S + half * 32, v);
-            put(0, row);
-            ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
-            put(2, row);
-            ptx::tmem_ld32(tmem + lane_base + T1_KH + half * 32, v);
-            put(3, row);
-        } else {
-            ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
-            put(1, row - 64);
-        }
+        ptx::tmem_ld32(tmem + lane_base + T1_SK + half * 32, v);
+        put(quad < 2 ? 0 : 3);
+        ptx::tmem_ld32(tmem + lane_base + T1_GC + half * 32, v);
+        put(quad < 2 ? 2 : 1);
         if (tid == 0) slot[4 * D * D] = gpow_n(g, C * N);
     } else if (tid == 0) {
         set_status(p.status, DEV_TIMEOUT);
         for (int b = 0; b < 2; ++b)
-            if (issued[b] > waited[b]) ptx::mbar_wait(&bar[b], (issued[b] - 1) & 1, 100000000ull);
-        ptx::umma_commit(ms.bar);
-        ptx::mbar_wait(ms.bar, ms.phase, 100000000ull);
+            if (ik[b] > wk[b]) ptx::mbar_wait(&bar_k[b], (ik[b] - 1) & 1, 100000000ull);
+        if (iqv > wqv) ptx::mbar_wait(bar_qv, (iqv - 1) & 1, 100000000ull);
+        ptx::umma_commit(bar_m);
+        ptx::mbar_wait(bar_m, phase, 100000000ull);
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+    if (warp == 1) ptx::tmem_dealloc(tmem, 256);
 }
 
 // ---------------------------------------------------------------- output walk
@@ -914,7 +934,8 @@ k_dwalk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensor
 
 namespace {
 // Segment plan of the decayed walk, from a makespan model in microseconds per CTA wave:
-// an output chunk ~7, a summary chunk ~3.5, set-up ~3 per walk, ~0.6 per folded slot.
+// an output chunk ~7 (one CTA per SM), a summary chunk ~4 (two CTAs per SM), set-up ~3 per
+// walk, ~0.6 per folded slot.
 // Summaries cover the chunks before the last output segment.
 struct DPlan {
     int NC, NCH, NS, NCHs, NSf, ratio;
@@ -923,6 +944,7 @@ DPlan dwalk_plan(int BH, int T, int seg_chunks) {
     DPlan pl;
     pl.NC = (T + C - 1) / C;
     auto waves = [](long long ctas) { return (double)((ctas + kSMs - 1) / kSMs); };
+    auto waves2 = [](long long ctas) { return (double)((ctas + 2 * kSMs - 1) / (2 * kSMs)); };   // two per SM
     double best = -1.0;
     pl.NCH = 1;
     pl.NCHs = 1;
@@ -932,7 +954,7 @@ DPlan dwalk_plan(int BH, int T, int seg_chunks) {
         const int ncsum = (NS - 1) * nch;
         for (int len = nch; len >= 1; len /= 2) {
             const double out = waves((long long)BH * NS) * (nch * 7.0 + 3.0 + 0.6 * (NS - 1) * (nch / len));
-            const double sum = ncsum ? waves((long long)BH * (ncsum / len)) * (len * 3.5 + 3.0) : 0.0;
+            const double sum = ncsum ? waves2((long long)BH * (ncsum / len)) * (len * 4.0 + 3.0) : 0.0;
             if (best < 0.0 || out + sum < best) {
                 best = out + sum;
                 pl.NCH = nch;
