@@ -172,7 +172,7 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
     chunk of c tokens, each 2 flop per multiply-add, divided by c (no discarded halves of
     stacked products, no state walk)."""
     D = w.d
-    c = 128 if path == "tc" else 64
+    c = 128 if path in ("tc", "tc-output") else 64
     if w.op in ("ahla", "ahlan", "ahlad"):
         # per token: A = Q K^T, Y = A V, O = A Y (2cD each), Q P0 and Q E0 (2D^2 each)
         flops = 6 * c * D + 4 * D * D
@@ -180,6 +180,10 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
         # per token: A* = Q K^T, P Q^T, A K, W V (2cD each); A A*^T (2c^2); Q S0, Q (S0 C0),
         # (A K) C0 (2D^2 each); S0 C0 once per chunk (2D^3 / c)
         flops = 8 * c * D + 2 * c * c + 6 * D * D + 2 * D ** 3 // c
+    elif path == "tc-output" and w.op == "hla3":
+        # the third-order output kernel on the tensor cores (c = 128): A* = Q K^T, P Q^T, A V,
+        # W Y (2cD each), A A^T (2c^2), Q S0, Q P0, Q F0 (2D^2 each), counted once (fp32)
+        flops = 8 * c * D + 2 * c * c + 6 * D * D
     elif w.op == "hla2d" and path == "tc":
         # the decayed output walker forms O and carries the state. Per token: A* = Q K^T,
         # Gam P Q^T, H K, W V (2cD each), At A^T and H U^T (2c^2 each), P = Q S0, Z C0, Q G0
@@ -190,7 +194,7 @@ def output_kernel_model(path: str, w: hla_inputs.Workload):
         flops = 2 * c * D + 2 * D * D + 2 * c * (D + c) + 2 * D * (D + c)
         if w.op in ("hla3", "hla3n", "hla3d"):
             flops += 2 * D * (D + c)      # the third order also forms Y = [Q|A][P0;V] before O = [Q|W][F0;Y]
-    return {"bound": "tensor" if path == "tc" else "alu", "flops_per_token": flops, "chunk": c}
+    return {"bound": "tensor" if path in ("tc", "tc-output") else "alu", "flops_per_token": flops, "chunk": c}
 
 
 def alu_peak_tflops(sm_mhz: float) -> float:
@@ -225,7 +229,7 @@ def run_ours(args):
     ws = hla.make_workspace(op, qd, vd, decayed=gd is not None)
     dcode = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
     launches_per_step = hla.kernel_launches(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv)
-    path = "tc" if hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv) else "simt"
+    path = {1: "tc", 2: "tc-output"}.get(hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv), "simt")
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     if args.segment_chunks:
         hla.set_segment_chunks(args.segment_chunks)
@@ -393,7 +397,11 @@ def parity_against_oracle(w, out, q, k, v, g):
 def roofline_of(path, w, out_ms, tokens, peaks, peak_kind):
     model = output_kernel_model(path, w)
     achieved = model["flops_per_token"] * tokens / (out_ms / 1e3) / 1e12
-    if model["bound"] == "tensor":
+    if model["bound"] == "tensor" and path == "tc-output":
+        # fp32 products from three bf16 products each (six for Q K^T): a third of the bf16 rate
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])) / 3
+        note = f"bf16 dense burst ({peak_kind}) / 3: each fp32 product is three bf16 products"
+    elif model["bound"] == "tensor":
         peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         note = f"bf16 dense burst ({peak_kind})"
     else:
@@ -429,7 +437,7 @@ def measure_workloads(dev, args, peaks, peak_kind, done):
         op = hla.OP_CODES[w.op]
         ws = hla.make_workspace(op, qd, vd, decayed=gd is not None)
         dcode = hla.HLA_BF16 if w.dtype == "bf16" else hla.HLA_F32
-        path = "tc" if hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv) else "simt"
+        path = {1: "tc", 2: "tc-output"}.get(hla.uses_tensor_cores(op, dcode, gd is not None, w.B, w.H, w.T, w.d, w.dv), "simt")
         for _ in range(max(3, args.warmup)):
             flush.zero_()
             hla.forward(w.op, qd, kd, vd, gamma=gd, eps=w.eps, out=out, workspace=ws)

@@ -154,8 +154,9 @@ def kernel_launches(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: 
     return int(load_library().hla_kernel_launches(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
 
 
-def uses_tensor_cores(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> bool:
-    return bool(load_library().hla_uses_tensor_cores(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
+def uses_tensor_cores(op: int, dtype_code: int, decayed: bool, B: int, H: int, T: int, d: int, dv: int) -> int:
+    """1: the whole forward on tcgen05; 2: its output kernel only; 0: CUDA cores (hla_uses_tensor_cores)."""
+    return int(load_library().hla_uses_tensor_cores(op, dtype_code, int(bool(decayed)), B, H, T, d, dv))
 
 
 def set_segment_chunks(chunks: int) -> None:

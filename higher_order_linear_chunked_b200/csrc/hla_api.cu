@@ -84,7 +84,7 @@ hla_status_t forward(hla_op_t op, const void* q, const void* k, const void* v, f
         e = hla::tc::forward(r.op, r.norm, q, k, v, gamma, eps, o, B * H, H, T, body, status, st, ev, r.seg);
     } else {
         e = hla::simt::forward(r.op, r.norm, r.bf16, r.d, q, k, v, gamma, eps, o, B * H, H, T,
-                               reinterpret_cast<float*>(body), st, ev);
+                               reinterpret_cast<float*>(body), status, st, ev);
     }
     return e == cudaSuccess ? HLA_OK : HLA_ERR_CUDA;
 }
@@ -135,7 +135,9 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
 
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
-    return use_tc(make_request(op, decayed != 0, dtype, B, H, T, d, dv)) ? 1 : 0;
+    const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
+    if (use_tc(r)) return 1;
+    return r.op == hla::OP_HLA3 && !r.norm && !r.bf16 && r.d == 32 ? 2 : 0;   // the tcgen05 output kernel
 }
 
 hla_status_t hla2_forward(const void* q, const void* k, const void* v, float* o, int B, int H, int T, int d,

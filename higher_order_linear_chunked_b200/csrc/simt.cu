@@ -30,6 +30,7 @@
 #include <algorithm>
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "common.cuh"
 #include "simt.h"
@@ -1097,9 +1098,15 @@ int scan_launches(int NCp) {
     return NCp == 1 ? 1 : 2 * levels;
 }
 
+// The plain third order with fp32 inputs and d = 32 takes the tcgen05 output kernel.
+template <int OP, bool NORM, int D, typename TIn>
+constexpr bool tc_third_order() {
+    return OP == OP_HLA3 && !NORM && D == 32 && std::is_same<TIn, float>::value;
+}
+
 template <int OP, bool NORM, int D, typename TIn>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* gamma, float eps, float* o,
-                       int BH, int H, int T, float* sums, cudaStream_t st, cudaEvent_t* ev) {
+                       int BH, int H, int T, float* sums, int* status, cudaStream_t st, cudaEvent_t* ev) {
     const int NC = (T + C - 1) / C;
     const int NCp = next_pow2(NC);
     auto ks = k_summary<OP, D, TIn>;
@@ -1124,50 +1131,57 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         return e;
     }
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    if ((e = launch_dep(ko, dim3(NC, BH), dim3(NT), s3, st, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H,
-                        T, NCp, (const float*)sums, o)) != cudaSuccess)
+    if (tc_third_order<OP, NORM, D, TIn>()) {
+        // the plain third order with fp32 inputs at d = 32: the output on the tensor cores
+        if ((e = tc::hla3_output((const float*)q, (const float*)k, (const float*)v, sums, NCp, Sum<OP, D>::SIZE, o, BH,
+                                 T, status, st)) != cudaSuccess)
+            return e;
+    } else if ((e = launch_dep(ko, dim3(NC, BH), dim3(NT), s3, st, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma,
+                               eps, H, T, NCp, (const float*)sums, o)) != cudaSuccess) {
         return e;
+    }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }
 
 template <typename TIn, int D>
 static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma,
-                               float eps, float* o, int BH, int H, int T, float* sums, cudaStream_t st,
+                               float eps, float* o, int BH, int H, int T, float* sums, int* status, cudaStream_t st,
                                cudaEvent_t* ev) {
     switch (op) {
     case OP_HLA2:
-        return norm ? run<OP_HLA2, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_HLA2, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_HLA2, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_HLA2, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     case OP_HLA2D:
-        return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     case OP_AHLA:
-        return norm ? run<OP_AHLA, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_AHLA, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     case OP_HLA3:
-        return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
-    case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+    case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     case OP_AHLAD:
-        return norm ? run<OP_AHLAD, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_AHLAD, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_AHLAD, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_AHLAD, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     case OP_HLA3D:
-        return norm ? run<OP_HLA3D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev)
-                    : run<OP_HLA3D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        return norm ? run<OP_HLA3D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
+                    : run<OP_HLA3D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     }
     return cudaErrorInvalidValue;
 }
 
 cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,
-                    const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, cudaStream_t st,
-                    cudaEvent_t* ev) {
+                    const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, int* status,
+                    cudaStream_t st, cudaEvent_t* ev) {
     if (bf16) {
-        if (d == 32) return dispatch_op<__nv_bfloat16, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
-        return dispatch_op<__nv_bfloat16, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+        if (d == 32)
+            return dispatch_op<__nv_bfloat16, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return dispatch_op<__nv_bfloat16, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
     }
-    if (d == 32) return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
-    return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, st, ev);
+    if (d == 32) return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+    return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
 }
 
 static bool uses_fold(int op, int d) {
@@ -2047,10 +2061,10 @@ cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, 
     if (bf16) k_fill_ones<__nv_bfloat16><<<blocks, NT, 0, st>>>(reinterpret_cast<__nv_bfloat16*>(ones), n);
     else k_fill_ones<float><<<blocks, NT, 0, st>>>(ones, n);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = forward(OP_HLA2, false, bf16, d, q, k, v, nullptr, 0.f, num, BH, 1, T, inner, st, nullptr)) !=
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, v, nullptr, 0.f, num, BH, 1, T, inner, status, st, nullptr)) !=
         cudaSuccess)
         return e;
-    if ((e = forward(OP_HLA2, false, bf16, d, q, k, ones, nullptr, 0.f, den, BH, 1, T, inner, st, nullptr)) !=
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, ones, nullptr, 0.f, den, BH, 1, T, inner, status, st, nullptr)) !=
         cudaSuccess)
         return e;
     const size_t rows = (size_t)BH * T;

@@ -24,7 +24,7 @@ int scan_launches(int NCp);
 // enqueue chunk kernel, Blelloch scan levels and output kernel on `st`; `ev` (NULL or
 // 4 events) is recorded before the chunk kernel, after it, after the scan, after the output kernel
 cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,
-                    const float* gamma, float eps, float* o, int BH, int H, int T, float* sums,
+                    const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, int* status,
                     cudaStream_t st, cudaEvent_t* ev);
 
 // Streaming state: one summary (summary_floats(op, d) floats) per head.

@@ -44,6 +44,12 @@ cudaError_t bwd_terms(const void* q, const void* v, const float* dout, float* te
 cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
                     const float* bw, float* dq, float* dk, float* dv, int BH, int T, int* status,
                     cudaStream_t st);
+// the third-order output (fp32 q, k, v, d = dv = 32, plain) on tcgen05 from three-term bf16
+// splits, 128-token chunks, after the CUDA-core summaries and factored prefix of 64-token chunks:
+// the prefix of 64-token chunk l of head bh is sums + (bh NCp + l) slot_floats (S0, P0, F0 at
+// matrices 0, 2, 3); launched as a programmatic dependent of the prefix kernels
+cudaError_t hla3_output(const float* q, const float* k, const float* v, const float* sums, int NCp, int slot_floats,
+                        float* o, int BH, int T, int* status, cudaStream_t st);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

@@ -1,0 +1,360 @@
+// tcgen05 output kernel of the third-order forward (fp32 inputs, d = dv = 32, not normalised,
+// no decay), fed by the CUDA-core chunk summaries and factored prefix.
+//
+// "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 3 (third
+// order) and Metodología 4 (chunked scan).  Per chunk of c = 128 tokens with the carried-in
+// key moment S0 and the carried-in P0, F0 of the third-order state (the exclusive prefix of the
+// 64-token chunk summaries at the chunk's first token):
+//     A = L (.) Q K^T,   P = Q S0,   W = L (.) (P Q^T + A A^T),
+//     Y = Q P0 + A V,    O = Q F0 + W Y.
+// fp32 accuracy from bf16 tensor-core products: a factor x is split into bf16 terms,
+// x = x1 + x2 (+ x3), each the bf16 rounding of what the earlier terms leave, and a product keeps
+// the terms of total order up to the split's: x1 y1 + x1 y2 + x2 y1 for two terms (about 2^-16
+// relative), x1 y1 + x1 y2 + x2 y1 + x1 y3 + x2 y2 + x3 y1 for three (about 2^-24).  The scores
+// Q K^T take three terms: with two, their error alone puts the output over a 1e-4 row error at
+// T = 4096 (an fp64 emulation of this kernel matched the GPU to three digits there).  Where the
+// contraction runs over the 32 features, the terms are one product over a concatenated K axis of
+// 192: A side [q1 | q1 | q2 | q1 | q2 | q3], B side [y1 | y2 | y1 | y3 | y2 | y1] (the state
+// products Q S0, Q P0, Q F0 ride along in the same B operand; P Q^T uses the first three
+// slots, [p1 | p2 | p1]).  Where it runs over the 128 tokens, the A side comes from TMEM as hi and
+// lo bf16 pairs and the B side is a [y_hi | y_lo] tile (64 columns) or separate hi and lo tiles.
+//
+// One CTA (8 warps, one TMEM lane quadrant per warp pair) per chunk x head:
+//   R1  [A* | P | Q P0 | Q F0] = [Q] [K ; S0^T ; P0^T ; F0^T]^T   (N = 224, K = 192 concatenated)
+//       -> E1: A = L (.) A* to hi / lo pairs (TMEM) and hi / lo tiles; P to its concatenated pairs
+//   R2  W = P Q^T + A A^T (hi.hi + hi.lo + lo.hi);  D_y = A [V_hi | V_lo]
+//       -> E2: W = L (.) W to hi / lo pairs; Y = Q P0 + D_y(hi) + D_y(lo) to a [Y_hi | Y_lo] tile
+//   R3  D_o = W [Y_hi | Y_lo]
+//       -> E3: O = Q F0 + D_o(hi) + D_o(lo), fp32 stores
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "tc.h"
+#include "tc_common.cuh"
+
+namespace hla {
+namespace tc {
+namespace {
+
+constexpr int D3 = 32;                      // head dim of this kernel
+constexpr int NT3 = 256;                    // 8 warps
+constexpr uint32_t BROWS = C + 3 * D3;      // rows of the R1 B operand: K, S0^T, P0^T, F0^T
+constexpr uint32_t BATOM = BROWS * 128;     // one 64-wide K atom of it (28 KB)
+
+// Shared memory (1024-byte aligned offsets)
+constexpr uint32_t X_QC = 0;                       // [q1 | q1 | q2 | q1 | q2 | q3], three atoms (48 KB)
+constexpr uint32_t X_BC = X_QC + 3 * TILE;         // [y1 | y2 | y1 | y3 | y2 | y1] rows K, S0^T, P0^T, F0^T
+constexpr uint32_t X_AH = X_BC + 3 * BATOM;        // A_hi [128][128], two atoms
+constexpr uint32_t X_AL = X_AH + 2 * TILE;         // A_lo
+constexpr uint32_t X_VC = X_AL + 2 * TILE;         // [V_hi | V_lo] [128 tokens][64], then [Y_hi | Y_lo]
+constexpr uint32_t X_YC = X_VC;
+constexpr uint32_t X_BAR = X_VC + TILE;
+constexpr uint32_t X_BYTES = X_BAR + 64 + 1024;    // + alignment slack
+
+// TMEM columns
+constexpr uint32_t T_X = 0;      // A*, then W (fp32, 128)
+constexpr uint32_t T_P = 128;    // P (32)
+constexpr uint32_t T_QP = 160;   // Q P0 (32)
+constexpr uint32_t T_QF = 192;   // Q F0 (32)
+constexpr uint32_t T_AH = 224;   // A_hi pairs, then W_hi pairs (64)
+constexpr uint32_t T_AL = 288;   // A_lo pairs, then W_lo pairs (64)
+constexpr uint32_t T_D = 352;    // D_y, then D_o (64)
+constexpr uint32_t T_PC = 416;   // [p1 | p2 | p1] pairs (48)
+
+__device__ __forceinline__ float hi_of(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+// three bf16 terms of x (each exact in bf16; x - x1 - x2 - x3 is about 2^-24 x)
+__device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
+    a = hi_of(x);
+    const float r = x - a;
+    b = hi_of(r);
+    c = hi_of(r - b);
+}
+
+// 16 values into columns c0 .. c0+15 of row `row` of a K-major tile whose 64-wide atoms lie
+// `atom` bytes apart (128B swizzle)
+__device__ __forceinline__ void put16(uint8_t* tile, uint32_t atom, int row, int c0, const float (&v)[16]) {
+    st_row16(tile, atom, row, c0, v);
+}
+
+struct H3Params {
+    int T, NCp, slot;     // slot: floats of one summary slot; the prefix of 64-token chunk l of head
+                          // bh sits at sums + (bh NCp + l) slot, S0 at matrix 0, P0 at 2, F0 at 3
+    const float* sums;
+    float* o;
+    int* status;
+};
+
+__global__ void __launch_bounds__(NT3, 1)
+k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, H3Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int t0 = chunk * C;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + X_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    // a row of the R1 B operand from the three terms of 16 of its features
+    auto put_b = [&](int r, int h, const float (&y1)[16], const float (&y2)[16], const float (&y3)[16]) {
+        put16(sm + X_BC, BATOM, r, 16 * h, y1);
+        put16(sm + X_BC, BATOM, r, 32 + 16 * h, y2);
+        put16(sm + X_BC, BATOM, r, 64 + 16 * h, y1);
+        put16(sm + X_BC, BATOM, r, 96 + 16 * h, y3);
+        put16(sm + X_BC, BATOM, r, 128 + 16 * h, y2);
+        put16(sm + X_BC, BATOM, r, 160 + 16 * h, y1);
+    };
+    // ---- Q, K, V rows to their split tiles: thread (r, h) takes columns 16h .. 16h+15 of row r
+    {
+        const int r = tid >> 1, h = tid & 1;
+        const bool in = t0 + r < p.T;
+        const size_t base = ((size_t)bh * p.T + t0 + r) * D3 + 16 * h;
+        float xq[16], xk[16], xv[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 a = in ? *reinterpret_cast<const float4*>(q + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 b = in ? *reinterpret_cast<const float4*>(k + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 c = in ? *reinterpret_cast<const float4*>(v + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            xq[4 * j] = a.x; xq[4 * j + 1] = a.y; xq[4 * j + 2] = a.z; xq[4 * j + 3] = a.w;
+            xk[4 * j] = b.x; xk[4 * j + 1] = b.y; xk[4 * j + 2] = b.z; xk[4 * j + 3] = b.w;
+            xv[4 * j] = c.x; xv[4 * j + 1] = c.y; xv[4 * j + 2] = c.z; xv[4 * j + 3] = c.w;
+        }
+        float x1[16], x2[16], x3[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) split3(xq[j], x1[j], x2[j], x3[j]);
+        put16(sm + X_QC, TILE, r, 16 * h, x1);
+        put16(sm + X_QC, TILE, r, 32 + 16 * h, x1);
+        put16(sm + X_QC, TILE, r, 64 + 16 * h, x2);
+        put16(sm + X_QC, TILE, r, 96 + 16 * h, x1);
+        put16(sm + X_QC, TILE, r, 128 + 16 * h, x2);
+        put16(sm + X_QC, TILE, r, 160 + 16 * h, x3);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) split3(xk[j], x1[j], x2[j], x3[j]);
+        put_b(r, h, x1, x2, x3);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            x1[j] = hi_of(xv[j]);
+            x2[j] = xv[j] - x1[j];
+        }
+        put16(sm + X_VC, TILE, r, 16 * h, x1);
+        put16(sm + X_VC, TILE, r, 32 + 16 * h, x2);
+    }
+    // A_hi / A_lo blocks above the diagonal are zero in every chunk
+#pragma unroll
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+        if (c0 > quad * 32 + 31) {
+            st_row32_zero(sm + X_AH, row, c0);
+            st_row32_zero(sm + X_AL, row, c0);
+        }
+    // the carried-in S0, P0, F0 come from the prefix kernels
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid < 3 * 2 * D3) {
+        // B rows 128 + 32 m + g: column g of matrix m (S0, P0, F0), split as the key rows
+        const int m = tid / (2 * D3), g = (tid >> 1) % D3, h = tid & 1;
+        const float* pre = p.sums + ((size_t)bh * p.NCp + 2 * chunk) * p.slot + (m == 0 ? 0 : m + 1) * D3 * D3;
+        float y1[16], y2[16], y3[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) split3(pre[(16 * h + j) * D3 + g], y1[j], y2[j], y3[j]);
+        put_b(C + m * D3 + g, h, y1, y2, y3);
+    }
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    auto st_pairs = [&](uint32_t tcol, const float* x) {          // 32 values -> 16 columns
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = ptx::pack_bf16(x[2 * i], x[2 * i + 1]);
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    auto st_zero16 = [&](uint32_t tcol) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    {
+        // pairs that stay zero: A / W above the diagonal
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+            if (c0 > quad * 32 + 31) {
+                st_zero16(T_AH + c0 / 2);
+                st_zero16(T_AL + c0 / 2);
+            }
+        ptx::tmem_st_wait();
+    }
+    constexpr uint32_t I_R1 = ptx::idesc_bf16(128, 224, false, false);
+    constexpr uint32_t I_W = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
+    uint32_t phase = 0;
+    auto mma_wait = [&]() {
+        bool good = true;
+        if (tid == 0) {
+            ptx::umma_commit(bar);
+            good = ptx::mbar_wait(bar, phase);
+        }
+        phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
+    auto sync_mma = [&]() {
+        ptx::tmem_st_wait();
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+    };
+    sync_mma();
+    bool ok = true;
+    if (tid == 0) {
+        for (int s = 0; s < 12; ++s)
+            ptx::umma_bf16(tmem + T_X, kdesc2(sb + X_QC, s),
+                           ptx::desc_sw128(sb + X_BC + (s >> 2) * BATOM + (s & 3) * 32, 16, 1024), I_R1, s > 0);
+    }
+    ok = mma_wait();                                                  // R1 done
+    if (ok) {
+        // E1: row `row` of A*, columns half*64 .. +63 in two blocks of 32: A = L (.) A*, split
+        float v[32], hi[32], lo[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 > quad * 32 + 31) continue;                          // zero since set-up
+            ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = (c0 + i <= row) ? v[i] : 0.f;
+                hi[i] = hi_of(x);
+                lo[i] = x - hi[i];
+            }
+            st_pairs(T_AH + c0 / 2, hi);
+            st_pairs(T_AL + c0 / 2, lo);
+            st_row32(sm + X_AH, row, c0, hi);
+            st_row32(sm + X_AL, row, c0, lo);
+        }
+        // P (32 columns) to [p1 | p2 | p1]: half 0 writes the two p1 slots, half 1 the p2 slot
+        ptx::tmem_ld32(tmem + lane_base + T_P, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            hi[i] = hi_of(v[i]);
+            lo[i] = v[i] - hi[i];
+        }
+        if (half == 0) {
+            st_pairs(T_PC, hi);
+            st_pairs(T_PC + 32, hi);
+        } else {
+            st_pairs(T_PC + 16, lo);
+        }
+        sync_mma();
+        if (tid == 0) {
+            const uint64_t dV = mdesc(sb + X_VC, TILE, 0);
+            for (int s = 0; s < 6; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_PC + 8 * s, kdesc2(sb + X_QC, s), I_W, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AL, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AL + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
+        }
+        ok = mma_wait();                                              // R2 done
+    }
+    if (ok) {
+        // E2: W = L (.) W to hi / lo pairs (over A's); Y = Q P0 + D_y(hi) + D_y(lo) to [Y_hi | Y_lo]
+        float v[32], hi[32], lo[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 > quad * 32 + 31) continue;
+            ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = (c0 + i <= row) ? v[i] : 0.f;
+                hi[i] = hi_of(x);
+                lo[i] = x - hi[i];
+            }
+            st_pairs(T_AH + c0 / 2, hi);
+            st_pairs(T_AL + c0 / 2, lo);
+        }
+        float a[16], b[16], c[16], yh[16], yl[16];
+        ptx::tmem_ld16(tmem + lane_base + T_QP + 16 * half, a);
+        ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
+        ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float y = a[i] + b[i] + c[i];
+            yh[i] = hi_of(y);
+            yl[i] = y - yh[i];
+        }
+        put16(sm + X_YC, TILE, row, 16 * half, yh);
+        put16(sm + X_YC, TILE, row, 32 + 16 * half, yl);
+        sync_mma();
+        if (tid == 0) {
+            const uint64_t dY = mdesc(sb + X_YC, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dY + (uint64_t)(s * 128), I_KM, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dY + (uint64_t)(s * 128), I_KM, 1);
+        }
+        ok = mma_wait();                                              // R3 done
+    }
+    if (ok) {
+        // E3: O = Q F0 + D_o(hi) + D_o(lo); this thread's 16 columns of its row
+        float a[16], b[16], c[16];
+        ptx::tmem_ld16(tmem + lane_base + T_QF + 16 * half, a);
+        ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
+        ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
+        if (t0 + row < p.T) {
+            float4* dst = reinterpret_cast<float4*>(p.o + ((size_t)bh * p.T + t0 + row) * D3 + 16 * half);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                dst[j] = make_float4(a[4 * j] + b[4 * j] + c[4 * j], a[4 * j + 1] + b[4 * j + 1] + c[4 * j + 1],
+                                     a[4 * j + 2] + b[4 * j + 2] + c[4 * j + 2], a[4 * j + 3] + b[4 * j + 3] + c[4 * j + 3]);
+        }
+    } else if (tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        ptx::umma_commit(bar);
+        ptx::mbar_wait(bar, phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t hla3_output(const float* q, const float* k, const float* v, const float* sums, int NCp, int slot_floats,
+                        float* o, int BH, int T, int* status, cudaStream_t st) {
+    H3Params prm;
+    prm.T = T;
+    prm.NCp = NCp;
+    prm.slot = slot_floats;
+    prm.sums = sums;
+    prm.o = o;
+    prm.status = status;
+    cudaError_t e;
+    if ((e = set_smem(k_hla3_out, X_BYTES)) != cudaSuccess) return e;
+    // a programmatic dependent of the prefix kernels: its Q, K, V loads overlap their end
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((T + C - 1) / C, BH);
+    cfg.blockDim = dim3(NT3);
+    cfg.dynamicSmemBytes = X_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_hla3_out, q, k, v, prm);
+}
+
+}  // namespace tc
+}  // namespace hla

@@ -180,9 +180,12 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
 int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
 
 /*
- * 1 when this request runs on the tcgen05 tensor-core kernels, 0 when it runs
- * on the CUDA-core (fp32 FFMA) kernels or is invalid.  Same arguments as
- * hla_workspace_bytes().
+ * 1 when this request runs on the tcgen05 tensor-core kernels, 2 when its
+ * output kernel runs on them and its chunk summaries and prefix on the CUDA
+ * cores (the plain third order with fp32 inputs at d = 32, whose output kernel
+ * takes fp32 accuracy from products of two- and three-term bf16 splits), 0 when
+ * it runs on the CUDA-core (fp32 FFMA) kernels or is invalid.  Same arguments
+ * as hla_workspace_bytes().
  */
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
 

@@ -81,6 +81,11 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert use(hla.OP_HLA2, f32, 0) == 0
     assert use(hla.OP_HLA2, bf16, 0, d=32) == 0
     assert use(hla.OP_HLA3, bf16, 0) == 0
+    # the plain third order with fp32 inputs at d = 32: the output kernel on the tensor cores (2),
+    # not the normalised or decayed forms, nor d = 64 or bf16 inputs
+    assert use(hla.OP_HLA3, f32, 0, d=32) == 2
+    assert use(hla.OP_HLA3, f32, 1, d=32) == 0 and use(hla.OP_HLA3_NORM, f32, 0, d=32) == 0
+    assert use(hla.OP_HLA3, f32, 0) == 0 and use(hla.OP_HLA3, bf16, 0, d=32) == 0
     assert use(hla.OP_HLA2_NORM, bf16, 1) == 0
     # launches per forward: summary walker, the prefix (with up to nine summary slots per head
     # folded into the output walker; else three kernels), output walker; the decayed second

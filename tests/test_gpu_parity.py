@@ -259,6 +259,29 @@ def test_decayed_walk_segment_plans(gam, nch, T):
     assert err <= TOL["bf16"], err
 
 
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 128, 129, 255, 257, 1000, 4097])
+def test_third_order_tensor_core_output(T):
+    """The plain third order with fp32 inputs at d = 32: CUDA-core summaries and prefix over
+    64-token chunks, the output on the tensor cores over 128-token chunks reading every other
+    prefix slot; ragged tails on both chunkings, fp32 tolerance."""
+    assert hla.uses_tensor_cores(hla.OP_HLA3, hla.HLA_F32, False, 1, 3, T, 32, 32) == 2
+    w = recipe("hla3", "f32", 1, 3, T, 32, seed=T + 17)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward("hla3", q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla3", q, k, v))
+    assert err <= TOL["f32"], err
+
+
+def test_third_order_tensor_core_output_large_values():
+    """Inputs 8x larger than the workload's (a wider dynamic range for the bf16 splits)."""
+    w = recipe("hla3", "f32", 1, 2, 2000, 32, seed=3)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    q, k, v = q * 8, k * 8, v * 8
+    o = gpu_forward("hla3", q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla3", q, k, v))
+    assert err <= TOL["f32"], err
+
+
 @pytest.mark.parametrize("gam", [0.5, 0.95, 0.999])
 def test_decay_strong_and_weak_tensor_cores(gam):
     """bf16 d = 64 decayed path for one gamma per run, strong to weak decay, ragged tail."""
