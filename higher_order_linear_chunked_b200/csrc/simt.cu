@@ -1098,7 +1098,7 @@ int scan_launches(int NCp) {
     return NCp == 1 ? 1 : 2 * levels;
 }
 
-// The plain third order with fp32 inputs and d = 32 takes the tcgen05 output kernel.
+// The plain third order with fp32 inputs and d = 32 takes the tcgen05 summary and output kernels.
 template <int OP, bool NORM, int D, typename TIn>
 constexpr bool tc_third_order() {
     return OP == OP_HLA3 && !NORM && D == 32 && std::is_same<TIn, float>::value;
@@ -1107,6 +1107,24 @@ constexpr bool tc_third_order() {
 template <int OP, bool NORM, int D, typename TIn>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* gamma, float eps, float* o,
                        int BH, int H, int T, float* sums, int* status, cudaStream_t st, cudaEvent_t* ev) {
+    if (tc_third_order<OP, NORM, D, TIn>()) {
+        // the plain third order with fp32 inputs at d = 32: summaries and output on the tensor
+        // cores over 128-token chunks, the factored prefix between them on the CUDA cores
+        const int NC2 = (T + 127) / 128;
+        cudaError_t e;
+        if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
+        if ((e = tc::hla3_summaries((const float*)q, (const float*)k, (const float*)v, sums, NC2, Sum<OP, D>::SIZE, BH,
+                                    T, status, st)) != cudaSuccess)
+            return e;
+        if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
+        if ((e = hla3_factored_prefix<OP, D>(sums, NC2, NC2, BH, st)) != cudaSuccess) return e;
+        if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
+        if ((e = tc::hla3_output((const float*)q, (const float*)k, (const float*)v, sums, NC2, Sum<OP, D>::SIZE, o, BH,
+                                 T, status, st)) != cudaSuccess)
+            return e;
+        if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
+        return cudaSuccess;
+    }
     const int NC = (T + C - 1) / C;
     const int NCp = next_pow2(NC);
     auto ks = k_summary<OP, D, TIn>;
@@ -1131,15 +1149,9 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
         return e;
     }
     if (ev && (e = cudaEventRecord(ev[2], st)) != cudaSuccess) return e;
-    if (tc_third_order<OP, NORM, D, TIn>()) {
-        // the plain third order with fp32 inputs at d = 32: the output on the tensor cores
-        if ((e = tc::hla3_output((const float*)q, (const float*)k, (const float*)v, sums, NCp, Sum<OP, D>::SIZE, o, BH,
-                                 T, status, st)) != cudaSuccess)
-            return e;
-    } else if ((e = launch_dep(ko, dim3(NC, BH), dim3(NT), s3, st, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma,
-                               eps, H, T, NCp, (const float*)sums, o)) != cudaSuccess) {
+    if ((e = launch_dep(ko, dim3(NC, BH), dim3(NT), s3, st, (const TIn*)q, (const TIn*)k, (const TIn*)v, gamma, eps, H,
+                        T, NCp, (const float*)sums, o)) != cudaSuccess)
         return e;
-    }
     if (ev && (e = cudaEventRecord(ev[3], st)) != cudaSuccess) return e;
     return cudaSuccess;
 }

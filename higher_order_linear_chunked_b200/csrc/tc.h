@@ -44,10 +44,13 @@ cudaError_t bwd_terms(const void* q, const void* v, const float* dout, float* te
 cudaError_t bwd_out(const void* q, const void* k, const void* v, const float* dout, const float* pre,
                     const float* bw, float* dq, float* dk, float* dv, int BH, int T, int* status,
                     cudaStream_t st);
-// the third-order output (fp32 q, k, v, d = dv = 32, plain) on tcgen05 from three-term bf16
-// splits, 128-token chunks, after the CUDA-core summaries and factored prefix of 64-token chunks:
-// the prefix of 64-token chunk l of head bh is sums + (bh NCp + l) slot_floats (S0, P0, F0 at
-// matrices 0, 2, 3); launched as a programmatic dependent of the prefix kernels
+// the third order (fp32 q, k, v, d = dv = 32, plain) on tcgen05 from two- and three-term bf16
+// splits, 128-token chunks: hla3_summaries writes chunk l's summary of head bh to
+// sums + (bh NC + l) slot_floats in the CUDA-core slot layout (the factored prefix then runs in
+// place over NC slots per head, NCp = NC); hla3_output reads the exclusive prefix of chunk l at
+// sums + (bh NCp + l) slot_floats (S0, P0, F0 at matrices 0, 2, 3) as a programmatic dependent
+cudaError_t hla3_summaries(const float* q, const float* k, const float* v, float* sums, int NC, int slot_floats,
+                           int BH, int T, int* status, cudaStream_t st);
 cudaError_t hla3_output(const float* q, const float* k, const float* v, const float* sums, int NCp, int slot_floats,
                         float* o, int BH, int T, int* status, cudaStream_t st);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)

@@ -1,10 +1,11 @@
-// tcgen05 output kernel of the third-order forward (fp32 inputs, d = dv = 32, not normalised,
-// no decay), fed by the CUDA-core chunk summaries and factored prefix.
+// tcgen05 kernels of the third-order forward (fp32 inputs, d = dv = 32, not normalised, no
+// decay): the 128-token chunk summaries and the output; the factored prefix between them runs on
+// the CUDA cores.
 //
 // "Higher-order Linear Attention" summary (gist.science 2510.27258), Metodología 3 (third
 // order) and Metodología 4 (chunked scan).  Per chunk of c = 128 tokens with the carried-in
 // key moment S0 and the carried-in P0, F0 of the third-order state (the exclusive prefix of the
-// 64-token chunk summaries at the chunk's first token):
+// chunk summaries):
 //     A = L (.) Q K^T,   P = Q S0,   W = L (.) (P Q^T + A A^T),
 //     Y = Q P0 + A V,    O = Q F0 + W Y.
 // fp32 accuracy from bf16 tensor-core products: a factor x is split into bf16 terms,
@@ -80,8 +81,8 @@ __device__ __forceinline__ void put16(uint8_t* tile, uint32_t atom, int row, int
 }
 
 struct H3Params {
-    int T, NCp, slot;     // slot: floats of one summary slot; the prefix of 64-token chunk l of head
-                          // bh sits at sums + (bh NCp + l) slot, S0 at matrix 0, P0 at 2, F0 at 3
+    int T, NCp, slot;     // slot: floats of one summary slot; the prefix of chunk l of head bh sits
+                          // at sums + (bh NCp + l) slot, S0 at matrix 0, P0 at 2, F0 at 3
     const float* sums;
     float* o;
     int* status;
@@ -162,7 +163,7 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
     if (tid < 3 * 2 * D3) {
         // B rows 128 + 32 m + g: column g of matrix m (S0, P0, F0), split as the key rows
         const int m = tid / (2 * D3), g = (tid >> 1) % D3, h = tid & 1;
-        const float* pre = p.sums + ((size_t)bh * p.NCp + 2 * chunk) * p.slot + (m == 0 ? 0 : m + 1) * D3 * D3;
+        const float* pre = p.sums + ((size_t)bh * p.NCp + chunk) * p.slot + (m == 0 ? 0 : m + 1) * D3 * D3;
         float y1[16], y2[16], y3[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) split3(pre[(16 * h + j) * D3 + g], y1[j], y2[j], y3[j]);
@@ -329,6 +330,297 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
     if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
+
+// ---------------------------------------------------------------- chunk summaries
+// The third-order summary of a 128-token chunk from the zero state (the slot layout of the
+// CUDA-core summaries: S = K^T K, Q2 = Q^T Q, P = K^T V, F = K^T (A^T (A V)), X = Q^T (A V),
+// Z = K^T (A^T Q) at matrices 0..5; the plain op needs no normaliser vectors, which stay zero).
+// Two-term bf16 splits throughout (an fp64 emulation of these summaries with the output kernel
+// above gave a 1.4e-5 row error on the fp32 workload).  The feature-side products are one MMA
+// over the stacked hi / lo tiles: A = [K_hi | K_lo ; Q_hi | Q_lo] (MN-major, M = 128) times
+// B = [K_hi | K_lo | V_hi | V_lo | Q_hi | Q_lo] gives every hi / lo block of K^T K, K^T V, Q^T Q;
+// a 32 x 32 result is the sum of its four blocks.
+//   R1  A* = Q K^T (concatenated K axis);  D1 = [KK ; QQ] [KK | VV | QQ]   -> E1: A hi / lo pairs
+//       and tiles; S, P, Q2 from D1
+//   R2  Yl = A [V_hi | V_lo];  AQ = A^T [Q_hi | Q_lo]                      -> E2: [Yl_hi | Yl_lo],
+//       [AQ_hi | AQ_lo] tiles
+//   R3  AY = A^T [Yl_hi | Yl_lo];  D3 = [KK ; QQ] [YY | AQ]                 -> E3: [AY_hi | AY_lo];
+//       X, Z from D3
+//   R4  D4 = [KK ; QQ] [AY]                                                 -> E4: F from D4
+constexpr uint32_t Y_QC = 0;                    // [q_hi | q_lo | q_hi | 0] (two atoms); AY later
+constexpr uint32_t Y_KC = Y_QC + 2 * TILE;      // [k_hi | k_hi | k_lo | 0]; fp32 staging later
+constexpr uint32_t Y_KK = Y_KC + 2 * TILE;      // [K_hi | K_lo] token rows }
+constexpr uint32_t Y_VV = Y_KK + TILE;          // [V_hi | V_lo]            } equally spaced: one
+constexpr uint32_t Y_QQ = Y_VV + TILE;          // [Q_hi | Q_lo]            } N = 192 operand
+constexpr uint32_t Y_AH = Y_QQ + TILE;          // A_hi [128][128], two atoms
+constexpr uint32_t Y_AL = Y_AH + 2 * TILE;      // A_lo
+constexpr uint32_t Y_YY = Y_AL + 2 * TILE;      // [Yl_hi | Yl_lo]  } one N = 128 operand
+constexpr uint32_t Y_AQ = Y_YY + TILE;          // [AQ_hi | AQ_lo]  }
+constexpr uint32_t Y_BAR = Y_AQ + TILE;
+constexpr uint32_t Y_BYTES = Y_BAR + 64 + 1024;
+// TMEM: A* 0-127, then Yl 0-63 and AQ 64-127, then D4 0-63; D1 128-319, then AY 128-191 and
+// D3 192-319; A pairs hi 320-383, lo 384-447
+
+struct H3SParams {
+    int T, NC, slot;
+    float* sums;
+    int* status;
+};
+
+__global__ void __launch_bounds__(NT3, 1)
+k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v, H3SParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    // the prefix kernels may be scheduled once every summary CTA has started
+    if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int t0 = chunk * C;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Y_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+    float* out = p.sums + ((size_t)bh * p.NC + chunk) * p.slot;
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 512);
+        ptx::tmem_relinquish();
+    }
+    {
+        // Q, K, V rows to their split tiles: thread (r, h) takes columns 16h .. 16h+15 of row r
+        const int r = tid >> 1, h = tid & 1;
+        const bool in = t0 + r < p.T;
+        const size_t base = ((size_t)bh * p.T + t0 + r) * D3 + 16 * h;
+        float xq[16], xk[16], xv[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 a = in ? *reinterpret_cast<const float4*>(q + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 b = in ? *reinterpret_cast<const float4*>(k + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 c = in ? *reinterpret_cast<const float4*>(v + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            xq[4 * j] = a.x; xq[4 * j + 1] = a.y; xq[4 * j + 2] = a.z; xq[4 * j + 3] = a.w;
+            xk[4 * j] = b.x; xk[4 * j + 1] = b.y; xk[4 * j + 2] = b.z; xk[4 * j + 3] = b.w;
+            xv[4 * j] = c.x; xv[4 * j + 1] = c.y; xv[4 * j + 2] = c.z; xv[4 * j + 3] = c.w;
+        }
+        float hi[16], lo[16], z[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            hi[j] = hi_of(xq[j]);
+            lo[j] = xq[j] - hi[j];
+            z[j] = 0.f;
+        }
+        put16(sm + Y_QC, TILE, r, 16 * h, hi);
+        put16(sm + Y_QC, TILE, r, 32 + 16 * h, lo);
+        put16(sm + Y_QC, TILE, r, 64 + 16 * h, hi);
+        put16(sm + Y_QC, TILE, r, 96 + 16 * h, z);
+        put16(sm + Y_QQ, TILE, r, 16 * h, hi);
+        put16(sm + Y_QQ, TILE, r, 32 + 16 * h, lo);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            hi[j] = hi_of(xk[j]);
+            lo[j] = xk[j] - hi[j];
+        }
+        put16(sm + Y_KC, TILE, r, 16 * h, hi);
+        put16(sm + Y_KC, TILE, r, 32 + 16 * h, hi);
+        put16(sm + Y_KC, TILE, r, 64 + 16 * h, lo);
+        put16(sm + Y_KC, TILE, r, 96 + 16 * h, z);
+        put16(sm + Y_KK, TILE, r, 16 * h, hi);
+        put16(sm + Y_KK, TILE, r, 32 + 16 * h, lo);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            hi[j] = hi_of(xv[j]);
+            lo[j] = xv[j] - hi[j];
+        }
+        put16(sm + Y_VV, TILE, r, 16 * h, hi);
+        put16(sm + Y_VV, TILE, r, 32 + 16 * h, lo);
+    }
+#pragma unroll
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+        if (c0 > quad * 32 + 31) {
+            st_row32_zero(sm + Y_AH, row, c0);
+            st_row32_zero(sm + Y_AL, row, c0);
+        }
+    ptx::fence_proxy_async();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sb = ptx::smem_u32(sm);
+    auto st_pairs = [&](uint32_t tcol, const float* x) {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = ptx::pack_bf16(x[2 * i], x[2 * i + 1]);
+        ptx::tmem_st16u(tmem + lane_base + tcol, r);
+    };
+    {
+        uint32_t zr[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) zr[i] = 0u;
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
+            if (c0 > quad * 32 + 31) {
+                ptx::tmem_st16u(tmem + lane_base + 320 + c0 / 2, zr);
+                ptx::tmem_st16u(tmem + lane_base + 384 + c0 / 2, zr);
+            }
+    }
+    constexpr uint32_t I_QK = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t I_D1 = ptx::idesc_bf16(128, 192, true, true);
+    constexpr uint32_t I_M128 = ptx::idesc_bf16(128, 128, true, true);
+    constexpr uint32_t I_M64 = ptx::idesc_bf16(128, 64, true, true);
+    constexpr uint32_t I_KM = ptx::idesc_bf16(128, 64, false, true);
+    uint32_t phase = 0;
+    auto mma_wait = [&]() {
+        bool good = true;
+        if (tid == 0) {
+            ptx::umma_commit(bar);
+            good = ptx::mbar_wait(bar, phase);
+        }
+        phase ^= 1;
+        good = __syncthreads_and(good) != 0;
+        ptx::tc_fence_after();
+        return good;
+    };
+    auto sync_mma = [&]() {
+        ptx::tmem_st_wait();
+        ptx::fence_proxy_async();
+        ptx::tc_fence_before();
+        __syncthreads();
+        ptx::tc_fence_after();
+    };
+    // fp32 staging of the 64 x 64 block sums (over the K^T operand once R1 has read it):
+    // a thread of lane quadrant q holds rows 32 (q mod 2) .. of one operand half
+    float* stg = reinterpret_cast<float*>(sm + Y_KC);            // [4][64][64 + 4]
+    constexpr int SLD = 68;
+    // the 32 x 32 result of a 64 x 64 block (hi / lo of x by hi / lo of y) at TMEM column c0 in the
+    // rows (lanes) lane0 .. lane0 + 63: staged by the threads of those lanes, summed by 256 threads
+    auto block_to_slot = [&](uint32_t col, int lane0, int m) {
+        if (row >= lane0 && row < lane0 + 64) {
+            float v[32];
+            ptx::tmem_ld32(tmem + lane_base + col + half * 32, v);
+            float* dst = stg + (row - lane0) * SLD + half * 32;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(dst + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+        __syncthreads();
+        for (int e = tid; e < D3 * D3; e += NT3) {
+            const int a = e / D3, b = e % D3;
+            out[m * D3 * D3 + e] = stg[a * SLD + b] + stg[a * SLD + 32 + b] + stg[(32 + a) * SLD + b] +
+                                   stg[(32 + a) * SLD + 32 + b];
+        }
+        __syncthreads();
+    };
+    sync_mma();
+    bool ok = true;
+    if (tid == 0) {
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, kdesc2(sb + Y_QC, s), kdesc2(sb + Y_KC, s), I_QK, s > 0);
+        const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dB = mdesc(sb + Y_KK, TILE, 0);
+        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dA + (uint64_t)(s * 128), dB + (uint64_t)(s * 128), I_D1, s > 0);
+    }
+    ok = mma_wait();                                                  // R1 done
+    if (ok) {
+        // E1: A = L (.) A* to hi / lo pairs and tiles
+        float v[32], hi[32], lo[32];
+#pragma unroll
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            if (c0 > quad * 32 + 31) continue;
+            ptx::tmem_ld32(tmem + lane_base + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = (c0 + i <= row) ? v[i] : 0.f;
+                hi[i] = hi_of(x);
+                lo[i] = x - hi[i];
+            }
+            st_pairs(320 + c0 / 2, hi);
+            st_pairs(384 + c0 / 2, lo);
+            st_row32(sm + Y_AH, row, c0, hi);
+            st_row32(sm + Y_AL, row, c0, lo);
+        }
+        sync_mma();
+        if (tid == 0) {
+            const uint64_t dV = mdesc(sb + Y_VV, TILE, 0), dQ = mdesc(sb + Y_QQ, TILE, 0);
+            const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 320 + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 384 + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAH + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAL + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, 1);
+        }
+        // S, P, Q2 from D1 (rows K_hi, K_lo, Q_hi, Q_lo; columns K, V, Q, each hi | lo) while R2 runs
+        block_to_slot(128, 0, 0);          // K^T K
+        block_to_slot(128 + 64, 0, 2);     // K^T V
+        block_to_slot(128 + 128, 64, 1);   // Q^T Q
+        ok = mma_wait();                                              // R2 done
+    }
+    if (ok) {
+        // E2: Yl = A V, AQ = A^T Q (each the sum of its hi and lo halves) to split tiles
+        float a[16], b[16], hi[16], lo[16];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t col = t == 0 ? 0 : 64;
+            ptx::tmem_ld16(tmem + lane_base + col + 16 * half, a);
+            ptx::tmem_ld16(tmem + lane_base + col + 32 + 16 * half, b);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float y = a[i] + b[i];
+                hi[i] = hi_of(y);
+                lo[i] = y - hi[i];
+            }
+            uint8_t* tile = sm + (t == 0 ? Y_YY : Y_AQ);
+            put16(tile, TILE, row, 16 * half, hi);
+            put16(tile, TILE, row, 32 + 16 * half, lo);
+        }
+        sync_mma();
+        if (tid == 0) {
+            const uint64_t dY = mdesc(sb + Y_YY, TILE, 0), dYA = mdesc(sb + Y_YY, TILE, 0);
+            const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
+            const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAH + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, s > 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAL + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 192, dA + (uint64_t)(s * 128), dYA + (uint64_t)(s * 128), I_M128, s > 0);
+        }
+        ok = mma_wait();                                              // R3 done
+    }
+    if (ok) {
+        // E3: AY = A^T Yl to a split tile (over the concatenated Q, which R1 was the last to read)
+        float a[16], b[16], hi[16], lo[16];
+        ptx::tmem_ld16(tmem + lane_base + 128 + 16 * half, a);
+        ptx::tmem_ld16(tmem + lane_base + 128 + 32 + 16 * half, b);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float y = a[i] + b[i];
+            hi[i] = hi_of(y);
+            lo[i] = y - hi[i];
+        }
+        put16(sm + Y_QC, TILE, row, 16 * half, hi);
+        put16(sm + Y_QC, TILE, row, 32 + 16 * half, lo);
+        sync_mma();
+        if (tid == 0) {
+            const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dAY = mdesc(sb + Y_QC, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, dA + (uint64_t)(s * 128), dAY + (uint64_t)(s * 128), I_M64, s > 0);
+        }
+        // X = Q^T Yl (rows Q, columns Yl) and Z = K^T (A^T Q) (rows K, columns AQ) from D3
+        block_to_slot(192, 64, 4);
+        block_to_slot(192 + 64, 0, 5);
+        ok = mma_wait();                                              // R4 done
+    }
+    if (ok) {
+        block_to_slot(0, 0, 3);            // F = K^T (A^T (A V))
+        for (int e = tid; e < p.slot - 6 * D3 * D3; e += NT3) out[6 * D3 * D3 + e] = 0.f;   // vectors, padding
+        __syncthreads();
+        if (tid == 0) out[6 * D3 * D3 + 3 * D3] = 1.f;           // rho of the plain op
+    } else if (tid == 0) {
+        set_status(p.status, DEV_TIMEOUT);
+        ptx::umma_commit(bar);
+        ptx::mbar_wait(bar, phase, 100000000ull);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
 }  // namespace
 
 cudaError_t hla3_output(const float* q, const float* k, const float* v, const float* sums, int NCp, int slot_floats,
@@ -354,6 +646,21 @@ cudaError_t hla3_output(const float* q, const float* k, const float* v, const fl
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k_hla3_out, q, k, v, prm);
+}
+
+
+cudaError_t hla3_summaries(const float* q, const float* k, const float* v, float* sums, int NC, int slot_floats,
+                           int BH, int T, int* status, cudaStream_t st) {
+    H3SParams prm;
+    prm.T = T;
+    prm.NC = NC;
+    prm.slot = slot_floats;
+    prm.sums = sums;
+    prm.status = status;
+    cudaError_t e;
+    if ((e = set_smem(k_hla3_sum, Y_BYTES)) != cudaSuccess) return e;
+    k_hla3_sum<<<dim3((T + C - 1) / C, BH), NT3, Y_BYTES, st>>>(q, k, v, prm);
+    return cudaGetLastError();
 }
 
 }  // namespace tc

@@ -181,9 +181,9 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
 
 /*
  * 1 when this request runs on the tcgen05 tensor-core kernels, 2 when its
- * output kernel runs on them and its chunk summaries and prefix on the CUDA
- * cores (the plain third order with fp32 inputs at d = 32, whose output kernel
- * takes fp32 accuracy from products of two- and three-term bf16 splits), 0 when
+ * chunk summaries and output kernel run on them and the prefix between them on
+ * the CUDA cores (the plain third order with fp32 inputs at d = 32, which takes
+ * fp32 accuracy from products of two- and three-term bf16 splits), 0 when
  * it runs on the CUDA-core (fp32 FFMA) kernels or is invalid.  Same arguments
  * as hla_workspace_bytes().
  */
