@@ -130,14 +130,17 @@ int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int 
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
     const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
     if (use_tc(r)) return hla::tc::kernel_launches(r.op, r.norm, B * H, T, r.seg);
-    return hla::simt::kernel_launches(r.op, r.d, T);
+    return hla::simt::kernel_launches(r.op, r.norm, r.bf16, r.d, T);
 }
 
 int hla_uses_tensor_cores(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv) {
     if (hla_workspace_bytes(op, dtype, decayed, B, H, T, d, dv) == 0) return 0;
     const Request r = make_request(op, decayed != 0, dtype, B, H, T, d, dv);
     if (use_tc(r)) return 1;
-    return r.op == hla::OP_HLA3 && !r.norm && !r.bf16 && r.d == 32 ? 2 : 0;   // the tcgen05 output kernel
+    if (r.norm || r.bf16 || r.d != 32) return 0;
+    if (r.op == hla::OP_HLA3) return 2;                       // tcgen05 summaries and output
+    if (r.op == hla::OP_HLA2 && (T + 127) / 128 <= hla::tc::hla2f_max_chunks()) return 2;
+    return 0;
 }
 
 hla_status_t hla2_forward(const void* q, const void* k, const void* v, float* o, int B, int H, int T, int d,
@@ -262,7 +265,7 @@ size_t hla_backward_workspace_bytes(hla_op_t op, hla_dtype_t dtype, int B, int H
 int hla_backward_kernel_launches(hla_op_t op, hla_dtype_t dtype, int B, int H, int T, int d, int dv) {
     if (hla_backward_workspace_bytes(op, dtype, B, H, T, d, dv) == 0) return 0;
     if (op == HLA_OP_AHLA) return hla::simt::ahla_backward_launches(d, T);
-    return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(d, T)
+    return op == HLA_OP_HLA2_NORM ? hla::simt::backward_normalized_launches(dtype == HLA_BF16, d, T)
                                   : hla::simt::backward_launches(dtype == HLA_BF16, d, T);
 }
 

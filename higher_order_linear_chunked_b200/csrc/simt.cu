@@ -1103,11 +1103,22 @@ template <int OP, bool NORM, int D, typename TIn>
 constexpr bool tc_third_order() {
     return OP == OP_HLA3 && !NORM && D == 32 && std::is_same<TIn, float>::value;
 }
+// So does the plain second order with fp32 inputs at d = 32, up to tc::hla2f_max_chunks()
+// 128-token chunks per head (its output CTAs fold the summaries themselves).
+template <int OP, bool NORM, int D, typename TIn>
+constexpr bool tc_second_order_f32() {
+    return OP == OP_HLA2 && !NORM && D == 32 && std::is_same<TIn, float>::value;
+}
+static bool tc_second_order_f32_fits(int T) { return (T + 127) / 128 <= tc::hla2f_max_chunks(); }
 
 template <int OP, bool NORM, int D, typename TIn>
 static cudaError_t run(const void* q, const void* k, const void* v, const float* gamma, float eps, float* o,
-                       int BH, int H, int T, float* sums, int* status, cudaStream_t st, cudaEvent_t* ev) {
-    if (tc_third_order<OP, NORM, D, TIn>()) {
+                       int BH, int H, int T, float* sums, int* status, cudaStream_t st, cudaEvent_t* ev,
+                       bool allow_tc) {
+    if (allow_tc && tc_second_order_f32<OP, NORM, D, TIn>() && tc_second_order_f32_fits(T))
+        return tc::hla2f_forward((const float*)q, (const float*)k, (const float*)v, sums, Sum<OP, D>::SIZE, o, BH, T,
+                                 status, st, ev);
+    if (allow_tc && tc_third_order<OP, NORM, D, TIn>()) {
         // the plain third order with fp32 inputs at d = 32: summaries and output on the tensor
         // cores over 128-token chunks, the factored prefix between them on the CUDA cores
         const int NC2 = (T + 127) / 128;
@@ -1159,41 +1170,44 @@ static cudaError_t run(const void* q, const void* k, const void* v, const float*
 template <typename TIn, int D>
 static cudaError_t dispatch_op(int op, bool norm, const void* q, const void* k, const void* v, const float* gamma,
                                float eps, float* o, int BH, int H, int T, float* sums, int* status, cudaStream_t st,
-                               cudaEvent_t* ev) {
+                               cudaEvent_t* ev, bool allow_tc) {
     switch (op) {
     case OP_HLA2:
-        return norm ? run<OP_HLA2, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_HLA2, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_HLA2, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_HLA2, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     case OP_HLA2D:
-        return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_HLA2D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_HLA2D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     case OP_AHLA:
-        return norm ? run<OP_AHLA, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_AHLA, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_AHLA, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     case OP_HLA3:
-        return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
-    case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_HLA3, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_HLA3, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
+    case OP_HLA2U: return run<OP_HLA2U, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     case OP_AHLAD:
-        return norm ? run<OP_AHLAD, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_AHLAD, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_AHLAD, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_AHLAD, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     case OP_HLA3D:
-        return norm ? run<OP_HLA3D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev)
-                    : run<OP_HLA3D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+        return norm ? run<OP_HLA3D, true, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc)
+                    : run<OP_HLA3D, false, D, TIn>(q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
     }
     return cudaErrorInvalidValue;
 }
 
 cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,
                     const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, int* status,
-                    cudaStream_t st, cudaEvent_t* ev) {
+                    cudaStream_t st, cudaEvent_t* ev, bool allow_tc) {
     if (bf16) {
         if (d == 32)
-            return dispatch_op<__nv_bfloat16, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
-        return dispatch_op<__nv_bfloat16, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+            return dispatch_op<__nv_bfloat16, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev,
+                                                  allow_tc);
+        return dispatch_op<__nv_bfloat16, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev,
+                                              allow_tc);
     }
-    if (d == 32) return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
-    return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev);
+    if (d == 32)
+        return dispatch_op<float, 32>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
+    return dispatch_op<float, 64>(op, norm, q, k, v, gamma, eps, o, BH, H, T, sums, status, st, ev, allow_tc);
 }
 
 static bool uses_fold(int op, int d) {
@@ -1209,7 +1223,8 @@ static bool uses_fold(int op, int d) {
     return false;
 }
 
-int kernel_launches(int op, int d, int T) {
+int kernel_launches(int op, bool norm, bool bf16, int d, int T) {
+    if (op == OP_HLA2 && !norm && !bf16 && d == 32 && tc_second_order_f32_fits(T)) return 2;   // tcgen05, folded prefix
     if (op == OP_HLA3 || op == OP_HLA3D) return 2 + 3;   // the factored prefix (decayed or not)
     return 2 + (uses_fold(op, d) ? 1 : scan_launches(next_pow2((T + C - 1) / C)));
 }
@@ -1940,7 +1955,7 @@ int backward_launches(bool bf16, int d, int T) {
     // term, gradients (128-token chunks); otherwise summaries, the scan, the same adjoint stages
     // (64-token chunks), gradients
     if (bf16 && d == 64) return 4 + 5;
-    return kernel_launches(OP_HLA2, d, T) - 1 + 5;
+    return kernel_launches(OP_HLA2, false, true, d, T) - 1 + 5;
 }
 
 template <int D, typename TIn>
@@ -2050,9 +2065,10 @@ size_t backward_normalized_workspace_floats(int d, int BH, int T) {
     return 8 * n + inner;
 }
 
-int backward_normalized_launches(int d, int T) {
+int backward_normalized_launches(bool bf16, int d, int T) {
     // two plain forwards, the ones, the gradient split, two plain backwards, two additions
-    return 2 * kernel_launches(OP_HLA2, d, T) + 1 + 1 + 2 * backward_launches(false, d, T) + 2;
+    // (the two forwards stay on the CUDA cores: the gradient combines them with cancellation)
+    return 2 * kernel_launches(OP_HLA2, false, true, d, T) + 1 + 1 + 2 * backward_launches(false, d, T) + 2;
 }
 
 cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
@@ -2073,10 +2089,10 @@ cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, 
     if (bf16) k_fill_ones<__nv_bfloat16><<<blocks, NT, 0, st>>>(reinterpret_cast<__nv_bfloat16*>(ones), n);
     else k_fill_ones<float><<<blocks, NT, 0, st>>>(ones, n);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = forward(OP_HLA2, false, bf16, d, q, k, v, nullptr, 0.f, num, BH, 1, T, inner, status, st, nullptr)) !=
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, v, nullptr, 0.f, num, BH, 1, T, inner, status, st, nullptr, false)) !=
         cudaSuccess)
         return e;
-    if ((e = forward(OP_HLA2, false, bf16, d, q, k, ones, nullptr, 0.f, den, BH, 1, T, inner, status, st, nullptr)) !=
+    if ((e = forward(OP_HLA2, false, bf16, d, q, k, ones, nullptr, 0.f, den, BH, 1, T, inner, status, st, nullptr, false)) !=
         cudaSuccess)
         return e;
     const size_t rows = (size_t)BH * T;
@@ -2205,7 +2221,7 @@ size_t ahla_backward_workspace_floats(int d, int BH, int T) {
 
 int ahla_backward_launches(int d, int T) {
     // summaries, the scan, chunk terms, two suffix sums, cross term, gradients
-    return kernel_launches(OP_AHLA, d, T) - 1 + 5;
+    return kernel_launches(OP_AHLA, false, true, d, T) - 1 + 5;
 }
 
 template <int D, typename TIn>

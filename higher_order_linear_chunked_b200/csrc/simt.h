@@ -10,7 +10,7 @@ namespace simt {
 size_t summary_floats(int op, int d);
 // kernels one forward enqueues (chunk kernel, the scan: one fold launch, or one launch per
 // tree level when three summaries do not fit in shared memory, output kernel)
-int kernel_launches(int op, int d, int T);
+int kernel_launches(int op, bool norm, bool bf16, int d, int T);
 // floats of workspace the path needs after the status block
 size_t workspace_floats(int op, int d, int BH, int T);
 // summary layout helpers for other paths: offsets (in floats) of matrix / vector slots
@@ -23,9 +23,10 @@ cudaError_t scan(int op, int d, float* sums, int NCp, int BH, cudaStream_t st);
 int scan_launches(int NCp);
 // enqueue chunk kernel, Blelloch scan levels and output kernel on `st`; `ev` (NULL or
 // 4 events) is recorded before the chunk kernel, after it, after the scan, after the output kernel
+// allow_tc = false keeps every kernel on the CUDA cores (fp32 FFMA throughout)
 cudaError_t forward(int op, bool norm, bool bf16, int d, const void* q, const void* k, const void* v,
                     const float* gamma, float eps, float* o, int BH, int H, int T, float* sums, int* status,
-                    cudaStream_t st, cudaEvent_t* ev);
+                    cudaStream_t st, cudaEvent_t* ev, bool allow_tc = true);
 
 // Streaming state: one summary (summary_floats(op, d) floats) per head.
 // state(): the state of each head after its T tokens (chunk kernel, up-sweep, copy of the
@@ -56,7 +57,7 @@ cudaError_t ahla_backward(bool bf16, int d, const void* q, const void* k, const 
 // The same for the ratio-normalised output (two plain forwards, two plain backwards, element-wise
 // glue); ws: backward_normalized_workspace_floats floats.
 size_t backward_normalized_workspace_floats(int d, int BH, int T);
-int backward_normalized_launches(int d, int T);
+int backward_normalized_launches(bool bf16, int d, int T);
 cudaError_t backward_normalized(bool bf16, int d, const void* q, const void* k, const void* v, const float* dout,
                                 float eps, float* dq, float* dk, float* dv, int BH, int T, float* ws, int* status,
                                 cudaStream_t st);

@@ -53,6 +53,13 @@ cudaError_t hla3_summaries(const float* q, const float* k, const float* v, float
                            int BH, int T, int* status, cudaStream_t st);
 cudaError_t hla3_output(const float* q, const float* k, const float* v, const float* sums, int NCp, int slot_floats,
                         float* o, int BH, int T, int* status, cudaStream_t st);
+// the plain second order (fp32 q, k, v, d = dv = 32) on tcgen05 from two- and three-term bf16
+// splits, 128-token chunks, for at most hla2f_max_chunks() chunks per head: the chunk summaries
+// into sums ([BH][chunks][slot_floats], the CUDA-core slot layout), then the output with each
+// CTA folding the summaries before its chunk; two launches, ev as for forward()
+int hla2f_max_chunks();
+cudaError_t hla2f_forward(const float* q, const float* k, const float* v, float* sums, int slot_floats, float* o,
+                          int BH, int T, int* status, cudaStream_t st, cudaEvent_t* ev);
 // one tcgen05 MMA on one CTA (layout self-check; see hla_selftest_umma in include/hla.h)
 cudaError_t selftest(int layout_case, const void* a, const void* b, float* d, int N, int K, cudaStream_t st);
 // a bounded wait that runs out (see hla_selftest_wait_timeout in include/hla.h)

@@ -99,6 +99,17 @@ __device__ __forceinline__ void st_row32_zero(uint8_t* tile, int row, int c0) {
     }
 }
 
+// ---------------------------------------------------------------- bf16 splits of fp32 values
+// x = x1 + x2 (+ x3): each term the bf16 rounding of what the earlier ones leave (exact in bf16);
+// the residual is about 2^-16 |x| after two terms and 2^-24 |x| after three.
+__device__ __forceinline__ float bf16_hi(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+__device__ __forceinline__ void bf16_split3(float x, float& a, float& b, float& c) {
+    a = bf16_hi(x);
+    const float r = x - a;
+    b = bf16_hi(r);
+    c = bf16_hi(r - b);
+}
+
 // ---------------------------------------------------------------- host side
 // Dynamic shared memory of a kernel, with the whole unified L1 / shared array preferred as shared
 // memory: the default carveout can leave room for only one CTA of ~100 KB on an SM, which would

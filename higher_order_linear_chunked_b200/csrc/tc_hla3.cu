@@ -65,14 +65,8 @@ constexpr uint32_t T_AL = 288;   // A_lo pairs, then W_lo pairs (64)
 constexpr uint32_t T_D = 352;    // D_y, then D_o (64)
 constexpr uint32_t T_PC = 416;   // [p1 | p2 | p1] pairs (48)
 
-__device__ __forceinline__ float hi_of(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
-// three bf16 terms of x (each exact in bf16; x - x1 - x2 - x3 is about 2^-24 x)
-__device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
-    a = hi_of(x);
-    const float r = x - a;
-    b = hi_of(r);
-    c = hi_of(r - b);
-}
+__device__ __forceinline__ float hi_of(float x) { return bf16_hi(x); }
+__device__ __forceinline__ void split3(float x, float& a, float& b, float& c) { bf16_split3(x, a, b, c); }
 
 // 16 values into columns c0 .. c0+15 of row `row` of a K-major tile whose 64-wide atoms lie
 // `atom` bytes apart (128B swizzle)

@@ -180,10 +180,12 @@ hla_status_t hla_forward_profiled(hla_op_t op, const void* q, const void* k, con
 int hla_kernel_launches(hla_op_t op, hla_dtype_t dtype, int decayed, int B, int H, int T, int d, int dv);
 
 /*
- * 1 when this request runs on the tcgen05 tensor-core kernels, 2 when its
- * chunk summaries and output kernel run on them and the prefix between them on
- * the CUDA cores (the plain third order with fp32 inputs at d = 32, which takes
- * fp32 accuracy from products of two- and three-term bf16 splits), 0 when
+ * 1 when this request runs on the tcgen05 tensor-core kernels, 2 when it takes
+ * the fp32-input tensor-core kernels that get fp32 accuracy from products of
+ * two- and three-term bf16 splits (the plain third order at d = 32: summaries
+ * and output, with the prefix between them on the CUDA cores; the plain second
+ * order at d = 32 with at most 64 chunks of 128 tokens per head: summaries and
+ * output, the prefix folded into the output kernel), 0 when
  * it runs on the CUDA-core (fp32 FFMA) kernels or is invalid.  Same arguments
  * as hla_workspace_bytes().
  */

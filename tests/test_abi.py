@@ -86,6 +86,12 @@ def test_tensor_core_routing_launches_and_workspace(lib):
     assert use(hla.OP_HLA3, f32, 0, d=32) == 2
     assert use(hla.OP_HLA3, f32, 1, d=32) == 0 and use(hla.OP_HLA3_NORM, f32, 0, d=32) == 0
     assert use(hla.OP_HLA3, f32, 0) == 0 and use(hla.OP_HLA3, bf16, 0, d=32) == 0
+    # the plain second order with fp32 inputs at d = 32: summaries and output on the tensor cores
+    # while the output CTAs can fold the summaries (up to 64 chunks of 128 tokens per head)
+    assert use(hla.OP_HLA2, f32, 0, d=32) == 2 and launches(hla.OP_HLA2, f32, 0, d=32) == 2
+    assert use(hla.OP_HLA2, f32, 0, T=8192, d=32) == 2 and use(hla.OP_HLA2, f32, 0, T=8193, d=32) == 0
+    assert launches(hla.OP_HLA2, f32, 0, T=8193, d=32) == 3
+    assert use(hla.OP_HLA2_NORM, f32, 0, d=32) == 0 and use(hla.OP_HLA2, f32, 1, d=32) == 0
     assert use(hla.OP_HLA2_NORM, bf16, 1) == 0
     # launches per forward: summary walker, the prefix (with up to nine summary slots per head
     # folded into the output walker; else three kernels), output walker; the decayed second

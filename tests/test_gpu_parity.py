@@ -272,6 +272,20 @@ def test_third_order_tensor_core_output(T):
     assert err <= TOL["f32"], err
 
 
+@pytest.mark.parametrize("T", [1, 100, 128, 129, 256, 1000, 4097, 8192, 8193])
+def test_second_order_fp32_tensor_cores(T):
+    """The plain second order with fp32 inputs at d = 32: tensor-core summaries and output with
+    the prefix folded into every output CTA, up to 64 chunks per head; one chunk more takes the
+    CUDA-core path.  fp32 tolerance either way."""
+    on_tc = hla.uses_tensor_cores(hla.OP_HLA2, hla.HLA_F32, False, 1, 2, T, 32, 32)
+    assert on_tc == (2 if T <= 8192 else 0)
+    w = recipe("hla2", "f32", 1, 2, T, 32, seed=T + 29)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward("hla2", q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2", q, k, v))
+    assert err <= TOL["f32"], err
+
+
 def test_third_order_tensor_core_output_large_values():
     """Inputs 8x larger than the workload's (a wider dynamic range for the bf16 splits)."""
     w = recipe("hla3", "f32", 1, 2, 2000, 32, seed=3)
