@@ -222,11 +222,17 @@ def test_normalized_constant_v_gives_den_ratio():
 
 
 def test_decay_gamma_one_matches_undecayed():
+    """gamma = 1 reduces the decayed op (CUDA cores, fp32 FFMA) to the undecayed one (at fp32 and
+    d = 32 the tensor-core kernels with split products, about 2e-5 from the oracle): both match
+    the oracle at the fp32 gate, and each other within two of it."""
     w = recipe("hla2", "f32", 1, 2, 200, 32, seed=4)
     q, k, v, _ = hla_inputs.make_inputs(w)
     a = gpu_forward("hla2d", q, k, v, torch.ones(2))
     b = gpu_forward("hla2", q, k, v, None)
-    assert oracle.max_row_rel_err(a.cpu(), b.cpu()) < 1e-5
+    ref = oracle.recur("hla2", q, k, v)
+    assert oracle.max_row_rel_err(a.cpu(), ref) <= TOL["f32"]
+    assert oracle.max_row_rel_err(b.cpu(), ref) <= TOL["f32"]
+    assert oracle.max_row_rel_err(a.cpu(), b.cpu()) <= 2 * TOL["f32"]
 
 
 @pytest.mark.parametrize("T", [300, 2049])
