@@ -56,23 +56,6 @@ __device__ __forceinline__ float gpow_n(float g, int n) {
     return r;
 }
 
-// Shared bounded commit-and-wait of the issuing thread; the block agrees on the result.
-struct MmaSync {
-    uint64_t* bar;
-    uint32_t phase;
-    __device__ bool commit_wait(bool issuer) {
-        bool good = true;
-        if (issuer) {
-            ptx::umma_commit(bar);
-            good = ptx::mbar_wait(bar, phase);
-        }
-        phase ^= 1;
-        good = __syncthreads_and(good) != 0;
-        ptx::tc_fence_after();
-        return good;
-    }
-};
-
 __device__ __forceinline__ void sync_for_mma() {
     ptx::fence_proxy_async();
     ptx::tc_fence_before();

@@ -212,6 +212,26 @@ def test_no_write_outside_output(op):
     assert hla.read_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("op", ["hla2", "hla3"])
+@pytest.mark.parametrize("T", [1, 190, 4097])
+def test_no_write_outside_output_fp32_tensor_cores(op, T):
+    """The fp32, d = 32 tensor-core kernels store O rows with plain stores: NaN guard bands on
+    both sides of the output stay untouched, and every output value is finite."""
+    w = recipe(op, "f32", 1, 2, T, 32, seed=T)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    dev = torch.device("cuda:0")
+    n = 2 * T * 32
+    guard = 4096
+    buf = torch.full((n + 2 * guard,), float("nan"), device=dev)
+    out = buf[guard:guard + n].view(1, 2, T, 32)
+    ws = hla.make_workspace(hla.OP_CODES[op], q.to(dev), v.to(dev), decayed=False)
+    hla.forward(op, q.to(dev), k.to(dev), v.to(dev), gamma=None, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:guard]).all() and torch.isnan(buf[guard + n:]).all()
+    assert torch.isfinite(out).all()
+    assert hla.read_device_status(ws) == 0
+
+
 def test_normalized_constant_v_gives_den_ratio():
     w = recipe("hla2n", "bf16", 1, 2, 300, 64, seed=9)
     q, k, _, _ = hla_inputs.make_inputs(w)
