@@ -51,7 +51,9 @@ struct Dim {
 // Programmatic dependent launch between the kernels of one forward: a kernel lets the next one
 // launch as soon as all of its CTAs have started (pdl_release), and the next one waits for its
 // completion (pdl_wait) before it reads what that kernel wrote; loads of the forward's inputs go
-// before the wait.  Both are no-ops for a kernel launched without the attribute.
+// before the wait.  Both are no-ops for a kernel launched without the attribute.  A pointer read
+// after the wait carries no __restrict__: with it the compiler may take the data as fixed for the
+// whole kernel and move a batch of its loads above the wait, before the earlier kernel is done.
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
@@ -114,65 +116,66 @@ __host__ __device__ constexpr bool decayed_op(int op) { return op == OP_HLA2D ||
 // ---------------------------------------------------------------------------
 // Block-cooperative small matrix products in shared/global memory.
 //   out(m,n) = init(m,n) + sum_k a1(m,k) b1(k,n) [+ sum_k a2(m,k) b2(k,n) ...]
-// Thread owns the 4x4 outputs (tm + i*M/4, tn + j*N/4): a() reads are
-// broadcasts within a warp, b() reads walk consecutive n (conflict-free).
+// Thread owns the R x R outputs (tm + i*M/R, tn + j*N/R), R = 4 unless a caller spreads a small
+// product over more threads: a() reads are broadcasts within a warp, b() reads walk consecutive
+// n (conflict-free).
 // ---------------------------------------------------------------------------
 struct Zero {
     __device__ float operator()(int, int) const { return 0.f; }
 };
 
-template <int M, int N, int K1, int K2, int K3, class A1, class B1, class A2, class B2, class A3,
+template <int M, int N, int K1, int K2, int K3, int R = 4, class A1, class B1, class A2, class B2, class A3,
           class B3, class FI, class FS>
 __device__ __forceinline__ void mm3(A1 a1, B1 b1, A2 a2, B2 b2, A3 a3, B3 b3, FI init, FS store) {
-    static_assert(M % 4 == 0 && N % 4 == 0, "tile");
-    constexpr int RM = M / 4, RN = N / 4;
+    static_assert(M % R == 0 && N % R == 0, "tile");
+    constexpr int RM = M / R, RN = N / R;
     for (int tile = threadIdx.x; tile < RM * RN; tile += blockDim.x) {
         const int tm = tile / RN, tn = tile % RN;
-        float acc[4][4];
+        float acc[R][R];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = init(tm + i * RM, tn + j * RN);
+            for (int j = 0; j < R; ++j) acc[i][j] = init(tm + i * RM, tn + j * RN);
 #pragma unroll 4
         for (int kk = 0; kk < K1; ++kk) {
-            float av[4], bv[4];
+            float av[R], bv[R];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) av[i] = a1(tm + i * RM, kk);
+            for (int i = 0; i < R; ++i) av[i] = a1(tm + i * RM, kk);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = b1(kk, tn + j * RN);
+            for (int j = 0; j < R; ++j) bv[j] = b1(kk, tn + j * RN);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < R; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                for (int j = 0; j < R; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
 #pragma unroll 4
         for (int kk = 0; kk < K2; ++kk) {
-            float av[4], bv[4];
+            float av[R], bv[R];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) av[i] = a2(tm + i * RM, kk);
+            for (int i = 0; i < R; ++i) av[i] = a2(tm + i * RM, kk);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = b2(kk, tn + j * RN);
+            for (int j = 0; j < R; ++j) bv[j] = b2(kk, tn + j * RN);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < R; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                for (int j = 0; j < R; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
 #pragma unroll 4
         for (int kk = 0; kk < K3; ++kk) {
-            float av[4], bv[4];
+            float av[R], bv[R];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) av[i] = a3(tm + i * RM, kk);
+            for (int i = 0; i < R; ++i) av[i] = a3(tm + i * RM, kk);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = b3(kk, tn + j * RN);
+            for (int j = 0; j < R; ++j) bv[j] = b3(kk, tn + j * RN);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < R; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                for (int j = 0; j < R; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) store(tm + i * RM, tn + j * RN, acc[i][j]);
+            for (int j = 0; j < R; ++j) store(tm + i * RM, tn + j * RN, acc[i][j]);
     }
 }
 
@@ -211,11 +214,25 @@ struct Put {                    // plain store into a tile
 // Load `rows` chunk rows (zero beyond T) of a [T][D] head slice into a padded fp32 tile.
 template <int D, typename TIn>
 __device__ __forceinline__ void load_rows(float* dst, const TIn* src, int t0, int T) {
-    constexpr int LD = Dim<D>::LD;
-    for (int e = threadIdx.x; e < C * D; e += blockDim.x) {
-        const int r = e / D, c = e % D;
-        const int t = t0 + r;
-        dst[r * LD + c] = (t < T) ? to_f32(src[(size_t)t * D + c]) : 0.f;
+    constexpr int LD = Dim<D>::LD, PER = C * D / NT;
+    static_assert(C * D % NT == 0, "whole tiles per pass");
+    if constexpr (PER > 8) {                 // d = 64: one value at a time (keeps the registers of
+        for (int e = threadIdx.x; e < C * D; e += blockDim.x) {     // the kernels around it)
+            const int t = t0 + e / D;
+            dst[(e / D) * LD + e % D] = (t < T) ? to_f32(src[(size_t)t * D + e % D]) : 0.f;
+        }
+    } else {                                 // d = 32: all loads of the tile in flight, then the stores
+        float x[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = threadIdx.x + i * NT, t = t0 + e / D;
+            x[i] = (t < T) ? to_f32(src[(size_t)t * D + e % D]) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = threadIdx.x + i * NT;
+            dst[(e / D) * LD + e % D] = x[i];
+        }
     }
 }
 
@@ -224,6 +241,33 @@ template <int D>
 __device__ __forceinline__ void load_mat(float* dst, const float* src) {
     constexpr int LD = Dim<D>::LD;
     for (int e = threadIdx.x; e < D * D; e += blockDim.x) dst[(e / D) * LD + (e % D)] = src[e];
+}
+
+// NM row-major D x D matrices from global memory into padded shared tiles, by a block of NT
+// threads: every load is issued before the first store, so one memory latency covers them all
+// (a store waits for its load, and a warp issues in order).
+// At d = 64 (16 values a thread per matrix) the matrices go one after the other, which keeps
+// the registers of the kernels around them.
+template <int D, int NM>
+__device__ __forceinline__ void load_mats(float* const (&dst)[NM], const float* const (&src)[NM]) {
+    constexpr int LD = Dim<D>::LD, PER = D * D / NT;
+    static_assert(D * D % NT == 0, "whole matrices per pass");
+    constexpr int G = PER * NM <= 24 ? NM : 1;          // matrices per batch of loads
+#pragma unroll
+    for (int m0 = 0; m0 < NM; m0 += G) {
+        float x[G][PER];
+#pragma unroll
+        for (int m = 0; m < G; ++m)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) x[m][i] = src[m0 + m][threadIdx.x + i * NT];
+#pragma unroll
+        for (int m = 0; m < G; ++m)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = threadIdx.x + i * NT;
+                dst[m0 + m][(e / D) * LD + (e % D)] = x[m][i];
+            }
+    }
 }
 
 __device__ __forceinline__ float gpow(float g, int n) {  // gamma^n, n >= 0
@@ -605,7 +649,7 @@ __device__ void combine_into(const float* A, const float* B, float* out, float* 
 }
 
 template <int OP, int D>
-__global__ void __launch_bounds__(NT) k_scan_level(float* __restrict__ sums, int NCp, int step, int down, int root) {
+__global__ void __launch_bounds__(NT) k_scan_level(float* sums, int NCp, int step, int down, int root) {
     using S = Sum<OP, D>;
     pdl_release();
     pdl_wait();
@@ -661,7 +705,7 @@ template <int OP, int D>
 constexpr bool fold_fits() { return OP != OP_HLA3 && OP != OP_HLA3D && fold_smem<OP, D>() <= 227 * 1024; }
 
 template <int OP, int D>
-__global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int NC, int NCp) {
+__global__ void __launch_bounds__(NT) k_scan_fold(float* sums, int NC, int NCp) {
     using S = Sum<OP, D>;
     constexpr int N4 = S::SIZE / 4, PER = (N4 + NT - 1) / NT;
     pdl_release();
@@ -718,7 +762,7 @@ __global__ void __launch_bounds__(NT) k_scan_fold(float* __restrict__ sums, int 
 // F_l + rho_l (...), with the same three launches.
 // ---------------------------------------------------------------------------
 template <int OP, int D>
-__global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ sums, int NC, int NCp, int which) {
+__global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* sums, int NC, int NCp, int which) {
     using S = Sum<OP, D>;
     pdl_release();
     pdl_wait();
@@ -734,16 +778,17 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ su
     float* p = sums + (size_t)blockIdx.y * NCp * S::SIZE + off;
     const float* rho = sums + (size_t)blockIdx.y * NCp * S::SIZE + S::SCAL;
     float run = 0.f;
-    for (int l0 = 0; l0 < NC; l0 += 8) {     // eight loads in flight, then the dependent adds
-        float y[8], r[8];
+    constexpr int B = 32;                    // B loads in flight, then the dependent adds
+    for (int l0 = 0; l0 < NC; l0 += B) {
+        float y[B], r[B];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < B; ++i)
             if (l0 + i < NC) {
                 y[i] = p[(size_t)(l0 + i) * S::SIZE];
                 r[i] = OP == OP_HLA3D ? rho[(size_t)(l0 + i) * S::SIZE] : 1.f;
             }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < B; ++i)
             if (l0 + i < NC) {
                 p[(size_t)(l0 + i) * S::SIZE] = run;
                 run = OP == OP_HLA3D ? fmaf(r[i], run, y[i]) : run + y[i];
@@ -752,7 +797,7 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_plain(float* __restrict__ su
 }
 
 template <int OP, int D>
-__global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ sums, int NCp) {
+__global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* sums, int NCp) {
     using S = Sum<OP, D>;
     pdl_release();
     pdl_wait();
@@ -767,23 +812,23 @@ __global__ void __launch_bounds__(NT) k_hla3_prefix_cross(float* __restrict__ su
     float* mk = Zs + D * LD;
     float* x1 = mk + D;
     float* slot = sums + ((size_t)blockIdx.y * NCp + blockIdx.x) * S::SIZE;
-    load_mat<D>(S0, slot + S::mat(0));       // S0(l) (the plain prefix, in place)
-    load_mat<D>(Q2, slot + S::mat(1));
-    load_mat<D>(P0, slot + S::mat(2));       // P0(l)
-    load_mat<D>(Xs, slot + S::mat(4));
-    load_mat<D>(Zs, slot + S::mat(5));
+    // S0(l) and P0(l) (the plain prefixes, in place), the chunk's Q2, X, Z
+    load_mats<D, 5>({S0, Q2, P0, Xs, Zs}, {slot + S::mat(0), slot + S::mat(1), slot + S::mat(2), slot + S::mat(4),
+                                          slot + S::mat(5)});
     for (int a = threadIdx.x; a < D; a += blockDim.x) {
         mk[a] = slot[S::vec(0) + a];
         x1[a] = slot[S::vec(1) + a];
     }
     __syncthreads();
-    mm<D, D, D>(Tile{S0, LD}, Tile{Q2, LD}, Zero{}, Put{SQ, LD});                  // S0 Q2
+    constexpr int R = D * D >= 16 * NT ? 4 : 2;       // 2 x 2 per thread at d = 32: every thread works
+    mm3<D, D, D, 0, 0, R>(Tile{S0, LD}, Tile{Q2, LD}, Tile{S0, LD}, Tile{Q2, LD}, Tile{S0, LD}, Tile{Q2, LD},
+                          Zero{}, Put{SQ, LD});                                  // S0 Q2
     __syncthreads();
     float* F = slot + S::mat(3);
     const float rho = OP == OP_HLA3D ? slot[S::SCAL] : 1.f;
     // F += rho ((S0 Q2) P0 + S0 X + Z P0)
-    mm3<D, D, D, D, D>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, Tile{Xs, LD}, Tile{Zs, LD}, Tile{P0, LD}, Zero{},
-                       [&](int r, int c, float x) { F[r * D + c] = fmaf(rho, x, F[r * D + c]); });
+    mm3<D, D, D, D, D, R>(Tile{SQ, LD}, Tile{P0, LD}, Tile{S0, LD}, Tile{Xs, LD}, Tile{Zs, LD}, Tile{P0, LD}, Zero{},
+                          [&](int r, int c, float x) { F[r * D + c] = fmaf(rho, x, F[r * D + c]); });
     for (int a = threadIdx.x; a < D; a += blockDim.x) {
         float s = 0.f;
         for (int b = 0; b < D; ++b) s += SQ[a * LD + b] * mk[b] + S0[a * LD + b] * x1[b] + Zs[a * LD + b] * mk[b];
@@ -809,7 +854,7 @@ static cudaError_t hla3_factored_prefix(float* sums, int NC, int NCp, int BH, cu
 template <int OP, bool NORM, int D, typename TIn>
 __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const TIn* __restrict__ k,
                                                const TIn* __restrict__ v, const float* __restrict__ gamma,
-                                               float eps, int H, int T, int NCp, const float* __restrict__ sums,
+                                               float eps, int H, int T, int NCp, const float* sums,
                                                float* __restrict__ o) {
     using S = Sum<OP, D>;
     constexpr int LD = Dim<D>::LD;
@@ -837,13 +882,10 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
     pdl_wait();                              // the prefixes below come from the scan
     float g = 1.f;
     if (OP == OP_HLA2) {
-        load_mat<D>(M0, pre + S::mat(0));   // S0
-        load_mat<D>(M1, pre + S::mat(2));   // R0
+        load_mats<D, 2>({M0, M1}, {pre + S::mat(0), pre + S::mat(2)});       // S0, R0
         for (int a = threadIdx.x; a < D; a += blockDim.x) vec[a] = pre[S::vec(1) + a];  // r0
     } else if (OP == OP_HLA2D) {
-        load_mat<D>(M0, pre + S::mat(0));   // S0
-        load_mat<D>(M1, pre + S::mat(1));   // C0
-        load_mat<D>(M2, pre + S::mat(2));   // G0
+        load_mats<D, 3>({M0, M1, M2}, {pre + S::mat(0), pre + S::mat(1), pre + S::mat(2)});   // S0, C0, G0
         for (int a = threadIdx.x; a < D; a += blockDim.x) {
             vec[a] = pre[S::vec(0) + a];      // m0
             vec[D + a] = pre[S::vec(1) + a];  // h0
@@ -851,19 +893,15 @@ __global__ void __launch_bounds__(NT) k_output(const TIn* __restrict__ q, const 
         g = gamma[bh % H];
         for (int j = threadIdx.x; j <= C; j += blockDim.x) gp[j] = gpow(g, j);
     } else if (OP == OP_HLA2U) {
-        load_mat<D>(M0, pre + S::mat(0));   // S0
-        load_mat<D>(M1, pre + S::mat(1));   // C0
+        load_mats<D, 2>({M0, M1}, {pre + S::mat(0), pre + S::mat(1)});       // S0, C0
     } else if (OP == OP_AHLA || OP == OP_AHLAD) {
-        load_mat<D>(M0, pre + S::mat(0));   // P0
-        load_mat<D>(M1, pre + S::mat(1));   // E0
+        load_mats<D, 2>({M0, M1}, {pre + S::mat(0), pre + S::mat(1)});       // P0, E0
         for (int a = threadIdx.x; a < D; a += blockDim.x) {
             vec[a] = pre[S::vec(0) + a];      // mK0
             vec[D + a] = pre[S::vec(1) + a];  // n0
         }
     } else {
-        load_mat<D>(M0, pre + S::mat(0));   // S0
-        load_mat<D>(M1, pre + S::mat(2));   // P0
-        load_mat<D>(M2, pre + S::mat(3));   // F0
+        load_mats<D, 3>({M0, M1, M2}, {pre + S::mat(0), pre + S::mat(2), pre + S::mat(3)});   // S0, P0, F0
         for (int a = threadIdx.x; a < D; a += blockDim.x) {
             vec[a] = pre[S::vec(0) + a];      // mK0
             vec[D + a] = pre[S::vec(2) + a];  // F1_0

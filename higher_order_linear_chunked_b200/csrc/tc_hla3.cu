@@ -20,7 +20,9 @@
 // slots, [p1 | p2 | p1]).  Where it runs over the 128 tokens, the A side comes from TMEM as hi and
 // lo bf16 pairs and the B side is a [y_hi | y_lo] tile (64 columns) or separate hi and lo tiles.
 //
-// One CTA (8 warps, one TMEM lane quadrant per warp pair) per chunk x head:
+// Both kernels are persistent: one CTA (8 warps, one TMEM lane quadrant per warp pair) per SM
+// walks the (chunk, head) items, and the next item's Q, K, V rows are in flight (in registers)
+// while the current item's products run.  The output kernel, per item:
 //   R1  [A* | P | Q P0 | Q F0] = [Q] [K ; S0^T ; P0^T ; F0^T]^T   (N = 224, K = 192 concatenated)
 //       -> E1: A = L (.) A* to hi / lo pairs (TMEM) and hi / lo tiles; P to its concatenated pairs
 //   R2  W = P Q^T + A A^T (hi.hi + hi.lo + lo.hi);  D_y = A [V_hi | V_lo]
@@ -77,6 +79,7 @@ __device__ __forceinline__ void put16(uint8_t* tile, uint32_t atom, int row, int
 struct H3Params {
     int T, NCp, slot;     // slot: floats of one summary slot; the prefix of chunk l of head bh sits
                           // at sums + (bh NCp + l) slot, S0 at matrix 0, P0 at 2, F0 at 3
+    int BH;
     const float* sums;
     float* o;
     int* status;
@@ -89,8 +92,7 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int chunk = blockIdx.x, bh = blockIdx.y;
-    const int t0 = chunk * C;
+    const int nchunks = (p.T + C - 1) / C, items = nchunks * p.BH;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + X_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
     if (tid == 0) {
@@ -110,12 +112,14 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
         put16(sm + X_BC, BATOM, r, 128 + 16 * h, y2);
         put16(sm + X_BC, BATOM, r, 160 + 16 * h, y1);
     };
-    // ---- Q, K, V rows to their split tiles: thread (r, h) takes columns 16h .. 16h+15 of row r
-    {
-        const int r = tid >> 1, h = tid & 1;
-        const bool in = t0 + r < p.T;
-        const size_t base = ((size_t)bh * p.T + t0 + r) * D3 + 16 * h;
-        float xq[16], xk[16], xv[16];
+    // ---- Q, K, V rows of one item (chunk, head): thread (r, h) takes columns 16h .. 16h+15 of
+    // row r.  The next item's rows are fetched into registers while this item's products run.
+    const int r_in = tid >> 1, h_in = tid & 1;
+    float xq[16], xk[16], xv[16];
+    auto fetch = [&](int item) {
+        const int t = (item % nchunks) * C + r_in, bh = item / nchunks;
+        const bool in = t < p.T;
+        const size_t base = ((size_t)bh * p.T + t) * D3 + 16 * h_in;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float4 a = in ? *reinterpret_cast<const float4*>(q + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -125,6 +129,10 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
             xk[4 * j] = b.x; xk[4 * j + 1] = b.y; xk[4 * j + 2] = b.z; xk[4 * j + 3] = b.w;
             xv[4 * j] = c.x; xv[4 * j + 1] = c.y; xv[4 * j + 2] = c.z; xv[4 * j + 3] = c.w;
         }
+    };
+    // the fetched rows to their split tiles
+    auto put_inputs = [&]() {
+        const int r = r_in, h = h_in;
         float x1[16], x2[16], x3[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) split3(xq[j], x1[j], x2[j], x3[j]);
@@ -144,7 +152,8 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
         }
         put16(sm + X_VC, TILE, r, 16 * h, x1);
         put16(sm + X_VC, TILE, r, 32 + 16 * h, x2);
-    }
+    };
+    if (blockIdx.x < items) fetch(blockIdx.x);
     // A_hi / A_lo blocks above the diagonal are zero in every chunk
 #pragma unroll
     for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
@@ -152,18 +161,6 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
             st_row32_zero(sm + X_AH, row, c0);
             st_row32_zero(sm + X_AL, row, c0);
         }
-    // the carried-in S0, P0, F0 come from the prefix kernels
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tid < 3 * 2 * D3) {
-        // B rows 128 + 32 m + g: column g of matrix m (S0, P0, F0), split as the key rows
-        const int m = tid / (2 * D3), g = (tid >> 1) % D3, h = tid & 1;
-        const float* pre = p.sums + ((size_t)bh * p.NCp + chunk) * p.slot + (m == 0 ? 0 : m + 1) * D3 * D3;
-        float y1[16], y2[16], y3[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) split3(pre[(16 * h + j) * D3 + g], y1[j], y2[j], y3[j]);
-        put_b(C + m * D3 + g, h, y1, y2, y3);
-    }
-    ptx::fence_proxy_async();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -214,107 +211,125 @@ k_hla3_out(const float* __restrict__ q, const float* __restrict__ k, const float
         __syncthreads();
         ptx::tc_fence_after();
     };
-    sync_mma();
     bool ok = true;
-    if (tid == 0) {
-        for (int s = 0; s < 12; ++s)
-            ptx::umma_bf16(tmem + T_X, kdesc2(sb + X_QC, s),
-                           ptx::desc_sw128(sb + X_BC + (s >> 2) * BATOM + (s & 3) * 32, 16, 1024), I_R1, s > 0);
-    }
-    ok = mma_wait();                                                  // R1 done
-    if (ok) {
-        // E1: row `row` of A*, columns half*64 .. +63 in two blocks of 32: A = L (.) A*, split
-        float v[32], hi[32], lo[32];
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const int chunk = item % nchunks, bh = item / nchunks, t0 = chunk * C;
+        put_inputs();
+        // the carried-in S0, P0, F0 come from the prefix kernels
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (tid < 3 * 2 * D3) {
+            // B rows 128 + 32 m + g: column g of matrix m (S0, P0, F0), split as the key rows
+            const int m = tid / (2 * D3), g = (tid >> 1) % D3, h = tid & 1;
+            const float* pre = p.sums + ((size_t)bh * p.NCp + chunk) * p.slot + (m == 0 ? 0 : m + 1) * D3 * D3;
+            float y1[16], y2[16], y3[16];
 #pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 > quad * 32 + 31) continue;                          // zero since set-up
-            ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x = (c0 + i <= row) ? v[i] : 0.f;
-                hi[i] = hi_of(x);
-                lo[i] = x - hi[i];
-            }
-            st_pairs(T_AH + c0 / 2, hi);
-            st_pairs(T_AL + c0 / 2, lo);
-            st_row32(sm + X_AH, row, c0, hi);
-            st_row32(sm + X_AL, row, c0, lo);
-        }
-        // P (32 columns) to [p1 | p2 | p1]: half 0 writes the two p1 slots, half 1 the p2 slot
-        ptx::tmem_ld32(tmem + lane_base + T_P, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            hi[i] = hi_of(v[i]);
-            lo[i] = v[i] - hi[i];
-        }
-        if (half == 0) {
-            st_pairs(T_PC, hi);
-            st_pairs(T_PC + 32, hi);
-        } else {
-            st_pairs(T_PC + 16, lo);
+            for (int j = 0; j < 16; ++j) split3(pre[(16 * h + j) * D3 + g], y1[j], y2[j], y3[j]);
+            put_b(C + m * D3 + g, h, y1, y2, y3);
         }
         sync_mma();
         if (tid == 0) {
-            const uint64_t dV = mdesc(sb + X_VC, TILE, 0);
-            for (int s = 0; s < 6; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_PC + 8 * s, kdesc2(sb + X_QC, s), I_W, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AL, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AL + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
+            for (int s = 0; s < 12; ++s)
+                ptx::umma_bf16(tmem + T_X, kdesc2(sb + X_QC, s),
+                               ptx::desc_sw128(sb + X_BC + (s >> 2) * BATOM + (s & 3) * 32, 16, 1024), I_R1, s > 0);
         }
-        ok = mma_wait();                                              // R2 done
-    }
-    if (ok) {
-        // E2: W = L (.) W to hi / lo pairs (over A's); Y = Q P0 + D_y(hi) + D_y(lo) to [Y_hi | Y_lo]
-        float v[32], hi[32], lo[32];
+        // the next item's rows, in flight while this item's products run
+        if (item + (int)gridDim.x < items) fetch(item + gridDim.x);
+        ok = mma_wait();                                                  // R1 done
+        if (ok) {
+            // E1: row `row` of A*, columns half*64 .. +63 in two blocks of 32: A = L (.) A*, split
+            float v[32], hi[32], lo[32];
 #pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 > quad * 32 + 31) continue;
-            ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) continue;                          // zero since set-up
+                ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float x = (c0 + i <= row) ? v[i] : 0.f;
+                    hi[i] = hi_of(x);
+                    lo[i] = x - hi[i];
+                }
+                st_pairs(T_AH + c0 / 2, hi);
+                st_pairs(T_AL + c0 / 2, lo);
+                st_row32(sm + X_AH, row, c0, hi);
+                st_row32(sm + X_AL, row, c0, lo);
+            }
+            // P (32 columns) to [p1 | p2 | p1]: half 0 writes the two p1 slots, half 1 the p2 slot
+            ptx::tmem_ld32(tmem + lane_base + T_P, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float x = (c0 + i <= row) ? v[i] : 0.f;
-                hi[i] = hi_of(x);
-                lo[i] = x - hi[i];
+                hi[i] = hi_of(v[i]);
+                lo[i] = v[i] - hi[i];
             }
-            st_pairs(T_AH + c0 / 2, hi);
-            st_pairs(T_AL + c0 / 2, lo);
+            if (half == 0) {
+                st_pairs(T_PC, hi);
+                st_pairs(T_PC + 32, hi);
+            } else {
+                st_pairs(T_PC + 16, lo);
+            }
+            sync_mma();
+            if (tid == 0) {
+                const uint64_t dV = mdesc(sb + X_VC, TILE, 0);
+                for (int s = 0; s < 6; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_PC + 8 * s, kdesc2(sb + X_QC, s), I_W, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AH + 8 * s, kdesc2(sb + X_AL, s), I_W, 1);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_X, tmem + T_AL + 8 * s, kdesc2(sb + X_AH, s), I_W, 1);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
+            }
+            ok = mma_wait();                                              // R2 done
         }
-        float a[16], b[16], c[16], yh[16], yl[16];
-        ptx::tmem_ld16(tmem + lane_base + T_QP + 16 * half, a);
-        ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
-        ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
+        if (ok) {
+            // E2: W = L (.) W to hi / lo pairs (over A's); Y = Q P0 + D_y(hi) + D_y(lo) to [Y_hi | Y_lo]
+            float v[32], hi[32], lo[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float y = a[i] + b[i] + c[i];
-            yh[i] = hi_of(y);
-            yl[i] = y - yh[i];
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) continue;
+                ptx::tmem_ld32(tmem + lane_base + T_X + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float x = (c0 + i <= row) ? v[i] : 0.f;
+                    hi[i] = hi_of(x);
+                    lo[i] = x - hi[i];
+                }
+                st_pairs(T_AH + c0 / 2, hi);
+                st_pairs(T_AL + c0 / 2, lo);
+            }
+            float a[16], b[16], c[16], yh[16], yl[16];
+            ptx::tmem_ld16(tmem + lane_base + T_QP + 16 * half, a);
+            ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
+            ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float y = a[i] + b[i] + c[i];
+                yh[i] = hi_of(y);
+                yl[i] = y - yh[i];
+            }
+            put16(sm + X_YC, TILE, row, 16 * half, yh);
+            put16(sm + X_YC, TILE, row, 32 + 16 * half, yl);
+            sync_mma();
+            if (tid == 0) {
+                const uint64_t dY = mdesc(sb + X_YC, TILE, 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dY + (uint64_t)(s * 128), I_KM, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dY + (uint64_t)(s * 128), I_KM, 1);
+            }
+            ok = mma_wait();                                              // R3 done
         }
-        put16(sm + X_YC, TILE, row, 16 * half, yh);
-        put16(sm + X_YC, TILE, row, 32 + 16 * half, yl);
-        sync_mma();
-        if (tid == 0) {
-            const uint64_t dY = mdesc(sb + X_YC, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AH + 8 * s, dY + (uint64_t)(s * 128), I_KM, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + T_D, tmem + T_AL + 8 * s, dY + (uint64_t)(s * 128), I_KM, 1);
+        if (ok) {
+            // E3: O = Q F0 + D_o(hi) + D_o(lo); this thread's 16 columns of its row
+            float a[16], b[16], c[16];
+            ptx::tmem_ld16(tmem + lane_base + T_QF + 16 * half, a);
+            ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
+            ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
+            if (t0 + row < p.T) {
+                float4* dst = reinterpret_cast<float4*>(p.o + ((size_t)bh * p.T + t0 + row) * D3 + 16 * half);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_float4(a[4 * j] + b[4 * j] + c[4 * j], a[4 * j + 1] + b[4 * j + 1] + c[4 * j + 1],
+                                         a[4 * j + 2] + b[4 * j + 2] + c[4 * j + 2], a[4 * j + 3] + b[4 * j + 3] + c[4 * j + 3]);
+            }
         }
-        ok = mma_wait();                                              // R3 done
     }
-    if (ok) {
-        // E3: O = Q F0 + D_o(hi) + D_o(lo); this thread's 16 columns of its row
-        float a[16], b[16], c[16];
-        ptx::tmem_ld16(tmem + lane_base + T_QF + 16 * half, a);
-        ptx::tmem_ld16(tmem + lane_base + T_D + 16 * half, b);
-        ptx::tmem_ld16(tmem + lane_base + T_D + 32 + 16 * half, c);
-        if (t0 + row < p.T) {
-            float4* dst = reinterpret_cast<float4*>(p.o + ((size_t)bh * p.T + t0 + row) * D3 + 16 * half);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                dst[j] = make_float4(a[4 * j] + b[4 * j] + c[4 * j], a[4 * j + 1] + b[4 * j + 1] + c[4 * j + 1],
-                                     a[4 * j + 2] + b[4 * j + 2] + c[4 * j + 2], a[4 * j + 3] + b[4 * j + 3] + c[4 * j + 3]);
-        }
-    } else if (tid == 0) {
+    if (!ok && tid == 0) {
         set_status(p.status, DEV_TIMEOUT);
         ptx::umma_commit(bar);
         ptx::mbar_wait(bar, phase, 100000000ull);
@@ -356,7 +371,7 @@ constexpr uint32_t Y_BYTES = Y_BAR + 64 + 1024;
 // D3 192-319; A pairs hi 320-383, lo 384-447
 
 struct H3SParams {
-    int T, NC, slot;
+    int T, NC, slot, BH;
     float* sums;
     int* status;
 };
@@ -368,13 +383,12 @@ k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, half = warp >> 2;
     const int row = quad * 32 + lane;
-    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int items = p.NC * p.BH;
     // the prefix kernels may be scheduled once every summary CTA has started
     if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int t0 = chunk * C;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Y_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
-    float* out = p.sums + ((size_t)bh * p.NC + chunk) * p.slot;
+    float* out = nullptr;                    // the slot of the item in hand
     if (tid == 0) {
         ptx::mbar_init(bar, 1);
         ptx::fence_mbar_init();
@@ -383,12 +397,14 @@ k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float
         ptx::tmem_alloc(tmem_slot, 512);
         ptx::tmem_relinquish();
     }
-    {
-        // Q, K, V rows to their split tiles: thread (r, h) takes columns 16h .. 16h+15 of row r
-        const int r = tid >> 1, h = tid & 1;
-        const bool in = t0 + r < p.T;
-        const size_t base = ((size_t)bh * p.T + t0 + r) * D3 + 16 * h;
-        float xq[16], xk[16], xv[16];
+    // Q, K, V rows of one item (chunk, head): thread (r, h) takes columns 16h .. 16h+15 of row
+    // r.  The next item's rows are fetched into registers while this item's products run.
+    const int r_in = tid >> 1, h_in = tid & 1;
+    float xq[16], xk[16], xv[16];
+    auto fetch = [&](int item) {
+        const int t = (item % p.NC) * C + r_in, bh = item / p.NC;
+        const bool in = t < p.T;
+        const size_t base = ((size_t)bh * p.T + t) * D3 + 16 * h_in;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float4 a = in ? *reinterpret_cast<const float4*>(q + base + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -398,6 +414,10 @@ k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float
             xk[4 * j] = b.x; xk[4 * j + 1] = b.y; xk[4 * j + 2] = b.z; xk[4 * j + 3] = b.w;
             xv[4 * j] = c.x; xv[4 * j + 1] = c.y; xv[4 * j + 2] = c.z; xv[4 * j + 3] = c.w;
         }
+    };
+    // the fetched rows to their split tiles
+    auto put_inputs = [&]() {
+        const int r = r_in, h = h_in;
         float hi[16], lo[16], z[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -429,7 +449,8 @@ k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float
         }
         put16(sm + Y_VV, TILE, r, 16 * h, hi);
         put16(sm + Y_VV, TILE, r, 32 + 16 * h, lo);
-    }
+    };
+    if (blockIdx.x < items) fetch(blockIdx.x);
 #pragma unroll
     for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32)
         if (c0 > quad * 32 + 31) {
@@ -507,105 +528,112 @@ k_hla3_sum(const float* __restrict__ q, const float* __restrict__ k, const float
         }
         __syncthreads();
     };
-    sync_mma();
     bool ok = true;
-    if (tid == 0) {
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, kdesc2(sb + Y_QC, s), kdesc2(sb + Y_KC, s), I_QK, s > 0);
-        const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dB = mdesc(sb + Y_KK, TILE, 0);
-        for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dA + (uint64_t)(s * 128), dB + (uint64_t)(s * 128), I_D1, s > 0);
-    }
-    ok = mma_wait();                                                  // R1 done
-    if (ok) {
-        // E1: A = L (.) A* to hi / lo pairs and tiles
-        float v[32], hi[32], lo[32];
-#pragma unroll
-        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            if (c0 > quad * 32 + 31) continue;
-            ptx::tmem_ld32(tmem + lane_base + c0, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x = (c0 + i <= row) ? v[i] : 0.f;
-                hi[i] = hi_of(x);
-                lo[i] = x - hi[i];
-            }
-            st_pairs(320 + c0 / 2, hi);
-            st_pairs(384 + c0 / 2, lo);
-            st_row32(sm + Y_AH, row, c0, hi);
-            st_row32(sm + Y_AL, row, c0, lo);
-        }
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        out = p.sums + (size_t)item * p.slot;       // item = bh NC + chunk
+        put_inputs();
         sync_mma();
         if (tid == 0) {
-            const uint64_t dV = mdesc(sb + Y_VV, TILE, 0), dQ = mdesc(sb + Y_QQ, TILE, 0);
-            const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 320 + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 384 + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAH + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAL + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, 1);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, kdesc2(sb + Y_QC, s), kdesc2(sb + Y_KC, s), I_QK, s > 0);
+            const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dB = mdesc(sb + Y_KK, TILE, 0);
+            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dA + (uint64_t)(s * 128), dB + (uint64_t)(s * 128), I_D1, s > 0);
         }
-        // S, P, Q2 from D1 (rows K_hi, K_lo, Q_hi, Q_lo; columns K, V, Q, each hi | lo) while R2 runs
-        block_to_slot(128, 0, 0);          // K^T K
-        block_to_slot(128 + 64, 0, 2);     // K^T V
-        block_to_slot(128 + 128, 64, 1);   // Q^T Q
-        ok = mma_wait();                                              // R2 done
-    }
-    if (ok) {
-        // E2: Yl = A V, AQ = A^T Q (each the sum of its hi and lo halves) to split tiles
-        float a[16], b[16], hi[16], lo[16];
+        // the next item's rows, in flight while this item's products run
+        if (item + (int)gridDim.x < items) fetch(item + gridDim.x);
+        ok = mma_wait();                                                  // R1 done
+        if (ok) {
+            // E1: A = L (.) A* to hi / lo pairs and tiles
+            float v[32], hi[32], lo[32];
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const uint32_t col = t == 0 ? 0 : 64;
-            ptx::tmem_ld16(tmem + lane_base + col + 16 * half, a);
-            ptx::tmem_ld16(tmem + lane_base + col + 32 + 16 * half, b);
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                if (c0 > quad * 32 + 31) continue;
+                ptx::tmem_ld32(tmem + lane_base + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float x = (c0 + i <= row) ? v[i] : 0.f;
+                    hi[i] = hi_of(x);
+                    lo[i] = x - hi[i];
+                }
+                st_pairs(320 + c0 / 2, hi);
+                st_pairs(384 + c0 / 2, lo);
+                st_row32(sm + Y_AH, row, c0, hi);
+                st_row32(sm + Y_AL, row, c0, lo);
+            }
+            sync_mma();
+            if (tid == 0) {
+                const uint64_t dV = mdesc(sb + Y_VV, TILE, 0), dQ = mdesc(sb + Y_QQ, TILE, 0);
+                const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 320 + 8 * s, dV + (uint64_t)(s * 128), I_KM, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16_ts(tmem + 0, tmem + 384 + 8 * s, dV + (uint64_t)(s * 128), I_KM, 1);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAH + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 64, dAL + (uint64_t)(s * 128), dQ + (uint64_t)(s * 128), I_M64, 1);
+            }
+            // S, P, Q2 from D1 (rows K_hi, K_lo, Q_hi, Q_lo; columns K, V, Q, each hi | lo) while R2 runs
+            block_to_slot(128, 0, 0);          // K^T K
+            block_to_slot(128 + 64, 0, 2);     // K^T V
+            block_to_slot(128 + 128, 64, 1);   // Q^T Q
+            ok = mma_wait();                                              // R2 done
+        }
+        if (ok) {
+            // E2: Yl = A V, AQ = A^T Q (each the sum of its hi and lo halves) to split tiles
+            float a[16], b[16], hi[16], lo[16];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const uint32_t col = t == 0 ? 0 : 64;
+                ptx::tmem_ld16(tmem + lane_base + col + 16 * half, a);
+                ptx::tmem_ld16(tmem + lane_base + col + 32 + 16 * half, b);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float y = a[i] + b[i];
+                    hi[i] = hi_of(y);
+                    lo[i] = y - hi[i];
+                }
+                uint8_t* tile = sm + (t == 0 ? Y_YY : Y_AQ);
+                put16(tile, TILE, row, 16 * half, hi);
+                put16(tile, TILE, row, 32 + 16 * half, lo);
+            }
+            sync_mma();
+            if (tid == 0) {
+                const uint64_t dY = mdesc(sb + Y_YY, TILE, 0), dYA = mdesc(sb + Y_YY, TILE, 0);
+                const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
+                const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAH + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, s > 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAL + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, 1);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 192, dA + (uint64_t)(s * 128), dYA + (uint64_t)(s * 128), I_M128, s > 0);
+            }
+            ok = mma_wait();                                              // R3 done
+        }
+        if (ok) {
+            // E3: AY = A^T Yl to a split tile (over the concatenated Q, which R1 was the last to read)
+            float a[16], b[16], hi[16], lo[16];
+            ptx::tmem_ld16(tmem + lane_base + 128 + 16 * half, a);
+            ptx::tmem_ld16(tmem + lane_base + 128 + 32 + 16 * half, b);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float y = a[i] + b[i];
                 hi[i] = hi_of(y);
                 lo[i] = y - hi[i];
             }
-            uint8_t* tile = sm + (t == 0 ? Y_YY : Y_AQ);
-            put16(tile, TILE, row, 16 * half, hi);
-            put16(tile, TILE, row, 32 + 16 * half, lo);
+            put16(sm + Y_QC, TILE, row, 16 * half, hi);
+            put16(sm + Y_QC, TILE, row, 32 + 16 * half, lo);
+            sync_mma();
+            if (tid == 0) {
+                const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dAY = mdesc(sb + Y_QC, TILE, 0);
+                for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, dA + (uint64_t)(s * 128), dAY + (uint64_t)(s * 128), I_M64, s > 0);
+            }
+            // X = Q^T Yl (rows Q, columns Yl) and Z = K^T (A^T Q) (rows K, columns AQ) from D3
+            block_to_slot(192, 64, 4);
+            block_to_slot(192 + 64, 0, 5);
+            ok = mma_wait();                                              // R4 done
         }
-        sync_mma();
-        if (tid == 0) {
-            const uint64_t dY = mdesc(sb + Y_YY, TILE, 0), dYA = mdesc(sb + Y_YY, TILE, 0);
-            const uint64_t dAH = mdesc(sb + Y_AH, TILE, 0), dAL = mdesc(sb + Y_AL, TILE, 0);
-            const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAH + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, s > 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 128, dAL + (uint64_t)(s * 128), dY + (uint64_t)(s * 128), I_M64, 1);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 192, dA + (uint64_t)(s * 128), dYA + (uint64_t)(s * 128), I_M128, s > 0);
+        if (ok) {
+            block_to_slot(0, 0, 3);            // F = K^T (A^T (A V))
+            for (int e = tid; e < p.slot - 6 * D3 * D3; e += NT3) out[6 * D3 * D3 + e] = 0.f;   // vectors, padding
+            __syncthreads();
+            if (tid == 0) out[6 * D3 * D3 + 3 * D3] = 1.f;           // rho of the plain op
         }
-        ok = mma_wait();                                              // R3 done
     }
-    if (ok) {
-        // E3: AY = A^T Yl to a split tile (over the concatenated Q, which R1 was the last to read)
-        float a[16], b[16], hi[16], lo[16];
-        ptx::tmem_ld16(tmem + lane_base + 128 + 16 * half, a);
-        ptx::tmem_ld16(tmem + lane_base + 128 + 32 + 16 * half, b);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float y = a[i] + b[i];
-            hi[i] = hi_of(y);
-            lo[i] = y - hi[i];
-        }
-        put16(sm + Y_QC, TILE, row, 16 * half, hi);
-        put16(sm + Y_QC, TILE, row, 32 + 16 * half, lo);
-        sync_mma();
-        if (tid == 0) {
-            const uint64_t dA = mdesc(sb + Y_KK, Y_QQ - Y_KK, 0), dAY = mdesc(sb + Y_QC, TILE, 0);
-            for (int s = 0; s < 8; ++s) ptx::umma_bf16(tmem + 0, dA + (uint64_t)(s * 128), dAY + (uint64_t)(s * 128), I_M64, s > 0);
-        }
-        // X = Q^T Yl (rows Q, columns Yl) and Z = K^T (A^T Q) (rows K, columns AQ) from D3
-        block_to_slot(192, 64, 4);
-        block_to_slot(192 + 64, 0, 5);
-        ok = mma_wait();                                              // R4 done
-    }
-    if (ok) {
-        block_to_slot(0, 0, 3);            // F = K^T (A^T (A V))
-        for (int e = tid; e < p.slot - 6 * D3 * D3; e += NT3) out[6 * D3 * D3 + e] = 0.f;   // vectors, padding
-        __syncthreads();
-        if (tid == 0) out[6 * D3 * D3 + 3 * D3] = 1.f;           // rho of the plain op
-    } else if (tid == 0) {
+    if (!ok && tid == 0) {
         set_status(p.status, DEV_TIMEOUT);
         ptx::umma_commit(bar);
         ptx::mbar_wait(bar, phase, 100000000ull);
@@ -626,11 +654,13 @@ cudaError_t hla3_output(const float* q, const float* k, const float* v, const fl
     prm.sums = sums;
     prm.o = o;
     prm.status = status;
+    prm.BH = BH;
     cudaError_t e;
     if ((e = set_smem(k_hla3_out, X_BYTES)) != cudaSuccess) return e;
     // a programmatic dependent of the prefix kernels: its Q, K, V loads overlap their end
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((T + C - 1) / C, BH);
+    const int items = (T + C - 1) / C * BH;
+    cfg.gridDim = dim3(items < kSMs ? items : kSMs);    // persistent: one CTA per SM walks the items
     cfg.blockDim = dim3(NT3);
     cfg.dynamicSmemBytes = X_BYTES;
     cfg.stream = st;
@@ -651,9 +681,11 @@ cudaError_t hla3_summaries(const float* q, const float* k, const float* v, float
     prm.slot = slot_floats;
     prm.sums = sums;
     prm.status = status;
+    prm.BH = BH;
     cudaError_t e;
     if ((e = set_smem(k_hla3_sum, Y_BYTES)) != cudaSuccess) return e;
-    k_hla3_sum<<<dim3((T + C - 1) / C, BH), NT3, Y_BYTES, st>>>(q, k, v, prm);
+    const int items = NC * BH;               // persistent: one CTA per SM walks the items
+    k_hla3_sum<<<items < kSMs ? items : kSMs, NT3, Y_BYTES, st>>>(q, k, v, prm);
     return cudaGetLastError();
 }
 
