@@ -287,9 +287,9 @@ def test_decayed_walk_segment_plans(gam, nch, T):
 
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 128, 129, 255, 257, 1000, 4097])
 def test_third_order_tensor_core_output(T):
-    """The plain third order with fp32 inputs at d = 32: CUDA-core summaries and prefix over
-    64-token chunks, the output on the tensor cores over 128-token chunks reading every other
-    prefix slot; ragged tails on both chunkings, fp32 tolerance."""
+    """The plain third order with fp32 inputs at d = 32: tensor-core summaries and output over
+    128-token chunks, the factored prefix on the CUDA cores between them; ragged tails, fp32
+    tolerance."""
     assert hla.uses_tensor_cores(hla.OP_HLA3, hla.HLA_F32, False, 1, 3, T, 32, 32) == 2
     w = recipe("hla3", "f32", 1, 3, T, 32, seed=T + 17)
     q, k, v, g = hla_inputs.make_inputs(w)
@@ -309,6 +309,18 @@ def test_second_order_fp32_tensor_cores(T):
     q, k, v, g = hla_inputs.make_inputs(w)
     o = gpu_forward("hla2", q, k, v, g)
     err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla2", q, k, v))
+    assert err <= TOL["f32"], err
+
+
+def test_third_order_tensor_cores_many_items_per_cta():
+    """21 heads x 33 chunks (the last one 1 token long) = 693 chunk x head items: every persistent
+    CTA of the summary and output kernels walks four or five of them, so the next item's loads,
+    the carried barrier phase and the reused TMEM and shared tiles all come into play, across
+    head boundaries and ragged tails."""
+    w = recipe("hla3", "f32", 3, 7, 4097, 32, seed=41)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward("hla3", q, k, v, g)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur("hla3", q, k, v))
     assert err <= TOL["f32"], err
 
 
