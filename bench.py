@@ -283,58 +283,47 @@ def run_ours(args):
     value = weak_scaling_value(tokens, world, ms_per_step / 1e3)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed
-    # region.  The heads are cut into slices that move through three streams in order: copies in
-    # (one stream, slice after slice, so the first slice is complete early), the forwards (one
-    # stream, each waiting for its slice's copies) and copies out (one stream, each waiting for
-    # its slice's forward).  A slice's copy out overlaps later slices' copies in, and only the
-    # first slice's copy in and the last one's copy out are not overlapped.
+    # region.  The batch is cut into per-batch-index slices, each on its own stream (copy in,
+    # forward, copy out), so one slice's copies overlap another slice's compute and the two
+    # copy directions overlap each other.
     e2e = None
     if args.e2e_steps > 0:
         qh, kh, vh = (x.pin_memory() for x in (q, k, v))
         oh = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32).pin_memory()
         main = torch.cuda.current_stream(dev)
-        hs = max(1, 8 // w.B)                 # head groups per batch index: about eight slices
-        while w.H % hs:
-            hs -= 1
-        hw = w.H // hs
-        slices = [(b, j * hw, (j + 1) * hw) for b in range(w.B) for j in range(hs)]
-        s_in, s_fw, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-        ws_e = hla.make_workspace(op, qd[0:1, 0:hw], vd[0:1, 0:hw], decayed=gd is not None)
+        G = w.B
+        streams = [torch.cuda.Stream(dev) for _ in range(G)]
+        gws = [hla.make_workspace(op, qd[b:b + 1], vd[b:b + 1], decayed=gd is not None) for b in range(G)]
         e_ms = []
         for i in range(args.e2e_steps + 2):
             flush.zero_()
             a, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(main)
-            s_in.wait_stream(main)
-            s_fw.wait_stream(main)
-            s_out.wait_stream(main)
-            for b, h0, h1 in slices:
-                ix = (slice(b, b + 1), slice(h0, h1))
-                with torch.cuda.stream(s_in):
-                    qd[ix].copy_(qh[ix], non_blocking=True)
-                    kd[ix].copy_(kh[ix], non_blocking=True)
-                    vd[ix].copy_(vh[ix], non_blocking=True)
-                s_fw.wait_stream(s_in)
-                with torch.cuda.stream(s_fw):
-                    hla.forward(w.op, qd[ix], kd[ix], vd[ix], gamma=gd[h0:h1] if gd is not None else None,
-                                eps=w.eps, out=out[ix], workspace=ws_e, stream=s_fw)
-                s_out.wait_stream(s_fw)
-                with torch.cuda.stream(s_out):
-                    oh[ix].copy_(out[ix], non_blocking=True)
-            main.wait_stream(s_out)
+            for b, s in enumerate(streams):
+                s.wait_stream(main)
+                with torch.cuda.stream(s):
+                    sl = slice(b, b + 1)
+                    qd[sl].copy_(qh[sl], non_blocking=True)
+                    kd[sl].copy_(kh[sl], non_blocking=True)
+                    vd[sl].copy_(vh[sl], non_blocking=True)
+                    hla.forward(w.op, qd[sl], kd[sl], vd[sl], gamma=gd, eps=w.eps, out=out[sl], workspace=gws[b],
+                                stream=s)
+                    oh[sl].copy_(out[sl], non_blocking=True)
+            for s in streams:
+                main.wait_stream(s)
             b_ev.record(main)
             torch.cuda.synchronize()
             if i >= 2:
                 e_ms.append(a.elapsed_time(b_ev))
-        if hla.read_device_status(ws_e) != 0:
-            raise SystemExit("device status word set during the end-to-end run")
+        for b in range(G):
+            if hla.read_device_status(gws[b]) != 0:
+                raise SystemExit("device status word set during the end-to-end run")
         e2e_ms = max_over_ranks(sum(e_ms) / len(e_ms), world, dev)
         h2d = sum(x.numel() * x.element_size() for x in (q, k, v))
         e2e = {"value": weak_scaling_value(tokens, world, e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": oh.numel() * oh.element_size(),
                "ms_per_step": e2e_ms,
-               "pipeline": f"{len(slices)} slices of {hw} heads through three streams in order: copies in, "
-                           "forwards, copies out"}
+               "pipeline": f"{G} batch slices on {G} streams: copy in, forward, copy out per slice"}
 
     peaks, peak_kind = load_peaks()
     decode = None
