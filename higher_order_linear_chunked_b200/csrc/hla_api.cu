@@ -27,6 +27,7 @@ hla_status_t check_shape(hla_dtype_t dtype, int B, int H, int T, int d, int dv) 
     if (dtype != HLA_F32 && dtype != HLA_BF16) return HLA_ERR_DTYPE;
     if (B < 1 || H < 1 || T < 1 || d < 1 || dv < 1) return HLA_ERR_SHAPE;
     if ((long long)B * H * T >= (1LL << 31)) return HLA_ERR_SHAPE;
+    if ((long long)B * H > 65535) return HLA_ERR_SHAPE;        // heads are a grid's y extent
     if (d != dv) return HLA_ERR_UNSUPPORTED;
     if (d != 32 && d != 64) return HLA_ERR_UNSUPPORTED;
     return HLA_OK;

@@ -38,11 +38,13 @@
  * type; o is always fp32.  gamma, when given, is fp32 [H], shared across B,
  * each value in (0, 1].  Base addresses must be 16-byte aligned.
  *
- * Supported shapes.  d == dv.  HLA_F32: d in {32, 64}, every op (fp32 CUDA-core
- * path).  HLA_BF16: d in {32, 64}, every op; with d == 64 the tcgen05
- * tensor-core path runs hla2 (with or without decay), hla2_normalized (without
- * decay) and ahla, and every other op runs on the CUDA cores.  T >= 1 (any
- * value; the tail chunk is padded), B, H >= 1, B*H*T < 2^31.  Anything else
+ * Supported shapes.  d == dv, d in {32, 64}, HLA_F32 or HLA_BF16, every op.
+ * The tcgen05 tensor-core kernels run bf16 d == 64 hla2 (with or without decay),
+ * hla2_normalized (without decay) and ahla (plain, normalised, decayed), and
+ * fp32 d == 32 hla3 and hla2 (plain; hla2 up to 64 chunks of 128 tokens per
+ * head); every other case runs on the CUDA cores (hla_uses_tensor_cores says
+ * which).  T >= 1 (any value; the tail chunk is padded), B, H >= 1,
+ * B*H <= 65535 (the heads are a grid dimension), B*H*T < 2^31.  Anything else
  * returns HLA_ERR_UNSUPPORTED or HLA_ERR_SHAPE before any launch.
  *
  * Memory ownership.  Every pointer (q, k, v, o, gamma, workspace) is DEVICE

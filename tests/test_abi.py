@@ -147,6 +147,8 @@ def test_argument_errors_are_reported_before_any_launch(lib, name):
     assert _call(lib, name, B=0) == 2                      # HLA_ERR_SHAPE
     assert _call(lib, name, T=0) == 2
     assert _call(lib, name, B=1 << 16, H=1 << 10, T=1 << 10) == 2
+    assert _call(lib, name, B=256, H=256, T=1) == 2        # B*H above 65535 heads
+    assert _call(lib, name, B=3, H=21845, T=1, ws=0) == 6  # 65535 heads: the shape passes
     assert _call(lib, name, dtype=5) == 4                  # HLA_ERR_DTYPE
     assert _call(lib, name, d=32, dv=64) == 5              # HLA_ERR_UNSUPPORTED
     assert _call(lib, name, d=48, dv=48) == 5
