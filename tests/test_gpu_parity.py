@@ -324,6 +324,19 @@ def test_third_order_tensor_cores_many_items_per_cta():
     assert err <= TOL["f32"], err
 
 
+@pytest.mark.parametrize("op,dtype,d", [("hla2n", "bf16", 64), ("ahla", "bf16", 64), ("hla2d", "bf16", 64),
+                                         ("hla3", "f32", 32)])
+def test_long_single_head(op, dtype, d):
+    """One head of 262,181 tokens (2,049 chunks of 128, the last one 37 tokens long): the
+    longest plans, with hundreds of summary slots per head and the many-slot prefix paths,
+    against the fp64 recurrence over the whole sequence."""
+    w = recipe(op, dtype, 1, 1, 262144 + 37, d, seed=5)
+    q, k, v, g = hla_inputs.make_inputs(w)
+    o = gpu_forward(w.op, q, k, v, g, eps=w.eps)
+    err = oracle.max_row_rel_err(o.cpu(), oracle.recur(w.op, q, k, v, gamma=g, eps=w.eps))
+    assert err <= TOL[dtype], err
+
+
 def test_third_order_tensor_core_output_large_values():
     """Inputs 8x larger than the workload's (a wider dynamic range for the bf16 splits)."""
     w = recipe("hla3", "f32", 1, 2, 2000, 32, seed=3)
