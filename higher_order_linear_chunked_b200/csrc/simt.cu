@@ -1875,13 +1875,13 @@ __global__ void __launch_bounds__(NT) k_bwd_suffix(float* __restrict__ bw, int N
     if (e >= D * D) return;
     float* p = bw + (size_t)blockIdx.y * NCp * Bwd<D>::SIZE + slot * D * D + e;
     float run = 0.f;
-    for (int c0 = NC - 1; c0 >= 0; c0 -= 8) {      // eight independent loads in flight
-        float y[8];
+    for (int c0 = NC - 1; c0 >= 0; c0 -= 32) {     // 32 independent loads in flight
+        float y[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (c0 - i >= 0) y[i] = p[(size_t)(c0 - i) * Bwd<D>::SIZE];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (c0 - i >= 0) {
                 p[(size_t)(c0 - i) * Bwd<D>::SIZE] = run;
                 run += y[i];

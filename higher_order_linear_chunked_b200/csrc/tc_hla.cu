@@ -692,7 +692,7 @@ k_walk(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorM
 //   k_prefix_sum (one thread per matrix element): R0(n) = sum_{l<n} Y_l in place.
 constexpr int PX_NT = 256;
 
-// S0(l) = sum_{m<l} S_m and m0(l) likewise, element-wise running sums (eight loads in flight).
+// S0(l) = sum_{m<l} S_m and m0(l) likewise, element-wise running sums (32 loads in flight).
 __global__ void __launch_bounds__(PX_NT) k_prefix_run(const float* __restrict__ sums, float* __restrict__ pre, int NS,
                                                       int NSp) {
     using S = simt_layout;
@@ -701,13 +701,13 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_run(const float* __restrict__ 
     const int off = e < D * D ? S::mat(0) + e : S::vec(0) + (e - D * D);
     const size_t base = (size_t)blockIdx.y * NSp * S::size + off;
     float run = 0.f;
-    for (int l0 = 0; l0 < NS; l0 += 8) {
-        float y[8];
+    for (int l0 = 0; l0 < NS; l0 += 32) {
+        float y[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (l0 + i < NS) y[i] = sums[base + (size_t)(l0 + i) * S::size];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (l0 + i < NS) {
                 pre[base + (size_t)(l0 + i) * S::size] = run;
                 run += y[i];
@@ -791,13 +791,13 @@ __global__ void __launch_bounds__(PX_NT) k_prefix_sum(float* __restrict__ pre, i
     const int off = e < D * D ? S::mat(2) + e : S::vec(1) + (e - D * D);
     float* p = pre + (size_t)blockIdx.y * NSp * S::size + off;
     float run = 0.f;
-    for (int l0 = 0; l0 < NS; l0 += 8) {
-        float y[8];
+    for (int l0 = 0; l0 < NS; l0 += 32) {    // 32 loads in flight, then the dependent adds
+        float y[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (l0 + i < NS) y[i] = p[(size_t)(l0 + i) * S::size];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             if (l0 + i < NS) {
                 p[(size_t)(l0 + i) * S::size] = run;
                 run += y[i];
