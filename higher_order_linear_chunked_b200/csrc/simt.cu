@@ -1895,8 +1895,7 @@ __global__ void __launch_bounds__(NT) k_bwd_cross(float* __restrict__ bw, int NC
     constexpr int LD = Dim<D>::LD;
     __shared__ float Cs[D * LD], Rs[D * LD];
     float* slot = bw + ((size_t)blockIdx.y * NCp + blockIdx.x) * Bwd<D>::SIZE;
-    load_mat<D>(Cs, slot + 2 * D * D);
-    load_mat<D>(Rs, slot);
+    load_mats<D, 2>({Cs, Rs}, {slot + 2 * D * D, slot});
     __syncthreads();
     float* U = slot + D * D;
     auto acc = [&](int r, int c) { return U[r * D + c]; };
@@ -2221,10 +2220,7 @@ __global__ void __launch_bounds__(NT) k_abwd_out(const TIn* __restrict__ q, cons
     load_rows<D>(Ks, k + head, t0, T);
     load_rows<D>(Vs, v + head, t0, T);
     load_rows<D>(Os, dout + head, t0, T);
-    load_mat<D>(P0, pre + S::mat(0));
-    load_mat<D>(E0, pre + S::mat(1));
-    load_mat<D>(dE, adj);
-    load_mat<D>(dP, adj + D * D);
+    load_mats<D, 4>({P0, E0, dE, dP}, {pre + S::mat(0), pre + S::mat(1), adj, adj + D * D});
     __syncthreads();
     mm<C, C, D>(Tile{Qs, LD}, TileT{Ks, LD}, Zero{}, PutMasked{As, LDC});                          // A
     __syncthreads();
