@@ -1122,7 +1122,10 @@ cudaError_t forward(int op, bool norm, const void* q, const void* k, const void*
         cudaSuccess)
         return e;
     if (ev && (e = cudaEventRecord(ev[0], st)) != cudaSuccess) return e;
-    k_walk<SUMMARY><<<dim3(pl.NSp, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
+    // one CTA per summary segment, plus the zero slot after them that the prefix kernels read
+    // (the folding output walk reads none); the other padding slots are never read
+    const int nsum = prm.fold ? (pl.NSf > 0 ? pl.NSf : 1) : pl.NSf + 1;
+    k_walk<SUMMARY><<<dim3(nsum, BH), NTH, SMEM_BYTES, st>>>(mq, mk, mv, mo, sprm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (ev && (e = cudaEventRecord(ev[1], st)) != cudaSuccess) return e;
     if (!prm.fold && (e = launch_prefix(prm.sums, prm.pre, pl.NSf + 1, pl.NSp, BH, st)) != cudaSuccess) return e;
